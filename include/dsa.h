@@ -1,0 +1,194 @@
+/*
+ * dsa.h - C ABI of the B200 (sm_100a) DSA decode path:
+ *   head gate -> kpool_compress (with k_norm) -> index_scores -> top-k pools
+ *   + token expansion -> NoPE sparse MLA.
+ *
+ * Sources, cited by page title and section:
+ *   [mod.rs] "spark_model/layers/glm5next_dsa/mod.rs": module doc "Shape of
+ *            the pipeline" and "Traps carried from Slice 8"; the docs of
+ *            KERNEL_KV_LORA_DIM, KERNEL_MAX_KPOOL, Glm5NextDsaKernels and
+ *            MASKED_ATTN_MAX_KEYS; Glm5NextDsaConfig::{select_k, out_width,
+ *            kv_cache_dim, validate}.
+ *   [PR227]  "feat(glm53): indexer fp32 head-gate split-K" (stkernel PR #227),
+ *            description and the splitk_applicable predicate.
+ *   [tap]    "glm53 step tap" README, "What it records".
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers unless stated otherwise. The caller owns
+ *     every buffer; no entry point allocates, frees or synchronises.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously. The calls capture into CUDA graphs.
+ *   - bf16 tensors are passed as `dsa_bf16` (raw bit patterns, uint16_t).
+ *   - Bulk tensors must be 16-byte aligned; int32 index arrays 4-byte aligned.
+ *   - Host-side checks run first. On any status other than DSA_OK nothing is
+ *     launched and no output is touched. DSA_ERR_CUDA means a launch failed
+ *     (cudaGetLastError after the launch); outputs are then undefined.
+ *   - There is no fallback path: an unsupported shape is refused with
+ *     DSA_ERR_UNSUPPORTED, never routed elsewhere ([mod.rs] Glm5NextDsaKernels
+ *     doc: a missing DSA entry point is a hard error).
+ *   - Request geometry lives on the device: request b owns cache rows
+ *     [req_start[b], req_start[b+1]) (T_b rows). Token ids are LOGICAL, i.e.
+ *     relative to the request; the physical row is req_start[b] + id ([tap]:
+ *     mla.topk logical vs mla.kvidx physical indices). Device-side values the
+ *     host cannot see (req_start, q_req, q_pos, ids) never cause an access out
+ *     of the documented buffers: a query whose q_req is outside [0, B) has no
+ *     candidates, and ids outside [0, T_b) are ignored.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t dsa_bf16;
+typedef struct CUstream_st *dsa_stream_t;
+
+enum dsa_status {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, inconsistent sizes */
+    DSA_ERR_UNSUPPORTED = 2,   /* valid request outside what the kernels implement */
+    DSA_ERR_ALIGNMENT = 3,     /* pointer not aligned as required */
+    DSA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+    DSA_ERR_CUDA = 5           /* the CUDA runtime reported a launch error */
+};
+
+/* Fixed geometry of the kernels (see each entry point). */
+#define DSA_INDEX_DIM 128          /* indexer head dim D */
+#define DSA_MAX_INDEX_HEADS 16     /* indexer heads H (= head-gate N) */
+#define DSA_MAX_KPOOL 8            /* [mod.rs] KERNEL_MAX_KPOOL */
+#define DSA_KV_LORA 512            /* [mod.rs] KERNEL_KV_LORA_DIM; NoPE: kv_cache_dim */
+#define DSA_MAX_SELECT 4096        /* largest select_k (pools per query) */
+#define DSA_MAX_MLA_HEADS 128      /* MLA heads per query */
+
+/*
+ * Sticky device-side error word. A kernel that gives up a bounded wait (an
+ * mbarrier phase that never completes) ORs a code into it and returns early
+ * instead of spinning; its outputs are then undefined. This call synchronises
+ * the current device, copies the word to *value (host pointer) and, if
+ * `reset` is nonzero, clears it. It is a diagnostic, not part of the hot path.
+ * Codes: 1 = a bounded wait timed out.
+ */
+int dsa_device_status(int *value, int reset);
+
+/* Name of a status code (static string, never NULL). */
+const char *dsa_status_string(int status);
+/* ABI revision of this header; bumps on any signature or contract change. */
+int dsa_abi_version(void);
+#define DSA_ABI_VERSION 1
+
+/*
+ * a1. Indexer head gate [PR227]: out[m, n] = sum_k hidden[m, k] * w[k, n].
+ *   hidden fp32 [M, K] row-major; w fp32 [K, N] row-major; out fp32 [M, N].
+ *   fp32 products and fp32 accumulation; K is split over a cluster of CTAs and
+ *   the partial sums are combined in a fixed order, so results are
+ *   deterministic (they differ from a sequential sum only in rounding).
+ *   Requires 1 <= N <= 16, K >= 1 with K % 4 == 0; M == 0 is a no-op.
+ *   Alignment: hidden 16 bytes; w and out 4 bytes.
+ */
+int dsa_head_gate(const float *hidden, const float *w, float *out, int M, int K, int N,
+                  dsa_stream_t stream);
+
+/*
+ * a2+a3. kpool_compress with the k_norm LayerNorm fused in
+ * ([mod.rs] "Shape of the pipeline" first arrow, traps 1-4, KERNEL_MAX_KPOOL).
+ *   k, gate   bf16 [total_tokens, D] row-major (indexer keys; per-token,
+ *             per-channel compress-gate logits)
+ *   tok_valid uint8 [total_tokens] (nonzero = valid)
+ *   req_start int32 [B + 1], non-decreasing, req_start[0] >= 0
+ *   ape       fp32 [kpool, D]; ln_w, ln_b bf16 [D]; eps >= 0 (LayerNorm eps)
+ * For request b: f_b = first valid token (T_b if none); pool p has slot
+ * tokens t_s = f_b + p*kpool + s; it is valid iff every t_s < T_b and is
+ * valid. kn_t = bf16(LayerNorm(k_t) * ln_w + ln_b) (biased variance); per
+ * channel c, w_s = softmax over s of (gate[t_s, c] + ape[s, c]);
+ * pooled[p, c] = bf16(sum_s w_s * kn_{t_s}[c]).
+ * Outputs:
+ *   pool_keys   bf16 [B, max_pools, D]: pooled key of each valid pool, zero for
+ *               an invalid pool p < n_span_b, rows p >= n_span_b NOT written,
+ *               with n_span_b = min(max_pools, floor((T_b - f_b) / kpool)).
+ *   pool_idx    int32 [B, max_pools, kpool]: t_s (logical) for valid pools,
+ *               -1 for every slot of an invalid pool (all rows written).
+ *   pool_valid  uint8 [B, max_pools] (all rows written).
+ *   first_valid int32 [B]: f_b.
+ * The caller sizes max_pools >= ceil(T_b / kpool) for every request; tokens
+ * past max_pools * kpool after f_b are not pooled.
+ * Requires D == 128, 1 <= kpool <= 8 (DSA_ERR_UNSUPPORTED otherwise: the page
+ * refuses larger kpool instead of truncating), B >= 0, max_pools >= 0.
+ */
+int dsa_kpool_compress(const dsa_bf16 *k, const dsa_bf16 *gate, const uint8_t *tok_valid,
+                       const int32_t *req_start, int B, int D, int kpool, int max_pools,
+                       const float *ape, const dsa_bf16 *ln_w, const dsa_bf16 *ln_b, float eps,
+                       dsa_bf16 *pool_keys, int32_t *pool_idx, uint8_t *pool_valid,
+                       int32_t *first_valid, dsa_stream_t stream);
+
+/*
+ * a4. index_scores ([mod.rs] "Shape of the pipeline" second arrow:
+ * [Q, P] scores plus candidate validity).
+ *   q_idx  bf16 [Q, H, D] indexer queries; gate_w fp32 [Q, H] (head gate of a1)
+ *   q_req, q_pos int32 [Q]: request and position of each query
+ *   pool_keys, pool_valid, first_valid: as written by dsa_kpool_compress
+ *   cand[q, p]   = pool_valid[b, p] and f_b + p*kpool + kpool - 1 <= q_pos[q]
+ *   scores[q, p] = sum_h gate_w[q, h] * max(0, <q_idx[q, h, :], pool_keys[b, p, :]>)
+ *                  in fp32, and -inf where cand is 0.
+ *   Outputs scores fp32 [Q, max_pools] and cand uint8 [Q, max_pools], fully
+ *   written. Pool keys of non-candidates are never read.
+ * Requires D == 128, 1 <= H <= 16, 1 <= kpool <= 8.
+ */
+int dsa_index_scores(const dsa_bf16 *q_idx, const float *gate_w, const int32_t *q_req,
+                     const int32_t *q_pos, int Q, int H, int D, const dsa_bf16 *pool_keys,
+                     const uint8_t *pool_valid, const int32_t *first_valid, int B, int kpool,
+                     int max_pools, float *scores, uint8_t *cand, dsa_stream_t stream);
+
+/*
+ * a5+a6. topk_pools + expand_selection ([mod.rs] "Shape of the pipeline" third
+ * and fourth arrows; Glm5NextDsaConfig::select_k and out_width; trap 6).
+ *   Candidates (cand != 0) of query q are ranked by (score descending, pool id
+ *   ascending); -0.0 equals +0.0 and a NaN score ranks as -inf.
+ *   n_q = min(select_k, number of candidates).
+ *   top_pools int32 [Q, select_k]: ranked pool ids, then -1.
+ *   token_ids int32 [Q, select_k * kpool]: token_ids[q, j*kpool + s] =
+ *             pool_idx[b, top_pools[q, j], s] for j < n_q, -1 after; every
+ *             element is written (the -1 sentinel tail in full).
+ *   Selection is exact and deterministic (ties go to the lowest pool id).
+ * Requires 1 <= kpool <= 8, 0 <= select_k <= 4096, max_pools >= 0.
+ */
+int dsa_topk_expand(const float *scores, const uint8_t *cand, const int32_t *pool_idx,
+                    const int32_t *q_req, int Q, int B, int max_pools, int kpool, int select_k,
+                    int32_t *top_pools, int32_t *token_ids, dsa_stream_t stream);
+
+/*
+ * a7. NoPE MLA restricted to the selected tokens ([mod.rs] "Shape of the
+ * pipeline" last arrow; MASKED_ATTN_MAX_KEYS doc: set-membership mask, so a
+ * per-row gather is exact; trap 5: qk_rope_head_dim == 0, the 512-wide latent
+ * row is both key and value).
+ *   q         bf16 [Q, Hm, 512] (queries absorbed into the latent space)
+ *   kv        bf16 [total_tokens, 512] latent cache
+ *   token_ids int32 [Q, W] logical ids; -1 and ids outside [0, T_b) ignored.
+ *             Ids in a row must be distinct (dsa_topk_expand guarantees it;
+ *             the set semantics of the page collapses duplicates).
+ *   For each head: z_j = sm_scale * <q[q,h,:], kv[row(j),:]>,
+ *   out[q,h,:] = bf16(sum_j softmax(z)_j * kv[row(j),:]) (fp32 accumulation),
+ *   lse[q,h] = log(sum_j exp(z_j)) (natural log; -inf and out = 0 when no id
+ *   is valid). lse may be NULL.
+ *   workspace: device scratch of dsa_sparse_mla_workspace_size(Q, Hm, W) bytes
+ *   (16-byte aligned; contents need no initialisation; not shared between
+ *   calls that may overlap).
+ * Requires kv_lora == 512 and rope_dim == 0 (DSA_ERR_UNSUPPORTED otherwise,
+ * as the page's config validation refuses any other latent width), Hm a
+ * multiple of 16 with 16 <= Hm <= 128, W >= 0.
+ */
+size_t dsa_sparse_mla_workspace_size(int Q, int Hm, int W);
+int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *req_start,
+                          const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
+                          int W, int kv_lora, int rope_dim, float sm_scale, dsa_bf16 *out,
+                          float *lse, void *workspace, size_t workspace_bytes,
+                          dsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

@@ -1,0 +1,86 @@
+// The C ABI of libdsa.so (declared in include/dsa.h). This file is the single
+// translation unit of the library: it includes every stage's kernels so the
+// sticky device error word is one symbol without relocatable device code.
+#include "common.cuh"
+#include "head_gate.cuh"
+#include "kpool_compress.cuh"
+#include "index_scores.cuh"
+#include "topk_expand.cuh"
+#include "sparse_mla.cuh"
+
+extern "C" {
+
+const char *dsa_status_string(int status) {
+    switch (status) {
+        case DSA_OK: return "DSA_OK";
+        case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+        case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+        case DSA_ERR_ALIGNMENT: return "DSA_ERR_ALIGNMENT";
+        case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+        case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+        default: return "DSA_ERR_UNKNOWN";
+    }
+}
+
+int dsa_abi_version(void) { return DSA_ABI_VERSION; }
+
+int dsa_device_status(int *value, int reset) {
+    if (!value) return DSA_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(value, dsa::g_device_error, sizeof(int)) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    if (reset) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(dsa::g_device_error, &zero, sizeof(int)) != cudaSuccess)
+            return DSA_ERR_CUDA;
+    }
+    return DSA_OK;
+}
+
+int dsa_head_gate(const float *hidden, const float *w, float *out, int M, int K, int N,
+                  dsa_stream_t stream) {
+    return dsa::head_gate_launch(hidden, w, out, M, K, N, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dsa_kpool_compress(const dsa_bf16 *k, const dsa_bf16 *gate, const uint8_t *tok_valid,
+                       const int32_t *req_start, int B, int D, int kpool, int max_pools,
+                       const float *ape, const dsa_bf16 *ln_w, const dsa_bf16 *ln_b, float eps,
+                       dsa_bf16 *pool_keys, int32_t *pool_idx, uint8_t *pool_valid,
+                       int32_t *first_valid, dsa_stream_t stream) {
+    return dsa::kpool_compress_launch(k, gate, tok_valid, req_start, B, D, kpool, max_pools, ape,
+                                      ln_w, ln_b, eps, pool_keys, pool_idx, pool_valid,
+                                      first_valid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dsa_index_scores(const dsa_bf16 *q_idx, const float *gate_w, const int32_t *q_req,
+                     const int32_t *q_pos, int Q, int H, int D, const dsa_bf16 *pool_keys,
+                     const uint8_t *pool_valid, const int32_t *first_valid, int B, int kpool,
+                     int max_pools, float *scores, uint8_t *cand, dsa_stream_t stream) {
+    return dsa::index_scores_launch(q_idx, gate_w, q_req, q_pos, Q, H, D, pool_keys, pool_valid,
+                                    first_valid, B, kpool, max_pools, scores, cand,
+                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dsa_topk_expand(const float *scores, const uint8_t *cand, const int32_t *pool_idx,
+                    const int32_t *q_req, int Q, int B, int max_pools, int kpool, int select_k,
+                    int32_t *top_pools, int32_t *token_ids, dsa_stream_t stream) {
+    return dsa::topk_expand_launch(scores, cand, pool_idx, q_req, Q, B, max_pools, kpool,
+                                   select_k, top_pools, token_ids,
+                                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_sparse_mla_workspace_size(int Q, int Hm, int W) {
+    return dsa::mla_workspace_bytes(Q, Hm, W);
+}
+
+int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *req_start,
+                          const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
+                          int W, int kv_lora, int rope_dim, float sm_scale, dsa_bf16 *out,
+                          float *lse, void *workspace, size_t workspace_bytes,
+                          dsa_stream_t stream) {
+    return dsa::sparse_mla_launch(q, kv, req_start, q_req, token_ids, Q, B, Hm, W, kv_lora,
+                                  rope_dim, sm_scale, out, lse, workspace, workspace_bytes,
+                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

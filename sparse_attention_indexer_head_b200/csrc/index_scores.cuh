@@ -1,0 +1,119 @@
+// a4. index_scores: [Q, P] head-gated ReLU dot scores plus candidate validity
+// ("spark_model/layers/glm5next_dsa/mod.rs", "Shape of the pipeline", second
+// arrow).
+//
+// Per query q of request b and pool p:
+//   cand = pool_valid[b,p] && last slot token of p <= q_pos[q]
+//   score = sum_h gate_w[q,h] * max(0, <q_idx[q,h,:], key[b,p,:]>), -inf if !cand.
+//
+// Kernel: a CTA scores 128 pools of one query, one thread per pool. The query
+// (16 heads x 128 channels) sits transposed in shared memory as fp32 and is
+// read by broadcast; the pool key row is read with 16-byte loads. Each head's
+// 128-term dot runs as 4 interleaved fp32 chains of 32 terms joined pairwise
+// (shorter chains keep the rounding error near the pairwise bound). Keys of
+// non-candidates are never read.
+#pragma once
+
+#include "common.cuh"
+
+namespace dsa {
+
+constexpr int kScoreThreads = 128;
+constexpr int kScoreHeads = DSA_MAX_INDEX_HEADS;   // 16
+
+__global__ void __launch_bounds__(kScoreThreads)
+index_scores_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__restrict__ gate_w,
+                    const int32_t *__restrict__ q_req, const int32_t *__restrict__ q_pos, int H,
+                    const __nv_bfloat16 *__restrict__ pool_keys,
+                    const uint8_t *__restrict__ pool_valid,
+                    const int32_t *__restrict__ first_valid, int B, int kpool, int max_pools,
+                    float *__restrict__ scores, uint8_t *__restrict__ cand) {
+    __shared__ __align__(16) float qs[kD * kScoreHeads];   // qs[c][h]
+    __shared__ float gs[kScoreHeads];
+
+    const int q = blockIdx.y;
+    const int tid = threadIdx.x;
+    const int b = q_req[q];
+    const bool req_ok = b >= 0 && b < B;
+
+    for (int i = tid; i < kD * kScoreHeads; i += kScoreThreads) {
+        const int c = i / kScoreHeads, h = i % kScoreHeads;
+        qs[i] = (req_ok && h < H) ? __bfloat162float(q_idx[((size_t)q * H + h) * kD + c]) : 0.f;
+    }
+    if (tid < kScoreHeads) gs[tid] = (req_ok && tid < H) ? gate_w[(size_t)q * H + tid] : 0.f;
+    __syncthreads();
+
+    const int p = blockIdx.x * kScoreThreads + tid;
+    if (p >= max_pools) return;
+    const size_t out_i = (size_t)q * max_pools + p;
+    bool is_cand = false;
+    if (req_ok) {
+        const long long last = (long long)first_valid[b] + (long long)p * kpool + kpool - 1;
+        is_cand = pool_valid[(size_t)b * max_pools + p] != 0 && last <= (long long)q_pos[q];
+    }
+    if (!is_cand) {
+        scores[out_i] = -INFINITY;
+        cand[out_i] = 0;
+        return;
+    }
+
+    const __nv_bfloat16 *key = pool_keys + ((size_t)b * max_pools + p) * kD;
+    float acc[4][kScoreHeads];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int h = 0; h < kScoreHeads; ++h) acc[u][h] = 0.f;
+
+#pragma unroll 1
+    for (int c8 = 0; c8 < kD / 8; ++c8) {
+        float kv[8];
+        unpack8(ldg_nc_v4(key + 8 * c8), kv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 *qr = reinterpret_cast<const float4 *>(qs + (8 * c8 + j) * kScoreHeads);
+            const int u = j & 3;
+#pragma unroll
+            for (int h4 = 0; h4 < 4; ++h4) {
+                const float4 qv = qr[h4];
+                acc[u][4 * h4 + 0] = fmaf(qv.x, kv[j], acc[u][4 * h4 + 0]);
+                acc[u][4 * h4 + 1] = fmaf(qv.y, kv[j], acc[u][4 * h4 + 1]);
+                acc[u][4 * h4 + 2] = fmaf(qv.z, kv[j], acc[u][4 * h4 + 2]);
+                acc[u][4 * h4 + 3] = fmaf(qv.w, kv[j], acc[u][4 * h4 + 3]);
+            }
+        }
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int h = 0; h < kScoreHeads; ++h) {
+        const float d = (acc[0][h] + acc[1][h]) + (acc[2][h] + acc[3][h]);
+        s = fmaf(gs[h], fmaxf(d, 0.f), s);
+    }
+    scores[out_i] = s;
+    cand[out_i] = 1;
+}
+
+inline int index_scores_launch(const void *q_idx, const float *gate_w, const int32_t *q_req,
+                               const int32_t *q_pos, int Q, int H, int D, const void *pool_keys,
+                               const uint8_t *pool_valid, const int32_t *first_valid, int B,
+                               int kpool, int max_pools, float *scores, uint8_t *cand,
+                               cudaStream_t stream) {
+    if (Q < 0 || H <= 0 || D <= 0 || B < 0 || kpool <= 0 || max_pools < 0)
+        return DSA_ERR_INVALID_ARG;
+    if (D != kD || H > kScoreHeads || kpool > DSA_MAX_KPOOL) return DSA_ERR_UNSUPPORTED;
+    if (Q == 0 || max_pools == 0) return DSA_OK;
+    if (Q > 65535) return DSA_ERR_UNSUPPORTED;
+    if (!q_idx || !gate_w || !q_req || !q_pos || !scores || !cand ||
+        (B > 0 && (!pool_keys || !pool_valid || !first_valid)))
+        return DSA_ERR_INVALID_ARG;
+    if (!aligned(q_idx, 16) || !aligned(gate_w, 4) || !aligned(q_req, 4) || !aligned(q_pos, 4) ||
+        !aligned(pool_keys, 16) || !aligned(first_valid, 4) || !aligned(scores, 4))
+        return DSA_ERR_ALIGNMENT;
+    dim3 grid(ceil_div(max_pools, kScoreThreads), Q);
+    index_scores_kernel<<<grid, kScoreThreads, 0, stream>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(q_idx), gate_w, q_req, q_pos, H,
+        reinterpret_cast<const __nv_bfloat16 *>(pool_keys), pool_valid, first_valid, B, kpool,
+        max_pools, scores, cand);
+    return launch_status();
+}
+
+}  // namespace dsa

@@ -1,0 +1,143 @@
+"""One DSA decode/prefill step on the GPU: device buffers plus the five C-ABI calls.
+
+PyTorch is used for device memory, pinned host memory and streams only; every
+stage runs in libdsa.so:
+  dsa_head_gate -> dsa_kpool_compress -> dsa_index_scores -> dsa_topk_expand
+  -> dsa_sparse_mla_decode.
+Cache-side tensors (k, gate logits, validity, latent kv, request offsets and
+the layer weights) are device-resident state; query-side tensors (hidden,
+indexer queries, MLA queries, query request/position) are the per-step inputs.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+from . import binding as B
+from .workloads import INDEX_DIM, INDEX_HEADS, KV_LORA, Workload
+
+QUERY_INPUTS = ("hidden", "q_idx", "q_mla", "q_req", "q_pos")
+
+
+def _bf16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+
+def host_tensors(wl: Workload) -> Dict[str, torch.Tensor]:
+    """CPU torch views of a workload's arrays (bf16 bit patterns as torch.bfloat16)."""
+    return {
+        "hidden": torch.from_numpy(wl.hidden),
+        "w_gate": torch.from_numpy(wl.w_gate),
+        "q_idx": _bf16(wl.q_idx),
+        "k": _bf16(wl.k),
+        "gate": _bf16(wl.gate),
+        "valid": torch.from_numpy(wl.valid),
+        "req_start": torch.from_numpy(wl.req_start),
+        "ape": torch.from_numpy(wl.ape),
+        "ln_w": _bf16(wl.ln_w),
+        "ln_b": _bf16(wl.ln_b),
+        "q_mla": _bf16(wl.q_mla),
+        "kv": _bf16(wl.kv),
+        "q_req": torch.from_numpy(wl.q_req),
+        "q_pos": torch.from_numpy(wl.q_pos),
+    }
+
+
+@dataclass
+class Geometry:
+    B: int
+    Q: int
+    kpool: int
+    max_pools: int
+    select_k: int
+    hm: int
+    eps: float
+    sm_scale: float
+
+    @property
+    def W(self) -> int:
+        return self.select_k * self.kpool
+
+
+class DecodeStep:
+    """Device buffers of one step; ``run()`` enqueues the five calls on a stream."""
+
+    def __init__(self, wl: Workload, device: str = "cuda", inputs: Optional[Dict] = None):
+        self.device = torch.device(device)
+        self.g = Geometry(wl.B, wl.Q, wl.kpool, wl.max_pools, wl.select_k, wl.hm, wl.eps,
+                          wl.sm_scale)
+        src = host_tensors(wl) if inputs is None else inputs
+        self.t = {k: v.to(self.device) for k, v in src.items()}
+        g, dev = self.g, self.device
+        self.gate_w = torch.empty(g.Q, INDEX_HEADS, dtype=torch.float32, device=dev)
+        self.pool_keys = torch.zeros(g.B, g.max_pools, INDEX_DIM, dtype=torch.bfloat16, device=dev)
+        self.pool_idx = torch.empty(g.B, g.max_pools, g.kpool, dtype=torch.int32, device=dev)
+        self.pool_valid = torch.empty(g.B, g.max_pools, dtype=torch.uint8, device=dev)
+        self.first_valid = torch.empty(g.B, dtype=torch.int32, device=dev)
+        self.scores = torch.empty(g.Q, g.max_pools, dtype=torch.float32, device=dev)
+        self.cand = torch.empty(g.Q, g.max_pools, dtype=torch.uint8, device=dev)
+        self.top_pools = torch.empty(g.Q, g.select_k, dtype=torch.int32, device=dev)
+        self.token_ids = torch.empty(g.Q, g.W, dtype=torch.int32, device=dev)
+        self.out = torch.empty(g.Q, g.hm, KV_LORA, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(g.Q, g.hm, dtype=torch.float32, device=dev)
+        ws = B.dsa_sparse_mla_workspace_size(g.Q, g.hm, g.W)
+        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+
+    # -- the five stages ---------------------------------------------------------------
+    def head_gate(self, stream=None):
+        g, t = self.g, self.t
+        B.dsa_head_gate(t["hidden"], t["w_gate"], self.gate_w, g.Q, t["hidden"].shape[1],
+                        INDEX_HEADS, stream)
+
+    def kpool_compress(self, stream=None):
+        g, t = self.g, self.t
+        B.dsa_kpool_compress(t["k"], t["gate"], t["valid"], t["req_start"], g.B, INDEX_DIM,
+                             g.kpool, g.max_pools, t["ape"], t["ln_w"], t["ln_b"], g.eps,
+                             self.pool_keys, self.pool_idx, self.pool_valid, self.first_valid,
+                             stream)
+
+    def index_scores(self, stream=None):
+        g, t = self.g, self.t
+        B.dsa_index_scores(t["q_idx"], self.gate_w, t["q_req"], t["q_pos"], g.Q, INDEX_HEADS,
+                           INDEX_DIM, self.pool_keys, self.pool_valid, self.first_valid, g.B,
+                           g.kpool, g.max_pools, self.scores, self.cand, stream)
+
+    def topk_expand(self, stream=None):
+        g, t = self.g, self.t
+        B.dsa_topk_expand(self.scores, self.cand, self.pool_idx, t["q_req"], g.Q, g.B,
+                          g.max_pools, g.kpool, g.select_k, self.top_pools, self.token_ids, stream)
+
+    def sparse_mla(self, stream=None):
+        g, t = self.g, self.t
+        B.dsa_sparse_mla_decode(t["q_mla"], t["kv"], t["req_start"], t["q_req"], self.token_ids,
+                                g.Q, g.B, g.hm, g.W, KV_LORA, 0, g.sm_scale, self.out, self.lse,
+                                self.ws, self.ws.numel(), stream)
+
+    def run(self, stream=None):
+        self.head_gate(stream)
+        self.kpool_compress(stream)
+        self.index_scores(stream)
+        self.topk_expand(stream)
+        self.sparse_mla(stream)
+
+    KERNELS_PER_STEP = 6   # gate, compress, scores, topk+expand, mla split, mla combine
+
+    def outputs_numpy(self) -> Dict[str, np.ndarray]:
+        def u16(x):
+            return x.view(torch.int16).cpu().numpy().view(np.uint16)
+        return {
+            "gate_w": self.gate_w.cpu().numpy(),
+            "pool_keys": u16(self.pool_keys),
+            "pool_idx": self.pool_idx.cpu().numpy(),
+            "pool_valid": self.pool_valid.cpu().numpy(),
+            "first_valid": self.first_valid.cpu().numpy(),
+            "scores": self.scores.cpu().numpy(),
+            "cand": self.cand.cpu().numpy(),
+            "top_pools": self.top_pools.cpu().numpy(),
+            "token_ids": self.token_ids.cpu().numpy(),
+            "out": u16(self.out),
+            "lse": self.lse.cpu().numpy(),
+        }

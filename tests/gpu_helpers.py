@@ -1,0 +1,127 @@
+"""Shared helpers of the GPU parity tests: tolerances and device plumbing.
+
+Tolerances (each derived from the arithmetic, see the docstrings):
+  * fp32 head gate: |gpu - ref| <= 1e-5 * max(1, |ref|).
+  * fp32 scores:    |gpu - ref| <= 1e-5 * max(1, S) with S = sum_h |g_h| relu(d_h),
+                    the magnitude of the summed terms (equal to |ref| when every
+                    gate weight is positive).
+  * bf16 pooled keys: |gpu - ref| <= ulp(ref) + max_s ulp(kn_s).
+  * bf16 MLA out:   max-abs 2e-2, and >= 99.9 % of elements within one bf16 ulp.
+"""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+import torch
+
+from sparse_attention_indexer_head_b200 import workloads as W
+
+
+def bf16f(bits) -> np.ndarray:
+    return W.bf16_bits_to_f32(np.asarray(bits, dtype=np.uint16)).astype(np.float64)
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 values at |x| (2^-133 in the subnormal range)."""
+    ax = np.abs(np.asarray(x, dtype=np.float64))
+    _, e = np.frexp(ax)                  # ax = m 2^e, m in [0.5, 1)
+    e = np.maximum(e - 1, -126)
+    return np.ldexp(1.0, e - 7)
+
+
+def assert_gate_close(gpu, ref, what="gate"):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(gpu - ref)
+    tol = 1e-5 * np.maximum(1.0, np.abs(ref))
+    bad = np.argwhere(err > tol)
+    assert bad.size == 0, f"{what}: {len(bad)} outside 1e-5*max(1,|ref|); worst {err.max():.3g}"
+    return float(err.max())
+
+
+def score_magnitude(q_idx_bits, gate_w, keys_bits, q_req, kpool=None):
+    """S[q,p] = sum_h |g_h| * relu(<q_h, key_p>) in fp64 (for the scores tolerance)."""
+    q = bf16f(q_idx_bits)                                   # [Q,H,D]
+    keys = bf16f(keys_bits)                                 # [B,P,D]
+    out = np.empty((q.shape[0], keys.shape[1]))
+    for i in range(q.shape[0]):
+        d = np.einsum("hc,pc->hp", q[i], keys[q_req[i]])
+        out[i] = (np.abs(gate_w[i]).astype(np.float64)[:, None] * np.maximum(d, 0)).sum(0)
+    return out
+
+
+def assert_scores_close(gpu, ref, cand, mag):
+    cand = cand.astype(bool)
+    assert np.isneginf(gpu[~cand]).all(), "scores of non-candidates must be -inf"
+    g, r, m = gpu[cand].astype(np.float64), ref[cand].astype(np.float64), mag[cand]
+    assert np.isfinite(g).all()
+    err = np.abs(g - r)
+    tol = 1e-5 * np.maximum(1.0, m)
+    assert (err <= tol).all(), f"scores: {(err > tol).sum()} outside tolerance; worst {err.max():.3g}"
+    plain = 1e-5 * np.maximum(1.0, np.abs(r))
+    return dict(max_abs=float(err.max(initial=0)), n=int(cand.sum()),
+                over_plain=int((err > plain).sum()))
+
+
+def kn_ulp_bound(k_bits, ln_w_bits, ln_b_bits, eps, rows):
+    """max over a pool's slots of ulp_bf16(kn) per channel; rows: [n_pools, kpool] token rows."""
+    x = bf16f(k_bits[rows.reshape(-1)])                     # [n*kp, D]
+    mu = x.mean(-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(-1, keepdims=True)
+    y = (x - mu) / np.sqrt(var + np.float32(eps)) * bf16f(ln_w_bits) + bf16f(ln_b_bits)
+    u = bf16_ulp(y * (1 + 2.0 ** -8))                      # a hair above: covers the rounded value
+    return u.reshape(rows.shape[0], rows.shape[1], -1).max(1)
+
+
+def assert_keys_close(gpu_keys, ref_keys, pool_valid, wl, first_valid):
+    """Pooled keys of valid pools: |gpu - ref| <= ulp(ref) + max_s ulp(kn_s)."""
+    b_idx, p_idx = np.nonzero(pool_valid)
+    if b_idx.size == 0:
+        return dict(n=0)
+    g = bf16f(gpu_keys[b_idx, p_idx])
+    r = bf16f(ref_keys[b_idx, p_idx])
+    rs = wl.req_start[b_idx].astype(np.int64) + first_valid[b_idx] + p_idx.astype(np.int64) * wl.kpool
+    rows = rs[:, None] + np.arange(wl.kpool)[None, :]
+    bound = bf16_ulp(r) + kn_ulp_bound(wl.k, wl.ln_w, wl.ln_b, wl.eps, rows)
+    err = np.abs(g - r)
+    assert (err <= bound).all(), f"pool keys: {(err > bound).sum()} outside ulp bound"
+    over1 = int((err > bf16_ulp(r)).sum())
+    frac = over1 / err.size
+    assert frac < 1e-3, f"pool keys: {over1} of {err.size} elements beyond 1 ulp"
+    return dict(n=int(err.size), exact=float((err == 0).mean()), over_1ulp=over1)
+
+
+def assert_mla_close(gpu_out, ref_out, gpu_lse, ref_lse, rows=None):
+    g, r = bf16f(gpu_out), bf16f(ref_out)
+    if rows is not None:
+        g, r = g[rows], r[rows]
+        gpu_lse, ref_lse = gpu_lse[rows], ref_lse[rows]
+    err = np.abs(g - r)
+    assert err.max(initial=0) <= 2e-2, f"mla out max-abs {err.max():.3g}"
+    within = (err <= bf16_ulp(r)).mean() if err.size else 1.0
+    assert within >= 0.999, f"mla out: only {within:.5f} within 1 bf16 ulp"
+    both_inf = np.isneginf(gpu_lse) & np.isneginf(ref_lse)
+    assert (np.isneginf(gpu_lse) == np.isneginf(ref_lse)).all()
+    lerr = np.abs(gpu_lse[~both_inf] - ref_lse[~both_inf])
+    assert lerr.max(initial=0) <= 1e-3, f"lse max-abs {lerr.max():.3g}"
+    return dict(max_abs=float(err.max(initial=0)), within_1ulp=float(within),
+                lse_max=float(lerr.max(initial=0)))
+
+
+@functools.lru_cache(maxsize=8)
+def workload(name: str, **kw):
+    return W.make(name, **kw)
+
+
+def device_status_clean(B):
+    assert B.dsa_device_status(reset=True) == 0, "a kernel gave up a bounded wait"
+
+
+def dev_bits(x: np.ndarray, device="cuda") -> torch.Tensor:
+    """bf16 bit array -> device bf16 tensor."""
+    return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def host_bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)

@@ -1,0 +1,143 @@
+"""The C-ABI library on the host (no GPU): it loads, exports every symbol the
+header declares, and refuses bad arguments with the documented status before
+launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+@pytest.fixture(scope="module")
+def B():
+    from sparse_attention_indexer_head_b200 import build
+    build.build()
+    from sparse_attention_indexer_head_b200 import binding
+    return binding
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_five_stages():
+    names = declared_functions()
+    for n in ("dsa_head_gate", "dsa_kpool_compress", "dsa_index_scores", "dsa_topk_expand",
+              "dsa_sparse_mla_decode"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(B):
+    for name in declared_functions():
+        assert hasattr(B.lib, name), name
+    assert set(declared_functions()) == set(B.EXPORTS)
+
+
+def test_status_strings_and_version(B):
+    assert B.dsa_abi_version() == 1
+    for code, name in [(0, "DSA_OK"), (1, "DSA_ERR_INVALID_ARG"), (2, "DSA_ERR_UNSUPPORTED"),
+                       (3, "DSA_ERR_ALIGNMENT"), (4, "DSA_ERR_WORKSPACE"), (5, "DSA_ERR_CUDA")]:
+        assert B.dsa_status_string(code) == name
+    assert B.dsa_status_string(99) == "DSA_ERR_UNKNOWN"
+
+
+FAKE = 1 << 20          # a 16-byte aligned non-null address; never dereferenced on these paths
+
+
+def test_head_gate_refusals(B):
+    L = B.lib
+    assert L.dsa_head_gate(None, None, None, 4, 4096, 16, None) == B.DSA_ERR_INVALID_ARG
+    assert L.dsa_head_gate(FAKE, FAKE, FAKE, 4, 4096, 17, None) == B.DSA_ERR_UNSUPPORTED
+    assert L.dsa_head_gate(FAKE, FAKE, FAKE, 4, 4094, 16, None) == B.DSA_ERR_UNSUPPORTED
+    assert L.dsa_head_gate(FAKE + 4, FAKE, FAKE, 4, 4096, 16, None) == B.DSA_ERR_ALIGNMENT
+    assert L.dsa_head_gate(FAKE, FAKE, FAKE, -1, 4096, 16, None) == B.DSA_ERR_INVALID_ARG
+    assert L.dsa_head_gate(None, None, None, 0, 4096, 16, None) == B.DSA_OK   # M == 0: no-op
+
+
+def _compress(lib, **kw):
+    a = dict(k=FAKE, gate=FAKE, valid=FAKE, req_start=FAKE, B=2, D=128, kpool=4, max_pools=8,
+             ape=FAKE, ln_w=FAKE, ln_b=FAKE, eps=1e-5, keys=FAKE, idx=FAKE, pv=FAKE, fv=FAKE)
+    a.update(kw)
+    return lib.lib.dsa_kpool_compress(a["k"], a["gate"], a["valid"], a["req_start"], a["B"], a["D"],
+                                     a["kpool"], a["max_pools"], a["ape"], a["ln_w"], a["ln_b"],
+                                     a["eps"], a["keys"], a["idx"], a["pv"], a["fv"], None)
+
+
+def test_kpool_compress_refusals(B):
+    assert _compress(B, kpool=9) == B.DSA_ERR_UNSUPPORTED        # KERNEL_MAX_KPOOL = 8
+    assert _compress(B, kpool=0) == B.DSA_ERR_INVALID_ARG
+    assert _compress(B, D=64) == B.DSA_ERR_UNSUPPORTED
+    assert _compress(B, k=None) == B.DSA_ERR_INVALID_ARG
+    assert _compress(B, k=FAKE + 8) == B.DSA_ERR_ALIGNMENT
+    assert _compress(B, eps=-1.0) == B.DSA_ERR_INVALID_ARG
+    assert _compress(B, eps=float("nan")) == B.DSA_ERR_INVALID_ARG
+    assert _compress(B, B=0) == B.DSA_OK
+
+
+def test_index_scores_refusals(B):
+    L = B.lib
+    args = [FAKE, FAKE, FAKE, FAKE, 4, 16, 128, FAKE, FAKE, FAKE, 4, 4, 64, FAKE, FAKE, None]
+    bad = list(args); bad[5] = 17
+    assert L.dsa_index_scores(*bad) == B.DSA_ERR_UNSUPPORTED
+    bad = list(args); bad[6] = 256
+    assert L.dsa_index_scores(*bad) == B.DSA_ERR_UNSUPPORTED
+    bad = list(args); bad[0] = None
+    assert L.dsa_index_scores(*bad) == B.DSA_ERR_INVALID_ARG
+    bad = list(args); bad[0] = FAKE + 2
+    assert L.dsa_index_scores(*bad) == B.DSA_ERR_ALIGNMENT
+    bad = list(args); bad[4] = 0
+    assert L.dsa_index_scores(*bad) == B.DSA_OK
+
+
+def test_topk_expand_refusals(B):
+    L = B.lib
+    args = [FAKE, FAKE, FAKE, FAKE, 4, 4, 64, 4, 16, FAKE, FAKE, None]
+    bad = list(args); bad[8] = 4097
+    assert L.dsa_topk_expand(*bad) == B.DSA_ERR_UNSUPPORTED
+    bad = list(args); bad[7] = 9
+    assert L.dsa_topk_expand(*bad) == B.DSA_ERR_UNSUPPORTED
+    bad = list(args); bad[9] = None
+    assert L.dsa_topk_expand(*bad) == B.DSA_ERR_INVALID_ARG
+    bad = list(args); bad[8] = 0
+    assert L.dsa_topk_expand(*bad) == B.DSA_OK
+
+
+def test_sparse_mla_refusals(B):
+    L = B.lib
+    ws = B.dsa_sparse_mla_workspace_size(16, 64, 2048)
+    assert ws > 0 and ws % 16 == 0
+
+    def call(**kw):
+        a = dict(q=FAKE, kv=FAKE, rs=FAKE, qr=FAKE, ids=FAKE, Q=16, B=16, Hm=64, W=2048, lora=512,
+                 rope=0, scale=0.044, out=FAKE, lse=FAKE, ws=FAKE, wsb=ws)
+        a.update(kw)
+        return L.dsa_sparse_mla_decode(a["q"], a["kv"], a["rs"], a["qr"], a["ids"], a["Q"], a["B"],
+                                       a["Hm"], a["W"], a["lora"], a["rope"], a["scale"], a["out"],
+                                       a["lse"], a["ws"], a["wsb"], None)
+
+    assert call(lora=576) == B.DSA_ERR_UNSUPPORTED      # KERNEL_KV_LORA_DIM = 512
+    assert call(rope=64) == B.DSA_ERR_UNSUPPORTED       # NoPE only
+    assert call(Hm=24) == B.DSA_ERR_UNSUPPORTED
+    assert call(Hm=144) == B.DSA_ERR_UNSUPPORTED
+    assert call(wsb=ws - 16) == B.DSA_ERR_WORKSPACE
+    assert call(ws=None) == B.DSA_ERR_WORKSPACE
+    assert call(q=None) == B.DSA_ERR_INVALID_ARG
+    assert call(scale=float("inf")) == B.DSA_ERR_INVALID_ARG
+    assert call(out=FAKE + 4) == B.DSA_ERR_ALIGNMENT
+    assert call(Q=0) == B.DSA_OK
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """The binding has no fallback: without libdsa.so the import raises."""
+    import importlib.util
+    src = os.path.join(ROOT, "sparse_attention_indexer_head_b200", "binding.py")
+    spec = importlib.util.spec_from_file_location("binding_copy", str(tmp_path / "binding.py"))
+    (tmp_path / "binding.py").write_text(open(src).read())
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)
