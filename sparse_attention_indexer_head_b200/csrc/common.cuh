@@ -111,6 +111,8 @@ DSA_DEVINL float ex2(float x) {
 template <typename T>
 DSA_DEVINL T ldg_nc(const T *p) { return __ldg(p); }
 
+DSA_DEVINL bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 DSA_DEVINL uint4 ldg_nc_v4(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
 
 // ---------------------------------------------------------------- host-side checks

@@ -42,31 +42,67 @@ head_gate_kernel(const float *__restrict__ hidden, const float *__restrict__ w,
 #pragma unroll
     for (int n = 0; n < kGateMaxN; ++n) acc[n] = 0.f;
 
+    // Each pass stages up to 512 rows of w and this thread's 8 vectors of hidden.
+    // All loads of a pass are issued before the first use, so one memory
+    // latency covers the pass instead of one per load.
+    const bool w_vec = N == kGateMaxN && aligned16(w);
     for (int k0 = kb; k0 < ke; k0 += kGateMaxSlice) {
         const int len = min(kGateMaxSlice, ke - k0);
-        __syncthreads();
-        for (int i = tid; i < len * kGateMaxN; i += kGateThreads) {
-            const int kk = i / kGateMaxN, n = i % kGateMaxN;
-            ws[i] = n < N ? __ldg(w + (size_t)(k0 + kk) * N + n) : 0.f;
+        float4 hv[kGateMaxSlice / 64];
+#pragma unroll
+        for (int u = 0; u < kGateMaxSlice / 64; ++u) {
+            const int kk = 4 * j + 64 * u;
+            hv[u] = (m < M && kk < len)
+                        ? __ldg(reinterpret_cast<const float4 *>(hidden + (size_t)m * K + k0 + kk))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        __syncthreads();   // the previous pass is done with ws
+        if (w_vec) {
+            const float4 *src = reinterpret_cast<const float4 *>(w + (size_t)k0 * kGateMaxN);
+            float4 tmp[kGateMaxSlice * kGateMaxN / 4 / kGateThreads];
+#pragma unroll
+            for (int u = 0; u < kGateMaxSlice * kGateMaxN / 4 / kGateThreads; ++u) {
+                const int i = tid + u * kGateThreads;
+                tmp[u] = i < len * 4 ? __ldg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < kGateMaxSlice * kGateMaxN / 4 / kGateThreads; ++u) {
+                const int i = tid + u * kGateThreads;
+                if (i < len * 4) reinterpret_cast<float4 *>(ws)[i] = tmp[u];
+            }
+        } else {
+            for (int i0 = 0; i0 < len * kGateMaxN; i0 += 8 * kGateThreads) {
+                float tmp[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + tid + u * kGateThreads;
+                    const int kk = i / kGateMaxN, n = i % kGateMaxN;
+                    tmp[u] = (i < len * kGateMaxN && n < N) ? __ldg(w + (size_t)(k0 + kk) * N + n)
+                                                            : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + tid + u * kGateThreads;
+                    if (i < len * kGateMaxN) ws[i] = tmp[u];
+                }
+            }
         }
         __syncthreads();
-        if (m < M) {
-            const float *hrow = hidden + (size_t)m * K + k0;
-            // lane j takes 4-wide vectors j, j+16, j+32, ... of the slice
-            for (int kk = 4 * j; kk < len; kk += 64) {
-                const float4 h = __ldg(reinterpret_cast<const float4 *>(hrow + kk));
-                const float hv[4] = {h.x, h.y, h.z, h.w};
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float4 *wr = reinterpret_cast<const float4 *>(ws + (kk + u) * kGateMaxN);
+        for (int u = 0; u < kGateMaxSlice / 64; ++u) {
+            const int kk = 4 * j + 64 * u;
+            if (kk >= len) break;
+            const float hvu[4] = {hv[u].x, hv[u].y, hv[u].z, hv[u].w};
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float4 wv = wr[q];
-                        acc[4 * q + 0] = fmaf(hv[u], wv.x, acc[4 * q + 0]);
-                        acc[4 * q + 1] = fmaf(hv[u], wv.y, acc[4 * q + 1]);
-                        acc[4 * q + 2] = fmaf(hv[u], wv.z, acc[4 * q + 2]);
-                        acc[4 * q + 3] = fmaf(hv[u], wv.w, acc[4 * q + 3]);
-                    }
+            for (int e = 0; e < 4; ++e) {
+                const float4 *wr = reinterpret_cast<const float4 *>(ws + (kk + e) * kGateMaxN);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 wv = wr[q];
+                    acc[4 * q + 0] = fmaf(hvu[e], wv.x, acc[4 * q + 0]);
+                    acc[4 * q + 1] = fmaf(hvu[e], wv.y, acc[4 * q + 1]);
+                    acc[4 * q + 2] = fmaf(hvu[e], wv.z, acc[4 * q + 2]);
+                    acc[4 * q + 3] = fmaf(hvu[e], wv.w, acc[4 * q + 3]);
                 }
             }
         }
@@ -91,15 +127,16 @@ head_gate_kernel(const float *__restrict__ hidden, const float *__restrict__ w,
         const int n = tid % kGateMaxN;
         const int mm = blockIdx.x * kGateRows + rr;
         const uint32_t local = smem_u32(&part[rr * kGateMaxN + n]);
-        float s = 0.f;
+        float v[kGateSplit];
 #pragma unroll
-        for (int c = 0; c < kGateSplit; ++c) {
+        for (int c = 0; c < kGateSplit; ++c) {   // all remote loads in flight at once
             uint32_t remote;
             asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(c));
-            float v;
-            asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-            s += v;
+            asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v[c]) : "r"(remote) : "memory");
         }
+        float s = 0.f;
+#pragma unroll
+        for (int c = 0; c < kGateSplit; ++c) s += v[c];
         if (mm < M && n < N) out[(size_t)mm * N + n] = s;
     }
     // Keep this CTA's shared memory alive until every rank has read it.

@@ -36,9 +36,13 @@ index_scores_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__rest
     const int b = q_req[q];
     const bool req_ok = b >= 0 && b < B;
 
-    for (int i = tid; i < kD * kScoreHeads; i += kScoreThreads) {
-        const int c = i / kScoreHeads, h = i % kScoreHeads;
-        qs[i] = (req_ok && h < H) ? __bfloat162float(q_idx[((size_t)q * H + h) * kD + c]) : 0.f;
+    // 16 heads x 16 vectors of 8 channels: coalesced 16-byte loads, stored transposed.
+    for (int i = tid; i < kScoreHeads * (kD / 8); i += kScoreThreads) {
+        const int h = i % kScoreHeads, c8 = i / kScoreHeads;   // consecutive threads: heads
+        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (req_ok && h < H) unpack8(ldg_nc_v4(q_idx + ((size_t)q * H + h) * kD + 8 * c8), x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qs[(8 * c8 + e) * kScoreHeads + h] = x[e];
     }
     if (tid < kScoreHeads) gs[tid] = (req_ok && tid < H) ? gate_w[(size_t)q * H + tid] : 0.f;
     __syncthreads();
@@ -58,16 +62,20 @@ index_scores_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__rest
     }
 
     const __nv_bfloat16 *key = pool_keys + ((size_t)b * max_pools + p) * kD;
+    uint4 kr[kD / 8];   // the whole 256-byte key row: 16 loads in flight at once
+#pragma unroll
+    for (int c8 = 0; c8 < kD / 8; ++c8) kr[c8] = ldg_nc_v4(key + 8 * c8);
+
     float acc[4][kScoreHeads];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
         for (int h = 0; h < kScoreHeads; ++h) acc[u][h] = 0.f;
 
-#pragma unroll 1
+#pragma unroll
     for (int c8 = 0; c8 < kD / 8; ++c8) {
         float kv[8];
-        unpack8(ldg_nc_v4(key + 8 * c8), kv);
+        unpack8(kr[c8], kv);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const float4 *qr = reinterpret_cast<const float4 *>(qs + (8 * c8 + j) * kScoreHeads);

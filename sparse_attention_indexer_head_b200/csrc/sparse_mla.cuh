@@ -4,125 +4,396 @@
 // set-membership mask, so gathering the selected rows is exact; trap 5: NoPE,
 // the 512-wide latent row is both key and value).
 //
-// Split-KV decode: a query's W selected ids are cut into S contiguous splits;
-// one CTA per (split, query) gathers its latent rows and runs an online
-// softmax for every head, writing an unnormalised partial (O, running max m,
-// running sum l); a combine kernel merges the S partials of each (query, head)
-// in split order (deterministic) and writes bf16 out and the log-sum-exp.
+// Split-KV decode on the 5th-generation tensor cores: a query's W selected ids
+// are cut into S contiguous splits; one CTA per (split, query, 64-head group)
+// gathers its latent rows and runs an online softmax for every head, writing an
+// unnormalised partial (O, running max m, running sum l) -- or, with a single
+// split, the normalised output directly; a combine kernel merges the S
+// partials of each (query, head) in split order (deterministic) and writes
+// bf16 out and the log-sum-exp.
 #pragma once
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace dsa {
 
 constexpr int kL = DSA_KV_LORA;      // 512
-constexpr int kMlaThreads = 256;     // 8 warps
-constexpr int kMlaWarps = 8;
-constexpr int kMlaHeadsPerPass = 8;  // heads a warp holds accumulators for
-constexpr int kMlaTargetCtas = 2 * 148;
-constexpr int kMlaMinSplitTokens = 64;
 // A partial row is O[512], m, l, padded to 516 floats so every row starts on a
-// 16-byte boundary (float4 stores).
+// 16-byte boundary (float4 loads in the combine).
 constexpr int kPartStride = kL + 4;
 
-inline int mla_num_splits(int Q, int W) {
-    if (Q <= 0 || W <= 0) return 1;
-    const int want = ceil_div(kMlaTargetCtas, Q);
-    const int most = ceil_div(W, kMlaMinSplitTokens);
-    return max(1, min(want, most));
-}
+// ---------------------------------------------------------------------------------------
+// tcgen05 split-KV kernel. One CTA per (split, query, group of 64 heads).
+//
+// Per chunk of 64 selected tokens:
+//   S[64 heads x 64 tokens]   = Q[64 x 512] . KV[64 x 512]^T   (M=64, N=64, 32 K-steps)
+//   softmax over the chunk's tokens, per head row, in registers (one thread per head)
+//   O^T[512 x 64 heads]      += KV^T[512 x 64] . P^T[64 x 64]  (4 x M=128, N=64, 4 K-steps)
+// The latent row is both key and value (NoPE), so one 128B-swizzled shared tile
+// of the gathered rows serves as the K-major B operand of S and as the MN-major A
+// operand of O^T. Accumulators live in tensor memory: O^T in columns [0,256)
+// (all 128 lanes), S double-buffered in columns [256,384) (lanes 0-15 of each
+// 32-lane quadrant, the M=64 layout).
+//
+// Warp roles (256 threads): warp 0 allocates tensor memory and one lane issues
+// every MMA; warps 1-3 gather the chunk's latent rows with 16-byte cp.async into
+// the swizzled layout (zero rows for ids that are -1 or outside the request);
+// warps 4-7 load Q, run the softmax (lane i < 16 of warp 4+w owns head 16w+i),
+// rescale O^T when a head's running max grows by more than 2^8 (lazy
+// rescaling), and write the epilogue.
+// ---------------------------------------------------------------------------------------
+constexpr int kTcThreads = 256;
+constexpr int kTcChunk = 64;
+constexpr int kTcHeads = 64;
+constexpr uint32_t kOffQ = 0;                       // 64 KB: 8 atoms x [64 rows x 128 B]
+constexpr uint32_t kOffKV = 64 * 1024;              // 2 stages x 64 KB
+constexpr uint32_t kOffP = 192 * 1024;              // 2 buffers x 8 KB
+constexpr uint32_t kOffCtl = 208 * 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLazyRescale = 8.0f;                // log2 units
 
-inline size_t mla_part_floats(int Q, int Hm, int S) {
-    return (size_t)Q * S * Hm * kPartStride;
+struct TcCtl {
+    uint64_t kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2];
+    uint64_t o_done, q_full, fin;
+    uint64_t vmask[2];
+    int32_t ids[2][kTcChunk];
+    float alpha[kTcHeads];
+    float lsum[kTcHeads];
+    uint32_t tmem_base;
+    volatile int abort;
+    int prod_abort[2];   // per chunk parity: read after the gather barrier of that chunk
+};
+constexpr int kTcSmemBytes = (int)kOffCtl + (int)sizeof(TcCtl) + 1024;   // + alignment slack
+
+struct MlaGeom {
+    int S;      // splits per query
+    int per;    // selected-id slots per split (a multiple of 64)
+};
+
+inline MlaGeom mla_geometry(int Q, int Hm, int W) {
+    MlaGeom g{1, kTcChunk};
+    if (Q <= 0 || W <= 0) return g;
+    const int groups = (Hm + kTcHeads - 1) / kTcHeads;
+    const int chunks = ceil_div(W, kTcChunk);
+    int S = max(1, min(chunks, (148 + Q * groups - 1) / (Q * groups)));
+    if (Q * groups >= 148) S = 1;
+    const int per = ceil_div(ceil_div(W, S), kTcChunk) * kTcChunk;
+    g.S = ceil_div(W, per);
+    g.per = per;
+    return g;
 }
 
 inline size_t mla_workspace_bytes(int Q, int Hm, int W) {
     if (Q <= 0 || Hm <= 0) return 0;
-    return mla_part_floats(Q, Hm, mla_num_splits(Q, W)) * sizeof(float);
+    const MlaGeom g = mla_geometry(Q, Hm, W);
+    if (g.S == 1) return 0;
+    return (size_t)Q * g.S * Hm * kPartStride * sizeof(float);
 }
 
-__global__ void __launch_bounds__(kMlaThreads)
-mla_split_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restrict__ kv,
-                 const int32_t *__restrict__ req_start, const int32_t *__restrict__ q_req,
-                 const int32_t *__restrict__ token_ids, int B, int Hm, int W, int S,
-                 float scale_log2, float *__restrict__ part) {
-    extern __shared__ __align__(16) uint8_t mla_smem[];
-    __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(mla_smem);   // [Hm][512]
+DSA_DEVINL bool tc_wait(TcCtl *ctl, uint64_t *bar, uint32_t parity) {
+    if (ctl->abort) return false;
+    if (!mbar_wait(bar, parity)) {
+        ctl->abort = 1;
+        return false;
+    }
+    return true;
+}
 
-    const int split = blockIdx.x, q = blockIdx.y;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = q_req[q];
+__global__ void __launch_bounds__(kTcThreads, 1)
+mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restrict__ kv,
+              const int32_t *__restrict__ req_start, const int32_t *__restrict__ q_req,
+              const int32_t *__restrict__ token_ids, int B, int Hm, int W, int S, int per,
+              float scale_log2, float *__restrict__ part, __nv_bfloat16 *__restrict__ out,
+              float *__restrict__ lse) {
+    extern __shared__ uint8_t mla_smem_raw[];
+    const uint32_t raw = smem_u32(mla_smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;           // 128B-swizzle atoms need 1 KB
+    uint8_t *gbase = mla_smem_raw + (base - raw);
+    TcCtl *ctl = reinterpret_cast<TcCtl *>(gbase + kOffCtl);
+    const uint32_t sQ = base + kOffQ;
+    const uint32_t sKV[2] = {base + kOffKV, base + kOffKV + 64 * 1024};
+    const uint32_t sP[2] = {base + kOffP, base + kOffP + 8 * 1024};
+
+    const int split = blockIdx.x, qi = blockIdx.y, hg = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = q_req[qi];
     const bool req_ok = b >= 0 && b < B;
     const int rs = req_ok ? req_start[b] : 0;
     const int T = req_ok ? max(0, req_start[b + 1] - rs) : 0;
-    const int per = (W + S - 1) / S;
     const int j0 = min(W, split * per), j1 = min(W, j0 + per);
+    const int ntok = j1 - j0;
+    const int nch = (ntok + kTcChunk - 1) / kTcChunk;
+    const int h0 = hg * kTcHeads, nh = min(kTcHeads, Hm - h0);
 
-    {
-        const uint4 *src = reinterpret_cast<const uint4 *>(qm + (size_t)q * Hm * kL);
-        uint4 *dst = reinterpret_cast<uint4 *>(qs);
-        for (int i = tid; i < Hm * kL / 8; i += kMlaThreads) dst[i] = __ldg(src + i);
+    if (warp == 0) {
+        tc::tmem_alloc(&ctl->tmem_base, kTmemCols);
+        tc::tmem_relinquish();
     }
+    if (tid == 32) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl->kv_full[i], 96);
+            mbar_init(&ctl->kv_empty[i], 1);
+            mbar_init(&ctl->s_full[i], 1);
+            mbar_init(&ctl->s_empty[i], 128);
+            mbar_init(&ctl->p_full[i], 128);
+            mbar_init(&ctl->p_empty[i], 1);
+        }
+        mbar_init(&ctl->o_done, 1);
+        mbar_init(&ctl->q_full, 128);
+        mbar_init(&ctl->fin, 1);
+        ctl->abort = 0;
+        fence_mbarrier_init();
+    }
+    tc::fence_before_sync();
     __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
 
-    const int heads_per_warp = Hm / kMlaWarps;   // Hm is a multiple of 16
-    for (int g0 = 0; g0 < heads_per_warp; g0 += kMlaHeadsPerPass) {
-        const int ng = min(kMlaHeadsPerPass, heads_per_warp - g0);
-        float acc[kMlaHeadsPerPass][16];
-        float m[kMlaHeadsPerPass], l[kMlaHeadsPerPass];
+    if (warp == 0) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0 && nch > 0) {
+            constexpr uint32_t idS = tc::idesc_bf16(64, 64, false, false);
+            constexpr uint32_t idPV = tc::idesc_bf16(128, 64, true, false);
+            auto issue_pv = [&](int cp) -> bool {
+                const int sp = cp & 1;
+                if (!tc_wait(ctl, &ctl->p_full[sp], (cp >> 1) & 1)) return false;
+                tc::fence_after_sync();
 #pragma unroll
-        for (int hh = 0; hh < kMlaHeadsPerPass; ++hh) {
-            m[hh] = -INFINITY;
-            l[hh] = 0.f;
+                for (int lb = 0; lb < 4; ++lb)
 #pragma unroll
-            for (int d = 0; d < 16; ++d) acc[hh][d] = 0.f;
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t a = tc::desc_sw128(sKV[sp] + lb * 2 * 8192 + ks * 2048, 8192, 1024);
+                        const uint64_t bd = tc::desc_sw128(sP[sp] + ks * 32, 16, 1024);
+                        tc::mma_bf16_ss(tmem + lb * 64, a, bd, idPV, (cp > 0 || ks > 0) ? 1u : 0u);
+                    }
+                tc::mma_commit(&ctl->kv_empty[sp]);
+                tc::mma_commit(&ctl->p_empty[sp]);
+                tc::mma_commit(&ctl->o_done);
+                return true;
+            };
+            bool ok = tc_wait(ctl, &ctl->q_full, 0);
+            for (int c = 0; ok && c < nch; ++c) {
+                const int s = c & 1;
+                if (!tc_wait(ctl, &ctl->kv_full[s], (c >> 1) & 1)) { ok = false; break; }
+                if (c >= 2 && !tc_wait(ctl, &ctl->s_empty[s], ((c >> 1) - 1) & 1)) { ok = false; break; }
+                tc::fence_after_sync();
+                const uint32_t d = tmem + 256 + s * 64;
+#pragma unroll
+                for (int kk = 0; kk < kL / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    tc::mma_bf16_ss(d, tc::desc_sw128(sQ + off, 16, 1024),
+                                    tc::desc_sw128(sKV[s] + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(&ctl->s_full[s]);
+                if (c >= 1 && !issue_pv(c - 1)) { ok = false; break; }
+            }
+            if (ok) issue_pv(nch - 1);
         }
-        for (int j = j0; j < j1; ++j) {
-            const int id = token_ids[(size_t)q * W + j];
-            if (id < 0 || id >= T) continue;   // warp-uniform
-            const uint4 *row = reinterpret_cast<const uint4 *>(kv + ((size_t)rs + id) * kL + 16 * lane);
-            float x[16];
-            unpack8(__ldg(row), *reinterpret_cast<float(*)[8]>(x));
-            unpack8(__ldg(row + 1), *reinterpret_cast<float(*)[8]>(x + 8));
+        __syncwarp();
+    } else if (warp < 4) {
+        // ------------------------------------------------------------------ gather (96 threads)
+        const int pt = tid - 32;
+        for (int c = 0; c < nch; ++c) {
+            const int s = c & 1;
+            if (pt == 0) {
+                if (c >= 2) tc_wait(ctl, &ctl->kv_empty[s], ((c >> 1) - 1) & 1);
+                ctl->prod_abort[s] = ctl->abort;
+            }
+            if (pt < 32) {
+                uint32_t m2[2];
 #pragma unroll
-            for (int hh = 0; hh < kMlaHeadsPerPass; ++hh) {
-                if (hh >= ng) break;
-                const int h = warp + kMlaWarps * (g0 + hh);
-                const uint4 *qr = reinterpret_cast<const uint4 *>(qs + (size_t)h * kL + 16 * lane);
-                float qv[16];
-                unpack8(qr[0], *reinterpret_cast<float(*)[8]>(qv));
-                unpack8(qr[1], *reinterpret_cast<float(*)[8]>(qv + 8));
-                float dot = 0.f;
-#pragma unroll
-                for (int d = 0; d < 16; ++d) dot = fmaf(qv[d], x[d], dot);
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-                const float z = dot * scale_log2;
-                const float mn = fmaxf(m[hh], z);
-                const float alpha = ex2(m[hh] - mn);
-                const float p = ex2(z - mn);
-                l[hh] = fmaf(l[hh], alpha, p);
-#pragma unroll
-                for (int d = 0; d < 16; ++d) acc[hh][d] = fmaf(acc[hh][d], alpha, p * x[d]);
-                m[hh] = mn;
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int r = pt + 32 * hh;
+                    const int j = c * kTcChunk + r;
+                    const int id = j < ntok ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
+                    const bool ok = id >= 0 && id < T;
+                    m2[hh] = __ballot_sync(0xffffffffu, ok);
+                    ctl->ids[s][r] = ok ? id : -1;
+                }
+                if (pt == 0) ctl->vmask[s] = (uint64_t)m2[0] | ((uint64_t)m2[1] << 32);
+            }
+            tc::named_bar_sync(1, 96);
+            if (ctl->prod_abort[s]) break;
+            const uint32_t dst0 = sKV[s];
+            for (int x = pt; x < kTcChunk * 64; x += 96) {
+                const int r = x >> 6, cc = x & 63;
+                const int id = ctl->ids[s][r];
+                const uint32_t dst = dst0 + (cc >> 3) * 8192 + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
+                if (id >= 0)
+                    tc::cp_async16(dst, kv + ((size_t)rs + id) * kL + cc * 8);
+                else
+                    tc::st_shared_zero16(dst);
+            }
+            tc::cp_async_wait_all();
+            tc::fence_proxy_async_smem();
+            mbar_arrive(&ctl->kv_full[s]);
+        }
+    } else {
+        // ------------------------------------------------------------------ softmax (128 threads)
+        const int st = tid - 128, wq = warp - 4;
+        const int hh = 16 * wq + lane;        // head row owned by lanes 0..15
+        const bool owner = lane < 16;
+        // Q tile: 64 rows x 64 16-byte chunks into the swizzled K-major layout.
+        for (int x = st; x < kTcHeads * 64; x += 128) {
+            const int h = x >> 6, cc = x & 63;
+            const uint32_t dst = sQ + (cc >> 3) * 8192 + h * 128 + (((cc & 7) ^ (h & 7)) << 4);
+            if (h < nh) {
+                const uint4 v = ldg_nc_v4(qm + ((size_t)qi * Hm + h0 + h) * kL + cc * 8);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x),
+                             "r"(v.y), "r"(v.z), "r"(v.w)
+                             : "memory");
+            } else {
+                tc::st_shared_zero16(dst);
             }
         }
+        tc::fence_proxy_async_smem();
+        mbar_arrive(&ctl->q_full);
+
+        const uint32_t tl = tmem + ((uint32_t)(32 * wq) << 16);
+        float m_used = -INFINITY, l = 0.f;
+        bool failed = false;
+        for (int c = 0; c < nch; ++c) {
+            const int s = c & 1;
+            bool bad = !tc_wait(ctl, &ctl->kv_full[s], (c >> 1) & 1);
+            bad = bad || !tc_wait(ctl, &ctl->s_full[s], (c >> 1) & 1);
+            if (tc::named_bar_or(2, 128, bad)) { failed = true; break; }
+            tc::fence_after_sync();
+            uint32_t r[2][32];
+            tc::tmem_ld32(tl + 256 + s * 64, r[0]);
+            tc::tmem_ld32(tl + 256 + s * 64 + 32, r[1]);
+            tc::tmem_wait_ld();
+            tc::fence_before_sync();
+            mbar_arrive(&ctl->s_empty[s]);
+
+            const uint64_t vm = ctl->vmask[s];
+            float mx = -INFINITY;
 #pragma unroll
-        for (int hh = 0; hh < kMlaHeadsPerPass; ++hh) {
-            if (hh >= ng) break;
-            const int h = warp + kMlaWarps * (g0 + hh);
-            float *po = part + (((size_t)q * S + split) * Hm + h) * kPartStride;
-            float4 *dst = reinterpret_cast<float4 *>(po + 16 * lane);
-#pragma unroll
-            for (int d4 = 0; d4 < 4; ++d4)
-                dst[d4] = make_float4(acc[hh][4 * d4], acc[hh][4 * d4 + 1], acc[hh][4 * d4 + 2],
-                                      acc[hh][4 * d4 + 3]);
-            if (lane == 0) {
-                po[kL] = m[hh];
-                po[kL + 1] = l[hh];
+            for (int j = 0; j < 64; ++j) {
+                const float z = ((vm >> j) & 1) ? __uint_as_float(r[j >> 5][j & 31]) * scale_log2
+                                                : -INFINITY;
+                r[j >> 5][j & 31] = __float_as_uint(z);
+                mx = fmaxf(mx, z);
             }
+            float alpha = 1.f;
+            if (mx > m_used + kLazyRescale) {
+                alpha = ex2(m_used - mx);
+                m_used = mx;
+            }
+            uint32_t pk[32];
+            float psum = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float z0 = __uint_as_float(r[(2 * j) >> 5][(2 * j) & 31]);
+                const float z1 = __uint_as_float(r[(2 * j + 1) >> 5][(2 * j + 1) & 31]);
+                const float p0 = z0 == -INFINITY ? 0.f : ex2(z0 - m_used);
+                const float p1 = z1 == -INFINITY ? 0.f : ex2(z1 - m_used);
+                pk[j] = pack_bf16x2(p0, p1);
+                psum += bf16lo(pk[j]) + bf16hi(pk[j]);   // the sum of the weights the MMA uses
+            }
+            l = fmaf(l, alpha, psum);
+            if (owner) ctl->alpha[hh] = alpha;
+
+            bad = c >= 2 && !tc_wait(ctl, &ctl->p_empty[s], ((c >> 1) - 1) & 1);
+            if (tc::named_bar_or(2, 128, bad)) { failed = true; break; }
+            const bool need = tc::named_bar_or(2, 128, owner && c >= 1 && alpha != 1.f);
+            if (owner) {
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const uint32_t dst = sP[s] + hh * 128 + ((c8 ^ (hh & 7)) << 4);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                                 "r"(pk[4 * c8]), "r"(pk[4 * c8 + 1]), "r"(pk[4 * c8 + 2]),
+                                 "r"(pk[4 * c8 + 3])
+                                 : "memory");
+                }
+            }
+            if (need) {
+                // O^T columns of rescaled heads times alpha, after PV(c-1) has landed.
+                bad = !tc_wait(ctl, &ctl->o_done, (c - 1) & 1);
+                if (tc::named_bar_or(2, 128, bad)) { failed = true; break; }
+                tc::fence_after_sync();
+#pragma unroll 1
+                for (int blk = 0; blk < 8; ++blk) {
+                    uint32_t o[32];
+                    const uint32_t ta = tl + (blk >> 1) * 64 + (blk & 1) * 32;
+                    tc::tmem_ld32(ta, o);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        o[j] = __float_as_uint(__uint_as_float(o[j]) * ctl->alpha[(blk & 1) * 32 + j]);
+                    tc::tmem_st32(ta, o);
+                }
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+            }
+            tc::fence_proxy_async_smem();
+            mbar_arrive(&ctl->p_full[s]);
+        }
+
+        // ------------------------------------------------------------------ epilogue
+        bool have_o = !failed && nch > 0;
+        if (have_o) {
+            const bool bad = !tc_wait(ctl, &ctl->o_done, (nch - 1) & 1);
+            have_o = !tc::named_bar_or(2, 128, bad);
+        }
+        if (owner) ctl->lsum[hh] = l;
+        tc::named_bar_sync(2, 128);
+        if (S > 1) {
+            float *pb = part + ((size_t)(qi * S + split) * Hm + h0) * kPartStride;
+            if (have_o) {
+                tc::fence_after_sync();
+#pragma unroll 1
+                for (int blk = 0; blk < 8; ++blk) {
+                    uint32_t o[32];
+                    tc::tmem_ld32(tl + (blk >> 1) * 64 + (blk & 1) * 32, o);
+                    tc::tmem_wait_ld();
+                    const int L = (blk >> 1) * 128 + 32 * wq + lane;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int h = (blk & 1) * 32 + j;
+                        if (h < nh) pb[(size_t)h * kPartStride + L] = __uint_as_float(o[j]);
+                    }
+                }
+            }
+            if (owner && hh < nh) {
+                pb[(size_t)hh * kPartStride + kL] = have_o ? m_used : -INFINITY;
+                pb[(size_t)hh * kPartStride + kL + 1] = have_o ? l : 0.f;
+            }
+        } else {
+            // single split: normalise here and write bf16 out and lse directly
+            __nv_bfloat16 *ob = out + ((size_t)qi * Hm + h0) * kL;
+            if (have_o) tc::fence_after_sync();
+#pragma unroll 1
+            for (int blk = 0; blk < 8; ++blk) {
+                uint32_t o[32];
+                if (have_o) {
+                    tc::tmem_ld32(tl + (blk >> 1) * 64 + (blk & 1) * 32, o);
+                    tc::tmem_wait_ld();
+                }
+                const int L = (blk >> 1) * 128 + 32 * wq + lane;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int h = (blk & 1) * 32 + j;
+                    const float lh = ctl->lsum[h];
+                    const float v = (have_o && lh > 0.f) ? __uint_as_float(o[j]) / lh : 0.f;
+                    if (h < nh) ob[(size_t)h * kL + L] = __float2bfloat16_rn(v);
+                }
+            }
+            if (lse && owner && hh < nh)
+                lse[(size_t)qi * Hm + h0 + hh] =
+                    (have_o && l > 0.f) ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
         }
     }
+
+    // Every MMA of this CTA has completed before tensor memory is released.
+    if (warp == 0 && lane == 0) {
+        tc::mma_commit(&ctl->fin);
+        (void)mbar_wait(&ctl->fin, 0);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
 // One CTA per (head, query); 128 threads x 4 channels.
@@ -176,19 +447,21 @@ inline int sparse_mla_launch(const void *q, const void *kv, const int32_t *req_s
     if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(req_start, 4) || !aligned(q_req, 4) ||
         !aligned(token_ids, 4) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(ws, 16))
         return DSA_ERR_ALIGNMENT;
-    const int S = mla_num_splits(Q, W);
-    if (!ws || ws_bytes < mla_workspace_bytes(Q, Hm, W)) return DSA_ERR_WORKSPACE;
-    float *part = reinterpret_cast<float *>(ws);
-    const int smem = Hm * kL * 2;
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_split_kernel), smem))
+    const MlaGeom g = mla_geometry(Q, Hm, W);
+    const size_t need = mla_workspace_bytes(Q, Hm, W);
+    if (need > 0 && (!ws || ws_bytes < need)) return DSA_ERR_WORKSPACE;
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel), kTcSmemBytes))
         return DSA_ERR_CUDA;
     const float scale_log2 = sm_scale * 1.4426950408889634f;
-    mla_split_kernel<<<dim3(S, Q), kMlaThreads, smem, stream>>>(
+    const int groups = (Hm + kTcHeads - 1) / kTcHeads;
+    float *part = reinterpret_cast<float *>(ws);
+    mla_tc_kernel<<<dim3(g.S, Q, groups), kTcThreads, kTcSmemBytes, stream>>>(
         reinterpret_cast<const __nv_bfloat16 *>(q), reinterpret_cast<const __nv_bfloat16 *>(kv),
-        req_start, q_req, token_ids, B, Hm, W, S, scale_log2, part);
+        req_start, q_req, token_ids, B, Hm, W, g.S, g.per, scale_log2, part,
+        reinterpret_cast<__nv_bfloat16 *>(out), lse);
     int st = launch_status();
-    if (st != DSA_OK) return st;
-    mla_combine_kernel<<<dim3(Hm, Q), 128, 0, stream>>>(part, Hm, S,
+    if (st != DSA_OK || g.S == 1) return st;
+    mla_combine_kernel<<<dim3(Hm, Q), 128, 0, stream>>>(part, Hm, g.S,
                                                           reinterpret_cast<__nv_bfloat16 *>(out),
                                                           lse);
     return launch_status();

@@ -97,9 +97,17 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
         for (int shift = 24; shift >= 0; shift -= 8) {
             if (tid < 256) hist[tid] = 0;
             __syncthreads();
-            for (int p = tid; p < P; p += kTopkThreads) {
-                const uint32_t k = key_at(p);
-                if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 0xFF], 1);
+            // Warp-aggregated increments: lanes with the same digit elect one
+            // leader, so a few crowded bins do not serialise the whole block.
+            for (int base = (tid & ~31); base < P; base += kTopkThreads) {
+                const int p = base + (tid & 31);
+                uint32_t d = 0x100u;   // no bin
+                if (p < P) {
+                    const uint32_t k = key_at(p);
+                    if ((k & pmask) == prefix) d = (k >> shift) & 0xFF;
+                }
+                const uint32_t peers = __match_any_sync(0xffffffffu, d);
+                if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
             }
             __syncthreads();
             if (tid < 32) {
@@ -169,7 +177,9 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     for (int i = nq + tid; i < n2; i += kTopkThreads) slist[i] = 0ull;
     __syncthreads();
 
-    // Bitonic sort, descending.
+    // Bitonic sort, descending. Element i is always handled by thread i mod 512,
+    // so a stage whose partner distance is below 32 stays inside one warp and
+    // needs only a warp barrier.
     for (int size = 2; size <= n2; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
             for (int i = tid; i < n2; i += kTopkThreads) {
@@ -183,9 +193,11 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
                     }
                 }
             }
-            __syncthreads();
+            if (stride >= 32) __syncthreads();
+            else __syncwarp();
         }
     }
+    __syncthreads();
 
     for (int j = tid; j < K; j += kTopkThreads)
         top_pools[(size_t)q * K + j] = j < nq ? (int32_t)(~(uint32_t)slist[j]) : -1;
