@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "../../include/dsa.h"
 
 #define DSA_DEVINL __device__ __forceinline__
@@ -126,6 +128,15 @@ inline int launch_status() {
 }
 
 inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+// Streaming-multiprocessor count of the current device (persistent grids).
+inline int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
 
 // Raise a kernel's dynamic shared-memory limit once per device (the attribute
 // is per device context). Returns false if the runtime refuses.

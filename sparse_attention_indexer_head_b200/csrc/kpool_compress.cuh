@@ -21,8 +21,11 @@
 
 namespace dsa {
 
-constexpr int kCmpThreads = 256;
-constexpr int kCmpTileTokens = 128;
+constexpr int kCmpConsumers = 256;                 // 8 consumer warps
+constexpr int kCmpThreads = kCmpConsumers + 32;   // + 1 producer warp
+constexpr int kCmpTileTokens = 128;               // token rows per tile (k and gate each)
+constexpr int kCmpStages = 3;
+constexpr int kCmpStageBytes = 2 * kCmpTileTokens * 128 * 2;   // 64 KB: k rows | gate rows
 constexpr int kD = DSA_INDEX_DIM;   // 128 channels
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -67,150 +70,195 @@ DSA_DEVINL float hsum16(float v) {
     return v;
 }
 
+// One pool on a half-warp: lane l owns channels 8l..8l+7 of the kpool slot rows
+// at krow/grow (shared memory). Returns the packed bf16 pooled key chunk (zero
+// when the pool is invalid).
 template <int KP>
-__global__ void __launch_bounds__(kCmpThreads)
+DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *grow,
+                               const float *s_ape, const float (&lw)[8], const float (&lb)[8],
+                               float eps, int l, bool ok) {
+    // Pass 1: LayerNorm statistics and pool logits (log2 units) per slot.
+    float mean[KP], rstd[KP], lg[KP][8];
+#pragma unroll
+    for (int s = 0; s < KP; ++s) {
+        float x[8];
+        unpack8(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) sum += x[c];
+        const float mu = hsum16(sum) * (1.0f / kD);
+        float sq = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float d = x[c] - mu;
+            sq = fmaf(d, d, sq);
+        }
+        const float var = hsum16(sq) * (1.0f / kD);
+        mean[s] = mu;
+        rstd[s] = __frsqrt_rn(var + eps);
+        float g[8];
+        unpack8(*reinterpret_cast<const uint4 *>(grow + s * kD), g);
+        const float4 a0 = *reinterpret_cast<const float4 *>(s_ape + s * kD + 8 * l);
+        const float4 a1 = *reinterpret_cast<const float4 *>(s_ape + s * kD + 8 * l + 4);
+        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+        for (int c = 0; c < 8; ++c) lg[s][c] = fmaf(g[c], kLog2e, av[c]);
+    }
+    // Pass 2: per-channel softmax over slots, weighted sum of the bf16 k_norm rows.
+    float mx[8], den[8], acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        mx[c] = lg[0][c];
+#pragma unroll
+        for (int s = 1; s < KP; ++s) mx[c] = fmaxf(mx[c], lg[s][c]);
+        den[c] = 0.f;
+        acc[c] = 0.f;
+    }
+#pragma unroll
+    for (int s = 0; s < KP; ++s) {
+        float x[8];
+        unpack8(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float y = fmaf((x[c] - mean[s]) * rstd[s], lw[c], lb[c]);
+            const float kn = round_bf16(y);
+            const float e = ex2(lg[s][c] - mx[c]);
+            den[c] += e;
+            acc[c] = fmaf(e, kn, acc[c]);
+        }
+    }
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (ok) {
+        float v[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) v[c] = __fdiv_rn(acc[c], den[c]);
+        o.x = pack_bf16x2(v[0], v[1]);
+        o.y = pack_bf16x2(v[2], v[3]);
+        o.z = pack_bf16x2(v[4], v[5]);
+        o.w = pack_bf16x2(v[6], v[7]);
+    }
+    return o;
+}
+
+struct CmpMeta {
+    int b, p0, p1, n_in, f, rs;
+};
+
+// Persistent kernel: CTA c owns a contiguous range of (request, pool-tile) work
+// items. Warp 8 is the producer: it finds each request's first valid token (a
+// warp ballot scan, cached across the request's tiles) and streams the tile's
+// contiguous k and gate rows into a 3-stage shared-memory ring with two 1-D
+// bulk copies per tile. Warps 0-7 consume: a half-warp per pool.
+template <int KP>
+__global__ void __launch_bounds__(kCmpThreads, 1)
 kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ gate,
                       const uint8_t *__restrict__ valid, const int32_t *__restrict__ req_start,
-                      int B, int max_pools, const float *__restrict__ ape,
-                      const __nv_bfloat16 *__restrict__ ln_w, const __nv_bfloat16 *__restrict__ ln_b,
-                      float eps, __nv_bfloat16 *__restrict__ pool_keys,
-                      int32_t *__restrict__ pool_idx, uint8_t *__restrict__ pool_valid,
-                      int32_t *__restrict__ first_valid) {
+                      int B, int max_pools, int tiles_per_req, int n_tiles,
+                      const float *__restrict__ ape, const __nv_bfloat16 *__restrict__ ln_w,
+                      const __nv_bfloat16 *__restrict__ ln_b, float eps,
+                      __nv_bfloat16 *__restrict__ pool_keys, int32_t *__restrict__ pool_idx,
+                      uint8_t *__restrict__ pool_valid, int32_t *__restrict__ first_valid) {
     constexpr int TP = kCmpTileTokens / KP;   // pools per tile
     extern __shared__ __align__(128) uint8_t cmp_smem[];
-    __nv_bfloat16 *sk = reinterpret_cast<__nv_bfloat16 *>(cmp_smem);
-    __nv_bfloat16 *sg = sk + TP * KP * kD;
     __shared__ __align__(16) float s_ape[KP * kD];   // ape * log2(e)
-    __shared__ __align__(8) uint64_t bar;
-    __shared__ int s_f;
+    __shared__ __align__(8) uint64_t full[kCmpStages], empty[kCmpStages];
+    __shared__ CmpMeta meta[kCmpStages];
 
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5;
-    const int b = blockIdx.y;
-    const int p0 = blockIdx.x * TP;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = gridDim.x;
+    const int t_begin = (int)((long long)blockIdx.x * n_tiles / G);
+    const int t_end = (int)((long long)(blockIdx.x + 1) * n_tiles / G);
 
-    const int rs = req_start[b];
-    const int T = max(0, req_start[b + 1] - rs);
-    if (warp == 0) {
-        const int f = first_valid_scan(valid, rs, T);
-        if (tid == 0) {
-            s_f = f;
-            mbar_init(&bar, 1);
-            fence_mbarrier_init();
+    if (tid == 0) {
+        for (int s = 0; s < kCmpStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kCmpConsumers / 32);
         }
+        fence_mbarrier_init();
     }
     for (int i = tid; i < KP * kD; i += kCmpThreads) s_ape[i] = ape[i] * kLog2e;
     __syncthreads();
-    const int f = s_f;
-    if (blockIdx.x == 0 && tid == 0) first_valid[b] = f;
-    if (p0 >= max_pools) return;
 
-    const int n_span = min(max_pools, (T - f) / KP);
-    const int p1 = min(p0 + TP, max_pools);
-    const int n_in = max(0, min(p1, n_span) - p0);   // pools of this tile inside the request
-
-    if (n_in > 0 && tid == 0) {
-        const uint32_t bytes = (uint32_t)(n_in * KP * kD * 2);
-        const size_t row0 = (size_t)rs + f + (size_t)p0 * KP;
-        mbar_arrive_expect_tx(&bar, 2 * bytes);
-        bulk_g2s(sk, k + row0 * kD, bytes, &bar);
-        bulk_g2s(sg, gate + row0 * kD, bytes, &bar);
+    if (warp == kCmpConsumers / 32) {
+        // ---------------------------------------------------------------- producer warp
+        int cur_b = -1, cur_f = 0, cur_rs = 0, cur_T = 0;
+        for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
+            const int s = i % kCmpStages;
+            bool ok = true;
+            if (i >= kCmpStages) ok = mbar_wait(&empty[s], ((i / kCmpStages) - 1) & 1);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const int b = t / tiles_per_req, j = t - b * tiles_per_req;
+            if (b != cur_b) {
+                cur_rs = req_start[b];
+                cur_T = max(0, req_start[b + 1] - cur_rs);
+                cur_f = first_valid_scan(valid, cur_rs, cur_T);
+                cur_b = b;
+            }
+            const int p0 = j * TP;
+            const int p1 = min(p0 + TP, max_pools);
+            const int n_span = min(max_pools, (cur_T - cur_f) / KP);
+            const int n_in = max(0, min(p1, n_span) - p0);
+            if (lane == 0) {
+                meta[s] = CmpMeta{b, p0, p1, n_in, cur_f, cur_rs};
+                if (n_in > 0) {
+                    const uint32_t bytes = (uint32_t)(n_in * KP * kD * 2);
+                    const size_t row0 = (size_t)cur_rs + cur_f + (size_t)p0 * KP;
+                    __nv_bfloat16 *sk = reinterpret_cast<__nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
+                    mbar_arrive_expect_tx(&full[s], 2 * bytes);
+                    bulk_g2s(sk, k + row0 * kD, bytes, &full[s]);
+                    bulk_g2s(sk + kCmpTileTokens * kD, gate + row0 * kD, bytes, &full[s]);
+                } else {
+                    mbar_arrive(&full[s]);
+                }
+            }
+            __syncwarp();
+        }
+        return;
     }
 
-    // Pools of this tile past the request's span: no key, index -1, invalid.
-    const size_t pool_base = (size_t)b * max_pools;
-    for (int i = n_in * KP + tid; i < (p1 - p0) * KP; i += kCmpThreads)
-        pool_idx[(pool_base + p0) * KP + i] = -1;
-    for (int i = n_in + tid; i < p1 - p0; i += kCmpThreads) pool_valid[pool_base + p0 + i] = 0;
-    if (n_in == 0) return;
-
+    // -------------------------------------------------------------------- consumer warps
     const int hw = tid >> 4;     // half-warp: one pool at a time
     const int l = tid & 15;      // channels 8l .. 8l+7
     float lw[8], lb[8];
     unpack8(ldg_nc_v4(ln_w + 8 * l), lw);
     unpack8(ldg_nc_v4(ln_b + 8 * l), lb);
 
-    if (!mbar_wait(&bar, 0)) return;
+    for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
+        const int s = i % kCmpStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / kCmpStages) & 1))) break;
+        const CmpMeta m = meta[s];
+        const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
+        const __nv_bfloat16 *sg = sk + kCmpTileTokens * kD;
+        const size_t pool_base = (size_t)m.b * max_pools;
+        if (m.p0 == 0 && tid == 0) first_valid[m.b] = m.f;
 
-    // Warp-uniform loop: the two half-warps of a warp take pools ii and ii+1;
-    // a half-warp past the tile computes on a loaded row and stores nothing.
-    for (int ii = 2 * warp; ii < n_in; ii += kCmpThreads / 16) {
-        const bool active = ii + (hw & 1) < n_in;
-        const int i = active ? ii + (hw & 1) : ii;
-        const int p = p0 + i;
-        const __nv_bfloat16 *krow = sk + (size_t)i * KP * kD + 8 * l;
-        const __nv_bfloat16 *grow = sg + (size_t)i * KP * kD + 8 * l;
+        // Pools of this tile past the request's span: no key, index -1, invalid.
+        for (int x = m.n_in * KP + tid; x < (m.p1 - m.p0) * KP; x += kCmpConsumers)
+            pool_idx[(pool_base + m.p0) * KP + x] = -1;
+        for (int x = m.n_in + tid; x < m.p1 - m.p0; x += kCmpConsumers)
+            pool_valid[pool_base + m.p0 + x] = 0;
 
-        // Slot validity: lane s < KP reads the valid byte of slot token s.
-        const size_t tok0 = (size_t)rs + f + (size_t)p * KP;
-        const bool lane_ok = l >= KP || valid[tok0 + l] != 0;
-        const uint32_t half_mask = 0xFFFFu << (tid & 16);
-        const bool ok = (__ballot_sync(0xffffffffu, lane_ok) & half_mask) == half_mask;
-
-        // Pass 1: LayerNorm statistics and pool logits (log2 units) per slot.
-        float mean[KP], rstd[KP], lg[KP][8];
-#pragma unroll
-        for (int s = 0; s < KP; ++s) {
-            float x[8];
-            unpack8(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
-            float sum = 0.f;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) sum += x[c];
-            const float mu = hsum16(sum) * (1.0f / kD);
-            float sq = 0.f;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float d = x[c] - mu;
-                sq = fmaf(d, d, sq);
-            }
-            const float var = hsum16(sq) * (1.0f / kD);
-            mean[s] = mu;
-            rstd[s] = __frsqrt_rn(var + eps);
-            float g[8];
-            unpack8(*reinterpret_cast<const uint4 *>(grow + s * kD), g);
-            const float4 a0 = *reinterpret_cast<const float4 *>(s_ape + s * kD + 8 * l);
-            const float4 a1 = *reinterpret_cast<const float4 *>(s_ape + s * kD + 8 * l + 4);
-            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-            for (int c = 0; c < 8; ++c) lg[s][c] = fmaf(g[c], kLog2e, av[c]);
+        // Warp-uniform loop: the two half-warps of a warp take pools ii and ii+1;
+        // a half-warp past the tile computes on a loaded row and stores nothing.
+        for (int ii = 2 * warp; ii < m.n_in; ii += kCmpConsumers / 16) {
+            const bool active = ii + (hw & 1) < m.n_in;
+            const int pi = active ? ii + (hw & 1) : ii;
+            const int p = m.p0 + pi;
+            // Slot validity: lane s < KP reads the valid byte of slot token s.
+            const size_t tok0 = (size_t)m.rs + m.f + (size_t)p * KP;
+            const bool lane_ok = l >= KP || valid[tok0 + l] != 0;
+            const uint32_t half_mask = 0xFFFFu << (tid & 16);
+            const bool ok = (__ballot_sync(0xffffffffu, lane_ok) & half_mask) == half_mask;
+            const uint4 o = compress_pool<KP>(sk + (size_t)pi * KP * kD + 8 * l,
+                                              sg + (size_t)pi * KP * kD + 8 * l, s_ape, lw, lb,
+                                              eps, l, ok);
+            if (!active) continue;
+            *reinterpret_cast<uint4 *>(pool_keys + (pool_base + p) * kD + 8 * l) = o;
+            if (l < KP) pool_idx[(pool_base + p) * KP + l] = ok ? m.f + p * KP + l : -1;
+            if (l == 0) pool_valid[pool_base + p] = ok ? 1 : 0;
         }
-        // Pass 2: per-channel softmax over slots, weighted sum of the bf16 k_norm rows.
-        float mx[8], den[8], acc[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            mx[c] = lg[0][c];
-#pragma unroll
-            for (int s = 1; s < KP; ++s) mx[c] = fmaxf(mx[c], lg[s][c]);
-            den[c] = 0.f;
-            acc[c] = 0.f;
-        }
-#pragma unroll
-        for (int s = 0; s < KP; ++s) {
-            float x[8];
-            unpack8(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float y = fmaf((x[c] - mean[s]) * rstd[s], lw[c], lb[c]);
-                const float kn = round_bf16(y);
-                const float e = ex2(lg[s][c] - mx[c]);
-                den[c] += e;
-                acc[c] = fmaf(e, kn, acc[c]);
-            }
-        }
-        uint4 o = make_uint4(0, 0, 0, 0);
-        if (ok) {
-            float v[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) v[c] = __fdiv_rn(acc[c], den[c]);
-            o.x = pack_bf16x2(v[0], v[1]);
-            o.y = pack_bf16x2(v[2], v[3]);
-            o.z = pack_bf16x2(v[4], v[5]);
-            o.w = pack_bf16x2(v[6], v[7]);
-        }
-        if (!active) continue;
-        *reinterpret_cast<uint4 *>(pool_keys + (pool_base + p) * kD + 8 * l) = o;
-        if (l < KP) pool_idx[(pool_base + p) * KP + l] = ok ? f + p * KP + l : -1;
-        if (l == 0) pool_valid[pool_base + p] = ok ? 1 : 0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
     }
 }
 
@@ -221,12 +269,16 @@ inline int kpool_compress_launch_kp(const __nv_bfloat16 *k, const __nv_bfloat16 
                                     const __nv_bfloat16 *ln_b, float eps, __nv_bfloat16 *keys,
                                     int32_t *idx, uint8_t *pv, int32_t *fv, cudaStream_t stream) {
     constexpr int TP = kCmpTileTokens / KP;
-    const int smem = 2 * TP * KP * kD * 2;
+    const int smem = kCmpStages * kCmpStageBytes;
     if (!ensure_smem_attr(reinterpret_cast<const void *>(kpool_compress_kernel<KP>), smem))
         return DSA_ERR_CUDA;
-    dim3 grid(max(1, ceil_div(max_pools, TP)), B);
+    const int tiles_per_req = max(1, ceil_div(max_pools, TP));
+    const long long n_tiles = (long long)tiles_per_req * B;
+    if (n_tiles > (1ll << 30)) return DSA_ERR_UNSUPPORTED;
+    const int grid = (int)std::min<long long>(n_tiles, sm_count());
     kpool_compress_kernel<KP><<<grid, kCmpThreads, smem, stream>>>(
-        k, gate, valid, req_start, B, max_pools, ape, ln_w, ln_b, eps, keys, idx, pv, fv);
+        k, gate, valid, req_start, B, max_pools, tiles_per_req, (int)n_tiles, ape, ln_w, ln_b, eps,
+        keys, idx, pv, fv);
     return launch_status();
 }
 
@@ -239,7 +291,6 @@ inline int kpool_compress_launch(const void *k, const void *gate, const uint8_t 
     if (!(eps >= 0.f) || eps > 1e30f) return DSA_ERR_INVALID_ARG;
     if (D != kD || kpool > DSA_MAX_KPOOL) return DSA_ERR_UNSUPPORTED;
     if (B == 0) return DSA_OK;
-    if (B > 65535) return DSA_ERR_UNSUPPORTED;
     if (!k || !gate || !valid || !req_start || !ape || !ln_w || !ln_b || !fv ||
         (max_pools > 0 && (!keys || !idx || !pv)))
         return DSA_ERR_INVALID_ARG;

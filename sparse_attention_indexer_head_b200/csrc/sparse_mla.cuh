@@ -289,7 +289,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                 const float p0 = z0 == -INFINITY ? 0.f : ex2(z0 - m_used);
                 const float p1 = z1 == -INFINITY ? 0.f : ex2(z1 - m_used);
                 pk[j] = pack_bf16x2(p0, p1);
-                psum += bf16lo(pk[j]) + bf16hi(pk[j]);   // the sum of the weights the MMA uses
+                psum += p0 + p1;     // fp32 weights: the row sum and lse stay exact to fp32
             }
             l = fmaf(l, alpha, psum);
             if (owner) ctl->alpha[hh] = alpha;

@@ -6,7 +6,8 @@ Tolerances (each derived from the arithmetic, see the docstrings):
                     the magnitude of the summed terms (equal to |ref| when every
                     gate weight is positive).
   * bf16 pooled keys: |gpu - ref| <= ulp(ref) + max_s ulp(kn_s).
-  * bf16 MLA out:   max-abs 2e-2, and >= 99.9 % of elements within one bf16 ulp.
+  * bf16 MLA out:   max-abs 2e-2 and |gpu - ref| <= ulp(ref) + 2^-8 max_j |v_j[c]|
+                    (bf16 softmax weights in the tensor-core PV product); lse 1e-4.
 """
 from __future__ import annotations
 
@@ -92,21 +93,47 @@ def assert_keys_close(gpu_keys, ref_keys, pool_valid, wl, first_valid):
     return dict(n=int(err.size), exact=float((err == 0).mean()), over_1ulp=over1)
 
 
-def assert_mla_close(gpu_out, ref_out, gpu_lse, ref_lse, rows=None):
+def mla_value_bound(kv_bits, req_start, q_req, token_ids):
+    """max_j |v_j[c]| over each query's selected latent rows: [Q, 512] (0 if none)."""
+    kv = bf16f(kv_bits) if kv_bits.dtype == np.uint16 else kv_bits
+    out = np.zeros((len(q_req), kv.shape[1]))
+    for i, b in enumerate(q_req):
+        T = req_start[b + 1] - req_start[b]
+        ids = token_ids[i][(token_ids[i] >= 0) & (token_ids[i] < T)]
+        if ids.size:
+            out[i] = np.abs(kv[req_start[b] + ids]).max(0)
+    return out
+
+
+def assert_mla_close(gpu_out, ref_out, gpu_lse, ref_lse, vbound=None, rows=None):
+    """MLA output parity.
+
+    The tensor-core PV product takes the softmax weights as bf16, so each weight
+    carries a relative rounding error of at most 2^-9. With the row sum taken
+    from the unrounded weights, out' - out = sum_j w_j e_j v_j / sum_j w_j, so
+    |out' - out| <= 2^-9 max_j |v_j[c]|; the bound used is ulp(ref) plus twice
+    that (fp32 accumulation and the exp2 approximation are far below it).
+    Also the spec max-abs 2e-2, and lse within 1e-4 (fp32 sums of
+    fp32 weights; one missing token among 2048 moves lse by ~1e-3).
+    """
     g, r = bf16f(gpu_out), bf16f(ref_out)
     if rows is not None:
         g, r = g[rows], r[rows]
         gpu_lse, ref_lse = gpu_lse[rows], ref_lse[rows]
+        if vbound is not None:
+            vbound = vbound[rows]
     err = np.abs(g - r)
     assert err.max(initial=0) <= 2e-2, f"mla out max-abs {err.max():.3g}"
-    within = (err <= bf16_ulp(r)).mean() if err.size else 1.0
-    assert within >= 0.999, f"mla out: only {within:.5f} within 1 bf16 ulp"
+    if vbound is not None:
+        bound = bf16_ulp(r) + 2.0 ** -8 * vbound[:, None, :]
+        assert (err <= bound).all(), f"mla out: {(err > bound).sum()} outside the weight-rounding bound"
+    within = float((err <= bf16_ulp(r)).mean()) if err.size else 1.0
     both_inf = np.isneginf(gpu_lse) & np.isneginf(ref_lse)
     assert (np.isneginf(gpu_lse) == np.isneginf(ref_lse)).all()
     lerr = np.abs(gpu_lse[~both_inf] - ref_lse[~both_inf])
-    assert lerr.max(initial=0) <= 1e-3, f"lse max-abs {lerr.max():.3g}"
-    return dict(max_abs=float(err.max(initial=0)), within_1ulp=float(within),
-                lse_max=float(lerr.max(initial=0)))
+    assert lerr.max(initial=0) <= 1e-4, f"lse max-abs {lerr.max():.3g}"
+    return dict(max_abs=float(err.max(initial=0)), rms=float(np.sqrt((err ** 2).mean())) if err.size else 0.0,
+                within_1ulp=within, lse_max=float(lerr.max(initial=0)))
 
 
 @functools.lru_cache(maxsize=8)

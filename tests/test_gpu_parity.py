@@ -12,7 +12,7 @@ import torch
 import oracle as O
 from gpu_helpers import (assert_gate_close, assert_keys_close, assert_mla_close,
                          assert_scores_close, bf16f, dev_bits, device_status_clean, host_bits,
-                         score_magnitude, workload)
+                         mla_value_bound, score_magnitude, workload)
 from sparse_attention_indexer_head_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -69,7 +69,8 @@ def stagewise(wl, g, queries=None):
     # a7 on GPU token ids
     out, lse = O.sparse_mla(wl.q_mla[qs], wl.kv, wl.req_start, wl.q_req[qs], g["token_ids"][qs],
                             wl.sm_scale)
-    rep["mla"] = assert_mla_close(g["out"][qs], out, g["lse"][qs], lse)
+    vb = mla_value_bound(wl.kv, wl.req_start, wl.q_req[qs], g["token_ids"][qs])
+    rep["mla"] = assert_mla_close(g["out"][qs], out, g["lse"][qs], lse, vbound=vb)
     return rep
 
 
@@ -102,8 +103,9 @@ def end_to_end(wl, g, queries=None):
     assert swaps <= max(1, 0.01 * K * len(qs)), f"{swaps} swapped pools"
     if agree_rows:
         rows = np.asarray(agree_rows)
+        vb = mla_value_bound(wl.kv, wl.req_start, wl.q_req[qs[rows]], ref["token_ids"][rows])
         assert_mla_close(g["out"][qs[rows]], ref["out"][rows], g["lse"][qs[rows]],
-                         ref["lse"][rows])
+                         ref["lse"][rows], vbound=vb)
     return dict(swaps=swaps, agree=len(agree_rows))
 
 
@@ -256,7 +258,7 @@ def test_mla_heads_and_id_edge_cases(B, hm):
     B.dsa_sparse_mla_decode(dev_bits(q), dev_bits(kv), d(rs), d(q_req), d(ids), 4, 3, hm, Wd, 512,
                             0, scale, out, lse, ws, ws_n)
     go, gl = host_bits(out), lse.cpu().numpy()
-    assert_mla_close(go, ref_out, gl, ref_lse)
+    assert_mla_close(go, ref_out, gl, ref_lse, vbound=mla_value_bound(kv, rs, q_req, ids))
     assert (go[2] == 0).all() and np.isneginf(gl[2]).all()      # empty request
     np.testing.assert_array_equal(go[3, 0], kv[123])                # single token: its row
     device_status_clean(B)
