@@ -55,7 +55,7 @@ constexpr float kLazyRescale = 8.0f;                // log2 units
 
 struct TcCtl {
     uint64_t kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2];
-    uint64_t o_done, q_full, fin;
+    uint64_t o_done, o_final, q_full, fin;
     uint64_t vmask[2];
     int32_t ids[2][kTcChunk];
     float alpha[kTcHeads];
@@ -140,6 +140,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             mbar_init(&ctl->p_empty[i], 1);
         }
         mbar_init(&ctl->o_done, 1);
+        mbar_init(&ctl->o_final, 1);
         mbar_init(&ctl->q_full, 128);
         mbar_init(&ctl->fin, 1);
         ctl->abort = 0;
@@ -188,7 +189,9 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                 tc::mma_commit(&ctl->s_full[s]);
                 if (c >= 1 && !issue_pv(c - 1)) { ok = false; break; }
             }
-            if (ok) issue_pv(nch - 1);
+            // o_final is single-use: once it completes every PV of this CTA has landed
+            // (a parity wait on o_done cannot tell the last two PVs apart).
+            if (ok && issue_pv(nch - 1)) tc::mma_commit(&ctl->o_final);
         }
         __syncwarp();
     } else if (warp < 4) {
@@ -333,7 +336,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         // ------------------------------------------------------------------ epilogue
         bool have_o = !failed && nch > 0;
         if (have_o) {
-            const bool bad = !tc_wait(ctl, &ctl->o_done, (nch - 1) & 1);
+            const bool bad = !tc_wait(ctl, &ctl->o_final, 0);
             have_o = !tc::named_bar_or(2, 128, bad);
         }
         if (owner) ctl->lsum[hh] = l;

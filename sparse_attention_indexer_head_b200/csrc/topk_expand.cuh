@@ -178,10 +178,15 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     __syncthreads();
 
     // Bitonic sort, descending. Element i is always handled by thread i mod 512,
-    // so a stage whose partner distance is below 32 stays inside one warp and
-    // needs only a warp barrier.
+    // so a stage whose partner distance is below 32 stays inside one warp: two
+    // consecutive such stages need only a warp barrier between them, any other
+    // pair a block barrier.
+    int prev_stride = n2;   // the compaction above was block-wide
     for (int size = 2; size <= n2; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride >= 32 || prev_stride >= 32) __syncthreads();
+            else __syncwarp();
+            prev_stride = stride;
             for (int i = tid; i < n2; i += kTopkThreads) {
                 const int l = i ^ stride;
                 if (l > i) {
@@ -193,8 +198,6 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
                     }
                 }
             }
-            if (stride >= 32) __syncthreads();
-            else __syncwarp();
         }
     }
     __syncthreads();
