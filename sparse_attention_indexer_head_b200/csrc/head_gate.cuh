@@ -3,9 +3,9 @@
 // [M,4096]x[4096,16] product that cuBLAS served with two CTAs).
 //
 // B200 design: K is split across a thread-block cluster of 8 CTAs; each CTA
-// owns 16 rows and a K/8 slice. A CTA stages its slice of w in shared memory,
-// 16 lanes per row sweep the slice with 16-byte loads of hidden, the 16
-// partial sums per row are folded with half-warp shuffles, and the 8 CTAs'
+// owns 16 rows and a K/8 slice, staged in shared memory with all global loads
+// in flight at once. 16 warps sweep the slice with a bank-conflict-free lane
+// mapping, their partials are folded in a fixed order, and the 8 CTAs'
 // partials are summed through distributed shared memory in rank order. One
 // launch, no atomics, no workspace, deterministic.
 #pragma once
@@ -16,116 +16,118 @@ namespace dsa {
 
 constexpr int kGateRows = 16;      // rows of hidden per CTA
 constexpr int kGateSplit = 8;      // CTAs per cluster (K split)
-constexpr int kGateThreads = 256;  // 16 rows x 16 k-lanes
+constexpr int kGateThreads = 512;  // 16 warps
+constexpr int kGateWarps = kGateThreads / 32;
 constexpr int kGateMaxN = 16;
-constexpr int kGateMaxSlice = 512; // K-slice rows staged per pass
+constexpr int kGateSlice = 512;    // k rows staged per pass
+constexpr int kGateHStride = kGateSlice + 1;   // padded hidden rows: conflict-free column reads
+constexpr int kGateSmem = (kGateRows * kGateHStride + kGateSlice * kGateMaxN +
+                           kGateWarps * kGateRows * kGateMaxN + kGateRows * kGateMaxN) * 4;
 
+// Lane mapping inside a warp: lane = 2*m + half, so a lane owns row m and
+// columns 8*half .. 8*half+7. For each k the 16 rows read 16 different
+// hidden values (padded row stride: distinct banks) and the 32 lanes read only
+// two distinct 32-byte pieces of the w row (broadcast), so shared memory is
+// conflict-free. Warp w covers k rows w, w+16, w+32, ... of the slice.
 __global__ void __cluster_dims__(1, kGateSplit, 1) __launch_bounds__(kGateThreads)
 head_gate_kernel(const float *__restrict__ hidden, const float *__restrict__ w,
                  float *__restrict__ out, int M, int K, int N) {
-    __shared__ __align__(16) float ws[kGateMaxSlice * kGateMaxN];  // w slice, zero-padded to 16 cols
-    __shared__ float part[kGateRows * kGateMaxN];                   // this CTA's partial sums
+    extern __shared__ __align__(16) float gate_smem[];
+    float *hs = gate_smem;                                   // [16][513]
+    float *ws = hs + kGateRows * kGateHStride;               // [512][16], zero-padded columns
+    float *red = ws + kGateSlice * kGateMaxN;                // [16 warps][16][16]
+    float *part = red + kGateWarps * kGateRows * kGateMaxN;  // [16][16] this CTA's partial
 
-    const int tid = threadIdx.x;
-    const int j = tid & 15;            // k-lane within the row
-    const int r = tid >> 4;            // row within the CTA
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = blockIdx.y;       // == cluster CTA rank (cluster dims 1 x 8)
-    const int m = blockIdx.x * kGateRows + r;
+    const int m0 = blockIdx.x * kGateRows;
+    const int rows = min(kGateRows, M - m0);
 
-    // This CTA's K range, in multiples of 4 (16-byte vectors of hidden).
     const int k4 = K >> 2;
     const int per = (k4 + kGateSplit - 1) / kGateSplit;
     const int kb = min(K, rank * per * 4);
     const int ke = min(K, (rank + 1) * per * 4);
 
-    float acc[kGateMaxN];
+    const int m = lane >> 1, n0 = (lane & 1) * 8;
+    float acc[8];
 #pragma unroll
-    for (int n = 0; n < kGateMaxN; ++n) acc[n] = 0.f;
+    for (int n = 0; n < 8; ++n) acc[n] = 0.f;
 
-    // Each pass stages up to 512 rows of w and this thread's 8 vectors of hidden.
-    // All loads of a pass are issued before the first use, so one memory
-    // latency covers the pass instead of one per load.
     const bool w_vec = N == kGateMaxN && aligned16(w);
-    for (int k0 = kb; k0 < ke; k0 += kGateMaxSlice) {
-        const int len = min(kGateMaxSlice, ke - k0);
-        float4 hv[kGateMaxSlice / 64];
+    for (int k0 = kb; k0 < ke; k0 += kGateSlice) {
+        const int len = min(kGateSlice, ke - k0);
+        // -- stage: every load of the pass is issued before the first store
+        constexpr int HV = kGateRows * kGateSlice / 4 / kGateThreads;    // 4 float4 of hidden
+        constexpr int WV = kGateSlice * kGateMaxN / 4 / kGateThreads;    // 4 float4 of w
+        float4 hv[HV], wv[WV];
 #pragma unroll
-        for (int u = 0; u < kGateMaxSlice / 64; ++u) {
-            const int kk = 4 * j + 64 * u;
-            hv[u] = (m < M && kk < len)
-                        ? __ldg(reinterpret_cast<const float4 *>(hidden + (size_t)m * K + k0 + kk))
+        for (int u = 0; u < HV; ++u) {
+            const int i = tid + u * kGateThreads;          // i = r * 128 + c4
+            const int r = i >> 7, c4 = (i & 127) * 4;
+            hv[u] = (r < rows && c4 < len)
+                        ? __ldg(reinterpret_cast<const float4 *>(hidden + (size_t)(m0 + r) * K + k0 + c4))
                         : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        __syncthreads();   // the previous pass is done with ws
         if (w_vec) {
             const float4 *src = reinterpret_cast<const float4 *>(w + (size_t)k0 * kGateMaxN);
-            float4 tmp[kGateMaxSlice * kGateMaxN / 4 / kGateThreads];
 #pragma unroll
-            for (int u = 0; u < kGateMaxSlice * kGateMaxN / 4 / kGateThreads; ++u) {
+            for (int u = 0; u < WV; ++u) {
                 const int i = tid + u * kGateThreads;
-                tmp[u] = i < len * 4 ? __ldg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < kGateMaxSlice * kGateMaxN / 4 / kGateThreads; ++u) {
-                const int i = tid + u * kGateThreads;
-                if (i < len * 4) reinterpret_cast<float4 *>(ws)[i] = tmp[u];
+                wv[u] = i < len * 4 ? __ldg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         } else {
-            for (int i0 = 0; i0 < len * kGateMaxN; i0 += 8 * kGateThreads) {
-                float tmp[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int i = i0 + tid + u * kGateThreads;
-                    const int kk = i / kGateMaxN, n = i % kGateMaxN;
-                    tmp[u] = (i < len * kGateMaxN && n < N) ? __ldg(w + (size_t)(k0 + kk) * N + n)
-                                                            : 0.f;
-                }
+            for (int u = 0; u < WV; ++u) {
+                const int i = tid + u * kGateThreads;      // float4 index: row i/4, cols 4(i%4)..
+                const int kk = i >> 2, c = (i & 3) * 4;
+                float t[4];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int i = i0 + tid + u * kGateThreads;
-                    if (i < len * kGateMaxN) ws[i] = tmp[u];
-                }
+                for (int e = 0; e < 4; ++e)
+                    t[e] = (kk < len && c + e < N) ? __ldg(w + (size_t)(k0 + kk) * N + c + e) : 0.f;
+                wv[u] = make_float4(t[0], t[1], t[2], t[3]);
             }
         }
+        __syncthreads();   // the previous pass is done with hs / ws
+#pragma unroll
+        for (int u = 0; u < HV; ++u) {
+            const int i = tid + u * kGateThreads;
+            const int r = i >> 7, c4 = (i & 127) * 4;
+            float *d = hs + r * kGateHStride + c4;
+            d[0] = hv[u].x; d[1] = hv[u].y; d[2] = hv[u].z; d[3] = hv[u].w;
+        }
+#pragma unroll
+        for (int u = 0; u < WV; ++u)
+            reinterpret_cast<float4 *>(ws)[tid + u * kGateThreads] = wv[u];
         __syncthreads();
-#pragma unroll
-        for (int u = 0; u < kGateMaxSlice / 64; ++u) {
-            const int kk = 4 * j + 64 * u;
-            if (kk >= len) break;
-            const float hvu[4] = {hv[u].x, hv[u].y, hv[u].z, hv[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float4 *wr = reinterpret_cast<const float4 *>(ws + (kk + e) * kGateMaxN);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 wv = wr[q];
-                    acc[4 * q + 0] = fmaf(hvu[e], wv.x, acc[4 * q + 0]);
-                    acc[4 * q + 1] = fmaf(hvu[e], wv.y, acc[4 * q + 1]);
-                    acc[4 * q + 2] = fmaf(hvu[e], wv.z, acc[4 * q + 2]);
-                    acc[4 * q + 3] = fmaf(hvu[e], wv.w, acc[4 * q + 3]);
-                }
-            }
+        // -- 8 independent accumulators per lane; 32 k rows per warp per pass
+        const float *hrow = hs + m * kGateHStride;
+#pragma unroll 4
+        for (int kk = warp; kk < len; kk += kGateWarps) {
+            const float h = hrow[kk];
+            const float4 wa = *reinterpret_cast<const float4 *>(ws + kk * kGateMaxN + n0);
+            const float4 wb = *reinterpret_cast<const float4 *>(ws + kk * kGateMaxN + n0 + 4);
+            acc[0] = fmaf(h, wa.x, acc[0]); acc[1] = fmaf(h, wa.y, acc[1]);
+            acc[2] = fmaf(h, wa.z, acc[2]); acc[3] = fmaf(h, wa.w, acc[3]);
+            acc[4] = fmaf(h, wb.x, acc[4]); acc[5] = fmaf(h, wb.y, acc[5]);
+            acc[6] = fmaf(h, wb.z, acc[6]); acc[7] = fmaf(h, wb.w, acc[7]);
         }
     }
 
-    // Fold the 16 k-lanes of each row (a fixed butterfly order).
+    // Fold the 16 warps (fixed order), then the 8 cluster ranks (rank order).
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1)
+    for (int n = 0; n < 8; ++n) red[(warp * kGateRows + m) * kGateMaxN + n0 + n] = acc[n];
+    __syncthreads();
+    if (tid < kGateRows * kGateMaxN) {
+        float sum = 0.f;
 #pragma unroll
-        for (int n = 0; n < kGateMaxN; ++n) acc[n] += __shfl_xor_sync(0xffffffffu, acc[n], off);
-    if (j == 0) {
-#pragma unroll
-        for (int n = 0; n < kGateMaxN; ++n) part[r * kGateMaxN + n] = acc[n];
+        for (int w2 = 0; w2 < kGateWarps; ++w2) sum += red[w2 * kGateRows * kGateMaxN + tid];
+        part[tid] = sum;
     }
-
-    // Cluster-wide: every CTA's partials visible, then rank c sums rows c and
-    // c + 8 over the 8 ranks in rank order.
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
     if (tid < 2 * kGateMaxN) {
         const int rr = rank + (tid >= kGateMaxN ? kGateSplit : 0);
         const int n = tid % kGateMaxN;
-        const int mm = blockIdx.x * kGateRows + rr;
         const uint32_t local = smem_u32(&part[rr * kGateMaxN + n]);
         float v[kGateSplit];
 #pragma unroll
@@ -137,7 +139,7 @@ head_gate_kernel(const float *__restrict__ hidden, const float *__restrict__ w,
         float s = 0.f;
 #pragma unroll
         for (int c = 0; c < kGateSplit; ++c) s += v[c];
-        if (mm < M && n < N) out[(size_t)mm * N + n] = s;
+        if (rr < rows && n < N) out[(size_t)(m0 + rr) * N + n] = s;
     }
     // Keep this CTA's shared memory alive until every rank has read it.
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
@@ -154,7 +156,9 @@ inline int head_gate_launch(const float *hidden, const float *w, float *out, int
     const int row_blocks = ceil_div(M, kGateRows);
     if (row_blocks > 65535 * 16) return DSA_ERR_UNSUPPORTED;
     dim3 grid(row_blocks, kGateSplit);
-    head_gate_kernel<<<grid, kGateThreads, 0, stream>>>(hidden, w, out, M, K, N);
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(head_gate_kernel), kGateSmem))
+        return DSA_ERR_CUDA;
+    head_gate_kernel<<<grid, kGateThreads, kGateSmem, stream>>>(hidden, w, out, M, K, N);
     return launch_status();
 }
 

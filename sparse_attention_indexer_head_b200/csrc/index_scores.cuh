@@ -6,11 +6,9 @@
 //   cand = pool_valid[b,p] && last slot token of p <= q_pos[q]
 //   score = sum_h gate_w[q,h] * max(0, <q_idx[q,h,:], key[b,p,:]>), -inf if !cand.
 //
-// Kernel: a CTA scores 128 pools of one query, one thread per pool. The query
-// (16 heads x 128 channels) sits transposed in shared memory as fp32 and is
-// read by broadcast; the pool key row is read with 16-byte loads. Each head's
-// 128-term dot runs as 4 interleaved fp32 chains of 32 terms joined pairwise
-// (shorter chains keep the rounding error near the pairwise bound). Keys of
+// Kernel: a CTA scores 32 pools of one query with four threads per pool (four
+// heads each). The query (16 heads x 128 channels) sits transposed in shared
+// memory as fp32; the pool key row is read with 16-byte loads. Keys of
 // non-candidates are never read.
 #pragma once
 
@@ -18,9 +16,16 @@
 
 namespace dsa {
 
-constexpr int kScoreThreads = 128;
-constexpr int kScoreHeads = DSA_MAX_INDEX_HEADS;   // 16
+constexpr int kScoreThreads = 128;                   // 32 pools x 4 head groups
+constexpr int kScorePools = kScoreThreads / 4;
+constexpr int kScoreHeads = DSA_MAX_INDEX_HEADS;     // 16
 
+// Thread (pool, hq) computes heads 4hq..4hq+3 of one pool over all 128
+// channels (two interleaved fp32 chains per head), adds g_h * relu(dot_h) for
+// its heads, and the four head groups of a pool are folded with two shuffles
+// in a fixed order. The four lanes of a pool read the same 256-byte key row
+// (served by L1 after the first); q is read from shared memory as one
+// broadcast 16-byte load per channel.
 __global__ void __launch_bounds__(kScoreThreads)
 index_scores_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__restrict__ gate_w,
                     const int32_t *__restrict__ q_req, const int32_t *__restrict__ q_pos, int H,
@@ -47,57 +52,46 @@ index_scores_kernel(const __nv_bfloat16 *__restrict__ q_idx, const float *__rest
     if (tid < kScoreHeads) gs[tid] = (req_ok && tid < H) ? gate_w[(size_t)q * H + tid] : 0.f;
     __syncthreads();
 
-    const int p = blockIdx.x * kScoreThreads + tid;
-    if (p >= max_pools) return;
-    const size_t out_i = (size_t)q * max_pools + p;
+    const int hq = tid & 3;
+    const int p = blockIdx.x * kScorePools + (tid >> 2);
     bool is_cand = false;
-    if (req_ok) {
+    if (req_ok && p < max_pools) {
         const long long last = (long long)first_valid[b] + (long long)p * kpool + kpool - 1;
         is_cand = pool_valid[(size_t)b * max_pools + p] != 0 && last <= (long long)q_pos[q];
     }
-    if (!is_cand) {
-        scores[out_i] = -INFINITY;
-        cand[out_i] = 0;
-        return;
-    }
-
-    const __nv_bfloat16 *key = pool_keys + ((size_t)b * max_pools + p) * kD;
-    uint4 kr[kD / 8];   // the whole 256-byte key row: 16 loads in flight at once
+    float part = 0.f;
+    if (is_cand) {
+        const __nv_bfloat16 *key = pool_keys + ((size_t)b * max_pools + p) * kD;
+        uint4 kr[kD / 8];   // the whole key row: 16 loads in flight at once
 #pragma unroll
-    for (int c8 = 0; c8 < kD / 8; ++c8) kr[c8] = ldg_nc_v4(key + 8 * c8);
-
-    float acc[4][kScoreHeads];
+        for (int c8 = 0; c8 < kD / 8; ++c8) kr[c8] = ldg_nc_v4(key + 8 * c8);
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+        for (int c8 = 0; c8 < kD / 8; ++c8) {
+            float kv[8];
+            unpack8(kr[c8], kv);
 #pragma unroll
-        for (int h = 0; h < kScoreHeads; ++h) acc[u][h] = 0.f;
-
-#pragma unroll
-    for (int c8 = 0; c8 < kD / 8; ++c8) {
-        float kv[8];
-        unpack8(kr[c8], kv);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float4 *qr = reinterpret_cast<const float4 *>(qs + (8 * c8 + j) * kScoreHeads);
-            const int u = j & 3;
-#pragma unroll
-            for (int h4 = 0; h4 < 4; ++h4) {
-                const float4 qv = qr[h4];
-                acc[u][4 * h4 + 0] = fmaf(qv.x, kv[j], acc[u][4 * h4 + 0]);
-                acc[u][4 * h4 + 1] = fmaf(qv.y, kv[j], acc[u][4 * h4 + 1]);
-                acc[u][4 * h4 + 2] = fmaf(qv.z, kv[j], acc[u][4 * h4 + 2]);
-                acc[u][4 * h4 + 3] = fmaf(qv.w, kv[j], acc[u][4 * h4 + 3]);
+            for (int j = 0; j < 8; ++j) {
+                const float4 qv = *reinterpret_cast<const float4 *>(qs + (8 * c8 + j) * kScoreHeads + 4 * hq);
+                float *a = acc[j & 1];
+                a[0] = fmaf(qv.x, kv[j], a[0]);
+                a[1] = fmaf(qv.y, kv[j], a[1]);
+                a[2] = fmaf(qv.z, kv[j], a[2]);
+                a[3] = fmaf(qv.w, kv[j], a[3]);
             }
         }
-    }
-    float s = 0.f;
 #pragma unroll
-    for (int h = 0; h < kScoreHeads; ++h) {
-        const float d = (acc[0][h] + acc[1][h]) + (acc[2][h] + acc[3][h]);
-        s = fmaf(gs[h], fmaxf(d, 0.f), s);
+        for (int u = 0; u < 4; ++u)
+            part = fmaf(gs[4 * hq + u], fmaxf(acc[0][u] + acc[1][u], 0.f), part);
     }
-    scores[out_i] = s;
-    cand[out_i] = 1;
+    // Fold the four head groups of the pool: (g0 + g1) + (g2 + g3).
+    part += __shfl_xor_sync(0xffffffffu, part, 1);
+    part += __shfl_xor_sync(0xffffffffu, part, 2);
+    if (hq == 0 && p < max_pools) {
+        const size_t out_i = (size_t)q * max_pools + p;
+        scores[out_i] = is_cand ? part : -INFINITY;
+        cand[out_i] = is_cand ? 1 : 0;
+    }
 }
 
 inline int index_scores_launch(const void *q_idx, const float *gate_w, const int32_t *q_req,
@@ -116,7 +110,7 @@ inline int index_scores_launch(const void *q_idx, const float *gate_w, const int
     if (!aligned(q_idx, 16) || !aligned(gate_w, 4) || !aligned(q_req, 4) || !aligned(q_pos, 4) ||
         !aligned(pool_keys, 16) || !aligned(first_valid, 4) || !aligned(scores, 4))
         return DSA_ERR_ALIGNMENT;
-    dim3 grid(ceil_div(max_pools, kScoreThreads), Q);
+    dim3 grid(ceil_div(max_pools, kScorePools), Q);
     index_scores_kernel<<<grid, kScoreThreads, 0, stream>>>(
         reinterpret_cast<const __nv_bfloat16 *>(q_idx), gate_w, q_req, q_pos, H,
         reinterpret_cast<const __nv_bfloat16 *>(pool_keys), pool_valid, first_valid, B, kpool,

@@ -21,11 +21,18 @@
 
 namespace dsa {
 
-constexpr int kCmpConsumers = 256;                 // 8 consumer warps
-constexpr int kCmpThreads = kCmpConsumers + 32;   // + 1 producer warp
-constexpr int kCmpTileTokens = 128;               // token rows per tile (k and gate each)
-constexpr int kCmpStages = 3;
-constexpr int kCmpStageBytes = 2 * kCmpTileTokens * 128 * 2;   // 64 KB: k rows | gate rows
+// Geometry per kpool: small pools get 12 consumer warps and 96-token tiles in a
+// 4-stage ring; kpool > 4 (more live registers per lane) 8 warps and 128-token
+// tiles in a 3-stage ring. A stage holds the tile's k rows then its gate rows.
+template <int KP> struct CmpCfg {
+    static constexpr int kWarps = KP <= 4 ? 12 : 8;             // consumer warps
+    static constexpr int kConsumers = kWarps * 32;
+    static constexpr int kThreads = kConsumers + 32;            // + 1 producer warp
+    static constexpr int kTileTokens = KP <= 4 ? 96 : 128;
+    static constexpr int kStages = KP <= 4 ? 4 : 3;
+    static constexpr int kStageBytes = 2 * kTileTokens * 128 * 2;
+    static constexpr int kTP = kTileTokens / KP;                // pools per tile
+};
 constexpr int kD = DSA_INDEX_DIM;   // 128 channels
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -71,71 +78,117 @@ DSA_DEVINL float hsum16(float v) {
 }
 
 // One pool on a half-warp: lane l owns channels 8l..8l+7 of the kpool slot rows
-// at krow/grow (shared memory). Returns the packed bf16 pooled key chunk (zero
-// when the pool is invalid).
+// at krow/grow (shared memory), held as four fp32 pairs so the arithmetic runs
+// as packed fp32x2 (FFMA2 / FADD2 / FMUL2) instructions. Returns the packed
+// bf16 pooled key chunk (zero when the pool is invalid).
+DSA_DEVINL void unpack8x2(const uint4 &v, float2 (&x)[4]) {
+    x[0] = make_float2(bf16lo(v.x), bf16hi(v.x));
+    x[1] = make_float2(bf16lo(v.y), bf16hi(v.y));
+    x[2] = make_float2(bf16lo(v.z), bf16hi(v.z));
+    x[3] = make_float2(bf16lo(v.w), bf16hi(v.w));
+}
+
+// Round a pair to bf16 (nearest even) and widen it back: the stored k_norm value.
+DSA_DEVINL float2 round_bf16x2(float2 y) {
+    const uint32_t p = pack_bf16x2(y.x, y.y);
+    return make_float2(bf16lo(p), bf16hi(p));
+}
+
 template <int KP>
 DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *grow,
-                               const float *s_ape, const float (&lw)[8], const float (&lb)[8],
+                               const float *s_ape, const float2 (&lw)[4], const float2 (&lb)[4],
                                float eps, int l, bool ok) {
-    // Pass 1: LayerNorm statistics and pool logits (log2 units) per slot.
-    float mean[KP], rstd[KP], lg[KP][8];
+    // kpool <= 4: the k rows and slot logits stay in registers between the two
+    // passes; larger pools re-read them from shared memory (register budget).
+    constexpr bool kKeep = KP <= 4;
+    const float2 log2e2 = make_float2(kLog2e, kLog2e);
+    float2 xk[kKeep ? KP : 1][4], lgk[kKeep ? KP : 1][4];
+    float rr[KP], nmr[KP];
+    float2 mx2[4];
 #pragma unroll
-    for (int s = 0; s < KP; ++s) {
-        float x[8];
-        unpack8(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
-        float sum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) sum += x[c];
-        const float mu = hsum16(sum) * (1.0f / kD);
-        float sq = 0.f;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const float d = x[c] - mu;
-            sq = fmaf(d, d, sq);
-        }
-        const float var = hsum16(sq) * (1.0f / kD);
-        mean[s] = mu;
-        rstd[s] = __frsqrt_rn(var + eps);
-        float g[8];
-        unpack8(*reinterpret_cast<const uint4 *>(grow + s * kD), g);
+    for (int c = 0; c < 4; ++c) mx2[c] = make_float2(-INFINITY, -INFINITY);
+
+    auto logits = [&](int s, float2 (&lg)[4]) {
+        float2 g[4];
+        unpack8x2(*reinterpret_cast<const uint4 *>(grow + s * kD), g);
         const float4 a0 = *reinterpret_cast<const float4 *>(s_ape + s * kD + 8 * l);
         const float4 a1 = *reinterpret_cast<const float4 *>(s_ape + s * kD + 8 * l + 4);
-        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        lg[0] = __ffma2_rn(g[0], log2e2, make_float2(a0.x, a0.y));
+        lg[1] = __ffma2_rn(g[1], log2e2, make_float2(a0.z, a0.w));
+        lg[2] = __ffma2_rn(g[2], log2e2, make_float2(a1.x, a1.y));
+        lg[3] = __ffma2_rn(g[3], log2e2, make_float2(a1.z, a1.w));
+    };
+
+    // Pass 1: LayerNorm statistics (two-pass mean / variance) and the running
+    // max of the slot logits (log2 units), per slot.
 #pragma unroll
-        for (int c = 0; c < 8; ++c) lg[s][c] = fmaf(g[c], kLog2e, av[c]);
+    for (int s = 0; s < KP; ++s) {
+        float2 x[4];
+        unpack8x2(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
+        const float2 s2 = __fadd2_rn(__fadd2_rn(x[0], x[1]), __fadd2_rn(x[2], x[3]));
+        const float mu = hsum16(s2.x + s2.y) * (1.0f / kD);
+        float2 q2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float2 d = __fadd2_rn(x[c], make_float2(-mu, -mu));
+            q2 = __ffma2_rn(d, d, q2);
+        }
+        const float var = hsum16(q2.x + q2.y) * (1.0f / kD);
+        rr[s] = __frsqrt_rn(var + eps);
+        nmr[s] = -mu * rr[s];
+        float2 lg[4];
+        logits(s, lg);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            mx2[c] = make_float2(fmaxf(mx2[c].x, lg[c].x), fmaxf(mx2[c].y, lg[c].y));
+            if constexpr (kKeep) {
+                xk[s][c] = x[c];
+                lgk[s][c] = lg[c];
+            }
+        }
     }
-    // Pass 2: per-channel softmax over slots, weighted sum of the bf16 k_norm rows.
-    float mx[8], den[8], acc[8];
+    // Pass 2: per-channel softmax over the slots, weighted sum of the bf16 k_norm rows.
+    float2 nmx[4], den[4], acc[4];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        mx[c] = lg[0][c];
-#pragma unroll
-        for (int s = 1; s < KP; ++s) mx[c] = fmaxf(mx[c], lg[s][c]);
-        den[c] = 0.f;
-        acc[c] = 0.f;
+    for (int c = 0; c < 4; ++c) {
+        nmx[c] = make_float2(-mx2[c].x, -mx2[c].y);
+        den[c] = make_float2(0.f, 0.f);
+        acc[c] = make_float2(0.f, 0.f);
     }
 #pragma unroll
     for (int s = 0; s < KP; ++s) {
-        float x[8];
-        unpack8(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
+        float2 x[4], lg[4];
+        if constexpr (kKeep) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const float y = fmaf((x[c] - mean[s]) * rstd[s], lw[c], lb[c]);
-            const float kn = round_bf16(y);
-            const float e = ex2(lg[s][c] - mx[c]);
-            den[c] += e;
-            acc[c] = fmaf(e, kn, acc[c]);
+            for (int c = 0; c < 4; ++c) {
+                x[c] = xk[s][c];
+                lg[c] = lgk[s][c];
+            }
+        } else {
+            unpack8x2(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
+            logits(s, lg);
+        }
+        const float2 r2 = make_float2(rr[s], rr[s]), nmr2 = make_float2(nmr[s], nmr[s]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float2 t = __ffma2_rn(x[c], r2, nmr2);              // (x - mu) * rstd
+            const float2 kn = round_bf16x2(__ffma2_rn(t, lw[c], lb[c]));
+            const float2 z = __fadd2_rn(lg[c], nmx[c]);
+            const float2 e = make_float2(ex2(z.x), ex2(z.y));
+            den[c] = __fadd2_rn(den[c], e);
+            acc[c] = __ffma2_rn(e, kn, acc[c]);
         }
     }
     uint4 o = make_uint4(0, 0, 0, 0);
     if (ok) {
-        float v[8];
+        uint32_t w[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) v[c] = __fdiv_rn(acc[c], den[c]);
-        o.x = pack_bf16x2(v[0], v[1]);
-        o.y = pack_bf16x2(v[2], v[3]);
-        o.z = pack_bf16x2(v[4], v[5]);
-        o.w = pack_bf16x2(v[6], v[7]);
+        for (int c = 0; c < 4; ++c) {
+            const float2 inv = make_float2(__frcp_rn(den[c].x), __frcp_rn(den[c].y));
+            const float2 v = __fmul2_rn(acc[c], inv);
+            w[c] = pack_bf16x2(v.x, v.y);
+        }
+        o = make_uint4(w[0], w[1], w[2], w[3]);
     }
     return o;
 }
@@ -150,7 +203,7 @@ struct CmpMeta {
 // contiguous k and gate rows into a 3-stage shared-memory ring with two 1-D
 // bulk copies per tile. Warps 0-7 consume: a half-warp per pool.
 template <int KP>
-__global__ void __launch_bounds__(kCmpThreads, 1)
+__global__ void __launch_bounds__(CmpCfg<KP>::kThreads, 1)
 kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ gate,
                       const uint8_t *__restrict__ valid, const int32_t *__restrict__ req_start,
                       int B, int max_pools, int tiles_per_req, int n_tiles,
@@ -158,7 +211,13 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
                       const __nv_bfloat16 *__restrict__ ln_b, float eps,
                       __nv_bfloat16 *__restrict__ pool_keys, int32_t *__restrict__ pool_idx,
                       uint8_t *__restrict__ pool_valid, int32_t *__restrict__ first_valid) {
-    constexpr int TP = kCmpTileTokens / KP;   // pools per tile
+    using C = CmpCfg<KP>;
+    constexpr int TP = C::kTP;
+    constexpr int kCmpStages = C::kStages;
+    constexpr int kCmpStageBytes = C::kStageBytes;
+    constexpr int kCmpTileTokens = C::kTileTokens;
+    constexpr int kCmpConsumers = C::kConsumers;
+    constexpr int kCmpThreads = C::kThreads;
     extern __shared__ __align__(128) uint8_t cmp_smem[];
     __shared__ __align__(16) float s_ape[KP * kD];   // ape * log2(e)
     __shared__ __align__(8) uint64_t full[kCmpStages], empty[kCmpStages];
@@ -219,9 +278,9 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     // -------------------------------------------------------------------- consumer warps
     const int hw = tid >> 4;     // half-warp: one pool at a time
     const int l = tid & 15;      // channels 8l .. 8l+7
-    float lw[8], lb[8];
-    unpack8(ldg_nc_v4(ln_w + 8 * l), lw);
-    unpack8(ldg_nc_v4(ln_b + 8 * l), lb);
+    float2 lw[4], lb[4];
+    unpack8x2(ldg_nc_v4(ln_w + 8 * l), lw);
+    unpack8x2(ldg_nc_v4(ln_b + 8 * l), lb);
 
     for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
         const int s = i % kCmpStages;
@@ -268,15 +327,16 @@ inline int kpool_compress_launch_kp(const __nv_bfloat16 *k, const __nv_bfloat16 
                                     int max_pools, const float *ape, const __nv_bfloat16 *ln_w,
                                     const __nv_bfloat16 *ln_b, float eps, __nv_bfloat16 *keys,
                                     int32_t *idx, uint8_t *pv, int32_t *fv, cudaStream_t stream) {
-    constexpr int TP = kCmpTileTokens / KP;
-    const int smem = kCmpStages * kCmpStageBytes;
+    using C = CmpCfg<KP>;
+    constexpr int TP = C::kTP;
+    const int smem = C::kStages * C::kStageBytes;
     if (!ensure_smem_attr(reinterpret_cast<const void *>(kpool_compress_kernel<KP>), smem))
         return DSA_ERR_CUDA;
     const int tiles_per_req = max(1, ceil_div(max_pools, TP));
     const long long n_tiles = (long long)tiles_per_req * B;
     if (n_tiles > (1ll << 30)) return DSA_ERR_UNSUPPORTED;
     const int grid = (int)std::min<long long>(n_tiles, sm_count());
-    kpool_compress_kernel<KP><<<grid, kCmpThreads, smem, stream>>>(
+    kpool_compress_kernel<KP><<<grid, C::kThreads, smem, stream>>>(
         k, gate, valid, req_start, B, max_pools, tiles_per_req, (int)n_tiles, ape, ln_w, ln_b, eps,
         keys, idx, pv, fv);
     return launch_status();

@@ -56,6 +56,57 @@ DSA_DEVINL int block_excl_scan(int v, int *s_warp, int *total) {
     return before;
 }
 
+// One warp-local bitonic stage in registers: v is element i, its partner is
+// i ^ stride (same warp since stride < 32); the lower index of a pair keeps the
+// larger key when the run of `size` containing it sorts descending.
+DSA_DEVINL unsigned long long bitonic_reg_stage(unsigned long long v, int i, int size, int stride) {
+    const unsigned long long p = __shfl_xor_sync(0xffffffffu, v, stride);
+    const bool desc = (i & size) == 0;
+    const bool lower = (i & stride) == 0;
+    const bool keep_max = lower == desc;
+    return keep_max ? (v > p ? v : p) : (v < p ? v : p);
+}
+
+// In-place descending bitonic sort of a[0..n2) in shared memory (n2 a power of
+// two, at most 8 * kTopkThreads). Called by the whole block.
+DSA_DEVINL void bitonic_sort_desc(unsigned long long *a, int n2) {
+    const int tid = threadIdx.x;
+    const int R = (n2 + kTopkThreads - 1) / kTopkThreads;   // elements per thread
+    auto reg_round = [&](int size_lo, int size_hi, int first_stride) {
+        // sizes size_lo..size_hi (powers of two); the first size starts at
+        // first_stride, later ones at size/2; every stride here is < 32.
+        for (int r = 0; r < R; ++r) {
+            const int i = tid + r * kTopkThreads;
+            unsigned long long v = i < n2 ? a[i] : 0ull;
+            for (int size = size_lo; size <= size_hi; size <<= 1)
+                for (int stride = (size == size_lo ? first_stride : size >> 1); stride > 0; stride >>= 1)
+                    v = bitonic_reg_stage(v, i, size, stride);
+            if (i < n2) a[i] = v;
+        }
+    };
+    __syncthreads();
+    reg_round(2, min(n2, 32), 1);
+    for (int size = 64; size <= n2; size <<= 1) {
+        for (int stride = size >> 1; stride >= 32; stride >>= 1) {
+            __syncthreads();
+            for (int i = tid; i < n2; i += kTopkThreads) {
+                const int l = i ^ stride;
+                if (l > i) {
+                    const unsigned long long x = a[i], y = a[l];
+                    const bool desc = (i & size) == 0;
+                    if (desc ? (x < y) : (x > y)) {
+                        a[i] = y;
+                        a[l] = x;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        reg_round(size, size, 16);
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(kTopkThreads)
 topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__ cand,
                    const int32_t *__restrict__ pool_idx, const int32_t *__restrict__ q_req, int B,
@@ -177,31 +228,12 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     for (int i = nq + tid; i < n2; i += kTopkThreads) slist[i] = 0ull;
     __syncthreads();
 
-    // Bitonic sort, descending. Element i is always handled by thread i mod 512,
-    // so a stage whose partner distance is below 32 stays inside one warp: two
-    // consecutive such stages need only a warp barrier between them, any other
-    // pair a block barrier.
-    int prev_stride = n2;   // the compaction above was block-wide
-    for (int size = 2; size <= n2; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            if (stride >= 32 || prev_stride >= 32) __syncthreads();
-            else __syncwarp();
-            prev_stride = stride;
-            for (int i = tid; i < n2; i += kTopkThreads) {
-                const int l = i ^ stride;
-                if (l > i) {
-                    const unsigned long long a = slist[i], c = slist[l];
-                    const bool desc = (i & size) == 0;
-                    if (desc ? (a < c) : (a > c)) {
-                        slist[i] = c;
-                        slist[l] = a;
-                    }
-                }
-            }
-        }
-    }
-    __syncthreads();
-
+    // Bitonic sort, descending, of n2 (a power of two, <= 4096) composite keys.
+    // Element i lives with thread i mod 512. Stages whose partner distance is
+    // below 32 stay inside a warp and run in registers with shuffles; the
+    // others (partner distance >= 32) run in shared memory between block
+    // barriers: 10 of the 45 stages for 512 elements.
+    bitonic_sort_desc(slist, n2);
     for (int j = tid; j < K; j += kTopkThreads)
         top_pools[(size_t)q * K + j] = j < nq ? (int32_t)(~(uint32_t)slist[j]) : -1;
     for (int e = tid; e < K * KP; e += kTopkThreads) {
