@@ -26,49 +26,53 @@ constexpr int kPartStride = kL + 4;
 // ---------------------------------------------------------------------------------------
 // tcgen05 split-KV kernel. One CTA per (split, query, group of 64 heads).
 //
-// Per chunk of 64 selected tokens:
-//   S[64 heads x 64 tokens]   = Q[64 x 512] . KV[64 x 512]^T   (M=64, N=64, 32 K-steps)
+// Per chunk of 32 selected tokens:
+//   S[64 heads x 32 tokens]   = Q[64 x 512] . KV[32 x 512]^T   (M=64, N=32, 32 K-steps)
 //   softmax over the chunk's tokens, per head row, in registers (one thread per head)
-//   O^T[512 x 64 heads]      += KV^T[512 x 64] . P^T[64 x 64]  (4 x M=128, N=64, 4 K-steps)
+//   O^T[512 x 64 heads]      += KV^T[512 x 32] . P^T[32 x 64]  (4 x M=128, N=64, 2 K-steps)
 // The latent row is both key and value (NoPE), so one 128B-swizzled shared tile
 // of the gathered rows serves as the K-major B operand of S and as the MN-major A
 // operand of O^T. Accumulators live in tensor memory: O^T in columns [0,256)
-// (all 128 lanes), S double-buffered in columns [256,384) (lanes 0-15 of each
+// (all 128 lanes), S double-buffered in columns [256,320) (lanes 0-15 of each
 // 32-lane quadrant, the M=64 layout).
 //
 // Warp roles (256 threads): warp 0 allocates tensor memory and one lane issues
-// every MMA; warps 1-3 gather the chunk's latent rows with 16-byte cp.async into
-// the swizzled layout (zero rows for ids that are -1 or outside the request);
-// warps 4-7 load Q, run the softmax (lane i < 16 of warp 4+w owns head 16w+i),
-// rescale O^T when a head's running max grows by more than 2^8 (lazy
-// rescaling), and write the epilogue.
+// every MMA; warps 1-3 gather, warp 1+(c mod 3) filling chunk c into a 4-stage
+// ring with 16-byte cp.async into the swizzled layout (zero rows for ids that are
+// -1 or outside the request; the next chunk's ids are prefetched), so up to
+// three chunks are in flight; warps 4-7 load Q, run the softmax (lane i < 16 of
+// warp 4+w owns head 16w+i), rescale O^T when a head's running max grows by
+// more than 2^8 (lazy rescaling), and write the epilogue.
 // ---------------------------------------------------------------------------------------
 constexpr int kTcThreads = 256;
-constexpr int kTcChunk = 64;
+constexpr int kTcChunk = 32;                        // tokens per chunk
+constexpr int kTcStages = 4;                        // gathered-row ring depth
 constexpr int kTcHeads = 64;
 constexpr uint32_t kOffQ = 0;                       // 64 KB: 8 atoms x [64 rows x 128 B]
-constexpr uint32_t kOffKV = 64 * 1024;              // 2 stages x 64 KB
-constexpr uint32_t kOffP = 192 * 1024;              // 2 buffers x 8 KB
-constexpr uint32_t kOffCtl = 208 * 1024;
+constexpr uint32_t kOffKV = 64 * 1024;              // 4 stages x 32 KB: 8 atoms x [32 rows x 128 B]
+constexpr uint32_t kStageKV = 32 * 1024;
+constexpr uint32_t kAtomKV = kTcChunk * 128;        // 4 KB: one 64-latent column of a stage
+constexpr uint32_t kOffP = 192 * 1024;              // 2 buffers x 4 KB: [64 heads x 64 B], 64B swizzle
+constexpr uint32_t kStageP = 4 * 1024;
+constexpr uint32_t kOffCtl = 200 * 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLazyRescale = 8.0f;                // log2 units
 
 struct TcCtl {
-    uint64_t kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2];
+    uint64_t kv_full[kTcStages], kv_empty[kTcStages];
+    uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
     uint64_t o_done, o_final, q_full, fin;
-    uint64_t vmask[2];
-    int32_t ids[2][kTcChunk];
+    uint32_t vmask[kTcStages];
     float alpha[kTcHeads];
     float lsum[kTcHeads];
     uint32_t tmem_base;
     volatile int abort;
-    int prod_abort[2];   // per chunk parity: read after the gather barrier of that chunk
 };
 constexpr int kTcSmemBytes = (int)kOffCtl + (int)sizeof(TcCtl) + 1024;   // + alignment slack
 
 struct MlaGeom {
     int S;      // splits per query
-    int per;    // selected-id slots per split (a multiple of 64)
+    int per;    // selected-id slots per split (a multiple of the chunk)
 };
 
 inline MlaGeom mla_geometry(int Q, int Hm, int W) {
@@ -112,8 +116,8 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     uint8_t *gbase = mla_smem_raw + (base - raw);
     TcCtl *ctl = reinterpret_cast<TcCtl *>(gbase + kOffCtl);
     const uint32_t sQ = base + kOffQ;
-    const uint32_t sKV[2] = {base + kOffKV, base + kOffKV + 64 * 1024};
-    const uint32_t sP[2] = {base + kOffP, base + kOffP + 8 * 1024};
+    const uint32_t sKV = base + kOffKV;                      // stage s at sKV + s * kStageKV
+    const uint32_t sP = base + kOffP;                        // buffer b at sP + b * kStageP
 
     const int split = blockIdx.x, qi = blockIdx.y, hg = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -131,9 +135,11 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         tc::tmem_relinquish();
     }
     if (tid == 32) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&ctl->kv_full[i], 96);
+        for (int i = 0; i < kTcStages; ++i) {
+            mbar_init(&ctl->kv_full[i], 32);
             mbar_init(&ctl->kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&ctl->s_full[i], 1);
             mbar_init(&ctl->s_empty[i], 128);
             mbar_init(&ctl->p_full[i], 128);
@@ -154,39 +160,44 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     if (warp == 0) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0 && nch > 0) {
-            constexpr uint32_t idS = tc::idesc_bf16(64, 64, false, false);
+            constexpr uint32_t idS = tc::idesc_bf16(64, kTcChunk, false, false);
             constexpr uint32_t idPV = tc::idesc_bf16(128, 64, true, false);
             auto issue_pv = [&](int cp) -> bool {
-                const int sp = cp & 1;
-                if (!tc_wait(ctl, &ctl->p_full[sp], (cp >> 1) & 1)) return false;
+                const int sp = cp % kTcStages, pb = cp & 1;
+                if (!tc_wait(ctl, &ctl->p_full[pb], (cp >> 1) & 1)) return false;
                 tc::fence_after_sync();
+                const uint32_t kvs = sKV + sp * kStageKV;
 #pragma unroll
                 for (int lb = 0; lb < 4; ++lb)
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t a = tc::desc_sw128(sKV[sp] + lb * 2 * 8192 + ks * 2048, 8192, 1024);
-                        const uint64_t bd = tc::desc_sw128(sP[sp] + ks * 32, 16, 1024);
+                    for (int ks = 0; ks < kTcChunk / 16; ++ks) {
+                        // V^T: MN-major, 64-latent atoms kAtomKV apart, 8-token groups 1 KB apart
+                        const uint64_t a = tc::desc_sw128(kvs + lb * 2 * kAtomKV + ks * 2048, kAtomKV, 1024);
+                        // P^T: K-major, 64-byte rows, 8-head groups 512 B apart
+                        const uint64_t bd = tc::desc_sw64(sP + pb * kStageP + ks * 32, 16, 512);
                         tc::mma_bf16_ss(tmem + lb * 64, a, bd, idPV, (cp > 0 || ks > 0) ? 1u : 0u);
                     }
                 tc::mma_commit(&ctl->kv_empty[sp]);
-                tc::mma_commit(&ctl->p_empty[sp]);
+                tc::mma_commit(&ctl->p_empty[pb]);
                 tc::mma_commit(&ctl->o_done);
                 return true;
             };
             bool ok = tc_wait(ctl, &ctl->q_full, 0);
             for (int c = 0; ok && c < nch; ++c) {
-                const int s = c & 1;
-                if (!tc_wait(ctl, &ctl->kv_full[s], (c >> 1) & 1)) { ok = false; break; }
-                if (c >= 2 && !tc_wait(ctl, &ctl->s_empty[s], ((c >> 1) - 1) & 1)) { ok = false; break; }
+                const int s = c % kTcStages, sb = c & 1;
+                if (!tc_wait(ctl, &ctl->kv_full[s], (c / kTcStages) & 1)) { ok = false; break; }
+                if (c >= 2 && !tc_wait(ctl, &ctl->s_empty[sb], ((c >> 1) - 1) & 1)) { ok = false; break; }
                 tc::fence_after_sync();
-                const uint32_t d = tmem + 256 + s * 64;
+                const uint32_t d = tmem + 256 + sb * kTcChunk;
+                const uint32_t kvs = sKV + s * kStageKV;
 #pragma unroll
                 for (int kk = 0; kk < kL / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    tc::mma_bf16_ss(d, tc::desc_sw128(sQ + off, 16, 1024),
-                                    tc::desc_sw128(sKV[s] + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+                    const uint32_t qo = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    const uint32_t ko = (kk >> 2) * kAtomKV + (kk & 3) * 32;
+                    tc::mma_bf16_ss(d, tc::desc_sw128(sQ + qo, 16, 1024),
+                                    tc::desc_sw128(kvs + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
                 }
-                tc::mma_commit(&ctl->s_full[s]);
+                tc::mma_commit(&ctl->s_full[sb]);
                 if (c >= 1 && !issue_pv(c - 1)) { ok = false; break; }
             }
             // o_final is single-use: once it completes every PV of this CTA has landed
@@ -195,39 +206,38 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         }
         __syncwarp();
     } else if (warp < 4) {
-        // ------------------------------------------------------------------ gather (96 threads)
-        const int pt = tid - 32;
-        for (int c = 0; c < nch; ++c) {
-            const int s = c & 1;
-            if (pt == 0) {
-                if (c >= 2) tc_wait(ctl, &ctl->kv_empty[s], ((c >> 1) - 1) & 1);
-                ctl->prod_abort[s] = ctl->abort;
-            }
-            if (pt < 32) {
-                uint32_t m2[2];
+        // ------------------------------------------------------------------ gather warps
+        // Warp 1+p fills chunks p, p+3, p+6, ...; lane r owns row r's id.
+        const int pw = warp - 1;
+        auto load_id = [&](int c) -> int {
+            const int j = c * kTcChunk + lane;
+            return (c < nch && j < ntok) ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
+        };
+        int next_id = load_id(pw);
+        for (int c = pw; c < nch; c += 3) {
+            const int s = c % kTcStages;
+            const int id = next_id;
+            next_id = load_id(c + 3);                      // in flight during this chunk's copies
+            bool ok = true;
+            if (c >= kTcStages) ok = tc_wait(ctl, &ctl->kv_empty[s], ((c / kTcStages) - 1) & 1);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const bool valid = id >= 0 && id < T;
+            const uint32_t vm = __ballot_sync(0xffffffffu, valid);
+            const int myid = valid ? id : -1;
+            const uint32_t dst0 = sKV + s * kStageKV;
+            for (int r = 0; r < kTcChunk; ++r) {
+                const int rid = __shfl_sync(0xffffffffu, myid, r);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const int r = pt + 32 * hh;
-                    const int j = c * kTcChunk + r;
-                    const int id = j < ntok ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
-                    const bool ok = id >= 0 && id < T;
-                    m2[hh] = __ballot_sync(0xffffffffu, ok);
-                    ctl->ids[s][r] = ok ? id : -1;
+                    const int cc = lane + 32 * hh;         // 16-byte piece of the 1 KB row
+                    const uint32_t dst = dst0 + (cc >> 3) * kAtomKV + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
+                    if (rid >= 0)
+                        tc::cp_async16(dst, kv + ((size_t)rs + rid) * kL + cc * 8);
+                    else
+                        tc::st_shared_zero16(dst);
                 }
-                if (pt == 0) ctl->vmask[s] = (uint64_t)m2[0] | ((uint64_t)m2[1] << 32);
             }
-            tc::named_bar_sync(1, 96);
-            if (ctl->prod_abort[s]) break;
-            const uint32_t dst0 = sKV[s];
-            for (int x = pt; x < kTcChunk * 64; x += 96) {
-                const int r = x >> 6, cc = x & 63;
-                const int id = ctl->ids[s][r];
-                const uint32_t dst = dst0 + (cc >> 3) * 8192 + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
-                if (id >= 0)
-                    tc::cp_async16(dst, kv + ((size_t)rs + id) * kL + cc * 8);
-                else
-                    tc::st_shared_zero16(dst);
-            }
+            if (lane == 0) ctl->vmask[s] = vm;
             tc::cp_async_wait_all();
             tc::fence_proxy_async_smem();
             mbar_arrive(&ctl->kv_full[s]);
@@ -257,25 +267,23 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         float m_used = -INFINITY, l = 0.f;
         bool failed = false;
         for (int c = 0; c < nch; ++c) {
-            const int s = c & 1;
-            bool bad = !tc_wait(ctl, &ctl->kv_full[s], (c >> 1) & 1);
-            bad = bad || !tc_wait(ctl, &ctl->s_full[s], (c >> 1) & 1);
+            const int s = c % kTcStages, sb = c & 1;
+            bool bad = !tc_wait(ctl, &ctl->kv_full[s], (c / kTcStages) & 1);
+            bad = bad || !tc_wait(ctl, &ctl->s_full[sb], (c >> 1) & 1);
             if (tc::named_bar_or(2, 128, bad)) { failed = true; break; }
             tc::fence_after_sync();
-            uint32_t r[2][32];
-            tc::tmem_ld32(tl + 256 + s * 64, r[0]);
-            tc::tmem_ld32(tl + 256 + s * 64 + 32, r[1]);
+            uint32_t r[kTcChunk];
+            tc::tmem_ld32(tl + 256 + sb * kTcChunk, r);
             tc::tmem_wait_ld();
             tc::fence_before_sync();
-            mbar_arrive(&ctl->s_empty[s]);
+            mbar_arrive(&ctl->s_empty[sb]);
 
-            const uint64_t vm = ctl->vmask[s];
+            const uint32_t vm = ctl->vmask[s];
             float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                const float z = ((vm >> j) & 1) ? __uint_as_float(r[j >> 5][j & 31]) * scale_log2
-                                                : -INFINITY;
-                r[j >> 5][j & 31] = __float_as_uint(z);
+            for (int j = 0; j < kTcChunk; ++j) {
+                const float z = ((vm >> j) & 1) ? __uint_as_float(r[j]) * scale_log2 : -INFINITY;
+                r[j] = __float_as_uint(z);
                 mx = fmaxf(mx, z);
             }
             float alpha = 1.f;
@@ -283,12 +291,11 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                 alpha = ex2(m_used - mx);
                 m_used = mx;
             }
-            uint32_t pk[32];
+            uint32_t pk[kTcChunk / 2];
             float psum = 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float z0 = __uint_as_float(r[(2 * j) >> 5][(2 * j) & 31]);
-                const float z1 = __uint_as_float(r[(2 * j + 1) >> 5][(2 * j + 1) & 31]);
+            for (int j = 0; j < kTcChunk / 2; ++j) {
+                const float z0 = __uint_as_float(r[2 * j]), z1 = __uint_as_float(r[2 * j + 1]);
                 const float p0 = z0 == -INFINITY ? 0.f : ex2(z0 - m_used);
                 const float p1 = z1 == -INFINITY ? 0.f : ex2(z1 - m_used);
                 pk[j] = pack_bf16x2(p0, p1);
@@ -297,16 +304,16 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             l = fmaf(l, alpha, psum);
             if (owner) ctl->alpha[hh] = alpha;
 
-            bad = c >= 2 && !tc_wait(ctl, &ctl->p_empty[s], ((c >> 1) - 1) & 1);
+            bad = c >= 2 && !tc_wait(ctl, &ctl->p_empty[sb], ((c >> 1) - 1) & 1);
             if (tc::named_bar_or(2, 128, bad)) { failed = true; break; }
             const bool need = tc::named_bar_or(2, 128, owner && c >= 1 && alpha != 1.f);
             if (owner) {
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    const uint32_t dst = sP[s] + hh * 128 + ((c8 ^ (hh & 7)) << 4);
+                for (int c4 = 0; c4 < kTcChunk / 8; ++c4) {
+                    const uint32_t dst = sP + sb * kStageP + hh * 64 + ((c4 ^ ((hh >> 1) & 3)) << 4);
                     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
-                                 "r"(pk[4 * c8]), "r"(pk[4 * c8 + 1]), "r"(pk[4 * c8 + 2]),
-                                 "r"(pk[4 * c8 + 3])
+                                 "r"(pk[4 * c4]), "r"(pk[4 * c4 + 1]), "r"(pk[4 * c4 + 2]),
+                                 "r"(pk[4 * c4 + 3])
                                  : "memory");
                 }
             }
@@ -330,7 +337,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                 tc::fence_before_sync();
             }
             tc::fence_proxy_async_smem();
-            mbar_arrive(&ctl->p_full[s]);
+            mbar_arrive(&ctl->p_full[sb]);
         }
 
         // ------------------------------------------------------------------ epilogue

@@ -20,6 +20,12 @@ DSA_DEVINL uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_
            ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// Same with the 64-byte swizzle (layout 4): rows of 64 bytes, 8-row atoms of 512 bytes.
+DSA_DEVINL uint64_t desc_sw64(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
+}
+
 // -- instruction descriptor, kind::f16 with bf16 inputs and an f32 accumulator ---------
 // bits [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,
 // bit 15 A major (1 = MN), bit 16 B major, [17,23) N >> 3, [24,29) M >> 4.
@@ -91,6 +97,17 @@ DSA_DEVINL void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
 }
 #undef DSA_R8
 #undef DSA_W8
+
+// 16 consecutive 32-bit columns of this thread's lane.
+DSA_DEVINL void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
 
 DSA_DEVINL void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 DSA_DEVINL void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
