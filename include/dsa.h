@@ -187,6 +187,37 @@ int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *
                           float *lse, void *workspace, size_t workspace_bytes,
                           dsa_stream_t stream);
 
+/*
+ * dsa_sparse_mla_decode without a workspace argument. The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory where they call the MLA: code that runs on an execution path whose
+ * memory is fixed before it starts (an engine that reserves every buffer at
+ * start-up and forbids allocation per step, or a plugin that only receives
+ * the input and output pointers of the op it implements). Such a caller has
+ * nowhere to take the split-KV scratch from, so this variant uses a scratch
+ * area owned by the library instead.
+ *   Arguments, outputs and refusals are those of dsa_sparse_mla_decode, and
+ *   the computation and results are the same.
+ *   The scratch is a static device array of DSA_NOALLOC_SCRATCH_BYTES bytes
+ *   that every GPU which loads the library keeps until the process exits. A
+ *   call whose split-KV scratch (dsa_sparse_mla_workspace_size(Q, Hm, W))
+ *   exceeds it returns DSA_ERR_WORKSPACE and launches nothing.
+ *   Nothing is allocated or freed: no cudaMalloc, no cudaFree, no allocating
+ *   library routine. The first call on a device looks up the scratch's device
+ *   address (cudaGetSymbolAddress, with that device current); make that first
+ *   call before any stream capture on that device.
+ *   Every call shares the one scratch area and leaves its last contents there;
+ *   nothing in it needs to start at zero (every value the merge reads is
+ *   written by the same call first). Calls whose kernels may overlap on the
+ *   GPU -- on different streams without ordering between them -- race on the
+ *   scratch and must not be made.
+ */
+#define DSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+int dsa_sparse_mla_decode_noalloc(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *req_start,
+                                  const int32_t *q_req, const int32_t *token_ids, int Q, int B,
+                                  int Hm, int W, int kv_lora, int rope_dim, float sm_scale,
+                                  dsa_bf16 *out, float *lse, dsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,8 +26,9 @@ DSA_ERR_CUDA = 5
 EXPORTS = (
     "dsa_status_string", "dsa_abi_version", "dsa_device_status", "dsa_head_gate",
     "dsa_kpool_compress", "dsa_index_scores", "dsa_topk_expand",
-    "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_decode",
+    "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_decode", "dsa_sparse_mla_decode_noalloc",
 )
+DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class DsaError(RuntimeError):
@@ -54,6 +55,7 @@ def _load() -> ctypes.CDLL:
         "dsa_topk_expand": ([P, P, P, P, I, I, I, I, I, P, P, P], I),
         "dsa_sparse_mla_workspace_size": ([I, I, I], Z),
         "dsa_sparse_mla_decode": ([P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P], I),
+        "dsa_sparse_mla_decode_noalloc": ([P, P, P, P, P, I, I, I, I, I, I, F, P, P, P], I),
     }
     for name, (argtypes, restype) in sig.items():
         fn = getattr(L, name)
@@ -142,3 +144,13 @@ def dsa_sparse_mla_decode(q, kv, req_start, q_req, token_ids, Q: int, B: int, Hm
         _ptr(q), _ptr(kv), _ptr(req_start), _ptr(q_req), _ptr(token_ids), Q, B, Hm, W, kv_lora,
         rope_dim, float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace), int(workspace_bytes),
         _stream(stream)))
+
+
+def dsa_sparse_mla_decode_noalloc(q, kv, req_start, q_req, token_ids, Q: int, B: int, Hm: int,
+                                  W: int, kv_lora: int, rope_dim: int, sm_scale: float, out, lse,
+                                  stream=None) -> None:
+    """dsa_sparse_mla_decode for callers that cannot allocate: the split-KV scratch is the
+    library's own static device area (see include/dsa.h)."""
+    _check("dsa_sparse_mla_decode_noalloc", lib.dsa_sparse_mla_decode_noalloc(
+        _ptr(q), _ptr(kv), _ptr(req_start), _ptr(q_req), _ptr(token_ids), Q, B, Hm, W, kv_lora,
+        rope_dim, float(sm_scale), _ptr(out), _ptr(lse), _stream(stream)))

@@ -8,6 +8,39 @@
 #include "topk_expand.cuh"
 #include "sparse_mla.cuh"
 
+#include <mutex>
+
+// ---------------------------------------------------------------------------------------
+// Library-owned scratch for dsa_sparse_mla_decode_noalloc: the split-KV partial
+// rows that dsa_sparse_mla_decode keeps in the caller's workspace. It is a
+// file-scope device array, so every GPU that loads this library holds
+// DSA_NOALLOC_SCRATCH_BYTES of it until the process exits. In host code the
+// name g_mla_scratch only stands in for the symbol; its device address comes
+// from cudaGetSymbolAddress, looked up once per device (with that device
+// current) on the first call made on it.
+// ---------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_mla_scratch[DSA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_addr[kMaxDevices] = {};
+
+int scratch_address(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_mla_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return DSA_OK;
+}
+}  // namespace
+
 extern "C" {
 
 const char *dsa_status_string(int status) {
@@ -80,6 +113,25 @@ int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *
                           dsa_stream_t stream) {
     return dsa::sparse_mla_launch(q, kv, req_start, q_req, token_ids, Q, B, Hm, W, kv_lora,
                                   rope_dim, sm_scale, out, lse, workspace, workspace_bytes,
+                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dsa_sparse_mla_decode_noalloc(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *req_start,
+                                  const int32_t *q_req, const int32_t *token_ids, int Q, int B,
+                                  int Hm, int W, int kv_lora, int rope_dim, float sm_scale,
+                                  dsa_bf16 *out, float *lse, dsa_stream_t stream) {
+    size_t need = 0;
+    if (Q > 0 && Hm > 0 && W >= 0) {
+        need = dsa::mla_workspace_bytes(Q, Hm, W);
+        if (need > (size_t)DSA_NOALLOC_SCRATCH_BYTES) return DSA_ERR_WORKSPACE;
+    }
+    void *scratch = nullptr;
+    if (need > 0) {
+        const int st = scratch_address(&scratch);
+        if (st != DSA_OK) return st;
+    }
+    return dsa::sparse_mla_launch(q, kv, req_start, q_req, token_ids, Q, B, Hm, W, kv_lora,
+                                  rope_dim, sm_scale, out, lse, scratch, need,
                                   reinterpret_cast<cudaStream_t>(stream));
 }
 
