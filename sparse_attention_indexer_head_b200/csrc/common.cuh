@@ -110,6 +110,19 @@ DSA_DEVINL float ex2(float x) {
     return y;
 }
 
+// MUFU reciprocal / reciprocal square root (relative error about 2^-23); used
+// where the result is rounded to bf16 afterwards.
+DSA_DEVINL float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+DSA_DEVINL float rsqrt_approx(float x) {
+    float y;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <typename T>
 DSA_DEVINL T ldg_nc(const T *p) { return __ldg(p); }
 

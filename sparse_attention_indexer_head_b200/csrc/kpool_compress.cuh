@@ -125,16 +125,28 @@ DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *g
     for (int s = 0; s < KP; ++s) {
         float2 x[4];
         unpack8x2(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
-        const float2 s2 = __fadd2_rn(__fadd2_rn(x[0], x[1]), __fadd2_rn(x[2], x[3]));
-        const float mu = hsum16(s2.x + s2.y) * (1.0f / kD);
-        float2 q2 = make_float2(0.f, 0.f);
+        // Shifted one-pass moments: sums of d = x - x0 and d^2 with x0 the row's
+        // channel 0 (within a few standard deviations of the mean, so the
+        // difference of moments does not cancel); both reduced in one chain.
+        const float x0 = __shfl_sync(0xffffffffu, x[0].x, 0, 16);
+        const float2 nx0 = make_float2(-x0, -x0);
+        float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            const float2 d = __fadd2_rn(x[c], make_float2(-mu, -mu));
-            q2 = __ffma2_rn(d, d, q2);
+            const float2 d = __fadd2_rn(x[c], nx0);
+            s1 = __fadd2_rn(s1, d);
+            s2 = __ffma2_rn(d, d, s2);
         }
-        const float var = hsum16(q2.x + q2.y) * (1.0f / kD);
-        rr[s] = __frsqrt_rn(var + eps);
+        float a1 = s1.x + s1.y, a2 = s2.x + s2.y;
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) {
+            a1 += __shfl_xor_sync(0xffffffffu, a1, off);
+            a2 += __shfl_xor_sync(0xffffffffu, a2, off);
+        }
+        const float dm = a1 * (1.0f / kD);
+        const float var = fmaxf(fmaf(-dm, dm, a2 * (1.0f / kD)), 0.f);
+        const float mu = x0 + dm;
+        rr[s] = rsqrt_approx(var + eps);
         nmr[s] = -mu * rr[s];
         float2 lg[4];
         logits(s, lg);
@@ -184,7 +196,7 @@ DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *g
         uint32_t w[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            const float2 inv = make_float2(__frcp_rn(den[c].x), __frcp_rn(den[c].y));
+            const float2 inv = make_float2(rcp_approx(den[c].x), rcp_approx(den[c].y));
             const float2 v = __fmul2_rn(acc[c], inv);
             w[c] = pack_bf16x2(v.x, v.y);
         }
@@ -195,6 +207,7 @@ DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *g
 
 struct CmpMeta {
     int b, p0, p1, n_in, f, rs;
+    uint32_t okmask[4];   // bit i: pool p0+i has every slot valid (i < 128)
 };
 
 // Persistent kernel: CTA c owns a contiguous range of (request, pool-tile) work
@@ -257,8 +270,26 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             const int p1 = min(p0 + TP, max_pools);
             const int n_span = min(max_pools, (cur_T - cur_f) / KP);
             const int n_in = max(0, min(p1, n_span) - p0);
+            // Pool validity for the tile (all slot tokens valid), one pool per lane,
+            // computed here so the consumers never wait on a global load.
+            uint32_t okm[4] = {0u, 0u, 0u, 0u};
+            const size_t tok_base = (size_t)cur_rs + cur_f + (size_t)p0 * KP;
+#pragma unroll
+            for (int w4 = 0; w4 < 4; ++w4) {
+                if (32 * w4 >= n_in) break;
+                const int i = 32 * w4 + lane;
+                bool pv = i < n_in;
+                if (pv) {
+                    uint8_t vb[KP];
+#pragma unroll
+                    for (int ss = 0; ss < KP; ++ss) vb[ss] = valid[tok_base + (size_t)i * KP + ss];
+#pragma unroll
+                    for (int ss = 0; ss < KP; ++ss) pv = pv && vb[ss] != 0;
+                }
+                okm[w4] = __ballot_sync(0xffffffffu, pv);
+            }
             if (lane == 0) {
-                meta[s] = CmpMeta{b, p0, p1, n_in, cur_f, cur_rs};
+                meta[s] = CmpMeta{b, p0, p1, n_in, cur_f, cur_rs, {okm[0], okm[1], okm[2], okm[3]}};
                 if (n_in > 0) {
                     const uint32_t bytes = (uint32_t)(n_in * KP * kD * 2);
                     const size_t row0 = (size_t)cur_rs + cur_f + (size_t)p0 * KP;
@@ -303,11 +334,7 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             const bool active = ii + (hw & 1) < m.n_in;
             const int pi = active ? ii + (hw & 1) : ii;
             const int p = m.p0 + pi;
-            // Slot validity: lane s < KP reads the valid byte of slot token s.
-            const size_t tok0 = (size_t)m.rs + m.f + (size_t)p * KP;
-            const bool lane_ok = l >= KP || valid[tok0 + l] != 0;
-            const uint32_t half_mask = 0xFFFFu << (tid & 16);
-            const bool ok = (__ballot_sync(0xffffffffu, lane_ok) & half_mask) == half_mask;
+            const bool ok = (m.okmask[pi >> 5] >> (pi & 31)) & 1u;
             const uint4 o = compress_pool<KP>(sk + (size_t)pi * KP * kD + 8 * l,
                                               sg + (size_t)pi * KP * kD + 8 * l, s_ape, lw, lb,
                                               eps, l, ok);

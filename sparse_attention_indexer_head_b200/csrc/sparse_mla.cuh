@@ -247,19 +247,17 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         const int st = tid - 128, wq = warp - 4;
         const int hh = 16 * wq + lane;        // head row owned by lanes 0..15
         const bool owner = lane < 16;
-        // Q tile: 64 rows x 64 16-byte chunks into the swizzled K-major layout.
+        // Q tile: 64 rows x 64 16-byte chunks into the swizzled K-major layout, all
+        // 32 copies of a thread in flight at once.
         for (int x = st; x < kTcHeads * 64; x += 128) {
             const int h = x >> 6, cc = x & 63;
             const uint32_t dst = sQ + (cc >> 3) * 8192 + h * 128 + (((cc & 7) ^ (h & 7)) << 4);
-            if (h < nh) {
-                const uint4 v = ldg_nc_v4(qm + ((size_t)qi * Hm + h0 + h) * kL + cc * 8);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x),
-                             "r"(v.y), "r"(v.z), "r"(v.w)
-                             : "memory");
-            } else {
+            if (h < nh)
+                tc::cp_async16(dst, qm + ((size_t)qi * Hm + h0 + h) * kL + cc * 8);
+            else
                 tc::st_shared_zero16(dst);
-            }
         }
+        tc::cp_async_wait_all();
         tc::fence_proxy_async_smem();
         mbar_arrive(&ctl->q_full);
 

@@ -131,11 +131,24 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
         return req_ok ? score_key(srow[p], crow[p] != 0) : 0u;
     };
 
+    // Keys: four loads of each array in flight per thread before any use.
     int cnt = 0;
-    for (int p = tid; p < P; p += kTopkThreads) {
-        const uint32_t k = req_ok ? score_key(srow[p], crow[p] != 0) : 0u;
-        if (keys_in_smem) skeys[p] = k;
-        cnt += k != 0u;
+    for (int p0 = 0; p0 < P; p0 += 4 * kTopkThreads) {
+        float sv[4];
+        uint8_t cv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int p = p0 + tid + u * kTopkThreads;
+            sv[u] = (req_ok && p < P) ? srow[p] : 0.f;
+            cv[u] = (req_ok && p < P) ? crow[p] : (uint8_t)0;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int p = p0 + tid + u * kTopkThreads;
+            const uint32_t k = score_key(sv[u], cv[u] != 0);
+            if (keys_in_smem && p < P) skeys[p] = k;
+            cnt += k != 0u;
+        }
     }
     int n_cand;
     (void)block_excl_scan(cnt, s_warp, &n_cand);
@@ -236,14 +249,24 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     bitonic_sort_desc(slist, n2);
     for (int j = tid; j < K; j += kTopkThreads)
         top_pools[(size_t)q * K + j] = j < nq ? (int32_t)(~(uint32_t)slist[j]) : -1;
-    for (int e = tid; e < K * KP; e += kTopkThreads) {
-        const int j = e / KP, s = e - j * KP;
-        int32_t v = -1;
-        if (j < nq) {
-            const int pid = (int)(~(uint32_t)slist[j]);
-            v = pool_idx[((size_t)b * P + pid) * KP + s];
+    // Expansion: four pool_idx gathers in flight per thread before the stores.
+    for (int e0 = 0; e0 < K * KP; e0 += 4 * kTopkThreads) {
+        int32_t v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = e0 + tid + u * kTopkThreads;
+            const int j = e / KP, s = e - j * KP;
+            v[u] = -1;
+            if (e < K * KP && j < nq) {
+                const int pid = (int)(~(uint32_t)slist[j]);
+                v[u] = pool_idx[((size_t)b * P + pid) * KP + s];
+            }
         }
-        token_ids[(size_t)q * K * KP + e] = v;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = e0 + tid + u * kTopkThreads;
+            if (e < K * KP) token_ids[(size_t)q * K * KP + e] = v[u];
+        }
     }
 }
 
