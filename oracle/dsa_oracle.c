@@ -278,9 +278,11 @@ int orc_index_scores(const uint16_t *q_idx, const float *gate_w, const int32_t *
  * a5+a6: topk_pools and expand_selection [mod.rs, "Shape of the pipeline"
  * third and fourth arrows; Glm5NextDsaConfig::select_k and out_width; trap 6].
  *   Candidates of query q are ranked by (score descending, pool id ascending)
- *   (READING: lowest pool id wins ties; a NaN score ranks as -inf).
- *   n_q = min(select_k, #candidates); top_pools[q, j] is the j-th ranked pool
- *   for j < n_q and -1 after.
+ *   (READING: lowest pool id wins ties; a NaN score ranks as -inf), and the
+ *   n_q = min(select_k, #candidates) best are selected.
+ *   READING: the page fixes which pools are selected, not their order in the
+ *   row; top_pools[q, :n_q] lists the selected pools in ascending pool id, and
+ *   -1 after.
  *   token_ids[q, j*kpool + s] = pool_idx[b, top_pools[q, j], s] for j < n_q and
  *   -1 for every later slot: out_width = select_k * kpool with the tail
  *   option off, and the -1 sentinel row is written in full.
@@ -293,6 +295,11 @@ static int orc_rank_cmp(const void *pa, const void *pb) {
     float sb = isnan(b->score) ? -INFINITY : b->score;
     if (sa > sb) return -1;
     if (sa < sb) return 1;
+    return (a->id > b->id) - (a->id < b->id);
+}
+
+static int orc_id_cmp(const void *pa, const void *pb) {
+    const orc_cand_t *a = (const orc_cand_t *)pa, *b = (const orc_cand_t *)pb;
     return (a->id > b->id) - (a->id < b->id);
 }
 
@@ -317,6 +324,7 @@ int orc_topk_expand(const float *scores, const uint8_t *cand, const int32_t *poo
                 }
             qsort(list, (size_t)n, sizeof(orc_cand_t), orc_rank_cmp);
             int nq = n < select_k ? n : select_k;
+            qsort(list, (size_t)nq, sizeof(orc_cand_t), orc_id_cmp);   /* selected set by id */
             int b = q_req[q];
             for (int j = 0; j < select_k; ++j) {
                 int pid = j < nq ? list[j].id : -1;

@@ -371,7 +371,8 @@ def test_topk_vs_sorted_with_ties(orc):
     for q in range(Q):
         cands = [p for p in range(P) if cand[q, p]]
         ranked = sorted(cands, key=lambda p: (-float(scores[q, p]), p))[:K]
-        expect = ranked + [-1] * (K - len(ranked))
+        chosen = sorted(ranked)              # the selected set, listed by pool id
+        expect = chosen + [-1] * (K - len(chosen))
         assert list(top[q]) == expect
         exp_ids = sum(([2 + p * kp + s for s in range(kp)] if p >= 0 else [-1] * kp
                        for p in expect), [])
@@ -392,10 +393,13 @@ def test_topk_all_equal_and_width(orc):
 
 
 def test_topk_nan_ranks_as_neg_inf(orc):
-    scores = np.array([[np.nan, -np.inf, 1.0, -5.0]], np.float32)
-    cand = np.ones((1, 4), np.uint8)
-    top, _ = orc.topk_expand(scores, cand, _pool_idx(4, 1), np.zeros(1, np.int32), 4)
-    assert list(top[0]) == [2, 3, 0, 1]
+    scores = np.array([[np.nan, -np.inf, 1.0, -5.0, 0.5]], np.float32)
+    cand = np.ones((1, 5), np.uint8)
+    # ranking 2 > 4 > 3 > {0 (NaN as -inf), 1 (-inf)}, tie -> lower id: 0 before 1
+    top, _ = orc.topk_expand(scores, cand, _pool_idx(5, 1), np.zeros(1, np.int32), 4)
+    assert list(top[0]) == [0, 2, 3, 4]
+    top, _ = orc.topk_expand(scores, cand, _pool_idx(5, 1), np.zeros(1, np.int32), 3)
+    assert list(top[0]) == [2, 3, 4]
 
 
 # --------------------------------------------------------------------------- a7 sparse MLA
