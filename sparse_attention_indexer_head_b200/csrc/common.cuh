@@ -82,12 +82,18 @@ DSA_DEVINL bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete. Gives up after a bounded
-// number of polls (each poll may itself suspend for a while), raises the device
-// error flag and returns false.
+// Wait for the phase with the given parity to complete. Gives up once about two
+// seconds of SM clock cycles have passed (each try_wait may itself suspend for
+// a while, so the bound is on elapsed cycles, not on the number of polls),
+// raises the device error flag and returns false.
+constexpr long long kWaitLimitCycles = 4000000000ll;
 DSA_DEVINL bool mbar_wait(uint64_t *bar, uint32_t phase) {
-    for (uint32_t i = 0; i < (1u << 24); ++i)
+    if (mbar_try_wait(bar, phase)) return true;
+    const long long t0 = clock64();
+    for (;;) {
         if (mbar_try_wait(bar, phase)) return true;
+        if (clock64() - t0 > kWaitLimitCycles) break;
+    }
     raise_device_error(kErrWaitTimeout);
     return false;
 }
