@@ -136,9 +136,38 @@ DSA_DEVINL bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p
 
 DSA_DEVINL uint4 ldg_nc_v4(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Every kernel of the path is launched with programmatic stream serialization:
+// it may start while its predecessor in the stream is still running. Each
+// kernel therefore (1) does only setup that reads nothing a predecessor writes
+// and writes nothing a predecessor reads, (2) waits for the predecessor grid to
+// complete (griddepcontrol.wait; a no-op without the launch attribute), then
+// (3) lets its own successor start launching. A kernel thus overlaps only its
+// immediate predecessor, whose own wait has already returned, so everything
+// earlier has completed.
+DSA_DEVINL void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+DSA_DEVINL void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- host-side checks
 inline bool aligned(const void *p, uintptr_t a) {
     return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+// Launch with the programmatic-stream-serialization attribute (see pdl_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 inline int launch_status() {

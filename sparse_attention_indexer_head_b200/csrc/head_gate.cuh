@@ -113,6 +113,11 @@ head_gate_kernel(const float *__restrict__ hidden, const float *__restrict__ w,
         }
     }
 
+    // Loads and arithmetic above touch only the step's inputs; from here on the
+    // CTA writes shared state and then the output, after the predecessor grid.
+    pdl_wait();
+    pdl_launch_dependents();
+
     // Fold the 16 warps (fixed order), then the 8 cluster ranks (rank order).
 #pragma unroll
     for (int n = 0; n < 8; ++n) red[(warp * kGateRows + m) * kGateMaxN + n0 + n] = acc[n];
@@ -158,7 +163,9 @@ inline int head_gate_launch(const float *hidden, const float *w, float *out, int
     dim3 grid(row_blocks, kGateSplit);
     if (!ensure_smem_attr(reinterpret_cast<const void *>(head_gate_kernel), kGateSmem))
         return DSA_ERR_CUDA;
-    head_gate_kernel<<<grid, kGateThreads, kGateSmem, stream>>>(hidden, w, out, M, K, N);
+    if (launch_pdl(head_gate_kernel, grid, dim3(kGateThreads), kGateSmem, stream, hidden, w, out,
+                   M, K, N) != cudaSuccess)
+        return DSA_ERR_CUDA;
     return launch_status();
 }
 

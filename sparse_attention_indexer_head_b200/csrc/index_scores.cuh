@@ -51,17 +51,6 @@ index_scores_kernel(const __grid_constant__ CUtensorMap key_map,
     const int tid = threadIdx.x, warp = tid >> 5;
     const int p0 = blockIdx.x * kScorePools;
     const int p = p0 + tid;
-    const int b = q_req[q];
-    const bool req_ok = b >= 0 && b < B;
-
-    bool is_cand = false;
-    if (req_ok && p < max_pools) {
-        const long long last = (long long)first_valid[b] + (long long)p * kpool + kpool - 1;
-        is_cand = pool_valid[(size_t)b * max_pools + p] != 0 && last <= (long long)q_pos[q];
-    }
-    float g[kScoreHeads];
-#pragma unroll
-    for (int h = 0; h < kScoreHeads; ++h) g[h] = (req_ok && h < H) ? __ldg(gate_w + (size_t)q * H + h) : 0.f;
 
     if (warp == 0) {
         tc::tmem_alloc(&tmem_base, 32);
@@ -72,6 +61,20 @@ index_scores_kernel(const __grid_constant__ CUtensorMap key_map,
         mbar_init(&mma_bar, 1);
         fence_mbarrier_init();
     }
+    pdl_wait();
+    pdl_launch_dependents();
+
+    const int b = q_req[q];
+    const bool req_ok = b >= 0 && b < B;
+    bool is_cand = false;
+    if (req_ok && p < max_pools) {
+        const long long last = (long long)first_valid[b] + (long long)p * kpool + kpool - 1;
+        is_cand = pool_valid[(size_t)b * max_pools + p] != 0 && last <= (long long)q_pos[q];
+    }
+    float g[kScoreHeads];
+#pragma unroll
+    for (int h = 0; h < kScoreHeads; ++h) g[h] = (req_ok && h < H) ? __ldg(gate_w + (size_t)q * H + h) : 0.f;
+
     tc::fence_before_sync();
     const bool any = __syncthreads_or(is_cand) != 0;
     tc::fence_after_sync();
@@ -153,9 +156,10 @@ inline int index_scores_launch(const void *q_idx, const float *gate_w, const int
     if (!ensure_smem_attr(reinterpret_cast<const void *>(index_scores_kernel), kScoreSmem))
         return DSA_ERR_CUDA;
     dim3 grid(ceil_div(max_pools, kScorePools), Q);
-    index_scores_kernel<<<grid, kScoreThreads, kScoreSmem, stream>>>(
-        key_map, q_map, gate_w, q_req, q_pos, H, pool_valid, first_valid, B, kpool, max_pools,
-        scores, cand);
+    if (launch_pdl(index_scores_kernel, grid, dim3(kScoreThreads), kScoreSmem, stream, key_map, q_map,
+                   gate_w, q_req, q_pos, H, pool_valid, first_valid, B, kpool, max_pools, scores,
+                   cand) != cudaSuccess)
+        return DSA_ERR_CUDA;
     return launch_status();
 }
 

@@ -250,6 +250,8 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     }
     for (int i = tid; i < KP * kD; i += kCmpThreads) s_ape[i] = ape[i] * kLog2e;
     __syncthreads();
+    pdl_wait();
+    pdl_launch_dependents();
 
     if (warp == kCmpConsumers / 32) {
         // ---------------------------------------------------------------- producer warp
@@ -363,9 +365,10 @@ inline int kpool_compress_launch_kp(const __nv_bfloat16 *k, const __nv_bfloat16 
     const long long n_tiles = (long long)tiles_per_req * B;
     if (n_tiles > (1ll << 30)) return DSA_ERR_UNSUPPORTED;
     const int grid = (int)std::min<long long>(n_tiles, sm_count());
-    kpool_compress_kernel<KP><<<grid, C::kThreads, smem, stream>>>(
-        k, gate, valid, req_start, B, max_pools, tiles_per_req, (int)n_tiles, ape, ln_w, ln_b, eps,
-        keys, idx, pv, fv);
+    if (launch_pdl(kpool_compress_kernel<KP>, dim3(grid), dim3(C::kThreads), smem, stream, k, gate,
+                   valid, req_start, B, max_pools, tiles_per_req, (int)n_tiles, ape, ln_w, ln_b, eps,
+                   keys, idx, pv, fv) != cudaSuccess)
+        return DSA_ERR_CUDA;
     return launch_status();
 }
 

@@ -121,14 +121,23 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
 
     const int split = blockIdx.x, qi = blockIdx.y, hg = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int b = q_req[qi];
-    const bool req_ok = b >= 0 && b < B;
-    const int rs = req_ok ? req_start[b] : 0;
-    const int T = req_ok ? max(0, req_start[b + 1] - rs) : 0;
     const int j0 = min(W, split * per), j1 = min(W, j0 + per);
     const int ntok = j1 - j0;
     const int nch = (ntok + kTcChunk - 1) / kTcChunk;
     const int h0 = hg * kTcHeads, nh = min(kTcHeads, Hm - h0);
+
+    if (warp >= 4) {
+        // Q tile (a step input): 64 rows x 64 16-byte chunks into the swizzled
+        // K-major layout, issued before the predecessor grid finishes.
+        for (int x = tid - 128; x < kTcHeads * 64; x += 128) {
+            const int h = x >> 6, cc = x & 63;
+            const uint32_t dst = sQ + (cc >> 3) * 8192 + h * 128 + (((cc & 7) ^ (h & 7)) << 4);
+            if (h < nh)
+                tc::cp_async16(dst, qm + ((size_t)qi * Hm + h0 + h) * kL + cc * 8);
+            else
+                tc::st_shared_zero16(dst);
+        }
+    }
 
     if (warp == 0) {
         tc::tmem_alloc(&ctl->tmem_base, kTmemCols);
@@ -156,6 +165,12 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
+    pdl_wait();                       // token ids come from the predecessor grid
+    pdl_launch_dependents();
+    const int b = q_req[qi];
+    const bool req_ok = b >= 0 && b < B;
+    const int rs = req_ok ? req_start[b] : 0;
+    const int T = req_ok ? max(0, req_start[b + 1] - rs) : 0;
 
     if (warp == 0) {
         // ------------------------------------------------------------------ MMA issuer
@@ -247,17 +262,8 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         const int st = tid - 128, wq = warp - 4;
         const int hh = 16 * wq + lane;        // head row owned by lanes 0..15
         const bool owner = lane < 16;
-        // Q tile: 64 rows x 64 16-byte chunks into the swizzled K-major layout, all
-        // 32 copies of a thread in flight at once.
-        for (int x = st; x < kTcHeads * 64; x += 128) {
-            const int h = x >> 6, cc = x & 63;
-            const uint32_t dst = sQ + (cc >> 3) * 8192 + h * 128 + (((cc & 7) ^ (h & 7)) << 4);
-            if (h < nh)
-                tc::cp_async16(dst, qm + ((size_t)qi * Hm + h0 + h) * kL + cc * 8);
-            else
-                tc::st_shared_zero16(dst);
-        }
-        tc::cp_async_wait_all();
+        (void)st;
+        tc::cp_async_wait_all();          // this thread's Q copies (issued at entry)
         tc::fence_proxy_async_smem();
         mbar_arrive(&ctl->q_full);
 
@@ -411,6 +417,8 @@ __global__ void __launch_bounds__(128)
 mla_combine_kernel(const float *__restrict__ part, int Hm, int S, __nv_bfloat16 *__restrict__ out,
                    float *__restrict__ lse) {
     const int h = blockIdx.x, q = blockIdx.y, tid = threadIdx.x;
+    pdl_wait();
+    pdl_launch_dependents();
     const float *base = part + ((size_t)q * S * Hm + h) * kPartStride;
     const size_t sstride = (size_t)Hm * kPartStride;
     float M = -INFINITY;
@@ -482,15 +490,17 @@ inline int sparse_mla_launch(const void *q, const void *kv, const int32_t *req_s
     const float scale_log2 = sm_scale * 1.4426950408889634f;
     const int groups = (Hm + kTcHeads - 1) / kTcHeads;
     float *part = reinterpret_cast<float *>(ws);
-    mla_tc_kernel<<<dim3(g.S, Q, groups), kTcThreads, kTcSmemBytes, stream>>>(
-        reinterpret_cast<const __nv_bfloat16 *>(q), reinterpret_cast<const __nv_bfloat16 *>(kv),
-        req_start, q_req, token_ids, B, Hm, W, g.S, g.per, scale_log2, part,
-        reinterpret_cast<__nv_bfloat16 *>(out), lse);
+    if (launch_pdl(mla_tc_kernel, dim3(g.S, Q, groups), dim3(kTcThreads), kTcSmemBytes, stream,
+                   reinterpret_cast<const __nv_bfloat16 *>(q),
+                   reinterpret_cast<const __nv_bfloat16 *>(kv), req_start, q_req, token_ids, B, Hm,
+                   W, g.S, g.per, scale_log2, part, reinterpret_cast<__nv_bfloat16 *>(out),
+                   lse) != cudaSuccess)
+        return DSA_ERR_CUDA;
     int st = launch_status();
     if (st != DSA_OK || g.S == 1) return st;
-    mla_combine_kernel<<<dim3(Hm, Q), 128, 0, stream>>>(part, Hm, g.S,
-                                                          reinterpret_cast<__nv_bfloat16 *>(out),
-                                                          lse);
+    if (launch_pdl(mla_combine_kernel, dim3(Hm, Q), dim3(128), 0, stream, part, Hm, g.S,
+                   reinterpret_cast<__nv_bfloat16 *>(out), lse) != cudaSuccess)
+        return DSA_ERR_CUDA;
     return launch_status();
 }
 

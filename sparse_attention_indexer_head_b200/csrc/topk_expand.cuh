@@ -69,6 +69,8 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
 
     const int tid = threadIdx.x;
     const int q = blockIdx.x;
+    pdl_wait();
+    pdl_launch_dependents();
     const int b = q_req[q];
     const bool req_ok = b >= 0 && b < B;
     const float *srow = scores + (size_t)q * P;
@@ -231,9 +233,10 @@ inline int topk_expand_launch(const float *scores, const uint8_t *cand, const in
     const int smem = select_k * 4 + (keys_in_smem ? max_pools * 4 : 0);
     if (!ensure_smem_attr(reinterpret_cast<const void *>(topk_expand_kernel), smem))
         return DSA_ERR_CUDA;
-    topk_expand_kernel<<<Q, kTopkThreads, smem, stream>>>(scores, cand, pool_idx, q_req, B,
-                                                          max_pools, kpool, select_k,
-                                                          keys_in_smem, top_pools, token_ids);
+    if (launch_pdl(topk_expand_kernel, dim3(Q), dim3(kTopkThreads), smem, stream, scores, cand,
+                   pool_idx, q_req, B, max_pools, kpool, select_k, keys_in_smem, top_pools,
+                   token_ids) != cudaSuccess)
+        return DSA_ERR_CUDA;
     return launch_status();
 }
 

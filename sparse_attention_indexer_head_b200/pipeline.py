@@ -117,8 +117,10 @@ class DecodeStep:
                                 self.ws, self.ws.numel(), stream)
 
     def run(self, stream=None):
-        self.head_gate(stream)
+        # compress first: the small head-gate grid then overlaps compress's tail
+        # (every kernel is launched with programmatic dependent launch).
         self.kpool_compress(stream)
+        self.head_gate(stream)
         self.index_scores(stream)
         self.topk_expand(stream)
         self.sparse_mla(stream)
