@@ -146,9 +146,11 @@ int dsa_index_scores(const dsa_bf16 *q_idx, const float *gate_w, const int32_t *
  * a5+a6. topk_pools + expand_selection ([mod.rs] "Shape of the pipeline" third
  * and fourth arrows; Glm5NextDsaConfig::select_k and out_width; trap 6).
  *   Candidates (cand != 0) of query q are ranked by (score descending, pool id
- *   ascending); -0.0 equals +0.0 and a NaN score ranks as -inf.
- *   n_q = min(select_k, number of candidates).
- *   top_pools int32 [Q, select_k]: ranked pool ids, then -1.
+ *   ascending); -0.0 equals +0.0 and a NaN score ranks as -inf. The first
+ *   n_q = min(select_k, number of candidates) of that ranking are selected.
+ *   top_pools int32 [Q, select_k]: the selected pool ids in ascending order,
+ *             then -1 (the pages fix no order for the list; by id it is
+ *             unique, and the expanded token ids ascend within a request).
  *   token_ids int32 [Q, select_k * kpool]: token_ids[q, j*kpool + s] =
  *             pool_idx[b, top_pools[q, j], s] for j < n_q, -1 after; every
  *             element is written (the -1 sentinel tail in full).
@@ -165,7 +167,12 @@ int dsa_topk_expand(const float *scores, const uint8_t *cand, const int32_t *poo
  * per-row gather is exact; trap 5: qk_rope_head_dim == 0, the 512-wide latent
  * row is both key and value).
  *   q         bf16 [Q, Hm, 512] (queries absorbed into the latent space)
- *   kv        bf16 [total_tokens, 512] latent cache
+ *   kv        bf16 [kv_rows, 512] latent cache (row stride 1024 bytes);
+ *             request b owns rows req_start[b] .. req_start[b+1]-1.
+ *   kv_rows   rows of kv, 0 <= kv_rows <= INT32_MAX (DSA_ERR_UNSUPPORTED
+ *             above: the row gather addresses rows with 32-bit coordinates);
+ *             kv may be NULL when it is 0. A row at or past kv_rows is never
+ *             read: its id counts as invalid.
  *   token_ids int32 [Q, W] logical ids; -1 and ids outside [0, T_b) ignored.
  *             Ids in a row must be distinct (dsa_topk_expand guarantees it;
  *             the set semantics of the page collapses duplicates).
@@ -176,13 +183,17 @@ int dsa_topk_expand(const float *scores, const uint8_t *cand, const int32_t *poo
  *   workspace: device scratch of dsa_sparse_mla_workspace_size(Q, Hm, W) bytes
  *   (16-byte aligned; contents need no initialisation; not shared between
  *   calls that may overlap).
+ *   When a query's ids are cut into 2..8 splits, the splits of a query run as
+ *   one thread-block cluster; a device on which such a cluster cannot be
+ *   resident (fewer free SMs per GPU processing cluster than splits) gets
+ *   DSA_ERR_UNSUPPORTED.
  * Requires kv_lora == 512 and rope_dim == 0 (DSA_ERR_UNSUPPORTED otherwise,
  * as the page's config validation refuses any other latent width), Hm a
  * multiple of 16 with 16 <= Hm <= 128, W >= 0.
  */
 size_t dsa_sparse_mla_workspace_size(int Q, int Hm, int W);
-int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *req_start,
-                          const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
+int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows,
+                          const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
                           int W, int kv_lora, int rope_dim, float sm_scale, dsa_bf16 *out,
                           float *lse, void *workspace, size_t workspace_bytes,
                           dsa_stream_t stream);
@@ -201,7 +212,10 @@ int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *
  *   The scratch is a static device array of DSA_NOALLOC_SCRATCH_BYTES bytes
  *   that every GPU which loads the library keeps until the process exits. A
  *   call whose split-KV scratch (dsa_sparse_mla_workspace_size(Q, Hm, W))
- *   exceeds it returns DSA_ERR_WORKSPACE and launches nothing.
+ *   exceeds it returns DSA_ERR_WORKSPACE and launches nothing. The split
+ *   geometry keeps every grid within 148 CTAs, so no call needs more than
+ *   148 x 64 x 516 x 4 bytes (about 19.6 MB): the refusal is a guard that no
+ *   present shape reaches.
  *   Nothing is allocated or freed: no cudaMalloc, no cudaFree, no allocating
  *   library routine. The first call on a device looks up the scratch's device
  *   address (cudaGetSymbolAddress, with that device current); make that first
@@ -213,8 +227,8 @@ int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *
  *   scratch and must not be made.
  */
 #define DSA_NOALLOC_SCRATCH_BYTES (32u << 20)
-int dsa_sparse_mla_decode_noalloc(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *req_start,
-                                  const int32_t *q_req, const int32_t *token_ids, int Q, int B,
+int dsa_sparse_mla_decode_noalloc(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows,
+                                  const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids, int Q, int B,
                                   int Hm, int W, int kv_lora, int rope_dim, float sm_scale,
                                   dsa_bf16 *out, float *lse, dsa_stream_t stream);
 

@@ -45,6 +45,7 @@ def _load() -> ctypes.CDLL:
             "`python -m sparse_attention_indexer_head_b200.build` (no fallback exists)")
     L = ctypes.CDLL(LIB_PATH)
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    I64 = ctypes.c_int64
     sig = {
         "dsa_status_string": ([I], ctypes.c_char_p),
         "dsa_abi_version": ([], I),
@@ -54,8 +55,8 @@ def _load() -> ctypes.CDLL:
         "dsa_index_scores": ([P, P, P, P, I, I, I, P, P, P, I, I, I, P, P, P], I),
         "dsa_topk_expand": ([P, P, P, P, I, I, I, I, I, P, P, P], I),
         "dsa_sparse_mla_workspace_size": ([I, I, I], Z),
-        "dsa_sparse_mla_decode": ([P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P], I),
-        "dsa_sparse_mla_decode_noalloc": ([P, P, P, P, P, I, I, I, I, I, I, F, P, P, P], I),
+        "dsa_sparse_mla_decode": ([P, P, I64, P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P], I),
+        "dsa_sparse_mla_decode_noalloc": ([P, P, I64, P, P, P, I, I, I, I, I, I, F, P, P, P], I),
     }
     for name, (argtypes, restype) in sig.items():
         fn = getattr(L, name)
@@ -137,20 +138,20 @@ def dsa_sparse_mla_workspace_size(Q: int, Hm: int, W: int) -> int:
     return int(lib.dsa_sparse_mla_workspace_size(Q, Hm, W))
 
 
-def dsa_sparse_mla_decode(q, kv, req_start, q_req, token_ids, Q: int, B: int, Hm: int, W: int,
-                          kv_lora: int, rope_dim: int, sm_scale: float, out, lse, workspace,
-                          workspace_bytes: int, stream=None) -> None:
+def dsa_sparse_mla_decode(q, kv, kv_rows: int, req_start, q_req, token_ids, Q: int, B: int,
+                          Hm: int, W: int, kv_lora: int, rope_dim: int, sm_scale: float, out, lse,
+                          workspace, workspace_bytes: int, stream=None) -> None:
     _check("dsa_sparse_mla_decode", lib.dsa_sparse_mla_decode(
-        _ptr(q), _ptr(kv), _ptr(req_start), _ptr(q_req), _ptr(token_ids), Q, B, Hm, W, kv_lora,
+        _ptr(q), _ptr(kv), int(kv_rows), _ptr(req_start), _ptr(q_req), _ptr(token_ids), Q, B, Hm, W, kv_lora,
         rope_dim, float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace), int(workspace_bytes),
         _stream(stream)))
 
 
-def dsa_sparse_mla_decode_noalloc(q, kv, req_start, q_req, token_ids, Q: int, B: int, Hm: int,
-                                  W: int, kv_lora: int, rope_dim: int, sm_scale: float, out, lse,
-                                  stream=None) -> None:
+def dsa_sparse_mla_decode_noalloc(q, kv, kv_rows: int, req_start, q_req, token_ids, Q: int,
+                                  B: int, Hm: int, W: int, kv_lora: int, rope_dim: int,
+                                  sm_scale: float, out, lse, stream=None) -> None:
     """dsa_sparse_mla_decode for callers that cannot allocate: the split-KV scratch is the
     library's own static device area (see include/dsa.h)."""
     _check("dsa_sparse_mla_decode_noalloc", lib.dsa_sparse_mla_decode_noalloc(
-        _ptr(q), _ptr(kv), _ptr(req_start), _ptr(q_req), _ptr(token_ids), Q, B, Hm, W, kv_lora,
+        _ptr(q), _ptr(kv), int(kv_rows), _ptr(req_start), _ptr(q_req), _ptr(token_ids), Q, B, Hm, W, kv_lora,
         rope_dim, float(sm_scale), _ptr(out), _ptr(lse), _stream(stream)))

@@ -106,18 +106,18 @@ size_t dsa_sparse_mla_workspace_size(int Q, int Hm, int W) {
     return dsa::mla_workspace_bytes(Q, Hm, W);
 }
 
-int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *req_start,
-                          const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
+int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows,
+                          const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
                           int W, int kv_lora, int rope_dim, float sm_scale, dsa_bf16 *out,
                           float *lse, void *workspace, size_t workspace_bytes,
                           dsa_stream_t stream) {
-    return dsa::sparse_mla_launch(q, kv, req_start, q_req, token_ids, Q, B, Hm, W, kv_lora,
-                                  rope_dim, sm_scale, out, lse, workspace, workspace_bytes,
+    return dsa::sparse_mla_launch(q, kv, kv_rows, req_start, q_req, token_ids, Q, B, Hm, W,
+                                  kv_lora, rope_dim, sm_scale, out, lse, workspace, workspace_bytes,
                                   reinterpret_cast<cudaStream_t>(stream));
 }
 
-int dsa_sparse_mla_decode_noalloc(const dsa_bf16 *q, const dsa_bf16 *kv, const int32_t *req_start,
-                                  const int32_t *q_req, const int32_t *token_ids, int Q, int B,
+int dsa_sparse_mla_decode_noalloc(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows,
+                                  const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids, int Q, int B,
                                   int Hm, int W, int kv_lora, int rope_dim, float sm_scale,
                                   dsa_bf16 *out, float *lse, dsa_stream_t stream) {
     size_t need = 0;
@@ -130,8 +130,8 @@ int dsa_sparse_mla_decode_noalloc(const dsa_bf16 *q, const dsa_bf16 *kv, const i
         const int st = scratch_address(&scratch);
         if (st != DSA_OK) return st;
     }
-    return dsa::sparse_mla_launch(q, kv, req_start, q_req, token_ids, Q, B, Hm, W, kv_lora,
-                                  rope_dim, sm_scale, out, lse, scratch, need,
+    return dsa::sparse_mla_launch(q, kv, kv_rows, req_start, q_req, token_ids, Q, B, Hm, W,
+                                  kv_lora, rope_dim, sm_scale, out, lse, scratch, need,
                                   reinterpret_cast<cudaStream_t>(stream));
 }
 

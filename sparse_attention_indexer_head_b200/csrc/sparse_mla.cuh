@@ -6,15 +6,22 @@
 //
 // Split-KV decode on the 5th-generation tensor cores: a query's W selected ids
 // are cut into S contiguous splits; one CTA per (split, query, 64-head group)
-// gathers its latent rows and runs an online softmax for every head, writing an
-// unnormalised partial (O, running max m, running sum l) -- or, with a single
-// split, the normalised output directly; a combine kernel merges the S
-// partials of each (query, head) in split order (deterministic) and writes
-// bf16 out and the log-sum-exp.
+// gathers its latent rows with TMA and runs an online softmax for every head.
+// The S partials (O, running max m, running sum l) of a (query, head group)
+// are merged in split order, so results do not depend on scheduling:
+//   S == 1       the CTA normalises and writes bf16 out and the lse itself;
+//   2 <= S <= 8  the S CTAs form a thread-block cluster and merge through
+//                distributed shared memory, each CTA writing its share of the
+//                heads (no partials in global memory, no second launch);
+//   S > 8        (few queries) the partials go to the workspace and a combine
+//                kernel merges them.
 #pragma once
+
+#include <atomic>
 
 #include "common.cuh"
 #include "tc_ptx.cuh"
+#include "tma.cuh"
 
 namespace dsa {
 
@@ -37,12 +44,15 @@ constexpr int kPartStride = kL + 4;
 // 32-lane quadrant, the M=64 layout).
 //
 // Warp roles (256 threads): warp 0 allocates tensor memory and one lane issues
-// every MMA; warps 1-3 gather, warp 1+(c mod 3) filling chunk c into a 4-stage
-// ring with 16-byte cp.async into the swizzled layout (zero rows for ids that are
-// -1 or outside the request; the next chunk's ids are prefetched), so up to
-// three chunks are in flight; warps 4-7 load Q, run the softmax (lane i < 16 of
-// warp 4+w owns head 16w+i), rescale O^T when a head's running max grows by
-// more than 2^8 (lazy rescaling), and write the epilogue.
+// every MMA; warp 1 is the producer: it turns the chunk's ids into cache rows
+// and gathers them with TMA (tile::gather4, four 128-byte rows per copy, eight
+// copies per group of four rows) straight into the swizzled 4-stage ring; an id
+// that is -1 or outside its request points past the end of the cache and reads
+// as a zero row. Nothing waits for a copy but the consumers, so all four stages
+// can be in flight. Warps 4-7 load Q, run the softmax (lane i < 16 of warp 4+w
+// owns head 16w+i), rescale O^T when a head's running max grows by more than
+// 2^8 (lazy rescaling), and write the epilogue. Warps 2-3 only take part in the
+// cluster merge.
 // ---------------------------------------------------------------------------------------
 constexpr int kTcThreads = 256;
 constexpr int kTcChunk = 32;                        // tokens per chunk
@@ -57,6 +67,11 @@ constexpr uint32_t kStageP = 4 * 1024;
 constexpr uint32_t kOffCtl = 200 * 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLazyRescale = 8.0f;                // log2 units
+constexpr int kMaxClusterSplits = 8;                // portable cluster size
+constexpr int kSmTarget = 148;                      // CTAs of one full wave (one CTA per SM)
+// The cluster merge reads each CTA's O^T, copied as fp32 [64 heads][512] into
+// the (then idle) gathered-row ring.
+static_assert(kTcStages * kStageKV == kTcHeads * kL * 4, "merge buffer must fit the ring");
 
 struct TcCtl {
     uint64_t kv_full[kTcStages], kv_empty[kTcStages];
@@ -65,33 +80,37 @@ struct TcCtl {
     uint32_t vmask[kTcStages];
     float alpha[kTcHeads];
     float lsum[kTcHeads];
+    float mfin[kTcHeads];
     uint32_t tmem_base;
     volatile int abort;
 };
 constexpr int kTcSmemBytes = (int)kOffCtl + (int)sizeof(TcCtl) + 1024;   // + alignment slack
 
 struct MlaGeom {
-    int S;      // splits per query
-    int per;    // selected-id slots per split (a multiple of the chunk)
+    int S;         // splits per (query, head group)
+    int per;       // selected-id slots per split (a multiple of the chunk)
+    bool cluster;  // splits merged inside a thread-block cluster
 };
 
+// As many splits as keep the grid within one wave of CTAs, no split holding
+// more chunks than needed for that; every split then holds at least one id.
 inline MlaGeom mla_geometry(int Q, int Hm, int W) {
-    MlaGeom g{1, kTcChunk};
+    MlaGeom g{1, kTcChunk, false};
     if (Q <= 0 || W <= 0) return g;
-    const int groups = (Hm + kTcHeads - 1) / kTcHeads;
+    const long long ctas = (long long)Q * ((Hm + kTcHeads - 1) / kTcHeads);
     const int chunks = ceil_div(W, kTcChunk);
-    int S = max(1, min(chunks, (148 + Q * groups - 1) / (Q * groups)));
-    if (Q * groups >= 148) S = 1;
-    const int per = ceil_div(ceil_div(W, S), kTcChunk) * kTcChunk;
-    g.S = ceil_div(W, per);
-    g.per = per;
+    int per_chunks = chunks;
+    if (ctas < kSmTarget) per_chunks = ceil_div(chunks, (int)(kSmTarget / ctas));
+    g.per = per_chunks * kTcChunk;
+    g.S = ceil_div(chunks, per_chunks);
+    g.cluster = g.S >= 2 && g.S <= kMaxClusterSplits;
     return g;
 }
 
 inline size_t mla_workspace_bytes(int Q, int Hm, int W) {
     if (Q <= 0 || Hm <= 0) return 0;
     const MlaGeom g = mla_geometry(Q, Hm, W);
-    if (g.S == 1) return 0;
+    if (g.S == 1 || g.cluster) return 0;
     return (size_t)Q * g.S * Hm * kPartStride * sizeof(float);
 }
 
@@ -104,12 +123,66 @@ DSA_DEVINL bool tc_wait(TcCtl *ctl, uint64_t *bar, uint32_t parity) {
     return true;
 }
 
+// Cluster merge of the S split partials of one (query, head group), held in the
+// shared memory of the cluster's S CTAs (m, l in TcCtl; O^T as fp32
+// [64 heads][512] at sO). The CTA of cluster rank r writes heads
+// [r*hp, min(nh, (r+1)*hp)), hp = ceil(nh / S), 256 threads x 4 latents per
+// head; splits enter in rank order.
+DSA_DEVINL void mla_cluster_merge(const TcCtl *ctl, uint32_t sO, int S, int nh, int rank, int tid,
+                                  __nv_bfloat16 *__restrict__ ob, float *__restrict__ lseb) {
+    const int hp = (nh + S - 1) / S;
+    const int hb = rank * hp, he = min(nh, hb + hp);
+    const int c4 = tid & 127;
+    for (int h = hb + (tid >> 7); h < he; h += 2) {
+        const uint32_t am = smem_u32(&ctl->mfin[h]), al = smem_u32(&ctl->lsum[h]);
+        const uint32_t ao = sO + (uint32_t)h * (kL * 4) + c4 * 16;
+        float ms[kMaxClusterSplits], ls[kMaxClusterSplits];
+        float4 v[kMaxClusterSplits];
+#pragma unroll
+        for (int r = 0; r < kMaxClusterSplits; ++r) {
+            ms[r] = -INFINITY;
+            ls[r] = 0.f;
+            v[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r < S) {
+                ms[r] = ld_cluster_f32(cluster_map(am, r));
+                ls[r] = ld_cluster_f32(cluster_map(al, r));
+                v[r] = ld_cluster_f32x4(cluster_map(ao, r));   // unused where m is -inf
+            }
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < kMaxClusterSplits; ++r) M = fmaxf(M, ms[r]);
+        float o[4] = {0.f, 0.f, 0.f, 0.f};
+        float lsum = 0.f;
+#pragma unroll
+        for (int r = 0; r < kMaxClusterSplits; ++r) {
+            if (ms[r] == -INFINITY) continue;
+            const float w = ex2(ms[r] - M);
+            lsum = fmaf(ls[r], w, lsum);
+            o[0] = fmaf(v[r].x, w, o[0]);
+            o[1] = fmaf(v[r].y, w, o[1]);
+            o[2] = fmaf(v[r].z, w, o[2]);
+            o[3] = fmaf(v[r].w, w, o[3]);
+        }
+        const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
+        uint2 packed;
+        packed.x = pack_bf16x2(o[0] * inv, o[1] * inv);
+        packed.y = pack_bf16x2(o[2] * inv, o[3] * inv);
+        *reinterpret_cast<uint2 *>(ob + (size_t)h * kL + 4 * c4) = packed;
+        if (lseb && c4 == 0)
+            lseb[h] = lsum > 0.f ? (M + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
+    }
+}
+
+// kv_map: the latent cache as [map_rows, 512] bf16 rows, box 64 x 1 with the
+// 128-byte swizzle; kv_rows of them are cache rows (map_rows = max(kv_rows, 1)).
+template <bool kCluster>
 __global__ void __launch_bounds__(kTcThreads, 1)
-mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restrict__ kv,
+mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __nv_bfloat16 *__restrict__ qm,
               const int32_t *__restrict__ req_start, const int32_t *__restrict__ q_req,
-              const int32_t *__restrict__ token_ids, int B, int Hm, int W, int S, int per,
-              float scale_log2, float *__restrict__ part, __nv_bfloat16 *__restrict__ out,
-              float *__restrict__ lse) {
+              const int32_t *__restrict__ token_ids, int B, int kv_rows, int map_rows, int Hm,
+              int W, int S, int per, float scale_log2, float *__restrict__ part,
+              __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
     extern __shared__ uint8_t mla_smem_raw[];
     const uint32_t raw = smem_u32(mla_smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;           // 128B-swizzle atoms need 1 KB
@@ -145,7 +218,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     }
     if (tid == 32) {
         for (int i = 0; i < kTcStages; ++i) {
-            mbar_init(&ctl->kv_full[i], 32);
+            mbar_init(&ctl->kv_full[i], 1);
             mbar_init(&ctl->kv_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -220,44 +293,50 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             if (ok && issue_pv(nch - 1)) tc::mma_commit(&ctl->o_final);
         }
         __syncwarp();
-    } else if (warp < 4) {
-        // ------------------------------------------------------------------ gather warps
-        // Warp 1+p fills chunks p, p+3, p+6, ...; lane r owns row r's id.
-        const int pw = warp - 1;
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ producer
+        // Lane r holds row r's id; lane i < 8 gathers rows 4i..4i+3 of the chunk
+        // (eight gather4 copies, one per 64-latent column atom).
         auto load_id = [&](int c) -> int {
             const int j = c * kTcChunk + lane;
             return (c < nch && j < ntok) ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
         };
-        int next_id = load_id(pw);
-        for (int c = pw; c < nch; c += 3) {
+        int next_id = load_id(0);
+        int issued = 0;
+        for (int c = 0; c < nch; ++c) {
             const int s = c % kTcStages;
             const int id = next_id;
-            next_id = load_id(c + 3);                      // in flight during this chunk's copies
+            next_id = load_id(c + 1);                      // in flight during this chunk's wait
             bool ok = true;
             if (c >= kTcStages) ok = tc_wait(ctl, &ctl->kv_empty[s], ((c / kTcStages) - 1) & 1);
             if (!__all_sync(0xffffffffu, ok)) break;
-            const bool valid = id >= 0 && id < T;
+            const bool valid = id >= 0 && id < T && (long long)rs + id < (long long)kv_rows;
             const uint32_t vm = __ballot_sync(0xffffffffu, valid);
-            const int myid = valid ? id : -1;
-            const uint32_t dst0 = sKV + s * kStageKV;
-            for (int r = 0; r < kTcChunk; ++r) {
-                const int rid = __shfl_sync(0xffffffffu, myid, r);
+            const int y = valid ? rs + id : map_rows;      // past the map: a zero row
+            int yy[4];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int cc = lane + 32 * hh;         // 16-byte piece of the 1 KB row
-                    const uint32_t dst = dst0 + (cc >> 3) * kAtomKV + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
-                    if (rid >= 0)
-                        tc::cp_async16(dst, kv + ((size_t)rs + rid) * kL + cc * 8);
-                    else
-                        tc::st_shared_zero16(dst);
-                }
+            for (int i = 0; i < 4; ++i) yy[i] = __shfl_sync(0xffffffffu, y, (4 * lane + i) & 31);
+            if (lane == 0) {
+                ctl->vmask[s] = vm;
+                mbar_arrive_expect_tx(&ctl->kv_full[s], kStageKV);
             }
-            if (lane == 0) ctl->vmask[s] = vm;
-            tc::cp_async_wait_all();
-            tc::fence_proxy_async_smem();
-            mbar_arrive(&ctl->kv_full[s]);
+            __syncwarp();
+            if (lane < kTcChunk / 4) {
+                const uint32_t dst = sKV + s * kStageKV + lane * 512;
+#pragma unroll
+                for (int cb = 0; cb < kL / 64; ++cb)
+                    tma_gather4(dst + cb * kAtomKV, &kv_map, cb * 64, yy[0], yy[1], yy[2], yy[3],
+                                &ctl->kv_full[s]);
+            }
+            issued = c + 1;
         }
-    } else {
+        // After an abort, copies may still be in flight: let them land (bounded)
+        // before the CTA moves on.
+        if (lane == 0)
+            for (int c = max(0, issued - kTcStages); c < issued; ++c)
+                (void)mbar_wait(&ctl->kv_full[c % kTcStages], (c / kTcStages) & 1);
+        __syncwarp();
+    } else if (warp >= 4) {
         // ------------------------------------------------------------------ softmax (128 threads)
         const int st = tid - 128, wq = warp - 4;
         const int hh = 16 * wq + lane;        // head row owned by lanes 0..15
@@ -352,7 +431,27 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         }
         if (owner) ctl->lsum[hh] = l;
         tc::named_bar_sync(2, 128);
-        if (S > 1) {
+        if constexpr (kCluster) {
+            // O^T -> fp32 [head][latent] in the ring (idle: every gathered chunk was
+            // consumed and every MMA has completed); merged after the cluster barrier.
+            if (owner) ctl->mfin[hh] = have_o ? m_used : -INFINITY;
+            if (have_o) {
+                tc::fence_after_sync();
+#pragma unroll 1
+                for (int blk = 0; blk < 8; ++blk) {
+                    uint32_t o[32];
+                    tc::tmem_ld32(tl + (blk >> 1) * 64 + (blk & 1) * 32, o);
+                    tc::tmem_wait_ld();
+                    const int L = (blk >> 1) * 128 + 32 * wq + lane;
+                    const uint32_t dst = sKV + ((uint32_t)((blk & 1) * 32) * kL + L) * 4;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        asm volatile("st.shared.f32 [%0], %1;" ::"r"(dst + (uint32_t)j * kL * 4),
+                                     "f"(__uint_as_float(o[j]))
+                                     : "memory");
+                }
+            }
+        } else if (S > 1) {
             float *pb = part + ((size_t)(qi * S + split) * Hm + h0) * kPartStride;
             if (have_o) {
                 tc::fence_after_sync();
@@ -407,6 +506,12 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    if constexpr (kCluster) {
+        cluster_sync_all();           // every split's m, l and O^T are in place
+        mla_cluster_merge(ctl, sKV, S, nh, split, tid, out + ((size_t)qi * Hm + h0) * kL,
+                          lse ? lse + (size_t)qi * Hm + h0 : nullptr);
+        cluster_sync_all();           // no CTA leaves while a peer still reads it
+    }
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
@@ -465,19 +570,50 @@ mla_combine_kernel(const float *__restrict__ part, int Hm, int S, __nv_bfloat16 
         lse[(size_t)q * Hm + h] = lsum > 0.f ? (M + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
 }
 
-inline int sparse_mla_launch(const void *q, const void *kv, const int32_t *req_start,
-                             const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
-                             int W, int kv_lora, int rope_dim, float sm_scale, void *out,
-                             float *lse, void *ws, size_t ws_bytes, cudaStream_t stream) {
-    if (Q < 0 || B < 0 || Hm <= 0 || W < 0 || kv_lora <= 0 || rope_dim < 0)
+// Whether clusters of `splits` CTAs of the cluster kernel can be resident on
+// the current device (asked once per device and size, after the kernel's
+// shared-memory limit is raised).
+inline bool mla_cluster_fits(int splits) {
+    static std::atomic<int> known[64][kMaxClusterSplits + 1];   // 0 unknown, 1 yes, 2 no
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    const int k = known[dev][splits].load(std::memory_order_relaxed);
+    if (k != 0) return k == 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(splits, 1, 1);
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = kTcSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const bool ok = cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel<true>, &cfg) == cudaSuccess &&
+                    n >= 1;
+    (void)cudaGetLastError();
+    known[dev][splits].store(ok ? 1 : 2, std::memory_order_relaxed);
+    return ok;
+}
+
+inline int sparse_mla_launch(const void *q, const void *kv, int64_t kv_rows,
+                             const int32_t *req_start, const int32_t *q_req,
+                             const int32_t *token_ids, int Q, int B, int Hm, int W, int kv_lora,
+                             int rope_dim, float sm_scale, void *out, float *lse, void *ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+    if (Q < 0 || B < 0 || Hm <= 0 || W < 0 || kv_lora <= 0 || rope_dim < 0 || kv_rows < 0)
         return DSA_ERR_INVALID_ARG;
     if (!(sm_scale == sm_scale) || sm_scale == INFINITY || sm_scale == -INFINITY)
         return DSA_ERR_INVALID_ARG;
     if (kv_lora != kL || rope_dim != 0 || Hm % 16 != 0 || Hm > DSA_MAX_MLA_HEADS)
         return DSA_ERR_UNSUPPORTED;
+    if (kv_rows > (int64_t)INT32_MAX) return DSA_ERR_UNSUPPORTED;   // TMA row coordinates are int32
     if (Q == 0) return DSA_OK;
     if (Q > 65535) return DSA_ERR_UNSUPPORTED;
-    if (!q || !q_req || !out || (W > 0 && !token_ids) || (B > 0 && (!kv || !req_start)))
+    if (!q || !q_req || !out || (W > 0 && !token_ids) || (B > 0 && !req_start) ||
+        (kv_rows > 0 && !kv))
         return DSA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(req_start, 4) || !aligned(q_req, 4) ||
         !aligned(token_ids, 4) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(ws, 16))
@@ -485,21 +621,41 @@ inline int sparse_mla_launch(const void *q, const void *kv, const int32_t *req_s
     const MlaGeom g = mla_geometry(Q, Hm, W);
     const size_t need = mla_workspace_bytes(Q, Hm, W);
     if (need > 0 && (!ws || ws_bytes < need)) return DSA_ERR_WORKSPACE;
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel), kTcSmemBytes))
+    if (g.cluster) {
+        if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true>), kTcSmemBytes))
+            return DSA_ERR_CUDA;
+        if (!mla_cluster_fits(g.S)) return DSA_ERR_UNSUPPORTED;
+    }
+    // With no cache rows the map spans q's first row; every id is then invalid
+    // and reads row 1, past the map.
+    const int map_rows = kv_rows > 0 ? (int)kv_rows : 1;
+    CUtensorMap kv_map;
+    if (!make_map_bf16_2d(&kv_map, kv_rows > 0 ? kv : q, (uint64_t)map_rows, kL, kL * 2, 64, 1))
         return DSA_ERR_CUDA;
     const float scale_log2 = sm_scale * 1.4426950408889634f;
     const int groups = (Hm + kTcHeads - 1) / kTcHeads;
     float *part = reinterpret_cast<float *>(ws);
-    if (launch_pdl(mla_tc_kernel, dim3(g.S, Q, groups), dim3(kTcThreads), kTcSmemBytes, stream,
-                   reinterpret_cast<const __nv_bfloat16 *>(q),
-                   reinterpret_cast<const __nv_bfloat16 *>(kv), req_start, q_req, token_ids, B, Hm,
-                   W, g.S, g.per, scale_log2, part, reinterpret_cast<__nv_bfloat16 *>(out),
-                   lse) != cudaSuccess)
+    const auto *qb = reinterpret_cast<const __nv_bfloat16 *>(q);
+    auto *ob = reinterpret_cast<__nv_bfloat16 *>(out);
+    const dim3 grid(g.S, Q, groups);
+    if (g.cluster) {
+        if (launch_pdl_cluster(mla_tc_kernel<true>, grid, dim3(kTcThreads), kTcSmemBytes, stream,
+                               g.S, kv_map, qb, req_start, q_req, token_ids, B, (int)kv_rows,
+                               map_rows, Hm, W, g.S, g.per, scale_log2, part, ob,
+                               lse) != cudaSuccess)
+            return DSA_ERR_CUDA;
+        return launch_status();
+    }
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<false>), kTcSmemBytes))
+        return DSA_ERR_CUDA;
+    if (launch_pdl(mla_tc_kernel<false>, grid, dim3(kTcThreads), kTcSmemBytes, stream, kv_map, qb,
+                   req_start, q_req, token_ids, B, (int)kv_rows, map_rows, Hm, W, g.S, g.per,
+                   scale_log2, part, ob, lse) != cudaSuccess)
         return DSA_ERR_CUDA;
     int st = launch_status();
     if (st != DSA_OK || g.S == 1) return st;
-    if (launch_pdl(mla_combine_kernel, dim3(Hm, Q), dim3(128), 0, stream, part, Hm, g.S,
-                   reinterpret_cast<__nv_bfloat16 *>(out), lse) != cudaSuccess)
+    if (launch_pdl(mla_combine_kernel, dim3(Hm, Q), dim3(128), 0, stream, part, Hm, g.S, ob,
+                   lse) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
 }

@@ -112,7 +112,8 @@ class DecodeStep:
 
     def sparse_mla(self, stream=None):
         g, t = self.g, self.t
-        B.dsa_sparse_mla_decode(t["q_mla"], t["kv"], t["req_start"], t["q_req"], self.token_ids,
+        B.dsa_sparse_mla_decode(t["q_mla"], t["kv"], t["kv"].shape[0], t["req_start"], t["q_req"],
+                                self.token_ids,
                                 g.Q, g.B, g.hm, g.W, KV_LORA, 0, g.sm_scale, self.out, self.lse,
                                 self.ws, self.ws.numel(), stream)
 

@@ -109,16 +109,21 @@ def test_topk_expand_refusals(B):
 
 def test_sparse_mla_refusals(B):
     L = B.lib
-    ws = B.dsa_sparse_mla_workspace_size(16, 64, 2048)
-    assert ws > 0 and ws % 16 == 0
+    # 2 queries: 64 splits of one chunk, merged through the workspace
+    ws = B.dsa_sparse_mla_workspace_size(2, 64, 2048)
+    assert ws == 2 * 64 * 64 * 516 * 4
+    # 16 queries: 8 splits per query merged inside a cluster, no workspace
+    assert B.dsa_sparse_mla_workspace_size(16, 64, 2048) == 0
+    # at least 148 CTAs without splitting: one split, no workspace
+    assert B.dsa_sparse_mla_workspace_size(148, 64, 2048) == 0
 
     def call(**kw):
-        a = dict(q=FAKE, kv=FAKE, rs=FAKE, qr=FAKE, ids=FAKE, Q=16, B=16, Hm=64, W=2048, lora=512,
-                 rope=0, scale=0.044, out=FAKE, lse=FAKE, ws=FAKE, wsb=ws)
+        a = dict(q=FAKE, kv=FAKE, rows=1 << 20, rs=FAKE, qr=FAKE, ids=FAKE, Q=2, B=2, Hm=64,
+                 W=2048, lora=512, rope=0, scale=0.044, out=FAKE, lse=FAKE, ws=FAKE, wsb=ws)
         a.update(kw)
-        return L.dsa_sparse_mla_decode(a["q"], a["kv"], a["rs"], a["qr"], a["ids"], a["Q"], a["B"],
-                                       a["Hm"], a["W"], a["lora"], a["rope"], a["scale"], a["out"],
-                                       a["lse"], a["ws"], a["wsb"], None)
+        return L.dsa_sparse_mla_decode(a["q"], a["kv"], a["rows"], a["rs"], a["qr"], a["ids"],
+                                       a["Q"], a["B"], a["Hm"], a["W"], a["lora"], a["rope"],
+                                       a["scale"], a["out"], a["lse"], a["ws"], a["wsb"], None)
 
     assert call(lora=576) == B.DSA_ERR_UNSUPPORTED      # KERNEL_KV_LORA_DIM = 512
     assert call(rope=64) == B.DSA_ERR_UNSUPPORTED       # NoPE only
@@ -128,6 +133,9 @@ def test_sparse_mla_refusals(B):
     assert call(ws=None) == B.DSA_ERR_WORKSPACE
     assert call(q=None) == B.DSA_ERR_INVALID_ARG
     assert call(scale=float("inf")) == B.DSA_ERR_INVALID_ARG
+    assert call(rows=-1) == B.DSA_ERR_INVALID_ARG
+    assert call(rows=1 << 31) == B.DSA_ERR_UNSUPPORTED  # 32-bit row coordinates
+    assert call(kv=None) == B.DSA_ERR_INVALID_ARG       # rows but no cache
     assert call(out=FAKE + 4) == B.DSA_ERR_ALIGNMENT
     assert call(Q=0) == B.DSA_OK
 
@@ -141,3 +149,18 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+def test_noalloc_scratch_covers_every_geometry(B):
+    # The split geometry keeps every grid within one wave of 148 CTAs, so the
+    # split-KV scratch of any call is at most 148 x 64 heads x 516 floats.
+    bound = 148 * 64 * 516 * 4
+    assert bound <= B.DSA_NOALLOC_SCRATCH_BYTES
+    worst = 0
+    for Q in list(range(1, 40)) + [64, 100, 147, 148, 149, 1000]:
+        for hm in range(16, 129, 16):
+            for W in (1, 31, 32, 33, 512, 2048, 4096 * 8, 1 << 20):
+                n = B.dsa_sparse_mla_workspace_size(Q, hm, W)
+                assert n % 16 == 0 and n <= bound, (Q, hm, W, n)
+                worst = max(worst, n)
+    assert worst > 0

@@ -255,8 +255,8 @@ def test_mla_heads_and_id_edge_cases(B, hm):
     lse = torch.empty(4, hm, dtype=torch.float32, device="cuda")
     ws_n = B.dsa_sparse_mla_workspace_size(4, hm, Wd)
     ws = torch.empty(ws_n, dtype=torch.uint8, device="cuda")
-    B.dsa_sparse_mla_decode(dev_bits(q), dev_bits(kv), d(rs), d(q_req), d(ids), 4, 3, hm, Wd, 512,
-                            0, scale, out, lse, ws, ws_n)
+    B.dsa_sparse_mla_decode(dev_bits(q), dev_bits(kv), kv.shape[0], d(rs), d(q_req), d(ids), 4, 3,
+                            hm, Wd, 512, 0, scale, out, lse, ws, ws_n)
     go, gl = host_bits(out), lse.cpu().numpy()
     assert_mla_close(go, ref_out, gl, ref_lse, vbound=mla_value_bound(kv, rs, q_req, ids))
     assert (go[2] == 0).all() and np.isneginf(gl[2]).all()      # empty request
