@@ -183,10 +183,12 @@ int dsa_topk_expand(const float *scores, const uint8_t *cand, const int32_t *poo
  *   workspace: device scratch of dsa_sparse_mla_workspace_size(Q, Hm, W) bytes
  *   (16-byte aligned; contents need no initialisation; not shared between
  *   calls that may overlap).
- *   When a query's ids are cut into 2..8 splits, the splits of a query run as
- *   one thread-block cluster; a device on which such a cluster cannot be
- *   resident (fewer free SMs per GPU processing cluster than splits) gets
- *   DSA_ERR_UNSUPPORTED.
+ *   A query's ids are cut into splits so the grid fills at most one wave of
+ *   148 CTAs. The workspace holds the splits' partial results for a merge
+ *   in global memory; when a query has 2..8 splits and all the launch's
+ *   clusters fit on the device at once, the splits of a query run as one
+ *   thread-block cluster, merge in shared memory and leave the workspace
+ *   untouched. Either way the splits are merged in split order.
  * Requires kv_lora == 512 and rope_dim == 0 (DSA_ERR_UNSUPPORTED otherwise,
  * as the page's config validation refuses any other latent width), Hm a
  * multiple of 16 with 16 <= Hm <= 128, W >= 0.

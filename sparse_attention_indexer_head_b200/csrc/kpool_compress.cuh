@@ -5,16 +5,18 @@
 // B200 design. The op streams the k and gate caches once (256 B per token row
 // each) and writes one 256 B key per pool: it is HBM-bound, so the kernel is a
 // TMA-fed stream with all arithmetic in registers:
-//   * a CTA owns a tile of TP = floor(128/kpool) consecutive pools of one
-//     request, i.e. up to 128 contiguous token rows of k and of gate; one
-//     thread issues two 1-D bulk copies (cp.async.bulk) of those rows into
-//     shared memory, completing on an mbarrier;
+//   * a persistent CTA owns a contiguous range of tiles; a tile is TP
+//     consecutive pools of one request, i.e. up to 128 contiguous token rows
+//     of k and of gate; a producer warp moves each tile with 1-D bulk copies
+//     (cp.async.bulk) into a shared-memory ring -- the k rows, the gate rows
+//     and the 16-byte-aligned span of validity bytes covering them -- all
+//     completing on one mbarrier, so no consumer waits on a global load;
 //   * a half-warp handles one pool; lane l owns channels 8l..8l+7 (one 16-byte
 //     vector of each row), LayerNorm statistics are half-warp shuffle sums;
 //   * the per-channel softmax over the kpool slots is done in fp32 registers
 //     (max-subtracted, exp2 with log2(e) folded into the logits);
-//   * the first valid token is found by a warp-wide ballot scan of the
-//     request's validity bytes (16-byte loads).
+//   * the first valid token of a request is found by a warp-wide ballot scan
+//     of its validity bytes (16-byte loads).
 #pragma once
 
 #include "common.cuh"
@@ -207,14 +209,17 @@ DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *g
 
 struct CmpMeta {
     int b, p0, p1, n_in, f, rs;
-    uint32_t okmask[4];   // bit i: pool p0+i has every slot valid (i < 128)
+    int voff;             // validity byte of the tile's first row in the stage's byte window
 };
+// A stage's validity window: the 16-byte-aligned span of validity bytes that
+// covers the tile's rows (at most 128 rows + 2 x 15 bytes of alignment).
+constexpr int kCmpValidWindow = 160;
 
 // Persistent kernel: CTA c owns a contiguous range of (request, pool-tile) work
-// items. Warp 8 is the producer: it finds each request's first valid token (a
-// warp ballot scan, cached across the request's tiles) and streams the tile's
-// contiguous k and gate rows into a 3-stage shared-memory ring with two 1-D
-// bulk copies per tile. Warps 0-7 consume: a half-warp per pool.
+// items. The last warp is the producer: it finds each request's first valid
+// token (a warp ballot scan, cached across the request's tiles) and streams each
+// tile's k rows, gate rows and validity bytes into the shared-memory ring. The
+// other warps consume: a half-warp per pool.
 template <int KP>
 __global__ void __launch_bounds__(CmpCfg<KP>::kThreads, 1)
 kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ gate,
@@ -235,6 +240,7 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     __shared__ __align__(16) float s_ape[KP * kD];   // ape * log2(e)
     __shared__ __align__(8) uint64_t full[kCmpStages], empty[kCmpStages];
     __shared__ CmpMeta meta[kCmpStages];
+    __shared__ __align__(16) uint8_t s_valid[kCmpStages][kCmpValidWindow];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x;
@@ -256,6 +262,7 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     if (warp == kCmpConsumers / 32) {
         // ---------------------------------------------------------------- producer warp
         int cur_b = -1, cur_f = 0, cur_rs = 0, cur_T = 0;
+        const long long total = req_start[B];      // rows of the validity array
         for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
             const int s = i % kCmpStages;
             bool ok = true;
@@ -272,33 +279,28 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             const int p1 = min(p0 + TP, max_pools);
             const int n_span = min(max_pools, (cur_T - cur_f) / KP);
             const int n_in = max(0, min(p1, n_span) - p0);
-            // Pool validity for the tile (all slot tokens valid), one pool per lane,
-            // computed here so the consumers never wait on a global load.
-            uint32_t okm[4] = {0u, 0u, 0u, 0u};
-            const size_t tok_base = (size_t)cur_rs + cur_f + (size_t)p0 * KP;
-#pragma unroll
-            for (int w4 = 0; w4 < 4; ++w4) {
-                if (32 * w4 >= n_in) break;
-                const int i = 32 * w4 + lane;
-                bool pv = i < n_in;
-                if (pv) {
-                    uint8_t vb[KP];
-#pragma unroll
-                    for (int ss = 0; ss < KP; ++ss) vb[ss] = valid[tok_base + (size_t)i * KP + ss];
-#pragma unroll
-                    for (int ss = 0; ss < KP; ++ss) pv = pv && vb[ss] != 0;
-                }
-                okm[w4] = __ballot_sync(0xffffffffu, pv);
-            }
+            // The tile's rows of k and gate, and the 16-byte-aligned span of
+            // validity bytes covering them, arrive together by bulk copy; the
+            // span stops at the last whole 16-byte chunk of the array and any
+            // rows past that (the array's last few bytes) are read by plain loads.
+            const long long row0 = (long long)cur_rs + cur_f + (long long)p0 * KP;
+            const long long row1 = row0 + (long long)n_in * KP;
+            const long long vs = row0 & ~15ll;
+            const long long ve = min((row1 + 15) & ~15ll, max(vs, total & ~15ll));
+            const uint32_t vbytes = n_in > 0 ? (uint32_t)(ve - vs) : 0u;
+            if (n_in > 0)
+                for (long long r = max(ve, row0) + lane; r < row1; r += 32)
+                    s_valid[s][r - vs] = valid[r];
+            __syncwarp();
             if (lane == 0) {
-                meta[s] = CmpMeta{b, p0, p1, n_in, cur_f, cur_rs, {okm[0], okm[1], okm[2], okm[3]}};
+                meta[s] = CmpMeta{b, p0, p1, n_in, cur_f, cur_rs, (int)(row0 - vs)};
                 if (n_in > 0) {
                     const uint32_t bytes = (uint32_t)(n_in * KP * kD * 2);
-                    const size_t row0 = (size_t)cur_rs + cur_f + (size_t)p0 * KP;
                     __nv_bfloat16 *sk = reinterpret_cast<__nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
-                    mbar_arrive_expect_tx(&full[s], 2 * bytes);
+                    mbar_arrive_expect_tx(&full[s], 2 * bytes + vbytes);
                     bulk_g2s(sk, k + row0 * kD, bytes, &full[s]);
                     bulk_g2s(sk + kCmpTileTokens * kD, gate + row0 * kD, bytes, &full[s]);
+                    if (vbytes > 0) bulk_g2s(&s_valid[s][0], valid + vs, vbytes, &full[s]);
                 } else {
                     mbar_arrive(&full[s]);
                 }
@@ -336,7 +338,10 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             const bool active = ii + (hw & 1) < m.n_in;
             const int pi = active ? ii + (hw & 1) : ii;
             const int p = m.p0 + pi;
-            const bool ok = (m.okmask[pi >> 5] >> (pi & 31)) & 1u;
+            // pool valid iff every slot token is valid (read from the stage's window)
+            bool ok = true;
+#pragma unroll
+            for (int ss = 0; ss < KP; ++ss) ok = ok && s_valid[s][m.voff + pi * KP + ss] != 0;
             const uint4 o = compress_pool<KP>(sk + (size_t)pi * KP * kD + 8 * l,
                                               sg + (size_t)pi * KP * kD + 8 * l, s_ape, lw, lb,
                                               eps, l, ok);

@@ -92,9 +92,11 @@ struct MlaGeom {
     bool cluster;  // splits merged inside a thread-block cluster
 };
 
-// As many splits as keep the grid within one wave of CTAs, no split holding
-// more chunks than needed for that; every split then holds at least one id.
-inline MlaGeom mla_geometry(int Q, int Hm, int W) {
+// The split plan, the same on every device: as many splits as keep the grid
+// within one wave of CTAs, no split holding more chunks than needed for that;
+// every split then holds at least one id. The workspace is sized for this plan
+// merged through global partials.
+inline MlaGeom mla_plan(int Q, int Hm, int W) {
     MlaGeom g{1, kTcChunk, false};
     if (Q <= 0 || W <= 0) return g;
     const long long ctas = (long long)Q * ((Hm + kTcHeads - 1) / kTcHeads);
@@ -103,14 +105,13 @@ inline MlaGeom mla_geometry(int Q, int Hm, int W) {
     if (ctas < kSmTarget) per_chunks = ceil_div(chunks, (int)(kSmTarget / ctas));
     g.per = per_chunks * kTcChunk;
     g.S = ceil_div(chunks, per_chunks);
-    g.cluster = g.S >= 2 && g.S <= kMaxClusterSplits;
     return g;
 }
 
 inline size_t mla_workspace_bytes(int Q, int Hm, int W) {
     if (Q <= 0 || Hm <= 0) return 0;
-    const MlaGeom g = mla_geometry(Q, Hm, W);
-    if (g.S == 1 || g.cluster) return 0;
+    const MlaGeom g = mla_plan(Q, Hm, W);
+    if (g.S == 1) return 0;
     return (size_t)Q * g.S * Hm * kPartStride * sizeof(float);
 }
 
@@ -301,15 +302,18 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __nv_bfloat16 *_
             const int j = c * kTcChunk + lane;
             return (c < nch && j < ntok) ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
         };
-        int next_id = load_id(0);
+        // The ids of the next eight chunks are in flight at any time: slot u of
+        // the queue holds chunk c0+u and is refilled with chunk c0+u+8 as soon as
+        // it is consumed (static slots, so no register waits on a pending load).
+        int idq[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) idq[i] = load_id(i);
         int issued = 0;
-        for (int c = 0; c < nch; ++c) {
+        auto gather_chunk = [&](int c, int id) -> bool {
             const int s = c % kTcStages;
-            const int id = next_id;
-            next_id = load_id(c + 1);                      // in flight during this chunk's wait
             bool ok = true;
             if (c >= kTcStages) ok = tc_wait(ctl, &ctl->kv_empty[s], ((c / kTcStages) - 1) & 1);
-            if (!__all_sync(0xffffffffu, ok)) break;
+            if (!__all_sync(0xffffffffu, ok)) return false;
             const bool valid = id >= 0 && id < T && (long long)rs + id < (long long)kv_rows;
             const uint32_t vm = __ballot_sync(0xffffffffu, valid);
             const int y = valid ? rs + id : map_rows;      // past the map: a zero row
@@ -329,6 +333,18 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __nv_bfloat16 *_
                                 &ctl->kv_full[s]);
             }
             issued = c + 1;
+            return true;
+        };
+        bool go = true;
+        for (int c0 = 0; go && c0 < nch; c0 += 8) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int c = c0 + u;
+                if (!go || c >= nch) break;
+                const int id = idq[u];
+                idq[u] = load_id(c + 8);
+                go = gather_chunk(c, id);
+            }
         }
         // After an abort, copies may still be in flight: let them land (bounded)
         // before the CTA moves on.
@@ -570,15 +586,15 @@ mla_combine_kernel(const float *__restrict__ part, int Hm, int S, __nv_bfloat16 
         lse[(size_t)q * Hm + h] = lsum > 0.f ? (M + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
 }
 
-// Whether clusters of `splits` CTAs of the cluster kernel can be resident on
-// the current device (asked once per device and size, after the kernel's
-// shared-memory limit is raised).
-inline bool mla_cluster_fits(int splits) {
-    static std::atomic<int> known[64][kMaxClusterSplits + 1];   // 0 unknown, 1 yes, 2 no
+// How many clusters of `splits` CTAs of the cluster kernel can be resident at
+// once on the current device (asked once per device and size, after the
+// kernel's shared-memory limit is raised); 0 when none or unknown.
+inline int mla_max_clusters(int splits) {
+    static std::atomic<int> known[64][kMaxClusterSplits + 1];   // count + 1; 0 = not asked
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     const int k = known[dev][splits].load(std::memory_order_relaxed);
-    if (k != 0) return k == 1;
+    if (k != 0) return k - 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(splits, 1, 1);
     cfg.blockDim = dim3(kTcThreads);
@@ -591,11 +607,29 @@ inline bool mla_cluster_fits(int splits) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    const bool ok = cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel<true>, &cfg) == cudaSuccess &&
-                    n >= 1;
+    if (cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel<true>, &cfg) != cudaSuccess) n = 0;
     (void)cudaGetLastError();
-    known[dev][splits].store(ok ? 1 : 2, std::memory_order_relaxed);
-    return ok;
+    known[dev][splits].store(n + 1, std::memory_order_relaxed);
+    return n;
+}
+
+// The launch: a plan of 2..8 splits runs as clusters when all of a grid's
+// clusters can be resident at once, shrinking the cluster (more chunks per CTA)
+// while that costs at most two chunks per CTA over the plan -- about what the
+// global merge costs; otherwise the plan runs with global partials.
+inline MlaGeom mla_launch_geometry(int Q, int Hm, int W) {
+    MlaGeom g = mla_plan(Q, Hm, W);
+    if (g.S < 2 || g.S > kMaxClusterSplits) return g;
+    const long long ctas = (long long)Q * ((Hm + kTcHeads - 1) / kTcHeads);
+    const int chunks = ceil_div(W, kTcChunk);
+    const int base = g.per / kTcChunk;
+    for (int s = g.S; s >= 2; --s) {
+        const int pc = ceil_div(chunks, s);
+        if (pc > base + 2) break;
+        const int ss = ceil_div(chunks, pc);
+        if ((long long)mla_max_clusters(ss) >= ctas) return MlaGeom{ss, pc * kTcChunk, true};
+    }
+    return g;
 }
 
 inline int sparse_mla_launch(const void *q, const void *kv, int64_t kv_rows,
@@ -618,14 +652,12 @@ inline int sparse_mla_launch(const void *q, const void *kv, int64_t kv_rows,
     if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(req_start, 4) || !aligned(q_req, 4) ||
         !aligned(token_ids, 4) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(ws, 16))
         return DSA_ERR_ALIGNMENT;
-    const MlaGeom g = mla_geometry(Q, Hm, W);
     const size_t need = mla_workspace_bytes(Q, Hm, W);
     if (need > 0 && (!ws || ws_bytes < need)) return DSA_ERR_WORKSPACE;
-    if (g.cluster) {
-        if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true>), kTcSmemBytes))
-            return DSA_ERR_CUDA;
-        if (!mla_cluster_fits(g.S)) return DSA_ERR_UNSUPPORTED;
-    }
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true>), kTcSmemBytes) ||
+        !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<false>), kTcSmemBytes))
+        return DSA_ERR_CUDA;
+    const MlaGeom g = mla_launch_geometry(Q, Hm, W);
     // With no cache rows the map spans q's first row; every id is then invalid
     // and reads row 1, past the map.
     const int map_rows = kv_rows > 0 ? (int)kv_rows : 1;
@@ -646,8 +678,6 @@ inline int sparse_mla_launch(const void *q, const void *kv, int64_t kv_rows,
             return DSA_ERR_CUDA;
         return launch_status();
     }
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<false>), kTcSmemBytes))
-        return DSA_ERR_CUDA;
     if (launch_pdl(mla_tc_kernel<false>, grid, dim3(kTcThreads), kTcSmemBytes, stream, kv_map, qb,
                    req_start, q_req, token_ids, B, (int)kv_rows, map_rows, Hm, W, g.S, g.per,
                    scale_log2, part, ob, lse) != cudaSuccess)

@@ -109,13 +109,14 @@ def test_topk_expand_refusals(B):
 
 def test_sparse_mla_refusals(B):
     L = B.lib
-    # 2 queries: 64 splits of one chunk, merged through the workspace
+    # partials of every split (the plan keeps the grid within 148 CTAs):
+    # 2 queries -> 64 splits of one chunk; 16 queries -> 8 splits of 8 chunks
     ws = B.dsa_sparse_mla_workspace_size(2, 64, 2048)
     assert ws == 2 * 64 * 64 * 516 * 4
-    # 16 queries: 8 splits per query merged inside a cluster, no workspace
-    assert B.dsa_sparse_mla_workspace_size(16, 64, 2048) == 0
+    assert B.dsa_sparse_mla_workspace_size(16, 64, 2048) == 16 * 8 * 64 * 516 * 4
     # at least 148 CTAs without splitting: one split, no workspace
     assert B.dsa_sparse_mla_workspace_size(148, 64, 2048) == 0
+    assert B.dsa_sparse_mla_workspace_size(74, 128, 2048) == 0
 
     def call(**kw):
         a = dict(q=FAKE, kv=FAKE, rows=1 << 20, rs=FAKE, qr=FAKE, ids=FAKE, Q=2, B=2, Hm=64,
