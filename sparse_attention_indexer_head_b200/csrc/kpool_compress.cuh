@@ -72,17 +72,9 @@ DSA_DEVINL int first_valid_scan(const uint8_t *__restrict__ valid, int rs, int T
     return T;
 }
 
-// Half-warp (16 lanes) butterfly sum; lanes of the other half-warp run their own.
-DSA_DEVINL float hsum16(float v) {
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    return v;
-}
-
 // One pool on a half-warp: lane l owns channels 8l..8l+7 of the kpool slot rows
 // at krow/grow (shared memory), held as four fp32 pairs so the arithmetic runs
-// as packed fp32x2 (FFMA2 / FADD2 / FMUL2) instructions. Returns the packed
-// bf16 pooled key chunk (zero when the pool is invalid).
+// as packed fp32x2 (FFMA2 / FADD2 / FMUL2) instructions.
 DSA_DEVINL void unpack8x2(const uint4 &v, float2 (&x)[4]) {
     x[0] = make_float2(bf16lo(v.x), bf16hi(v.x));
     x[1] = make_float2(bf16lo(v.y), bf16hi(v.y));
@@ -96,72 +88,107 @@ DSA_DEVINL float2 round_bf16x2(float2 y) {
     return make_float2(bf16lo(p), bf16hi(p));
 }
 
+// LayerNorm statistics of a tile's token rows, four threads per row: thread q of
+// a row's group sums the 16-byte pieces q, q+4, q+8, q+12 (rotated by four
+// pieces on odd rows, so the eight threads of a shared-memory phase touch eight
+// distinct bank groups). The moments are shifted by a sample of the row (the
+// group's first loaded value), which lies within a few standard deviations of
+// the mean, so their difference does not cancel. Stores (rstd, -mu * rstd).
+// Every thread of the consumer group calls it (warp-uniform loop).
+DSA_DEVINL void token_stats(const __nv_bfloat16 *sk, int ntok, float eps, float2 *stat, int ctid,
+                            int nthreads) {
+    const int q = ctid & 3, lane = ctid & 31;
+    for (int tok0 = 0; tok0 < ntok; tok0 += nthreads / 4) {
+        const int tok = tok0 + (ctid >> 2);
+        const bool act = tok < ntok;
+        const int rot = 4 * (tok & 1);
+        uint4 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int piece = (q + 4 * i + rot) & 15;
+            v[i] = act ? *reinterpret_cast<const uint4 *>(sk + (size_t)tok * kD + piece * 8)
+                       : make_uint4(0u, 0u, 0u, 0u);
+        }
+        const float x0 = __shfl_sync(0xffffffffu, bf16lo(v[0].x), lane & ~3);
+        const float2 nx0 = make_float2(-x0, -x0);
+        float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 x[4];
+            unpack8x2(v[i], x);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float2 d = __fadd2_rn(x[c], nx0);
+                s1 = __fadd2_rn(s1, d);
+                s2 = __ffma2_rn(d, d, s2);
+            }
+        }
+        float a1 = s1.x + s1.y, a2 = s2.x + s2.y;
+        a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+        a2 += __shfl_xor_sync(0xffffffffu, a2, 1);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+        a2 += __shfl_xor_sync(0xffffffffu, a2, 2);
+        const float dm = a1 * (1.0f / kD);
+        const float var = fmaxf(fmaf(-dm, dm, a2 * (1.0f / kD)), 0.f);
+        const float mu = x0 + dm;
+        const float r = rsqrt_approx(var + eps);
+        if (act && q == 0) stat[tok] = make_float2(r, -mu * r);
+    }
+}
+
+// The pooled key chunk of lane l (channels 8l..8l+7) from the pool's kpool
+// k rows and gate rows, with the rows' LayerNorm statistics st[s]. s_ape holds
+// ape * log2(e) laid out [slot][half][lane][4] so a half-warp's loads are
+// contiguous. Returns the packed bf16 chunk (zero when the pool is invalid).
 template <int KP>
 DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *grow,
-                               const float *s_ape, const float2 (&lw)[4], const float2 (&lb)[4],
-                               float eps, int l, bool ok) {
-    // kpool <= 4: the k rows and slot logits stay in registers between the two
-    // passes; larger pools re-read them from shared memory (register budget).
+                               const float2 *st, const float *s_ape, const float2 (&lw)[4],
+                               const float2 (&lb)[4], int l, bool ok) {
+    // kpool <= 4: the k_norm rows and slot logits stay in registers between the
+    // two passes; larger pools recompute them from shared memory (register budget).
     constexpr bool kKeep = KP <= 4;
     const float2 log2e2 = make_float2(kLog2e, kLog2e);
-    float2 xk[kKeep ? KP : 1][4], lgk[kKeep ? KP : 1][4];
-    float rr[KP], nmr[KP];
+    float2 knk[kKeep ? KP : 1][4], lgk[kKeep ? KP : 1][4];
     float2 mx2[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) mx2[c] = make_float2(-INFINITY, -INFINITY);
 
+    auto knorm = [&](int s, float2 (&kn)[4]) {
+        const float2 rs = st[s];
+        const float2 r2 = make_float2(rs.x, rs.x), n2 = make_float2(rs.y, rs.y);
+        float2 x[4];
+        unpack8x2(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            kn[c] = round_bf16x2(__ffma2_rn(__ffma2_rn(x[c], r2, n2), lw[c], lb[c]));
+    };
     auto logits = [&](int s, float2 (&lg)[4]) {
         float2 g[4];
         unpack8x2(*reinterpret_cast<const uint4 *>(grow + s * kD), g);
-        const float4 a0 = *reinterpret_cast<const float4 *>(s_ape + s * kD + 8 * l);
-        const float4 a1 = *reinterpret_cast<const float4 *>(s_ape + s * kD + 8 * l + 4);
+        const float4 a0 = *reinterpret_cast<const float4 *>(s_ape + (s * 2) * 64 + 4 * l);
+        const float4 a1 = *reinterpret_cast<const float4 *>(s_ape + (s * 2 + 1) * 64 + 4 * l);
         lg[0] = __ffma2_rn(g[0], log2e2, make_float2(a0.x, a0.y));
         lg[1] = __ffma2_rn(g[1], log2e2, make_float2(a0.z, a0.w));
         lg[2] = __ffma2_rn(g[2], log2e2, make_float2(a1.x, a1.y));
         lg[3] = __ffma2_rn(g[3], log2e2, make_float2(a1.z, a1.w));
     };
 
-    // Pass 1: LayerNorm statistics (two-pass mean / variance) and the running
-    // max of the slot logits (log2 units), per slot.
+    // Pass 1: bf16 k_norm rows, slot logits (log2 units) and their running max.
 #pragma unroll
     for (int s = 0; s < KP; ++s) {
-        float2 x[4];
-        unpack8x2(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
-        // Shifted one-pass moments: sums of d = x - x0 and d^2 with x0 the row's
-        // channel 0 (within a few standard deviations of the mean, so the
-        // difference of moments does not cancel); both reduced in one chain.
-        const float x0 = __shfl_sync(0xffffffffu, x[0].x, 0, 16);
-        const float2 nx0 = make_float2(-x0, -x0);
-        float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const float2 d = __fadd2_rn(x[c], nx0);
-            s1 = __fadd2_rn(s1, d);
-            s2 = __ffma2_rn(d, d, s2);
-        }
-        float a1 = s1.x + s1.y, a2 = s2.x + s2.y;
-#pragma unroll
-        for (int off = 8; off > 0; off >>= 1) {
-            a1 += __shfl_xor_sync(0xffffffffu, a1, off);
-            a2 += __shfl_xor_sync(0xffffffffu, a2, off);
-        }
-        const float dm = a1 * (1.0f / kD);
-        const float var = fmaxf(fmaf(-dm, dm, a2 * (1.0f / kD)), 0.f);
-        const float mu = x0 + dm;
-        rr[s] = rsqrt_approx(var + eps);
-        nmr[s] = -mu * rr[s];
-        float2 lg[4];
+        float2 kn[4], lg[4];
+        knorm(s, kn);
         logits(s, lg);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             mx2[c] = make_float2(fmaxf(mx2[c].x, lg[c].x), fmaxf(mx2[c].y, lg[c].y));
             if constexpr (kKeep) {
-                xk[s][c] = x[c];
+                knk[s][c] = kn[c];
                 lgk[s][c] = lg[c];
             }
         }
     }
-    // Pass 2: per-channel softmax over the slots, weighted sum of the bf16 k_norm rows.
+    // Pass 2: per-channel softmax over the slots, weighted sum of the k_norm rows.
     float2 nmx[4], den[4], acc[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -171,26 +198,23 @@ DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *g
     }
 #pragma unroll
     for (int s = 0; s < KP; ++s) {
-        float2 x[4], lg[4];
+        float2 kn[4], lg[4];
         if constexpr (kKeep) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                x[c] = xk[s][c];
+                kn[c] = knk[s][c];
                 lg[c] = lgk[s][c];
             }
         } else {
-            unpack8x2(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
+            knorm(s, kn);
             logits(s, lg);
         }
-        const float2 r2 = make_float2(rr[s], rr[s]), nmr2 = make_float2(nmr[s], nmr[s]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            const float2 t = __ffma2_rn(x[c], r2, nmr2);              // (x - mu) * rstd
-            const float2 kn = round_bf16x2(__ffma2_rn(t, lw[c], lb[c]));
             const float2 z = __fadd2_rn(lg[c], nmx[c]);
             const float2 e = make_float2(ex2(z.x), ex2(z.y));
             den[c] = __fadd2_rn(den[c], e);
-            acc[c] = __ffma2_rn(e, kn, acc[c]);
+            acc[c] = __ffma2_rn(e, kn[c], acc[c]);
         }
     }
     uint4 o = make_uint4(0, 0, 0, 0);
@@ -237,7 +261,8 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     constexpr int kCmpConsumers = C::kConsumers;
     constexpr int kCmpThreads = C::kThreads;
     extern __shared__ __align__(128) uint8_t cmp_smem[];
-    __shared__ __align__(16) float s_ape[KP * kD];   // ape * log2(e)
+    __shared__ __align__(16) float s_ape[KP * kD];   // ape * log2(e), [slot][half][lane][4]
+    __shared__ __align__(16) float2 s_stat[kCmpStages][kCmpTileTokens];   // (rstd, -mu*rstd)
     __shared__ __align__(8) uint64_t full[kCmpStages], empty[kCmpStages];
     __shared__ CmpMeta meta[kCmpStages];
     __shared__ __align__(16) uint8_t s_valid[kCmpStages][kCmpValidWindow];
@@ -254,7 +279,10 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         }
         fence_mbarrier_init();
     }
-    for (int i = tid; i < KP * kD; i += kCmpThreads) s_ape[i] = ape[i] * kLog2e;
+    for (int i = tid; i < KP * kD; i += kCmpThreads) {
+        const int sl = i / kD, c = i % kD;
+        s_ape[(sl * 2 + ((c >> 2) & 1)) * 64 + 4 * (c >> 3) + (c & 3)] = ape[i] * kLog2e;
+    }
     __syncthreads();
     pdl_wait();
     pdl_launch_dependents();
@@ -332,6 +360,10 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         for (int x = m.n_in + tid; x < m.p1 - m.p0; x += kCmpConsumers)
             pool_valid[pool_base + m.p0 + x] = 0;
 
+        // LayerNorm statistics of the tile's rows, then every pool of the tile.
+        token_stats(sk, m.n_in * KP, eps, &s_stat[s][0], tid, kCmpConsumers);
+        asm volatile("bar.sync 1, %0;" ::"n"(kCmpConsumers) : "memory");
+
         // Warp-uniform loop: the two half-warps of a warp take pools ii and ii+1;
         // a half-warp past the tile computes on a loaded row and stores nothing.
         for (int ii = 2 * warp; ii < m.n_in; ii += kCmpConsumers / 16) {
@@ -343,8 +375,8 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
 #pragma unroll
             for (int ss = 0; ss < KP; ++ss) ok = ok && s_valid[s][m.voff + pi * KP + ss] != 0;
             const uint4 o = compress_pool<KP>(sk + (size_t)pi * KP * kD + 8 * l,
-                                              sg + (size_t)pi * KP * kD + 8 * l, s_ape, lw, lb,
-                                              eps, l, ok);
+                                              sg + (size_t)pi * KP * kD + 8 * l,
+                                              &s_stat[s][pi * KP], s_ape, lw, lb, l, ok);
             if (!active) continue;
             *reinterpret_cast<uint4 *>(pool_keys + (pool_base + p) * kD + 8 * l) = o;
             if (l < KP) pool_idx[(pool_base + p) * KP + l] = ok ? m.f + p * KP + l : -1;

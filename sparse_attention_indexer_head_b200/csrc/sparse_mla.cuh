@@ -239,12 +239,13 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __nv_bfloat16 *_
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
-    pdl_wait();                       // token ids come from the predecessor grid
-    pdl_launch_dependents();
+    // Request geometry is a step input: read before the wait on the predecessor.
     const int b = q_req[qi];
     const bool req_ok = b >= 0 && b < B;
     const int rs = req_ok ? req_start[b] : 0;
     const int T = req_ok ? max(0, req_start[b + 1] - rs) : 0;
+    pdl_wait();                       // token ids come from the predecessor grid
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------------ MMA issuer
@@ -354,10 +355,14 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __nv_bfloat16 *_
         __syncwarp();
     } else if (warp >= 4) {
         // ------------------------------------------------------------------ softmax (128 threads)
-        const int st = tid - 128, wq = warp - 4;
-        const int hh = 16 * wq + lane;        // head row owned by lanes 0..15
-        const bool owner = lane < 16;
-        (void)st;
+        // S is read with the 16x64b tensor-memory shape, so every lane works:
+        // thread t of warp 4+w holds head row hh = 16w + (t>>2) + 8(t&1) and the
+        // chunk's tokens of parity par = (t>>1)&1; its partner t^2 holds the
+        // other parity of the same head. Row max and sum take one exchange.
+        const int wq = warp - 4;
+        const int hh = 16 * wq + (lane >> 2) + 8 * (lane & 1);
+        const int par = (lane >> 1) & 1;
+        const bool owner = par == 0;          // writes the head's per-row values
         tc::cp_async_wait_all();          // this thread's Q copies (issued at entry)
         tc::fence_proxy_async_smem();
         mbar_arrive(&ctl->q_full);
@@ -369,52 +374,61 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __nv_bfloat16 *_
             const int s = c % kTcStages, sb = c & 1;
             bool bad = !tc_wait(ctl, &ctl->kv_full[s], (c / kTcStages) & 1);
             bad = bad || !tc_wait(ctl, &ctl->s_full[sb], (c >> 1) & 1);
-            if (tc::named_bar_or(2, 128, bad)) { failed = true; break; }
             tc::fence_after_sync();
-            uint32_t r[kTcChunk];
-            tc::tmem_ld32(tl + 256 + sb * kTcChunk, r);
+            uint32_t r[kTcChunk / 2];
+            tc::tmem_ld16x64b_x16(tl + 256 + sb * kTcChunk, r);
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             mbar_arrive(&ctl->s_empty[sb]);
 
-            const uint32_t vm = ctl->vmask[s];
+            const uint32_t vm = ctl->vmask[s] >> par;        // bit 2i: token par + 2i
+            float z[kTcChunk / 2];
             float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < kTcChunk; ++j) {
-                const float z = ((vm >> j) & 1) ? __uint_as_float(r[j]) * scale_log2 : -INFINITY;
-                r[j] = __float_as_uint(z);
-                mx = fmaxf(mx, z);
+            for (int i = 0; i < kTcChunk / 2; ++i) {
+                z[i] = ((vm >> (2 * i)) & 1) ? __uint_as_float(r[i]) * scale_log2 : -INFINITY;
+                mx = fmaxf(mx, z[i]);
             }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
             float alpha = 1.f;
             if (mx > m_used + kLazyRescale) {
                 alpha = ex2(m_used - mx);
                 m_used = mx;
             }
-            uint32_t pk[kTcChunk / 2];
+            float pv[kTcChunk / 2];
             float psum = 0.f;
 #pragma unroll
-            for (int j = 0; j < kTcChunk / 2; ++j) {
-                const float z0 = __uint_as_float(r[2 * j]), z1 = __uint_as_float(r[2 * j + 1]);
-                const float p0 = z0 == -INFINITY ? 0.f : ex2(z0 - m_used);
-                const float p1 = z1 == -INFINITY ? 0.f : ex2(z1 - m_used);
-                pk[j] = pack_bf16x2(p0, p1);
-                psum += p0 + p1;     // fp32 weights: the row sum and lse stay exact to fp32
+            for (int i = 0; i < kTcChunk / 2; ++i) {
+                pv[i] = z[i] == -INFINITY ? 0.f : ex2(z[i] - m_used);
+                psum += pv[i];       // fp32 weights: the row sum and lse stay exact to fp32
             }
+            psum += __shfl_xor_sync(0xffffffffu, psum, 2);
             l = fmaf(l, alpha, psum);
             if (owner) ctl->alpha[hh] = alpha;
-
-            bad = c >= 2 && !tc_wait(ctl, &ctl->p_empty[sb], ((c >> 1) - 1) & 1);
-            if (tc::named_bar_or(2, 128, bad)) { failed = true; break; }
-            const bool need = tc::named_bar_or(2, 128, owner && c >= 1 && alpha != 1.f);
-            if (owner) {
+            // bf16 P row of the head: this thread packs tokens 16par .. 16par+15,
+            // taking the other parity from its partner.
+            uint32_t pk[8];
 #pragma unroll
-                for (int c4 = 0; c4 < kTcChunk / 8; ++c4) {
-                    const uint32_t dst = sP + sb * kStageP + hh * 64 + ((c4 ^ ((hh >> 1) & 3)) << 4);
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
-                                 "r"(pk[4 * c4]), "r"(pk[4 * c4 + 1]), "r"(pk[4 * c4 + 2]),
-                                 "r"(pk[4 * c4 + 3])
-                                 : "memory");
-                }
+            for (int k = 0; k < 8; ++k) {
+                const float recv = __shfl_xor_sync(0xffffffffu, par ? pv[k] : pv[k + 8], 2);
+                pk[k] = par ? pack_bf16x2(recv, pv[k + 8]) : pack_bf16x2(pv[k], recv);
+            }
+
+            bad = bad || (c >= 2 && !tc_wait(ctl, &ctl->p_empty[sb], ((c >> 1) - 1) & 1));
+            // One barrier per chunk; a second only when some head rescales or a wait failed.
+            bool need = false;
+            if (tc::named_bar_or(2, 128, bad || (owner && c >= 1 && alpha != 1.f))) {
+                if (tc::named_bar_or(2, 128, bad)) { failed = true; break; }
+                need = true;
+            }
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int c4 = 2 * par + h2;      // 16-byte piece of the 64-byte row
+                const uint32_t dst = sP + sb * kStageP + hh * 64 + ((c4 ^ ((hh >> 1) & 3)) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                             "r"(pk[4 * h2]), "r"(pk[4 * h2 + 1]), "r"(pk[4 * h2 + 2]),
+                             "r"(pk[4 * h2 + 3])
+                             : "memory");
             }
             if (need) {
                 // O^T columns of rescaled heads times alpha, after PV(c-1) has landed.
