@@ -23,17 +23,19 @@
 
 namespace dsa {
 
-// Geometry per kpool: small pools get 12 consumer warps and 96-token tiles in a
-// 4-stage ring; kpool > 4 (more live registers per lane) 8 warps and 128-token
-// tiles in a 3-stage ring. A stage holds the tile's k rows then its gate rows.
+// Geometry per kpool. kpool <= 4: 15 consumer warps (with the producer, four
+// warps per scheduler, so 128 registers a thread) and 120-token tiles -- four
+// threads per row in the statistics phase, two pools per warp (30 pools at kpool
+// 4); larger pools (more live registers) 8 warps and floor(128 / kpool) pools.
+// A stage holds the tile's k rows then its gate rows; three stages in the ring.
 template <int KP> struct CmpCfg {
-    static constexpr int kWarps = KP <= 4 ? 12 : 8;             // consumer warps
+    static constexpr int kWarps = KP <= 4 ? 15 : 8;             // consumer warps
     static constexpr int kConsumers = kWarps * 32;
     static constexpr int kThreads = kConsumers + 32;            // + 1 producer warp
-    static constexpr int kTileTokens = KP <= 4 ? 96 : 128;
-    static constexpr int kStages = KP <= 4 ? 4 : 3;
+    static constexpr int kTP = KP <= 4 ? 120 / KP : 128 / KP;   // pools per tile
+    static constexpr int kTileTokens = kTP * KP;
+    static constexpr int kStages = 3;
     static constexpr int kStageBytes = 2 * kTileTokens * 128 * 2;
-    static constexpr int kTP = kTileTokens / KP;                // pools per tile
 };
 constexpr int kD = DSA_INDEX_DIM;   // 128 channels
 constexpr float kLog2e = 1.4426950408889634f;
@@ -144,11 +146,12 @@ template <int KP>
 DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *grow,
                                const float2 *st, const float *s_ape, const float2 (&lw)[4],
                                const float2 (&lb)[4], int l, bool ok) {
-    // kpool <= 4: the k_norm rows and slot logits stay in registers between the
-    // two passes; larger pools recompute them from shared memory (register budget).
+    // Pass 1 forms the slot logits and their per-channel max; pass 2 forms the
+    // bf16 k_norm rows and the softmax-weighted sum. kpool <= 4 keeps the logits
+    // in registers between the passes, larger pools recompute them.
     constexpr bool kKeep = KP <= 4;
     const float2 log2e2 = make_float2(kLog2e, kLog2e);
-    float2 knk[kKeep ? KP : 1][4], lgk[kKeep ? KP : 1][4];
+    float2 lgk[kKeep ? KP : 1][4];
     float2 mx2[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) mx2[c] = make_float2(-INFINITY, -INFINITY);
@@ -173,22 +176,16 @@ DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *g
         lg[3] = __ffma2_rn(g[3], log2e2, make_float2(a1.z, a1.w));
     };
 
-    // Pass 1: bf16 k_norm rows, slot logits (log2 units) and their running max.
 #pragma unroll
     for (int s = 0; s < KP; ++s) {
-        float2 kn[4], lg[4];
-        knorm(s, kn);
+        float2 lg[4];
         logits(s, lg);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             mx2[c] = make_float2(fmaxf(mx2[c].x, lg[c].x), fmaxf(mx2[c].y, lg[c].y));
-            if constexpr (kKeep) {
-                knk[s][c] = kn[c];
-                lgk[s][c] = lg[c];
-            }
+            if constexpr (kKeep) lgk[s][c] = lg[c];
         }
     }
-    // Pass 2: per-channel softmax over the slots, weighted sum of the k_norm rows.
     float2 nmx[4], den[4], acc[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -201,14 +198,11 @@ DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *g
         float2 kn[4], lg[4];
         if constexpr (kKeep) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                kn[c] = knk[s][c];
-                lg[c] = lgk[s][c];
-            }
+            for (int c = 0; c < 4; ++c) lg[c] = lgk[s][c];
         } else {
-            knorm(s, kn);
             logits(s, lg);
         }
+        knorm(s, kn);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const float2 z = __fadd2_rn(lg[c], nmx[c]);

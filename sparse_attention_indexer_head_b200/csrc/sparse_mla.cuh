@@ -6,7 +6,7 @@
 //
 // Split-KV decode on the 5th-generation tensor cores: a query's W selected ids
 // are cut into S contiguous splits; one CTA per (split, query, 64-head group)
-// gathers its latent rows with TMA and runs an online softmax for every head.
+// gathers its latent rows and runs an online softmax for every head.
 // The S partials (O, running max m, running sum l) of a (query, head group)
 // are merged in split order, so results do not depend on scheduling:
 //   S == 1       the CTA normalises and writes bf16 out and the lse itself;
@@ -21,7 +21,6 @@
 
 #include "common.cuh"
 #include "tc_ptx.cuh"
-#include "tma.cuh"
 
 namespace dsa {
 
@@ -44,15 +43,15 @@ constexpr int kPartStride = kL + 4;
 // 32-lane quadrant, the M=64 layout).
 //
 // Warp roles (256 threads): warp 0 allocates tensor memory and one lane issues
-// every MMA; warp 1 is the producer: it turns the chunk's ids into cache rows
-// and gathers them with TMA (tile::gather4, four 128-byte rows per copy, eight
-// copies per group of four rows) straight into the swizzled 4-stage ring; an id
-// that is -1 or outside its request points past the end of the cache and reads
-// as a zero row. Nothing waits for a copy but the consumers, so all four stages
-// can be in flight. Warps 4-7 load Q, run the softmax (lane i < 16 of warp 4+w
-// owns head 16w+i), rescale O^T when a head's running max grows by more than
-// 2^8 (lazy rescaling), and write the epilogue. Warps 2-3 only take part in the
-// cluster merge.
+// every MMA; warps 1-3 gather, warp 1+(c mod 3) filling chunk c of a 4-stage
+// ring with 16-byte cp.async pieces straight into the 128B-swizzled layout (a
+// zero fill for ids that are -1 or outside the request). The copies' landing is
+// tracked by the stage's mbarrier (cp.async.mbarrier.arrive), so no gather warp
+// waits for its own copies and all four stages can be in flight. (Per-row TMA
+// copies -- tile::gather4 or a 1-D bulk copy per 1 KB row -- move only 12-20 GB/s
+// per SM here: their per-instruction cost, not the depth of the ring, bounds
+// them.) Warps 4-7 load Q, run the softmax, rescale O^T when a head's running
+// max grows by more than 2^8 (lazy rescaling), and write the epilogue.
 // ---------------------------------------------------------------------------------------
 constexpr int kTcThreads = 256;
 constexpr int kTcChunk = 32;                        // tokens per chunk
@@ -175,14 +174,13 @@ DSA_DEVINL void mla_cluster_merge(const TcCtl *ctl, uint32_t sO, int S, int nh, 
     }
 }
 
-// kv_map: the latent cache as [map_rows, 512] bf16 rows, box 64 x 1 with the
-// 128-byte swizzle; kv_rows of them are cache rows (map_rows = max(kv_rows, 1)).
+// kv: the latent cache, kv_rows rows of 512 bf16.
 template <bool kCluster>
 __global__ void __launch_bounds__(kTcThreads, 1)
-mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __nv_bfloat16 *__restrict__ qm,
+mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restrict__ kv,
               const int32_t *__restrict__ req_start, const int32_t *__restrict__ q_req,
-              const int32_t *__restrict__ token_ids, int B, int kv_rows, int map_rows, int Hm,
-              int W, int S, int per, float scale_log2, float *__restrict__ part,
+              const int32_t *__restrict__ token_ids, int B, int kv_rows, int Hm, int W, int S,
+              int per, float scale_log2, float *__restrict__ part,
               __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
     extern __shared__ uint8_t mla_smem_raw[];
     const uint32_t raw = smem_u32(mla_smem_raw);
@@ -219,7 +217,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __nv_bfloat16 *_
     }
     if (tid == 32) {
         for (int i = 0; i < kTcStages; ++i) {
-            mbar_init(&ctl->kv_full[i], 1);
+            mbar_init(&ctl->kv_full[i], 33);    // 32 lanes' copies + lane 0's arrive
             mbar_init(&ctl->kv_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -278,6 +276,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __nv_bfloat16 *_
                 if (!tc_wait(ctl, &ctl->kv_full[s], (c / kTcStages) & 1)) { ok = false; break; }
                 if (c >= 2 && !tc_wait(ctl, &ctl->s_empty[sb], ((c >> 1) - 1) & 1)) { ok = false; break; }
                 tc::fence_after_sync();
+                tc::fence_proxy_async_smem();     // the stage was written by cp.async
                 const uint32_t d = tmem + 256 + sb * kTcChunk;
                 const uint32_t kvs = sKV + s * kStageKV;
 #pragma unroll
@@ -295,21 +294,18 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __nv_bfloat16 *_
             if (ok && issue_pv(nch - 1)) tc::mma_commit(&ctl->o_final);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ producer
-        // Lane r holds row r's id; lane i < 8 gathers rows 4i..4i+3 of the chunk
-        // (eight gather4 copies, one per 64-latent column atom).
+    } else if (warp < 4) {
+        // ------------------------------------------------------------------ gather warps
+        // Warp 1+p fills chunks p, p+3, p+6, ...: lane r holds row r's id and the
+        // warp copies the chunk's 32 rows as 16-byte cp.async pieces into the
+        // swizzled stage (zero-filled for invalid ids). Each lane's copies arrive
+        // on the stage's barrier as they land, so no warp waits for its own copies
+        // and all four stages can be in flight.
+        const int pw = warp - 1;
         auto load_id = [&](int c) -> int {
             const int j = c * kTcChunk + lane;
             return (c < nch && j < ntok) ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
         };
-        // The ids of the next eight chunks are in flight at any time: slot u of
-        // the queue holds chunk c0+u and is refilled with chunk c0+u+8 as soon as
-        // it is consumed (static slots, so no register waits on a pending load).
-        int idq[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) idq[i] = load_id(i);
-        int issued = 0;
         auto gather_chunk = [&](int c, int id) -> bool {
             const int s = c % kTcStages;
             bool ok = true;
@@ -317,42 +313,41 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __nv_bfloat16 *_
             if (!__all_sync(0xffffffffu, ok)) return false;
             const bool valid = id >= 0 && id < T && (long long)rs + id < (long long)kv_rows;
             const uint32_t vm = __ballot_sync(0xffffffffu, valid);
-            const int y = valid ? rs + id : map_rows;      // past the map: a zero row
-            int yy[4];
+            const int myrow = valid ? rs + id : -1;
+            const uint32_t dst0 = sKV + s * kStageKV;
+#pragma unroll 4
+            for (int r = 0; r < kTcChunk; ++r) {
+                const int row = __shfl_sync(0xffffffffu, myrow, r);
+                const __nv_bfloat16 *src = row >= 0 ? kv + (size_t)row * kL : qm;   // qm: never read
+                const uint32_t nb = row >= 0 ? 16u : 0u;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) yy[i] = __shfl_sync(0xffffffffu, y, (4 * lane + i) & 31);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int cc = lane + 32 * hh;         // 16-byte piece of the 1 KB row
+                    const uint32_t dst = dst0 + (cc >> 3) * kAtomKV + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
+                    tc::cp_async16_zfill(dst, row >= 0 ? src + cc * 8 : src, nb);
+                }
+            }
             if (lane == 0) {
                 ctl->vmask[s] = vm;
-                mbar_arrive_expect_tx(&ctl->kv_full[s], kStageKV);
+                mbar_arrive(&ctl->kv_full[s]);             // releases vmask
             }
-            __syncwarp();
-            if (lane < kTcChunk / 4) {
-                const uint32_t dst = sKV + s * kStageKV + lane * 512;
-#pragma unroll
-                for (int cb = 0; cb < kL / 64; ++cb)
-                    tma_gather4(dst + cb * kAtomKV, &kv_map, cb * 64, yy[0], yy[1], yy[2], yy[3],
-                                &ctl->kv_full[s]);
-            }
-            issued = c + 1;
+            tc::cp_async_arrive_noinc(&ctl->kv_full[s]);
             return true;
         };
+        // ids of this warp's next two chunks are in flight (static queue slots)
+        int idq[2] = {load_id(pw), load_id(pw + 3)};
         bool go = true;
-        for (int c0 = 0; go && c0 < nch; c0 += 8) {
+        for (int c0 = pw; go && c0 < nch; c0 += 6) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int c = c0 + u;
+            for (int u = 0; u < 2; ++u) {
+                const int c = c0 + 3 * u;
                 if (!go || c >= nch) break;
                 const int id = idq[u];
-                idq[u] = load_id(c + 8);
+                idq[u] = load_id(c + 6);
                 go = gather_chunk(c, id);
             }
         }
-        // After an abort, copies may still be in flight: let them land (bounded)
-        // before the CTA moves on.
-        if (lane == 0)
-            for (int c = max(0, issued - kTcStages); c < issued; ++c)
-                (void)mbar_wait(&ctl->kv_full[c % kTcStages], (c / kTcStages) & 1);
-        __syncwarp();
+        tc::cp_async_wait_all();          // nothing of this warp in flight past here
     } else if (warp >= 4) {
         // ------------------------------------------------------------------ softmax (128 threads)
         // S is read with the 16x64b tensor-memory shape, so every lane works:
@@ -672,29 +667,23 @@ inline int sparse_mla_launch(const void *q, const void *kv, int64_t kv_rows,
         !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<false>), kTcSmemBytes))
         return DSA_ERR_CUDA;
     const MlaGeom g = mla_launch_geometry(Q, Hm, W);
-    // With no cache rows the map spans q's first row; every id is then invalid
-    // and reads row 1, past the map.
-    const int map_rows = kv_rows > 0 ? (int)kv_rows : 1;
-    CUtensorMap kv_map;
-    if (!make_map_bf16_2d(&kv_map, kv_rows > 0 ? kv : q, (uint64_t)map_rows, kL, kL * 2, 64, 1))
-        return DSA_ERR_CUDA;
     const float scale_log2 = sm_scale * 1.4426950408889634f;
     const int groups = (Hm + kTcHeads - 1) / kTcHeads;
     float *part = reinterpret_cast<float *>(ws);
     const auto *qb = reinterpret_cast<const __nv_bfloat16 *>(q);
+    const auto *kvb = reinterpret_cast<const __nv_bfloat16 *>(kv);
     auto *ob = reinterpret_cast<__nv_bfloat16 *>(out);
     const dim3 grid(g.S, Q, groups);
     if (g.cluster) {
         if (launch_pdl_cluster(mla_tc_kernel<true>, grid, dim3(kTcThreads), kTcSmemBytes, stream,
-                               g.S, kv_map, qb, req_start, q_req, token_ids, B, (int)kv_rows,
-                               map_rows, Hm, W, g.S, g.per, scale_log2, part, ob,
-                               lse) != cudaSuccess)
+                               g.S, qb, kvb, req_start, q_req, token_ids, B, (int)kv_rows, Hm,
+                               W, g.S, g.per, scale_log2, part, ob, lse) != cudaSuccess)
             return DSA_ERR_CUDA;
         return launch_status();
     }
-    if (launch_pdl(mla_tc_kernel<false>, grid, dim3(kTcThreads), kTcSmemBytes, stream, kv_map, qb,
-                   req_start, q_req, token_ids, B, (int)kv_rows, map_rows, Hm, W, g.S, g.per,
-                   scale_log2, part, ob, lse) != cudaSuccess)
+    if (launch_pdl(mla_tc_kernel<false>, grid, dim3(kTcThreads), kTcSmemBytes, stream, qb, kvb,
+                   req_start, q_req, token_ids, B, (int)kv_rows, Hm, W, g.S, g.per, scale_log2,
+                   part, ob, lse) != cudaSuccess)
         return DSA_ERR_CUDA;
     int st = launch_status();
     if (st != DSA_OK || g.S == 1) return st;

@@ -128,6 +128,19 @@ DSA_DEVINL void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" :
 DSA_DEVINL void cp_async16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+// 16-byte copy of which the first src_bytes (0 or 16) come from src and the rest
+// are zero-filled; with 0 nothing is read.
+DSA_DEVINL void cp_async16_zfill(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+// Arrive on bar once every cp.async this thread issued so far has landed (the
+// arrival is counted in the barrier's expected count: no pending increment).
+DSA_DEVINL void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
 DSA_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 DSA_DEVINL void st_shared_zero16(uint32_t dst) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
