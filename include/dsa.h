@@ -26,6 +26,14 @@
  *   - There is no fallback path: an unsupported shape is refused with
  *     DSA_ERR_UNSUPPORTED, never routed elsewhere ([mod.rs] Glm5NextDsaKernels
  *     doc: a missing DSA entry point is a hard error).
+ *   - Every kernel is launched with programmatic dependent launch: it may
+ *     start while the kernel before it on the stream drains, and waits for
+ *     that kernel (griddepcontrol.wait) before reading anything an earlier
+ *     stage of this path writes. Before that wait it already reads inputs the
+ *     path never writes: hidden and w (head gate); ape (kpool_compress); q,
+ *     q_req and req_start (sparse MLA). Write those before the kernel that
+ *     immediately precedes the call on the stream, or separate that kernel
+ *     from the call by a copy, an event wait or a host synchronisation.
  *   - Request geometry lives on the device: request b owns cache rows
  *     [req_start[b], req_start[b+1]) (T_b rows). Token ids are LOGICAL, i.e.
  *     relative to the request; the physical row is req_start[b] + id ([tap]:
