@@ -23,17 +23,16 @@
 
 namespace dsa {
 
-// Geometry: kpool <= 4 runs 31 consumer warps + 1 producer (1024 threads, so
-// at most 64 registers a thread), larger pools 23 + 1 (80 registers); a tile is
-// floor(124 / kpool) pools (up to 124 token rows); a stage holds the tile's k
-// rows then its gate rows (62 KB), three stages in the ring. The statistics
-// phase runs eight threads per row (992 threads = 124 rows); the pool phase one
-// warp per pool.
+// Geometry per kpool. kpool <= 4: 15 consumer warps (with the producer, four
+// warps per scheduler, so 128 registers a thread) and 120-token tiles -- four
+// threads per row in the statistics phase, two pools per warp (30 pools at kpool
+// 4); larger pools (more live registers) 8 warps and floor(128 / kpool) pools.
+// A stage holds the tile's k rows then its gate rows; three stages in the ring.
 template <int KP> struct CmpCfg {
-    static constexpr int kWarps = KP <= 4 ? 31 : 23;            // consumer warps
+    static constexpr int kWarps = KP <= 4 ? 15 : 8;             // consumer warps
     static constexpr int kConsumers = kWarps * 32;
     static constexpr int kThreads = kConsumers + 32;            // + 1 producer warp
-    static constexpr int kTP = 124 / KP;                        // pools per tile
+    static constexpr int kTP = KP <= 4 ? 120 / KP : 128 / KP;   // pools per tile
     static constexpr int kTileTokens = kTP * KP;
     static constexpr int kStages = 3;
     static constexpr int kStageBytes = 2 * kTileTokens * 128 * 2;
@@ -75,15 +74,14 @@ DSA_DEVINL int first_valid_scan(const uint8_t *__restrict__ valid, int rs, int T
     return T;
 }
 
+// One pool on a half-warp: lane l owns channels 8l..8l+7 of the kpool slot rows
+// at krow/grow (shared memory), held as four fp32 pairs so the arithmetic runs
+// as packed fp32x2 (FFMA2 / FADD2 / FMUL2) instructions.
 DSA_DEVINL void unpack8x2(const uint4 &v, float2 (&x)[4]) {
     x[0] = make_float2(bf16lo(v.x), bf16hi(v.x));
     x[1] = make_float2(bf16lo(v.y), bf16hi(v.y));
     x[2] = make_float2(bf16lo(v.z), bf16hi(v.z));
     x[3] = make_float2(bf16lo(v.w), bf16hi(v.w));
-}
-DSA_DEVINL void unpack4x2(const uint2 &v, float2 (&x)[2]) {
-    x[0] = make_float2(bf16lo(v.x), bf16hi(v.x));
-    x[1] = make_float2(bf16lo(v.y), bf16hi(v.y));
 }
 
 // Round a pair to bf16 (nearest even) and widen it back: the stored k_norm value.
@@ -92,29 +90,32 @@ DSA_DEVINL float2 round_bf16x2(float2 y) {
     return make_float2(bf16lo(p), bf16hi(p));
 }
 
-// LayerNorm statistics of a tile's token rows, eight threads per row: thread q
-// of a row's group sums the 16-byte pieces q and q+8 (a shared-memory phase of
-// eight threads reads one row's 128 contiguous bytes: no bank conflict). The
-// moments are shifted by a sample of the row (the group's first loaded value),
-// which lies within a few standard deviations of the mean, so their difference
-// does not cancel. Stores (rstd, -mu * rstd). Every consumer thread calls it
-// (warp-uniform loop).
+// LayerNorm statistics of a tile's token rows, four threads per row: thread q of
+// a row's group sums the 16-byte pieces q, q+4, q+8, q+12 (rotated by four
+// pieces on odd rows, so the eight threads of a shared-memory phase touch eight
+// distinct bank groups). The moments are shifted by a sample of the row (the
+// group's first loaded value), which lies within a few standard deviations of
+// the mean, so their difference does not cancel. Stores (rstd, -mu * rstd).
+// Every thread of the consumer group calls it (warp-uniform loop).
 DSA_DEVINL void token_stats(const __nv_bfloat16 *sk, int ntok, float eps, float2 *stat, int ctid,
                             int nthreads) {
-    const int q = ctid & 7, lane = ctid & 31;
-    for (int tok0 = 0; tok0 < ntok; tok0 += nthreads / 8) {
-        const int tok = tok0 + (ctid >> 3);
+    const int q = ctid & 3, lane = ctid & 31;
+    for (int tok0 = 0; tok0 < ntok; tok0 += nthreads / 4) {
+        const int tok = tok0 + (ctid >> 2);
         const bool act = tok < ntok;
-        uint4 v[2];
+        const int rot = 4 * (tok & 1);
+        uint4 v[4];
 #pragma unroll
-        for (int i = 0; i < 2; ++i)
-            v[i] = act ? *reinterpret_cast<const uint4 *>(sk + (size_t)tok * kD + (q + 8 * i) * 8)
+        for (int i = 0; i < 4; ++i) {
+            const int piece = (q + 4 * i + rot) & 15;
+            v[i] = act ? *reinterpret_cast<const uint4 *>(sk + (size_t)tok * kD + piece * 8)
                        : make_uint4(0u, 0u, 0u, 0u);
-        const float x0 = __shfl_sync(0xffffffffu, bf16lo(v[0].x), lane & ~7);
+        }
+        const float x0 = __shfl_sync(0xffffffffu, bf16lo(v[0].x), lane & ~3);
         const float2 nx0 = make_float2(-x0, -x0);
         float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 4; ++i) {
             float2 x[4];
             unpack8x2(v[i], x);
 #pragma unroll
@@ -125,11 +126,10 @@ DSA_DEVINL void token_stats(const __nv_bfloat16 *sk, int ntok, float eps, float2
             }
         }
         float a1 = s1.x + s1.y, a2 = s2.x + s2.y;
-#pragma unroll
-        for (int off = 1; off < 8; off <<= 1) {
-            a1 += __shfl_xor_sync(0xffffffffu, a1, off);
-            a2 += __shfl_xor_sync(0xffffffffu, a2, off);
-        }
+        a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+        a2 += __shfl_xor_sync(0xffffffffu, a2, 1);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+        a2 += __shfl_xor_sync(0xffffffffu, a2, 2);
         const float dm = a1 * (1.0f / kD);
         const float var = fmaxf(fmaf(-dm, dm, a2 * (1.0f / kD)), 0.f);
         const float mu = x0 + dm;
@@ -138,84 +138,89 @@ DSA_DEVINL void token_stats(const __nv_bfloat16 *sk, int ntok, float eps, float2
     }
 }
 
-// One pool on a warp: lane l owns channels 4l..4l+3 of the kpool slot rows at
-// krow/grow (shared memory) as two fp32 pairs (packed fp32x2 arithmetic), with
-// the rows' LayerNorm statistics st[s] and s_ape = ape * log2(e) ([slot][128]).
-// Pass 1 forms the slot logits and their per-channel max; pass 2 the bf16
-// k_norm rows and the softmax-weighted sum. kpool <= 4 keeps the logits in
-// registers between the passes, larger pools recompute them. Returns the
-// packed bf16 chunk (zero when the pool is invalid).
+// The pooled key chunk of lane l (channels 8l..8l+7) from the pool's kpool
+// k rows and gate rows, with the rows' LayerNorm statistics st[s]. s_ape holds
+// ape * log2(e) laid out [slot][half][lane][4] so a half-warp's loads are
+// contiguous. Returns the packed bf16 chunk (zero when the pool is invalid).
 template <int KP>
-DSA_DEVINL uint2 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *grow,
-                               const float2 *st, const float *s_ape, const float2 (&lw)[2],
-                               const float2 (&lb)[2], int l, bool ok) {
+DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *grow,
+                               const float2 *st, const float *s_ape, const float2 (&lw)[4],
+                               const float2 (&lb)[4], int l, bool ok) {
+    // Pass 1 forms the slot logits and their per-channel max; pass 2 forms the
+    // bf16 k_norm rows and the softmax-weighted sum. kpool <= 4 keeps the logits
+    // in registers between the passes, larger pools recompute them.
     constexpr bool kKeep = KP <= 4;
     const float2 log2e2 = make_float2(kLog2e, kLog2e);
-    float2 lgk[kKeep ? KP : 1][2];
-    float2 mx2[2] = {make_float2(-INFINITY, -INFINITY), make_float2(-INFINITY, -INFINITY)};
+    float2 lgk[kKeep ? KP : 1][4];
+    float2 mx2[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) mx2[c] = make_float2(-INFINITY, -INFINITY);
 
-    auto knorm = [&](int s, float2 (&kn)[2]) {
+    auto knorm = [&](int s, float2 (&kn)[4]) {
         const float2 rs = st[s];
         const float2 r2 = make_float2(rs.x, rs.x), n2 = make_float2(rs.y, rs.y);
-        float2 x[2];
-        unpack4x2(*reinterpret_cast<const uint2 *>(krow + s * kD), x);
+        float2 x[4];
+        unpack8x2(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < 4; ++c)
             kn[c] = round_bf16x2(__ffma2_rn(__ffma2_rn(x[c], r2, n2), lw[c], lb[c]));
     };
-    auto logits = [&](int s, float2 (&lg)[2]) {
-        float2 g[2];
-        unpack4x2(*reinterpret_cast<const uint2 *>(grow + s * kD), g);
-        const float4 a = *reinterpret_cast<const float4 *>(s_ape + s * kD + 4 * l);
-        lg[0] = __ffma2_rn(g[0], log2e2, make_float2(a.x, a.y));
-        lg[1] = __ffma2_rn(g[1], log2e2, make_float2(a.z, a.w));
+    auto logits = [&](int s, float2 (&lg)[4]) {
+        float2 g[4];
+        unpack8x2(*reinterpret_cast<const uint4 *>(grow + s * kD), g);
+        const float4 a0 = *reinterpret_cast<const float4 *>(s_ape + (s * 2) * 64 + 4 * l);
+        const float4 a1 = *reinterpret_cast<const float4 *>(s_ape + (s * 2 + 1) * 64 + 4 * l);
+        lg[0] = __ffma2_rn(g[0], log2e2, make_float2(a0.x, a0.y));
+        lg[1] = __ffma2_rn(g[1], log2e2, make_float2(a0.z, a0.w));
+        lg[2] = __ffma2_rn(g[2], log2e2, make_float2(a1.x, a1.y));
+        lg[3] = __ffma2_rn(g[3], log2e2, make_float2(a1.z, a1.w));
     };
 
 #pragma unroll
     for (int s = 0; s < KP; ++s) {
-        float2 lg[2];
+        float2 lg[4];
         logits(s, lg);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
             mx2[c] = make_float2(fmaxf(mx2[c].x, lg[c].x), fmaxf(mx2[c].y, lg[c].y));
             if constexpr (kKeep) lgk[s][c] = lg[c];
         }
     }
-    float2 nmx[2], den[2], acc[2];
+    float2 nmx[4], den[4], acc[4];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < 4; ++c) {
         nmx[c] = make_float2(-mx2[c].x, -mx2[c].y);
         den[c] = make_float2(0.f, 0.f);
         acc[c] = make_float2(0.f, 0.f);
     }
 #pragma unroll
     for (int s = 0; s < KP; ++s) {
-        float2 kn[2], lg[2];
+        float2 kn[4], lg[4];
         if constexpr (kKeep) {
 #pragma unroll
-            for (int c = 0; c < 2; ++c) lg[c] = lgk[s][c];
+            for (int c = 0; c < 4; ++c) lg[c] = lgk[s][c];
         } else {
             logits(s, lg);
         }
         knorm(s, kn);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
             const float2 z = __fadd2_rn(lg[c], nmx[c]);
             const float2 e = make_float2(ex2(z.x), ex2(z.y));
             den[c] = __fadd2_rn(den[c], e);
             acc[c] = __ffma2_rn(e, kn[c], acc[c]);
         }
     }
-    uint2 o = make_uint2(0u, 0u);
+    uint4 o = make_uint4(0, 0, 0, 0);
     if (ok) {
-        uint32_t w[2];
+        uint32_t w[4];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
             const float2 inv = make_float2(rcp_approx(den[c].x), rcp_approx(den[c].y));
             const float2 v = __fmul2_rn(acc[c], inv);
             w[c] = pack_bf16x2(v.x, v.y);
         }
-        o = make_uint2(w[0], w[1]);
+        o = make_uint4(w[0], w[1], w[2], w[3]);
     }
     return o;
 }
@@ -250,7 +255,7 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     constexpr int kCmpConsumers = C::kConsumers;
     constexpr int kCmpThreads = C::kThreads;
     extern __shared__ __align__(128) uint8_t cmp_smem[];
-    __shared__ __align__(16) float s_ape[KP * kD];   // ape * log2(e)
+    __shared__ __align__(16) float s_ape[KP * kD];   // ape * log2(e), [slot][half][lane][4]
     __shared__ __align__(16) float2 s_stat[kCmpStages][kCmpTileTokens];   // (rstd, -mu*rstd)
     __shared__ __align__(8) uint64_t full[kCmpStages], empty[kCmpStages];
     __shared__ CmpMeta meta[kCmpStages];
@@ -268,7 +273,10 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         }
         fence_mbarrier_init();
     }
-    for (int i = tid; i < KP * kD; i += kCmpThreads) s_ape[i] = ape[i] * kLog2e;
+    for (int i = tid; i < KP * kD; i += kCmpThreads) {
+        const int sl = i / kD, c = i % kD;
+        s_ape[(sl * 2 + ((c >> 2) & 1)) * 64 + 4 * (c >> 3) + (c & 3)] = ape[i] * kLog2e;
+    }
     __syncthreads();
     pdl_wait();
     pdl_launch_dependents();
@@ -325,10 +333,11 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     }
 
     // -------------------------------------------------------------------- consumer warps
-    // lane owns channels 4*lane .. 4*lane+3 of every pool of its warp
-    float2 lw[2], lb[2];
-    unpack4x2(__ldg(reinterpret_cast<const uint2 *>(ln_w) + lane), lw);
-    unpack4x2(__ldg(reinterpret_cast<const uint2 *>(ln_b) + lane), lb);
+    const int hw = tid >> 4;     // half-warp: one pool at a time
+    const int l = tid & 15;      // channels 8l .. 8l+7
+    float2 lw[4], lb[4];
+    unpack8x2(ldg_nc_v4(ln_w + 8 * l), lw);
+    unpack8x2(ldg_nc_v4(ln_b + 8 * l), lb);
 
     for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
         const int s = i % kCmpStages;
@@ -349,19 +358,23 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         token_stats(sk, m.n_in * KP, eps, &s_stat[s][0], tid, kCmpConsumers);
         asm volatile("bar.sync 1, %0;" ::"n"(kCmpConsumers) : "memory");
 
-        // One pool per warp (warp-uniform loop).
-        for (int pi = warp; pi < m.n_in; pi += kCmpConsumers / 32) {
+        // Warp-uniform loop: the two half-warps of a warp take pools ii and ii+1;
+        // a half-warp past the tile computes on a loaded row and stores nothing.
+        for (int ii = 2 * warp; ii < m.n_in; ii += kCmpConsumers / 16) {
+            const bool active = ii + (hw & 1) < m.n_in;
+            const int pi = active ? ii + (hw & 1) : ii;
             const int p = m.p0 + pi;
             // pool valid iff every slot token is valid (read from the stage's window)
             bool ok = true;
 #pragma unroll
             for (int ss = 0; ss < KP; ++ss) ok = ok && s_valid[s][m.voff + pi * KP + ss] != 0;
-            const uint2 o = compress_pool<KP>(sk + (size_t)pi * KP * kD + 4 * lane,
-                                              sg + (size_t)pi * KP * kD + 4 * lane,
-                                              &s_stat[s][pi * KP], s_ape, lw, lb, lane, ok);
-            *reinterpret_cast<uint2 *>(pool_keys + (pool_base + p) * kD + 4 * lane) = o;
-            if (lane < KP) pool_idx[(pool_base + p) * KP + lane] = ok ? m.f + p * KP + lane : -1;
-            if (lane == 0) pool_valid[pool_base + p] = ok ? 1 : 0;
+            const uint4 o = compress_pool<KP>(sk + (size_t)pi * KP * kD + 8 * l,
+                                              sg + (size_t)pi * KP * kD + 8 * l,
+                                              &s_stat[s][pi * KP], s_ape, lw, lb, l, ok);
+            if (!active) continue;
+            *reinterpret_cast<uint4 *>(pool_keys + (pool_base + p) * kD + 8 * l) = o;
+            if (l < KP) pool_idx[(pool_base + p) * KP + l] = ok ? m.f + p * KP + l : -1;
+            if (l == 0) pool_valid[pool_base + p] = ok ? 1 : 0;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);

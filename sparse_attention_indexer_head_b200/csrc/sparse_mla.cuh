@@ -54,23 +54,23 @@ constexpr int kPartStride = kL + 4;
 // max grows by more than 2^8 (lazy rescaling), and write the epilogue.
 // ---------------------------------------------------------------------------------------
 constexpr int kTcThreads = 256;
-constexpr int kTcChunk = 32;                        // tokens per chunk
-constexpr int kTcStages = 4;                        // gathered-row ring depth
+constexpr int kTcChunk = 64;                        // tokens per chunk (one S tile, one PV pass)
+constexpr int kTcSub = 32;                          // tokens per gathered stage
+constexpr int kTcStages = 4;                        // 32-token stages; chunk c uses 2(c&1), 2(c&1)+1
 constexpr int kTcHeads = 64;
 constexpr uint32_t kOffQ = 0;                       // 64 KB: 8 atoms x [64 rows x 128 B]
-constexpr uint32_t kOffKV = 64 * 1024;              // 4 stages x 32 KB: 8 atoms x [32 rows x 128 B]
-constexpr uint32_t kStageKV = 32 * 1024;
-constexpr uint32_t kAtomKV = kTcChunk * 128;        // 4 KB: one 64-latent column of a stage
-constexpr uint32_t kOffP = 192 * 1024;              // 2 buffers x 4 KB: [64 heads x 64 B], 64B swizzle
-constexpr uint32_t kStageP = 4 * 1024;
-constexpr uint32_t kOffCtl = 200 * 1024;
+constexpr uint32_t kOffKV = 64 * 1024;              // 128 KB: 8 atoms x [128 rows x 128 B]
+constexpr uint32_t kAtomKV = 128 * 128;             // 16 KB: one 64-latent column of all stages
+constexpr uint32_t kOffP = 192 * 1024;              // 2 buffers x 8 KB: [64 heads x 128 B], 128B swizzle
+constexpr uint32_t kStageP = 8 * 1024;
+constexpr uint32_t kOffCtl = 208 * 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLazyRescale = 8.0f;                // log2 units
 constexpr int kMaxClusterSplits = 8;                // portable cluster size
 constexpr int kSmTarget = 148;                      // CTAs of one full wave (one CTA per SM)
 // The cluster merge reads each CTA's O^T, copied as fp32 [64 heads][512] into
 // the (then idle) gathered-row ring.
-static_assert(kTcStages * kStageKV == kTcHeads * kL * 4, "merge buffer must fit the ring");
+static_assert(8 * kAtomKV == kTcHeads * kL * 4, "merge buffer must fit the ring");
 
 struct TcCtl {
     uint64_t kv_full[kTcStages], kv_empty[kTcStages];
@@ -188,7 +188,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     uint8_t *gbase = mla_smem_raw + (base - raw);
     TcCtl *ctl = reinterpret_cast<TcCtl *>(gbase + kOffCtl);
     const uint32_t sQ = base + kOffQ;
-    const uint32_t sKV = base + kOffKV;                      // stage s at sKV + s * kStageKV
+    const uint32_t sKV = base + kOffKV;                      // stage s: rows [32s, 32s+32) of each atom
     const uint32_t sP = base + kOffP;                        // buffer b at sP + b * kStageP
 
     const int split = blockIdx.x, qi = blockIdx.y, hg = blockIdx.z;
@@ -250,41 +250,44 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         if (lane == 0 && nch > 0) {
             constexpr uint32_t idS = tc::idesc_bf16(64, kTcChunk, false, false);
             constexpr uint32_t idPV = tc::idesc_bf16(128, 64, true, false);
+            // Chunk c lives in stages 2h, 2h+1 (h = c & 1): rows [64h, 64h+64) of
+            // every 128-row column atom.
             auto issue_pv = [&](int cp) -> bool {
-                const int sp = cp % kTcStages, pb = cp & 1;
+                const int hp = cp & 1, pb = cp & 1;
                 if (!tc_wait(ctl, &ctl->p_full[pb], (cp >> 1) & 1)) return false;
                 tc::fence_after_sync();
-                const uint32_t kvs = sKV + sp * kStageKV;
 #pragma unroll
                 for (int lb = 0; lb < 4; ++lb)
 #pragma unroll
                     for (int ks = 0; ks < kTcChunk / 16; ++ks) {
                         // V^T: MN-major, 64-latent atoms kAtomKV apart, 8-token groups 1 KB apart
-                        const uint64_t a = tc::desc_sw128(kvs + lb * 2 * kAtomKV + ks * 2048, kAtomKV, 1024);
-                        // P^T: K-major, 64-byte rows, 8-head groups 512 B apart
-                        const uint64_t bd = tc::desc_sw64(sP + pb * kStageP + ks * 32, 16, 512);
+                        const uint64_t a = tc::desc_sw128(sKV + lb * 2 * kAtomKV + hp * 8192 + ks * 2048,
+                                                          kAtomKV, 1024);
+                        // P^T: K-major, 128-byte rows (64 tokens), 8-head groups 1 KB apart
+                        const uint64_t bd = tc::desc_sw128(sP + pb * kStageP + ks * 32, 16, 1024);
                         tc::mma_bf16_ss(tmem + lb * 64, a, bd, idPV, (cp > 0 || ks > 0) ? 1u : 0u);
                     }
-                tc::mma_commit(&ctl->kv_empty[sp]);
+                tc::mma_commit(&ctl->kv_empty[2 * hp]);
+                tc::mma_commit(&ctl->kv_empty[2 * hp + 1]);
                 tc::mma_commit(&ctl->p_empty[pb]);
                 tc::mma_commit(&ctl->o_done);
                 return true;
             };
             bool ok = tc_wait(ctl, &ctl->q_full, 0);
             for (int c = 0; ok && c < nch; ++c) {
-                const int s = c % kTcStages, sb = c & 1;
-                if (!tc_wait(ctl, &ctl->kv_full[s], (c / kTcStages) & 1)) { ok = false; break; }
+                const int h = c & 1, sb = c & 1;
+                if (!tc_wait(ctl, &ctl->kv_full[2 * h], (c >> 1) & 1) ||
+                    !tc_wait(ctl, &ctl->kv_full[2 * h + 1], (c >> 1) & 1)) { ok = false; break; }
                 if (c >= 2 && !tc_wait(ctl, &ctl->s_empty[sb], ((c >> 1) - 1) & 1)) { ok = false; break; }
                 tc::fence_after_sync();
-                tc::fence_proxy_async_smem();     // the stage was written by cp.async
+                tc::fence_proxy_async_smem();     // the stages were written by cp.async
                 const uint32_t d = tmem + 256 + sb * kTcChunk;
-                const uint32_t kvs = sKV + s * kStageKV;
 #pragma unroll
                 for (int kk = 0; kk < kL / 16; ++kk) {
                     const uint32_t qo = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    const uint32_t ko = (kk >> 2) * kAtomKV + (kk & 3) * 32;
+                    const uint32_t ko = (kk >> 2) * kAtomKV + h * 8192 + (kk & 3) * 32;
                     tc::mma_bf16_ss(d, tc::desc_sw128(sQ + qo, 16, 1024),
-                                    tc::desc_sw128(kvs + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
+                                    tc::desc_sw128(sKV + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(&ctl->s_full[sb]);
                 if (c >= 1 && !issue_pv(c - 1)) { ok = false; break; }
@@ -302,9 +305,10 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         // on the stage's barrier as they land, so no warp waits for its own copies
         // and all four stages can be in flight.
         const int pw = warp - 1;
+        const int nsub = 2 * nch;                          // 32-token stages to fill
         auto load_id = [&](int c) -> int {
-            const int j = c * kTcChunk + lane;
-            return (c < nch && j < ntok) ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
+            const int j = c * kTcSub + lane;
+            return (c < nsub && j < ntok) ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
         };
         auto gather_chunk = [&](int c, int id) -> bool {
             const int s = c % kTcStages;
@@ -314,9 +318,9 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             const bool valid = id >= 0 && id < T && (long long)rs + id < (long long)kv_rows;
             const uint32_t vm = __ballot_sync(0xffffffffu, valid);
             const int myrow = valid ? rs + id : -1;
-            const uint32_t dst0 = sKV + s * kStageKV;
+            const uint32_t dst0 = sKV + s * (kTcSub * 128);   // rows [32s, 32s+32) of each atom
 #pragma unroll 4
-            for (int r = 0; r < kTcChunk; ++r) {
+            for (int r = 0; r < kTcSub; ++r) {
                 const int row = __shfl_sync(0xffffffffu, myrow, r);
                 const __nv_bfloat16 *src = row >= 0 ? kv + (size_t)row * kL : qm;   // qm: never read
                 const uint32_t nb = row >= 0 ? 16u : 0u;
@@ -337,11 +341,11 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         // ids of this warp's next two chunks are in flight (static queue slots)
         int idq[2] = {load_id(pw), load_id(pw + 3)};
         bool go = true;
-        for (int c0 = pw; go && c0 < nch; c0 += 6) {
+        for (int c0 = pw; go && c0 < nsub; c0 += 6) {
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int c = c0 + 3 * u;
-                if (!go || c >= nch) break;
+                if (!go || c >= nsub) break;
                 const int id = idq[u];
                 idq[u] = load_id(c + 6);
                 go = gather_chunk(c, id);
@@ -366,22 +370,26 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         float m_used = -INFINITY, l = 0.f;
         bool failed = false;
         for (int c = 0; c < nch; ++c) {
-            const int s = c % kTcStages, sb = c & 1;
-            bool bad = !tc_wait(ctl, &ctl->kv_full[s], (c / kTcStages) & 1);
+            const int h = c & 1, sb = c & 1;
+            bool bad = !tc_wait(ctl, &ctl->kv_full[2 * h], (c >> 1) & 1);
+            bad = bad || !tc_wait(ctl, &ctl->kv_full[2 * h + 1], (c >> 1) & 1);
             bad = bad || !tc_wait(ctl, &ctl->s_full[sb], (c >> 1) & 1);
             tc::fence_after_sync();
             uint32_t r[kTcChunk / 2];
-            tc::tmem_ld16x64b_x16(tl + 256 + sb * kTcChunk, r);
+            tc::tmem_ld16x64b_x16(tl + 256 + sb * kTcChunk, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+            tc::tmem_ld16x64b_x16(tl + 256 + sb * kTcChunk + 32, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             mbar_arrive(&ctl->s_empty[sb]);
 
-            const uint32_t vm = ctl->vmask[s] >> par;        // bit 2i: token par + 2i
+            // token par + 2i: i < 16 in the first stage of the pair, i >= 16 in the second
+            const uint32_t vm0 = ctl->vmask[2 * h] >> par, vm1 = ctl->vmask[2 * h + 1] >> par;
             float z[kTcChunk / 2];
             float mx = -INFINITY;
 #pragma unroll
             for (int i = 0; i < kTcChunk / 2; ++i) {
-                z[i] = ((vm >> (2 * i)) & 1) ? __uint_as_float(r[i]) * scale_log2 : -INFINITY;
+                const uint32_t bit = i < 16 ? (vm0 >> (2 * i)) & 1 : (vm1 >> (2 * i - 32)) & 1;
+                z[i] = bit ? __uint_as_float(r[i]) * scale_log2 : -INFINITY;
                 mx = fmaxf(mx, z[i]);
             }
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -400,13 +408,13 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             psum += __shfl_xor_sync(0xffffffffu, psum, 2);
             l = fmaf(l, alpha, psum);
             if (owner) ctl->alpha[hh] = alpha;
-            // bf16 P row of the head: this thread packs tokens 16par .. 16par+15,
+            // bf16 P row of the head: this thread packs tokens 32par .. 32par+31,
             // taking the other parity from its partner.
-            uint32_t pk[8];
+            uint32_t pk[16];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const float recv = __shfl_xor_sync(0xffffffffu, par ? pv[k] : pv[k + 8], 2);
-                pk[k] = par ? pack_bf16x2(recv, pv[k + 8]) : pack_bf16x2(pv[k], recv);
+            for (int k = 0; k < 16; ++k) {
+                const float recv = __shfl_xor_sync(0xffffffffu, par ? pv[k] : pv[k + 16], 2);
+                pk[k] = par ? pack_bf16x2(recv, pv[k + 16]) : pack_bf16x2(pv[k], recv);
             }
 
             bad = bad || (c >= 2 && !tc_wait(ctl, &ctl->p_empty[sb], ((c >> 1) - 1) & 1));
@@ -417,12 +425,12 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                 need = true;
             }
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const int c4 = 2 * par + h2;      // 16-byte piece of the 64-byte row
-                const uint32_t dst = sP + sb * kStageP + hh * 64 + ((c4 ^ ((hh >> 1) & 3)) << 4);
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const int c16 = 4 * par + q4;     // 16-byte piece of the 128-byte row
+                const uint32_t dst = sP + sb * kStageP + hh * 128 + ((c16 ^ (hh & 7)) << 4);
                 asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
-                             "r"(pk[4 * h2]), "r"(pk[4 * h2 + 1]), "r"(pk[4 * h2 + 2]),
-                             "r"(pk[4 * h2 + 3])
+                             "r"(pk[4 * q4]), "r"(pk[4 * q4 + 1]), "r"(pk[4 * q4 + 2]),
+                             "r"(pk[4 * q4 + 3])
                              : "memory");
             }
             if (need) {

@@ -109,10 +109,10 @@ def test_topk_expand_refusals(B):
 
 def test_sparse_mla_refusals(B):
     L = B.lib
-    # partials of every split (the plan keeps the grid within 148 CTAs):
-    # 2 queries -> 64 splits of one chunk; 16 queries -> 8 splits of 8 chunks
+    # partials of every split (the plan keeps the grid within 148 CTAs; 64-token
+    # chunks): 2 queries -> 32 splits of one chunk; 16 queries -> 8 splits of 4
     ws = B.dsa_sparse_mla_workspace_size(2, 64, 2048)
-    assert ws == 2 * 64 * 64 * 516 * 4
+    assert ws == 2 * 32 * 64 * 516 * 4
     assert B.dsa_sparse_mla_workspace_size(16, 64, 2048) == 16 * 8 * 64 * 516 * 4
     # at least 148 CTAs without splitting: one split, no workspace
     assert B.dsa_sparse_mla_workspace_size(148, 64, 2048) == 0
