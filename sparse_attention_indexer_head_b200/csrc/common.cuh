@@ -87,6 +87,19 @@ DSA_DEVINL bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
 // a while, so the bound is on elapsed cycles, not on the number of polls),
 // raises the device error flag and returns false.
 constexpr long long kWaitLimitCycles = 4000000000ll;
+// Non-blocking probe: has the phase with this parity completed?
+DSA_DEVINL bool mbar_test(uint64_t *bar, uint32_t phase) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(phase)
+        : "memory");
+    return ok != 0;
+}
+
 DSA_DEVINL bool mbar_wait(uint64_t *bar, uint32_t phase) {
     if (mbar_try_wait(bar, phase)) return true;
     const long long t0 = clock64();

@@ -252,14 +252,15 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             constexpr uint32_t idPV = tc::idesc_bf16(128, 64, true, false);
             // Chunk c lives in stages 2h, 2h+1 (h = c & 1): rows [64h, 64h+64) of
             // every 128-row column atom.
-            auto issue_pv = [&](int cp) -> bool {
+            // PV(cp): O^T += V^T P^T over the chunk's 64 tokens; the K-steps of its
+            // first stage go first so that stage is released as early as possible.
+            auto issue_pv = [&](int cp) {
                 const int hp = cp & 1, pb = cp & 1;
-                if (!tc_wait(ctl, &ctl->p_full[pb], (cp >> 1) & 1)) return false;
                 tc::fence_after_sync();
 #pragma unroll
-                for (int lb = 0; lb < 4; ++lb)
+                for (int ks = 0; ks < kTcChunk / 16; ++ks) {
 #pragma unroll
-                    for (int ks = 0; ks < kTcChunk / 16; ++ks) {
+                    for (int lb = 0; lb < 4; ++lb) {
                         // V^T: MN-major, 64-latent atoms kAtomKV apart, 8-token groups 1 KB apart
                         const uint64_t a = tc::desc_sw128(sKV + lb * 2 * kAtomKV + hp * 8192 + ks * 2048,
                                                           kAtomKV, 1024);
@@ -267,18 +268,15 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                         const uint64_t bd = tc::desc_sw128(sP + pb * kStageP + ks * 32, 16, 1024);
                         tc::mma_bf16_ss(tmem + lb * 64, a, bd, idPV, (cp > 0 || ks > 0) ? 1u : 0u);
                     }
-                tc::mma_commit(&ctl->kv_empty[2 * hp]);
+                    if (ks == 1) tc::mma_commit(&ctl->kv_empty[2 * hp]);
+                }
                 tc::mma_commit(&ctl->kv_empty[2 * hp + 1]);
                 tc::mma_commit(&ctl->p_empty[pb]);
                 tc::mma_commit(&ctl->o_done);
-                return true;
             };
-            bool ok = tc_wait(ctl, &ctl->q_full, 0);
-            for (int c = 0; ok && c < nch; ++c) {
+            // S(c) = Q K^T over chunk c's 64 tokens into S buffer c & 1.
+            auto issue_s = [&](int c) {
                 const int h = c & 1, sb = c & 1;
-                if (!tc_wait(ctl, &ctl->kv_full[2 * h], (c >> 1) & 1) ||
-                    !tc_wait(ctl, &ctl->kv_full[2 * h + 1], (c >> 1) & 1)) { ok = false; break; }
-                if (c >= 2 && !tc_wait(ctl, &ctl->s_empty[sb], ((c >> 1) - 1) & 1)) { ok = false; break; }
                 tc::fence_after_sync();
                 tc::fence_proxy_async_smem();     // the stages were written by cp.async
                 const uint32_t d = tmem + 256 + sb * kTcChunk;
@@ -290,11 +288,39 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                                     tc::desc_sw128(sKV + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(&ctl->s_full[sb]);
-                if (c >= 1 && !issue_pv(c - 1)) { ok = false; break; }
+            };
+            // Event loop: issue whichever product is ready, PV first (it frees a
+            // stage pair for the gathers); give up after the wait bound without progress.
+            bool ok = tc_wait(ctl, &ctl->q_full, 0);
+            int ns = 0, np = 0;
+            long long t_last = clock64();
+            while (ok && np < nch) {
+                if (np < ns && mbar_test(&ctl->p_full[np & 1], (np >> 1) & 1)) {
+                    issue_pv(np++);
+                    t_last = clock64();
+                    continue;
+                }
+                if (ns < nch) {
+                    const int h = ns & 1;
+                    const bool ready = mbar_test(&ctl->kv_full[2 * h], (ns >> 1) & 1) &&
+                                       mbar_test(&ctl->kv_full[2 * h + 1], (ns >> 1) & 1) &&
+                                       (ns < 2 || mbar_test(&ctl->s_empty[h], ((ns >> 1) - 1) & 1));
+                    if (ready) {
+                        issue_s(ns++);
+                        t_last = clock64();
+                        continue;
+                    }
+                }
+                if (ctl->abort) { ok = false; break; }
+                if (clock64() - t_last > kWaitLimitCycles) {
+                    raise_device_error(kErrWaitTimeout);
+                    ctl->abort = 1;
+                    ok = false;
+                }
             }
             // o_final is single-use: once it completes every PV of this CTA has landed
             // (a parity wait on o_done cannot tell the last two PVs apart).
-            if (ok && issue_pv(nch - 1)) tc::mma_commit(&ctl->o_final);
+            if (ok) tc::mma_commit(&ctl->o_final);
         }
         __syncwarp();
     } else if (warp < 4) {
