@@ -364,6 +364,26 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             tc::cp_async_arrive_noinc(&ctl->kv_full[s]);
             return true;
         };
+        // The rows of this warp's first eight stages (24 of the split's) are
+        // prefetched into L2 up front, so DRAM streams them at once and the ring
+        // refills come from L2. Their ids are loaded together first.
+        {
+            int pid[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) pid[u] = load_id(pw + 3 * u);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const bool valid = pid[u] >= 0 && pid[u] < T && (long long)rs + pid[u] < (long long)kv_rows;
+                const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+                const int row = valid ? rs + pid[u] : 0;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {            // 8 lines of 128 B per 1 KB row
+                    const int r = (lane >> 3) + 4 * k;   // row r, line lane & 7
+                    const int rr = __shfl_sync(0xffffffffu, row, r);
+                    if ((vmask >> r) & 1) tc::prefetch_l2(kv + (size_t)rr * kL + (lane & 7) * 64);
+                }
+            }
+        }
         // ids of this warp's next two chunks are in flight (static queue slots)
         int idq[2] = {load_id(pw), load_id(pw + 3)};
         bool go = true;

@@ -141,6 +141,11 @@ DSA_DEVINL void cp_async_arrive_noinc(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
 }
+// Hint: bring the 128-byte line at p into L2 (no data returned, never faults on
+// the valid addresses it is given).
+DSA_DEVINL void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 DSA_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 DSA_DEVINL void st_shared_zero16(uint32_t dst) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
