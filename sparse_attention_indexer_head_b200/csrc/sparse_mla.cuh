@@ -42,18 +42,21 @@ constexpr int kPartStride = kL + 4;
 // (all 128 lanes), S double-buffered in columns [256,320) (lanes 0-15 of each
 // 32-lane quadrant, the M=64 layout).
 //
-// Warp roles (256 threads): warp 0 allocates tensor memory and one lane issues
-// every MMA; warps 1-3 gather, warp 1+(c mod 3) filling chunk c of a 4-stage
-// ring with 16-byte cp.async pieces straight into the 128B-swizzled layout (a
-// zero fill for ids that are -1 or outside the request). The copies' landing is
-// tracked by the stage's mbarrier (cp.async.mbarrier.arrive), so no gather warp
-// waits for its own copies and all four stages can be in flight. (Per-row TMA
-// copies -- tile::gather4 or a 1-D bulk copy per 1 KB row -- move only 12-20 GB/s
-// per SM here: their per-instruction cost, not the depth of the ring, bounds
-// them.) Warps 4-7 load Q, run the softmax, rescale O^T when a head's running
-// max grows by more than 2^8 (lazy rescaling), and write the epilogue.
+// Warp roles (512 threads): warp 0 allocates tensor memory and one lane issues
+// every MMA (an event loop over the barriers: a PV as soon as its P is ready, an
+// S as soon as its two stages have landed); warps 8-15 gather, two groups of
+// four warps filling alternate 32-token stages of a 4-stage ring with 16-byte
+// cp.async pieces straight into the 128B-swizzled layout (a zero fill for ids
+// that are -1 or outside the request). The copies' landing is tracked by the
+// stage's mbarrier (cp.async.mbarrier.arrive), so no gather warp waits for its
+// own copies. (Per-row TMA copies -- tile::gather4 or a 1-D bulk copy per 1 KB
+// row -- move only 12-20 GB/s per SM here, bounded by their per-instruction
+// cost; cp.async reaches about 37 GB/s per SM once a stage is spread over four
+// warps.) Warps 4-7 load Q, run the softmax, rescale O^T when a head's running
+// max grows by more than 2^8 (lazy rescaling), and write the epilogue. Warps
+// 1-3 take part only in the cluster merge.
 // ---------------------------------------------------------------------------------------
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 512;
 constexpr int kTcChunk = 64;                        // tokens per chunk (one S tile, one PV pass)
 constexpr int kTcSub = 32;                          // tokens per gathered stage
 constexpr int kTcStages = 4;                        // 32-token stages; chunk c uses 2(c&1), 2(c&1)+1
@@ -198,7 +201,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     const int nch = (ntok + kTcChunk - 1) / kTcChunk;
     const int h0 = hg * kTcHeads, nh = min(kTcHeads, Hm - h0);
 
-    if (warp >= 4) {
+    if (warp >= 4 && warp < 8) {
         // Q tile (a step input): 64 rows x 64 16-byte chunks into the swizzled
         // K-major layout, issued before the predecessor grid finishes.
         for (int x = tid - 128; x < kTcHeads * 64; x += 128) {
@@ -217,7 +220,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     }
     if (tid == 32) {
         for (int i = 0; i < kTcStages; ++i) {
-            mbar_init(&ctl->kv_full[i], 33);    // 32 lanes' copies + lane 0's arrive
+            mbar_init(&ctl->kv_full[i], 4 * 32 + 1);   // four warps' lanes' copies + the mask's arrive
             mbar_init(&ctl->kv_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -323,20 +326,20 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             if (ok) tc::mma_commit(&ctl->o_final);
         }
         __syncwarp();
-    } else if (warp < 4) {
+    } else if (warp >= 8) {
         // ------------------------------------------------------------------ gather warps
-        // Warp 1+p fills chunks p, p+3, p+6, ...: lane r holds row r's id and the
-        // warp copies the chunk's 32 rows as 16-byte cp.async pieces into the
-        // swizzled stage (zero-filled for invalid ids). Each lane's copies arrive
-        // on the stage's barrier as they land, so no warp waits for its own copies
-        // and all four stages can be in flight.
-        const int pw = warp - 1;
+        // Two groups of four warps (warps 8-11, 12-15) fill alternate 32-token
+        // stages (group p: stages g = p, p+2, ...); warp i of a group copies rows
+        // 8i..8i+7 of the stage as 16-byte cp.async pieces straight into the
+        // swizzled layout (zero-filled for invalid ids). Each lane's copies arrive
+        // on the stage's barrier as they land, so no warp waits for its own copies.
+        const int grp = (warp - 8) >> 2, sub = (warp - 8) & 3;
         const int nsub = 2 * nch;                          // 32-token stages to fill
         auto load_id = [&](int c) -> int {
             const int j = c * kTcSub + lane;
             return (c < nsub && j < ntok) ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
         };
-        auto gather_chunk = [&](int c, int id) -> bool {
+        auto gather_stage = [&](int c, int id) -> bool {
             const int s = c % kTcStages;
             bool ok = true;
             if (c >= kTcStages) ok = tc_wait(ctl, &ctl->kv_empty[s], ((c / kTcStages) - 1) & 1);
@@ -345,8 +348,9 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             const uint32_t vm = __ballot_sync(0xffffffffu, valid);
             const int myrow = valid ? rs + id : -1;
             const uint32_t dst0 = sKV + s * (kTcSub * 128);   // rows [32s, 32s+32) of each atom
-#pragma unroll 4
-            for (int r = 0; r < kTcSub; ++r) {
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+                const int r = 8 * sub + rr;
                 const int row = __shfl_sync(0xffffffffu, myrow, r);
                 const __nv_bfloat16 *src = row >= 0 ? kv + (size_t)row * kL : qm;   // qm: never read
                 const uint32_t nb = row >= 0 ? 16u : 0u;
@@ -357,49 +361,29 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                     tc::cp_async16_zfill(dst, row >= 0 ? src + cc * 8 : src, nb);
                 }
             }
-            if (lane == 0) {
+            if (sub == 0 && lane == 0) {
                 ctl->vmask[s] = vm;
                 mbar_arrive(&ctl->kv_full[s]);             // releases vmask
             }
             tc::cp_async_arrive_noinc(&ctl->kv_full[s]);
             return true;
         };
-        // The rows of this warp's first eight stages (24 of the split's) are
-        // prefetched into L2 up front, so DRAM streams them at once and the ring
-        // refills come from L2. Their ids are loaded together first.
-        {
-            int pid[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) pid[u] = load_id(pw + 3 * u);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const bool valid = pid[u] >= 0 && pid[u] < T && (long long)rs + pid[u] < (long long)kv_rows;
-                const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-                const int row = valid ? rs + pid[u] : 0;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {            // 8 lines of 128 B per 1 KB row
-                    const int r = (lane >> 3) + 4 * k;   // row r, line lane & 7
-                    const int rr = __shfl_sync(0xffffffffu, row, r);
-                    if ((vmask >> r) & 1) tc::prefetch_l2(kv + (size_t)rr * kL + (lane & 7) * 64);
-                }
-            }
-        }
-        // ids of this warp's next two chunks are in flight (static queue slots)
-        int idq[2] = {load_id(pw), load_id(pw + 3)};
+        // ids of the group's next two stages are in flight (static queue slots)
+        int idq[2] = {load_id(grp), load_id(grp + 2)};
         bool go = true;
-        for (int c0 = pw; go && c0 < nsub; c0 += 6) {
+        for (int c0 = grp; go && c0 < nsub; c0 += 4) {
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-                const int c = c0 + 3 * u;
+                const int c = c0 + 2 * u;
                 if (!go || c >= nsub) break;
                 const int id = idq[u];
-                idq[u] = load_id(c + 6);
-                go = gather_chunk(c, id);
+                idq[u] = load_id(c + 4);
+                go = gather_stage(c, id);
             }
         }
         tc::cp_async_wait_all();          // nothing of this warp in flight past here
     } else if (warp >= 4) {
-        // ------------------------------------------------------------------ softmax (128 threads)
+        // ------------------------------------------------------------------ softmax (warps 4-7)
         // S is read with the 16x64b tensor-memory shape, so every lane works:
         // thread t of warp 4+w holds head row hh = 16w + (t>>2) + 8(t&1) and the
         // chunk's tokens of parity par = (t>>1)&1; its partner t^2 holds the
@@ -587,8 +571,9 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     tc::fence_after_sync();
     if constexpr (kCluster) {
         cluster_sync_all();           // every split's m, l and O^T are in place
-        mla_cluster_merge(ctl, sKV, S, nh, split, tid, out + ((size_t)qi * Hm + h0) * kL,
-                          lse ? lse + (size_t)qi * Hm + h0 : nullptr);
+        if (tid < 256)
+            mla_cluster_merge(ctl, sKV, S, nh, split, tid, out + ((size_t)qi * Hm + h0) * kL,
+                              lse ? lse + (size_t)qi * Hm + h0 : nullptr);
         cluster_sync_all();           // no CTA leaves while a peer still reads it
     }
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
