@@ -57,29 +57,30 @@ constexpr int kPartStride = kL + 4;
 // 1-3 take part only in the cluster merge.
 // ---------------------------------------------------------------------------------------
 constexpr int kTcThreads = 512;
-constexpr int kTcChunk = 64;                        // tokens per chunk (one S tile, one PV pass)
-constexpr int kTcSub = 32;                          // tokens per gathered stage
-constexpr int kTcStages = 4;                        // 32-token stages; chunk c uses 2(c&1), 2(c&1)+1
+constexpr int kTcChunk = 48;                        // tokens per chunk (one S tile, one PV pass)
+constexpr int kTcSlots = 3;                         // ring slots, one chunk each
 constexpr int kTcHeads = 64;
 constexpr uint32_t kOffQ = 0;                       // 64 KB: 8 atoms x [64 rows x 128 B]
-constexpr uint32_t kOffKV = 64 * 1024;              // 128 KB: 8 atoms x [128 rows x 128 B]
-constexpr uint32_t kAtomKV = 128 * 128;             // 16 KB: one 64-latent column of all stages
-constexpr uint32_t kOffP = 192 * 1024;              // 2 buffers x 8 KB: [64 heads x 128 B], 128B swizzle
+constexpr uint32_t kOffKV = 64 * 1024;              // 144 KB: 8 atoms x [144 rows x 128 B]
+constexpr uint32_t kAtomKV = kTcSlots * kTcChunk * 128;   // 18 KB: one 64-latent column of the ring
+constexpr uint32_t kSlotRows = kTcChunk * 128;      // 6 KB: a slot's rows within an atom
+constexpr uint32_t kOffP = kOffKV + 8 * kAtomKV;    // 2 buffers x 8 KB: [64 heads x 128 B], 128B swizzle
 constexpr uint32_t kStageP = 8 * 1024;
-constexpr uint32_t kOffCtl = 208 * 1024;
+constexpr uint32_t kOffCtl = kOffP + 2 * kStageP;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLazyRescale = 8.0f;                // log2 units
 constexpr int kMaxClusterSplits = 8;                // portable cluster size
 constexpr int kSmTarget = 148;                      // CTAs of one full wave (one CTA per SM)
 // The cluster merge reads each CTA's O^T, copied as fp32 [64 heads][512] into
 // the (then idle) gathered-row ring.
-static_assert(8 * kAtomKV == kTcHeads * kL * 4, "merge buffer must fit the ring");
+static_assert(8 * kAtomKV >= kTcHeads * kL * 4, "merge buffer must fit the ring");
+static_assert(kOffP % 1024 == 0, "P buffers hold 128B-swizzle atoms");
 
 struct TcCtl {
-    uint64_t kv_full[kTcStages], kv_empty[kTcStages];
+    uint64_t kv_full[kTcSlots], kv_empty[kTcSlots];
     uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
     uint64_t o_done, o_final, q_full, fin;
-    uint32_t vmask[kTcStages];
+    uint16_t vmask[kTcSlots][4];          // validity of a slot's rows, 12 rows per gather warp
     float alpha[kTcHeads];
     float lsum[kTcHeads];
     float mfin[kTcHeads];
@@ -87,6 +88,7 @@ struct TcCtl {
     volatile int abort;
 };
 constexpr int kTcSmemBytes = (int)kOffCtl + (int)sizeof(TcCtl) + 1024;   // + alignment slack
+static_assert(kTcSmemBytes <= 232448, "shared memory per block");
 
 struct MlaGeom {
     int S;         // splits per (query, head group)
@@ -219,8 +221,8 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         tc::tmem_relinquish();
     }
     if (tid == 32) {
-        for (int i = 0; i < kTcStages; ++i) {
-            mbar_init(&ctl->kv_full[i], 4 * 32 + 1);   // four warps' lanes' copies + the mask's arrive
+        for (int i = 0; i < kTcSlots; ++i) {
+            mbar_init(&ctl->kv_full[i], 4 * 32 + 4);   // four warps' lanes' copies + their masks' arrives
             mbar_init(&ctl->kv_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -253,40 +255,38 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         if (lane == 0 && nch > 0) {
             constexpr uint32_t idS = tc::idesc_bf16(64, kTcChunk, false, false);
             constexpr uint32_t idPV = tc::idesc_bf16(128, 64, true, false);
-            // Chunk c lives in stages 2h, 2h+1 (h = c & 1): rows [64h, 64h+64) of
-            // every 128-row column atom.
-            // PV(cp): O^T += V^T P^T over the chunk's 64 tokens; the K-steps of its
-            // first stage go first so that stage is released as early as possible.
+            // Chunk c lives in ring slot c % 3: rows [48 slot, 48 slot + 48) of every
+            // 144-row column atom.
+            // PV(cp): O^T += V^T P^T over the chunk's 48 tokens (three K-steps).
             auto issue_pv = [&](int cp) {
-                const int hp = cp & 1, pb = cp & 1;
+                const int slot = cp % kTcSlots, pb = cp & 1;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int ks = 0; ks < kTcChunk / 16; ++ks) {
 #pragma unroll
                     for (int lb = 0; lb < 4; ++lb) {
                         // V^T: MN-major, 64-latent atoms kAtomKV apart, 8-token groups 1 KB apart
-                        const uint64_t a = tc::desc_sw128(sKV + lb * 2 * kAtomKV + hp * 8192 + ks * 2048,
+                        const uint64_t a = tc::desc_sw128(sKV + lb * 2 * kAtomKV + slot * kSlotRows + ks * 2048,
                                                           kAtomKV, 1024);
-                        // P^T: K-major, 128-byte rows (64 tokens), 8-head groups 1 KB apart
+                        // P^T: K-major, 128-byte rows (48 of 64 tokens used), 8-head groups 1 KB apart
                         const uint64_t bd = tc::desc_sw128(sP + pb * kStageP + ks * 32, 16, 1024);
                         tc::mma_bf16_ss(tmem + lb * 64, a, bd, idPV, (cp > 0 || ks > 0) ? 1u : 0u);
                     }
-                    if (ks == 1) tc::mma_commit(&ctl->kv_empty[2 * hp]);
                 }
-                tc::mma_commit(&ctl->kv_empty[2 * hp + 1]);
+                tc::mma_commit(&ctl->kv_empty[slot]);
                 tc::mma_commit(&ctl->p_empty[pb]);
                 tc::mma_commit(&ctl->o_done);
             };
-            // S(c) = Q K^T over chunk c's 64 tokens into S buffer c & 1.
+            // S(c) = Q K^T over chunk c's 48 tokens into S buffer c & 1.
             auto issue_s = [&](int c) {
-                const int h = c & 1, sb = c & 1;
+                const int slot = c % kTcSlots, sb = c & 1;
                 tc::fence_after_sync();
-                tc::fence_proxy_async_smem();     // the stages were written by cp.async
+                tc::fence_proxy_async_smem();     // the slot was written by cp.async
                 const uint32_t d = tmem + 256 + sb * kTcChunk;
 #pragma unroll
                 for (int kk = 0; kk < kL / 16; ++kk) {
                     const uint32_t qo = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    const uint32_t ko = (kk >> 2) * kAtomKV + h * 8192 + (kk & 3) * 32;
+                    const uint32_t ko = (kk >> 2) * kAtomKV + slot * kSlotRows + (kk & 3) * 32;
                     tc::mma_bf16_ss(d, tc::desc_sw128(sQ + qo, 16, 1024),
                                     tc::desc_sw128(sKV + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
                 }
@@ -304,10 +304,8 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                     continue;
                 }
                 if (ns < nch) {
-                    const int h = ns & 1;
-                    const bool ready = mbar_test(&ctl->kv_full[2 * h], (ns >> 1) & 1) &&
-                                       mbar_test(&ctl->kv_full[2 * h + 1], (ns >> 1) & 1) &&
-                                       (ns < 2 || mbar_test(&ctl->s_empty[h], ((ns >> 1) - 1) & 1));
+                    const bool ready = mbar_test(&ctl->kv_full[ns % kTcSlots], (ns / kTcSlots) & 1) &&
+                                       (ns < 2 || mbar_test(&ctl->s_empty[ns & 1], ((ns >> 1) - 1) & 1));
                     if (ready) {
                         issue_s(ns++);
                         t_last = clock64();
@@ -328,30 +326,30 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         __syncwarp();
     } else if (warp >= 8) {
         // ------------------------------------------------------------------ gather warps
-        // Two groups of four warps (warps 8-11, 12-15) fill alternate 32-token
-        // stages (group p: stages g = p, p+2, ...); warp i of a group copies rows
-        // 8i..8i+7 of the stage as 16-byte cp.async pieces straight into the
-        // swizzled layout (zero-filled for invalid ids). Each lane's copies arrive
-        // on the stage's barrier as they land, so no warp waits for its own copies.
+        // Two groups of four warps (warps 8-11, 12-15) fill alternate chunks
+        // (group p: chunks p, p+2, ...); warp i of a group copies rows 12i..12i+11
+        // of the chunk's slot as 16-byte cp.async pieces straight into the swizzled
+        // layout (zero-filled for invalid ids) and records their validity. Each
+        // lane's copies arrive on the slot's barrier as they land, so no warp waits
+        // for its own copies.
         const int grp = (warp - 8) >> 2, sub = (warp - 8) & 3;
-        const int nsub = 2 * nch;                          // 32-token stages to fill
-        auto load_id = [&](int c) -> int {
-            const int j = c * kTcSub + lane;
-            return (c < nsub && j < ntok) ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
+        auto load_id = [&](int c) -> int {         // lane l < 12: row 12 sub + l of chunk c
+            const int j = c * kTcChunk + 12 * sub + lane;
+            return (lane < 12 && c < nch && j < ntok) ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
         };
-        auto gather_stage = [&](int c, int id) -> bool {
-            const int s = c % kTcStages;
+        auto gather_chunk = [&](int c, int id) -> bool {
+            const int slot = c % kTcSlots;
             bool ok = true;
-            if (c >= kTcStages) ok = tc_wait(ctl, &ctl->kv_empty[s], ((c / kTcStages) - 1) & 1);
+            if (c >= kTcSlots) ok = tc_wait(ctl, &ctl->kv_empty[slot], ((c / kTcSlots) - 1) & 1);
             if (!__all_sync(0xffffffffu, ok)) return false;
             const bool valid = id >= 0 && id < T && (long long)rs + id < (long long)kv_rows;
-            const uint32_t vm = __ballot_sync(0xffffffffu, valid);
+            const uint32_t vm = __ballot_sync(0xffffffffu, valid);   // bits 0..11
             const int myrow = valid ? rs + id : -1;
-            const uint32_t dst0 = sKV + s * (kTcSub * 128);   // rows [32s, 32s+32) of each atom
+            const uint32_t dst0 = sKV + slot * kSlotRows;
 #pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-                const int r = 8 * sub + rr;
-                const int row = __shfl_sync(0xffffffffu, myrow, r);
+            for (int rr = 0; rr < 12; ++rr) {
+                const int r = 12 * sub + rr;                 // row within the chunk
+                const int row = __shfl_sync(0xffffffffu, myrow, rr);
                 const __nv_bfloat16 *src = row >= 0 ? kv + (size_t)row * kL : qm;   // qm: never read
                 const uint32_t nb = row >= 0 ? 16u : 0u;
 #pragma unroll
@@ -361,24 +359,24 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                     tc::cp_async16_zfill(dst, row >= 0 ? src + cc * 8 : src, nb);
                 }
             }
-            if (sub == 0 && lane == 0) {
-                ctl->vmask[s] = vm;
-                mbar_arrive(&ctl->kv_full[s]);             // releases vmask
+            if (lane == 0) {
+                ctl->vmask[slot][sub] = (uint16_t)vm;
+                mbar_arrive(&ctl->kv_full[slot]);          // releases this warp's mask
             }
-            tc::cp_async_arrive_noinc(&ctl->kv_full[s]);
+            tc::cp_async_arrive_noinc(&ctl->kv_full[slot]);
             return true;
         };
-        // ids of the group's next two stages are in flight (static queue slots)
+        // ids of the group's next two chunks are in flight (static queue slots)
         int idq[2] = {load_id(grp), load_id(grp + 2)};
         bool go = true;
-        for (int c0 = grp; go && c0 < nsub; c0 += 4) {
+        for (int c0 = grp; go && c0 < nch; c0 += 4) {
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int c = c0 + 2 * u;
-                if (!go || c >= nsub) break;
+                if (!go || c >= nch) break;
                 const int id = idq[u];
                 idq[u] = load_id(c + 4);
-                go = gather_stage(c, id);
+                go = gather_chunk(c, id);
             }
         }
         tc::cp_async_wait_all();          // nothing of this warp in flight past here
@@ -400,26 +398,27 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         float m_used = -INFINITY, l = 0.f;
         bool failed = false;
         for (int c = 0; c < nch; ++c) {
-            const int h = c & 1, sb = c & 1;
-            bool bad = !tc_wait(ctl, &ctl->kv_full[2 * h], (c >> 1) & 1);
-            bad = bad || !tc_wait(ctl, &ctl->kv_full[2 * h + 1], (c >> 1) & 1);
+            const int slot = c % kTcSlots, sb = c & 1;
+            bool bad = !tc_wait(ctl, &ctl->kv_full[slot], (c / kTcSlots) & 1);
             bad = bad || !tc_wait(ctl, &ctl->s_full[sb], (c >> 1) & 1);
             tc::fence_after_sync();
-            uint32_t r[kTcChunk / 2];
+            // 48 columns: this thread's 24 tokens par + 2i, i < 24
+            uint32_t r[24];
             tc::tmem_ld16x64b_x16(tl + 256 + sb * kTcChunk, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-            tc::tmem_ld16x64b_x16(tl + 256 + sb * kTcChunk + 32, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+            tc::tmem_ld16x64b_x8(tl + 256 + sb * kTcChunk + 32, *reinterpret_cast<uint32_t(*)[8]>(&r[16]));
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             mbar_arrive(&ctl->s_empty[sb]);
 
-            // token par + 2i: i < 16 in the first stage of the pair, i >= 16 in the second
-            const uint32_t vm0 = ctl->vmask[2 * h] >> par, vm1 = ctl->vmask[2 * h + 1] >> par;
-            float z[kTcChunk / 2];
+            // validity of the chunk's 48 rows (12 per gather warp), then bit 2i: token par + 2i
+            const uint64_t vm48 = (uint64_t)ctl->vmask[slot][0] | ((uint64_t)ctl->vmask[slot][1] << 12) |
+                                  ((uint64_t)ctl->vmask[slot][2] << 24) | ((uint64_t)ctl->vmask[slot][3] << 36);
+            const uint64_t vmp = vm48 >> par;
+            float z[24];
             float mx = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < kTcChunk / 2; ++i) {
-                const uint32_t bit = i < 16 ? (vm0 >> (2 * i)) & 1 : (vm1 >> (2 * i - 32)) & 1;
-                z[i] = bit ? __uint_as_float(r[i]) * scale_log2 : -INFINITY;
+            for (int i = 0; i < 24; ++i) {
+                z[i] = ((vmp >> (2 * i)) & 1) ? __uint_as_float(r[i]) * scale_log2 : -INFINITY;
                 mx = fmaxf(mx, z[i]);
             }
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -428,23 +427,23 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                 alpha = ex2(m_used - mx);
                 m_used = mx;
             }
-            float pv[kTcChunk / 2];
+            float pv[24];
             float psum = 0.f;
 #pragma unroll
-            for (int i = 0; i < kTcChunk / 2; ++i) {
+            for (int i = 0; i < 24; ++i) {
                 pv[i] = z[i] == -INFINITY ? 0.f : ex2(z[i] - m_used);
                 psum += pv[i];       // fp32 weights: the row sum and lse stay exact to fp32
             }
             psum += __shfl_xor_sync(0xffffffffu, psum, 2);
             l = fmaf(l, alpha, psum);
             if (owner) ctl->alpha[hh] = alpha;
-            // bf16 P row of the head: this thread packs tokens 32par .. 32par+31,
+            // bf16 P row of the head: this thread packs tokens 24par .. 24par+23,
             // taking the other parity from its partner.
-            uint32_t pk[16];
+            uint32_t pk[12];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float recv = __shfl_xor_sync(0xffffffffu, par ? pv[k] : pv[k + 16], 2);
-                pk[k] = par ? pack_bf16x2(recv, pv[k + 16]) : pack_bf16x2(pv[k], recv);
+            for (int k = 0; k < 12; ++k) {
+                const float recv = __shfl_xor_sync(0xffffffffu, par ? pv[k] : pv[k + 12], 2);
+                pk[k] = par ? pack_bf16x2(recv, pv[k + 12]) : pack_bf16x2(pv[k], recv);
             }
 
             bad = bad || (c >= 2 && !tc_wait(ctl, &ctl->p_empty[sb], ((c >> 1) - 1) & 1));
@@ -455,12 +454,12 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                 need = true;
             }
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                const int c16 = 4 * par + q4;     // 16-byte piece of the 128-byte row
+            for (int q3 = 0; q3 < 3; ++q3) {
+                const int c16 = 3 * par + q3;     // 16-byte piece of the 128-byte row (pieces 6, 7 unused)
                 const uint32_t dst = sP + sb * kStageP + hh * 128 + ((c16 ^ (hh & 7)) << 4);
                 asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
-                             "r"(pk[4 * q4]), "r"(pk[4 * q4 + 1]), "r"(pk[4 * q4 + 2]),
-                             "r"(pk[4 * q4 + 3])
+                             "r"(pk[4 * q3]), "r"(pk[4 * q3 + 1]), "r"(pk[4 * q3 + 2]),
+                             "r"(pk[4 * q3 + 3])
                              : "memory");
             }
             if (need) {

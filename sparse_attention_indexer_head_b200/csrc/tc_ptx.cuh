@@ -121,6 +121,14 @@ DSA_DEVINL void tmem_ld16x64b_x16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
 }
 
+// The same shape over 16 columns: r[i] = column ((t >> 1) & 1) + 2i, i < 8.
+DSA_DEVINL void tmem_ld16x64b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.16x64b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+
 DSA_DEVINL void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 DSA_DEVINL void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 

@@ -109,11 +109,12 @@ def test_topk_expand_refusals(B):
 
 def test_sparse_mla_refusals(B):
     L = B.lib
-    # partials of every split (the plan keeps the grid within 148 CTAs; 64-token
-    # chunks): 2 queries -> 32 splits of one chunk; 16 queries -> 8 splits of 4
+    # partials of every split (the plan keeps the grid within 148 CTAs; 48-token
+    # chunks, 43 of them for 2048 ids): 2 queries -> 43 splits of one chunk;
+    # 16 queries -> 9 splits of 5 chunks
     ws = B.dsa_sparse_mla_workspace_size(2, 64, 2048)
-    assert ws == 2 * 32 * 64 * 516 * 4
-    assert B.dsa_sparse_mla_workspace_size(16, 64, 2048) == 16 * 8 * 64 * 516 * 4
+    assert ws == 2 * 43 * 64 * 516 * 4
+    assert B.dsa_sparse_mla_workspace_size(16, 64, 2048) == 16 * 9 * 64 * 516 * 4
     # at least 148 CTAs without splitting: one split, no workspace
     assert B.dsa_sparse_mla_workspace_size(148, 64, 2048) == 0
     assert B.dsa_sparse_mla_workspace_size(74, 128, 2048) == 0
