@@ -28,31 +28,33 @@ DSA_DEVINL uint32_t score_key(float s, bool is_cand) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive prefix sum of v over the block (thread order); *total gets the sum.
-DSA_DEVINL int block_excl_scan(int v, int *s_warp, int *total) {
+// Exclusive prefix sums of (a, b) over the block in one pass; *ta, *tb get the sums.
+DSA_DEVINL int2 block_excl_scan2(int a, int b, int2 *s_warp2, int *ta, int *tb) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
+    int x = a, y = b;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, off);
-        if (lane >= off) x += y;
+        const int u = __shfl_up_sync(0xffffffffu, x, off);
+        const int v = __shfl_up_sync(0xffffffffu, y, off);
+        if (lane >= off) { x += u; y += v; }
     }
-    if (lane == 31) s_warp[warp] = x;
+    if (lane == 31) s_warp2[warp] = make_int2(x, y);
     __syncthreads();
     if (warp == 0) {
-        int w = lane < kTopkWarps ? s_warp[lane] : 0;
+        int2 w = lane < kTopkWarps ? s_warp2[lane] : make_int2(0, 0);
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, w, off);
-            if (lane >= off) w += y;
+            const int u = __shfl_up_sync(0xffffffffu, w.x, off);
+            const int v = __shfl_up_sync(0xffffffffu, w.y, off);
+            if (lane >= off) { w.x += u; w.y += v; }
         }
-        if (lane < kTopkWarps) s_warp[lane] = w;   // inclusive warp totals
+        if (lane < kTopkWarps) s_warp2[lane] = w;   // inclusive warp totals
     }
     __syncthreads();
-    const int before = (warp ? s_warp[warp - 1] : 0) + x - v;
-    *total = s_warp[kTopkWarps - 1];
-    __syncthreads();
-    return before;
+    const int2 before = warp ? s_warp2[warp - 1] : make_int2(0, 0);
+    *ta = s_warp2[kTopkWarps - 1].x;
+    *tb = s_warp2[kTopkWarps - 1].y;
+    return make_int2(before.x + x - a, before.y + y - b);
 }
 
 __global__ void __launch_bounds__(kTopkThreads)
@@ -63,9 +65,10 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     extern __shared__ __align__(16) uint8_t topk_smem[];
     int32_t *slist = reinterpret_cast<int32_t *>(topk_smem);                  // [K] selected ids
     uint32_t *skeys = reinterpret_cast<uint32_t *>(topk_smem) + K;           // [P] if cached
-    __shared__ int hist[256];
-    __shared__ int s_warp[kTopkWarps];
-    __shared__ int s_pick[2];
+    __shared__ int hist[2][256];          // double-buffered radix histograms
+    __shared__ int2 s_warp2[kTopkWarps];
+    __shared__ int s_pick[2][2];          // per pass parity: (digit, count above it)
+    __shared__ int s_ncand;
 
     const int tid = threadIdx.x;
     const int q = blockIdx.x;
@@ -82,8 +85,13 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     };
 
     // Keys: four loads of each array in flight per thread before any use; the
-    // histogram of the top byte (the first radix pass) is built on the way.
-    if (tid < 256) hist[tid] = 0;
+    // histogram of the top byte (the first radix pass) and the candidate count
+    // are built on the way.
+    if (tid < 256) {
+        hist[0][tid] = 0;
+        hist[1][tid] = 0;
+    }
+    if (tid == 0) s_ncand = 0;
     __syncthreads();
     int cnt = 0;
     for (int p0 = 0; p0 < P; p0 += 4 * kTopkThreads) {
@@ -103,21 +111,27 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
             cnt += k != 0u;
             const uint32_t d = p < P ? (k >> 24) : 0x100u;
             const uint32_t peers = __match_any_sync(0xffffffffu, d);
-            if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
+            if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[0][d], __popc(peers));
         }
     }
-    int n_cand;
-    (void)block_excl_scan(cnt, s_warp, &n_cand);
-    const int nq = min(K, n_cand);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    if ((tid & 31) == 0) atomicAdd(&s_ncand, cnt);
+    __syncthreads();
+    const int nq = min(K, s_ncand);
 
-    // Radix select of the nq-th largest key, 8 bits per pass, most significant first.
+    // Radix select of the nq-th largest key, 8 bits per pass, most significant
+    // first. Pass i builds its histogram in hist[i & 1] (cleared one pass
+    // earlier) and its pick in s_pick[i & 1], so a pass takes two barriers.
     uint32_t prefix = 0, pmask = 0;
     int remaining = nq;
     if (nq > 0) {
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            if (shift != 24) {
-                if (tid < 256) hist[tid] = 0;
-                __syncthreads();
+#pragma unroll 1
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass, hb = pass & 1;
+            if (pass > 0) {
+                // the other buffer's pass is over (its pick was read): clear it for the next
+                if (tid < 256) hist[hb ^ 1][tid] = 0;
                 // Warp-aggregated increments: lanes with the same digit elect one
                 // leader, so a few crowded bins do not serialise the whole block.
                 for (int base = (tid & ~31); base < P; base += kTopkThreads) {
@@ -128,7 +142,7 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
                         if ((k & pmask) == prefix) d = (k >> shift) & 0xFF;
                     }
                     const uint32_t peers = __match_any_sync(0xffffffffu, d);
-                    if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
+                    if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[hb][d], __popc(peers));
                 }
                 __syncthreads();
             }
@@ -137,7 +151,7 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
                 int c[8], sum = 0;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    c[i] = hist[255 - 8 * tid - i];
+                    c[i] = hist[hb][255 - 8 * tid - i];
                     sum += c[i];
                 }
                 int above = sum;   // inclusive scan over lanes (descending bins)
@@ -150,17 +164,16 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     if (run < remaining && remaining <= run + c[i]) {
-                        s_pick[0] = 255 - 8 * tid - i;
-                        s_pick[1] = run;
+                        s_pick[hb][0] = 255 - 8 * tid - i;
+                        s_pick[hb][1] = run;
                     }
                     run += c[i];
                 }
             }
             __syncthreads();
-            remaining -= s_pick[1];
-            prefix |= (uint32_t)s_pick[0] << shift;
+            remaining -= s_pick[hb][1];
+            prefix |= (uint32_t)s_pick[hb][0] << shift;
             pmask |= 0xFFu << shift;
-            __syncthreads();
         }
     }
     const uint32_t tau = prefix;   // the nq-th largest key (when nq > 0)
@@ -176,9 +189,9 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
             gt += k > tau;
             eq += k == tau;
         }
-    int tot;
-    const int gt_before = block_excl_scan(gt, s_warp, &tot);
-    const int eq_before = block_excl_scan(eq, s_warp, &tot);
+    int tot_gt, tot_eq;
+    const int2 before = block_excl_scan2(gt, eq, s_warp2, &tot_gt, &tot_eq);
+    const int gt_before = before.x, eq_before = before.y;
     // The winners in ascending pool id: every key above tau, then the r lowest-id
     // keys equal to tau, each placed at its id-order position.
     if (nq > 0) {
