@@ -578,42 +578,38 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-// One CTA per (head, query); 128 threads x 4 channels. The split loop is
-// unrolled by 8 so eight partial rows are in flight at once; splits are merged
-// in split order (deterministic).
+// One CTA per (head, query); 128 threads x 4 channels. Up to 16 splits are
+// merged from one round of loads (every split's m, l and row in flight at once);
+// more splits take a first round for the maxima. Splits are merged in split
+// order (deterministic).
 __global__ void __launch_bounds__(128)
 mla_combine_kernel(const float *__restrict__ part, int Hm, int S, __nv_bfloat16 *__restrict__ out,
                    float *__restrict__ lse) {
+    constexpr int kRound = 16;
     const int h = blockIdx.x, q = blockIdx.y, tid = threadIdx.x;
     pdl_wait();
     pdl_launch_dependents();
     const float *base = part + ((size_t)q * S * Hm + h) * kPartStride;
     const size_t sstride = (size_t)Hm * kPartStride;
     float M = -INFINITY;
-    for (int s0 = 0; s0 < S; s0 += 8) {
-        float mv[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mv[u] = s0 + u < S ? __ldg(base + (s0 + u) * sstride + kL) : -INFINITY;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) M = fmaxf(M, mv[u]);
-    }
     float o[4] = {0.f, 0.f, 0.f, 0.f};
     float lsum = 0.f;
-    if (M != -INFINITY) {
-        for (int s0 = 0; s0 < S; s0 += 8) {
-            float mv[8], lv[8];
-            float4 v[8];
+    if (S <= kRound) {
+        float mv[kRound], lv[kRound];
+        float4 v[kRound];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const bool in = s0 + u < S;
-                const float *ps = base + (s0 + u) * sstride;
-                mv[u] = in ? __ldg(ps + kL) : -INFINITY;
-                lv[u] = in ? __ldg(ps + kL + 1) : 0.f;
-                v[u] = in ? __ldg(reinterpret_cast<const float4 *>(ps + 4 * tid))
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+        for (int u = 0; u < kRound; ++u) {
+            const bool in = u < S;
+            const float *ps = base + u * sstride;
+            mv[u] = in ? __ldg(ps + kL) : -INFINITY;
+            lv[u] = in ? __ldg(ps + kL + 1) : 0.f;
+            v[u] = in ? __ldg(reinterpret_cast<const float4 *>(ps + 4 * tid)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < kRound; ++u) M = fmaxf(M, mv[u]);
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int u = 0; u < kRound; ++u) {
                 if (mv[u] == -INFINITY) continue;
                 const float w = ex2(mv[u] - M);
                 lsum = fmaf(lv[u], w, lsum);
@@ -621,6 +617,39 @@ mla_combine_kernel(const float *__restrict__ part, int Hm, int S, __nv_bfloat16 
                 o[1] = fmaf(v[u].y, w, o[1]);
                 o[2] = fmaf(v[u].z, w, o[2]);
                 o[3] = fmaf(v[u].w, w, o[3]);
+            }
+        }
+    } else {
+        for (int s0 = 0; s0 < S; s0 += 8) {
+            float mv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mv[u] = s0 + u < S ? __ldg(base + (s0 + u) * sstride + kL) : -INFINITY;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) M = fmaxf(M, mv[u]);
+        }
+        if (M != -INFINITY) {
+            for (int s0 = 0; s0 < S; s0 += 8) {
+                float mv[8], lv[8];
+                float4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const bool in = s0 + u < S;
+                    const float *ps = base + (s0 + u) * sstride;
+                    mv[u] = in ? __ldg(ps + kL) : -INFINITY;
+                    lv[u] = in ? __ldg(ps + kL + 1) : 0.f;
+                    v[u] = in ? __ldg(reinterpret_cast<const float4 *>(ps + 4 * tid))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (mv[u] == -INFINITY) continue;
+                    const float w = ex2(mv[u] - M);
+                    lsum = fmaf(lv[u], w, lsum);
+                    o[0] = fmaf(v[u].x, w, o[0]);
+                    o[1] = fmaf(v[u].y, w, o[1]);
+                    o[2] = fmaf(v[u].z, w, o[2]);
+                    o[3] = fmaf(v[u].w, w, o[3]);
+                }
             }
         }
     }
