@@ -262,3 +262,37 @@ def test_mla_heads_and_id_edge_cases(B, hm):
     assert (go[2] == 0).all() and np.isneginf(gl[2]).all()      # empty request
     np.testing.assert_array_equal(go[3, 0], kv[123])                # single token: its row
     device_status_clean(B)
+
+
+def test_mla_rows_past_kv_rows_are_not_read(B):
+    # kv_rows bounds the cache: an id whose row falls at or past it counts as
+    # invalid (it is neither read nor weighted). Request 1 owns rows 300..389;
+    # the cache is declared to hold 350 rows, so its ids 50..89 drop out.
+    rng = np.random.default_rng(11)
+    hm, Wd = 64, 160
+    rs = np.array([0, 300, 390], np.int32)
+    kv_full = W.f32_to_bf16_bits(rng.standard_normal((390, 512)).astype(np.float32))
+    q = W.f32_to_bf16_bits(rng.standard_normal((2, hm, 512)).astype(np.float32))
+    q_req = np.array([0, 1], np.int32)
+    ids = np.full((2, Wd), -1, np.int32)
+    ids[0, :140] = rng.choice(300, 140, replace=False)
+    ids[1, :90] = rng.permutation(90)
+    kv_rows = 350
+    ids_ref = ids.copy()
+    ids_ref[1][(ids_ref[1] >= 0) & (rs[1] + ids_ref[1] >= kv_rows)] = -1
+    scale = float(1 / np.sqrt(512))
+    ref_out, ref_lse = O.sparse_mla(q, kv_full, rs, q_req, ids_ref, scale)
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    out = torch.empty(2, hm, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(2, hm, dtype=torch.float32, device="cuda")
+    ws_n = B.dsa_sparse_mla_workspace_size(2, hm, Wd)
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device="cuda")
+    # the rows past kv_rows hold NaN on the device: reading any of them would show
+    kv_dev = kv_full.copy()
+    kv_dev[kv_rows:] = 0x7FC0
+    B.dsa_sparse_mla_decode(dev_bits(q), dev_bits(kv_dev), kv_rows, d(rs), d(q_req), d(ids), 2, 2,
+                            hm, Wd, 512, 0, scale, out, lse, ws, ws_n)
+    assert np.isfinite(lse.cpu().numpy()).all()
+    assert_mla_close(host_bits(out), ref_out, lse.cpu().numpy(), ref_lse,
+                     vbound=mla_value_bound(kv_full, rs, q_req, ids_ref))
+    device_status_clean(B)
