@@ -30,8 +30,8 @@
  *     start while the kernel before it on the stream drains, and waits for
  *     that kernel (griddepcontrol.wait) before reading anything an earlier
  *     stage of this path writes. Before that wait it already reads inputs the
- *     path never writes: hidden and w (head gate); ape (kpool_compress); q,
- *     q_req and req_start (sparse MLA). Write those before the kernel that
+ *     path never writes: hidden and w (head gate); ape (kpool_compress); q_idx
+ *     (index_scores); q, q_req and req_start (sparse MLA). Write those before the kernel that
  *     immediately precedes the call on the stream, or separate that kernel
  *     from the call by a copy, an event wait or a host synchronisation.
  *   - Request geometry lives on the device: request b owns cache rows

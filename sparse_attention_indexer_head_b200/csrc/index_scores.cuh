@@ -40,7 +40,7 @@ index_scores_kernel(const __grid_constant__ CUtensorMap key_map,
                     const int32_t *__restrict__ first_valid, int B, int kpool, int max_pools,
                     float *__restrict__ scores, uint8_t *__restrict__ cand) {
     extern __shared__ uint8_t sc_smem_raw[];
-    __shared__ __align__(8) uint64_t load_bar, mma_bar;
+    __shared__ __align__(8) uint64_t q_bar, load_bar, mma_bar;
     __shared__ uint32_t tmem_base;
 
     const uint32_t raw = smem_u32(sc_smem_raw);
@@ -56,10 +56,15 @@ index_scores_kernel(const __grid_constant__ CUtensorMap key_map,
         tc::tmem_alloc(&tmem_base, 32);
         tc::tmem_relinquish();
     }
-    if (tid == 32) {
+    if (tid == 0) {
+        mbar_init(&q_bar, 1);
         mbar_init(&load_bar, 1);
         mbar_init(&mma_bar, 1);
         fence_mbarrier_init();
+        // the query's 16 x 128 head rows are a step input: in flight before the wait
+        mbar_arrive_expect_tx(&q_bar, 2 * kScoreQAtom);
+        tma_load_2d(sQ, &q_map, 0, q * H, &q_bar);
+        tma_load_2d(sQ + kScoreQAtom, &q_map, 64, q * H, &q_bar);
     }
     pdl_wait();
     pdl_launch_dependents();
@@ -83,13 +88,11 @@ index_scores_kernel(const __grid_constant__ CUtensorMap key_map,
     bool ok = true;
     if (any) {
         if (tid == 0) {
-            mbar_arrive_expect_tx(&load_bar, 2 * kScoreKeyAtom + 2 * kScoreQAtom);
+            mbar_arrive_expect_tx(&load_bar, 2 * kScoreKeyAtom);
             const int row = b * max_pools + p0;
             tma_load_2d(sK, &key_map, 0, row, &load_bar);
             tma_load_2d(sK + kScoreKeyAtom, &key_map, 64, row, &load_bar);
-            tma_load_2d(sQ, &q_map, 0, q * H, &load_bar);
-            tma_load_2d(sQ + kScoreQAtom, &q_map, 64, q * H, &load_bar);
-            ok = mbar_wait(&load_bar, 0);
+            ok = mbar_wait(&load_bar, 0) && mbar_wait(&q_bar, 0);
             if (ok) {
                 tc::fence_after_sync();
                 constexpr uint32_t idesc = tc::idesc_bf16(kScorePools, kScoreHeads, false, false);
@@ -108,6 +111,8 @@ index_scores_kernel(const __grid_constant__ CUtensorMap key_map,
         ok = __syncthreads_and(ok) != 0;
         tc::fence_after_sync();
     }
+
+    if (!any && tid == 0) (void)mbar_wait(&q_bar, 0);   // the query rows land before the CTA leaves
 
     float score = -INFINITY;
     if (any && ok) {

@@ -132,8 +132,9 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
             if (pass > 0) {
                 // the other buffer's pass is over (its pick was read): clear it for the next
                 if (tid < 256) hist[hb ^ 1][tid] = 0;
-                // Warp-aggregated increments: lanes with the same digit elect one
-                // leader, so a few crowded bins do not serialise the whole block.
+                // Only keys under the chosen prefix count, and they spread over the
+                // next byte: plain shared atomics, except in a warp where many lanes
+                // match (crowded bins, e.g. equal scores), which aggregates per digit.
                 for (int base = (tid & ~31); base < P; base += kTopkThreads) {
                     const int p = base + (tid & 31);
                     uint32_t d = 0x100u;   // no bin
@@ -141,8 +142,13 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
                         const uint32_t k = key_at(p);
                         if ((k & pmask) == prefix) d = (k >> shift) & 0xFF;
                     }
-                    const uint32_t peers = __match_any_sync(0xffffffffu, d);
-                    if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[hb][d], __popc(peers));
+                    const uint32_t act = __ballot_sync(0xffffffffu, d != 0x100u);
+                    if (__popc(act) > 8) {
+                        const uint32_t peers = __match_any_sync(0xffffffffu, d);
+                        if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[hb][d], __popc(peers));
+                    } else if (d != 0x100u) {
+                        atomicAdd(&hist[hb][d], 1);
+                    }
                 }
                 __syncthreads();
             }
