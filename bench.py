@@ -154,7 +154,9 @@ def traffic_for(kernel: str, kernel_file: str, units_scale: float = 1.0):
     return float(t["dram_bytes_per_launch"]) * units_scale
 
 
-def dist_setup():
+def dist_setup(backend: str = "nccl"):
+    """Rank, world size and local rank from the launcher's environment; joins the
+    process group when world > 1 (NCCL on GPUs; gloo serves the CPU tests)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -162,20 +164,29 @@ def dist_setup():
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return rank, world, local
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The maximum of x over all ranks (the step time every rank reports)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(queries_per_rank: int, world: int, steps: int, seconds: float) -> float:
+    """Whole-job queries/s: every rank runs its own batch each step (weak scaling),
+    timed by the slowest rank."""
+    return queries_per_rank * world * steps / seconds
 
 
 def barrier(world: int):
@@ -298,7 +309,7 @@ def gpu_arm(args, wl_fn):
     ms_local = ev0.elapsed_time(ev1)
     ms_total = max_over_ranks(ms_local, world)
     ms_per_step = ms_total / args.steps
-    value = wl.Q * world * args.steps / (ms_total / 1e3)
+    value = replica_throughput(wl.Q, world, args.steps, ms_total / 1e3)
     clk = clocks.summary(t_wall0 - 0.05, t_wall1 + 0.05) if clocks else None
 
     # ---- per-stage device time. Each stage is bracketed by events and preceded by a
@@ -346,7 +357,7 @@ def gpu_arm(args, wl_fn):
             out_host.copy_(s0.out, non_blocking=True)
             stream.synchronize()
     e2e_s = max_over_ranks(time.perf_counter() - t0, world)
-    e2e_value = wl.Q * world * e2e_steps / e2e_s
+    e2e_value = replica_throughput(wl.Q, world, e2e_steps, e2e_s)
 
     if clocks:
         clocks.stop()
