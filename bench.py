@@ -404,7 +404,7 @@ def gpu_arm(args, wl_fn):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "path": "pinned host query inputs -> H2D -> 5 ABI calls -> D2H of out, "
                         "synchronised each step"},
-        "gpu_launches": DecodeStep.KERNELS_PER_STEP * args.steps,
+        "gpu_launches": steps[0].kernels_per_step() * args.steps,
         "clocks": clk,
         "device_error": B.dsa_device_status(reset=True),
     }

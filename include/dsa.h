@@ -202,6 +202,13 @@ int dsa_topk_expand(const float *scores, const uint8_t *cand, const int32_t *poo
  * multiple of 16 with 16 <= Hm <= 128, W >= 0.
  */
 size_t dsa_sparse_mla_workspace_size(int Q, int Hm, int W);
+/*
+ * Number of kernels dsa_sparse_mla_decode launches for this shape on the
+ * current device (1, or 2 when the splits merge through the workspace); 0 for
+ * an empty or invalid shape. An inspection aid for callers that account for
+ * launches; it launches nothing.
+ */
+int dsa_sparse_mla_launch_count(int Q, int Hm, int W);
 int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows,
                           const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
                           int W, int kv_lora, int rope_dim, float sm_scale, dsa_bf16 *out,

@@ -26,7 +26,8 @@ DSA_ERR_CUDA = 5
 EXPORTS = (
     "dsa_status_string", "dsa_abi_version", "dsa_device_status", "dsa_head_gate",
     "dsa_kpool_compress", "dsa_index_scores", "dsa_topk_expand",
-    "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_decode", "dsa_sparse_mla_decode_noalloc",
+    "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_launch_count", "dsa_sparse_mla_decode",
+    "dsa_sparse_mla_decode_noalloc",
 )
 DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -55,6 +56,7 @@ def _load() -> ctypes.CDLL:
         "dsa_index_scores": ([P, P, P, P, I, I, I, P, P, P, I, I, I, P, P, P], I),
         "dsa_topk_expand": ([P, P, P, P, I, I, I, I, I, P, P, P], I),
         "dsa_sparse_mla_workspace_size": ([I, I, I], Z),
+        "dsa_sparse_mla_launch_count": ([I, I, I], I),
         "dsa_sparse_mla_decode": ([P, P, I64, P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P], I),
         "dsa_sparse_mla_decode_noalloc": ([P, P, I64, P, P, P, I, I, I, I, I, I, F, P, P, P], I),
     }
@@ -136,6 +138,10 @@ def dsa_topk_expand(scores, cand, pool_idx, q_req, Q: int, B: int, max_pools: in
 
 def dsa_sparse_mla_workspace_size(Q: int, Hm: int, W: int) -> int:
     return int(lib.dsa_sparse_mla_workspace_size(Q, Hm, W))
+
+
+def dsa_sparse_mla_launch_count(Q: int, Hm: int, W: int) -> int:
+    return int(lib.dsa_sparse_mla_launch_count(Q, Hm, W))
 
 
 def dsa_sparse_mla_decode(q, kv, kv_rows: int, req_start, q_req, token_ids, Q: int, B: int,

@@ -106,6 +106,10 @@ size_t dsa_sparse_mla_workspace_size(int Q, int Hm, int W) {
     return dsa::mla_workspace_bytes(Q, Hm, W);
 }
 
+int dsa_sparse_mla_launch_count(int Q, int Hm, int W) {
+    return dsa::sparse_mla_launch_count(Q, Hm, W);
+}
+
 int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows,
                           const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
                           int W, int kv_lora, int rope_dim, float sm_scale, dsa_bf16 *out,

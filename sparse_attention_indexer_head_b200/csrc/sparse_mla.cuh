@@ -708,6 +708,15 @@ inline MlaGeom mla_launch_geometry(int Q, int Hm, int W) {
     return g;
 }
 
+// Kernels sparse_mla_launch runs for this shape on the current device: the
+// split kernel, plus the combine when the splits merge through the workspace.
+inline int sparse_mla_launch_count(int Q, int Hm, int W) {
+    if (Q <= 0 || Hm <= 0 || W < 0) return 0;
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true>), kTcSmemBytes)) return 0;
+    const MlaGeom g = mla_launch_geometry(Q, Hm, W);
+    return (g.S > 1 && !g.cluster) ? 2 : 1;
+}
+
 inline int sparse_mla_launch(const void *q, const void *kv, int64_t kv_rows,
                              const int32_t *req_start, const int32_t *q_req,
                              const int32_t *token_ids, int Q, int B, int Hm, int W, int kv_lora,

@@ -126,7 +126,11 @@ class DecodeStep:
         self.topk_expand(stream)
         self.sparse_mla(stream)
 
-    KERNELS_PER_STEP = 6   # gate, compress, scores, topk+expand, mla split, mla combine
+    def kernels_per_step(self) -> int:
+        """Launches of run(): gate, compress, scores, topk+expand, and the MLA's one or
+        two kernels (split kernel, plus the combine when splits merge in the workspace)."""
+        g = self.g
+        return 4 + B.dsa_sparse_mla_launch_count(g.Q, g.hm, g.W)
 
     def outputs_numpy(self) -> Dict[str, np.ndarray]:
         def u16(x):

@@ -296,3 +296,12 @@ def test_mla_rows_past_kv_rows_are_not_read(B):
     assert_mla_close(host_bits(out), ref_out, lse.cpu().numpy(), ref_lse,
                      vbound=mla_value_bound(kv_full, rs, q_req, ids_ref))
     device_status_clean(B)
+
+
+def test_mla_launch_count(B):
+    # one split: the split kernel alone; more than 8 splits: always the workspace
+    # merge, so a combine kernel too; 2..8 splits: 1 or 2 (clusters where they fit)
+    assert B.dsa_sparse_mla_launch_count(148, 64, 2048) == 1
+    assert B.dsa_sparse_mla_launch_count(2, 64, 2048) == 2
+    assert B.dsa_sparse_mla_launch_count(16, 64, 2048) in (1, 2)
+    assert B.dsa_sparse_mla_launch_count(0, 64, 2048) == 0
