@@ -339,9 +339,43 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     unpack8x2(ldg_nc_v4(ln_w + 8 * l), lw);
     unpack8x2(ldg_nc_v4(ln_b + 8 * l), lb);
 
-    for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
+    // Consumer-wide barrier (named barrier 1) that also ORs a stop flag, so every
+    // consumer thread takes the same decision to leave.
+    auto bar_or = [&](bool v) -> bool {
+        uint32_t r;
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+            "bar.red.or.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(r)
+            : "r"((uint32_t)v), "n"(kCmpConsumers)
+            : "memory");
+        return r != 0;
+    };
+    // Tile i's LayerNorm statistics are computed one iteration early, next to
+    // tile i-1's pools (different stage buffers); the one barrier of an
+    // iteration separates a tile's statistics from its pools.
+    const int n_t = t_end - t_begin;
+    auto tile_ready = [&](int i) -> bool {
+        return !__any_sync(0xffffffffu, !mbar_wait(&full[i % kCmpStages], (i / kCmpStages) & 1));
+    };
+    auto stats_of = [&](int i) {
         const int s = i % kCmpStages;
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / kCmpStages) & 1))) break;
+        const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
+        token_stats(sk, meta[s].n_in * KP, eps, &s_stat[s][0], tid, kCmpConsumers);
+    };
+    bool bad = false;
+    if (n_t > 0) {
+        bad = !tile_ready(0);
+        if (!bad) stats_of(0);
+    }
+    bool stop = bar_or(bad);
+    for (int i = 0; !stop && i < n_t; ++i) {
+        const int s = i % kCmpStages;
+        bool bad_next = false;
+        if (i + 1 < n_t) {
+            bad_next = !tile_ready(i + 1);
+            if (!bad_next) stats_of(i + 1);
+        }
         const CmpMeta m = meta[s];
         const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
         const __nv_bfloat16 *sg = sk + kCmpTileTokens * kD;
@@ -353,10 +387,6 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             pool_idx[(pool_base + m.p0) * KP + x] = -1;
         for (int x = m.n_in + tid; x < m.p1 - m.p0; x += kCmpConsumers)
             pool_valid[pool_base + m.p0 + x] = 0;
-
-        // LayerNorm statistics of the tile's rows, then every pool of the tile.
-        token_stats(sk, m.n_in * KP, eps, &s_stat[s][0], tid, kCmpConsumers);
-        asm volatile("bar.sync 1, %0;" ::"n"(kCmpConsumers) : "memory");
 
         // Warp-uniform loop: the two half-warps of a warp take pools ii and ii+1;
         // a half-warp past the tile computes on a loaded row and stores nothing.
@@ -378,6 +408,7 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
+        stop = bar_or(bad_next);
     }
 }
 
