@@ -351,31 +351,16 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             : "memory");
         return r != 0;
     };
-    // Tile i's LayerNorm statistics are computed one iteration early, next to
-    // tile i-1's pools (different stage buffers); the one barrier of an
-    // iteration separates a tile's statistics from its pools.
-    const int n_t = t_end - t_begin;
-    auto tile_ready = [&](int i) -> bool {
-        return !__any_sync(0xffffffffu, !mbar_wait(&full[i % kCmpStages], (i / kCmpStages) & 1));
-    };
-    auto stats_of = [&](int i) {
+    // Per tile: wait for its data, its LayerNorm statistics, the barrier (which
+    // also decides, for every consumer alike, whether a wait gave up), its pools.
+    for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
         const int s = i % kCmpStages;
-        const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
-        token_stats(sk, meta[s].n_in * KP, eps, &s_stat[s][0], tid, kCmpConsumers);
-    };
-    bool bad = false;
-    if (n_t > 0) {
-        bad = !tile_ready(0);
-        if (!bad) stats_of(0);
-    }
-    bool stop = bar_or(bad);
-    for (int i = 0; !stop && i < n_t; ++i) {
-        const int s = i % kCmpStages;
-        bool bad_next = false;
-        if (i + 1 < n_t) {
-            bad_next = !tile_ready(i + 1);
-            if (!bad_next) stats_of(i + 1);
+        const bool bad = __any_sync(0xffffffffu, !mbar_wait(&full[s], (i / kCmpStages) & 1));
+        if (!bad) {
+            const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
+            token_stats(sk, meta[s].n_in * KP, eps, &s_stat[s][0], tid, kCmpConsumers);
         }
+        if (bar_or(bad)) break;
         const CmpMeta m = meta[s];
         const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
         const __nv_bfloat16 *sg = sk + kCmpTileTokens * kD;
@@ -408,7 +393,6 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
-        stop = bar_or(bad_next);
     }
 }
 
