@@ -277,31 +277,25 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                 tc::mma_commit(&ctl->p_empty[pb]);
                 tc::mma_commit(&ctl->o_done);
             };
-            // Quarter qt (8 of the 32 K-steps) of S(c) = Q K^T over chunk c's 48 tokens
-            // into S buffer c & 1; the last quarter commits s_full.
-            auto issue_s_quarter = [&](int c, int qt) {
+            // S(c) = Q K^T over chunk c's 48 tokens into S buffer c & 1.
+            auto issue_s = [&](int c) {
                 const int slot = c % kTcSlots, sb = c & 1;
-                if (qt == 0) {
-                    tc::fence_after_sync();
-                    tc::fence_proxy_async_smem();     // the slot was written by cp.async
-                }
+                tc::fence_after_sync();
+                tc::fence_proxy_async_smem();     // the slot was written by cp.async
                 const uint32_t d = tmem + 256 + sb * kTcChunk;
 #pragma unroll
-                for (int k8 = 0; k8 < 8; ++k8) {
-                    const int kk = qt * 8 + k8;
+                for (int kk = 0; kk < kL / 16; ++kk) {
                     const uint32_t qo = (kk >> 2) * 8192 + (kk & 3) * 32;
                     const uint32_t ko = (kk >> 2) * kAtomKV + slot * kSlotRows + (kk & 3) * 32;
                     tc::mma_bf16_ss(d, tc::desc_sw128(sQ + qo, 16, 1024),
                                     tc::desc_sw128(sKV + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
                 }
-                if (qt == 3) tc::mma_commit(&ctl->s_full[sb]);
+                tc::mma_commit(&ctl->s_full[sb]);
             };
             // Event loop: issue whichever product is ready, PV first (it frees a
-            // ring slot for the gathers), S a quarter at a time so a PV that becomes
-            // ready meanwhile is not queued behind a whole S; give up after the wait
-            // bound without progress.
+            // stage pair for the gathers); give up after the wait bound without progress.
             bool ok = tc_wait(ctl, &ctl->q_full, 0);
-            int ns = 0, sq = 0, np = 0;
+            int ns = 0, np = 0;
             long long t_last = clock64();
             while (ok && np < nch) {
                 if (np < ns && mbar_test(&ctl->p_full[np & 1], (np >> 1) & 1)) {
@@ -310,15 +304,10 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                     continue;
                 }
                 if (ns < nch) {
-                    const bool ready = sq > 0 ||
-                                       (mbar_test(&ctl->kv_full[ns % kTcSlots], (ns / kTcSlots) & 1) &&
-                                        (ns < 2 || mbar_test(&ctl->s_empty[ns & 1], ((ns >> 1) - 1) & 1)));
+                    const bool ready = mbar_test(&ctl->kv_full[ns % kTcSlots], (ns / kTcSlots) & 1) &&
+                                       (ns < 2 || mbar_test(&ctl->s_empty[ns & 1], ((ns >> 1) - 1) & 1));
                     if (ready) {
-                        issue_s_quarter(ns, sq);
-                        if (++sq == 4) {
-                            sq = 0;
-                            ++ns;
-                        }
+                        issue_s(ns++);
                         t_last = clock64();
                         continue;
                     }
