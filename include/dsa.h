@@ -30,10 +30,11 @@
  *     start while the kernel before it on the stream drains, and waits for
  *     that kernel (griddepcontrol.wait) before reading anything an earlier
  *     stage of this path writes. Before that wait it already reads inputs the
- *     path never writes: hidden and w (head gate); ape (kpool_compress); q_idx
- *     (index_scores); q, q_req and req_start (sparse MLA). Write those before the kernel that
- *     immediately precedes the call on the stream, or separate that kernel
- *     from the call by a copy, an event wait or a host synchronisation.
+ *     path never writes: hidden and w (head gate); ape (kpool_compress and
+ *     kpool_compress_tokens); q_idx (index_scores); q, q_req and req_start
+ *     (sparse MLA). Write those before the kernel that immediately precedes
+ *     the call on the stream, or separate that kernel from the call by a
+ *     copy, an event wait or a host synchronisation.
  *   - Request geometry lives on the device: request b owns cache rows
  *     [req_start[b], req_start[b+1]) (T_b rows). Token ids are LOGICAL, i.e.
  *     relative to the request; the physical row is req_start[b] + id ([tap]:
@@ -131,6 +132,56 @@ int dsa_kpool_compress(const dsa_bf16 *k, const dsa_bf16 *gate, const uint8_t *t
                        const float *ape, const dsa_bf16 *ln_w, const dsa_bf16 *ln_b, float eps,
                        dsa_bf16 *pool_keys, int32_t *pool_idx, uint8_t *pool_valid,
                        int32_t *first_valid, dsa_stream_t stream);
+
+/*
+ * f1. indexer_store ([mod.rs] Glm5NextDsaKernels::indexer_store: the staged
+ * indexer row is placed at a position resolved on the device and marked
+ * valid, so a captured graph replays over the live position).
+ *   k_new, gate_new bf16 [n, D]: the new tokens' indexer keys and gate logits
+ *   valid_new uint8 [n] (nonzero = valid) or NULL (every new token valid)
+ *   tok_req, tok_pos int32 [n]: request b and position t of each new token
+ *   req_start int32 [B + 1]: as for dsa_kpool_compress
+ *   For each i with 0 <= tok_req[i] < B and 0 <= tok_pos[i] < T_b, row
+ *   r = req_start[b] + tok_pos[i] gets k[r, :] = k_new[i, :],
+ *   gate[r, :] = gate_new[i, :] and tok_valid[r] = valid_new[i] != 0 (1 when
+ *   valid_new is NULL); other new tokens are skipped and nothing else is
+ *   written. Two new tokens for one row race (the caller keeps them distinct).
+ * Requires D == 128, n >= 0, B >= 0; n == 0 or B == 0 launches nothing.
+ * Alignment: k_new, gate_new, k, gate 16 bytes; tok_req, tok_pos, req_start 4.
+ */
+int dsa_indexer_store(const dsa_bf16 *k_new, const dsa_bf16 *gate_new, const uint8_t *valid_new,
+                      const int32_t *tok_req, const int32_t *tok_pos, int n, int D,
+                      const int32_t *req_start, int B, dsa_bf16 *k, dsa_bf16 *gate,
+                      uint8_t *tok_valid, dsa_stream_t stream);
+
+/*
+ * f1. kpool_compress of the pools that hold a range of new tokens (the pooled
+ * keys updated in place at the new tokens' pools instead of compressed anew:
+ * PR #290 page, the later commit that keeps KPOOL_UPDATE_DIRECT_POS in the
+ * profile; pool arithmetic as for dsa_kpool_compress).
+ *   Inputs and outputs are those of dsa_kpool_compress, plus
+ *   tok_begin, tok_end int32 [B]: request b's changed token rows are
+ *             [tok_begin[b], tok_end[b]) (clamped to [0, T_b); empty allowed).
+ *   first_valid int32 [B] is read, then written: on entry it holds f_b as
+ *   the previous compress of the request left it (any other value, e.g. -1,
+ *   asks for every pool of b). If the new f_b differs from it, every pool
+ *   row p < max_pools of b is written as dsa_kpool_compress writes it.
+ *   Otherwise exactly the pools p < max_pools that hold a changed token,
+ *   f_b + p*kpool <= tok_end[b]-1 and f_b + (p+1)*kpool - 1 >= tok_begin[b],
+ *   are; every other pool row is left untouched.
+ *   So, with req_start unchanged and every row changed since the outputs
+ *   held dsa_kpool_compress's result inside the ranges given, the outputs
+ *   hold dsa_kpool_compress's result again (byte for byte: the pooled keys
+ *   are computed in the same order).
+ * Requires D == 128, 1 <= kpool <= 8, B >= 0, max_pools >= 0. One CTA per
+ * request; its time grows with the pools it writes.
+ */
+int dsa_kpool_compress_tokens(const dsa_bf16 *k, const dsa_bf16 *gate, const uint8_t *tok_valid,
+                              const int32_t *req_start, int B, int D, int kpool, int max_pools,
+                              const float *ape, const dsa_bf16 *ln_w, const dsa_bf16 *ln_b,
+                              float eps, const int32_t *tok_begin, const int32_t *tok_end,
+                              dsa_bf16 *pool_keys, int32_t *pool_idx, uint8_t *pool_valid,
+                              int32_t *first_valid, dsa_stream_t stream);
 
 /*
  * a4. index_scores ([mod.rs] "Shape of the pipeline" second arrow:

@@ -122,6 +122,31 @@ def kpool_compress(k, gate, valid, req_start, kpool: int, max_pools: int, ape, l
     return keys, idx, pv, fv
 
 
+def indexer_store(k, gate, valid, req_start, k_new, gate_new, valid_new, tok_req, tok_pos):
+    """The indexer cache after a step's new rows are stored: copies of (k, gate, valid).
+
+    "spark_model/layers/glm5next_dsa/mod.rs", Glm5NextDsaKernels::indexer_store:
+    each staged row goes to the cache row of its request at its position, and
+    that token is marked valid. A row whose request or position falls outside
+    the cache is not stored (the plainest reading where the page says nothing
+    about them); valid_new None marks every stored token valid.
+    """
+    k, gate, valid = np.array(k, np.uint16), np.array(gate, np.uint16), np.array(valid, np.uint8)
+    req_start = np.asarray(req_start, np.int64)
+    B = req_start.shape[0] - 1
+    for i in range(len(tok_req)):
+        b, pos = int(tok_req[i]), int(tok_pos[i])
+        if not (0 <= b < B):
+            continue
+        if not (0 <= pos < req_start[b + 1] - req_start[b]):
+            continue
+        row = req_start[b] + pos
+        k[row] = k_new[i]
+        gate[row] = gate_new[i]
+        valid[row] = 1 if valid_new is None or valid_new[i] != 0 else 0
+    return k, gate, valid
+
+
 def index_scores(q_idx, gate_w, q_req, q_pos, pool_keys, pool_valid, first_valid, kpool: int,
                  threads: int = 0):
     """Returns (scores [Q,P] f32, cand [Q,P] u8)."""

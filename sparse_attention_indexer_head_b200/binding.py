@@ -25,7 +25,8 @@ DSA_ERR_CUDA = 5
 # Every symbol include/dsa.h declares.
 EXPORTS = (
     "dsa_status_string", "dsa_abi_version", "dsa_device_status", "dsa_head_gate",
-    "dsa_kpool_compress", "dsa_index_scores", "dsa_topk_expand",
+    "dsa_kpool_compress", "dsa_indexer_store", "dsa_kpool_compress_tokens",
+    "dsa_index_scores", "dsa_topk_expand",
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_launch_count", "dsa_sparse_mla_decode",
     "dsa_sparse_mla_decode_noalloc",
 )
@@ -53,6 +54,9 @@ def _load() -> ctypes.CDLL:
         "dsa_device_status": ([ctypes.POINTER(I), I], I),
         "dsa_head_gate": ([P, P, P, I, I, I, P], I),
         "dsa_kpool_compress": ([P, P, P, P, I, I, I, I, P, P, P, F, P, P, P, P, P], I),
+        "dsa_indexer_store": ([P, P, P, P, P, I, I, P, I, P, P, P, P], I),
+        "dsa_kpool_compress_tokens": ([P, P, P, P, I, I, I, I, P, P, P, F, P, P, P, P, P, P, P],
+                                      I),
         "dsa_index_scores": ([P, P, P, P, I, I, I, P, P, P, I, I, I, P, P, P], I),
         "dsa_topk_expand": ([P, P, P, P, I, I, I, I, I, P, P, P], I),
         "dsa_sparse_mla_workspace_size": ([I, I, I], Z),
@@ -118,6 +122,22 @@ def dsa_kpool_compress(k, gate, tok_valid, req_start, B: int, D: int, kpool: int
         _ptr(k), _ptr(gate), _ptr(tok_valid), _ptr(req_start), B, D, kpool, max_pools, _ptr(ape),
         _ptr(ln_w), _ptr(ln_b), float(eps), _ptr(pool_keys), _ptr(pool_idx), _ptr(pool_valid),
         _ptr(first_valid), _stream(stream)))
+
+
+def dsa_indexer_store(k_new, gate_new, valid_new, tok_req, tok_pos, n: int, D: int, req_start,
+                      B: int, k, gate, tok_valid, stream=None) -> None:
+    _check("dsa_indexer_store", lib.dsa_indexer_store(
+        _ptr(k_new), _ptr(gate_new), _ptr(valid_new), _ptr(tok_req), _ptr(tok_pos), n, D,
+        _ptr(req_start), B, _ptr(k), _ptr(gate), _ptr(tok_valid), _stream(stream)))
+
+
+def dsa_kpool_compress_tokens(k, gate, tok_valid, req_start, B: int, D: int, kpool: int,
+                              max_pools: int, ape, ln_w, ln_b, eps: float, tok_begin, tok_end,
+                              pool_keys, pool_idx, pool_valid, first_valid, stream=None) -> None:
+    _check("dsa_kpool_compress_tokens", lib.dsa_kpool_compress_tokens(
+        _ptr(k), _ptr(gate), _ptr(tok_valid), _ptr(req_start), B, D, kpool, max_pools, _ptr(ape),
+        _ptr(ln_w), _ptr(ln_b), float(eps), _ptr(tok_begin), _ptr(tok_end), _ptr(pool_keys),
+        _ptr(pool_idx), _ptr(pool_valid), _ptr(first_valid), _stream(stream)))
 
 
 def dsa_index_scores(q_idx, gate_w, q_req, q_pos, Q: int, H: int, D: int, pool_keys, pool_valid,

@@ -4,6 +4,7 @@
 #include "common.cuh"
 #include "head_gate.cuh"
 #include "kpool_compress.cuh"
+#include "indexer_store.cuh"
 #include "index_scores.cuh"
 #include "topk_expand.cuh"
 #include "sparse_mla.cuh"
@@ -83,6 +84,26 @@ int dsa_kpool_compress(const dsa_bf16 *k, const dsa_bf16 *gate, const uint8_t *t
     return dsa::kpool_compress_launch(k, gate, tok_valid, req_start, B, D, kpool, max_pools, ape,
                                       ln_w, ln_b, eps, pool_keys, pool_idx, pool_valid,
                                       first_valid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dsa_indexer_store(const dsa_bf16 *k_new, const dsa_bf16 *gate_new, const uint8_t *valid_new,
+                      const int32_t *tok_req, const int32_t *tok_pos, int n, int D,
+                      const int32_t *req_start, int B, dsa_bf16 *k, dsa_bf16 *gate,
+                      uint8_t *tok_valid, dsa_stream_t stream) {
+    return dsa::indexer_store_launch(k_new, gate_new, valid_new, tok_req, tok_pos, n, D, req_start,
+                                     B, k, gate, tok_valid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dsa_kpool_compress_tokens(const dsa_bf16 *k, const dsa_bf16 *gate, const uint8_t *tok_valid,
+                              const int32_t *req_start, int B, int D, int kpool, int max_pools,
+                              const float *ape, const dsa_bf16 *ln_w, const dsa_bf16 *ln_b,
+                              float eps, const int32_t *tok_begin, const int32_t *tok_end,
+                              dsa_bf16 *pool_keys, int32_t *pool_idx, uint8_t *pool_valid,
+                              int32_t *first_valid, dsa_stream_t stream) {
+    return dsa::kpool_compress_tokens_launch(k, gate, tok_valid, req_start, B, D, kpool, max_pools,
+                                             ape, ln_w, ln_b, eps, tok_begin, tok_end, pool_keys,
+                                             pool_idx, pool_valid, first_valid,
+                                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dsa_index_scores(const dsa_bf16 *q_idx, const float *gate_w, const int32_t *q_req,

@@ -126,6 +126,68 @@ class DecodeStep:
         self.topk_expand(stream)
         self.sparse_mla(stream)
 
+    # -- incremental decode: the step's new token rows update the pooled-key cache -------
+    def stage_new_tokens(self, k_new=None, gate_new=None, valid_new=None, tok_req=None,
+                         tok_pos=None):
+        """Device buffers of a step's new indexer rows and the token ranges they change.
+
+        Default: one new token per request, its last row (position T_b - 1), with
+        the k and gate values the cache already holds there, so a step that
+        stores it leaves the cache as it was and its outputs can be compared
+        with the full step's. Requests with no rows get none.
+        """
+        g, t, dev = self.g, self.t, self.device
+        rs = t["req_start"].to("cpu").numpy().astype(np.int64)
+        lengths = rs[1:] - rs[:-1]
+        if tok_req is None:
+            have = np.nonzero(lengths > 0)[0]
+            tok_req = have.astype(np.int32)
+            tok_pos = (lengths[have] - 1).astype(np.int32)
+            rows = torch.from_numpy(rs[have] + tok_pos).to(dev)
+            k_new = t["k"].index_select(0, rows)
+            gate_new = t["gate"].index_select(0, rows)
+            valid_new = t["valid"].index_select(0, rows)
+        tok_req = np.asarray(tok_req, np.int32)
+        tok_pos = np.asarray(tok_pos, np.int32)
+        begin = np.full(g.B, 0, np.int32)
+        end = np.full(g.B, 0, np.int32)
+        for b in range(g.B):                   # the smallest range holding b's new rows
+            mine = tok_pos[tok_req == b]
+            if mine.size:
+                begin[b], end[b] = mine.min(), mine.max() + 1
+        self.new = {
+            "k": torch.as_tensor(k_new).to(dev), "gate": torch.as_tensor(gate_new).to(dev),
+            "valid": None if valid_new is None else torch.as_tensor(valid_new).to(dev),
+            "tok_req": torch.from_numpy(tok_req).to(dev), "tok_pos": torch.from_numpy(tok_pos).to(dev),
+            "n": int(tok_req.shape[0]),
+            "tok_begin": torch.from_numpy(begin).to(dev), "tok_end": torch.from_numpy(end).to(dev),
+        }
+
+    def indexer_store(self, stream=None):
+        g, t, n = self.g, self.t, self.new
+        B.dsa_indexer_store(n["k"], n["gate"], n["valid"], n["tok_req"], n["tok_pos"], n["n"],
+                            INDEX_DIM, t["req_start"], g.B, t["k"], t["gate"], t["valid"], stream)
+
+    def kpool_compress_tokens(self, stream=None):
+        g, t, n = self.g, self.t, self.new
+        B.dsa_kpool_compress_tokens(t["k"], t["gate"], t["valid"], t["req_start"], g.B, INDEX_DIM,
+                                    g.kpool, g.max_pools, t["ape"], t["ln_w"], t["ln_b"], g.eps,
+                                    n["tok_begin"], n["tok_end"], self.pool_keys, self.pool_idx,
+                                    self.pool_valid, self.first_valid, stream)
+
+    def run_incremental(self, stream=None):
+        """A decode step that stores the new rows and recomputes only their pools.
+
+        The pooled-key outputs must already hold the compress result of the
+        cache before the new rows (run() or kpool_compress() once).
+        """
+        self.indexer_store(stream)
+        self.kpool_compress_tokens(stream)
+        self.head_gate(stream)
+        self.index_scores(stream)
+        self.topk_expand(stream)
+        self.sparse_mla(stream)
+
     def kernels_per_step(self) -> int:
         """Launches of run(): gate, compress, scores, topk+expand, and the MLA's one or
         two kernels (split kernel, plus the combine when splits merge in the workspace)."""

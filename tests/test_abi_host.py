@@ -79,6 +79,52 @@ def test_kpool_compress_refusals(B):
     assert _compress(B, B=0) == B.DSA_OK
 
 
+def test_indexer_store_refusals(B):
+    L = B.lib
+    args = [FAKE, FAKE, None, FAKE, FAKE, 8, 128, FAKE, 2, FAKE, FAKE, FAKE, None]
+    bad = list(args); bad[6] = 64
+    assert L.dsa_indexer_store(*bad) == B.DSA_ERR_UNSUPPORTED        # D is the indexer dim 128
+    bad = list(args); bad[5] = -1
+    assert L.dsa_indexer_store(*bad) == B.DSA_ERR_INVALID_ARG
+    bad = list(args); bad[0] = None
+    assert L.dsa_indexer_store(*bad) == B.DSA_ERR_INVALID_ARG
+    bad = list(args); bad[9] = None
+    assert L.dsa_indexer_store(*bad) == B.DSA_ERR_INVALID_ARG       # no destination cache
+    bad = list(args); bad[1] = FAKE + 4
+    assert L.dsa_indexer_store(*bad) == B.DSA_ERR_ALIGNMENT
+    bad = list(args); bad[3] = FAKE + 2
+    assert L.dsa_indexer_store(*bad) == B.DSA_ERR_ALIGNMENT
+    bad = list(args); bad[5] = 0
+    assert L.dsa_indexer_store(*bad) == B.DSA_OK                     # nothing to store
+    bad = list(args); bad[8] = 0; bad[7] = None; bad[9] = bad[10] = bad[11] = None
+    assert L.dsa_indexer_store(*bad) == B.DSA_OK                     # no request to store into
+
+
+def _compress_tokens(lib, **kw):
+    a = dict(k=FAKE, gate=FAKE, valid=FAKE, req_start=FAKE, B=2, D=128, kpool=4, max_pools=8,
+             ape=FAKE, ln_w=FAKE, ln_b=FAKE, eps=1e-5, tb=FAKE, te=FAKE, keys=FAKE, idx=FAKE,
+             pv=FAKE, fv=FAKE)
+    a.update(kw)
+    return lib.lib.dsa_kpool_compress_tokens(
+        a["k"], a["gate"], a["valid"], a["req_start"], a["B"], a["D"], a["kpool"], a["max_pools"],
+        a["ape"], a["ln_w"], a["ln_b"], a["eps"], a["tb"], a["te"], a["keys"], a["idx"], a["pv"],
+        a["fv"], None)
+
+
+def test_kpool_compress_tokens_refusals(B):
+    assert _compress_tokens(B, kpool=9) == B.DSA_ERR_UNSUPPORTED
+    assert _compress_tokens(B, kpool=0) == B.DSA_ERR_INVALID_ARG
+    assert _compress_tokens(B, D=256) == B.DSA_ERR_UNSUPPORTED
+    assert _compress_tokens(B, tb=None) == B.DSA_ERR_INVALID_ARG
+    assert _compress_tokens(B, te=None) == B.DSA_ERR_INVALID_ARG
+    assert _compress_tokens(B, fv=None) == B.DSA_ERR_INVALID_ARG
+    assert _compress_tokens(B, keys=None) == B.DSA_ERR_INVALID_ARG
+    assert _compress_tokens(B, te=FAKE + 1) == B.DSA_ERR_ALIGNMENT
+    assert _compress_tokens(B, eps=float("inf")) == B.DSA_ERR_INVALID_ARG
+    assert _compress_tokens(B, max_pools=-1) == B.DSA_ERR_INVALID_ARG
+    assert _compress_tokens(B, B=0) == B.DSA_OK
+
+
 def test_index_scores_refusals(B):
     L = B.lib
     args = [FAKE, FAKE, FAKE, FAKE, 4, 16, 128, FAKE, FAKE, FAKE, 4, 4, 64, FAKE, FAKE, None]

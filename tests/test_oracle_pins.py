@@ -487,3 +487,58 @@ def test_mla_physical_rows_are_request_relative(orc):
     rs = np.array([0, 10, 20], np.int32)
     out, _ = orc.sparse_mla(q, kv, rs, np.array([1], np.int32), np.array([[4]], np.int32), 0.1)
     np.testing.assert_array_equal(out[0, 0], kv[14])
+
+
+def test_indexer_store_places_rows_by_request_and_position(orc):
+    """Stored rows land at req_start[b] + pos, marked valid; out-of-range rows are dropped."""
+    req_start = np.array([0, 3, 3, 7], np.int32)          # request 1 is empty
+    k = np.zeros((7, 2), np.uint16)
+    gate = np.zeros((7, 2), np.uint16)
+    valid = np.zeros(7, np.uint8)
+    k_new = np.array([[1, 2], [3, 4], [5, 6], [7, 8], [9, 10]], np.uint16)
+    g_new = k_new + 100
+    tok_req = np.array([0, 2, 1, 2, 3])                  # request 1 has no row 0; request 3 is none
+    tok_pos = np.array([2, 0, 0, 4, 0])                  # position 4 is past request 2's 4 rows
+    k2, g2, v2 = orc.indexer_store(k, gate, valid, req_start, k_new, g_new, None, tok_req, tok_pos)
+    want_k = np.zeros((7, 2), np.uint16)
+    want_k[2] = [1, 2]
+    want_k[3] = [3, 4]
+    np.testing.assert_array_equal(k2, want_k)
+    np.testing.assert_array_equal(g2[[2, 3]], [[101, 102], [103, 104]])
+    assert g2[[0, 1, 4, 5, 6]].sum() == 0
+    np.testing.assert_array_equal(v2, [0, 0, 1, 1, 0, 0, 0])
+    assert valid.sum() == 0 and k.sum() == 0               # inputs are not modified
+    # an explicit validity byte is stored as given (nonzero -> 1)
+    _, _, v3 = orc.indexer_store(k, gate, np.ones(7, np.uint8), req_start, k_new[:2], g_new[:2],
+                                 np.array([0, 7], np.uint8), tok_req[:2], tok_pos[:2])
+    np.testing.assert_array_equal(v3, [1, 1, 0, 1, 1, 1, 1])
+
+
+def test_compress_after_store_only_changes_pools_of_new_tokens(orc):
+    """Appending tokens to a capacity-sized request changes only the pools that hold them.
+
+    This is what lets the incremental update recompute those pools alone
+    (pooled keys of a pool depend only on its own kpool token rows, given f_b).
+    """
+    rng = np.random.default_rng(11)
+    kp, cap = 4, 40
+    req_start = np.array([0, cap], np.int32)
+    k = rng.integers(0x3C00, 0x4000, size=(cap, 128)).astype(np.uint16)     # bf16 values in [1, 2)
+    gate = rng.integers(0x3C00, 0x4000, size=(cap, 128)).astype(np.uint16)
+    valid = np.zeros(cap, np.uint8)
+    valid[3:21] = 1                                        # f = 3, tokens 3..20 present
+    ape = rng.standard_normal((kp, 128)).astype(np.float32) * np.float32(0.02)
+    ln_w = np.full(128, 0x3F80, np.uint16)
+    ln_b = np.zeros(128, np.uint16)
+    before = orc.kpool_compress(k, gate, valid, req_start, kp, 10, ape, ln_w, ln_b, 1e-5)
+    k2, g2, v2 = orc.indexer_store(k, gate, valid, req_start, k[21:24] ^ 1, gate[21:24], None,
+                                   [0, 0, 0], [21, 22, 23])
+    after = orc.kpool_compress(k2, g2, v2, req_start, kp, 10, ape, ln_w, ln_b, 1e-5)
+    assert before[3][0] == after[3][0] == 3
+    # pools 0..3 (tokens 3..18) unchanged; pool 4 (tokens 19..22) and 5 (23..26) hold new tokens
+    for a, b in zip(before[:3], after[:3]):
+        np.testing.assert_array_equal(a[0, :4], b[0, :4])
+        np.testing.assert_array_equal(a[0, 6:], b[0, 6:])
+    assert before[2][0, 4] == 0 and after[2][0, 4] == 1    # pool 4 complete now
+    assert after[2][0, 5] == 0                             # pool 5 still lacks tokens 24..26
+    assert not np.array_equal(before[0][0, 4], after[0][0, 4])
