@@ -333,6 +333,60 @@ def gpu_arm(args, wl_fn):
                                    for r in range(n_rep))
                 for i, n in enumerate(names)}
 
+    # ---- incremental decode step: the cache update stores each request's new
+    # indexer row and recomputes only the pools holding it, in place of the full
+    # compress (the pooled keys already hold the compress result of the cache).
+    for s in steps:
+        s.stage_new_tokens()
+    with torch.cuda.stream(stream):
+        for s in steps:
+            s.run_incremental(stream)
+    stream.synchronize()
+    inc_graphs = []
+    for s in steps:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            s.run_incremental()
+        inc_graphs.append(g)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            inc_graphs[i % len(inc_graphs)].replay()
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(2_000_000)
+        ev0.record(stream)
+        for i in range(args.steps):
+            inc_graphs[i % len(inc_graphs)].replay()
+        ev1.record(stream)
+    stream.synchronize()
+    barrier(world)
+    inc_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    inc_names = ["indexer_store", "kpool_compress_tokens"]
+    inc_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_rep)]
+    with torch.cuda.stream(stream):
+        for r in range(n_rep):
+            s = steps[r % len(steps)]
+            for i, n in enumerate(inc_names):
+                torch.cuda._sleep(200_000)
+                inc_evs[r][2 * i].record(stream)
+                getattr(s, n)(stream)
+                inc_evs[r][2 * i + 1].record(stream)
+    stream.synchronize()
+    inc_stage_us = {n: 1e3 * statistics.mean(inc_evs[r][2 * i].elapsed_time(inc_evs[r][2 * i + 1])
+                                             for r in range(n_rep))
+                    for i, n in enumerate(inc_names)}
+    incremental = {
+        "value": replica_throughput(wl.Q, world, args.steps, inc_ms / 1e3), "unit": "queries/s",
+        "ms_per_step": inc_ms / args.steps, "steps": args.steps,
+        "gpu_launches": steps[0].kernels_per_step_incremental() * args.steps,
+        "stage_us": inc_stage_us, "new_rows_per_step": steps[0].new["n"],
+        "path": "dsa_indexer_store of each request's new row -> dsa_kpool_compress_tokens "
+                "over its pools -> gate, scores, top-k, MLA as in the step above",
+    }
+    del inc_graphs
+
     # ---- end to end through the public API with host buffers
     pinned_in = {k: host[k].pin_memory() for k in QUERY_INPUTS}
     s0 = steps[0]
@@ -405,6 +459,7 @@ def gpu_arm(args, wl_fn):
                 "path": "pinned host query inputs -> H2D -> 5 ABI calls -> D2H of out, "
                         "synchronised each step"},
         "gpu_launches": steps[0].kernels_per_step() * args.steps,
+        "incremental": incremental,
         "clocks": clk,
         "device_error": B.dsa_device_status(reset=True),
     }

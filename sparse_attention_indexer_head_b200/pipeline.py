@@ -194,6 +194,12 @@ class DecodeStep:
         g = self.g
         return 4 + B.dsa_sparse_mla_launch_count(g.Q, g.hm, g.W)
 
+    def kernels_per_step_incremental(self) -> int:
+        """Launches of run_incremental(): store (when there are new rows), token-range
+        compress, gate, scores, topk+expand and the MLA's kernels."""
+        g = self.g
+        return (1 if self.new["n"] > 0 else 0) + 4 + B.dsa_sparse_mla_launch_count(g.Q, g.hm, g.W)
+
     def outputs_numpy(self) -> Dict[str, np.ndarray]:
         def u16(x):
             return x.view(torch.int16).cpu().numpy().view(np.uint16)
