@@ -456,7 +456,7 @@ kpool_compress_tokens_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfl
     __shared__ __align__(16) float s_ape[KP * kD];         // ape * log2(e), [slot][half][lane][4]
     __shared__ __align__(16) __nv_bfloat16 s_rows[kHW][2][KP][kD];   // per half-warp: k rows, gate rows
     __shared__ __align__(16) float2 s_st[kHW][KP];         // per half-warp: (rstd, -mu * rstd)
-    __shared__ int s_f, s_all;
+    __shared__ int s_f, s_fold, s_tb, s_te;
 
     const int b = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -475,20 +475,20 @@ kpool_compress_tokens_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfl
     const int T = max(0, req_start[b + 1] - rs);
     if (warp == 0) {
         const int f = first_valid_scan(valid, rs, T);
-        if (lane == 0) {
-            // a first valid token that moved shifts every pool: recompute them all
-            s_all = first_valid[b] != f;
-            s_f = f;
-            first_valid[b] = f;
-        }
+        if (lane == 0) s_f = f;
+    } else if (tid == 32) {        // the request's range and previous first valid token, meanwhile
+        s_tb = tok_begin[b];
+        s_te = tok_end[b];
+        s_fold = first_valid[b];
     }
     __syncthreads();
     const int f = s_f;
+    if (tid == 0) first_valid[b] = f;
     if (max_pools <= 0) return;
     const int n_span = min(max_pools, (T - f) / KP);
     int p_lo = 0, p_hi = max_pools - 1;
-    if (!s_all) {
-        const int tb = max(tok_begin[b], 0), te = min(tok_end[b], T);
+    if (s_fold == f) {             // a first valid token that moved shifts every pool: all of them
+        const int tb = max(s_tb, 0), te = min(s_te, T);
         if (te <= tb || te - 1 < f) return;      // no pool holds the range
         p_lo = tb > f ? (tb - f) / KP : 0;
         p_hi = min(max_pools - 1, (te - 1 - f) / KP);
