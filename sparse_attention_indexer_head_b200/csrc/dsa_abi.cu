@@ -4,6 +4,7 @@
 #include "common.cuh"
 #include "head_gate.cuh"
 #include "kpool_compress.cuh"
+#include "kpool_compress_tokens.cuh"
 #include "indexer_store.cuh"
 #include "index_scores.cuh"
 #include "topk_expand.cuh"

@@ -85,6 +85,7 @@ struct TcCtl {
     float lsum[kTcHeads];
     float mfin[kTcHeads];
     uint32_t tmem_base;
+    int have_o;                           // the epilogue reads O^T (set by the softmax warps)
     volatile int abort;
 };
 constexpr int kTcSmemBytes = (int)kOffCtl + (int)sizeof(TcCtl) + 1024;   // + alignment slack
@@ -513,48 +514,11 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                                      : "memory");
                 }
             }
-        } else if (S > 1) {
-            float *pb = part + ((size_t)(qi * S + split) * Hm + h0) * kPartStride;
-            if (have_o) {
-                tc::fence_after_sync();
-#pragma unroll 1
-                for (int blk = 0; blk < 8; ++blk) {
-                    uint32_t o[32];
-                    tc::tmem_ld32(tl + (blk >> 1) * 64 + (blk & 1) * 32, o);
-                    tc::tmem_wait_ld();
-                    const int L = (blk >> 1) * 128 + 32 * wq + lane;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int h = (blk & 1) * 32 + j;
-                        if (h < nh) pb[(size_t)h * kPartStride + L] = __uint_as_float(o[j]);
-                    }
-                }
-            }
-            if (owner && hh < nh) {
-                pb[(size_t)hh * kPartStride + kL] = have_o ? m_used : -INFINITY;
-                pb[(size_t)hh * kPartStride + kL + 1] = have_o ? l : 0.f;
-            }
         } else {
-            // single split: normalise here and write bf16 out and lse directly
-            __nv_bfloat16 *ob = out + ((size_t)qi * Hm + h0) * kL;
-            if (have_o) tc::fence_after_sync();
-#pragma unroll 1
-            for (int blk = 0; blk < 8; ++blk) {
-                uint32_t o[32];
-                if (have_o) {
-                    tc::tmem_ld32(tl + (blk >> 1) * 64 + (blk & 1) * 32, o);
-                    tc::tmem_wait_ld();
-                }
-                const int L = (blk >> 1) * 128 + 32 * wq + lane;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int h = (blk & 1) * 32 + j;
-                    const float lh = ctl->lsum[h];
-                    const float v = (have_o && lh > 0.f) ? __uint_as_float(o[j]) / lh : 0.f;
-                    if (h < nh) ob[(size_t)h * kL + L] = __float2bfloat16_rn(v);
-                }
-            }
-            if (lse && owner && hh < nh)
+            // O^T is written after the CTA barrier below, by all sixteen warps.
+            if (owner) ctl->mfin[hh] = have_o ? m_used : -INFINITY;
+            if (tid == 128) ctl->have_o = have_o ? 1 : 0;
+            if (S == 1 && lse && owner && hh < nh)
                 lse[(size_t)qi * Hm + h0 + hh] =
                     (have_o && l > 0.f) ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
         }
@@ -568,6 +532,59 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    if constexpr (!kCluster) {
+        // O^T out of tensor memory by all sixteen warps: warp w reads the lane
+        // quarter w % 4 (32 latent rows of each 128-row block) for two of the
+        // eight (latent block, 32-head half) pieces; each store writes 32
+        // consecutive latent values of one head (128 bytes).
+        const int quarter = warp & 3;
+        const uint32_t tq = tmem + ((uint32_t)(32 * quarter) << 16);
+        const bool have_o = ctl->have_o != 0;
+        if (S > 1) {
+            float *pb = part + ((size_t)(qi * S + split) * Hm + h0) * kPartStride;
+            if (have_o) {
+#pragma unroll 1
+                for (int bi = 0; bi < 2; ++bi) {
+                    const int blk = 2 * (warp >> 2) + bi;
+                    uint32_t o[32];
+                    tc::tmem_ld32(tq + (blk >> 1) * 64 + (blk & 1) * 32, o);
+                    tc::tmem_wait_ld();
+                    const int L = (blk >> 1) * 128 + 32 * quarter + lane;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int h = (blk & 1) * 32 + j;
+                        if (h < nh) pb[(size_t)h * kPartStride + L] = __uint_as_float(o[j]);
+                    }
+                }
+            }
+            if (tid < kTcHeads && tid < nh) {
+                pb[(size_t)tid * kPartStride + kL] = ctl->mfin[tid];
+                pb[(size_t)tid * kPartStride + kL + 1] = have_o ? ctl->lsum[tid] : 0.f;
+            }
+        } else {
+            // single split: normalise here and write bf16 out directly
+            __nv_bfloat16 *ob = out + ((size_t)qi * Hm + h0) * kL;
+#pragma unroll 1
+            for (int bi = 0; bi < 2; ++bi) {
+                const int blk = 2 * (warp >> 2) + bi;
+                uint32_t o[32];
+                if (have_o) {
+                    tc::tmem_ld32(tq + (blk >> 1) * 64 + (blk & 1) * 32, o);
+                    tc::tmem_wait_ld();
+                }
+                const int L = (blk >> 1) * 128 + 32 * quarter + lane;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int h = (blk & 1) * 32 + j;
+                    const float lh = ctl->lsum[h];
+                    const float v = (have_o && lh > 0.f) ? __uint_as_float(o[j]) / lh : 0.f;
+                    if (h < nh) ob[(size_t)h * kL + L] = __float2bfloat16_rn(v);
+                }
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();              // every tensor-memory read is done before the release
+    }
     if constexpr (kCluster) {
         cluster_sync_all();           // every split's m, l and O^T are in place
         if (tid < 256)

@@ -4,8 +4,10 @@
 // sentinel row written in full).
 //
 // One CTA per query. Scores become order-preserving uint32 keys (candidates
-// only; -0 folded onto +0, NaN onto -inf, non-candidates 0). A 4-pass 8-bit
-// MSB radix select finds the n_q-th largest key tau exactly; the winners are
+// only; -0 folded onto +0, NaN onto -inf, non-candidates 0). An 8-bit MSB
+// radix select finds the n_q-th largest key tau exactly: two passes, then,
+// when at most 32 keys share those 16 bits with tau, a rank among them on one
+// warp, else two more passes; the winners are
 // every key above tau plus the lowest-id keys equal to tau (an id-ordered
 // block scan), written in ascending pool id, so the result is bit-exact and
 // deterministic. The expansion gathers pool_idx rows and writes every slot of
@@ -67,8 +69,9 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     uint32_t *skeys = reinterpret_cast<uint32_t *>(topk_smem) + K;           // [P] if cached
     __shared__ int hist[2][256];          // double-buffered radix histograms
     __shared__ int2 s_warp2[kTopkWarps];
-    __shared__ int s_pick[2][2];          // per pass parity: (digit, count above it)
-    __shared__ int s_ncand;
+    __shared__ int s_pick[2][3];          // per pass parity: (digit, count above it, count in it)
+    __shared__ int s_ncand, s_nsmall, s_req;
+    __shared__ uint32_t s_small[32], s_tau;
 
     const int tid = threadIdx.x;
     const int q = blockIdx.x;
@@ -91,7 +94,10 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
         hist[0][tid] = 0;
         hist[1][tid] = 0;
     }
-    if (tid == 0) s_ncand = 0;
+    if (tid == 0) {
+        s_ncand = 0;
+        s_nsmall = 0;
+    }
     __syncthreads();
     int cnt = 0;
     for (int p0 = 0; p0 < P; p0 += 4 * kTopkThreads) {
@@ -172,6 +178,7 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
                     if (run < remaining && remaining <= run + c[i]) {
                         s_pick[hb][0] = 255 - 8 * tid - i;
                         s_pick[hb][1] = run;
+                        s_pick[hb][2] = c[i];
                     }
                     run += c[i];
                 }
@@ -180,6 +187,44 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
             remaining -= s_pick[hb][1];
             prefix |= (uint32_t)s_pick[hb][0] << shift;
             pmask |= 0xFFu << shift;
+            if (pass == 1 && s_pick[hb][2] <= 32) {
+                // At most 32 keys share the top 16 bits of the answer (the usual
+                // case: keys of similar magnitude differ from the second byte on).
+                // Gather them and rank them on one warp instead of two more passes.
+                const int lane = tid & 31;
+                for (int base = (tid & ~31); base < P; base += kTopkThreads) {
+                    const int p = base + lane;
+                    const uint32_t k = p < P ? key_at(p) : 0u;
+                    const bool m = p < P && (k & pmask) == prefix;
+                    const uint32_t bal = __ballot_sync(0xffffffffu, m);
+                    if (bal) {
+                        int off = 0;
+                        if (lane == 0) off = atomicAdd(&s_nsmall, __popc(bal));
+                        off = __shfl_sync(0xffffffffu, off, 0);
+                        if (m) s_small[off + __popc(bal & ((1u << lane) - 1u))] = k;
+                    }
+                }
+                __syncthreads();
+                if (tid < 32) {
+                    const int n = s_nsmall;            // the bin's count, <= 32
+                    const uint32_t mine = tid < n ? s_small[tid] : 0u;
+                    int gt = 0, ge = 0;
+                    for (int j = 0; j < n; ++j) {
+                        const uint32_t kj = s_small[j];
+                        gt += kj > mine;
+                        ge += kj >= mine;
+                    }
+                    // the remaining-th largest of the bin (equal keys write equal values)
+                    if (tid < n && gt < remaining && remaining <= ge) {
+                        s_tau = mine;
+                        s_req = remaining - gt;
+                    }
+                }
+                __syncthreads();
+                prefix = s_tau;
+                remaining = s_req;
+                break;
+            }
         }
     }
     const uint32_t tau = prefix;   // the nq-th largest key (when nq > 0)
