@@ -221,6 +221,29 @@ int dsa_topk_expand(const float *scores, const uint8_t *cand, const int32_t *poo
                     int32_t *top_pools, int32_t *token_ids, dsa_stream_t stream);
 
 /*
+ * f4. topk_pools + expand_selection with always_select_tail ([mod.rs]
+ * Glm5NextDsaConfig::out_width: the tail adds kpool - 1 slots to the index
+ * row; the step tap's idx.tail_slot).
+ *   As dsa_topk_expand, but token_ids rows are out_width = select_k * kpool +
+ *   kpool - 1 wide: the first select_k * kpool slots as dsa_topk_expand writes
+ *   them, then kpool - 1 tail slots for the query's trailing partial pool.
+ *   With f = first_valid[b] and n = (q_pos[q] - f + 1) mod kpool (the tokens
+ *   after the query's last complete pool), tail slot s holds the logical id
+ *   q_pos[q] + 1 - n + s when s < n, that token is < T_b and tok_valid marks it
+ *   valid; every other tail slot is -1 (all of them when q_pos[q] < f or the
+ *   query's request is out of range). Those tokens are in no selectable pool
+ *   (the pool holding them ends after q_pos), so the row has no duplicates.
+ *   q_pos int32 [Q]; first_valid int32 [B] (as written by dsa_kpool_compress);
+ *   tok_valid uint8 [total_tokens]; req_start int32 [B + 1].
+ * Requires what dsa_topk_expand requires; select_k == 0 writes the tail only.
+ */
+int dsa_topk_expand_tail(const float *scores, const uint8_t *cand, const int32_t *pool_idx,
+                         const int32_t *q_req, const int32_t *q_pos, const int32_t *first_valid,
+                         const uint8_t *tok_valid, const int32_t *req_start, int Q, int B,
+                         int max_pools, int kpool, int select_k, int32_t *top_pools,
+                         int32_t *token_ids, dsa_stream_t stream);
+
+/*
  * a7. NoPE MLA restricted to the selected tokens ([mod.rs] "Shape of the
  * pipeline" last arrow; MASKED_ATTN_MAX_KEYS doc: set-membership mask, so a
  * per-row gather is exact; trap 5: qk_rope_head_dim == 0, the 512-wide latent

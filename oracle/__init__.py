@@ -185,6 +185,36 @@ def topk_expand(scores, cand, pool_idx, q_req, select_k: int, threads: int = 0):
     return top, ids
 
 
+def tail_slots(q_req, q_pos, first_valid, valid, req_start, kpool: int) -> np.ndarray:
+    """The kpool - 1 tail slots of each query's index row under always_select_tail.
+
+    "spark_model/layers/glm5next_dsa/mod.rs", Glm5NextDsaConfig::out_width: the
+    tail adds kpool - 1 slots to the row (the step tap names them idx.tail_slot).
+    Reading: they hold the query's trailing partial pool -- the tokens after its
+    last complete pool up to and including q_pos, counted on the pool grid that
+    starts at the request's first valid token -- in position order, a token that
+    is missing or not valid as -1, and -1 past them.
+    """
+    req_start = np.asarray(req_start, np.int64)
+    B = req_start.shape[0] - 1
+    Q = len(q_req)
+    out = np.full((Q, max(kpool - 1, 0)), -1, dtype=np.int32)
+    for q in range(Q):
+        b = int(q_req[q])
+        if not (0 <= b < B):
+            continue
+        f, qp = int(first_valid[b]), int(q_pos[q])
+        T = int(req_start[b + 1] - req_start[b])
+        if qp < f:
+            continue
+        n_tail = (qp - f + 1) % kpool          # tokens past the last complete pool
+        for s in range(n_tail):
+            t = qp + 1 - n_tail + s
+            if 0 <= t < T and valid[req_start[b] + t] != 0:
+                out[q, s] = t
+    return out
+
+
 def sparse_mla(q, kv, req_start, q_req, token_ids, sm_scale: float, threads: int = 0):
     """Returns (out [Q,Hm,L] u16 bf16 bits, lse [Q,Hm] f32)."""
     q = _c(q, np.uint16)

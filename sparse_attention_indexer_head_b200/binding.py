@@ -26,7 +26,7 @@ DSA_ERR_CUDA = 5
 EXPORTS = (
     "dsa_status_string", "dsa_abi_version", "dsa_device_status", "dsa_head_gate",
     "dsa_kpool_compress", "dsa_indexer_store", "dsa_kpool_compress_tokens",
-    "dsa_index_scores", "dsa_topk_expand",
+    "dsa_index_scores", "dsa_topk_expand", "dsa_topk_expand_tail",
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_launch_count", "dsa_sparse_mla_decode",
     "dsa_sparse_mla_decode_noalloc",
 )
@@ -59,6 +59,7 @@ def _load() -> ctypes.CDLL:
                                       I),
         "dsa_index_scores": ([P, P, P, P, I, I, I, P, P, P, I, I, I, P, P, P], I),
         "dsa_topk_expand": ([P, P, P, P, I, I, I, I, I, P, P, P], I),
+        "dsa_topk_expand_tail": ([P, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P], I),
         "dsa_sparse_mla_workspace_size": ([I, I, I], Z),
         "dsa_sparse_mla_launch_count": ([I, I, I], I),
         "dsa_sparse_mla_decode": ([P, P, I64, P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P], I),
@@ -154,6 +155,15 @@ def dsa_topk_expand(scores, cand, pool_idx, q_req, Q: int, B: int, max_pools: in
     _check("dsa_topk_expand", lib.dsa_topk_expand(
         _ptr(scores), _ptr(cand), _ptr(pool_idx), _ptr(q_req), Q, B, max_pools, kpool, select_k,
         _ptr(top_pools), _ptr(token_ids), _stream(stream)))
+
+
+def dsa_topk_expand_tail(scores, cand, pool_idx, q_req, q_pos, first_valid, tok_valid, req_start,
+                         Q: int, B: int, max_pools: int, kpool: int, select_k: int, top_pools,
+                         token_ids, stream=None) -> None:
+    _check("dsa_topk_expand_tail", lib.dsa_topk_expand_tail(
+        _ptr(scores), _ptr(cand), _ptr(pool_idx), _ptr(q_req), _ptr(q_pos), _ptr(first_valid),
+        _ptr(tok_valid), _ptr(req_start), Q, B, max_pools, kpool, select_k, _ptr(top_pools),
+        _ptr(token_ids), _stream(stream)))
 
 
 def dsa_sparse_mla_workspace_size(Q: int, Hm: int, W: int) -> int:

@@ -119,8 +119,21 @@ int dsa_index_scores(const dsa_bf16 *q_idx, const float *gate_w, const int32_t *
 int dsa_topk_expand(const float *scores, const uint8_t *cand, const int32_t *pool_idx,
                     const int32_t *q_req, int Q, int B, int max_pools, int kpool, int select_k,
                     int32_t *top_pools, int32_t *token_ids, dsa_stream_t stream) {
+    const dsa::TailArgs no_tail{nullptr, nullptr, nullptr, nullptr, 0};
     return dsa::topk_expand_launch(scores, cand, pool_idx, q_req, Q, B, max_pools, kpool,
-                                   select_k, top_pools, token_ids,
+                                   select_k, no_tail, top_pools, token_ids,
+                                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dsa_topk_expand_tail(const float *scores, const uint8_t *cand, const int32_t *pool_idx,
+                         const int32_t *q_req, const int32_t *q_pos, const int32_t *first_valid,
+                         const uint8_t *tok_valid, const int32_t *req_start, int Q, int B,
+                         int max_pools, int kpool, int select_k, int32_t *top_pools,
+                         int32_t *token_ids, dsa_stream_t stream) {
+    if (kpool <= 0) return DSA_ERR_INVALID_ARG;
+    const dsa::TailArgs tail{q_pos, first_valid, tok_valid, req_start, kpool - 1};
+    return dsa::topk_expand_launch(scores, cand, pool_idx, q_req, Q, B, max_pools, kpool,
+                                   select_k, tail, top_pools, token_ids,
                                    reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -59,10 +59,23 @@ DSA_DEVINL int2 block_excl_scan2(int a, int b, int2 *s_warp2, int *ta, int *tb) 
     return make_int2(before.x + x - a, before.y + y - b);
 }
 
+// Tail slots (always_select_tail): after the K * KP pool slots, a row carries
+// KP - 1 slots for the query's trailing partial pool. With f the request's first
+// valid token and n = (q_pos - f + 1) mod KP tokens past the query's last
+// complete pool, slot s < n holds token q_pos + 1 - n + s when it exists and is
+// valid; every other tail slot is -1 (also when q_pos < f).
+struct TailArgs {
+    const int32_t *q_pos;
+    const int32_t *first_valid;
+    const uint8_t *valid;
+    const int32_t *req_start;
+    int slots;              // 0 (no tail) or KP - 1
+};
+
 __global__ void __launch_bounds__(kTopkThreads)
 topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__ cand,
                    const int32_t *__restrict__ pool_idx, const int32_t *__restrict__ q_req, int B,
-                   int P, int KP, int K, int keys_in_smem,
+                   int P, int KP, int K, int keys_in_smem, TailArgs tail,
                    int32_t *__restrict__ top_pools, int32_t *__restrict__ token_ids) {
     extern __shared__ __align__(16) uint8_t topk_smem[];
     int32_t *slist = reinterpret_cast<int32_t *>(topk_smem);                  // [K] selected ids
@@ -260,6 +273,20 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     }
     __syncthreads();
 
+    const size_t wout = (size_t)K * KP + tail.slots;   // row width of token_ids
+    if (tid < tail.slots) {
+        int id = -1;
+        if (req_ok) {
+            const int f = tail.first_valid[b], qp = tail.q_pos[q];
+            const int rs = tail.req_start[b], T = tail.req_start[b + 1] - rs;
+            if (qp >= f) {
+                const int n = (int)(((long long)qp - f + 1) % KP);
+                const long long t = (long long)qp + 1 - n + tid;
+                if (tid < n && t >= 0 && t < T && tail.valid[(size_t)rs + t] != 0) id = (int)t;
+            }
+        }
+        token_ids[(size_t)q * wout + (size_t)K * KP + tid] = id;
+    }
     for (int j = tid; j < K; j += kTopkThreads)
         top_pools[(size_t)q * K + j] = j < nq ? slist[j] : -1;
     // Expansion: four pool_idx gathers in flight per thread before the stores.
@@ -275,30 +302,33 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int e = e0 + tid + u * kTopkThreads;
-            if (e < K * KP) token_ids[(size_t)q * K * KP + e] = v[u];
+            if (e < K * KP) token_ids[(size_t)q * wout + e] = v[u];
         }
     }
 }
 
 inline int topk_expand_launch(const float *scores, const uint8_t *cand, const int32_t *pool_idx,
                               const int32_t *q_req, int Q, int B, int max_pools, int kpool,
-                              int select_k, int32_t *top_pools, int32_t *token_ids,
-                              cudaStream_t stream) {
+                              int select_k, const TailArgs &tail, int32_t *top_pools,
+                              int32_t *token_ids, cudaStream_t stream) {
     if (Q < 0 || B < 0 || max_pools < 0 || kpool <= 0 || select_k < 0) return DSA_ERR_INVALID_ARG;
     if (kpool > DSA_MAX_KPOOL || select_k > DSA_MAX_SELECT) return DSA_ERR_UNSUPPORTED;
-    if (Q == 0 || select_k == 0) return DSA_OK;
-    if (!q_req || !top_pools || !token_ids ||
+    if (Q == 0 || (select_k == 0 && tail.slots == 0)) return DSA_OK;
+    if (!q_req || (select_k > 0 && !top_pools) || !token_ids ||
         (max_pools > 0 && (!scores || !cand || (B > 0 && !pool_idx))))
         return DSA_ERR_INVALID_ARG;
+    if (tail.slots > 0 && (!tail.q_pos || (B > 0 && (!tail.first_valid || !tail.valid || !tail.req_start))))
+        return DSA_ERR_INVALID_ARG;
     if (!aligned(scores, 4) || !aligned(pool_idx, 4) || !aligned(q_req, 4) ||
-        !aligned(top_pools, 4) || !aligned(token_ids, 4))
+        !aligned(top_pools, 4) || !aligned(token_ids, 4) || !aligned(tail.q_pos, 4) ||
+        !aligned(tail.first_valid, 4) || !aligned(tail.req_start, 4))
         return DSA_ERR_ALIGNMENT;
     const int keys_in_smem = max_pools <= kTopkSmemKeys ? 1 : 0;
     const int smem = select_k * 4 + (keys_in_smem ? max_pools * 4 : 0);
     if (!ensure_smem_attr(reinterpret_cast<const void *>(topk_expand_kernel), smem))
         return DSA_ERR_CUDA;
     if (launch_pdl(topk_expand_kernel, dim3(Q), dim3(kTopkThreads), smem, stream, scores, cand,
-                   pool_idx, q_req, B, max_pools, kpool, select_k, keys_in_smem, top_pools,
+                   pool_idx, q_req, B, max_pools, kpool, select_k, keys_in_smem, tail, top_pools,
                    token_ids) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();

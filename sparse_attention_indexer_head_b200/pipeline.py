@@ -56,19 +56,21 @@ class Geometry:
     hm: int
     eps: float
     sm_scale: float
+    tail: int = 0           # always_select_tail: kpool - 1 extra slots per index row
 
     @property
     def W(self) -> int:
-        return self.select_k * self.kpool
+        return self.select_k * self.kpool + self.tail
 
 
 class DecodeStep:
     """Device buffers of one step; ``run()`` enqueues the five calls on a stream."""
 
-    def __init__(self, wl: Workload, device: str = "cuda", inputs: Optional[Dict] = None):
+    def __init__(self, wl: Workload, device: str = "cuda", inputs: Optional[Dict] = None,
+                 always_select_tail: bool = False):
         self.device = torch.device(device)
         self.g = Geometry(wl.B, wl.Q, wl.kpool, wl.max_pools, wl.select_k, wl.hm, wl.eps,
-                          wl.sm_scale)
+                          wl.sm_scale, wl.kpool - 1 if always_select_tail else 0)
         src = host_tensors(wl) if inputs is None else inputs
         self.t = {k: v.to(self.device) for k, v in src.items()}
         g, dev = self.g, self.device
@@ -107,8 +109,15 @@ class DecodeStep:
 
     def topk_expand(self, stream=None):
         g, t = self.g, self.t
-        B.dsa_topk_expand(self.scores, self.cand, self.pool_idx, t["q_req"], g.Q, g.B,
-                          g.max_pools, g.kpool, g.select_k, self.top_pools, self.token_ids, stream)
+        if g.tail:
+            B.dsa_topk_expand_tail(self.scores, self.cand, self.pool_idx, t["q_req"], t["q_pos"],
+                                   self.first_valid, t["valid"], t["req_start"], g.Q, g.B,
+                                   g.max_pools, g.kpool, g.select_k, self.top_pools,
+                                   self.token_ids, stream)
+        else:
+            B.dsa_topk_expand(self.scores, self.cand, self.pool_idx, t["q_req"], g.Q, g.B,
+                              g.max_pools, g.kpool, g.select_k, self.top_pools, self.token_ids,
+                              stream)
 
     def sparse_mla(self, stream=None):
         g, t = self.g, self.t

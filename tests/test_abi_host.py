@@ -153,6 +153,27 @@ def test_topk_expand_refusals(B):
     assert L.dsa_topk_expand(*bad) == B.DSA_OK
 
 
+def test_topk_expand_tail_refusals(B):
+    L = B.lib
+    # scores, cand, pool_idx, q_req, q_pos, first_valid, tok_valid, req_start, Q, B, P, kpool, K
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 4, 64, 4, 16, FAKE, FAKE, None]
+    bad = list(args); bad[11] = 0
+    assert L.dsa_topk_expand_tail(*bad) == B.DSA_ERR_INVALID_ARG
+    bad = list(args); bad[11] = 9
+    assert L.dsa_topk_expand_tail(*bad) == B.DSA_ERR_UNSUPPORTED
+    bad = list(args); bad[4] = None
+    assert L.dsa_topk_expand_tail(*bad) == B.DSA_ERR_INVALID_ARG       # the tail needs q_pos
+    bad = list(args); bad[5] = None
+    assert L.dsa_topk_expand_tail(*bad) == B.DSA_ERR_INVALID_ARG       # ... and first_valid
+    bad = list(args); bad[4] = FAKE + 2
+    assert L.dsa_topk_expand_tail(*bad) == B.DSA_ERR_ALIGNMENT
+    bad = list(args); bad[8] = 0
+    assert L.dsa_topk_expand_tail(*bad) == B.DSA_OK
+    # kpool 1 has no tail: select_k 0 then writes nothing at all
+    bad = list(args); bad[11] = 1; bad[12] = 0
+    assert L.dsa_topk_expand_tail(*bad) == B.DSA_OK
+
+
 def test_sparse_mla_refusals(B):
     L = B.lib
     # partials of every split (the plan keeps the grid within 148 CTAs; 48-token

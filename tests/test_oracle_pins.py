@@ -542,3 +542,40 @@ def test_compress_after_store_only_changes_pools_of_new_tokens(orc):
     assert before[2][0, 4] == 0 and after[2][0, 4] == 1    # pool 4 complete now
     assert after[2][0, 5] == 0                             # pool 5 still lacks tokens 24..26
     assert not np.array_equal(before[0][0, 4], after[0][0, 4])
+
+
+def test_tail_slots_hold_the_trailing_partial_pool(orc):
+    """Tail slots: the tokens after the query's last complete pool, up to q_pos."""
+    req_start = np.array([0, 20, 30, 30], np.int32)         # request 2 is empty
+    valid = np.ones(30, np.uint8)
+    valid[0:3] = 0                                          # request 0: f = 3
+    valid[20 + 8] = 0                                       # request 1: a hole at token 8
+    first_valid = np.array([3, 0, 0], np.int32)
+    kp = 4
+    q_req = np.array([0, 0, 0, 0, 1, 1, 2, 7])
+    q_pos = np.array([9, 10, 14, 2, 9, 5, 0, 3])
+    got = orc.tail_slots(q_req, q_pos, first_valid, valid, req_start, kp)
+    want = np.array([
+        [7, 8, 9],      # tokens 3..6 form pool 0; 7, 8, 9 trail
+        [-1, -1, -1],   # 3..10 are two complete pools: nothing trails
+        [-1, -1, -1],   # 3..14 three complete pools
+        [-1, -1, -1],   # q_pos before the first valid token
+        [-1, 9, -1],    # pools 0..3, 4..7; 8 (a hole) and 9 trail: the hole's slot is -1
+        [4, 5, -1],
+        [-1, -1, -1],   # empty request: f = T = 0 but token 0 does not exist
+        [-1, -1, -1],   # request out of range
+    ], np.int32)
+    np.testing.assert_array_equal(got, want)
+    # kpool 1: no tail slots at all
+    assert orc.tail_slots(q_req, q_pos, first_valid, valid, req_start, 1).shape == (8, 0)
+    # the tail never repeats a token of a candidate pool: candidates end at or before q_pos
+    rng = np.random.default_rng(3)
+    for _ in range(50):
+        kp = int(rng.integers(2, 9))
+        f = int(rng.integers(0, 5))
+        qp = int(rng.integers(f, 60))
+        t = orc.tail_slots([0], [qp], [f], np.ones(64, np.uint8), [0, 64], kp)[0]
+        last_cand_end = f + ((qp - f + 1) // kp) * kp - 1   # last token of the last candidate pool
+        ids = t[t >= 0]
+        assert (ids > last_cand_end).all() and (ids <= qp).all()
+        assert len(ids) == (qp - f + 1) % kp
