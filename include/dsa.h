@@ -290,6 +290,33 @@ int dsa_sparse_mla_decode(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows
                           dsa_stream_t stream);
 
 /*
+ * f2. Sparse MLA over a block-table paged latent cache ([mod.rs] the serve
+ * path is the block-table paged MLA decode taught to walk a selected-index
+ * row instead of 0..seq_len).
+ *   Arguments, outputs, workspace and refusals are those of
+ *   dsa_sparse_mla_decode, except for where a token's latent row lives:
+ *   kv          bf16 [kv_rows, 512]: the pool of cache pages, page_size rows
+ *               each (kv_rows a multiple of page_size is not required).
+ *   block_table int32 [B, max_blocks]: request b's logical token t is in page
+ *               block_table[b, t / page_size], row t % page_size of it, i.e.
+ *               cache row block_table[b, t / page_size] * page_size + t % page_size.
+ *   seq_len     int32 [B]: T_b, the request's token count.
+ *   An id is ignored (like -1) when it is outside [0, T_b), its page index is
+ *   >= max_blocks, its block number is negative, or its row is >= kv_rows.
+ *   Results equal dsa_sparse_mla_decode's on the contiguous cache holding the
+ *   same rows (the kernels are the same but for the row lookup).
+ * Requires page_size >= 1 and max_blocks >= 0 (DSA_ERR_INVALID_ARG otherwise).
+ * seq_len joins q, q_req and req_start among the inputs read before the wait
+ * on the preceding kernel; block_table is read after it.
+ */
+int dsa_sparse_mla_decode_paged(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows,
+                                const int32_t *block_table, int max_blocks, int page_size,
+                                const int32_t *seq_len, const int32_t *q_req,
+                                const int32_t *token_ids, int Q, int B, int Hm, int W, int kv_lora,
+                                int rope_dim, float sm_scale, dsa_bf16 *out, float *lse,
+                                void *workspace, size_t workspace_bytes, dsa_stream_t stream);
+
+/*
  * dsa_sparse_mla_decode without a workspace argument. The pages have no
  * counterpart to this call; it exists for callers that cannot allocate device
  * memory where they call the MLA: code that runs on an execution path whose

@@ -233,6 +233,49 @@ def sparse_mla(q, kv, req_start, q_req, token_ids, sm_scale: float, threads: int
     return out, lse
 
 
+def sparse_mla_paged(q, kv, block_table, page_size: int, seq_len, q_req, token_ids,
+                     sm_scale: float, threads: int = 0):
+    """Sparse MLA over a block-table paged latent cache: (out, lse) as sparse_mla.
+
+    "spark_model/layers/glm5next_dsa/mod.rs", MASKED_ATTN_MAX_KEYS doc: the serve
+    path is the block-table paged MLA decode walking a selected-index row. The
+    block table only says where a token's latent row is stored: request b's
+    token t is row block_table[b, t // page_size] * page_size + t % page_size.
+    Written out as that lookup followed by the contiguous definition: each
+    request's rows are copied into a contiguous cache, and an id whose page is
+    missing (index past the table, negative block, row past the cache) is
+    dropped like -1.
+    """
+    kv = np.asarray(kv, np.uint16)
+    block_table = np.asarray(block_table, np.int64)
+    B, max_blocks = block_table.shape
+    token_ids = np.array(token_ids, np.int32)
+    lengths = [max(int(seq_len[b]), 0) for b in range(B)]
+    req_start = np.zeros(B + 1, np.int32)
+    req_start[1:] = np.cumsum(lengths)
+    flat = np.zeros((int(req_start[-1]), kv.shape[1]), np.uint16)
+    present = np.zeros(int(req_start[-1]), bool)
+    for b in range(B):
+        for t in range(lengths[b]):
+            pi = t // page_size
+            if pi >= max_blocks or block_table[b, pi] < 0:
+                continue
+            row = int(block_table[b, pi]) * page_size + t % page_size
+            if row >= kv.shape[0]:
+                continue
+            flat[req_start[b] + t] = kv[row]
+            present[req_start[b] + t] = True
+    for i in range(token_ids.shape[0]):
+        b = int(q_req[i])
+        if not (0 <= b < B):
+            continue
+        for j in range(token_ids.shape[1]):
+            t = int(token_ids[i, j])
+            if 0 <= t < lengths[b] and not present[req_start[b] + t]:
+                token_ids[i, j] = -1
+    return sparse_mla(q, flat, req_start, q_req, token_ids, sm_scale, threads)
+
+
 def pipeline(wl, threads: int = 0, queries: Optional[np.ndarray] = None) -> dict:
     """All stages on a workload's raw inputs (optionally a subset of queries)."""
     qsel = np.arange(wl.Q) if queries is None else np.asarray(queries)

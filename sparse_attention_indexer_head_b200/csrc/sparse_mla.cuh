@@ -180,11 +180,24 @@ DSA_DEVINL void mla_cluster_merge(const TcCtl *ctl, uint32_t sO, int S, int nh, 
     }
 }
 
+// Where a request's logical token t lives in the latent cache. Contiguous:
+// row req_start[b] + t, t < T_b = req_start[b+1] - req_start[b]. Paged (a
+// block table, block_table != nullptr): row block_table[b][t / page] * page +
+// t % page, t < T_b = seq_len[b]; a negative block number or a block index past
+// max_blocks makes the token invalid. Either way a row at or past kv_rows is
+// never read (the token counts as invalid).
+struct KvMap {
+    const int32_t *req_start;
+    const int32_t *block_table;   // [B, max_blocks] or nullptr
+    const int32_t *seq_len;       // [B] (paged)
+    int max_blocks, page;
+};
+
 // kv: the latent cache, kv_rows rows of 512 bf16.
-template <bool kCluster>
+template <bool kCluster, bool kPaged>
 __global__ void __launch_bounds__(kTcThreads, 1)
 mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restrict__ kv,
-              const int32_t *__restrict__ req_start, const int32_t *__restrict__ q_req,
+              const KvMap map, const int32_t *__restrict__ q_req,
               const int32_t *__restrict__ token_ids, int B, int kv_rows, int Hm, int W, int S,
               int per, float scale_log2, float *__restrict__ part,
               __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
@@ -246,8 +259,15 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     // Request geometry is a step input: read before the wait on the predecessor.
     const int b = q_req[qi];
     const bool req_ok = b >= 0 && b < B;
-    const int rs = req_ok ? req_start[b] : 0;
-    const int T = req_ok ? max(0, req_start[b + 1] - rs) : 0;
+    int rs = 0, T = 0;
+    if (req_ok) {
+        if constexpr (kPaged) {
+            T = max(0, map.seq_len[b]);
+        } else {
+            rs = map.req_start[b];
+            T = max(0, map.req_start[b + 1] - rs);
+        }
+    }
     pdl_wait();                       // token ids come from the predecessor grid
     pdl_launch_dependents();
 
@@ -338,14 +358,27 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             const int j = c * kTcChunk + 12 * sub + lane;
             return (lane < 12 && c < nch && j < ntok) ? __ldg(token_ids + (size_t)qi * W + j0 + j) : -1;
         };
-        auto gather_chunk = [&](int c, int id) -> bool {
+        // cache row of a logical id, -1 when the id is not a valid token
+        auto resolve = [&](int id) -> int {
+            if (id < 0 || id >= T) return -1;
+            long long r;
+            if constexpr (kPaged) {
+                const int bi = id / map.page;
+                if (bi >= map.max_blocks) return -1;
+                const int blk = __ldg(map.block_table + (size_t)b * map.max_blocks + bi);
+                if (blk < 0) return -1;
+                r = (long long)blk * map.page + (id - bi * map.page);
+            } else {
+                r = (long long)rs + id;
+            }
+            return r < (long long)kv_rows ? (int)r : -1;
+        };
+        auto gather_chunk = [&](int c, int myrow) -> bool {
             const int slot = c % kTcSlots;
             bool ok = true;
             if (c >= kTcSlots) ok = tc_wait(ctl, &ctl->kv_empty[slot], ((c / kTcSlots) - 1) & 1);
             if (!__all_sync(0xffffffffu, ok)) return false;
-            const bool valid = id >= 0 && id < T && (long long)rs + id < (long long)kv_rows;
-            const uint32_t vm = __ballot_sync(0xffffffffu, valid);   // bits 0..11
-            const int myrow = valid ? rs + id : -1;
+            const uint32_t vm = __ballot_sync(0xffffffffu, myrow >= 0);   // bits 0..11
             const uint32_t dst0 = sKV + slot * kSlotRows;
 #pragma unroll
             for (int rr = 0; rr < 12; ++rr) {
@@ -367,17 +400,35 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             tc::cp_async_arrive_noinc(&ctl->kv_full[slot]);
             return true;
         };
-        // ids of the group's next two chunks are in flight (static queue slots)
-        int idq[2] = {load_id(grp), load_id(grp + 2)};
         bool go = true;
-        for (int c0 = grp; go && c0 < nch; c0 += 4) {
+        if constexpr (!kPaged) {
+            // ids of the group's next two chunks are in flight (static queue slots)
+            int idq[2] = {load_id(grp), load_id(grp + 2)};
+            for (int c0 = grp; go && c0 < nch; c0 += 4) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int c = c0 + 2 * u;
-                if (!go || c >= nch) break;
-                const int id = idq[u];
-                idq[u] = load_id(c + 4);
-                go = gather_chunk(c, id);
+                for (int u = 0; u < 2; ++u) {
+                    const int c = c0 + 2 * u;
+                    if (!go || c >= nch) break;
+                    const int id = idq[u];
+                    idq[u] = load_id(c + 4);
+                    go = gather_chunk(c, resolve(id));
+                }
+            }
+        } else {
+            // The block-table lookup is a second dependent load: rows are resolved
+            // two of the group's chunks ahead, ids loaded four ahead.
+            int rq[2] = {resolve(load_id(grp)), resolve(load_id(grp + 2))};
+            int idq[2] = {load_id(grp + 4), load_id(grp + 6)};
+            for (int c0 = grp; go && c0 < nch; c0 += 4) {
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int c = c0 + 2 * u;
+                    if (!go || c >= nch) break;
+                    const int row = rq[u];
+                    rq[u] = resolve(idq[u]);
+                    idq[u] = load_id(c + 8);
+                    go = gather_chunk(c, row);
+                }
             }
         }
         tc::cp_async_wait_all();          // nothing of this warp in flight past here
@@ -700,7 +751,7 @@ inline int mla_max_clusters(int splits) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel<true>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel<true, false>, &cfg) != cudaSuccess) n = 0;
     (void)cudaGetLastError();
     known[dev][splits].store(n + 1, std::memory_order_relaxed);
     return n;
@@ -729,35 +780,41 @@ inline MlaGeom mla_launch_geometry(int Q, int Hm, int W) {
 // split kernel, plus the combine when the splits merge through the workspace.
 inline int sparse_mla_launch_count(int Q, int Hm, int W) {
     if (Q <= 0 || Hm <= 0 || W < 0) return 0;
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true>), kTcSmemBytes)) return 0;
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, false>), kTcSmemBytes))
+        return 0;
     const MlaGeom g = mla_launch_geometry(Q, Hm, W);
     return (g.S > 1 && !g.cluster) ? 2 : 1;
 }
 
-inline int sparse_mla_launch(const void *q, const void *kv, int64_t kv_rows,
-                             const int32_t *req_start, const int32_t *q_req,
-                             const int32_t *token_ids, int Q, int B, int Hm, int W, int kv_lora,
-                             int rope_dim, float sm_scale, void *out, float *lse, void *ws,
-                             size_t ws_bytes, cudaStream_t stream) {
+template <bool kPaged>
+inline int sparse_mla_launch_map(const void *q, const void *kv, int64_t kv_rows, const KvMap &map,
+                                 const int32_t *q_req, const int32_t *token_ids, int Q, int B,
+                                 int Hm, int W, int kv_lora, int rope_dim, float sm_scale,
+                                 void *out, float *lse, void *ws, size_t ws_bytes,
+                                 cudaStream_t stream) {
     if (Q < 0 || B < 0 || Hm <= 0 || W < 0 || kv_lora <= 0 || rope_dim < 0 || kv_rows < 0)
         return DSA_ERR_INVALID_ARG;
     if (!(sm_scale == sm_scale) || sm_scale == INFINITY || sm_scale == -INFINITY)
         return DSA_ERR_INVALID_ARG;
+    if (kPaged && (map.page <= 0 || map.max_blocks < 0)) return DSA_ERR_INVALID_ARG;
     if (kv_lora != kL || rope_dim != 0 || Hm % 16 != 0 || Hm > DSA_MAX_MLA_HEADS)
         return DSA_ERR_UNSUPPORTED;
-    if (kv_rows > (int64_t)INT32_MAX) return DSA_ERR_UNSUPPORTED;   // TMA row coordinates are int32
+    if (kv_rows > (int64_t)INT32_MAX) return DSA_ERR_UNSUPPORTED;   // rows are 32-bit indices
     if (Q == 0) return DSA_OK;
     if (Q > 65535) return DSA_ERR_UNSUPPORTED;
-    if (!q || !q_req || !out || (W > 0 && !token_ids) || (B > 0 && !req_start) ||
-        (kv_rows > 0 && !kv))
+    if (!q || !q_req || !out || (W > 0 && !token_ids) || (kv_rows > 0 && !kv))
         return DSA_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(req_start, 4) || !aligned(q_req, 4) ||
+    if (B > 0 && (kPaged ? (!map.seq_len || (map.max_blocks > 0 && !map.block_table)) : !map.req_start))
+        return DSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(map.req_start, 4) ||
+        !aligned(map.block_table, 4) || !aligned(map.seq_len, 4) || !aligned(q_req, 4) ||
         !aligned(token_ids, 4) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(ws, 16))
         return DSA_ERR_ALIGNMENT;
     const size_t need = mla_workspace_bytes(Q, Hm, W);
     if (need > 0 && (!ws || ws_bytes < need)) return DSA_ERR_WORKSPACE;
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true>), kTcSmemBytes) ||
-        !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<false>), kTcSmemBytes))
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, kPaged>), kTcSmemBytes) ||
+        !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<false, kPaged>), kTcSmemBytes) ||
+        !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, false>), kTcSmemBytes))
         return DSA_ERR_CUDA;
     const MlaGeom g = mla_launch_geometry(Q, Hm, W);
     const float scale_log2 = sm_scale * 1.4426950408889634f;
@@ -768,14 +825,14 @@ inline int sparse_mla_launch(const void *q, const void *kv, int64_t kv_rows,
     auto *ob = reinterpret_cast<__nv_bfloat16 *>(out);
     const dim3 grid(g.S, Q, groups);
     if (g.cluster) {
-        if (launch_pdl_cluster(mla_tc_kernel<true>, grid, dim3(kTcThreads), kTcSmemBytes, stream,
-                               g.S, qb, kvb, req_start, q_req, token_ids, B, (int)kv_rows, Hm,
+        if (launch_pdl_cluster(mla_tc_kernel<true, kPaged>, grid, dim3(kTcThreads), kTcSmemBytes,
+                               stream, g.S, qb, kvb, map, q_req, token_ids, B, (int)kv_rows, Hm,
                                W, g.S, g.per, scale_log2, part, ob, lse) != cudaSuccess)
             return DSA_ERR_CUDA;
         return launch_status();
     }
-    if (launch_pdl(mla_tc_kernel<false>, grid, dim3(kTcThreads), kTcSmemBytes, stream, qb, kvb,
-                   req_start, q_req, token_ids, B, (int)kv_rows, Hm, W, g.S, g.per, scale_log2,
+    if (launch_pdl(mla_tc_kernel<false, kPaged>, grid, dim3(kTcThreads), kTcSmemBytes, stream, qb,
+                   kvb, map, q_req, token_ids, B, (int)kv_rows, Hm, W, g.S, g.per, scale_log2,
                    part, ob, lse) != cudaSuccess)
         return DSA_ERR_CUDA;
     int st = launch_status();
@@ -784,6 +841,28 @@ inline int sparse_mla_launch(const void *q, const void *kv, int64_t kv_rows,
                    lse) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
+}
+
+inline int sparse_mla_launch(const void *q, const void *kv, int64_t kv_rows,
+                             const int32_t *req_start, const int32_t *q_req,
+                             const int32_t *token_ids, int Q, int B, int Hm, int W, int kv_lora,
+                             int rope_dim, float sm_scale, void *out, float *lse, void *ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+    const KvMap map{req_start, nullptr, nullptr, 0, 1};
+    return sparse_mla_launch_map<false>(q, kv, kv_rows, map, q_req, token_ids, Q, B, Hm, W,
+                                        kv_lora, rope_dim, sm_scale, out, lse, ws, ws_bytes,
+                                        stream);
+}
+
+inline int sparse_mla_launch_paged(const void *q, const void *kv, int64_t kv_rows,
+                                   const int32_t *block_table, int max_blocks, int page_size,
+                                   const int32_t *seq_len, const int32_t *q_req,
+                                   const int32_t *token_ids, int Q, int B, int Hm, int W,
+                                   int kv_lora, int rope_dim, float sm_scale, void *out, float *lse,
+                                   void *ws, size_t ws_bytes, cudaStream_t stream) {
+    const KvMap map{nullptr, block_table, seq_len, max_blocks, page_size};
+    return sparse_mla_launch_map<true>(q, kv, kv_rows, map, q_req, token_ids, Q, B, Hm, W,
+                                       kv_lora, rope_dim, sm_scale, out, lse, ws, ws_bytes, stream);
 }
 
 }  // namespace dsa

@@ -579,3 +579,45 @@ def test_tail_slots_hold_the_trailing_partial_pool(orc):
         ids = t[t >= 0]
         assert (ids > last_cand_end).all() and (ids <= qp).all()
         assert len(ids) == (qp - f + 1) % kp
+
+
+def test_paged_mla_single_token_reads_its_page_row(orc):
+    """One selected token: out is its latent row, wherever its page sits."""
+    rng = np.random.default_rng(5)
+    L, page = 512, 2
+    kv = W.f32_to_bf16_bits(rng.standard_normal((8, L), dtype=np.float32))   # 4 pages
+    block_table = np.array([[3, 0, -1], [1, 2, -1]], np.int32)   # request 0: pages 3, 0
+    seq_len = np.array([4, 3], np.int32)
+    q = W.f32_to_bf16_bits(rng.standard_normal((3, 16, L), dtype=np.float32))
+    q_req = np.array([0, 0, 1])
+    ids = np.array([[2, -1], [1, -1], [2, 7]], np.int32)       # 7 is past request 1's tokens
+    out, lse = orc.sparse_mla_paged(q, kv, block_table, page, seq_len, q_req, ids, 0.05)
+    # request 0 token 2 -> page 0 row 0 = cache row 0; token 1 -> page 3 row 1 = cache row 7;
+    # request 1 token 2 -> page 2 row 0 = cache row 4
+    for i, row in enumerate([0, 7, 4]):
+        for h in range(16):
+            np.testing.assert_array_equal(out[i, h], kv[row])
+    # a token on a missing page is dropped: nothing valid -> out 0, lse -inf
+    out2, lse2 = orc.sparse_mla_paged(q[:1], kv, np.array([[-1, 0]], np.int32), page, [4], [0],
+                                      np.array([[0, 1]], np.int32), 0.05)
+    assert (out2 == 0).all() and np.isneginf(lse2).all()
+
+
+def test_paged_mla_is_invariant_to_page_placement(orc):
+    """Moving the pages of a cache (and its table with them) leaves the result unchanged."""
+    rng = np.random.default_rng(9)
+    L, page, T = 512, 4, 22
+    n_pages = (T + page - 1) // page                              # 6 pages
+    kv_c = W.f32_to_bf16_bits(rng.standard_normal((T, L), dtype=np.float32))
+    perm = rng.permutation(10)[:n_pages]                         # 6 of 10 physical pages
+    pool = np.zeros((10 * page, L), np.uint16)
+    for pi in range(n_pages):
+        rows = kv_c[pi * page:(pi + 1) * page]
+        pool[perm[pi] * page:perm[pi] * page + len(rows)] = rows
+    table = perm[None, :].astype(np.int32)
+    q = W.f32_to_bf16_bits(rng.standard_normal((2, 16, L), dtype=np.float32))
+    ids = np.array([rng.permutation(T)[:9], rng.permutation(T)[:9]], np.int32)
+    a = orc.sparse_mla_paged(q, pool, table, page, [T], [0, 0], ids, 0.06)
+    b = orc.sparse_mla(q, kv_c, [0, T], [0, 0], ids, 0.06)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
