@@ -122,12 +122,6 @@ DSA_DEVINL void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes, u
         : "memory");
 }
 
-// L2 prefetch of `bytes` (multiple of 16) of global memory from a 16-byte
-// aligned address; nothing is returned to the SM, so it only warms L2.
-DSA_DEVINL void bulk_prefetch_l2(const void *gmem_src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem_src), "r"(bytes) : "memory");
-}
-
 // ---------------------------------------------------------------- misc
 DSA_DEVINL float ex2(float x) {
     float y;

@@ -288,26 +288,6 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         s_ape[(sl * 2 + ((c >> 2) & 1)) * 64 + 4 * (c >> 3) + (c & 3)] = ape[i] * kLog2e;
     }
     __syncthreads();
-    if (tid == 0) {
-        // Warm L2 with the k and gate rows of this CTA's first tiles while the
-        // preceding kernel drains. The rows are guessed from req_start and the
-        // first valid token the previous call left in first_valid; a wrong guess
-        // only prefetches other rows. Nothing read here is used past the wait.
-        const long long total = req_start[B];
-        for (int i = 0; i < kCmpStages && t_begin + i < t_end; ++i) {
-            const int t = t_begin + i;
-            const int b = t / tiles_per_req, j = t - b * tiles_per_req;
-            const long long rs = req_start[b], T = req_start[b + 1] - rs;
-            long long fo = first_valid[b];
-            if (fo < 0 || fo > T) fo = 0;
-            const long long r0 = max(0ll, rs + fo + (long long)j * kCmpTileTokens);
-            const long long r1 = min(min(r0 + kCmpTileTokens, rs + T), total);
-            if (r1 > r0) {
-                bulk_prefetch_l2(k + r0 * kD, (uint32_t)((r1 - r0) * kD * 2));
-                bulk_prefetch_l2(gate + r0 * kD, (uint32_t)((r1 - r0) * kD * 2));
-            }
-        }
-    }
     pdl_wait();
     pdl_launch_dependents();
 
