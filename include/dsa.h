@@ -332,8 +332,8 @@ int dsa_sparse_mla_decode_paged(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t k
  *   call whose split-KV scratch (dsa_sparse_mla_workspace_size(Q, Hm, W))
  *   exceeds it returns DSA_ERR_WORKSPACE and launches nothing. The split
  *   geometry keeps every grid within 148 CTAs, so no call needs more than
- *   148 x 64 x 516 x 4 bytes (about 19.6 MB): the refusal is a guard that no
- *   present shape reaches.
+ *   148 x 64 x 1032 bytes (about 9.8 MB: a bf16 row of 512 plus m and l per
+ *   head and split): the refusal is a guard that no present shape reaches.
  *   Nothing is allocated or freed: no cudaMalloc, no cudaFree, no allocating
  *   library routine. The first call on a device looks up the scratch's device
  *   address (cudaGetSymbolAddress, with that device current); make that first
@@ -344,7 +344,7 @@ int dsa_sparse_mla_decode_paged(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t k
  *   GPU -- on different streams without ordering between them -- race on the
  *   scratch and must not be made.
  */
-#define DSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+#define DSA_NOALLOC_SCRATCH_BYTES (16u << 20)
 int dsa_sparse_mla_decode_noalloc(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows,
                                   const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids, int Q, int B,
                                   int Hm, int W, int kv_lora, int rope_dim, float sm_scale,

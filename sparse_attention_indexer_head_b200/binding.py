@@ -30,7 +30,7 @@ EXPORTS = (
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_launch_count", "dsa_sparse_mla_decode",
     "dsa_sparse_mla_decode_noalloc", "dsa_sparse_mla_decode_paged",
 )
-DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
+DSA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class DsaError(RuntimeError):

@@ -25,9 +25,11 @@
 namespace dsa {
 
 constexpr int kL = DSA_KV_LORA;      // 512
-// A partial row is O[512], m, l, padded to 516 floats so every row starts on a
-// 16-byte boundary (float4 loads in the combine).
-constexpr int kPartStride = kL + 4;
+// Split partials in the workspace: the unnormalised O rows as bf16
+// [Q][S][Hm][512] (1 KB a row), then (m, l) as float2 [Q][S][Hm]. O is rounded
+// to bf16 once, like the P weights of the PV product: each rounding moves an
+// output by at most 2^-9 of the largest selected value in its channel.
+constexpr size_t kPartRowBytes = kL * 2 + 8;
 
 // ---------------------------------------------------------------------------------------
 // tcgen05 split-KV kernel. One CTA per (split, query, group of 64 heads).
@@ -117,7 +119,7 @@ inline size_t mla_workspace_bytes(int Q, int Hm, int W) {
     if (Q <= 0 || Hm <= 0) return 0;
     const MlaGeom g = mla_plan(Q, Hm, W);
     if (g.S == 1) return 0;
-    return (size_t)Q * g.S * Hm * kPartStride * sizeof(float);
+    return (size_t)Q * g.S * Hm * kPartRowBytes;
 }
 
 DSA_DEVINL bool tc_wait(TcCtl *ctl, uint64_t *bar, uint32_t parity) {
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restrict__ kv,
               const KvMap map, const int32_t *__restrict__ q_req,
               const int32_t *__restrict__ token_ids, int B, int kv_rows, int Hm, int W, int S,
-              int per, float scale_log2, float *__restrict__ part,
+              int per, float scale_log2, uint8_t *__restrict__ part,
               __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
     extern __shared__ uint8_t mla_smem_raw[];
     const uint32_t raw = smem_u32(mla_smem_raw);
@@ -592,26 +594,32 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
         const uint32_t tq = tmem + ((uint32_t)(32 * quarter) << 16);
         const bool have_o = ctl->have_o != 0;
         if (S > 1) {
-            float *pb = part + ((size_t)(qi * S + split) * Hm + h0) * kPartStride;
+            const size_t row0 = (size_t)(qi * S + split) * Hm + h0;
+            __nv_bfloat16 *po = reinterpret_cast<__nv_bfloat16 *>(part) + row0 * kL;
+            float2 *pml = reinterpret_cast<float2 *>(part + (size_t)gridDim.y * S * Hm * kL * 2) + row0;
             if (have_o) {
+                // Lanes 2i and 2i+1 hold latent columns L, L+1: the even lane
+                // writes both columns of heads j, the odd lane of heads j+1.
+                const bool odd = lane & 1;
 #pragma unroll 1
                 for (int bi = 0; bi < 2; ++bi) {
                     const int blk = 2 * (warp >> 2) + bi;
                     uint32_t o[32];
                     tc::tmem_ld32(tq + (blk >> 1) * 64 + (blk & 1) * 32, o);
                     tc::tmem_wait_ld();
-                    const int L = (blk >> 1) * 128 + 32 * quarter + lane;
+                    const int L2 = (blk >> 1) * 128 + 32 * quarter + (lane & ~1);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int h = (blk & 1) * 32 + j;
-                        if (h < nh) pb[(size_t)h * kPartStride + L] = __uint_as_float(o[j]);
+                    for (int j = 0; j < 32; j += 2) {
+                        const float x = __shfl_xor_sync(0xffffffffu, __uint_as_float(odd ? o[j] : o[j + 1]), 1);
+                        const int h = (blk & 1) * 32 + j + (odd ? 1 : 0);
+                        const uint32_t v = odd ? pack_bf16x2(x, __uint_as_float(o[j + 1]))
+                                               : pack_bf16x2(__uint_as_float(o[j]), x);
+                        if (h < nh) *reinterpret_cast<uint32_t *>(po + (size_t)h * kL + L2) = v;
                     }
                 }
             }
-            if (tid < kTcHeads && tid < nh) {
-                pb[(size_t)tid * kPartStride + kL] = ctl->mfin[tid];
-                pb[(size_t)tid * kPartStride + kL + 1] = have_o ? ctl->lsum[tid] : 0.f;
-            }
+            if (tid < kTcHeads && tid < nh)
+                pml[tid] = make_float2(ctl->mfin[tid], have_o ? ctl->lsum[tid] : 0.f);
         } else {
             // single split: normalise here and write bf16 out directly
             __nv_bfloat16 *ob = out + ((size_t)qi * Hm + h0) * kL;
@@ -651,73 +659,64 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
 // more splits take a first round for the maxima. Splits are merged in split
 // order (deterministic).
 __global__ void __launch_bounds__(128)
-mla_combine_kernel(const float *__restrict__ part, int Hm, int S, __nv_bfloat16 *__restrict__ out,
+mla_combine_kernel(const uint8_t *__restrict__ part, int Hm, int S, __nv_bfloat16 *__restrict__ out,
                    float *__restrict__ lse) {
     constexpr int kRound = 16;
     const int h = blockIdx.x, q = blockIdx.y, tid = threadIdx.x;
     pdl_wait();
     pdl_launch_dependents();
-    const float *base = part + ((size_t)q * S * Hm + h) * kPartStride;
-    const size_t sstride = (size_t)Hm * kPartStride;
+    const size_t row0 = (size_t)q * S * Hm + h;                  // split u: row0 + u * Hm
+    const __nv_bfloat16 *po = reinterpret_cast<const __nv_bfloat16 *>(part) + row0 * kL + 4 * tid;
+    const float2 *pml = reinterpret_cast<const float2 *>(part + (size_t)gridDim.y * S * Hm * kL * 2) + row0;
+    const size_t sstride = (size_t)Hm * kL;
     float M = -INFINITY;
     float o[4] = {0.f, 0.f, 0.f, 0.f};
     float lsum = 0.f;
+    auto accum = [&](float m, float l, uint2 v) {
+        if (m == -INFINITY) return;
+        const float w = ex2(m - M);
+        lsum = fmaf(l, w, lsum);
+        o[0] = fmaf(bf16lo(v.x), w, o[0]);
+        o[1] = fmaf(bf16hi(v.x), w, o[1]);
+        o[2] = fmaf(bf16lo(v.y), w, o[2]);
+        o[3] = fmaf(bf16hi(v.y), w, o[3]);
+    };
     if (S <= kRound) {
-        float mv[kRound], lv[kRound];
-        float4 v[kRound];
+        float2 ml[kRound];
+        uint2 v[kRound];
 #pragma unroll
         for (int u = 0; u < kRound; ++u) {
             const bool in = u < S;
-            const float *ps = base + u * sstride;
-            mv[u] = in ? __ldg(ps + kL) : -INFINITY;
-            lv[u] = in ? __ldg(ps + kL + 1) : 0.f;
-            v[u] = in ? __ldg(reinterpret_cast<const float4 *>(ps + 4 * tid)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            ml[u] = in ? __ldg(pml + (size_t)u * Hm) : make_float2(-INFINITY, 0.f);
+            v[u] = in ? __ldg(reinterpret_cast<const uint2 *>(po + u * sstride)) : make_uint2(0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < kRound; ++u) M = fmaxf(M, mv[u]);
+        for (int u = 0; u < kRound; ++u) M = fmaxf(M, ml[u].x);
         if (M != -INFINITY) {
 #pragma unroll
-            for (int u = 0; u < kRound; ++u) {
-                if (mv[u] == -INFINITY) continue;
-                const float w = ex2(mv[u] - M);
-                lsum = fmaf(lv[u], w, lsum);
-                o[0] = fmaf(v[u].x, w, o[0]);
-                o[1] = fmaf(v[u].y, w, o[1]);
-                o[2] = fmaf(v[u].z, w, o[2]);
-                o[3] = fmaf(v[u].w, w, o[3]);
-            }
+            for (int u = 0; u < kRound; ++u) accum(ml[u].x, ml[u].y, v[u]);
         }
     } else {
         for (int s0 = 0; s0 < S; s0 += 8) {
             float mv[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) mv[u] = s0 + u < S ? __ldg(base + (s0 + u) * sstride + kL) : -INFINITY;
+            for (int u = 0; u < 8; ++u) mv[u] = s0 + u < S ? __ldg(pml + (size_t)(s0 + u) * Hm).x : -INFINITY;
 #pragma unroll
             for (int u = 0; u < 8; ++u) M = fmaxf(M, mv[u]);
         }
         if (M != -INFINITY) {
             for (int s0 = 0; s0 < S; s0 += 8) {
-                float mv[8], lv[8];
-                float4 v[8];
+                float2 ml[8];
+                uint2 v[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const bool in = s0 + u < S;
-                    const float *ps = base + (s0 + u) * sstride;
-                    mv[u] = in ? __ldg(ps + kL) : -INFINITY;
-                    lv[u] = in ? __ldg(ps + kL + 1) : 0.f;
-                    v[u] = in ? __ldg(reinterpret_cast<const float4 *>(ps + 4 * tid))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                    ml[u] = in ? __ldg(pml + (size_t)(s0 + u) * Hm) : make_float2(-INFINITY, 0.f);
+                    v[u] = in ? __ldg(reinterpret_cast<const uint2 *>(po + (s0 + u) * sstride))
+                              : make_uint2(0u, 0u);
                 }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    if (mv[u] == -INFINITY) continue;
-                    const float w = ex2(mv[u] - M);
-                    lsum = fmaf(lv[u], w, lsum);
-                    o[0] = fmaf(v[u].x, w, o[0]);
-                    o[1] = fmaf(v[u].y, w, o[1]);
-                    o[2] = fmaf(v[u].z, w, o[2]);
-                    o[3] = fmaf(v[u].w, w, o[3]);
-                }
+                for (int u = 0; u < 8; ++u) accum(ml[u].x, ml[u].y, v[u]);
             }
         }
     }
@@ -819,7 +818,7 @@ inline int sparse_mla_launch_map(const void *q, const void *kv, int64_t kv_rows,
     const MlaGeom g = mla_launch_geometry(Q, Hm, W);
     const float scale_log2 = sm_scale * 1.4426950408889634f;
     const int groups = (Hm + kTcHeads - 1) / kTcHeads;
-    float *part = reinterpret_cast<float *>(ws);
+    auto *part = reinterpret_cast<uint8_t *>(ws);
     const auto *qb = reinterpret_cast<const __nv_bfloat16 *>(q);
     const auto *kvb = reinterpret_cast<const __nv_bfloat16 *>(kv);
     auto *ob = reinterpret_cast<__nv_bfloat16 *>(out);

@@ -6,8 +6,9 @@ Tolerances (each derived from the arithmetic, see the docstrings):
                     the magnitude of the summed terms (equal to |ref| when every
                     gate weight is positive).
   * bf16 pooled keys: |gpu - ref| <= ulp(ref) + max_s ulp(kn_s).
-  * bf16 MLA out:   max-abs 2e-2 and |gpu - ref| <= ulp(ref) + 2^-8 max_j |v_j[c]|
-                    (bf16 softmax weights in the tensor-core PV product); lse 1e-4.
+  * bf16 MLA out:   max-abs 2e-2 and |gpu - ref| <= ulp(ref) + (2^-8 + 2^-12) max_j |v_j[c]|
+                    (bf16 softmax weights in the tensor-core PV product, bf16
+                    split partials); lse 1e-4.
 """
 from __future__ import annotations
 
@@ -111,8 +112,12 @@ def assert_mla_close(gpu_out, ref_out, gpu_lse, ref_lse, vbound=None, rows=None)
     The tensor-core PV product takes the softmax weights as bf16, so each weight
     carries a relative rounding error of at most 2^-9. With the row sum taken
     from the unrounded weights, out' - out = sum_j w_j e_j v_j / sum_j w_j, so
-    |out' - out| <= 2^-9 max_j |v_j[c]|; the bound used is ulp(ref) plus twice
-    that (fp32 accumulation and the exp2 approximation are far below it).
+    |out' - out| <= 2^-9 max_j |v_j[c]|. When a query's splits merge through
+    the workspace, each split's O row is stored as bf16 once more: another
+    relative 2^-9 of |O_s[c]| <= l_s max_j |v_j[c]|, i.e. at most
+    2^-9 max_j |v_j[c]| after the merge. The bound used is ulp(ref) plus
+    (2^-8 + 2^-12) max_j |v_j[c]|: the two roundings and a margin for fp32
+    accumulation and the exp2 approximation, which are far below 2^-12.
     Also the spec max-abs 2e-2, and lse within 1e-4 (fp32 sums of
     fp32 weights; one missing token among 2048 moves lse by ~1e-3).
     """
@@ -125,7 +130,7 @@ def assert_mla_close(gpu_out, ref_out, gpu_lse, ref_lse, vbound=None, rows=None)
     err = np.abs(g - r)
     assert err.max(initial=0) <= 2e-2, f"mla out max-abs {err.max():.3g}"
     if vbound is not None:
-        bound = bf16_ulp(r) + 2.0 ** -8 * vbound[:, None, :]
+        bound = bf16_ulp(r) + (2.0 ** -8 + 2.0 ** -12) * vbound[:, None, :]
         assert (err <= bound).all(), f"mla out: {(err > bound).sum()} outside the weight-rounding bound"
     within = float((err <= bf16_ulp(r)).mean()) if err.size else 1.0
     both_inf = np.isneginf(gpu_lse) & np.isneginf(ref_lse)

@@ -180,8 +180,8 @@ def test_sparse_mla_refusals(B):
     # chunks, 43 of them for 2048 ids): 2 queries -> 43 splits of one chunk;
     # 16 queries -> 9 splits of 5 chunks
     ws = B.dsa_sparse_mla_workspace_size(2, 64, 2048)
-    assert ws == 2 * 43 * 64 * 516 * 4
-    assert B.dsa_sparse_mla_workspace_size(16, 64, 2048) == 16 * 9 * 64 * 516 * 4
+    assert ws == 2 * 43 * 64 * (512 * 2 + 8)
+    assert B.dsa_sparse_mla_workspace_size(16, 64, 2048) == 16 * 9 * 64 * (512 * 2 + 8)
     # at least 148 CTAs without splitting: one split, no workspace
     assert B.dsa_sparse_mla_workspace_size(148, 64, 2048) == 0
     assert B.dsa_sparse_mla_workspace_size(74, 128, 2048) == 0
@@ -222,8 +222,8 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
 
 def test_noalloc_scratch_covers_every_geometry(B):
     # The split geometry keeps every grid within one wave of 148 CTAs, so the
-    # split-KV scratch of any call is at most 148 x 64 heads x 516 floats.
-    bound = 148 * 64 * 516 * 4
+    # split-KV scratch of any call is at most 148 x 64 heads x (a bf16 row + m, l).
+    bound = 148 * 64 * (512 * 2 + 8)
     assert bound <= B.DSA_NOALLOC_SCRATCH_BYTES
     worst = 0
     for Q in list(range(1, 40)) + [64, 100, 147, 148, 149, 1000]:
