@@ -259,3 +259,70 @@ def test_incremental_step_equals_full_step(B, name):
     for key in a:
         assert np.array_equal(a[key], b[key], equal_nan=key in ("scores", "lse")), key
     device_status_clean(B)
+
+
+@pytest.mark.parametrize("kpool", [3, 4])
+def test_decode_sequence_stays_equal_to_full_compress(B, kpool):
+    """Twelve decode steps, each storing one new token per request (some invalid,
+    some requests idle), through one captured CUDA graph: after every step the
+    incremental outputs equal the full compress of the grown cache, byte for byte."""
+    caps = [96, 64, 80, 33]
+    lens = [40, 0, 77, 10]                  # request 1 starts empty
+    wl = _capacity_workload(kpool, caps, lens, [3, 0, 0, 0], seed=60 + kpool)
+    c = Cache(wl)
+    inc = c.outputs()
+    c.compress(B, inc)
+    rng = np.random.default_rng(kpool + 100)
+    nb = wl.B
+    # device-side step inputs, refilled in place each step so a graph can replay them
+    k_new = torch.empty(nb, 128, dtype=torch.bfloat16, device="cuda")
+    g_new = torch.empty_like(k_new)
+    v_new = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    t_req = torch.arange(nb, dtype=torch.int32, device="cuda")
+    t_pos = torch.empty(nb, dtype=torch.int32, device="cuda")
+    t_beg = torch.empty(nb, dtype=torch.int32, device="cuda")
+    t_end = torch.empty(nb, dtype=torch.int32, device="cuda")
+
+    def step(stream=None):
+        B.dsa_indexer_store(k_new, g_new, v_new, t_req, t_pos, nb, 128, c.req_start, nb, c.k,
+                            c.gate, c.valid, stream)
+        B.dsa_kpool_compress_tokens(c.k, c.gate, c.valid, c.req_start, nb, 128, kpool,
+                                    wl.max_pools, c.ape, c.ln_w, c.ln_b, wl.eps, t_beg, t_end,
+                                    inc["keys"], inc["idx"], inc["pv"], inc["fv"], stream)
+
+    s = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    pos = np.array(lens)
+
+    def fill():
+        active = (rng.random(nb) < 0.8) & (pos < np.array(caps))
+        k_new.copy_(dev_bits(W.f32_to_bf16_bits(rng.standard_normal((nb, 128), dtype=np.float32))))
+        g_new.copy_(dev_bits(W.f32_to_bf16_bits(rng.standard_normal((nb, 128), dtype=np.float32))))
+        v_new.copy_(_u8((rng.random(nb) < 0.9).astype(np.uint8)))
+        p = np.where(active, pos, -1).astype(np.int32)        # -1: no new token this step
+        t_pos.copy_(_i32(p))
+        t_beg.copy_(_i32(np.where(active, pos, 0)))
+        t_end.copy_(_i32(np.where(active, pos + 1, 0)))
+        return active
+
+    for it in range(12):
+        active = fill()
+        torch.cuda.synchronize()
+        if it == 0:
+            with torch.cuda.stream(s):
+                step()                                        # eager first (sets attributes)
+            s.synchronize()
+            with torch.cuda.graph(graph, stream=s):
+                step()
+        else:
+            graph.replay()
+        torch.cuda.synchronize()
+        pos = pos + active
+        full = c.outputs()
+        # the full reference must start from the same unwritten-row contents
+        full["keys"].copy_(inc["keys"])
+        c.compress(B, full)
+        torch.cuda.synchronize()
+        _assert_same(_np(inc), _np(full), f"step {it}")
+    del graph
+    device_status_clean(B)
