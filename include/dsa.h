@@ -83,6 +83,17 @@ enum dsa_status {
  */
 int dsa_device_status(int *value, int reset);
 
+/*
+ * Failure-detection self-check. Launches one CTA that waits, through the
+ * bounded wait every kernel of the path uses, on an mbarrier phase that nothing
+ * completes. The wait gives up after its bound (about two seconds of SM clock
+ * cycles), ORs code 1 into the device error word and the kernel writes 0 to
+ * *result (a device int; 1 would mean the wait completed). The kernel then
+ * returns normally, so the context stays usable. A diagnostic for tests: it
+ * occupies the stream for about two seconds.
+ */
+int dsa_selftest_bounded_wait(int *result, dsa_stream_t stream);
+
 /* Name of a status code (static string, never NULL). */
 const char *dsa_status_string(int status);
 /* ABI revision of this header; bumps on any signature or contract change. */

@@ -24,7 +24,8 @@ DSA_ERR_CUDA = 5
 
 # Every symbol include/dsa.h declares.
 EXPORTS = (
-    "dsa_status_string", "dsa_abi_version", "dsa_device_status", "dsa_head_gate",
+    "dsa_status_string", "dsa_abi_version", "dsa_device_status", "dsa_selftest_bounded_wait",
+    "dsa_head_gate",
     "dsa_kpool_compress", "dsa_indexer_store", "dsa_kpool_compress_tokens",
     "dsa_index_scores", "dsa_topk_expand", "dsa_topk_expand_tail",
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_launch_count", "dsa_sparse_mla_decode",
@@ -52,6 +53,7 @@ def _load() -> ctypes.CDLL:
         "dsa_status_string": ([I], ctypes.c_char_p),
         "dsa_abi_version": ([], I),
         "dsa_device_status": ([ctypes.POINTER(I), I], I),
+        "dsa_selftest_bounded_wait": ([P, P], I),
         "dsa_head_gate": ([P, P, P, I, I, I, P], I),
         "dsa_kpool_compress": ([P, P, P, P, I, I, I, I, P, P, P, F, P, P, P, P, P], I),
         "dsa_indexer_store": ([P, P, P, P, P, I, I, P, I, P, P, P, P], I),
@@ -111,6 +113,10 @@ def dsa_device_status(reset: bool = True) -> int:
     v = ctypes.c_int(0)
     _check("dsa_device_status", lib.dsa_device_status(ctypes.byref(v), int(reset)))
     return v.value
+
+
+def dsa_selftest_bounded_wait(result, stream=None) -> None:
+    _check("dsa_selftest_bounded_wait", lib.dsa_selftest_bounded_wait(_ptr(result), _stream(stream)))
 
 
 def dsa_head_gate(hidden, w, out, M: int, K: int, N: int, stream=None) -> None:

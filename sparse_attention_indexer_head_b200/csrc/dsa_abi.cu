@@ -43,6 +43,19 @@ int scratch_address(void **out) {
 }
 }  // namespace
 
+// Failure-detection self-check: one CTA waits on an mbarrier phase that nothing
+// completes, through the same bounded wait as every kernel of the path.
+static __global__ void selftest_wait_kernel(int *result) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        dsa::mbar_init(&bar, 1);
+        dsa::fence_mbarrier_init();
+    }
+    __syncthreads();
+    const bool ok = dsa::mbar_wait(&bar, 0);   // phase 0 never completes: gives up
+    if (threadIdx.x == 0) *result = ok ? 1 : 0;
+}
+
 extern "C" {
 
 const char *dsa_status_string(int status) {
@@ -70,6 +83,13 @@ int dsa_device_status(int *value, int reset) {
             return DSA_ERR_CUDA;
     }
     return DSA_OK;
+}
+
+int dsa_selftest_bounded_wait(int *result, dsa_stream_t stream) {
+    if (!result) return DSA_ERR_INVALID_ARG;
+    if (!dsa::aligned(result, 4)) return DSA_ERR_ALIGNMENT;
+    selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(result);
+    return dsa::launch_status();
 }
 
 int dsa_head_gate(const float *hidden, const float *w, float *out, int M, int K, int N,

@@ -49,6 +49,11 @@ def test_status_strings_and_version(B):
 FAKE = 1 << 20          # a 16-byte aligned non-null address; never dereferenced on these paths
 
 
+def test_selftest_refusals(B):
+    assert B.lib.dsa_selftest_bounded_wait(None, None) == B.DSA_ERR_INVALID_ARG
+    assert B.lib.dsa_selftest_bounded_wait(FAKE + 2, None) == B.DSA_ERR_ALIGNMENT
+
+
 def test_head_gate_refusals(B):
     L = B.lib
     assert L.dsa_head_gate(None, None, None, 4, 4096, 16, None) == B.DSA_ERR_INVALID_ARG
