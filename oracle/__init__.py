@@ -40,8 +40,11 @@ def lib():
         L.orc_index_scores.argtypes = [P, P, P, P, I, I, I, P, P, P, I, I, I, P, P, I]
         L.orc_topk_expand.argtypes = [P, P, P, P, I, I, I, I, I, P, P, I]
         L.orc_sparse_mla.argtypes = [P, P, P, P, P, I, I, I, I, I, D, P, P, I]
+        L.orc_sparse_mla_fp8.argtypes = [P, P, D, P, P, P, I, I, I, I, I, D, P, P, I]
+        L.orc_f64_from_e4m3.argtypes = [ctypes.c_uint8]
+        L.orc_f64_from_e4m3.restype = D
         for f in ("orc_head_gate", "orc_layernorm_row", "orc_kpool_compress",
-                  "orc_index_scores", "orc_topk_expand", "orc_sparse_mla"):
+                  "orc_index_scores", "orc_topk_expand", "orc_sparse_mla", "orc_sparse_mla_fp8"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -66,6 +69,10 @@ def default_threads() -> int:
 
 def bf16_from_f64(x: float) -> int:
     return int(lib().orc_bf16_from_f64(float(x)))
+
+
+def f64_from_e4m3(code: int) -> float:
+    return float(lib().orc_f64_from_e4m3(int(code)))
 
 
 def f64_from_bf16(bits: int) -> float:
@@ -230,6 +237,30 @@ def sparse_mla(q, kv, req_start, q_req, token_ids, sm_scale: float, threads: int
     _check(lib().orc_sparse_mla(_p(q), _p(kv), _p(req_start), _p(q_req), _p(token_ids), Q, B, Hm,
                                 W, L, float(np.float32(sm_scale)), _p(out), _p(lse),
                                 threads or default_threads()), "sparse_mla")
+    return out, lse
+
+
+def sparse_mla_fp8(q, kv8, kv_scale: float, req_start, q_req, token_ids, sm_scale: float,
+                   threads: int = 0):
+    """sparse_mla over an fp8 latent cache: row values kv_scale * E4M3(kv8).
+
+    The pages name an fp8 variant of the paged MLA decode and give no scale
+    layout; the reading taken is one fp32 scale for the whole cache.
+    """
+    q = _c(q, np.uint16)
+    kv8 = _c(kv8, np.uint8)
+    req_start = _c(req_start, np.int32)
+    q_req = _c(q_req, np.int32)
+    token_ids = _c(token_ids, np.int32)
+    Q, Hm, L = q.shape
+    W = token_ids.shape[1]
+    B = req_start.shape[0] - 1
+    out = np.empty((Q, Hm, L), dtype=np.uint16)
+    lse = np.empty((Q, Hm), dtype=np.float32)
+    _check(lib().orc_sparse_mla_fp8(_p(q), _p(kv8), float(np.float32(kv_scale)), _p(req_start),
+                                    _p(q_req), _p(token_ids), Q, B, Hm, W, L,
+                                    float(np.float32(sm_scale)), _p(out), _p(lse),
+                                    threads or default_threads()), "sparse_mla_fp8")
     return out, lse
 
 

@@ -80,6 +80,19 @@ uint16_t orc_bf16_from_f64(double x) {
 
 static float orc_f32(double x) { return (float)x; }   /* round to nearest even */
 
+/*
+ * OCP 8-bit floating point, E4M3 (the "fn" variant: no infinities): sign bit,
+ * 4 exponent bits with bias 7, 3 mantissa bits. Exponent field 0 is subnormal,
+ * m/8 * 2^-6; otherwise (1 + m/8) * 2^(e-7); the codes S.1111.111 are NaN, so
+ * the largest magnitude is 1.75 * 2^8 = 448.
+ */
+double orc_f64_from_e4m3(uint8_t b) {
+    int s = b >> 7, e = (b >> 3) & 0xF, m = b & 0x7;
+    if (e == 0xF && m == 0x7) return NAN;
+    double v = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
 /* ------------------------------------------------------------------------ */
 /* a1: head gate [PR227]. out[m,n] = sum_k hidden[m,k] * w[k,n], fp32 result. */
 int orc_head_gate(const float *hidden, const float *w, float *out, int M, int K, int N,
@@ -356,9 +369,17 @@ int orc_topk_expand(const float *scores, const uint8_t *cand, const int32_t *poo
  *   An empty mask gives out = 0 and lse = -inf.
  * READING: sm_scale is an argument (the pages do not print it).
  */
-int orc_sparse_mla(const uint16_t *q, const uint16_t *kv, const int32_t *req_start,
-                   const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
-                   int W, int L, double sm_scale, uint16_t *out, float *lse, int threads) {
+/* latent value c of cache row r: bf16, or E4M3 times one cache-wide scale */
+static double orc_kv_at(const uint16_t *kv, const uint8_t *kv8, double kv_scale, size_t r, int L,
+                        int c) {
+    if (kv) return orc_f64_from_bf16(kv[r * (size_t)L + c]);
+    return kv_scale * orc_f64_from_e4m3(kv8[r * (size_t)L + c]);
+}
+
+static int orc_sparse_mla_any(const uint16_t *q, const uint16_t *kv, const uint8_t *kv8,
+                              double kv_scale, const int32_t *req_start, const int32_t *q_req,
+                              const int32_t *token_ids, int Q, int B, int Hm, int W, int L,
+                              double sm_scale, uint16_t *out, float *lse, int threads) {
     if (Q < 0 || Hm <= 0 || W < 0 || L <= 0) return ORC_EINVAL;
     for (int i = 0; i < Q; ++i)
         if (q_req[i] < 0 || q_req[i] >= B) return ORC_EINVAL;
@@ -394,10 +415,10 @@ int orc_sparse_mla(const uint16_t *q, const uint16_t *kv, const int32_t *req_sta
             int any = 0;
             for (int t = 0; t < T; ++t) {
                 if (!mask[t]) continue;
-                const uint16_t *row = kv + (size_t)(rs + t) * L;
                 double dot = 0.0;
                 for (int c = 0; c < L; ++c)
-                    dot += orc_f64_from_bf16(qh[c]) * orc_f64_from_bf16(row[c]);
+                    dot += orc_f64_from_bf16(qh[c]) *
+                           orc_kv_at(kv, kv8, kv_scale, (size_t)(rs + t), L, c);
                 z[t] = sm_scale * dot;
                 if (z[t] > mx) mx = z[t];
                 any = 1;
@@ -415,8 +436,8 @@ int orc_sparse_mla(const uint16_t *q, const uint16_t *kv, const int32_t *req_sta
             for (int t = 0; t < T; ++t) {
                 if (!mask[t]) continue;
                 double pr = exp(z[t] - mx) / den;
-                const uint16_t *row = kv + (size_t)(rs + t) * L;
-                for (int c = 0; c < L; ++c) acc[c] += pr * orc_f64_from_bf16(row[c]);
+                for (int c = 0; c < L; ++c)
+                    acc[c] += pr * orc_kv_at(kv, kv8, kv_scale, (size_t)(rs + t), L, c);
             }
             for (int c = 0; c < L; ++c) o[c] = orc_bf16_from_f64(acc[c]);
             if (lse) lse[(size_t)i * Hm + h] = orc_f32(mx + log(den));
@@ -426,4 +447,27 @@ int orc_sparse_mla(const uint16_t *q, const uint16_t *kv, const int32_t *req_sta
         free(acc);
     }
     return 0;
+}
+
+int orc_sparse_mla(const uint16_t *q, const uint16_t *kv, const int32_t *req_start,
+                   const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
+                   int W, int L, double sm_scale, uint16_t *out, float *lse, int threads) {
+    if (!kv && Q > 0 && W > 0) return ORC_EINVAL;
+    return orc_sparse_mla_any(q, kv, NULL, 0.0, req_start, q_req, token_ids, Q, B, Hm, W, L,
+                              sm_scale, out, lse, threads);
+}
+
+/*
+ * f2: the same attention over an fp8 latent cache: row value c is
+ * kv_scale * E4M3(kv8[row, c]) (one scale for the whole cache).
+ * READING: the pages name an fp8 variant of the paged MLA decode and give no
+ * scale layout; one cache-wide fp32 scale is the plainest.
+ */
+int orc_sparse_mla_fp8(const uint16_t *q, const uint8_t *kv8, double kv_scale,
+                       const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids,
+                       int Q, int B, int Hm, int W, int L, double sm_scale, uint16_t *out,
+                       float *lse, int threads) {
+    if (!kv8 && Q > 0 && W > 0) return ORC_EINVAL;
+    return orc_sparse_mla_any(q, NULL, kv8, kv_scale, req_start, q_req, token_ids, Q, B, Hm, W, L,
+                              sm_scale, out, lse, threads);
 }

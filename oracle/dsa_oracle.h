@@ -56,6 +56,12 @@ int orc_topk_expand(const float *scores, const uint8_t *cand, const int32_t *poo
 int orc_sparse_mla(const uint16_t *q, const uint16_t *kv, const int32_t *req_start,
                    const int32_t *q_req, const int32_t *token_ids, int Q, int B, int Hm,
                    int W, int L, double sm_scale, uint16_t *out, float *lse, int threads);
+/* f2 the same over an fp8 (E4M3) latent cache with one cache-wide scale. */
+double orc_f64_from_e4m3(uint8_t b);
+int orc_sparse_mla_fp8(const uint16_t *q, const uint8_t *kv8, double kv_scale,
+                       const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids,
+                       int Q, int B, int Hm, int W, int L, double sm_scale, uint16_t *out,
+                       float *lse, int threads);
 
 #ifdef __cplusplus
 }

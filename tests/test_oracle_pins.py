@@ -621,3 +621,36 @@ def test_paged_mla_is_invariant_to_page_placement(orc):
     b = orc.sparse_mla(q, kv_c, [0, T], [0, 0], ids, 0.06)
     np.testing.assert_array_equal(a[0], b[0])
     np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_e4m3_decode_vs_torch_and_definition(orc):
+    """Every E4M3 code against torch's float8_e4m3fn and the format's landmarks."""
+    codes = np.arange(256, dtype=np.uint8)
+    mine = np.array([orc.f64_from_e4m3(int(c)) for c in codes])
+    lib_vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(lib_vals)
+    assert (np.isnan(mine) == nan).all() and nan.sum() == 2            # S.1111.111 only
+    np.testing.assert_array_equal(mine[~nan], lib_vals[~nan])
+    assert orc.f64_from_e4m3(0x7E) == 448.0 and orc.f64_from_e4m3(0x01) == 2.0 ** -9
+    assert orc.f64_from_e4m3(0x38) == 1.0 and orc.f64_from_e4m3(0xB8) == -1.0
+
+
+def test_fp8_mla_single_token_and_scale(orc):
+    """One selected token: out = bf16(kv_scale * decoded row); the scale enters the logits."""
+    rng = np.random.default_rng(12)
+    L = 512
+    kv8 = rng.integers(0, 256, size=(5, L)).astype(np.uint8)
+    kv8[(kv8 & 0x7F) == 0x7F] = 0x3C                                    # no NaN codes
+    q = W.f32_to_bf16_bits(rng.standard_normal((2, 16, L), dtype=np.float32))
+    ids = np.array([[3, -1], [1, 4]], np.int32)
+    out, lse = orc.sparse_mla_fp8(q, kv8, 0.5, [0, 5], [0, 0], ids, 0.01)
+    dec = np.array([[orc.f64_from_e4m3(int(c)) for c in row] for row in kv8])
+    want = np.array([orc.bf16_from_f64(0.5 * v) for v in dec[3]], np.uint16)
+    for h in range(16):        # as values: a sum that starts at +0 turns a -0 row entry into +0
+        np.testing.assert_array_equal(W.bf16_bits_to_f32(out[0, h]), W.bf16_bits_to_f32(want))
+    # a power-of-two scale is exact, so the fp8 result equals the bf16 result on the
+    # decoded-and-scaled cache (each scaled value is a bf16 value)
+    kv_bf16 = np.array([[orc.bf16_from_f64(0.5 * v) for v in row] for row in dec], np.uint16)
+    out_b, lse_b = orc.sparse_mla(q, kv_bf16, [0, 5], [0, 0], ids, 0.01)
+    np.testing.assert_array_equal(out, out_b)
+    np.testing.assert_array_equal(lse, lse_b)
