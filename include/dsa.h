@@ -328,6 +328,26 @@ int dsa_sparse_mla_decode_paged(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t k
                                 void *workspace, size_t workspace_bytes, dsa_stream_t stream);
 
 /*
+ * f2. The paged sparse MLA over an fp8 latent cache ([mod.rs] names the fp8
+ * variant of the block-table paged MLA decode; it gives no scale layout).
+ *   As dsa_sparse_mla_decode_paged, except that
+ *   kv8       uint8 [kv_rows, 512]: OCP FP8 E4M3 codes (S.1111.111 is NaN),
+ *   kv_scale  one fp32 scale for the whole cache (finite, > 0): latent value
+ *             = kv_scale * E4M3(code).
+ *   The rows enter the tensor-core products widened to bf16, which is exact;
+ *   kv_scale is applied to the logits and to the output, so the result is
+ *   that of the bf16 kernel on the scaled cache up to fp32 rounding.
+ * DSA_ERR_INVALID_ARG for a kv_scale that is not finite and positive.
+ */
+int dsa_sparse_mla_decode_paged_fp8(const dsa_bf16 *q, const uint8_t *kv8, float kv_scale,
+                                    int64_t kv_rows, const int32_t *block_table, int max_blocks,
+                                    int page_size, const int32_t *seq_len, const int32_t *q_req,
+                                    const int32_t *token_ids, int Q, int B, int Hm, int W,
+                                    int kv_lora, int rope_dim, float sm_scale, dsa_bf16 *out,
+                                    float *lse, void *workspace, size_t workspace_bytes,
+                                    dsa_stream_t stream);
+
+/*
  * dsa_sparse_mla_decode without a workspace argument. The pages have no
  * counterpart to this call; it exists for callers that cannot allocate device
  * memory where they call the MLA: code that runs on an execution path whose

@@ -30,6 +30,7 @@ EXPORTS = (
     "dsa_index_scores", "dsa_topk_expand", "dsa_topk_expand_tail",
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_launch_count", "dsa_sparse_mla_decode",
     "dsa_sparse_mla_decode_noalloc", "dsa_sparse_mla_decode_paged",
+    "dsa_sparse_mla_decode_paged_fp8",
 )
 DSA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -68,6 +69,8 @@ def _load() -> ctypes.CDLL:
         "dsa_sparse_mla_decode_noalloc": ([P, P, I64, P, P, P, I, I, I, I, I, I, F, P, P, P], I),
         "dsa_sparse_mla_decode_paged": ([P, P, I64, P, I, I, P, P, P, I, I, I, I, I, I, F, P, P, P,
                                          Z, P], I),
+        "dsa_sparse_mla_decode_paged_fp8": ([P, P, F, I64, P, I, I, P, P, P, I, I, I, I, I, I, F, P,
+                                             P, P, Z, P], I),
     }
     for name, (argtypes, restype) in sig.items():
         fn = getattr(L, name)
@@ -209,3 +212,14 @@ def dsa_sparse_mla_decode_paged(q, kv, kv_rows: int, block_table, max_blocks: in
         _ptr(q), _ptr(kv), kv_rows, _ptr(block_table), max_blocks, page_size, _ptr(seq_len),
         _ptr(q_req), _ptr(token_ids), Q, B, Hm, W, kv_lora, rope_dim, float(sm_scale), _ptr(out),
         _ptr(lse), _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def dsa_sparse_mla_decode_paged_fp8(q, kv8, kv_scale: float, kv_rows: int, block_table,
+                                    max_blocks: int, page_size: int, seq_len, q_req, token_ids,
+                                    Q: int, B: int, Hm: int, W: int, kv_lora: int, rope_dim: int,
+                                    sm_scale: float, out, lse, workspace, workspace_bytes: int,
+                                    stream=None) -> None:
+    _check("dsa_sparse_mla_decode_paged_fp8", lib.dsa_sparse_mla_decode_paged_fp8(
+        _ptr(q), _ptr(kv8), float(kv_scale), kv_rows, _ptr(block_table), max_blocks, page_size,
+        _ptr(seq_len), _ptr(q_req), _ptr(token_ids), Q, B, Hm, W, kv_lora, rope_dim,
+        float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace_bytes, _stream(stream)))

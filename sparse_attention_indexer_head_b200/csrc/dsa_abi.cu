@@ -187,6 +187,19 @@ int dsa_sparse_mla_decode_paged(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t k
                                         reinterpret_cast<cudaStream_t>(stream));
 }
 
+int dsa_sparse_mla_decode_paged_fp8(const dsa_bf16 *q, const uint8_t *kv8, float kv_scale,
+                                    int64_t kv_rows, const int32_t *block_table, int max_blocks,
+                                    int page_size, const int32_t *seq_len, const int32_t *q_req,
+                                    const int32_t *token_ids, int Q, int B, int Hm, int W,
+                                    int kv_lora, int rope_dim, float sm_scale, dsa_bf16 *out,
+                                    float *lse, void *workspace, size_t workspace_bytes,
+                                    dsa_stream_t stream) {
+    return dsa::sparse_mla_launch_paged_fp8(q, kv8, kv_scale, kv_rows, block_table, max_blocks,
+                                            page_size, seq_len, q_req, token_ids, Q, B, Hm, W,
+                                            kv_lora, rope_dim, sm_scale, out, lse, workspace,
+                                            workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int dsa_sparse_mla_decode_noalloc(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows,
                                   const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids, int Q, int B,
                                   int Hm, int W, int kv_lora, int rope_dim, float sm_scale,

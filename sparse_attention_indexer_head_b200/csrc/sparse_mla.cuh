@@ -137,7 +137,8 @@ DSA_DEVINL bool tc_wait(TcCtl *ctl, uint64_t *bar, uint32_t parity) {
 // [r*hp, min(nh, (r+1)*hp)), hp = ceil(nh / S), 256 threads x 4 latents per
 // head; splits enter in rank order.
 DSA_DEVINL void mla_cluster_merge(const TcCtl *ctl, uint32_t sO, int S, int nh, int rank, int tid,
-                                  __nv_bfloat16 *__restrict__ ob, float *__restrict__ lseb) {
+                                  float out_scale, __nv_bfloat16 *__restrict__ ob,
+                                  float *__restrict__ lseb) {
     const int hp = (nh + S - 1) / S;
     const int hb = rank * hp, he = min(nh, hb + hp);
     const int c4 = tid & 127;
@@ -172,7 +173,7 @@ DSA_DEVINL void mla_cluster_merge(const TcCtl *ctl, uint32_t sO, int S, int nh, 
             o[2] = fmaf(v[r].z, w, o[2]);
             o[3] = fmaf(v[r].w, w, o[3]);
         }
-        const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
+        const float inv = lsum > 0.f ? out_scale / lsum : 0.f;
         uint2 packed;
         packed.x = pack_bf16x2(o[0] * inv, o[1] * inv);
         packed.y = pack_bf16x2(o[2] * inv, o[3] * inv);
@@ -180,6 +181,18 @@ DSA_DEVINL void mla_cluster_merge(const TcCtl *ctl, uint32_t sO, int S, int nh, 
         if (lseb && c4 == 0)
             lseb[h] = lsum > 0.f ? (M + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
     }
+}
+
+// Two E4M3 values (low byte first) widened to a bf16 pair: through f16, exact
+// for every E4M3 value (at most 4 significant bits, exponents 2^-9 .. 2^8).
+DSA_DEVINL uint32_t e4m3x2_to_bf16x2(uint16_t v) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(v));
+    float lo, hi;
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h2));
+    return pack_bf16x2(lo, hi);
 }
 
 // Where a request's logical token t lives in the latent cache. Contiguous:
@@ -195,13 +208,15 @@ struct KvMap {
     int max_blocks, page;
 };
 
-// kv: the latent cache, kv_rows rows of 512 bf16.
-template <bool kCluster, bool kPaged>
+// kv: the latent cache, kv_rows rows of 512 bf16, or of 512 E4M3 bytes (kFp8:
+// the MMA takes them widened to bf16, which is exact; the cache-wide scale is
+// folded into scale_log2 and out_scale).
+template <bool kCluster, bool kPaged, bool kFp8>
 __global__ void __launch_bounds__(kTcThreads, 1)
-mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restrict__ kv,
+mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_raw,
               const KvMap map, const int32_t *__restrict__ q_req,
               const int32_t *__restrict__ token_ids, int B, int kv_rows, int Hm, int W, int S,
-              int per, float scale_log2, uint8_t *__restrict__ part,
+              int per, float scale_log2, float out_scale, uint8_t *__restrict__ part,
               __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
     extern __shared__ uint8_t mla_smem_raw[];
     const uint32_t raw = smem_u32(mla_smem_raw);
@@ -382,24 +397,62 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
             if (!__all_sync(0xffffffffu, ok)) return false;
             const uint32_t vm = __ballot_sync(0xffffffffu, myrow >= 0);   // bits 0..11
             const uint32_t dst0 = sKV + slot * kSlotRows;
+            if constexpr (!kFp8) {
+                const auto *kv = reinterpret_cast<const __nv_bfloat16 *>(kv_raw);
 #pragma unroll
-            for (int rr = 0; rr < 12; ++rr) {
-                const int r = 12 * sub + rr;                 // row within the chunk
-                const int row = __shfl_sync(0xffffffffu, myrow, rr);
-                const __nv_bfloat16 *src = row >= 0 ? kv + (size_t)row * kL : qm;   // qm: never read
-                const uint32_t nb = row >= 0 ? 16u : 0u;
+                for (int rr = 0; rr < 12; ++rr) {
+                    const int r = 12 * sub + rr;                 // row within the chunk
+                    const int row = __shfl_sync(0xffffffffu, myrow, rr);
+                    const __nv_bfloat16 *src = row >= 0 ? kv + (size_t)row * kL : qm;   // qm: never read
+                    const uint32_t nb = row >= 0 ? 16u : 0u;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int cc = lane + 32 * hh;         // 16-byte piece of the 1 KB row
-                    const uint32_t dst = dst0 + (cc >> 3) * kAtomKV + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
-                    tc::cp_async16_zfill(dst, row >= 0 ? src + cc * 8 : src, nb);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int cc = lane + 32 * hh;         // 16-byte piece of the 1 KB row
+                        const uint32_t dst = dst0 + (cc >> 3) * kAtomKV + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
+                        tc::cp_async16_zfill(dst, row >= 0 ? src + cc * 8 : src, nb);
+                    }
                 }
+                if (lane == 0) {
+                    ctl->vmask[slot][sub] = (uint16_t)vm;
+                    mbar_arrive(&ctl->kv_full[slot]);          // releases this warp's mask
+                }
+                tc::cp_async_arrive_noinc(&ctl->kv_full[slot]);
+            } else {
+                // E4M3 rows of 512 bytes: lane l loads channels 16l..16l+15 of each of
+                // the warp's 12 rows (all loads in flight first), widens them to bf16
+                // exactly and stores the two 16-byte pieces into the swizzled layout.
+                const auto *kv8 = reinterpret_cast<const uint8_t *>(kv_raw);
+                uint4 raw[12];
+#pragma unroll
+                for (int rr = 0; rr < 12; ++rr) {
+                    const int row = __shfl_sync(0xffffffffu, myrow, rr);
+                    raw[rr] = row >= 0 ? ldg_nc_v4(kv8 + (size_t)row * kL + 16 * lane)
+                                       : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int rr = 0; rr < 12; ++rr) {
+                    const int r = 12 * sub + rr;
+                    const uint32_t w[4] = {raw[rr].x, raw[rr].y, raw[rr].z, raw[rr].w};
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int cc = 2 * lane + hh;          // 16-byte piece of the bf16 row
+                        const uint32_t dst = dst0 + (cc >> 3) * kAtomKV + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
+                        const uint32_t a = w[2 * hh], bword = w[2 * hh + 1];
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                                     "r"(e4m3x2_to_bf16x2((uint16_t)(a & 0xFFFFu))),
+                                     "r"(e4m3x2_to_bf16x2((uint16_t)(a >> 16))),
+                                     "r"(e4m3x2_to_bf16x2((uint16_t)(bword & 0xFFFFu))),
+                                     "r"(e4m3x2_to_bf16x2((uint16_t)(bword >> 16)))
+                                     : "memory");
+                    }
+                }
+                tc::fence_proxy_async_smem();               // generic stores -> tensor-core reads
+                if (lane == 0) {
+                    ctl->vmask[slot][sub] = (uint16_t)vm;
+                    mbar_arrive(&ctl->kv_full[slot]);
+                }
+                mbar_arrive(&ctl->kv_full[slot]);            // this lane's rows are in place
             }
-            if (lane == 0) {
-                ctl->vmask[slot][sub] = (uint16_t)vm;
-                mbar_arrive(&ctl->kv_full[slot]);          // releases this warp's mask
-            }
-            tc::cp_async_arrive_noinc(&ctl->kv_full[slot]);
             return true;
         };
         bool go = true;
@@ -636,7 +689,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
                 for (int j = 0; j < 32; ++j) {
                     const int h = (blk & 1) * 32 + j;
                     const float lh = ctl->lsum[h];
-                    const float v = (have_o && lh > 0.f) ? __uint_as_float(o[j]) / lh : 0.f;
+                    const float v = (have_o && lh > 0.f) ? __uint_as_float(o[j]) / lh * out_scale : 0.f;
                     if (h < nh) ob[(size_t)h * kL + L] = __float2bfloat16_rn(v);
                 }
             }
@@ -647,7 +700,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
     if constexpr (kCluster) {
         cluster_sync_all();           // every split's m, l and O^T are in place
         if (tid < 256)
-            mla_cluster_merge(ctl, sKV, S, nh, split, tid, out + ((size_t)qi * Hm + h0) * kL,
+            mla_cluster_merge(ctl, sKV, S, nh, split, tid, out_scale, out + ((size_t)qi * Hm + h0) * kL,
                               lse ? lse + (size_t)qi * Hm + h0 : nullptr);
         cluster_sync_all();           // no CTA leaves while a peer still reads it
     }
@@ -659,8 +712,8 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const __nv_bfloat16 *__restr
 // more splits take a first round for the maxima. Splits are merged in split
 // order (deterministic).
 __global__ void __launch_bounds__(128)
-mla_combine_kernel(const uint8_t *__restrict__ part, int Hm, int S, __nv_bfloat16 *__restrict__ out,
-                   float *__restrict__ lse) {
+mla_combine_kernel(const uint8_t *__restrict__ part, int Hm, int S, float out_scale,
+                   __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
     constexpr int kRound = 16;
     const int h = blockIdx.x, q = blockIdx.y, tid = threadIdx.x;
     pdl_wait();
@@ -720,7 +773,7 @@ mla_combine_kernel(const uint8_t *__restrict__ part, int Hm, int S, __nv_bfloat1
             }
         }
     }
-    const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
+    const float inv = lsum > 0.f ? out_scale / lsum : 0.f;
     uint2 packed;
     packed.x = pack_bf16x2(o[0] * inv, o[1] * inv);
     packed.y = pack_bf16x2(o[2] * inv, o[3] * inv);
@@ -750,7 +803,7 @@ inline int mla_max_clusters(int splits) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel<true, false>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel<true, false, false>, &cfg) != cudaSuccess) n = 0;
     (void)cudaGetLastError();
     known[dev][splits].store(n + 1, std::memory_order_relaxed);
     return n;
@@ -779,23 +832,24 @@ inline MlaGeom mla_launch_geometry(int Q, int Hm, int W) {
 // split kernel, plus the combine when the splits merge through the workspace.
 inline int sparse_mla_launch_count(int Q, int Hm, int W) {
     if (Q <= 0 || Hm <= 0 || W < 0) return 0;
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, false>), kTcSmemBytes))
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, false, false>), kTcSmemBytes))
         return 0;
     const MlaGeom g = mla_launch_geometry(Q, Hm, W);
     return (g.S > 1 && !g.cluster) ? 2 : 1;
 }
 
-template <bool kPaged>
+template <bool kPaged, bool kFp8>
 inline int sparse_mla_launch_map(const void *q, const void *kv, int64_t kv_rows, const KvMap &map,
-                                 const int32_t *q_req, const int32_t *token_ids, int Q, int B,
-                                 int Hm, int W, int kv_lora, int rope_dim, float sm_scale,
-                                 void *out, float *lse, void *ws, size_t ws_bytes,
+                                 float kv_scale, const int32_t *q_req, const int32_t *token_ids,
+                                 int Q, int B, int Hm, int W, int kv_lora, int rope_dim,
+                                 float sm_scale, void *out, float *lse, void *ws, size_t ws_bytes,
                                  cudaStream_t stream) {
     if (Q < 0 || B < 0 || Hm <= 0 || W < 0 || kv_lora <= 0 || rope_dim < 0 || kv_rows < 0)
         return DSA_ERR_INVALID_ARG;
     if (!(sm_scale == sm_scale) || sm_scale == INFINITY || sm_scale == -INFINITY)
         return DSA_ERR_INVALID_ARG;
     if (kPaged && (map.page <= 0 || map.max_blocks < 0)) return DSA_ERR_INVALID_ARG;
+    if (kFp8 && !(kv_scale > 0.f && kv_scale < INFINITY)) return DSA_ERR_INVALID_ARG;
     if (kv_lora != kL || rope_dim != 0 || Hm % 16 != 0 || Hm > DSA_MAX_MLA_HEADS)
         return DSA_ERR_UNSUPPORTED;
     if (kv_rows > (int64_t)INT32_MAX) return DSA_ERR_UNSUPPORTED;   // rows are 32-bit indices
@@ -811,33 +865,35 @@ inline int sparse_mla_launch_map(const void *q, const void *kv, int64_t kv_rows,
         return DSA_ERR_ALIGNMENT;
     const size_t need = mla_workspace_bytes(Q, Hm, W);
     if (need > 0 && (!ws || ws_bytes < need)) return DSA_ERR_WORKSPACE;
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, kPaged>), kTcSmemBytes) ||
-        !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<false, kPaged>), kTcSmemBytes) ||
-        !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, false>), kTcSmemBytes))
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, kPaged, kFp8>), kTcSmemBytes) ||
+        !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<false, kPaged, kFp8>), kTcSmemBytes) ||
+        !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, false, false>), kTcSmemBytes))
         return DSA_ERR_CUDA;
     const MlaGeom g = mla_launch_geometry(Q, Hm, W);
-    const float scale_log2 = sm_scale * 1.4426950408889634f;
+    // fp8: S = sm_scale * q . (s k8) = (sm_scale * s) q . k8, and O = s * (P V8)
+    const float out_scale = kFp8 ? kv_scale : 1.0f;
+    const float scale_log2 = (kFp8 ? sm_scale * kv_scale : sm_scale) * 1.4426950408889634f;
     const int groups = (Hm + kTcHeads - 1) / kTcHeads;
     auto *part = reinterpret_cast<uint8_t *>(ws);
     const auto *qb = reinterpret_cast<const __nv_bfloat16 *>(q);
-    const auto *kvb = reinterpret_cast<const __nv_bfloat16 *>(kv);
     auto *ob = reinterpret_cast<__nv_bfloat16 *>(out);
     const dim3 grid(g.S, Q, groups);
     if (g.cluster) {
-        if (launch_pdl_cluster(mla_tc_kernel<true, kPaged>, grid, dim3(kTcThreads), kTcSmemBytes,
-                               stream, g.S, qb, kvb, map, q_req, token_ids, B, (int)kv_rows, Hm,
-                               W, g.S, g.per, scale_log2, part, ob, lse) != cudaSuccess)
+        if (launch_pdl_cluster(mla_tc_kernel<true, kPaged, kFp8>, grid, dim3(kTcThreads),
+                               kTcSmemBytes, stream, g.S, qb, kv, map, q_req, token_ids, B,
+                               (int)kv_rows, Hm, W, g.S, g.per, scale_log2, out_scale, part, ob,
+                               lse) != cudaSuccess)
             return DSA_ERR_CUDA;
         return launch_status();
     }
-    if (launch_pdl(mla_tc_kernel<false, kPaged>, grid, dim3(kTcThreads), kTcSmemBytes, stream, qb,
-                   kvb, map, q_req, token_ids, B, (int)kv_rows, Hm, W, g.S, g.per, scale_log2,
-                   part, ob, lse) != cudaSuccess)
+    if (launch_pdl(mla_tc_kernel<false, kPaged, kFp8>, grid, dim3(kTcThreads), kTcSmemBytes,
+                   stream, qb, kv, map, q_req, token_ids, B, (int)kv_rows, Hm, W, g.S, g.per,
+                   scale_log2, out_scale, part, ob, lse) != cudaSuccess)
         return DSA_ERR_CUDA;
     int st = launch_status();
     if (st != DSA_OK || g.S == 1) return st;
-    if (launch_pdl(mla_combine_kernel, dim3(Hm, Q), dim3(128), 0, stream, part, Hm, g.S, ob,
-                   lse) != cudaSuccess)
+    if (launch_pdl(mla_combine_kernel, dim3(Hm, Q), dim3(128), 0, stream, part, Hm, g.S,
+                   out_scale, ob, lse) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
 }
@@ -848,9 +904,9 @@ inline int sparse_mla_launch(const void *q, const void *kv, int64_t kv_rows,
                              int rope_dim, float sm_scale, void *out, float *lse, void *ws,
                              size_t ws_bytes, cudaStream_t stream) {
     const KvMap map{req_start, nullptr, nullptr, 0, 1};
-    return sparse_mla_launch_map<false>(q, kv, kv_rows, map, q_req, token_ids, Q, B, Hm, W,
-                                        kv_lora, rope_dim, sm_scale, out, lse, ws, ws_bytes,
-                                        stream);
+    return sparse_mla_launch_map<false, false>(q, kv, kv_rows, map, 1.0f, q_req, token_ids, Q, B,
+                                               Hm, W, kv_lora, rope_dim, sm_scale, out, lse, ws,
+                                               ws_bytes, stream);
 }
 
 inline int sparse_mla_launch_paged(const void *q, const void *kv, int64_t kv_rows,
@@ -860,8 +916,21 @@ inline int sparse_mla_launch_paged(const void *q, const void *kv, int64_t kv_row
                                    int kv_lora, int rope_dim, float sm_scale, void *out, float *lse,
                                    void *ws, size_t ws_bytes, cudaStream_t stream) {
     const KvMap map{nullptr, block_table, seq_len, max_blocks, page_size};
-    return sparse_mla_launch_map<true>(q, kv, kv_rows, map, q_req, token_ids, Q, B, Hm, W,
-                                       kv_lora, rope_dim, sm_scale, out, lse, ws, ws_bytes, stream);
+    return sparse_mla_launch_map<true, false>(q, kv, kv_rows, map, 1.0f, q_req, token_ids, Q, B,
+                                              Hm, W, kv_lora, rope_dim, sm_scale, out, lse, ws,
+                                              ws_bytes, stream);
+}
+
+inline int sparse_mla_launch_paged_fp8(const void *q, const void *kv8, float kv_scale,
+                                       int64_t kv_rows, const int32_t *block_table, int max_blocks,
+                                       int page_size, const int32_t *seq_len, const int32_t *q_req,
+                                       const int32_t *token_ids, int Q, int B, int Hm, int W,
+                                       int kv_lora, int rope_dim, float sm_scale, void *out,
+                                       float *lse, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    const KvMap map{nullptr, block_table, seq_len, max_blocks, page_size};
+    return sparse_mla_launch_map<true, true>(q, kv8, kv_rows, map, kv_scale, q_req, token_ids, Q,
+                                             B, Hm, W, kv_lora, rope_dim, sm_scale, out, lse, ws,
+                                             ws_bytes, stream);
 }
 
 }  // namespace dsa

@@ -214,6 +214,30 @@ def test_sparse_mla_refusals(B):
     assert call(Q=0) == B.DSA_OK
 
 
+def test_paged_mla_refusals(B):
+    L = B.lib
+    # q, kv, kv_rows, table, max_blocks, page, seq_len, q_req, ids, Q, B, Hm, W, lora, rope, scale,
+    # out, lse, ws, ws_bytes, stream
+    args = [FAKE, FAKE, 1024, FAKE, 8, 16, FAKE, FAKE, FAKE, 2, 2, 64, 64, 512, 0, 0.04, FAKE,
+            FAKE, FAKE, 1 << 30, None]
+    bad = list(args); bad[5] = 0
+    assert L.dsa_sparse_mla_decode_paged(*bad) == B.DSA_ERR_INVALID_ARG      # page size 0
+    bad = list(args); bad[4] = -1
+    assert L.dsa_sparse_mla_decode_paged(*bad) == B.DSA_ERR_INVALID_ARG
+    bad = list(args); bad[6] = None
+    assert L.dsa_sparse_mla_decode_paged(*bad) == B.DSA_ERR_INVALID_ARG      # no seq_len
+    bad = list(args); bad[3] = FAKE + 2
+    assert L.dsa_sparse_mla_decode_paged(*bad) == B.DSA_ERR_ALIGNMENT
+    bad = list(args); bad[13] = 576
+    assert L.dsa_sparse_mla_decode_paged(*bad) == B.DSA_ERR_UNSUPPORTED
+    fp8 = args[:2] + [0.5] + args[2:]
+    for s in (0.0, -1.0, float("inf"), float("nan")):
+        bad = list(fp8); bad[2] = s
+        assert L.dsa_sparse_mla_decode_paged_fp8(*bad) == B.DSA_ERR_INVALID_ARG
+    bad = list(fp8); bad[10] = 0
+    assert L.dsa_sparse_mla_decode_paged_fp8(*bad) == B.DSA_OK               # Q == 0
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     """The binding has no fallback: without libdsa.so the import raises."""
     import importlib.util

@@ -1,4 +1,4 @@
-"""Sparse MLA over a block-table paged latent cache on the GPU.
+"""Sparse MLA over a block-table paged latent cache (bf16 or fp8 E4M3) on the GPU.
 
 The same rows stored in pages at scattered places must give the contiguous
 call's results bit for bit (the kernels differ only in the row lookup); ids on
@@ -103,4 +103,76 @@ def test_paged_missing_pages_and_short_sequences(B):
     vb = mla_value_bound(wl.kv, wl.req_start, wl.q_req, ids)
     assert_mla_close(out, ref_out, lse, ref_lse, vbound=vb)
     assert np.isfinite(W.bf16_bits_to_f32(out)).all()    # no NaN page was read
+    device_status_clean(B)
+
+
+def _fp8_cache(wl, rng):
+    """An E4M3 latent cache of the workload's shape (no NaN codes)."""
+    kv8 = rng.integers(0, 256, size=wl.kv.shape).astype(np.uint8)
+    kv8[(kv8 & 0x7F) == 0x7F] = 0x3C
+    return kv8
+
+
+def _paged_call_fp8(B, step, pool8, scale, table, seq_len, page):
+    g, t = step.g, step.t
+    out = torch.empty_like(step.out)
+    lse = torch.empty_like(step.lse)
+    ws = torch.empty(max(16, B.dsa_sparse_mla_workspace_size(g.Q, g.hm, g.W)), dtype=torch.uint8,
+                     device="cuda")
+    B.dsa_sparse_mla_decode_paged_fp8(
+        t["q_mla"], torch.from_numpy(pool8).cuda(), scale, pool8.shape[0],
+        torch.from_numpy(table).cuda(), table.shape[1], page, torch.from_numpy(seq_len).cuda(),
+        t["q_req"], step.token_ids, g.Q, g.B, g.hm, g.W, 512, 0, g.sm_scale, out, lse, ws,
+        ws.numel())
+    torch.cuda.synchronize()
+    return out.view(torch.int16).cpu().numpy().view(np.uint16), lse.cpu().numpy()
+
+
+@pytest.mark.parametrize("name,page", [("tiny", 16), ("batched", 64)])
+def test_paged_fp8_against_oracle_and_bf16(B, name, page):
+    from sparse_attention_indexer_head_b200.pipeline import DecodeStep
+    wl = W.make(name)
+    rng = np.random.default_rng(31)
+    kv8 = _fp8_cache(wl, rng)
+    step = DecodeStep(wl)
+    step.run()
+    torch.cuda.synchronize()
+    ids = step.token_ids.cpu().numpy()
+    # the same fp8 rows scattered over pages (unused pages hold NaN codes)
+    lengths = [int(x) for x in np.diff(wl.req_start)]
+    n_pages = [(t + page - 1) // page for t in lengths]
+    total = sum(n_pages) + 2
+    perm = rng.permutation(total)
+    pool8 = np.full((total * page, 512), 0x7F, np.uint8)
+    table = np.full((wl.B, max(n_pages) + 1), -1, np.int32)
+    k = 0
+    for b, T in enumerate(lengths):
+        for pi in range(n_pages[b]):
+            blk = int(perm[k]); k += 1
+            table[b, pi] = blk
+            rows = kv8[wl.req_start[b] + pi * page: wl.req_start[b] + min(T, (pi + 1) * page)]
+            pool8[blk * page: blk * page + len(rows)] = rows
+    seq_len = np.asarray(lengths, np.int32)
+    # a scale that is not a power of two: against the oracle
+    out, lse = _paged_call_fp8(B, step, pool8, 0.37, table, seq_len, page)
+    ref_out, ref_lse = O.sparse_mla_fp8(wl.q_mla, kv8, 0.37, wl.req_start, wl.q_req, ids,
+                                        wl.sm_scale)
+    dec = np.array([O.f64_from_e4m3(c) for c in range(256)])
+    vb = mla_value_bound(0.37 * dec[kv8], wl.req_start, wl.q_req, ids)
+    assert_mla_close(out, ref_out, lse, ref_lse, vbound=vb)
+    assert np.isfinite(W.bf16_bits_to_f32(out)).all()
+    # a power-of-two scale: bit-identical to the bf16 kernel on the decoded, scaled cache
+    kv_b = W.f32_to_bf16_bits((0.5 * dec[kv8]).astype(np.float32))
+    pool_b = np.zeros((pool8.shape[0], 512), np.uint16)
+    used = table[table >= 0]
+    for b, T in enumerate(lengths):
+        for pi in range(n_pages[b]):
+            blk = table[b, pi]
+            rows = kv_b[wl.req_start[b] + pi * page: wl.req_start[b] + min(T, (pi + 1) * page)]
+            pool_b[blk * page: blk * page + len(rows)] = rows
+    out8, lse8 = _paged_call_fp8(B, step, pool8, 0.5, table, seq_len, page)
+    outb, lseb = _paged_call(B, step, pool_b, table, seq_len, page)
+    np.testing.assert_array_equal(out8, outb)
+    np.testing.assert_array_equal(lse8, lseb)
+    assert used.size == sum(n_pages)
     device_status_clean(B)
