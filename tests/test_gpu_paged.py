@@ -106,11 +106,11 @@ def test_paged_missing_pages_and_short_sequences(B):
     device_status_clean(B)
 
 
-def _fp8_cache(wl, rng):
-    """An E4M3 latent cache of the workload's shape (no NaN codes)."""
-    kv8 = rng.integers(0, 256, size=wl.kv.shape).astype(np.uint8)
-    kv8[(kv8 & 0x7F) == 0x7F] = 0x3C
-    return kv8
+def _fp8_cache(wl, scale):
+    """The workload's latent cache quantised to E4M3 codes for the given scale (input
+    generation: torch's float8_e4m3fn cast of kv / scale)."""
+    x = torch.from_numpy(W.bf16_bits_to_f32(wl.kv)) / scale
+    return x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
 
 
 def _paged_call_fp8(B, step, pool8, scale, table, seq_len, page):
@@ -133,7 +133,7 @@ def test_paged_fp8_against_oracle_and_bf16(B, name, page):
     from sparse_attention_indexer_head_b200.pipeline import DecodeStep
     wl = W.make(name)
     rng = np.random.default_rng(31)
-    kv8 = _fp8_cache(wl, rng)
+    kv8 = _fp8_cache(wl, 0.37)
     step = DecodeStep(wl)
     step.run()
     torch.cuda.synchronize()
