@@ -29,9 +29,10 @@ constexpr int kScoreSmem = 2 * kScoreKeyAtom + 2 * kScoreQAtom + 1024;   // + al
 // as 8 tcgen05 MMAs (M=128, N=16, K=16) into tensor memory. Both operands come
 // in by 2-D TMA tile loads into the 128B-swizzled K-major layout (two 64-channel
 // atoms each). Thread t then owns pool p0+t: it reads its 16 head dots from
-// tensor memory and adds g_h * relu(dot_h) over h in order. Tiles with no
-// candidate pool skip the loads and MMAs. Keys of non-candidates inside a tile
-// are read (one 32 KB box) but do not enter any score.
+// tensor memory and adds g_h * relu(dot_h) over h in order. The key tile is
+// requested right after the dependency wait, before the candidate flags are
+// known; tiles with no candidate pool skip the MMAs. Keys of non-candidates
+// inside a tile are read (one 32 KB box) but do not enter any score.
 __global__ void __launch_bounds__(kScoreThreads)
 index_scores_kernel(const __grid_constant__ CUtensorMap key_map,
                     const __grid_constant__ CUtensorMap q_map, const float *__restrict__ gate_w,
@@ -68,9 +69,17 @@ index_scores_kernel(const __grid_constant__ CUtensorMap key_map,
     }
     pdl_wait();
     pdl_launch_dependents();
-
     const int b = q_req[q];
     const bool req_ok = b >= 0 && b < B;
+    if (tid == 0 && req_ok) {
+        // The key tile (written by the predecessor) is requested at once, while
+        // the candidate flags are read; rows past the key map read as zeros.
+        mbar_arrive_expect_tx(&load_bar, 2 * kScoreKeyAtom);
+        const int row = b * max_pools + p0;
+        tma_load_2d(sK, &key_map, 0, row, &load_bar);
+        tma_load_2d(sK + kScoreKeyAtom, &key_map, 64, row, &load_bar);
+    }
+
     bool is_cand = false;
     if (req_ok && p < max_pools) {
         const long long last = (long long)first_valid[b] + (long long)p * kpool + kpool - 1;
@@ -88,10 +97,6 @@ index_scores_kernel(const __grid_constant__ CUtensorMap key_map,
     bool ok = true;
     if (any) {
         if (tid == 0) {
-            mbar_arrive_expect_tx(&load_bar, 2 * kScoreKeyAtom);
-            const int row = b * max_pools + p0;
-            tma_load_2d(sK, &key_map, 0, row, &load_bar);
-            tma_load_2d(sK + kScoreKeyAtom, &key_map, 64, row, &load_bar);
             ok = mbar_wait(&load_bar, 0) && mbar_wait(&q_bar, 0);
             if (ok) {
                 tc::fence_after_sync();
@@ -112,7 +117,10 @@ index_scores_kernel(const __grid_constant__ CUtensorMap key_map,
         tc::fence_after_sync();
     }
 
-    if (!any && tid == 0) (void)mbar_wait(&q_bar, 0);   // the query rows land before the CTA leaves
+    if (!any && tid == 0) {   // every copy lands before the CTA leaves
+        (void)mbar_wait(&q_bar, 0);
+        if (req_ok) (void)mbar_wait(&load_bar, 0);
+    }
 
     float score = -INFINITY;
     if (any && ok) {
