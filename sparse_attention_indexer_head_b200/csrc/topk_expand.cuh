@@ -75,12 +75,11 @@ struct TailArgs {
 __global__ void __launch_bounds__(kTopkThreads)
 topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__ cand,
                    const int32_t *__restrict__ pool_idx, const int32_t *__restrict__ q_req, int B,
-                   int P, int KP, int K, int keys_in_smem, int idx_in_smem, TailArgs tail,
+                   int P, int KP, int K, int keys_in_smem, TailArgs tail,
                    int32_t *__restrict__ top_pools, int32_t *__restrict__ token_ids) {
     extern __shared__ __align__(16) uint8_t topk_smem[];
     int32_t *slist = reinterpret_cast<int32_t *>(topk_smem);                  // [K] selected ids
     uint32_t *skeys = reinterpret_cast<uint32_t *>(topk_smem) + K;           // [P] if cached
-    int32_t *sidx = reinterpret_cast<int32_t *>(skeys + P);                   // [P * KP] if cached
     __shared__ int hist[2][256];          // double-buffered radix histograms
     __shared__ int2 s_warp2[kTopkWarps];
     __shared__ int s_pick[2][3];          // per pass parity: (digit, count above it, count in it)
@@ -113,12 +112,6 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
         s_nsmall = 0;
     }
     __syncthreads();
-    // The request's pool_idx rows, when cached, load beside the keys so the
-    // expansion at the end reads shared memory instead of gathering from L2.
-    if (idx_in_smem && req_ok) {
-        const int32_t *irow = pool_idx + (size_t)b * P * KP;
-        for (int e = tid; e < P * KP; e += kTopkThreads) sidx[e] = __ldg(irow + e);
-    }
     int cnt = 0;
     for (int p0 = 0; p0 < P; p0 += 4 * kTopkThreads) {
         float sv[4];
@@ -304,8 +297,7 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
             const int e = e0 + tid + u * kTopkThreads;
             const int j = e / KP, s = e - j * KP;
             v[u] = -1;
-            if (e < K * KP && j < nq)
-                v[u] = idx_in_smem ? sidx[slist[j] * KP + s] : pool_idx[((size_t)b * P + slist[j]) * KP + s];
+            if (e < K * KP && j < nq) v[u] = pool_idx[((size_t)b * P + slist[j]) * KP + s];
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -332,15 +324,12 @@ inline int topk_expand_launch(const float *scores, const uint8_t *cand, const in
         !aligned(tail.first_valid, 4) || !aligned(tail.req_start, 4))
         return DSA_ERR_ALIGNMENT;
     const int keys_in_smem = max_pools <= kTopkSmemKeys ? 1 : 0;
-    // pool_idx rows cached too when they fit in 64 KB (e.g. 2048 pools of 4 or 8 slots)
-    const int idx_in_smem = keys_in_smem && (long long)max_pools * kpool * 4 <= (64 << 10) ? 1 : 0;
-    const int smem = select_k * 4 + (keys_in_smem ? max_pools * 4 : 0) +
-                     (idx_in_smem ? max_pools * kpool * 4 : 0);
+    const int smem = select_k * 4 + (keys_in_smem ? max_pools * 4 : 0);
     if (!ensure_smem_attr(reinterpret_cast<const void *>(topk_expand_kernel), smem))
         return DSA_ERR_CUDA;
     if (launch_pdl(topk_expand_kernel, dim3(Q), dim3(kTopkThreads), smem, stream, scores, cand,
-                   pool_idx, q_req, B, max_pools, kpool, select_k, keys_in_smem, idx_in_smem, tail,
-                   top_pools, token_ids) != cudaSuccess)
+                   pool_idx, q_req, B, max_pools, kpool, select_k, keys_in_smem, tail, top_pools,
+                   token_ids) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
 }
