@@ -68,10 +68,21 @@ def _paged_call(B, step, pool, table, seq_len, page):
     return out.view(torch.int16).cpu().numpy().view(np.uint16), lse.cpu().numpy()
 
 
-@pytest.mark.parametrize("name,page", [("tiny", 16), ("tiny", 7), ("tiny", 1), ("batched", 64)])
+def _workload(name):
+    if name == "cluster":
+        # 32 decode queries: each query's ids split 4 ways and merge inside a cluster
+        lengths = [600 + 37 * i for i in range(32)]
+        return W.build("cluster", lengths=lengths, pads=[i % 5 for i in range(32)], kpool=4,
+                       max_pools=(max(lengths) + 3) // 4, select_k=512, hm=64,
+                       q_req=list(range(32)), q_pos=[t - 1 for t in lengths], seed=17)
+    return W.make(name)
+
+
+@pytest.mark.parametrize("name,page", [("tiny", 16), ("tiny", 7), ("tiny", 1), ("batched", 64),
+                                       ("cluster", 32)])
 def test_paged_equals_contiguous(B, name, page):
     from sparse_attention_indexer_head_b200.pipeline import DecodeStep
-    wl = W.make(name)
+    wl = _workload(name)
     step = DecodeStep(wl)
     step.run()
     torch.cuda.synchronize()
@@ -128,10 +139,10 @@ def _paged_call_fp8(B, step, pool8, scale, table, seq_len, page):
     return out.view(torch.int16).cpu().numpy().view(np.uint16), lse.cpu().numpy()
 
 
-@pytest.mark.parametrize("name,page", [("tiny", 16), ("batched", 64)])
+@pytest.mark.parametrize("name,page", [("tiny", 16), ("batched", 64), ("cluster", 32)])
 def test_paged_fp8_against_oracle_and_bf16(B, name, page):
     from sparse_attention_indexer_head_b200.pipeline import DecodeStep
-    wl = W.make(name)
+    wl = _workload(name)
     rng = np.random.default_rng(31)
     kv8 = _fp8_cache(wl, 0.37)
     step = DecodeStep(wl)
@@ -176,3 +187,9 @@ def test_paged_fp8_against_oracle_and_bf16(B, name, page):
     np.testing.assert_array_equal(lse8, lseb)
     assert used.size == sum(n_pages)
     device_status_clean(B)
+
+
+def test_cluster_workload_takes_the_cluster_path(B):
+    """The 32-query case above merges its splits inside clusters: one MLA launch."""
+    assert B.dsa_sparse_mla_launch_count(32, 64, 2048) == 1
+    assert B.dsa_sparse_mla_workspace_size(32, 64, 2048) > 0      # sized for the global plan
