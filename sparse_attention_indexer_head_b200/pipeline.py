@@ -225,3 +225,80 @@ class DecodeStep:
             "out": u16(self.out),
             "lse": self.lse.cpu().numpy(),
         }
+
+
+class StreamedDecode:
+    """Decode steps served from and to pinned host memory, overlapped across steps.
+
+    Each step copies its query inputs host -> device, runs the five calls
+    (replayed from a CUDA graph captured once per slot) and copies the output
+    device -> host. The three run on their own streams and the steps rotate over
+    `slots` device buffer sets, so step i's copies overlap the compute of its
+    neighbours; events keep a slot's inputs and output from being overwritten
+    while still in use. `submit` enqueues a step; `result(i)` waits for step
+    i's output to reach the host and returns it (the slot's pinned buffer,
+    valid until that slot is submitted again).
+    """
+
+    def __init__(self, wl: Workload, device: str = "cuda", slots: int = 2,
+                 inputs: Optional[Dict] = None):
+        self.device = torch.device(device)
+        self.steps = [DecodeStep(wl, device=device, inputs=inputs) for _ in range(slots)]
+        self.s_in = torch.cuda.Stream(device=self.device)
+        self.s_run = torch.cuda.Stream(device=self.device)
+        self.s_out = torch.cuda.Stream(device=self.device)
+        self.graphs = []
+        with torch.cuda.stream(self.s_run):
+            for st in self.steps:
+                st.run()                                  # sets kernel attributes eagerly
+        self.s_run.synchronize()
+        for st in self.steps:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.s_run):
+                st.run()
+            self.graphs.append(g)
+        torch.cuda.synchronize(self.device)
+        n = len(self.steps)
+        self.in_done = [torch.cuda.Event() for _ in range(n)]
+        self.run_done = [torch.cuda.Event() for _ in range(n)]
+        self.out_done = [torch.cuda.Event() for _ in range(n)]
+        self.out_host = [torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+                         for st in self.steps]
+        self.submitted = 0
+
+    def submit(self, host_inputs: Dict[str, torch.Tensor]) -> int:
+        """Enqueue one step on pinned host inputs (names of QUERY_INPUTS); returns its index."""
+        i = self.submitted
+        k = i % len(self.steps)
+        st = self.steps[k]
+        # inputs: after the slot's previous step has finished reading them
+        self.s_in.wait_event(self.run_done[k])
+        with torch.cuda.stream(self.s_in):
+            for name, v in host_inputs.items():
+                st.t[name].copy_(v, non_blocking=True)
+        self.in_done[k].record(self.s_in)
+        # compute: after its inputs landed and the slot's previous output left
+        self.s_run.wait_event(self.in_done[k])
+        self.s_run.wait_event(self.out_done[k])
+        with torch.cuda.stream(self.s_run):
+            self.graphs[k].replay()
+        self.run_done[k].record(self.s_run)
+        # output back to the host
+        self.s_out.wait_event(self.run_done[k])
+        with torch.cuda.stream(self.s_out):
+            self.out_host[k].copy_(st.out, non_blocking=True)
+        self.out_done[k].record(self.s_out)
+        self.submitted += 1
+        return i
+
+    def result(self, i: int) -> torch.Tensor:
+        """Step i's output [Q, Hm, 512] bf16 on the host (step i must be among the
+        last `slots` submitted)."""
+        if not (self.submitted - len(self.steps) <= i < self.submitted):
+            raise ValueError("step is not among the slots in flight")
+        k = i % len(self.steps)
+        self.out_done[k].synchronize()
+        return self.out_host[k]
+
+    def kernels_per_step(self) -> int:
+        return self.steps[0].kernels_per_step()
