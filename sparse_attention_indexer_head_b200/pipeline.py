@@ -230,7 +230,8 @@ class DecodeStep:
 class StreamedDecode:
     """Decode steps served from and to pinned host memory, overlapped across steps.
 
-    Each step copies its query inputs host -> device, runs the five calls
+    Each step copies its query inputs host -> device (one copy of a packed
+    pinned buffer), runs the five calls
     (replayed from a CUDA graph captured once per slot) and copies the output
     device -> host. The three run on their own streams and the steps rotate over
     `slots` device buffer sets, so step i's copies overlap the compute of its
@@ -244,6 +245,23 @@ class StreamedDecode:
                  inputs: Optional[Dict] = None):
         self.device = torch.device(device)
         self.steps = [DecodeStep(wl, device=device, inputs=inputs) for _ in range(slots)]
+        # A slot's query inputs live in one device buffer, so a step's inputs are
+        # one host-to-device copy from a packed pinned buffer (see pack()).
+        self.layout, nbytes = {}, 0
+        for name in QUERY_INPUTS:
+            t = self.steps[0].t[name]
+            nbytes = (nbytes + 255) // 256 * 256
+            self.layout[name] = (nbytes, t.dtype, tuple(t.shape))
+            nbytes += t.numel() * t.element_size()
+        self.nbytes = nbytes
+        self.dev_in = []
+        for st in self.steps:
+            buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+            for name, (off, dtype, shape) in self.layout.items():
+                view = self._view(buf, off, dtype, shape)
+                view.copy_(st.t[name])
+                st.t[name] = view
+            self.dev_in.append(buf)
         self.s_in = torch.cuda.Stream(device=self.device)
         self.s_run = torch.cuda.Stream(device=self.device)
         self.s_out = torch.cuda.Stream(device=self.device)
@@ -266,17 +284,31 @@ class StreamedDecode:
                          for st in self.steps]
         self.submitted = 0
 
-    def submit(self, host_inputs: Dict[str, torch.Tensor]) -> int:
-        """Enqueue one step on pinned host inputs (names of QUERY_INPUTS); returns its index."""
+    @staticmethod
+    def _view(buf: torch.Tensor, off: int, dtype, shape) -> torch.Tensor:
+        n = 1
+        for d in shape:
+            n *= d
+        size = n * torch.empty((), dtype=dtype).element_size()
+        return buf[off:off + size].view(dtype).view(shape)
+
+    def pack(self, host_inputs: Dict[str, torch.Tensor]) -> torch.Tensor:
+        """The query inputs (names of QUERY_INPUTS) packed into one pinned buffer."""
+        out = torch.empty(self.nbytes, dtype=torch.uint8).pin_memory()
+        for name, (off, dtype, shape) in self.layout.items():
+            self._view(out, off, dtype, shape).copy_(host_inputs[name])
+        return out
+
+    def submit(self, packed: torch.Tensor) -> int:
+        """Enqueue one step on pinned packed inputs (from pack()); returns its index."""
         i = self.submitted
         k = i % len(self.steps)
-        st = self.steps[k]
         # inputs: after the slot's previous step has finished reading them
         self.s_in.wait_event(self.run_done[k])
         with torch.cuda.stream(self.s_in):
-            for name, v in host_inputs.items():
-                st.t[name].copy_(v, non_blocking=True)
+            self.dev_in[k].copy_(packed, non_blocking=True)
         self.in_done[k].record(self.s_in)
+        st = self.steps[k]
         # compute: after its inputs landed and the slot's previous output left
         self.s_run.wait_event(self.in_done[k])
         self.s_run.wait_event(self.out_done[k])

@@ -344,9 +344,10 @@ def test_streamed_decode_matches_eager_steps(B):
         torch.cuda.synchronize()
         ref.append(st.out.view(torch.int16).cpu().numpy())
     sd = StreamedDecode(wl_a, slots=2)
+    packed = [sd.pack(q) for q in ins]
     got = []
     for i in range(7):
-        sd.submit(ins[i % 2])
+        sd.submit(packed[i % 2])
         if i >= 1:
             got.append(sd.result(i - 1).view(torch.int16).numpy().copy())
     got.append(sd.result(6).view(torch.int16).numpy().copy())
