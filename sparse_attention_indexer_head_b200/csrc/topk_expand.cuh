@@ -4,10 +4,10 @@
 // sentinel row written in full).
 //
 // One CTA per query. Scores become order-preserving uint32 keys (candidates
-// only; -0 folded onto +0, NaN onto -inf, non-candidates 0). An MSB radix
-// select finds the n_q-th largest key tau exactly: 8-bit digits from the
-// highest bit where the candidate keys differ, until at most 32 keys share
-// the bits fixed so far, which one warp then ranks; the winners are
+// only; -0 folded onto +0, NaN onto -inf, non-candidates 0). An 8-bit MSB
+// radix select finds the n_q-th largest key tau exactly: two passes, then,
+// when at most 32 keys share those 16 bits with tau, a rank among them on one
+// warp, else two more passes; the winners are
 // every key above tau plus the lowest-id keys equal to tau (an id-ordered
 // block scan), written in ascending pool id, so the result is bit-exact and
 // deterministic. The expansion gathers pool_idx rows and writes every slot of
@@ -84,7 +84,7 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     __shared__ int2 s_warp2[kTopkWarps];
     __shared__ int s_pick[2][3];          // per pass parity: (digit, count above it, count in it)
     __shared__ int s_ncand, s_nsmall, s_req;
-    __shared__ uint32_t s_small[32], s_tau, s_kmin, s_kmax;
+    __shared__ uint32_t s_small[32], s_tau;
 
     const int tid = threadIdx.x;
     const int q = blockIdx.x;
@@ -101,8 +101,8 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     };
 
     // Keys: four loads of each array in flight per thread before any use; the
-    // candidate count and the smallest and largest candidate key are taken on
-    // the way.
+    // histogram of the top byte (the first radix pass) and the candidate count
+    // are built on the way.
     if (tid < 256) {
         hist[0][tid] = 0;
         hist[1][tid] = 0;
@@ -110,12 +110,9 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     if (tid == 0) {
         s_ncand = 0;
         s_nsmall = 0;
-        s_kmin = 0xFFFFFFFFu;
-        s_kmax = 0u;
     }
     __syncthreads();
     int cnt = 0;
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
     for (int p0 = 0; p0 < P; p0 += 4 * kTopkThreads) {
         float sv[4];
         uint8_t cv[4];
@@ -130,139 +127,116 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
             const int p = p0 + tid + u * kTopkThreads;
             const uint32_t k = score_key(sv[u], cv[u] != 0);
             if (keys_in_smem && p < P) skeys[p] = k;
-            if (k != 0u) {
-                ++cnt;
-                kmin = min(kmin, k);
-                kmax = max(kmax, k);
-            }
+            cnt += k != 0u;
+            const uint32_t d = p < P ? (k >> 24) : 0x100u;
+            const uint32_t peers = __match_any_sync(0xffffffffu, d);
+            if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[0][d], __popc(peers));
         }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
-        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
-    }
-    if ((tid & 31) == 0) {
-        atomicAdd(&s_ncand, cnt);
-        atomicMin(&s_kmin, kmin);
-        atomicMax(&s_kmax, kmax);
-    }
+    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    if ((tid & 31) == 0) atomicAdd(&s_ncand, cnt);
     __syncthreads();
     const int nq = min(K, s_ncand);
 
-    // Radix select of the nq-th largest key, most significant digit first. Every
-    // candidate key shares the bits above hb, the highest bit where the smallest
-    // and the largest differ, so the first digit is bits hb..hb-7 (scores of one
-    // magnitude share their top byte, which would cost a pass for nothing). Pass
-    // i builds its histogram in hist[i & 1] (cleared one pass earlier) and its
-    // pick in s_pick[i & 1]: two barriers a pass. Non-candidates (key 0) rank
-    // below every candidate and never reach the answer (nq <= candidates).
+    // Radix select of the nq-th largest key, 8 bits per pass, most significant
+    // first. Pass i builds its histogram in hist[i & 1] (cleared one pass
+    // earlier) and its pick in s_pick[i & 1], so a pass takes two barriers.
     uint32_t prefix = 0, pmask = 0;
     int remaining = nq;
     if (nq > 0) {
-        const uint32_t diff = s_kmin ^ s_kmax;
-        if (diff == 0u) {
-            prefix = s_kmax;                       // every candidate key is equal
-        } else {
-            const int hb = 31 - __clz(diff);
-            pmask = hb == 31 ? 0u : ~((2u << hb) - 1u);
-            prefix = s_kmax & pmask;
-            int width = min(8, hb + 1);
-            int shift = hb + 1 - width;
 #pragma unroll 1
-            for (int pass = 0;; ++pass) {
-                const int hbuf = pass & 1;
-                const uint32_t dmask = (1u << width) - 1u;
-                if (pass > 0 && tid < 256) hist[hbuf ^ 1][tid] = 0;   // the other buffer's pick was read
-                // Keys under the chosen prefix spread over the digit: plain shared
-                // atomics, except in a warp where many lanes match (crowded bins,
-                // e.g. equal scores), which aggregates per digit.
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass, hb = pass & 1;
+            if (pass > 0) {
+                // the other buffer's pass is over (its pick was read): clear it for the next
+                if (tid < 256) hist[hb ^ 1][tid] = 0;
+                // Only keys under the chosen prefix count, and they spread over the
+                // next byte: plain shared atomics, except in a warp where many lanes
+                // match (crowded bins, e.g. equal scores), which aggregates per digit.
                 for (int base = (tid & ~31); base < P; base += kTopkThreads) {
                     const int p = base + (tid & 31);
                     uint32_t d = 0x100u;   // no bin
                     if (p < P) {
                         const uint32_t k = key_at(p);
-                        if ((k & pmask) == prefix) d = (k >> shift) & dmask;
+                        if ((k & pmask) == prefix) d = (k >> shift) & 0xFF;
                     }
                     const uint32_t act = __ballot_sync(0xffffffffu, d != 0x100u);
                     if (__popc(act) > 8) {
                         const uint32_t peers = __match_any_sync(0xffffffffu, d);
-                        if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[hbuf][d], __popc(peers));
+                        if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[hb][d], __popc(peers));
                     } else if (d != 0x100u) {
-                        atomicAdd(&hist[hbuf][d], 1);
+                        atomicAdd(&hist[hb][d], 1);
+                    }
+                }
+                __syncthreads();
+            }
+            if (tid < 32) {
+                // lane l owns bins 255-8l down to 248-8l
+                int c[8], sum = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    c[i] = hist[hb][255 - 8 * tid - i];
+                    sum += c[i];
+                }
+                int above = sum;   // inclusive scan over lanes (descending bins)
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, above, off);
+                    if (tid >= off) above += y;
+                }
+                int run = above - sum;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (run < remaining && remaining <= run + c[i]) {
+                        s_pick[hb][0] = 255 - 8 * tid - i;
+                        s_pick[hb][1] = run;
+                        s_pick[hb][2] = c[i];
+                    }
+                    run += c[i];
+                }
+            }
+            __syncthreads();
+            remaining -= s_pick[hb][1];
+            prefix |= (uint32_t)s_pick[hb][0] << shift;
+            pmask |= 0xFFu << shift;
+            if (pass == 1 && s_pick[hb][2] <= 32) {
+                // At most 32 keys share the top 16 bits of the answer (the usual
+                // case: keys of similar magnitude differ from the second byte on).
+                // Gather them and rank them on one warp instead of two more passes.
+                const int lane = tid & 31;
+                for (int base = (tid & ~31); base < P; base += kTopkThreads) {
+                    const int p = base + lane;
+                    const uint32_t k = p < P ? key_at(p) : 0u;
+                    const bool m = p < P && (k & pmask) == prefix;
+                    const uint32_t bal = __ballot_sync(0xffffffffu, m);
+                    if (bal) {
+                        int off = 0;
+                        if (lane == 0) off = atomicAdd(&s_nsmall, __popc(bal));
+                        off = __shfl_sync(0xffffffffu, off, 0);
+                        if (m) s_small[off + __popc(bal & ((1u << lane) - 1u))] = k;
                     }
                 }
                 __syncthreads();
                 if (tid < 32) {
-                    // lane l owns bins 255-8l down to 248-8l (bins past dmask stay 0)
-                    int c[8], sum = 0;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        c[i] = hist[hbuf][255 - 8 * tid - i];
-                        sum += c[i];
+                    const int n = s_nsmall;            // the bin's count, <= 32
+                    const uint32_t mine = tid < n ? s_small[tid] : 0u;
+                    int gt = 0, ge = 0;
+                    for (int j = 0; j < n; ++j) {
+                        const uint32_t kj = s_small[j];
+                        gt += kj > mine;
+                        ge += kj >= mine;
                     }
-                    int above = sum;   // inclusive scan over lanes (descending bins)
-#pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const int y = __shfl_up_sync(0xffffffffu, above, off);
-                        if (tid >= off) above += y;
-                    }
-                    int run = above - sum;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        if (run < remaining && remaining <= run + c[i]) {
-                            s_pick[hbuf][0] = 255 - 8 * tid - i;
-                            s_pick[hbuf][1] = run;
-                            s_pick[hbuf][2] = c[i];
-                        }
-                        run += c[i];
+                    // the remaining-th largest of the bin (equal keys write equal values)
+                    if (tid < n && gt < remaining && remaining <= ge) {
+                        s_tau = mine;
+                        s_req = remaining - gt;
                     }
                 }
                 __syncthreads();
-                remaining -= s_pick[hbuf][1];
-                prefix |= (uint32_t)s_pick[hbuf][0] << shift;
-                pmask |= dmask << shift;
-                if (shift == 0) break;                       // every bit is fixed
-                if (s_pick[hbuf][2] <= 32) {
-                    // At most 32 keys share the answer's bits so far (the usual case
-                    // after one pass): gather them and rank them on one warp.
-                    const int lane = tid & 31;
-                    for (int base = (tid & ~31); base < P; base += kTopkThreads) {
-                        const int p = base + lane;
-                        const uint32_t k = p < P ? key_at(p) : 0u;
-                        const bool m = p < P && (k & pmask) == prefix;
-                        const uint32_t bal = __ballot_sync(0xffffffffu, m);
-                        if (bal) {
-                            int off = 0;
-                            if (lane == 0) off = atomicAdd(&s_nsmall, __popc(bal));
-                            off = __shfl_sync(0xffffffffu, off, 0);
-                            if (m) s_small[off + __popc(bal & ((1u << lane) - 1u))] = k;
-                        }
-                    }
-                    __syncthreads();
-                    if (tid < 32) {
-                        const int n = s_nsmall;            // the bin's count, <= 32
-                        const uint32_t mine = tid < n ? s_small[tid] : 0u;
-                        int gt = 0, ge = 0;
-                        for (int j = 0; j < n; ++j) {
-                            const uint32_t kj = s_small[j];
-                            gt += kj > mine;
-                            ge += kj >= mine;
-                        }
-                        // the remaining-th largest of the bin (equal keys write equal values)
-                        if (tid < n && gt < remaining && remaining <= ge) {
-                            s_tau = mine;
-                            s_req = remaining - gt;
-                        }
-                    }
-                    __syncthreads();
-                    prefix = s_tau;
-                    remaining = s_req;
-                    break;
-                }
-                width = min(8, shift);
-                shift -= width;
+                prefix = s_tau;
+                remaining = s_req;
+                break;
             }
         }
     }
