@@ -305,3 +305,21 @@ def test_mla_launch_count(B):
     assert B.dsa_sparse_mla_launch_count(2, 64, 2048) == 2
     assert B.dsa_sparse_mla_launch_count(16, 64, 2048) in (1, 2)
     assert B.dsa_sparse_mla_launch_count(0, 64, 2048) == 0
+
+
+def test_maximum_select_k_and_kpool(B):
+    """select_k = 4096 (the largest), kpool = 8: a 32768-id row, whose MLA splits 69 ways
+    per query (138 CTAs) and merges more than 16 splits in the combine (its
+    multi-round path)."""
+    T = 40000
+    wl = W.build("max select", lengths=[T, 700], pads=[3, 0], kpool=8, max_pools=(T + 7) // 8,
+                 select_k=4096, hm=16, q_req=[0, 1], q_pos=[T - 1, 699], seed=23)
+    assert wl.out_width == 32768
+    assert B.dsa_sparse_mla_launch_count(2, 16, 32768) == 2
+    step, g = run_step(wl)
+    stagewise(wl, g)
+    n0 = int((g["top_pools"][0] >= 0).sum())
+    assert n0 == 4096                                    # 4999 candidate pools, 4096 taken
+    assert int((g["top_pools"][1] >= 0).sum()) == 87     # request 1: all its 87 pools
+    assert (g["token_ids"][1][87 * 8:] == -1).all()
+    device_status_clean(B)
