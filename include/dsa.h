@@ -113,6 +113,14 @@ int dsa_head_gate(const float *hidden, const float *w, float *out, int M, int K,
                   dsa_stream_t stream);
 
 /*
+ * Routing predicate of the head gate (the PR's splitk_applicable, as a status):
+ * the status dsa_head_gate returns for these sizes before it looks at any
+ * pointer -- DSA_OK when the kernel serves them, DSA_ERR_UNSUPPORTED or
+ * DSA_ERR_INVALID_ARG otherwise. Launches nothing.
+ */
+int dsa_head_gate_supported(int M, int K, int N);
+
+/*
  * a2+a3. kpool_compress with the k_norm LayerNorm fused in
  * ([mod.rs] "Shape of the pipeline" first arrow, traps 1-4, KERNEL_MAX_KPOOL).
  *   k, gate   bf16 [total_tokens, D] row-major (indexer keys; per-token,

@@ -25,7 +25,7 @@ DSA_ERR_CUDA = 5
 # Every symbol include/dsa.h declares.
 EXPORTS = (
     "dsa_status_string", "dsa_abi_version", "dsa_device_status", "dsa_selftest_bounded_wait",
-    "dsa_head_gate",
+    "dsa_head_gate", "dsa_head_gate_supported",
     "dsa_kpool_compress", "dsa_indexer_store", "dsa_kpool_compress_tokens",
     "dsa_index_scores", "dsa_topk_expand", "dsa_topk_expand_tail",
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_launch_count", "dsa_sparse_mla_decode",
@@ -56,6 +56,7 @@ def _load() -> ctypes.CDLL:
         "dsa_device_status": ([ctypes.POINTER(I), I], I),
         "dsa_selftest_bounded_wait": ([P, P], I),
         "dsa_head_gate": ([P, P, P, I, I, I, P], I),
+        "dsa_head_gate_supported": ([I, I, I], I),
         "dsa_kpool_compress": ([P, P, P, P, I, I, I, I, P, P, P, F, P, P, P, P, P], I),
         "dsa_indexer_store": ([P, P, P, P, P, I, I, P, I, P, P, P, P], I),
         "dsa_kpool_compress_tokens": ([P, P, P, P, I, I, I, I, P, P, P, F, P, P, P, P, P, P, P],
@@ -120,6 +121,10 @@ def dsa_device_status(reset: bool = True) -> int:
 
 def dsa_selftest_bounded_wait(result, stream=None) -> None:
     _check("dsa_selftest_bounded_wait", lib.dsa_selftest_bounded_wait(_ptr(result), _stream(stream)))
+
+
+def dsa_head_gate_supported(M: int, K: int, N: int) -> bool:
+    return int(lib.dsa_head_gate_supported(M, K, N)) == DSA_OK
 
 
 def dsa_head_gate(hidden, w, out, M: int, K: int, N: int, stream=None) -> None:

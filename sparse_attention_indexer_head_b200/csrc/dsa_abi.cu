@@ -92,6 +92,8 @@ int dsa_selftest_bounded_wait(int *result, dsa_stream_t stream) {
     return dsa::launch_status();
 }
 
+int dsa_head_gate_supported(int M, int K, int N) { return dsa::head_gate_shape_status(M, K, N); }
+
 int dsa_head_gate(const float *hidden, const float *w, float *out, int M, int K, int N,
                   dsa_stream_t stream) {
     return dsa::head_gate_launch(hidden, w, out, M, K, N, reinterpret_cast<cudaStream_t>(stream));

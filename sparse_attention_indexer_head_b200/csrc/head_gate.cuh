@@ -151,10 +151,18 @@ head_gate_kernel(const float *__restrict__ hidden, const float *__restrict__ w,
                      : "memory");
 }
 
-inline int head_gate_launch(const float *hidden, const float *w, float *out, int M, int K, int N,
-                            cudaStream_t stream) {
+// The size checks of head_gate_launch, on their own (no pointer is looked at).
+inline int head_gate_shape_status(int M, int K, int N) {
     if (M < 0 || K <= 0 || N <= 0) return DSA_ERR_INVALID_ARG;
     if (N > kGateMaxN || (K & 3) != 0) return DSA_ERR_UNSUPPORTED;
+    if (ceil_div(M, kGateRows) > 65535 * 16) return DSA_ERR_UNSUPPORTED;
+    return DSA_OK;
+}
+
+inline int head_gate_launch(const float *hidden, const float *w, float *out, int M, int K, int N,
+                            cudaStream_t stream) {
+    const int st = head_gate_shape_status(M, K, N);
+    if (st != DSA_OK) return st;
     if (M == 0) return DSA_OK;
     if (!hidden || !w || !out) return DSA_ERR_INVALID_ARG;
     if (!aligned(hidden, 16) || !aligned(w, 4) || !aligned(out, 4)) return DSA_ERR_ALIGNMENT;

@@ -64,6 +64,19 @@ def test_head_gate_refusals(B):
     assert L.dsa_head_gate(None, None, None, 0, 4096, 16, None) == B.DSA_OK   # M == 0: no-op
 
 
+def test_head_gate_routing_predicate(B):
+    assert B.dsa_head_gate_supported(16, 4096, 16)
+    assert B.dsa_head_gate_supported(0, 4096, 16)                 # empty batch: served (no-op)
+    assert not B.dsa_head_gate_supported(16, 4096, 17)            # more than 16 heads
+    assert not B.dsa_head_gate_supported(16, 4094, 16)            # K not a multiple of 4
+    assert B.lib.dsa_head_gate_supported(-1, 4096, 16) == B.DSA_ERR_INVALID_ARG
+    # the predicate and the call agree on every shape
+    for M, K, N in [(16, 4096, 16), (3, 4, 1), (5, 4096, 17), (2, 4098, 8), (-1, 8, 1)]:
+        want = B.lib.dsa_head_gate_supported(M, K, N)
+        got = B.lib.dsa_head_gate(FAKE, FAKE, FAKE, M, K, N, None) if want != B.DSA_OK else want
+        assert got == want
+
+
 def _compress(lib, **kw):
     a = dict(k=FAKE, gate=FAKE, valid=FAKE, req_start=FAKE, B=2, D=128, kpool=4, max_pools=8,
              ape=FAKE, ln_w=FAKE, ln_b=FAKE, eps=1e-5, keys=FAKE, idx=FAKE, pv=FAKE, fv=FAKE)
