@@ -20,12 +20,6 @@ DSA_DEVINL uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_
            ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Same with the 64-byte swizzle (layout 4): rows of 64 bytes, 8-row atoms of 512 bytes.
-DSA_DEVINL uint64_t desc_sw64(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
-}
-
 // -- instruction descriptor, kind::f16 with bf16 inputs and an f32 accumulator ---------
 // bits [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,
 // bit 15 A major (1 = MN), bit 16 B major, [17,23) N >> 3, [24,29) M >> 4.
@@ -148,11 +142,6 @@ DSA_DEVINL void cp_async16_zfill(uint32_t dst, const void *src, uint32_t src_byt
 DSA_DEVINL void cp_async_arrive_noinc(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
-}
-// Hint: bring the 128-byte line at p into L2 (no data returned, never faults on
-// the valid addresses it is given).
-DSA_DEVINL void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 DSA_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 DSA_DEVINL void st_shared_zero16(uint32_t dst) {

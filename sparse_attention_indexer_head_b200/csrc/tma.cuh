@@ -56,18 +56,4 @@ DSA_DEVINL void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, 
         : "memory");
 }
 
-// Gather of four whole-box rows: rows y0..y3 of the map (box one row high,
-// box_cols wide) at column x land one after another at dst (4 x 128 bytes for
-// a 64-column bf16 box with the 128-byte swizzle). A row outside the map reads
-// as zeros. x is a multiple of 64 elements at every call site.
-DSA_DEVINL void tma_gather4(uint32_t dst, const CUtensorMap *map, int x, int y0, int y1, int y2,
-                            int y3, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
-        "r"(smem_u32(bar))
-        : "memory");
-}
-
 }  // namespace dsa
