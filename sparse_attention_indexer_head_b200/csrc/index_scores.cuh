@@ -67,10 +67,10 @@ index_scores_kernel(const __grid_constant__ CUtensorMap key_map,
         tma_load_2d(sQ, &q_map, 0, q * H, &q_bar);
         tma_load_2d(sQ + kScoreQAtom, &q_map, 64, q * H, &q_bar);
     }
+    const int b = q_req[q];                   // a step input, like the query rows
+    const bool req_ok = b >= 0 && b < B;
     pdl_wait();
     pdl_launch_dependents();
-    const int b = q_req[q];
-    const bool req_ok = b >= 0 && b < B;
     if (tid == 0 && req_ok) {
         // The key tile (written by the predecessor) is requested at once, while
         // the candidate flags are read; rows past the key map read as zeros.

@@ -288,13 +288,22 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         s_ape[(sl * 2 + ((c >> 2) & 1)) * 64 + 4 * (c >> 3) + (c & 3)] = ape[i] * kLog2e;
     }
     __syncthreads();
+    // Request offsets are a step input the path never writes: the producer has
+    // its first request's rows before the wait on the preceding kernel.
+    long long total = 0;
+    int first_rs = 0, first_re = 0;
+    if (warp == kCmpConsumers / 32 && t_begin < t_end) {
+        const int b0 = t_begin / tiles_per_req;
+        total = req_start[B];                       // rows of the validity array
+        first_rs = req_start[b0];
+        first_re = req_start[b0 + 1];
+    }
     pdl_wait();
     pdl_launch_dependents();
 
     if (warp == kCmpConsumers / 32) {
         // ---------------------------------------------------------------- producer warp
         int cur_b = -1, cur_f = 0, cur_rs = 0, cur_T = 0;
-        const long long total = req_start[B];      // rows of the validity array
         for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
             const int s = i % kCmpStages;
             bool ok = true;
@@ -302,8 +311,9 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             if (!__all_sync(0xffffffffu, ok)) break;
             const int b = t / tiles_per_req, j = t - b * tiles_per_req;
             if (b != cur_b) {
-                cur_rs = req_start[b];
-                cur_T = max(0, req_start[b + 1] - cur_rs);
+                const bool first = i == 0;
+                cur_rs = first ? first_rs : req_start[b];
+                cur_T = max(0, (first ? first_re : req_start[b + 1]) - cur_rs);
                 cur_f = first_valid_scan(valid, cur_rs, cur_T);
                 cur_b = b;
             }

@@ -88,10 +88,10 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
 
     const int tid = threadIdx.x;
     const int q = blockIdx.x;
+    const int b = q_req[q];                   // a step input: read before the wait
+    const bool req_ok = b >= 0 && b < B;
     pdl_wait();
     pdl_launch_dependents();
-    const int b = q_req[q];
-    const bool req_ok = b >= 0 && b < B;
     const float *srow = scores + (size_t)q * P;
     const uint8_t *crow = cand + (size_t)q * P;
 
