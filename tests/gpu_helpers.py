@@ -118,7 +118,7 @@ def assert_mla_close(gpu_out, ref_out, gpu_lse, ref_lse, vbound=None, rows=None)
     2^-9 max_j |v_j[c]| after the merge. The bound used is ulp(ref) plus
     (2^-8 + 2^-12) max_j |v_j[c]|: the two roundings and a margin for fp32
     accumulation and the exp2 approximation, which are far below 2^-12.
-    Also the spec max-abs 2e-2, and lse within 1e-4 (fp32 sums of
+    Also the stated max-abs 2e-2, and lse within 1e-4 (fp32 sums of
     fp32 weights; one missing token among 2048 moves lse by ~1e-3).
     """
     g, r = bf16f(gpu_out), bf16f(ref_out)
