@@ -228,25 +228,23 @@ class DecodeStep:
 
 
 class StreamedDecode:
-    """Decode steps served from and to pinned host memory, overlapped across steps.
+    """Decode steps served from and to pinned host memory.
 
-    Each step copies its query inputs host -> device (one copy of a packed
-    pinned buffer), runs the five calls
-    (replayed from a CUDA graph captured once per slot) and copies the output
-    device -> host. The three run on their own streams and the steps rotate over
-    `slots` device buffer sets, so step i's copies overlap the compute of its
-    neighbours; events keep a slot's inputs and output from being overwritten
-    while still in use. `submit` enqueues a step; `result(i)` waits for step
-    i's output to reach the host and returns it (the slot's pinned buffer,
-    valid until that slot is submitted again).
+    Each slot owns a pinned host input buffer (the query inputs packed, see
+    `write_inputs`), device buffers and a pinned host output buffer, and a CUDA
+    graph that copies the inputs host -> device, runs the five calls and copies
+    the output device -> host, on the slot's own stream. Steps rotate over the
+    slots, so consecutive steps run on different streams and overlap on the
+    GPU (their copies and kernels interleave). Step i uses slot i % slots: its
+    inputs must be in that slot's buffer when it is submitted, and the buffer
+    may be refilled for step i + slots once result(i) has returned.
     """
 
     def __init__(self, wl: Workload, device: str = "cuda", slots: int = 2,
                  inputs: Optional[Dict] = None):
         self.device = torch.device(device)
         self.steps = [DecodeStep(wl, device=device, inputs=inputs) for _ in range(slots)]
-        # A slot's query inputs live in one device buffer, so a step's inputs are
-        # one host-to-device copy from a packed pinned buffer (see pack()).
+        # A slot's query inputs live in one device buffer: one copy per step.
         self.layout, nbytes = {}, 0
         for name in QUERY_INPUTS:
             t = self.steps[0].t[name]
@@ -254,34 +252,32 @@ class StreamedDecode:
             self.layout[name] = (nbytes, t.dtype, tuple(t.shape))
             nbytes += t.numel() * t.element_size()
         self.nbytes = nbytes
-        self.dev_in = []
+        self.dev_in, self.in_host, self.out_host, self.streams = [], [], [], []
         for st in self.steps:
             buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+            host = torch.zeros(nbytes, dtype=torch.uint8).pin_memory()
             for name, (off, dtype, shape) in self.layout.items():
                 view = self._view(buf, off, dtype, shape)
                 view.copy_(st.t[name])
+                self._view(host, off, dtype, shape).copy_(st.t[name].cpu())
                 st.t[name] = view
             self.dev_in.append(buf)
-        self.s_in = torch.cuda.Stream(device=self.device)
-        self.s_run = torch.cuda.Stream(device=self.device)
-        self.s_out = torch.cuda.Stream(device=self.device)
+            self.in_host.append(host)
+            self.out_host.append(torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory())
+            self.streams.append(torch.cuda.Stream(device=self.device))
         self.graphs = []
-        with torch.cuda.stream(self.s_run):
-            for st in self.steps:
+        for k, st in enumerate(self.steps):
+            with torch.cuda.stream(self.streams[k]):
                 st.run()                                  # sets kernel attributes eagerly
-        self.s_run.synchronize()
-        for st in self.steps:
+            self.streams[k].synchronize()
             g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=self.s_run):
+            with torch.cuda.graph(g, stream=self.streams[k]):
+                self.dev_in[k].copy_(self.in_host[k], non_blocking=True)
                 st.run()
+                self.out_host[k].copy_(st.out, non_blocking=True)
             self.graphs.append(g)
         torch.cuda.synchronize(self.device)
-        n = len(self.steps)
-        self.in_done = [torch.cuda.Event() for _ in range(n)]
-        self.run_done = [torch.cuda.Event() for _ in range(n)]
-        self.out_done = [torch.cuda.Event() for _ in range(n)]
-        self.out_host = [torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
-                         for st in self.steps]
+        self.done = [torch.cuda.Event() for _ in self.steps]
         self.submitted = 0
 
     @staticmethod
@@ -292,34 +288,22 @@ class StreamedDecode:
         size = n * torch.empty((), dtype=dtype).element_size()
         return buf[off:off + size].view(dtype).view(shape)
 
-    def pack(self, host_inputs: Dict[str, torch.Tensor]) -> torch.Tensor:
-        """The query inputs (names of QUERY_INPUTS) packed into one pinned buffer."""
-        out = torch.empty(self.nbytes, dtype=torch.uint8).pin_memory()
-        for name, (off, dtype, shape) in self.layout.items():
-            self._view(out, off, dtype, shape).copy_(host_inputs[name])
-        return out
+    def slot(self, i: int) -> int:
+        return i % len(self.steps)
 
-    def submit(self, packed: torch.Tensor) -> int:
-        """Enqueue one step on pinned packed inputs (from pack()); returns its index."""
+    def write_inputs(self, i: int, host_inputs: Dict[str, torch.Tensor]) -> None:
+        """Pack step i's query inputs (names of QUERY_INPUTS) into its slot's buffer."""
+        buf = self.in_host[self.slot(i)]
+        for name, (off, dtype, shape) in self.layout.items():
+            self._view(buf, off, dtype, shape).copy_(host_inputs[name])
+
+    def submit(self) -> int:
+        """Enqueue the next step on its slot's stream; returns its index."""
         i = self.submitted
-        k = i % len(self.steps)
-        # inputs: after the slot's previous step has finished reading them
-        self.s_in.wait_event(self.run_done[k])
-        with torch.cuda.stream(self.s_in):
-            self.dev_in[k].copy_(packed, non_blocking=True)
-        self.in_done[k].record(self.s_in)
-        st = self.steps[k]
-        # compute: after its inputs landed and the slot's previous output left
-        self.s_run.wait_event(self.in_done[k])
-        self.s_run.wait_event(self.out_done[k])
-        with torch.cuda.stream(self.s_run):
+        k = self.slot(i)
+        with torch.cuda.stream(self.streams[k]):
             self.graphs[k].replay()
-        self.run_done[k].record(self.s_run)
-        # output back to the host
-        self.s_out.wait_event(self.run_done[k])
-        with torch.cuda.stream(self.s_out):
-            self.out_host[k].copy_(st.out, non_blocking=True)
-        self.out_done[k].record(self.s_out)
+            self.done[k].record(self.streams[k])
         self.submitted += 1
         return i
 
@@ -328,9 +312,8 @@ class StreamedDecode:
         last `slots` submitted)."""
         if not (self.submitted - len(self.steps) <= i < self.submitted):
             raise ValueError("step is not among the slots in flight")
-        k = i % len(self.steps)
-        self.out_done[k].synchronize()
-        return self.out_host[k]
+        self.done[self.slot(i)].synchronize()
+        return self.out_host[self.slot(i)]
 
     def kernels_per_step(self) -> int:
         return self.steps[0].kernels_per_step()

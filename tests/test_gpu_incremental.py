@@ -329,8 +329,9 @@ def test_decode_sequence_stays_equal_to_full_compress(B, kpool):
 
 
 def test_streamed_decode_matches_eager_steps(B):
-    """StreamedDecode (H2D, graph replay, D2H over two overlapped slots) returns each
-    step's output exactly as an eager step on the same inputs does."""
+    """StreamedDecode (H2D, the step and D2H in one graph per slot, consecutive steps on
+    two streams) returns each step's output exactly as an eager step on the same
+    inputs does."""
     from sparse_attention_indexer_head_b200.pipeline import (QUERY_INPUTS, DecodeStep,
                                                             StreamedDecode, host_tensors)
     wl_a, wl_b = W.make("tiny", seed=0), W.make("tiny", seed=1)
@@ -344,10 +345,10 @@ def test_streamed_decode_matches_eager_steps(B):
         torch.cuda.synchronize()
         ref.append(st.out.view(torch.int16).cpu().numpy())
     sd = StreamedDecode(wl_a, slots=2)
-    packed = [sd.pack(q) for q in ins]
     got = []
     for i in range(7):
-        sd.submit(packed[i % 2])
+        sd.write_inputs(i, ins[i % 2])       # its slot's previous step was read (below)
+        sd.submit()
         if i >= 1:
             got.append(sd.result(i - 1).view(torch.int16).numpy().copy())
     got.append(sd.result(6).view(torch.int16).numpy().copy())
