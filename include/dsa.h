@@ -281,7 +281,10 @@ int dsa_topk_expand_tail(const float *scores, const uint8_t *cand, const int32_t
  *   For each head: z_j = sm_scale * <q[q,h,:], kv[row(j),:]>,
  *   out[q,h,:] = bf16(sum_j softmax(z)_j * kv[row(j),:]) (fp32 accumulation),
  *   lse[q,h] = log(sum_j exp(z_j)) (natural log; -inf and out = 0 when no id
- *   is valid). lse may be NULL.
+ *   is valid). lse may be NULL. Precision: the P.V product takes the softmax
+ *   weights as bf16, and split partials merged through the workspace are
+ *   stored as bf16 rows; each moves an output by at most 2^-9 of the largest
+ *   selected value in its channel (the row sums and lse stay fp32).
  *   workspace: device scratch of dsa_sparse_mla_workspace_size(Q, Hm, W) bytes
  *   (16-byte aligned; contents need no initialisation; not shared between
  *   calls that may overlap).
