@@ -5,10 +5,9 @@
 //
 // One CTA per query. Scores become order-preserving uint32 keys (candidates
 // only; -0 folded onto +0, NaN onto -inf, non-candidates 0). An 8-bit MSB
-// radix select finds the n_q-th largest key tau exactly: the first pass while
-// the keys load, the second on one warp -- which, when at most 32 keys share
-// those 16 bits with tau, ranks them and ends the select -- else two more
-// passes; the winners are
+// radix select finds the n_q-th largest key tau exactly: two passes, then,
+// when at most 32 keys share those 16 bits with tau, a rank among them on one
+// warp, else two more passes; the winners are
 // every key above tau plus the lowest-id keys equal to tau (an id-ordered
 // block scan), written in ascending pool id, so the result is bit-exact and
 // deterministic. The expansion gathers pool_idx rows and writes every slot of
@@ -84,7 +83,7 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     __shared__ int hist[2][256];          // double-buffered radix histograms
     __shared__ int2 s_warp2[kTopkWarps];
     __shared__ int s_pick[2][3];          // per pass parity: (digit, count above it, count in it)
-    __shared__ int s_ncand, s_req;
+    __shared__ int s_ncand, s_nsmall, s_req;
     __shared__ uint32_t s_small[32], s_tau;
 
     const int tid = threadIdx.x;
@@ -108,7 +107,10 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
         hist[0][tid] = 0;
         hist[1][tid] = 0;
     }
-    if (tid == 0) s_ncand = 0;
+    if (tid == 0) {
+        s_ncand = 0;
+        s_nsmall = 0;
+    }
     __syncthreads();
     int cnt = 0;
     for (int p0 = 0; p0 < P; p0 += 4 * kTopkThreads) {
@@ -146,100 +148,6 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
 #pragma unroll 1
         for (int pass = 0; pass < 4; ++pass) {
             const int shift = 24 - 8 * pass, hb = pass & 1;
-            if (pass == 1) {
-                // Pass 1 on one warp, no block barrier inside: its histogram, its
-                // pick and, when at most 32 keys share the 16 bits then fixed (the
-                // usual case: scores of one magnitude differ from the second byte
-                // on), the rank among them that ends the select. The other threads
-                // clear the buffer of pass 2 meanwhile.
-                if (tid >= 32 && tid < 256 + 32) hist[0][tid - 32] = 0;
-                if (tid < 32) {
-                    const int lane = tid;
-                    for (int p0 = 0; p0 < P; p0 += 4 * 32) {
-                        uint32_t kk[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int p = p0 + 32 * u + lane;
-                            kk[u] = p < P ? key_at(p) : 0u;
-                        }
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int p = p0 + 32 * u + lane;
-                            if (p < P && (kk[u] & pmask) == prefix) atomicAdd(&hist[1][(kk[u] >> 16) & 0xFF], 1);
-                        }
-                    }
-                    __syncwarp();
-                    int c[8], sum = 0;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        c[i] = hist[1][255 - 8 * lane - i];
-                        sum += c[i];
-                    }
-                    int above = sum;
-#pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const int y = __shfl_up_sync(0xffffffffu, above, off);
-                        if (lane >= off) above += y;
-                    }
-                    int run = above - sum, pick = -1, pick_run = 0, pick_cnt = 0;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        if (run < remaining && remaining <= run + c[i]) {
-                            pick = 255 - 8 * lane - i;
-                            pick_run = run;
-                            pick_cnt = c[i];
-                        }
-                        run += c[i];
-                    }
-                    const int src = __ffs(__ballot_sync(0xffffffffu, pick >= 0)) - 1;
-                    pick = __shfl_sync(0xffffffffu, pick, src);
-                    pick_run = __shfl_sync(0xffffffffu, pick_run, src);
-                    pick_cnt = __shfl_sync(0xffffffffu, pick_cnt, src);
-                    const int rem1 = remaining - pick_run;
-                    const uint32_t pre1 = prefix | ((uint32_t)pick << 16), msk1 = pmask | 0xFF0000u;
-                    int done = 0;
-                    if (pick_cnt <= 32) {
-                        int n = 0;
-                        for (int p0 = 0; p0 < P; p0 += 32) {
-                            const int p = p0 + lane;
-                            const uint32_t k = p < P ? key_at(p) : 0u;
-                            const bool m = p < P && (k & msk1) == pre1;
-                            const uint32_t bal = __ballot_sync(0xffffffffu, m);
-                            if (m) s_small[n + __popc(bal & ((1u << lane) - 1u))] = k;
-                            n += __popc(bal);
-                        }
-                        __syncwarp();
-                        const uint32_t mine = lane < n ? s_small[lane] : 0u;
-                        int gt = 0, ge = 0;
-                        for (int j = 0; j < n; ++j) {
-                            const uint32_t kj = s_small[j];
-                            gt += kj > mine;
-                            ge += kj >= mine;
-                        }
-                        // the rem1-th largest of the bin (equal keys write equal values)
-                        if (lane < n && gt < rem1 && rem1 <= ge) {
-                            s_tau = mine;
-                            s_req = rem1 - gt;
-                        }
-                        done = 1;
-                    }
-                    if (lane == 0) {
-                        s_pick[1][0] = pick;
-                        s_pick[1][1] = pick_run;
-                        s_pick[1][2] = done;
-                    }
-                }
-                __syncthreads();
-                remaining -= s_pick[1][1];
-                prefix |= (uint32_t)s_pick[1][0] << 16;
-                pmask |= 0xFF0000u;
-                if (s_pick[1][2]) {
-                    prefix = s_tau;
-                    remaining = s_req;
-                    break;
-                }
-                continue;
-            }
             if (pass > 0) {
                 // the other buffer's pass is over (its pick was read): clear it for the next
                 if (tid < 256) hist[hb ^ 1][tid] = 0;
@@ -292,6 +200,44 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
             remaining -= s_pick[hb][1];
             prefix |= (uint32_t)s_pick[hb][0] << shift;
             pmask |= 0xFFu << shift;
+            if (pass == 1 && s_pick[hb][2] <= 32) {
+                // At most 32 keys share the top 16 bits of the answer (the usual
+                // case: keys of similar magnitude differ from the second byte on).
+                // Gather them and rank them on one warp instead of two more passes.
+                const int lane = tid & 31;
+                for (int base = (tid & ~31); base < P; base += kTopkThreads) {
+                    const int p = base + lane;
+                    const uint32_t k = p < P ? key_at(p) : 0u;
+                    const bool m = p < P && (k & pmask) == prefix;
+                    const uint32_t bal = __ballot_sync(0xffffffffu, m);
+                    if (bal) {
+                        int off = 0;
+                        if (lane == 0) off = atomicAdd(&s_nsmall, __popc(bal));
+                        off = __shfl_sync(0xffffffffu, off, 0);
+                        if (m) s_small[off + __popc(bal & ((1u << lane) - 1u))] = k;
+                    }
+                }
+                __syncthreads();
+                if (tid < 32) {
+                    const int n = s_nsmall;            // the bin's count, <= 32
+                    const uint32_t mine = tid < n ? s_small[tid] : 0u;
+                    int gt = 0, ge = 0;
+                    for (int j = 0; j < n; ++j) {
+                        const uint32_t kj = s_small[j];
+                        gt += kj > mine;
+                        ge += kj >= mine;
+                    }
+                    // the remaining-th largest of the bin (equal keys write equal values)
+                    if (tid < n && gt < remaining && remaining <= ge) {
+                        s_tau = mine;
+                        s_req = remaining - gt;
+                    }
+                }
+                __syncthreads();
+                prefix = s_tau;
+                remaining = s_req;
+                break;
+            }
         }
     }
     const uint32_t tau = prefix;   // the nq-th largest key (when nq > 0)
