@@ -220,7 +220,9 @@ def reference_arm(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    n_req = 2
+    # one request (one decode query) per step keeps --steps K within a few minutes
+    # at the K the GPU arm uses (about 27 ms a step on 16 host cores)
+    n_req = 2 if args.steps + args.warmup <= 200 else 1
     import oracle as O
     from sparse_attention_indexer_head_b200 import workloads as W
     sub = W.build(wl.name, lengths=wl.lengths[:n_req], pads=wl.pads[:n_req], kpool=wl.kpool,
@@ -471,7 +473,7 @@ def gpu_arm(args, wl_fn):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=8000)
+    ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sets", type=int, default=3)
