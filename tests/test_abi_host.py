@@ -1,7 +1,6 @@
 """The C-ABI library on the host (no GPU): it loads, exports every symbol the
 header declares, and refuses bad arguments with the documented status before
 launching anything."""
-import ctypes
 import os
 import re
 

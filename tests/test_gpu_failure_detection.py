@@ -1,7 +1,6 @@
 """Failure detection on the GPU without a fault: a bounded wait that nothing
 completes gives up, raises the device error word, and the context keeps
 working (the wait bound is about two seconds)."""
-import numpy as np
 import pytest
 import torch
 

@@ -11,7 +11,7 @@ import torch
 
 import oracle as O
 from gpu_helpers import (assert_gate_close, assert_keys_close, assert_mla_close,
-                         assert_scores_close, bf16f, dev_bits, device_status_clean, host_bits,
+                         assert_scores_close, dev_bits, device_status_clean, host_bits,
                          mla_value_bound, score_magnitude, workload)
 from sparse_attention_indexer_head_b200 import workloads as W
 
