@@ -378,9 +378,15 @@ int dsa_sparse_mla_decode_paged_fp8(const dsa_bf16 *q, const uint8_t *kv8, float
  *   148 x 64 x 1032 bytes (about 9.8 MB: a bf16 row of 512 plus m and l per
  *   head and split): the refusal is a guard that no present shape reaches.
  *   Nothing is allocated or freed: no cudaMalloc, no cudaFree, no allocating
- *   library routine. The first call on a device looks up the scratch's device
- *   address (cudaGetSymbolAddress, with that device current); make that first
- *   call before any stream capture on that device.
+ *   library routine. Each call looks up the scratch's device address
+ *   (cudaGetSymbolAddress with the calling thread's device current: a host
+ *   query that launches nothing), so the address stays right after a
+ *   cudaDeviceReset. The array itself comes into being when the CUDA runtime
+ *   loads this library's device code on a device, which under the default
+ *   lazy module loading happens at the first call into the library there: if
+ *   that first call is this one, the load (and its allocation) happens inside
+ *   it. So make one call of any entry point on each device before the region
+ *   where nothing may be allocated, and before any stream capture on it.
  *   Every call shares the one scratch area and leaves its last contents there;
  *   nothing in it needs to start at zero (every value the merge reads is
  *   written by the same call first). Calls whose kernels may overlap on the
@@ -388,6 +394,8 @@ int dsa_sparse_mla_decode_paged_fp8(const dsa_bf16 *q, const uint8_t *kv8, float
  *   scratch and must not be made.
  */
 #define DSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+/* DSA_NOALLOC_SCRATCH_BYTES as the loaded library was built with it. */
+size_t dsa_noalloc_scratch_bytes(void);
 int dsa_sparse_mla_decode_noalloc(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows,
                                   const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids, int Q, int B,
                                   int Hm, int W, int kv_lora, int rope_dim, float sm_scale,

@@ -30,9 +30,8 @@ EXPORTS = (
     "dsa_index_scores", "dsa_topk_expand", "dsa_topk_expand_tail",
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_launch_count", "dsa_sparse_mla_decode",
     "dsa_sparse_mla_decode_noalloc", "dsa_sparse_mla_decode_paged",
-    "dsa_sparse_mla_decode_paged_fp8",
+    "dsa_sparse_mla_decode_paged_fp8", "dsa_noalloc_scratch_bytes",
 )
-DSA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class DsaError(RuntimeError):
@@ -68,6 +67,7 @@ def _load() -> ctypes.CDLL:
         "dsa_sparse_mla_launch_count": ([I, I, I], I),
         "dsa_sparse_mla_decode": ([P, P, I64, P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P], I),
         "dsa_sparse_mla_decode_noalloc": ([P, P, I64, P, P, P, I, I, I, I, I, I, F, P, P, P], I),
+        "dsa_noalloc_scratch_bytes": ([], Z),
         "dsa_sparse_mla_decode_paged": ([P, P, I64, P, I, I, P, P, P, I, I, I, I, I, I, F, P, P, P,
                                          Z, P], I),
         "dsa_sparse_mla_decode_paged_fp8": ([P, P, F, I64, P, I, I, P, P, P, I, I, I, I, I, I, F, P,
@@ -81,6 +81,8 @@ def _load() -> ctypes.CDLL:
 
 
 lib = _load()
+# Size of the library's own scratch for dsa_sparse_mla_decode_noalloc, as built.
+DSA_NOALLOC_SCRATCH_BYTES = int(lib.dsa_noalloc_scratch_bytes())
 
 
 def _ptr(x) -> Optional[int]:

@@ -10,35 +10,28 @@
 #include "topk_expand.cuh"
 #include "sparse_mla.cuh"
 
-#include <mutex>
-
 // ---------------------------------------------------------------------------------------
 // Library-owned scratch for dsa_sparse_mla_decode_noalloc: the split-KV partial
 // rows that dsa_sparse_mla_decode keeps in the caller's workspace. It is a
 // file-scope device array, so every GPU that loads this library holds
 // DSA_NOALLOC_SCRATCH_BYTES of it until the process exits. In host code the
 // name g_mla_scratch only stands in for the symbol; its device address comes
-// from cudaGetSymbolAddress, looked up once per device (with that device
-// current) on the first call made on it.
+// from cudaGetSymbolAddress with the call's device current.
 // ---------------------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_mla_scratch[DSA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxDevices] = {};
-
+// The scratch's device address on the current device, looked up on every call:
+// a host-side query that launches and allocates nothing. Nothing is cached, so
+// after cudaDeviceReset (the module, and the array with it, is loaded anew and
+// may sit elsewhere) the next call still passes the right address.
 int scratch_address(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_mla_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_mla_scratch) != cudaSuccess || !p) {
+        (void)cudaGetLastError();
+        return DSA_ERR_CUDA;
     }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return DSA_OK;
 }
 }  // namespace
@@ -201,6 +194,8 @@ int dsa_sparse_mla_decode_paged_fp8(const dsa_bf16 *q, const uint8_t *kv8, float
                                             kv_lora, rope_dim, sm_scale, out, lse, workspace,
                                             workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
+
+size_t dsa_noalloc_scratch_bytes(void) { return (size_t)DSA_NOALLOC_SCRATCH_BYTES; }
 
 int dsa_sparse_mla_decode_noalloc(const dsa_bf16 *q, const dsa_bf16 *kv, int64_t kv_rows,
                                   const int32_t *req_start, const int32_t *q_req, const int32_t *token_ids, int Q, int B,

@@ -266,6 +266,9 @@ def test_noalloc_scratch_covers_every_geometry(B):
     # split-KV scratch of any call is at most 148 x 64 heads x (a bf16 row + m, l).
     bound = 148 * 64 * (512 * 2 + 8)
     assert bound <= B.DSA_NOALLOC_SCRATCH_BYTES
+    # the binding reads the size from the library; it is the header's constant
+    m = re.search(r"#define DSA_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", open(HEADER).read())
+    assert m and B.DSA_NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
     worst = 0
     for Q in list(range(1, 40)) + [64, 100, 147, 148, 149, 1000]:
         for hm in range(16, 129, 16):
