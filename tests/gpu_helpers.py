@@ -2,10 +2,15 @@
 
 Tolerances (each derived from the arithmetic, see the docstrings):
   * fp32 head gate: |gpu - ref| <= 1e-5 * max(1, |ref|).
-  * fp32 scores:    |gpu - ref| <= 1e-5 * max(1, S) with S = sum_h |g_h| relu(d_h),
-                    the magnitude of the summed terms (equal to |ref| when every
-                    gate weight is positive).
-  * bf16 pooled keys: |gpu - ref| <= ulp(ref) + max_s ulp(kn_s).
+  * fp32 scores:    |gpu - ref| <= 1e-5 * max(1, |ref|), and the looser
+                    1e-5 * max(1, S) with S = sum_h |g_h| relu(d_h), the magnitude
+                    of the summed terms, is reported beside it.
+  * bf16 pooled keys: |gpu - ref| <= ulp(ref) + max_s ulp(kn_s), at most 0.1 %
+                    of elements beyond 1 ulp(ref) (one-ulp k_norm flips).
+  * end to end (oracle from raw inputs): every score within its own bound (the
+                    gate and arithmetic tolerances plus the propagated pooled-key
+                    difference); a pool may be swapped only when that bound
+                    explains the swap (see end_to_end in test_gpu_parity.py).
   * bf16 MLA out:   max-abs 2e-2 and |gpu - ref| <= ulp(ref) + (2^-8 + 2^-12) max_j |v_j[c]|
                     (bf16 softmax weights in the tensor-core PV product, bf16
                     split partials); lse 1e-4.
@@ -54,6 +59,8 @@ def score_magnitude(q_idx_bits, gate_w, keys_bits, q_req, kpool=None):
 
 
 def assert_scores_close(gpu, ref, cand, mag):
+    """Scores of candidates within 1e-5 * max(1, S) and, as the specification states
+    it, within 1e-5 * max(1, |ref|); -inf exactly at non-candidates."""
     cand = cand.astype(bool)
     assert np.isneginf(gpu[~cand]).all(), "scores of non-candidates must be -inf"
     g, r, m = gpu[cand].astype(np.float64), ref[cand].astype(np.float64), mag[cand]
@@ -62,8 +69,10 @@ def assert_scores_close(gpu, ref, cand, mag):
     tol = 1e-5 * np.maximum(1.0, m)
     assert (err <= tol).all(), f"scores: {(err > tol).sum()} outside tolerance; worst {err.max():.3g}"
     plain = 1e-5 * np.maximum(1.0, np.abs(r))
-    return dict(max_abs=float(err.max(initial=0)), n=int(cand.sum()),
-                over_plain=int((err > plain).sum()))
+    over_plain = int((err > plain).sum())
+    assert over_plain == 0, (f"scores: {over_plain} outside 1e-5*max(1,|ref|); "
+                             f"worst {(err / plain).max():.3g} x the bound")
+    return dict(max_abs=float(err.max(initial=0)), n=int(cand.sum()), over_plain=over_plain)
 
 
 def kn_ulp_bound(k_bits, ln_w_bits, ln_b_bits, eps, rows):
@@ -77,7 +86,20 @@ def kn_ulp_bound(k_bits, ln_w_bits, ln_b_bits, eps, rows):
 
 
 def assert_keys_close(gpu_keys, ref_keys, pool_valid, wl, first_valid):
-    """Pooled keys of valid pools: |gpu - ref| <= ulp(ref) + max_s ulp(kn_s)."""
+    """Pooled keys of valid pools: |gpu - ref| <= ulp(ref) + max_s ulp(kn_s), and at
+    most 0.1 % of the elements more than 1 ulp(ref) away.
+
+    The kernel takes each token's LayerNorm mean and rstd in fp32 and rounds
+    kn = (k - mu) * rstd * w + b to bf16 as the specification stores it. Where the exact kn
+    lies within fp32 error of a bf16 rounding boundary, the two roundings can
+    differ by one bf16 ulp of kn; that kn enters the pooled value with its
+    softmax weight w_s <= 1, moving it by at most w_s * ulp(kn_s) <= max_s
+    ulp(kn_s) before the final rounding, which adds at most ulp(ref). A flip
+    needs the exact kn within fp32 error (about 2^-21 relative) of a bf16
+    boundary, about one kn in 2^12, and it carries a pooled element more than
+    1 ulp(ref) away only when that element also lies near its own boundary:
+    the 0.1 % cap on such elements is far above what that allows.
+    """
     b_idx, p_idx = np.nonzero(pool_valid)
     if b_idx.size == 0:
         return dict(n=0)

@@ -11,7 +11,7 @@ import torch
 
 import oracle as O
 from gpu_helpers import (assert_gate_close, assert_keys_close, assert_mla_close,
-                         assert_scores_close, dev_bits, device_status_clean, host_bits,
+                         assert_scores_close, bf16f, dev_bits, device_status_clean, host_bits,
                          mla_value_bound, score_magnitude, workload)
 from sparse_attention_indexer_head_b200 import workloads as W
 
@@ -74,39 +74,85 @@ def stagewise(wl, g, queries=None):
     return rep
 
 
+def e2e_score_bound(wl, qs, g, gate_ref, keys_ref):
+    """Per-pool bound of |GPU score - oracle score from raw inputs|, [len(qs), P].
+
+    The GPU scores a pool from its own head gate and pooled keys; the oracle
+    from its own. In exact arithmetic the two scores differ by
+      sum_h (g_gpu_h - g_ref_h) relu(d_gpu_h) + sum_h g_ref_h (relu(d_gpu_h) - relu(d_ref_h))
+    (d: the head dots with each side's pooled key), and the GPU's fp32 score is
+    within 1e-5 max(1, |score|) of its exact value (the stage-wise tolerance),
+    the oracle's within half an fp32 ulp. The bound is the sum of those terms'
+    magnitudes: where both sides hold the same pooled key it is the gate and
+    arithmetic tolerances alone.
+    """
+    q = bf16f(wl.q_idx[qs])
+    kg, kr = bf16f(g["pool_keys"]), bf16f(keys_ref)
+    gg = g["gate_w"][qs].astype(np.float64)
+    gr = gate_ref.astype(np.float64)
+    out = np.zeros((len(qs), kg.shape[1]))
+    for i in range(len(qs)):
+        b = wl.q_req[qs[i]]
+        dg = np.maximum(q[i] @ kg[b].T, 0.0)                 # [H, P]
+        dr = np.maximum(q[i] @ kr[b].T, 0.0)
+        s_exact = gg[i] @ dg
+        out[i] = (1e-5 * np.maximum(1.0, np.abs(s_exact)) + np.abs(gg[i] - gr[i]) @ dg
+                  + np.abs(gr[i]) @ np.abs(dg - dr) + 2.0 ** -24 * np.abs(gr[i] @ dr))
+    return out
+
+
 def end_to_end(wl, g, queries=None):
-    """Oracle from raw inputs vs the GPU: selections may differ only near the K-th score."""
+    """Oracle from raw inputs vs the GPU.
+
+    Validity, candidates and pool indices are bit-exact. Every candidate's GPU
+    score lies within its bound E (e2e_score_bound). The selections may differ
+    only by swaps that those bounds explain: for every pool p the oracle selects
+    and the GPU does not, and every pool p' the GPU selects and the oracle does
+    not, s_ref[p] - E[p] <= s_ref[p'] + E[p']. Where both sides hold the same
+    pooled keys, E is the gate and arithmetic tolerance (about 2e-5 of the
+    score's terms), so swaps stay within the specification's score gap. Rows
+    whose selections agree have bit-exact token ids and their MLA output is
+    compared with the oracle's.
+    """
     qs = np.arange(wl.Q) if queries is None else np.asarray(queries)
-    ref = O.pipeline(wl, queries=qs)
-    np.testing.assert_array_equal(g["pool_valid"], ref["pool_valid"])
-    np.testing.assert_array_equal(g["cand"][qs], ref["cand"])
+    gate_ref = O.head_gate(wl.hidden[qs], wl.w_gate)
+    keys, idx, pv, fv = O.kpool_compress(wl.k, wl.gate, wl.valid, wl.req_start, wl.kpool,
+                                         wl.max_pools, wl.ape, wl.ln_w, wl.ln_b, wl.eps)
+    np.testing.assert_array_equal(g["pool_valid"], pv)
+    np.testing.assert_array_equal(g["pool_idx"], idx)
+    np.testing.assert_array_equal(g["first_valid"], fv)
+    s_ref, c_ref = O.index_scores(wl.q_idx[qs], gate_ref, wl.q_req[qs], wl.q_pos[qs], keys, pv, fv,
+                                  wl.kpool)
+    np.testing.assert_array_equal(g["cand"][qs], c_ref)
+    top_ref, ids_ref = O.topk_expand(s_ref, c_ref, idx, wl.q_req[qs], wl.select_k)
+    E = e2e_score_bound(wl, qs, g, gate_ref, keys)
+    cand = c_ref.astype(bool)
+    s_gpu = g["scores"][qs].astype(np.float64)
+    sr = s_ref.astype(np.float64)
+    err = np.abs(s_gpu - sr)
+    assert (err[cand] <= E[cand]).all(), f"{(err[cand] > E[cand]).sum()} scores outside their bound"
     agree_rows = []
     swaps = 0
     for i, q in enumerate(qs):
-        a = set(ref["top_pools"][i][ref["top_pools"][i] >= 0].tolist())
-        gg = set(g["top_pools"][q][g["top_pools"][q] >= 0].tolist())
-        assert len(a) == len(gg)
-        diff = a ^ gg
-        if not diff:
+        a = set(top_ref[i][top_ref[i] >= 0].tolist())
+        gs = set(g["top_pools"][q][g["top_pools"][q] >= 0].tolist())
+        assert len(a) == len(gs)
+        if a == gs:
             agree_rows.append(i)
+            np.testing.assert_array_equal(g["token_ids"][q], ids_ref[i])
             continue
-        swaps += len(diff) // 2
-        s_ref = ref["scores"][i].astype(np.float64)
-        s_gpu = g["scores"][q].astype(np.float64)
-        fin = np.isfinite(s_ref)
-        delta = np.abs(s_gpu[fin] - s_ref[fin]).max()
-        kth = np.sort(s_ref[list(a)])[0]
-        for p in diff:
-            gap = abs(s_ref[p] - kth)
-            assert gap <= 2 * delta + 2e-5 * max(1.0, abs(kth)), (q, p, gap, delta)
-    K = wl.select_k
-    assert swaps <= max(1, 0.01 * K * len(qs)), f"{swaps} swapped pools"
+        out_, in_ = np.array(sorted(a - gs)), np.array(sorted(gs - a))
+        swaps += len(out_)
+        worst_out = (sr[i, out_] - E[i, out_]).max()
+        best_in = (sr[i, in_] + E[i, in_]).min()
+        assert worst_out <= best_in, (int(q), worst_out, best_in)
     if agree_rows:
         rows = np.asarray(agree_rows)
-        vb = mla_value_bound(wl.kv, wl.req_start, wl.q_req[qs[rows]], ref["token_ids"][rows])
-        assert_mla_close(g["out"][qs[rows]], ref["out"][rows], g["lse"][qs[rows]],
-                         ref["lse"][rows], vbound=vb)
-    return dict(swaps=swaps, agree=len(agree_rows))
+        out, lse = O.sparse_mla(wl.q_mla[qs[rows]], wl.kv, wl.req_start, wl.q_req[qs[rows]],
+                                ids_ref[rows], wl.sm_scale)
+        vb = mla_value_bound(wl.kv, wl.req_start, wl.q_req[qs[rows]], ids_ref[rows])
+        assert_mla_close(g["out"][qs[rows]], out, g["lse"][qs[rows]], lse, vbound=vb)
+    return dict(swaps=swaps, agree=len(agree_rows), max_err_over_bound=float((err[cand] / E[cand]).max()))
 
 
 # ----------------------------------------------------------------------------- configurations
@@ -124,7 +170,7 @@ def test_config_ragged(B):
     wl = workload("ragged")
     step, g = run_step(wl)
     rep = stagewise(wl, g)
-    print("ragged", rep)
+    print("ragged", rep, end_to_end(wl, g))
     device_status_clean(B)
 
 
@@ -136,8 +182,10 @@ def test_config_long_context(B):
     device_status_clean(B)
 
 
-def test_config_prefill_sampled(B):
-    """2048 queries: scores/top-k/expand for every query, gate and MLA on a sample."""
+def test_config_prefill(B):
+    """2048 queries: gate, scores, top-k and expand for every query; the end-to-end
+    check compares the MLA output of every query whose selection agrees with the
+    oracle's; the stage-wise MLA check on the GPU's own ids takes a sample."""
     wl = workload("prefill")
     step, g = run_step(wl)
     sample = np.r_[0:8, 1020:1028, 2040:2048]
@@ -150,7 +198,9 @@ def test_config_prefill_sampled(B):
     # causality: every selected token is at or before its query's position
     sel = g["token_ids"]
     assert ((sel < 0) | (sel <= wl.q_pos[:, None])).all()
-    print("prefill", rep)
+    e2e = end_to_end(wl, g)
+    assert e2e["agree"] > 0
+    print("prefill", rep, e2e)
     device_status_clean(B)
 
 
