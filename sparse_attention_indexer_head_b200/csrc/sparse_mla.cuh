@@ -809,20 +809,22 @@ inline int mla_max_clusters(int splits) {
     return n;
 }
 
-// The launch: a plan of 2..8 splits runs as clusters when all of a grid's
-// clusters can be resident at once, shrinking the cluster (more chunks per CTA)
-// while that costs at most two chunks per CTA over the plan -- about what the
-// global merge costs; otherwise the plan runs with global partials.
+// The launch: a plan of 2 or more splits runs as clusters of at most 8 CTAs
+// when all of a grid's clusters can be resident at once, shrinking the cluster
+// (more chunks per CTA) while that costs at most two chunks per CTA over the
+// plan -- about what the global merge and its second launch cost; otherwise
+// the plan runs with global partials.
 inline MlaGeom mla_launch_geometry(int Q, int Hm, int W) {
     MlaGeom g = mla_plan(Q, Hm, W);
-    if (g.S < 2 || g.S > kMaxClusterSplits) return g;
+    if (g.S < 2) return g;
     const long long ctas = (long long)Q * ((Hm + kTcHeads - 1) / kTcHeads);
     const int chunks = ceil_div(W, kTcChunk);
     const int base = g.per / kTcChunk;
-    for (int s = g.S; s >= 2; --s) {
+    for (int s = std::min(g.S, kMaxClusterSplits); s >= 2; --s) {
         const int pc = ceil_div(chunks, s);
         if (pc > base + 2) break;
         const int ss = ceil_div(chunks, pc);
+        if (ss < 2) break;
         if ((long long)mla_max_clusters(ss) >= ctas) return MlaGeom{ss, pc * kTcChunk, true};
     }
     return g;
