@@ -68,8 +68,12 @@ def algorithmic_bytes(wl) -> dict:
     n_sel = np.minimum(wl.select_k, n_span[wl.q_req])          # pools selected (decode: all cand)
     topk = int(Q * P * 5 + (n_sel * kp * 4).sum() + Q * (4 * wl.select_k + 4 * wl.out_width + 4))
     mla = int((n_sel * kp * L * 2).sum() + Q * (wl.hm * L * 2 * 2 + 4 * wl.out_width + 4 * wl.hm + 4))
-    return dict(head_gate=gate, kpool_compress=compress, index_scores=scores,
-                topk_expand=topk, sparse_mla=mla)
+    out = dict(head_gate=gate, kpool_compress=compress, index_scores=scores,
+               topk_expand=topk, sparse_mla=mla)
+    # the fused indexer moves the three stages' bytes but the ones they pass each other
+    # through memory: the gate rows the scores read, the scores and flags top-k reads
+    out["indexer"] = gate + scores + topk - Q * 4 * H - Q * P * 5
+    return out
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -168,7 +172,7 @@ def kernel_source_sha(kernel_file: str) -> str:
 # kernel source of each stage (its DRAM traffic is valid only for that source)
 STAGE_SOURCE = {"head_gate": "head_gate.cuh", "kpool_compress": "kpool_compress.cuh",
                 "index_scores": "index_scores.cuh", "topk_expand": "topk_expand.cuh",
-                "sparse_mla": "sparse_mla.cuh"}
+                "indexer": "indexer.cuh", "sparse_mla": "sparse_mla.cuh"}
 
 
 def traffic_for(kernel: str, kernel_file: str, workload: str):
@@ -328,9 +332,6 @@ def reference_arm(args, wl):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-STAGES = ["head_gate", "kpool_compress", "index_scores", "topk_expand", "sparse_mla"]
-
-
 def stage_times(steps, stream, names, n_rep):
     """Mean device time (ms) of each stage on its own. Each stage is bracketed by events
     and preceded by a short device sleep, so the CPU has enqueued the event/kernel/event
@@ -380,11 +381,16 @@ def measure(args, wl, dev, rank, world, local, headline: bool) -> dict:
     from sparse_attention_indexer_head_b200 import binding as B
     from sparse_attention_indexer_head_b200.pipeline import (QUERY_INPUTS, DecodeStep,
                                                              StreamedDecode, host_tensors)
-    per_stage_bytes = algorithmic_bytes(wl)
+    fused = args.path == "fused"
+    all_bytes = algorithmic_bytes(wl)
+    host = host_tensors(wl)
+    steps = [DecodeStep(wl, device=str(dev), inputs=host, fused_indexer=fused)]
+    names = steps[0].stages()
+    per_stage_bytes = {n: all_bytes[n] for n in names}
     step_bytes = sum(per_stage_bytes.values())
     n_sets = input_sets(step_bytes, args.sets)
-    host = host_tensors(wl)
-    steps = [DecodeStep(wl, device=str(dev), inputs=host) for _ in range(n_sets)]
+    steps += [DecodeStep(wl, device=str(dev), inputs=host, fused_indexer=fused)
+              for _ in range(n_sets - 1)]
     stream = torch.cuda.Stream(device=dev)
     clocks = ClockSampler(local) if rank == 0 else None
 
@@ -413,7 +419,7 @@ def measure(args, wl, dev, rank, world, local, headline: bool) -> dict:
     clk = clocks.summary(t_wall0, t_wall1) if clocks else None
 
     n_rep = max(5, min(args.steps, 100))
-    stage_ms = stage_times(steps, stream, STAGES, n_rep)
+    stage_ms = stage_times(steps, stream, names, n_rep)
 
     incremental = None
     if headline:
@@ -446,7 +452,7 @@ def measure(args, wl, dev, rank, world, local, headline: bool) -> dict:
             "stage_us": {k: 1e3 * v for k, v in inc_stage.items()},
             "new_rows_per_step": steps[0].new["n"],
             "path": "dsa_indexer_store of each request's new row -> dsa_kpool_compress_tokens "
-                    "over its pools -> gate, scores, top-k, MLA as in the step above",
+                    "over its pools -> the indexer stage(s) and the MLA as in the step above",
         }
         del inc_graphs
 
@@ -459,7 +465,7 @@ def measure(args, wl, dev, rank, world, local, headline: bool) -> dict:
     # back, with consecutive steps on two streams; every step's output is read on the
     # host (step i-1's while step i is enqueued) inside the timed region. The loop
     # runs at least --e2e-seconds, whatever --steps is, so it measures steady state.
-    sd = StreamedDecode(wl, device=str(dev), slots=2, inputs=host)
+    sd = StreamedDecode(wl, device=str(dev), slots=2, inputs=host, fused_indexer=fused)
     for k in range(2):
         sd.write_inputs(k, {n: host[n] for n in QUERY_INPUTS})
     h2d = sd.nbytes
@@ -523,7 +529,7 @@ def measure(args, wl, dev, rank, world, local, headline: bool) -> dict:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/f32",
         "data": "synthetic",
-        "config": {"workload": wl.name, "global_batch": wl.Q * world,
+        "config": {"workload": wl.name, "path": args.path, "global_batch": wl.Q * world,
                    "seq_len": int(max(wl.lengths)), "parallelism": f"replicas x{world}",
                    "l2": f"inputs rotated over {n_sets} device-resident sets "
                          f"({n_sets * step_bytes / 1e9:.2f} GB > L2)",
@@ -538,7 +544,7 @@ def measure(args, wl, dev, rank, world, local, headline: bool) -> dict:
         "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "seconds": e2e_s,
                 "path": "StreamedDecode: per step one graph replay of H2D of the packed pinned "
-                        "query inputs -> the five ABI calls -> D2H of out, consecutive steps "
+                        "query inputs -> the step's ABI calls -> D2H of out, consecutive steps "
                         "on two streams; each step's output read on the host"},
         "gpu_launches": launches,
         "incremental": incremental,
@@ -578,6 +584,8 @@ def main():
     ap.add_argument("--config", default="batched",
                     choices=["tiny", "batched", "ragged", "long", "prefill", "all"])
     ap.add_argument("--sets", type=int, default=0, help="input sets to rotate (0: enough for L2)")
+    ap.add_argument("--path", default="fused", choices=["fused", "staged"],
+                    help="fused: compress -> dsa_indexer_select -> MLA; staged: the five calls")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--cpu-queries", type=int, default=16)
     ap.add_argument("--e2e-seconds", type=float, default=0.5)

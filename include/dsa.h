@@ -264,6 +264,40 @@ int dsa_topk_expand_tail(const float *scores, const uint8_t *cand, const int32_t
                          int32_t *token_ids, dsa_stream_t stream);
 
 /*
+ * f3. The fused indexer: a1 + a4 + a5 + a6 in one launch ([PR227] the
+ * FUSED_K_GATE arm, which computes the head gate inside the indexer instead of
+ * as a separate GEMM; [mod.rs] "Shape of the pipeline" second to fourth
+ * arrows).
+ *   hidden fp32 [Q, K], w fp32 [K, H]: the head gate's operands; one gate row
+ *             per query (gate_w[q, h] = sum_k hidden[q, k] * w[k, h]).
+ *   q_idx, q_req, q_pos, pool_keys, pool_valid, first_valid: as for
+ *             dsa_index_scores; pool_idx, select_k: as for dsa_topk_expand.
+ * Outputs, each as the separate call writes it: gate_w fp32 [Q, H] (as
+ * dsa_head_gate), scores fp32 [Q, max_pools] and cand uint8 [Q, max_pools]
+ * (as dsa_index_scores, from this gate_w), top_pools int32 [Q, select_k] and
+ * token_ids int32 [Q, select_k * kpool] (as dsa_topk_expand, from these
+ * scores: the same ranking, ties and -1 tail).
+ * One thread-block cluster of up to 8 CTAs per query splits K for the gate and
+ * the pools for the scores; partial gates and the top-k histograms meet
+ * through distributed shared memory, so nothing but the outputs goes to
+ * global memory and results are deterministic. The gate's K-split differs from
+ * dsa_head_gate's, so gate_w (and the scores after it) may differ from the
+ * separate calls' in the last bits; both are held to the same tolerance.
+ * hidden, w, q_idx, q_req and q_pos are read before the wait on the preceding
+ * kernel (see the conventions above).
+ * Requires D == 128, 1 <= H <= 16, K >= 1, 1 <= kpool <= 8,
+ * 0 <= select_k <= 4096 and max_pools <= 32768 (DSA_ERR_UNSUPPORTED above:
+ * dsa_index_scores + dsa_topk_expand serve larger pool counts).
+ * Alignment: hidden, w 4 bytes; q_idx, pool_keys 16; int32 arrays 4.
+ */
+int dsa_indexer_select(const float *hidden, const float *w, int K, const dsa_bf16 *q_idx,
+                       const int32_t *q_req, const int32_t *q_pos, int Q, int H, int D,
+                       const dsa_bf16 *pool_keys, const uint8_t *pool_valid,
+                       const int32_t *first_valid, const int32_t *pool_idx, int B, int kpool,
+                       int max_pools, int select_k, float *gate_w, float *scores, uint8_t *cand,
+                       int32_t *top_pools, int32_t *token_ids, dsa_stream_t stream);
+
+/*
  * a7. NoPE MLA restricted to the selected tokens ([mod.rs] "Shape of the
  * pipeline" last arrow; MASKED_ATTN_MAX_KEYS doc: set-membership mask, so a
  * per-row gather is exact; trap 5: qk_rope_head_dim == 0, the 512-wide latent

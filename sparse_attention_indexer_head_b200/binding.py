@@ -27,7 +27,7 @@ EXPORTS = (
     "dsa_status_string", "dsa_abi_version", "dsa_device_status", "dsa_selftest_bounded_wait",
     "dsa_head_gate", "dsa_head_gate_supported",
     "dsa_kpool_compress", "dsa_indexer_store", "dsa_kpool_compress_tokens",
-    "dsa_index_scores", "dsa_topk_expand", "dsa_topk_expand_tail",
+    "dsa_index_scores", "dsa_topk_expand", "dsa_topk_expand_tail", "dsa_indexer_select",
     "dsa_sparse_mla_workspace_size", "dsa_sparse_mla_launch_count", "dsa_sparse_mla_decode",
     "dsa_sparse_mla_decode_noalloc", "dsa_sparse_mla_decode_paged",
     "dsa_sparse_mla_decode_paged_fp8", "dsa_noalloc_scratch_bytes",
@@ -63,6 +63,8 @@ def _load() -> ctypes.CDLL:
         "dsa_index_scores": ([P, P, P, P, I, I, I, P, P, P, I, I, I, P, P, P], I),
         "dsa_topk_expand": ([P, P, P, P, I, I, I, I, I, P, P, P], I),
         "dsa_topk_expand_tail": ([P, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P], I),
+        "dsa_indexer_select": ([P, P, I, P, P, P, I, I, I, P, P, P, P, I, I, I, I, P, P, P, P, P, P],
+                               I),
         "dsa_sparse_mla_workspace_size": ([I, I, I], Z),
         "dsa_sparse_mla_launch_count": ([I, I, I], I),
         "dsa_sparse_mla_decode": ([P, P, I64, P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P], I),
@@ -182,6 +184,16 @@ def dsa_topk_expand_tail(scores, cand, pool_idx, q_req, q_pos, first_valid, tok_
         _ptr(scores), _ptr(cand), _ptr(pool_idx), _ptr(q_req), _ptr(q_pos), _ptr(first_valid),
         _ptr(tok_valid), _ptr(req_start), Q, B, max_pools, kpool, select_k, _ptr(top_pools),
         _ptr(token_ids), _stream(stream)))
+
+
+def dsa_indexer_select(hidden, w, K: int, q_idx, q_req, q_pos, Q: int, H: int, D: int, pool_keys,
+                       pool_valid, first_valid, pool_idx, B: int, kpool: int, max_pools: int,
+                       select_k: int, gate_w, scores, cand, top_pools, token_ids,
+                       stream=None) -> None:
+    _check("dsa_indexer_select", lib.dsa_indexer_select(
+        _ptr(hidden), _ptr(w), K, _ptr(q_idx), _ptr(q_req), _ptr(q_pos), Q, H, D, _ptr(pool_keys),
+        _ptr(pool_valid), _ptr(first_valid), _ptr(pool_idx), B, kpool, max_pools, select_k,
+        _ptr(gate_w), _ptr(scores), _ptr(cand), _ptr(top_pools), _ptr(token_ids), _stream(stream)))
 
 
 def dsa_sparse_mla_workspace_size(Q: int, Hm: int, W: int) -> int:

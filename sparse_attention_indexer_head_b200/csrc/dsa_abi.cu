@@ -8,6 +8,7 @@
 #include "indexer_store.cuh"
 #include "index_scores.cuh"
 #include "topk_expand.cuh"
+#include "indexer.cuh"
 #include "sparse_mla.cuh"
 
 // ---------------------------------------------------------------------------------------
@@ -150,6 +151,18 @@ int dsa_topk_expand_tail(const float *scores, const uint8_t *cand, const int32_t
     return dsa::topk_expand_launch(scores, cand, pool_idx, q_req, Q, B, max_pools, kpool,
                                    select_k, tail, top_pools, token_ids,
                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dsa_indexer_select(const float *hidden, const float *w, int K, const dsa_bf16 *q_idx,
+                       const int32_t *q_req, const int32_t *q_pos, int Q, int H, int D,
+                       const dsa_bf16 *pool_keys, const uint8_t *pool_valid,
+                       const int32_t *first_valid, const int32_t *pool_idx, int B, int kpool,
+                       int max_pools, int select_k, float *gate_w, float *scores, uint8_t *cand,
+                       int32_t *top_pools, int32_t *token_ids, dsa_stream_t stream) {
+    return dsa::indexer_launch(hidden, w, K, q_idx, q_req, q_pos, Q, H, D, pool_keys, pool_valid,
+                               first_valid, pool_idx, B, kpool, max_pools, select_k, gate_w,
+                               scores, cand, top_pools, token_ids,
+                               reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t dsa_sparse_mla_workspace_size(int Q, int Hm, int W) {

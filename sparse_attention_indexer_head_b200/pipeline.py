@@ -1,9 +1,11 @@
-"""One DSA decode/prefill step on the GPU: device buffers plus the five C-ABI calls.
+"""One DSA decode/prefill step on the GPU: device buffers plus the C-ABI calls.
 
 PyTorch is used for device memory, pinned host memory and streams only; every
 stage runs in libdsa.so:
-  dsa_head_gate -> dsa_kpool_compress -> dsa_index_scores -> dsa_topk_expand
-  -> dsa_sparse_mla_decode.
+  dsa_kpool_compress -> dsa_head_gate -> dsa_index_scores -> dsa_topk_expand
+  -> dsa_sparse_mla_decode,
+or, with the fused indexer, dsa_kpool_compress -> dsa_indexer_select (gate,
+scores, top-k and expansion in one launch) -> dsa_sparse_mla_decode.
 Cache-side tensors (k, gate logits, validity, latent kv, request offsets and
 the layer weights) are device-resident state; query-side tensors (hidden,
 indexer queries, MLA queries, query request/position) are the per-step inputs.
@@ -67,8 +69,11 @@ class DecodeStep:
     """Device buffers of one step; ``run()`` enqueues the five calls on a stream."""
 
     def __init__(self, wl: Workload, device: str = "cuda", inputs: Optional[Dict] = None,
-                 always_select_tail: bool = False):
+                 always_select_tail: bool = False, fused_indexer: bool = False):
         self.device = torch.device(device)
+        # fused_indexer: gate, scores, top-k and expansion in one dsa_indexer_select
+        # call (not with always_select_tail, whose tail slots only dsa_topk_expand_tail writes)
+        self.fused = bool(fused_indexer) and not always_select_tail
         self.g = Geometry(wl.B, wl.Q, wl.kpool, wl.max_pools, wl.select_k, wl.hm, wl.eps,
                           wl.sm_scale, wl.kpool - 1 if always_select_tail else 0)
         src = host_tensors(wl) if inputs is None else inputs
@@ -126,14 +131,26 @@ class DecodeStep:
                                 g.Q, g.B, g.hm, g.W, KV_LORA, 0, g.sm_scale, self.out, self.lse,
                                 self.ws, self.ws.numel(), stream)
 
-    def run(self, stream=None):
+    def indexer(self, stream=None):
+        """a1 + a4 + a5 + a6 in one launch (dsa_indexer_select)."""
+        g, t = self.g, self.t
+        B.dsa_indexer_select(t["hidden"], t["w_gate"], t["hidden"].shape[1], t["q_idx"], t["q_req"],
+                             t["q_pos"], g.Q, INDEX_HEADS, INDEX_DIM, self.pool_keys,
+                             self.pool_valid, self.first_valid, self.pool_idx, g.B, g.kpool,
+                             g.max_pools, g.select_k, self.gate_w, self.scores, self.cand,
+                             self.top_pools, self.token_ids, stream)
+
+    def stages(self):
+        """Names of the stage methods run() calls, in order."""
+        if self.fused:
+            return ["kpool_compress", "indexer", "sparse_mla"]
         # compress first: the small head-gate grid then overlaps compress's tail
         # (every kernel is launched with programmatic dependent launch).
-        self.kpool_compress(stream)
-        self.head_gate(stream)
-        self.index_scores(stream)
-        self.topk_expand(stream)
-        self.sparse_mla(stream)
+        return ["kpool_compress", "head_gate", "index_scores", "topk_expand", "sparse_mla"]
+
+    def run(self, stream=None):
+        for name in self.stages():
+            getattr(self, name)(stream)
 
     # -- incremental decode: the step's new token rows update the pooled-key cache -------
     def stage_new_tokens(self, k_new=None, gate_new=None, valid_new=None, tok_req=None,
@@ -192,22 +209,20 @@ class DecodeStep:
         """
         self.indexer_store(stream)
         self.kpool_compress_tokens(stream)
-        self.head_gate(stream)
-        self.index_scores(stream)
-        self.topk_expand(stream)
-        self.sparse_mla(stream)
+        for name in self.stages()[1:]:
+            getattr(self, name)(stream)
 
     def kernels_per_step(self) -> int:
-        """Launches of run(): gate, compress, scores, topk+expand, and the MLA's one or
-        two kernels (split kernel, plus the combine when splits merge in the workspace)."""
+        """Launches of run(): compress, then gate, scores and topk+expand (or the one fused
+        indexer), and the MLA's one or two kernels (split kernel, plus the combine when
+        splits merge in the workspace)."""
         g = self.g
-        return 4 + B.dsa_sparse_mla_launch_count(g.Q, g.hm, g.W)
+        return len(self.stages()) - 1 + B.dsa_sparse_mla_launch_count(g.Q, g.hm, g.W)
 
     def kernels_per_step_incremental(self) -> int:
         """Launches of run_incremental(): store (when there are new rows), token-range
-        compress, gate, scores, topk+expand and the MLA's kernels."""
-        g = self.g
-        return (1 if self.new["n"] > 0 else 0) + 4 + B.dsa_sparse_mla_launch_count(g.Q, g.hm, g.W)
+        compress, the indexer stage(s) and the MLA's kernels."""
+        return (1 if self.new["n"] > 0 else 0) + self.kernels_per_step()
 
     def outputs_numpy(self) -> Dict[str, np.ndarray]:
         def u16(x):
@@ -241,9 +256,10 @@ class StreamedDecode:
     """
 
     def __init__(self, wl: Workload, device: str = "cuda", slots: int = 2,
-                 inputs: Optional[Dict] = None):
+                 inputs: Optional[Dict] = None, fused_indexer: bool = False):
         self.device = torch.device(device)
-        self.steps = [DecodeStep(wl, device=device, inputs=inputs) for _ in range(slots)]
+        self.steps = [DecodeStep(wl, device=device, inputs=inputs, fused_indexer=fused_indexer)
+                      for _ in range(slots)]
         # A slot's query inputs live in one device buffer: one copy per step.
         self.layout, nbytes = {}, 0
         for name in QUERY_INPUTS:

@@ -22,6 +22,7 @@ import functools
 import numpy as np
 import torch
 
+import oracle as O
 from sparse_attention_indexer_head_b200 import workloads as W
 
 
@@ -179,3 +180,132 @@ def dev_bits(x: np.ndarray, device="cuda") -> torch.Tensor:
 
 def host_bits(t: torch.Tensor) -> np.ndarray:
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+# ----------------------------------------------------------------------------- path checks
+def run_step(wl, canary=True, fused=False):
+    """One step of the path on the workload (the fused indexer when fused is set),
+    with every output first filled with 0x7F bytes so a missed write shows."""
+    from sparse_attention_indexer_head_b200.pipeline import DecodeStep
+    step = DecodeStep(wl, fused_indexer=fused)
+    if canary:   # every output the contract says is written must lose the 0x7F fill
+        for t in (step.gate_w, step.pool_idx, step.pool_valid, step.first_valid, step.scores,
+                  step.cand, step.top_pools, step.token_ids, step.out, step.lse):
+            t.view(torch.uint8).fill_(0x7F)
+    step.run()
+    torch.cuda.synchronize()
+    return step, step.outputs_numpy()
+
+
+def stagewise(wl, g, queries=None):
+    """Each oracle stage on the GPU's inputs to that stage; returns a report dict."""
+    rep = {}
+    qs = np.arange(wl.Q) if queries is None else np.asarray(queries)
+    # a1
+    ref_gate = O.head_gate(wl.hidden[qs], wl.w_gate)
+    rep["gate_max_abs"] = assert_gate_close(g["gate_w"][qs], ref_gate)
+    # a2+a3
+    keys, idx, pv, fv = O.kpool_compress(wl.k, wl.gate, wl.valid, wl.req_start, wl.kpool,
+                                         wl.max_pools, wl.ape, wl.ln_w, wl.ln_b, wl.eps)
+    np.testing.assert_array_equal(g["first_valid"], fv)
+    np.testing.assert_array_equal(g["pool_valid"], pv)
+    np.testing.assert_array_equal(g["pool_idx"], idx)
+    rep["keys"] = assert_keys_close(g["pool_keys"], keys, pv, wl, fv)
+    # a4 on GPU gate_w and GPU pool tensors
+    sc, cd = O.index_scores(wl.q_idx[qs], g["gate_w"][qs], wl.q_req[qs], wl.q_pos[qs],
+                            g["pool_keys"], g["pool_valid"], g["first_valid"], wl.kpool)
+    np.testing.assert_array_equal(g["cand"][qs], cd)
+    mag = score_magnitude(wl.q_idx[qs], g["gate_w"][qs], g["pool_keys"], wl.q_req[qs])
+    rep["scores"] = assert_scores_close(g["scores"][qs], sc, cd, mag)
+    # a5+a6 on GPU scores: bit-exact
+    top, ids = O.topk_expand(g["scores"][qs], g["cand"][qs], g["pool_idx"], wl.q_req[qs],
+                             wl.select_k)
+    np.testing.assert_array_equal(g["top_pools"][qs], top)
+    np.testing.assert_array_equal(g["token_ids"][qs], ids)
+    # a7 on GPU token ids
+    out, lse = O.sparse_mla(wl.q_mla[qs], wl.kv, wl.req_start, wl.q_req[qs], g["token_ids"][qs],
+                            wl.sm_scale)
+    vb = mla_value_bound(wl.kv, wl.req_start, wl.q_req[qs], g["token_ids"][qs])
+    rep["mla"] = assert_mla_close(g["out"][qs], out, g["lse"][qs], lse, vbound=vb)
+    return rep
+
+
+def e2e_score_bound(wl, qs, g, gate_ref, keys_ref):
+    """Per-pool bound of |GPU score - oracle score from raw inputs|, [len(qs), P].
+
+    The GPU scores a pool from its own head gate and pooled keys; the oracle
+    from its own. In exact arithmetic the two scores differ by
+      sum_h (g_gpu_h - g_ref_h) relu(d_gpu_h) + sum_h g_ref_h (relu(d_gpu_h) - relu(d_ref_h))
+    (d: the head dots with each side's pooled key), and the GPU's fp32 score is
+    within 1e-5 max(1, |score|) of its exact value (the stage-wise tolerance),
+    the oracle's within half an fp32 ulp. The bound is the sum of those terms'
+    magnitudes: where both sides hold the same pooled key it is the gate and
+    arithmetic tolerances alone.
+    """
+    q = bf16f(wl.q_idx[qs])
+    kg, kr = bf16f(g["pool_keys"]), bf16f(keys_ref)
+    gg = g["gate_w"][qs].astype(np.float64)
+    gr = gate_ref.astype(np.float64)
+    out = np.zeros((len(qs), kg.shape[1]))
+    for i in range(len(qs)):
+        b = wl.q_req[qs[i]]
+        dg = np.maximum(q[i] @ kg[b].T, 0.0)                 # [H, P]
+        dr = np.maximum(q[i] @ kr[b].T, 0.0)
+        s_exact = gg[i] @ dg
+        out[i] = (1e-5 * np.maximum(1.0, np.abs(s_exact)) + np.abs(gg[i] - gr[i]) @ dg
+                  + np.abs(gr[i]) @ np.abs(dg - dr) + 2.0 ** -24 * np.abs(gr[i] @ dr))
+    return out
+
+
+def end_to_end(wl, g, queries=None):
+    """Oracle from raw inputs vs the GPU.
+
+    Validity, candidates and pool indices are bit-exact. Every candidate's GPU
+    score lies within its bound E (e2e_score_bound). The selections may differ
+    only by swaps that those bounds explain: for every pool p the oracle selects
+    and the GPU does not, and every pool p' the GPU selects and the oracle does
+    not, s_ref[p] - E[p] <= s_ref[p'] + E[p']. Where both sides hold the same
+    pooled keys, E is the gate and arithmetic tolerance (about 2e-5 of the
+    score's terms), so swaps stay within the specification's score gap. Rows
+    whose selections agree have bit-exact token ids and their MLA output is
+    compared with the oracle's.
+    """
+    qs = np.arange(wl.Q) if queries is None else np.asarray(queries)
+    gate_ref = O.head_gate(wl.hidden[qs], wl.w_gate)
+    keys, idx, pv, fv = O.kpool_compress(wl.k, wl.gate, wl.valid, wl.req_start, wl.kpool,
+                                         wl.max_pools, wl.ape, wl.ln_w, wl.ln_b, wl.eps)
+    np.testing.assert_array_equal(g["pool_valid"], pv)
+    np.testing.assert_array_equal(g["pool_idx"], idx)
+    np.testing.assert_array_equal(g["first_valid"], fv)
+    s_ref, c_ref = O.index_scores(wl.q_idx[qs], gate_ref, wl.q_req[qs], wl.q_pos[qs], keys, pv, fv,
+                                  wl.kpool)
+    np.testing.assert_array_equal(g["cand"][qs], c_ref)
+    top_ref, ids_ref = O.topk_expand(s_ref, c_ref, idx, wl.q_req[qs], wl.select_k)
+    E = e2e_score_bound(wl, qs, g, gate_ref, keys)
+    cand = c_ref.astype(bool)
+    s_gpu = g["scores"][qs].astype(np.float64)
+    sr = s_ref.astype(np.float64)
+    err = np.abs(s_gpu - sr)
+    assert (err[cand] <= E[cand]).all(), f"{(err[cand] > E[cand]).sum()} scores outside their bound"
+    agree_rows = []
+    swaps = 0
+    for i, q in enumerate(qs):
+        a = set(top_ref[i][top_ref[i] >= 0].tolist())
+        gs = set(g["top_pools"][q][g["top_pools"][q] >= 0].tolist())
+        assert len(a) == len(gs)
+        if a == gs:
+            agree_rows.append(i)
+            np.testing.assert_array_equal(g["token_ids"][q], ids_ref[i])
+            continue
+        out_, in_ = np.array(sorted(a - gs)), np.array(sorted(gs - a))
+        swaps += len(out_)
+        worst_out = (sr[i, out_] - E[i, out_]).max()
+        best_in = (sr[i, in_] + E[i, in_]).min()
+        assert worst_out <= best_in, (int(q), worst_out, best_in)
+    if agree_rows:
+        rows = np.asarray(agree_rows)
+        out, lse = O.sparse_mla(wl.q_mla[qs[rows]], wl.kv, wl.req_start, wl.q_req[qs[rows]],
+                                ids_ref[rows], wl.sm_scale)
+        vb = mla_value_bound(wl.kv, wl.req_start, wl.q_req[qs[rows]], ids_ref[rows])
+        assert_mla_close(g["out"][qs[rows]], out, g["lse"][qs[rows]], lse, vbound=vb)
+    return dict(swaps=swaps, agree=len(agree_rows), max_err_over_bound=float((err[cand] / E[cand]).max()))

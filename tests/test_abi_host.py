@@ -250,6 +250,33 @@ def test_paged_mla_refusals(B):
     assert L.dsa_sparse_mla_decode_paged_fp8(*bad) == B.DSA_OK               # Q == 0
 
 
+def test_indexer_select_refusals(B):
+    L = B.lib
+    #       hidden w     K     q_idx q_req q_pos Q  H   D    keys  pv    fv    pidx  B  kp mp    sk
+    args = [FAKE, FAKE, 4096, FAKE, FAKE, FAKE, 4, 16, 128, FAKE, FAKE, FAKE, FAKE, 2, 4, 2048, 512,
+            FAKE, FAKE, FAKE, FAKE, FAKE, None]
+    bad = list(args); bad[7] = 17
+    assert L.dsa_indexer_select(*bad) == B.DSA_ERR_UNSUPPORTED      # more than 16 heads
+    bad = list(args); bad[8] = 64
+    assert L.dsa_indexer_select(*bad) == B.DSA_ERR_UNSUPPORTED      # D is 128
+    bad = list(args); bad[14] = 9
+    assert L.dsa_indexer_select(*bad) == B.DSA_ERR_UNSUPPORTED      # kpool <= 8
+    bad = list(args); bad[15] = 32769
+    assert L.dsa_indexer_select(*bad) == B.DSA_ERR_UNSUPPORTED      # 8 CTAs x 4096 pools at most
+    bad = list(args); bad[16] = 4097
+    assert L.dsa_indexer_select(*bad) == B.DSA_ERR_UNSUPPORTED
+    bad = list(args); bad[2] = 0
+    assert L.dsa_indexer_select(*bad) == B.DSA_ERR_INVALID_ARG
+    bad = list(args); bad[0] = None
+    assert L.dsa_indexer_select(*bad) == B.DSA_ERR_INVALID_ARG
+    bad = list(args); bad[21] = None
+    assert L.dsa_indexer_select(*bad) == B.DSA_ERR_INVALID_ARG      # no token-id output
+    bad = list(args); bad[3] = FAKE + 8
+    assert L.dsa_indexer_select(*bad) == B.DSA_ERR_ALIGNMENT
+    bad = list(args); bad[6] = 0
+    assert L.dsa_indexer_select(*bad) == B.DSA_OK                   # Q == 0: nothing to do
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     """The binding has no fallback: without libdsa.so the import raises."""
     import importlib.util
