@@ -62,6 +62,8 @@ struct IxCtl {
     uint32_t tau;
     int req;
     int cnt[2];                         // this CTA's keys above / equal to tau (read by the cluster)
+    int base[2];                        // the lower-ranked CTAs' keys above / equal to tau
+    int tot[256];                       // the current pass's histogram summed over the cluster
     volatile int abort;
 };
 
@@ -242,8 +244,12 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     cluster_sync_all();
     if (tid < kIxHeads) {
         const uint32_t a = smem_u32(&ctl->gpart[tid]);
+        float v[kIxMaxCluster];
+#pragma unroll
+        for (int c = 0; c < kIxMaxCluster; ++c) v[c] = c < C ? ld_cluster_f32(cluster_map(a, c)) : 0.f;
         float g = 0.f;
-        for (int c = 0; c < C; ++c) g += ld_cluster_f32(cluster_map(a, c));
+#pragma unroll
+        for (int c = 0; c < kIxMaxCluster; ++c) g += v[c];      // rank order
         ctl->gate[tid] = tid < H ? g : 0.f;
         if (r == 0 && tid < H) gate_w[(size_t)q * H + tid] = g;
     }
@@ -327,7 +333,14 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     __syncthreads();
     cluster_sync_all();                           // histograms of pass 0 and candidate counts
     int ncand = 0;
-    for (int c = 0; c < C; ++c) ncand += ld_cluster_s32(cluster_map(smem_u32(&ctl->ncand), c));
+    {
+        int v[kIxMaxCluster];
+#pragma unroll
+        for (int c = 0; c < kIxMaxCluster; ++c)
+            v[c] = c < C ? ld_cluster_s32(cluster_map(smem_u32(&ctl->ncand), c)) : 0;
+#pragma unroll
+        for (int c = 0; c < kIxMaxCluster; ++c) ncand += v[c];
+    }
     const int nq = min(SK, ncand);
     const int nloc = rg.p_hi - rg.p_lo;
     uint32_t prefix = 0, pmask = 0;
@@ -343,16 +356,25 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
                 }
                 cluster_sync_all();
             }
+            {
+                // thread t sums bin t over the cluster (all loads in flight at once)
+                const uint32_t a = smem_u32(&ctl->hist[hb][tid]);
+                int v[kIxMaxCluster];
+#pragma unroll
+                for (int c = 0; c < kIxMaxCluster; ++c) v[c] = c < C ? ld_cluster_s32(cluster_map(a, c)) : 0;
+                int t = 0;
+#pragma unroll
+                for (int c = 0; c < kIxMaxCluster; ++c) t += v[c];
+                ctl->tot[tid] = t;
+            }
+            __syncthreads();
             if (tid < 32) {
-                // lane l owns bins 255-8l down to 248-8l, summed over the cluster
+                // lane l owns bins 255-8l down to 248-8l
                 int cbin[8], sum = 0;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const uint32_t a = smem_u32(&ctl->hist[hb][255 - 8 * tid - i]);
-                    int v = 0;
-                    for (int c = 0; c < C; ++c) v += ld_cluster_s32(cluster_map(a, c));
-                    cbin[i] = v;
-                    sum += v;
+                    cbin[i] = ctl->tot[255 - 8 * tid - i];
+                    sum += cbin[i];
                 }
                 int above = sum;
 #pragma unroll
@@ -397,15 +419,25 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
                 }
                 cluster_sync_all();
                 if (tid < 32) {
-                    // this lane's key: entry tid of the cluster's concatenated lists
-                    uint32_t mine = 0u;
-                    int n = 0;
-                    for (int c = 0; c < C; ++c) {
-                        const int nc = ld_cluster_s32(cluster_map(smem_u32(&ctl->nsmall), c));
-                        if (tid >= n && tid < n + nc)
-                            mine = ld_cluster_u32(cluster_map(smem_u32(&ctl->small[tid - n]), c));
-                        n += nc;
+                    // lane c < C reads CTA c's list length; lane tid then loads entry tid of
+                    // the cluster's lists concatenated in rank order
+                    const int nc = tid < C ? ld_cluster_s32(cluster_map(smem_u32(&ctl->nsmall), tid)) : 0;
+                    int incl = nc;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+                        if (tid >= off) incl += y;
                     }
+                    const int n = __shfl_sync(0xffffffffu, incl, 31);
+                    int owner = 0, start = 0;
+#pragma unroll
+                    for (int c = 0; c < kIxMaxCluster; ++c) {
+                        const int e = __shfl_sync(0xffffffffu, incl, c);      // end of CTA c's list
+                        const int b0 = e - __shfl_sync(0xffffffffu, nc, c);
+                        if (c < C && tid >= b0 && tid < e) { owner = c; start = b0; }
+                    }
+                    const uint32_t mine =
+                        tid < n ? ld_cluster_u32(cluster_map(smem_u32(&ctl->small[tid - start]), owner)) : 0u;
                     int gt = 0, ge = 0;
                     for (int j = 0; j < n; ++j) {
                         const uint32_t kj = __shfl_sync(0xffffffffu, mine, j);
@@ -444,11 +476,25 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         ctl->cnt[1] = tot_eq;
     }
     cluster_sync_all();
-    int base_gt = 0, base_eq = 0;
-    for (int c = 0; c < r; ++c) {
-        base_gt += ld_cluster_s32(cluster_map(smem_u32(&ctl->cnt[0]), c));
-        base_eq += ld_cluster_s32(cluster_map(smem_u32(&ctl->cnt[1]), c));
+    if (tid < 32) {
+        // counts of the lower-ranked CTAs, summed on one warp
+        int g = 0, e = 0;
+        if (tid < r) {
+            g = ld_cluster_s32(cluster_map(smem_u32(&ctl->cnt[0]), tid));
+            e = ld_cluster_s32(cluster_map(smem_u32(&ctl->cnt[1]), tid));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, off);
+            e += __shfl_xor_sync(0xffffffffu, e, off);
+        }
+        if (tid == 0) {
+            ctl->base[0] = g;
+            ctl->base[1] = e;
+        }
     }
+    __syncthreads();
+    const int base_gt = ctl->base[0], base_eq = ctl->base[1];
     const size_t wrow = (size_t)SK * KP;
     if (nq > 0) {
         const int eq0 = base_eq + before.y;
@@ -485,8 +531,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     if (warp == 0) tc::tmem_dealloc(tmem, 32);
 }
 
-// Cluster size for P pools: one CTA per 128-pool tile up to 8.
-inline int indexer_cluster(int P) { return std::max(1, std::min(kIxMaxCluster, ceil_div(P, kIxTile))); }
+// Cluster size: 8 CTAs whatever P (the gate's K-split uses every CTA; one with no
+// pool tile only adds its gate slice and takes part in the select).
+inline int indexer_cluster(int) { return kIxMaxCluster; }
 
 inline int indexer_launch(const float *hidden, const float *w, int K, const void *q_idx,
                           const int32_t *q_req, const int32_t *q_pos, int Q, int H, int D,
