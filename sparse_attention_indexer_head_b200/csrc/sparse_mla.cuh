@@ -70,6 +70,15 @@ constexpr uint32_t kOffP = kOffKV + 8 * kAtomKV;    // 2 buffers x 8 KB: [64 hea
 constexpr uint32_t kStageP = 8 * 1024;
 constexpr uint32_t kOffCtl = kOffP + 2 * kStageP;
 constexpr uint32_t kTmemCols = 512;
+// MMAs are issued by one thread in each of warps 0-3: a single issuing thread
+// starts about one tcgen05.mma every 128 cycles whatever the tile, and issuers
+// in different warps proceed in parallel. Warps 0 and 1 issue the two K-halves
+// of S into separate accumulators (added by the softmax); each of the four
+// issues the PV of one 128-latent block of O^T.
+constexpr int kIssuers = 4;
+constexpr int kSParts = 2;
+constexpr uint32_t kSCol = 256;                     // S buffers: [256, 256 + 2 * kSParts * chunk)
+static_assert(kSCol + 2 * kSParts * kTcChunk <= kTmemCols, "tensor memory columns");
 constexpr float kLazyRescale = 8.0f;                // log2 units
 constexpr int kMaxClusterSplits = 8;                // portable cluster size
 constexpr int kSmTarget = 148;                      // CTAs of one full wave (one CTA per SM)
@@ -254,18 +263,18 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
     if (tid == 32) {
         for (int i = 0; i < kTcSlots; ++i) {
             mbar_init(&ctl->kv_full[i], 4 * 32 + 4);   // four warps' lanes' copies + their masks' arrives
-            mbar_init(&ctl->kv_empty[i], 1);
+            mbar_init(&ctl->kv_empty[i], kIssuers);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&ctl->s_full[i], 1);
+            mbar_init(&ctl->s_full[i], kSParts);
             mbar_init(&ctl->s_empty[i], 128);
             mbar_init(&ctl->p_full[i], 128);
-            mbar_init(&ctl->p_empty[i], 1);
+            mbar_init(&ctl->p_empty[i], kIssuers);
         }
-        mbar_init(&ctl->o_done, 1);
-        mbar_init(&ctl->o_final, 1);
+        mbar_init(&ctl->o_done, kIssuers);
+        mbar_init(&ctl->o_final, kIssuers);
         mbar_init(&ctl->q_full, 128);
-        mbar_init(&ctl->fin, 1);
+        mbar_init(&ctl->fin, kIssuers);
         ctl->abort = 0;
         fence_mbarrier_init();
     }
@@ -288,60 +297,67 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
     pdl_wait();                       // token ids come from the predecessor grid
     pdl_launch_dependents();
 
-    if (warp == 0) {
-        // ------------------------------------------------------------------ MMA issuer
+    if (warp < kIssuers) {
+        // ------------------------------------------------------------------ MMA issuers
+        // Lane 0 of warp w issues the PV of latent block w and, for w < 2, the
+        // K-half w of every S.
         if (lane == 0 && nch > 0) {
+            const int w = warp;
+            const bool s_issuer = w < kSParts;
             constexpr uint32_t idS = tc::idesc_bf16(64, kTcChunk, false, false);
             constexpr uint32_t idPV = tc::idesc_bf16(128, 64, true, false);
             // Chunk c lives in ring slot c % 3: rows [48 slot, 48 slot + 48) of every
             // 144-row column atom.
-            // PV(cp): O^T += V^T P^T over the chunk's 48 tokens (three K-steps).
+            // PV(cp), block w: O^T[128w .. 128w+127] += V^T P^T over the chunk's 48
+            // tokens (three K-steps).
             auto issue_pv = [&](int cp) {
                 const int slot = cp % kTcSlots, pb = cp & 1;
                 tc::fence_after_sync();
+                tc::fence_proxy_async_smem();     // the slot was written by cp.async
 #pragma unroll
                 for (int ks = 0; ks < kTcChunk / 16; ++ks) {
-#pragma unroll
-                    for (int lb = 0; lb < 4; ++lb) {
-                        // V^T: MN-major, 64-latent atoms kAtomKV apart, 8-token groups 1 KB apart
-                        const uint64_t a = tc::desc_sw128(sKV + lb * 2 * kAtomKV + slot * kSlotRows + ks * 2048,
-                                                          kAtomKV, 1024);
-                        // P^T: K-major, 128-byte rows (48 of 64 tokens used), 8-head groups 1 KB apart
-                        const uint64_t bd = tc::desc_sw128(sP + pb * kStageP + ks * 32, 16, 1024);
-                        tc::mma_bf16_ss(tmem + lb * 64, a, bd, idPV, (cp > 0 || ks > 0) ? 1u : 0u);
-                    }
+                    // V^T: MN-major, 64-latent atoms kAtomKV apart, 8-token groups 1 KB apart
+                    const uint64_t a = tc::desc_sw128(sKV + w * 2 * kAtomKV + slot * kSlotRows + ks * 2048,
+                                                      kAtomKV, 1024);
+                    // P^T: K-major, 128-byte rows (48 of 64 tokens used), 8-head groups 1 KB apart
+                    const uint64_t bd = tc::desc_sw128(sP + pb * kStageP + ks * 32, 16, 1024);
+                    tc::mma_bf16_ss(tmem + w * 64, a, bd, idPV, (cp > 0 || ks > 0) ? 1u : 0u);
                 }
                 tc::mma_commit(&ctl->kv_empty[slot]);
                 tc::mma_commit(&ctl->p_empty[pb]);
                 tc::mma_commit(&ctl->o_done);
             };
-            // S(c) = Q K^T over chunk c's 48 tokens into S buffer c & 1.
+            // S(c), K-half w = Q K^T over latent [256w, 256w + 256) of chunk c's 48
+            // tokens, into S buffer c & 1, part w.
             auto issue_s = [&](int c) {
                 const int slot = c % kTcSlots, sb = c & 1;
                 tc::fence_after_sync();
                 tc::fence_proxy_async_smem();     // the slot was written by cp.async
-                const uint32_t d = tmem + 256 + sb * kTcChunk;
+                const uint32_t d = tmem + kSCol + (uint32_t)((sb * kSParts + w) * kTcChunk);
+                constexpr int kHalf = kL / 16 / kSParts;
 #pragma unroll
-                for (int kk = 0; kk < kL / 16; ++kk) {
+                for (int k2 = 0; k2 < kHalf; ++k2) {
+                    const int kk = w * kHalf + k2;
                     const uint32_t qo = (kk >> 2) * 8192 + (kk & 3) * 32;
                     const uint32_t ko = (kk >> 2) * kAtomKV + slot * kSlotRows + (kk & 3) * 32;
                     tc::mma_bf16_ss(d, tc::desc_sw128(sQ + qo, 16, 1024),
-                                    tc::desc_sw128(sKV + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
+                                    tc::desc_sw128(sKV + ko, 16, 1024), idS, k2 > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(&ctl->s_full[sb]);
             };
             // Event loop: issue whichever product is ready, PV first (it frees a
-            // stage pair for the gathers); give up after the wait bound without progress.
+            // slot for the gathers); give up after the wait bound without progress.
             bool ok = tc_wait(ctl, &ctl->q_full, 0);
-            int ns = 0, np = 0;
+            int ns = s_issuer ? 0 : nch, np = 0;
             long long t_last = clock64();
             while (ok && np < nch) {
-                if (np < ns && mbar_test(&ctl->p_full[np & 1], (np >> 1) & 1)) {
+                if ((np < ns || !s_issuer) && mbar_test(&ctl->p_full[np & 1], (np >> 1) & 1)) {
+                    // the softmax of chunk np waited for its rows: they have landed
                     issue_pv(np++);
                     t_last = clock64();
                     continue;
                 }
-                if (ns < nch) {
+                if (s_issuer && ns < nch) {
                     const bool ready = mbar_test(&ctl->kv_full[ns % kTcSlots], (ns / kTcSlots) & 1) &&
                                        (ns < 2 || mbar_test(&ctl->s_empty[ns & 1], ((ns >> 1) - 1) & 1));
                     if (ready) {
@@ -360,6 +376,8 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
             // o_final is single-use: once it completes every PV of this CTA has landed
             // (a parity wait on o_done cannot tell the last two PVs apart).
             if (ok) tc::mma_commit(&ctl->o_final);
+            // every MMA of this issuer has completed before tensor memory is released
+            tc::mma_commit(&ctl->fin);
         }
         __syncwarp();
     } else if (warp >= 8) {
@@ -509,10 +527,13 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
             bool bad = !tc_wait(ctl, &ctl->kv_full[slot], (c / kTcSlots) & 1);
             bad = bad || !tc_wait(ctl, &ctl->s_full[sb], (c >> 1) & 1);
             tc::fence_after_sync();
-            // 48 columns: this thread's 24 tokens par + 2i, i < 24
-            uint32_t r[24];
-            tc::tmem_ld16x64b_x16(tl + 256 + sb * kTcChunk, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-            tc::tmem_ld16x64b_x8(tl + 256 + sb * kTcChunk + 32, *reinterpret_cast<uint32_t(*)[8]>(&r[16]));
+            // 48 columns of each S part: this thread's 24 tokens par + 2i, i < 24
+            uint32_t r[24], r2[24];
+            const uint32_t sc0 = tl + kSCol + (uint32_t)(sb * kSParts * kTcChunk);
+            tc::tmem_ld16x64b_x16(sc0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+            tc::tmem_ld16x64b_x8(sc0 + 32, *reinterpret_cast<uint32_t(*)[8]>(&r[16]));
+            tc::tmem_ld16x64b_x16(sc0 + kTcChunk, *reinterpret_cast<uint32_t(*)[16]>(&r2[0]));
+            tc::tmem_ld16x64b_x8(sc0 + kTcChunk + 32, *reinterpret_cast<uint32_t(*)[8]>(&r2[16]));
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             mbar_arrive(&ctl->s_empty[sb]);
@@ -525,7 +546,8 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
             float mx = -INFINITY;
 #pragma unroll
             for (int i = 0; i < 24; ++i) {
-                z[i] = ((vmp >> (2 * i)) & 1) ? __uint_as_float(r[i]) * scale_log2 : -INFINITY;
+                z[i] = ((vmp >> (2 * i)) & 1) ? (__uint_as_float(r[i]) + __uint_as_float(r2[i])) * scale_log2
+                                              : -INFINITY;
                 mx = fmaxf(mx, z[i]);
             }
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -631,10 +653,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
     }
 
     // Every MMA of this CTA has completed before tensor memory is released.
-    if (warp == 0 && lane == 0) {
-        tc::mma_commit(&ctl->fin);
-        (void)mbar_wait(&ctl->fin, 0);
-    }
+    if (warp == 0 && lane == 0 && nch > 0) (void)mbar_wait(&ctl->fin, 0);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
