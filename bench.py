@@ -381,11 +381,12 @@ def measure(args, wl, dev, rank, world, local, headline: bool) -> dict:
     from sparse_attention_indexer_head_b200 import binding as B
     from sparse_attention_indexer_head_b200.pipeline import (QUERY_INPUTS, DecodeStep,
                                                              StreamedDecode, host_tensors)
-    fused = args.path == "fused"
+    fused = {"fused": True, "staged": False, "auto": "auto"}[args.path]
     all_bytes = algorithmic_bytes(wl)
     host = host_tensors(wl)
     steps = [DecodeStep(wl, device=str(dev), inputs=host, fused_indexer=fused)]
     names = steps[0].stages()
+    steps_fused = steps[0].fused
     per_stage_bytes = {n: all_bytes[n] for n in names}
     step_bytes = sum(per_stage_bytes.values())
     n_sets = input_sets(step_bytes, args.sets)
@@ -529,7 +530,8 @@ def measure(args, wl, dev, rank, world, local, headline: bool) -> dict:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/f32",
         "data": "synthetic",
-        "config": {"workload": wl.name, "path": args.path, "global_batch": wl.Q * world,
+        "config": {"workload": wl.name, "path": "fused" if steps_fused else "staged",
+                   "global_batch": wl.Q * world,
                    "seq_len": int(max(wl.lengths)), "parallelism": f"replicas x{world}",
                    "l2": f"inputs rotated over {n_sets} device-resident sets "
                          f"({n_sets * step_bytes / 1e9:.2f} GB > L2)",
@@ -584,8 +586,9 @@ def main():
     ap.add_argument("--config", default="batched",
                     choices=["tiny", "batched", "ragged", "long", "prefill", "all"])
     ap.add_argument("--sets", type=int, default=0, help="input sets to rotate (0: enough for L2)")
-    ap.add_argument("--path", default="fused", choices=["fused", "staged"],
-                    help="fused: compress -> dsa_indexer_select -> MLA; staged: the five calls")
+    ap.add_argument("--path", default="auto", choices=["auto", "fused", "staged"],
+                    help="fused: compress -> dsa_indexer_select -> MLA; staged: the five calls; "
+                         "auto: fused for decode-sized batches")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--cpu-queries", type=int, default=16)
     ap.add_argument("--e2e-seconds", type=float, default=0.5)

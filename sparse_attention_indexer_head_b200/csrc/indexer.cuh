@@ -6,25 +6,26 @@
 // to fourth arrows: [Q, P] scores with candidate validity, the top-k select,
 // the expansion to a [Q, select_k * kpool] token-id row; trap 6).
 //
-// One thread-block cluster of C CTAs per query (C <= 8). CTA r of the cluster
+// One thread-block cluster of 8 CTAs per query. CTA r of the cluster
 //   1. sums its K-slice of the query's head gate (hidden[q] . w) before the
 //      wait on the preceding kernel (both are step inputs the path never
-//      writes); the C partials meet through distributed shared memory and are
-//      added in rank order, so every CTA holds the same gate_w[q];
+//      writes) and pushes the partial into every CTA's shared memory; each CTA
+//      adds the 8 partials in rank order, so all hold the same gate_w[q];
 //   2. scores its share of the pools, 128-pool tiles of TMA-loaded pooled keys
 //      on the tensor cores (D[128 pools x 16 heads] = keys . q_idx^T), one
-//      thread per pool summing g_h * relu(dot_h) in head order, and writes
-//      scores and cand;
-//   3. takes part in an exact 8-bit MSB radix select of the n_q-th largest
-//      candidate key over the whole cluster: each pass's 256-bin histograms
-//      are added across the cluster through distributed shared memory; after
-//      two passes, when at most 32 keys of the cluster share the answer's top
-//      16 bits, one warp ranks them;
-//   4. writes its selected pools in ascending id order at positions offset by
-//      the lower-ranked CTAs' counts, expands them to token ids and writes its
-//      stripe of the -1 tail.
-// The selection is the one dsa_topk_expand makes (ties to the lowest pool id,
-// -0 equal to +0, NaN as -inf), so results are deterministic.
+//      thread per pool summing g_h * relu(dot_h) in head order; it writes
+//      scores and cand and pushes each pool's radix key into the shared
+//      memory of the cluster's first CTA (the leader);
+//   3. the leader selects: an exact 8-bit MSB radix select of the n_q-th
+//      largest candidate key over the query's pools, with, after two passes,
+//      a one-warp rank of the at most 32 keys that share the answer's top 16
+//      bits; the winners are placed in ascending pool id and expanded to
+//      token ids, and the -1 tail is written.
+// Pushes are distributed-shared-memory stores followed by a release arrive on
+// the receiver's mbarrier, so the only cluster-wide rendezvous is the one that
+// guarantees every CTA has started (its arrive is issued before the gate's
+// loads). The selection is the one dsa_topk_expand makes (ties to the lowest
+// pool id, -0 equal to +0, NaN as -inf), so results are deterministic.
 #pragma once
 
 #include "common.cuh"
@@ -38,32 +39,35 @@ constexpr int kIxThreads = 256;
 constexpr int kIxWarps = kIxThreads / 32;
 constexpr int kIxTile = 128;                                // pools per MMA tile (M)
 constexpr int kIxHeads = DSA_MAX_INDEX_HEADS;               // 16 (N)
-constexpr int kIxMaxCluster = 8;
-constexpr int kIxMaxTilesPerCta = 32;                       // 4096 pools a CTA: max_pools <= 32768
+constexpr int kIxCluster = 8;                               // CTAs per query
+constexpr int kIxMaxPools = 32768;                          // keys the leader holds
 constexpr uint32_t kIxKeyAtom = kIxTile * 128;              // 16 KB: one 64-channel column
 constexpr uint32_t kIxKeyTile = 2 * kIxKeyAtom;             // 32 KB
 constexpr uint32_t kIxQAtom = kIxHeads * 128;               // 2 KB
 constexpr uint32_t kIxOffQ = 2 * kIxKeyTile;                // after the two-stage key ring
-constexpr uint32_t kIxOffKeys = kIxOffQ + 2 * kIxQAtom;     // radix keys of the CTA's pools
-constexpr int kIxSmem = (int)kIxOffKeys + kIxMaxTilesPerCta * kIxTile * 4 + 1024;
+constexpr uint32_t kIxOffKeys = kIxOffQ + 2 * kIxQAtom;     // the query's radix keys (leader)
+
+// Dynamic shared memory: the key ring, the query rows, P radix keys and the
+// select_k selected ids (used by the leader, sized alike on every CTA).
+inline int indexer_smem_bytes(int P, int SK) { return (int)kIxOffKeys + 4 * P + 4 * SK + 1024; }
 
 struct IxCtl {
     uint64_t q_bar, load_full[2], mma_done[2], d_empty[2];
+    uint64_t gate_bar;                  // the cluster's gate partials have arrived
+    uint64_t keys_bar;                  // the cluster's radix keys have arrived (leader)
     uint32_t tmem_base;
     int hist[2][256];
     float red[64][kIxHeads];            // gate partials per row-part
-    float gpart[kIxHeads];              // this CTA's gate partial (read by the cluster)
+    float gate_in[kIxCluster][kIxHeads];// the cluster's gate partials, by rank
     float gate[kIxHeads];               // the query's gate weights
+    int ncand_in[kIxCluster];           // the cluster's candidate counts, by rank (leader)
     int2 warp2[kIxWarps];
     int pick[3];                        // (digit, count above, count in it) of the current pass
-    int ncand;                          // this CTA's candidates (read by the cluster)
-    int nsmall;                         // this CTA's keys in the small bin (read by the cluster)
+    int ncand;                          // this CTA's candidates
+    int nsmall;
     uint32_t small[32];
     uint32_t tau;
     int req;
-    int cnt[2];                         // this CTA's keys above / equal to tau (read by the cluster)
-    int base[2];                        // the lower-ranked CTAs' keys above / equal to tau
-    int tot[256];                       // the current pass's histogram summed over the cluster
     volatile int abort;
 };
 
@@ -89,16 +93,43 @@ DSA_DEVINL bool ix_wait(IxCtl *c, uint64_t *bar, uint32_t parity) {
     return true;
 }
 
-DSA_DEVINL int ld_cluster_s32(uint32_t addr) {
-    int v;
-    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
+// Bounded wait with cluster-scope acquire: writes that other CTAs of the cluster
+// made before their release arrive on this (local) barrier are visible after it.
+DSA_DEVINL bool mbar_wait_cluster(uint64_t *bar, uint32_t phase) {
+    auto try_once = [&]() {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(phase)
+            : "memory");
+        return ok != 0;
+    };
+    if (try_once()) return true;
+    const long long t0 = clock64();
+    for (;;) {
+        if (try_once()) return true;
+        if (clock64() - t0 > kWaitLimitCycles) break;
+    }
+    raise_device_error(kErrWaitTimeout);
+    return false;
 }
-DSA_DEVINL uint32_t ld_cluster_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
+
+// Release arrive on the mbarrier at shared::cluster address `remote` (another
+// CTA's, or this one's through its cluster address).
+DSA_DEVINL void mbar_arrive_remote(uint32_t remote) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote)
+                 : "memory");
 }
+DSA_DEVINL void st_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+DSA_DEVINL void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+DSA_DEVINL void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
 // Exclusive prefix sums of (a, b) over the CTA's kIxThreads threads; *ta, *tb get the sums.
 DSA_DEVINL int2 ix_excl_scan2(int a, int b, int2 *s_warp2, int *ta, int *tb) {
@@ -139,7 +170,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     const uint32_t raw = smem_u32(ix_smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = ix_smem_raw + (base - raw);
-    uint32_t *skeys = reinterpret_cast<uint32_t *>(gbase + kIxOffKeys);
+    uint32_t *akeys = reinterpret_cast<uint32_t *>(gbase + kIxOffKeys);                 // [P]
+    int32_t *slist = reinterpret_cast<int32_t *>(gbase + kIxOffKeys + 4 * (size_t)P);   // [SK]
     const uint32_t sQ = base + kIxOffQ;
 
     const int C = gridDim.x, r = blockIdx.x, q = blockIdx.y;
@@ -158,6 +190,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
             mbar_init(&ctl->mma_done[i], 1);
             mbar_init(&ctl->d_empty[i], kIxTile);
         }
+        mbar_init(&ctl->gate_bar, C);
+        mbar_init(&ctl->keys_bar, C);
         ctl->abort = 0;
         ctl->ncand = 0;
         ctl->nsmall = 0;
@@ -168,6 +202,12 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         tma_load_2d(sQ + kIxQAtom, &q_map, 64, q * H, &ctl->q_bar);
     }
     for (int i = tid; i < 2 * 256; i += kIxThreads) (&ctl->hist[0][0])[i] = 0;
+    // Every CTA of the cluster has started and initialised its barriers once the
+    // cluster wait below returns; the arrive goes out now, so the rendezvous
+    // overlaps the gate's loads.
+    tc::fence_before_sync();
+    __syncthreads();
+    cluster_arrive_relaxed();
 
     // ---- 1. this CTA's K-slice of the head gate (step inputs: before the wait).
     // Thread (kp, hq) takes rows k = kb + kp, kb + kp + 64, ... in order (all of a
@@ -212,21 +252,32 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     const int b = q_req[q];                       // a step input, like the query rows
     const bool req_ok = b >= 0 && b < B;
     const int qp = q_pos[q];
-    tc::fence_before_sync();
     __syncthreads();
-    tc::fence_after_sync();
     if (tid < kIxHeads) {
-        float s = 0.f;
-#pragma unroll
-        for (int kp = 0; kp < 64; ++kp) s += ctl->red[kp][tid];
-        ctl->gpart[tid] = s;
+        float gpart = 0.f;
+        for (int kp = 0; kp < 64; ++kp) gpart += ctl->red[kp][tid];
+        ctl->gate[tid] = gpart;                   // this CTA's partial, until the sum below
     }
     const uint32_t tmem = ctl->tmem_base;
+    tc::fence_after_sync();
+    __syncthreads();
+    cluster_wait();
+    // push: thread (c, h) of warps 0-3 writes this CTA's partial of head h into
+    // slot r of CTA c; one thread per receiver then arrives on its barrier
+    if (warp < 4) {
+        const int c = tid >> 4, h = tid & 15;
+        if (c < C) st_cluster_u32(cluster_map(smem_u32(&ctl->gate_in[r][h]), c), __float_as_uint(ctl->gate[h]));
+    }
+    __syncthreads();
+    if (tid < C) {
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        mbar_arrive_remote(cluster_map(smem_u32(&ctl->gate_bar), tid));
+    }
 
     pdl_wait();                                   // pooled keys and flags come from compress
     pdl_launch_dependents();
 
-    // ---- 2. tiles: a producer thread loads keys and issues the MMAs, warps 0-3 drain
+    // ---- 2. tiles: two issuing threads load keys and issue the MMAs, warps 0-3 drain
     auto load = [&](int i) {
         const int s = i & 1;
         mbar_arrive_expect_tx(&ctl->load_full[s], kIxKeyTile);
@@ -235,30 +286,29 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         tma_load_2d(dst, &key_map, 0, row, &ctl->load_full[s]);
         tma_load_2d(dst + kIxKeyAtom, &key_map, 64, row, &ctl->load_full[s]);
     };
-    if (tid == 128 && req_ok) {
-        if (ntile > 0) load(0);
-        if (ntile > 1) load(1);
-    }
-
-    // every CTA's gate partial is in place: add them in rank order
-    cluster_sync_all();
+    // tiles i = 0, 2, 4 ... go through stage 0 and the issuer in warp 4, tiles
+    // 1, 3, 5 ... through stage 1 and the issuer in warp 5 (a single thread
+    // starts about one MMA per 128 cycles; two in separate warps run in parallel)
+    const bool issuer = (tid == 128 || tid == 160) && req_ok;
+    const int my_s = (tid - 128) >> 5;
+    if (issuer && my_s < ntile) load(my_s);
+    // the cluster's gate partials, added in rank order
     if (tid < kIxHeads) {
-        const uint32_t a = smem_u32(&ctl->gpart[tid]);
-        float v[kIxMaxCluster];
-#pragma unroll
-        for (int c = 0; c < kIxMaxCluster; ++c) v[c] = c < C ? ld_cluster_f32(cluster_map(a, c)) : 0.f;
         float g = 0.f;
-#pragma unroll
-        for (int c = 0; c < kIxMaxCluster; ++c) g += v[c];      // rank order
+        if (mbar_wait_cluster(&ctl->gate_bar, 0)) {
+            for (int c = 0; c < C; ++c) g += ctl->gate_in[c][tid];
+        } else {
+            ctl->abort = 1;
+        }
         ctl->gate[tid] = tid < H ? g : 0.f;
         if (r == 0 && tid < H) gate_w[(size_t)q * H + tid] = g;
     }
     __syncthreads();
 
-    if (tid == 128 && req_ok) {
-        bool ok = ntile == 0 || ix_wait(ctl, &ctl->q_bar, 0);
+    if (issuer) {
+        bool ok = my_s >= ntile || ix_wait(ctl, &ctl->q_bar, 0);
         constexpr uint32_t idesc = tc::idesc_bf16(kIxTile, kIxHeads, false, false);
-        for (int i = 0; ok && i < ntile; ++i) {
+        for (int i = my_s; ok && i < ntile; i += 2) {
             const int s = i & 1;
             ok = ix_wait(ctl, &ctl->load_full[s], (i >> 1) & 1);
             if (ok && i >= 2) ok = ix_wait(ctl, &ctl->d_empty[s], ((i >> 1) - 1) & 1);
@@ -282,6 +332,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         if (!ok) ctl->abort = 1;
     }
 
+    const uint32_t lead_keys = cluster_map(smem_u32(akeys), 0);   // the leader's key array
     int local_cand = 0;
     if (warp < 4) {
         float g[kIxHeads];
@@ -315,225 +366,183 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
             if (p < P) {
                 scores[(size_t)q * P + p] = is_cand ? score : -INFINITY;
                 cand[(size_t)q * P + p] = is_cand ? 1 : 0;
+                const uint32_t k = score_key(score, is_cand);
+                st_cluster_u32(lead_keys + 4u * (uint32_t)p, k);
+                local_cand += k != 0u;
             }
-            const int lp = p - rg.p_lo;
-            const uint32_t k = score_key(score, is_cand);
-            if (p < P) skeys[lp] = k;
-            local_cand += k != 0u;
-            const uint32_t dgt = (p < P) ? (k >> 24) : 0x100u;
-            const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
-            if (dgt != 0x100u && lane == __ffs(peers) - 1) atomicAdd(&ctl->hist[0][dgt], __popc(peers));
         }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) local_cand += __shfl_xor_sync(0xffffffffu, local_cand, off);
     if (lane == 0 && local_cand) atomicAdd(&ctl->ncand, local_cand);
-
-    // ---- 3. radix select over the cluster
     __syncthreads();
-    cluster_sync_all();                           // histograms of pass 0 and candidate counts
-    int ncand = 0;
-    {
-        int v[kIxMaxCluster];
-#pragma unroll
-        for (int c = 0; c < kIxMaxCluster; ++c)
-            v[c] = c < C ? ld_cluster_s32(cluster_map(smem_u32(&ctl->ncand), c)) : 0;
-#pragma unroll
-        for (int c = 0; c < kIxMaxCluster; ++c) ncand += v[c];
+    if (tid == 0) {
+        // this CTA's candidate count to the leader, then its release arrive (after
+        // every key this CTA pushed: the CTA barrier above orders them before it)
+        st_cluster_u32(cluster_map(smem_u32(&ctl->ncand_in[r]), 0), (uint32_t)ctl->ncand);
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        mbar_arrive_remote(cluster_map(smem_u32(&ctl->keys_bar), 0));
     }
-    const int nq = min(SK, ncand);
-    const int nloc = rg.p_hi - rg.p_lo;
-    uint32_t prefix = 0, pmask = 0;
-    int remaining = nq;
-    if (nq > 0) {
+
+    if (r == 0) {
+        // ---- 3. the leader selects over the query's P keys
+        if (tid == 0) {
+            int n = 0;
+            if (mbar_wait_cluster(&ctl->keys_bar, 0)) {
+                for (int c = 0; c < C; ++c) n += ctl->ncand_in[c];
+            } else {
+                ctl->abort = 1;
+            }
+            ctl->req = ctl->abort ? 0 : n;
+        }
+        __syncthreads();
+        const int nq = min(SK, ctl->req);
+
+        uint32_t prefix = 0, pmask = 0;
+        int remaining = nq;
+        if (nq > 0) {
+            // pass 0's histogram: the top byte of every key
+            for (int p0 = 0; p0 < P; p0 += kIxThreads) {
+                const int p = p0 + tid;
+                const uint32_t dgt = p < P ? (akeys[p] >> 24) : 0x100u;
+                const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
+                if (dgt != 0x100u && lane == __ffs(peers) - 1) atomicAdd(&ctl->hist[0][dgt], __popc(peers));
+            }
+            __syncthreads();
 #pragma unroll 1
-        for (int pass = 0; pass < 4; ++pass) {
-            const int shift = 24 - 8 * pass, hb = pass & 1;
-            if (pass > 0) {
-                for (int i = tid; i < nloc; i += kIxThreads) {
-                    const uint32_t k = skeys[i];
-                    if ((k & pmask) == prefix) atomicAdd(&ctl->hist[hb][(k >> shift) & 0xFF], 1);
-                }
-                cluster_sync_all();
-            }
-            {
-                // thread t sums bin t over the cluster (all loads in flight at once)
-                const uint32_t a = smem_u32(&ctl->hist[hb][tid]);
-                int v[kIxMaxCluster];
-#pragma unroll
-                for (int c = 0; c < kIxMaxCluster; ++c) v[c] = c < C ? ld_cluster_s32(cluster_map(a, c)) : 0;
-                int t = 0;
-#pragma unroll
-                for (int c = 0; c < kIxMaxCluster; ++c) t += v[c];
-                ctl->tot[tid] = t;
-            }
-            __syncthreads();
-            if (tid < 32) {
-                // lane l owns bins 255-8l down to 248-8l
-                int cbin[8], sum = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    cbin[i] = ctl->tot[255 - 8 * tid - i];
-                    sum += cbin[i];
-                }
-                int above = sum;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int y = __shfl_up_sync(0xffffffffu, above, off);
-                    if (tid >= off) above += y;
-                }
-                int run = above - sum;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (run < remaining && remaining <= run + cbin[i]) {
-                        ctl->pick[0] = 255 - 8 * tid - i;
-                        ctl->pick[1] = run;
-                        ctl->pick[2] = cbin[i];
+            for (int pass = 0; pass < 4; ++pass) {
+                const int shift = 24 - 8 * pass, hb = pass & 1;
+                if (pass > 0) {
+                    for (int p = tid; p < P; p += kIxThreads) {
+                        const uint32_t k = akeys[p];
+                        if ((k & pmask) == prefix) atomicAdd(&ctl->hist[hb][(k >> shift) & 0xFF], 1);
                     }
-                    run += cbin[i];
+                    __syncthreads();
                 }
-            }
-            __syncthreads();
-            remaining -= ctl->pick[1];
-            prefix |= (uint32_t)ctl->pick[0] << shift;
-            pmask |= 0xFFu << shift;
-            const int in_bin = ctl->pick[2];
-            // the other histogram buffer was last read by the cluster before the
-            // barrier above: clear it for the next pass
-            for (int i = tid; i < 256; i += kIxThreads) ctl->hist[hb ^ 1][i] = 0;
-            __syncthreads();
-            if (pass == 1 && in_bin <= 32) {
-                // At most 32 keys of the cluster share the answer's top 16 bits:
-                // gather them and rank them on one warp instead of two more passes.
-                for (int base0 = (tid & ~31); base0 < nloc; base0 += kIxThreads) {
-                    const int i = base0 + lane;
-                    const uint32_t k = i < nloc ? skeys[i] : 0u;
-                    const bool m = i < nloc && (k & pmask) == prefix;
-                    const uint32_t bal = __ballot_sync(0xffffffffu, m);
-                    if (bal) {
-                        int off = 0;
-                        if (lane == 0) off = atomicAdd(&ctl->nsmall, __popc(bal));
-                        off = __shfl_sync(0xffffffffu, off, 0);
-                        if (m) ctl->small[off + __popc(bal & ((1u << lane) - 1u))] = k;
-                    }
-                }
-                cluster_sync_all();
                 if (tid < 32) {
-                    // lane c < C reads CTA c's list length; lane tid then loads entry tid of
-                    // the cluster's lists concatenated in rank order
-                    const int nc = tid < C ? ld_cluster_s32(cluster_map(smem_u32(&ctl->nsmall), tid)) : 0;
-                    int incl = nc;
+                    // lane l owns bins 255-8l down to 248-8l
+                    int cbin[8], sum = 0;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        cbin[i] = ctl->hist[hb][255 - 8 * tid - i];
+                        sum += cbin[i];
+                    }
+                    int above = sum;
 #pragma unroll
                     for (int off = 1; off < 32; off <<= 1) {
-                        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-                        if (tid >= off) incl += y;
+                        const int y = __shfl_up_sync(0xffffffffu, above, off);
+                        if (tid >= off) above += y;
                     }
-                    const int n = __shfl_sync(0xffffffffu, incl, 31);
-                    int owner = 0, start = 0;
+                    int run = above - sum;
 #pragma unroll
-                    for (int c = 0; c < kIxMaxCluster; ++c) {
-                        const int e = __shfl_sync(0xffffffffu, incl, c);      // end of CTA c's list
-                        const int b0 = e - __shfl_sync(0xffffffffu, nc, c);
-                        if (c < C && tid >= b0 && tid < e) { owner = c; start = b0; }
-                    }
-                    const uint32_t mine =
-                        tid < n ? ld_cluster_u32(cluster_map(smem_u32(&ctl->small[tid - start]), owner)) : 0u;
-                    int gt = 0, ge = 0;
-                    for (int j = 0; j < n; ++j) {
-                        const uint32_t kj = __shfl_sync(0xffffffffu, mine, j);
-                        gt += kj > mine;
-                        ge += kj >= mine;
-                    }
-                    if (tid < n && gt < remaining && remaining <= ge) {
-                        ctl->tau = mine;
-                        ctl->req = remaining - gt;
+                    for (int i = 0; i < 8; ++i) {
+                        if (run < remaining && remaining <= run + cbin[i]) {
+                            ctl->pick[0] = 255 - 8 * tid - i;
+                            ctl->pick[1] = run;
+                            ctl->pick[2] = cbin[i];
+                        }
+                        run += cbin[i];
                     }
                 }
                 __syncthreads();
-                prefix = ctl->tau;
-                remaining = ctl->req;
-                break;
+                remaining -= ctl->pick[1];
+                prefix |= (uint32_t)ctl->pick[0] << shift;
+                pmask |= 0xFFu << shift;
+                const int in_bin = ctl->pick[2];
+                for (int i = tid; i < 256; i += kIxThreads) ctl->hist[hb ^ 1][i] = 0;
+                __syncthreads();
+                if (pass == 1 && in_bin <= 32) {
+                    // At most 32 keys share the answer's top 16 bits: gather them and
+                    // rank them on one warp instead of two more passes.
+                    for (int base0 = (tid & ~31); base0 < P; base0 += kIxThreads) {
+                        const int p = base0 + lane;
+                        const uint32_t k = p < P ? akeys[p] : 0u;
+                        const bool m = p < P && (k & pmask) == prefix;
+                        const uint32_t bal = __ballot_sync(0xffffffffu, m);
+                        if (bal) {
+                            int off = 0;
+                            if (lane == 0) off = atomicAdd(&ctl->nsmall, __popc(bal));
+                            off = __shfl_sync(0xffffffffu, off, 0);
+                            if (m) ctl->small[off + __popc(bal & ((1u << lane) - 1u))] = k;
+                        }
+                    }
+                    __syncthreads();
+                    if (tid < 32) {
+                        const int n = ctl->nsmall;
+                        const uint32_t mine = tid < n ? ctl->small[tid] : 0u;
+                        int gt = 0, ge = 0;
+                        for (int j = 0; j < n; ++j) {
+                            const uint32_t kj = ctl->small[j];
+                            gt += kj > mine;
+                            ge += kj >= mine;
+                        }
+                        if (tid < n && gt < remaining && remaining <= ge) {
+                            ctl->tau = mine;
+                            ctl->pick[0] = remaining - gt;
+                        }
+                    }
+                    __syncthreads();
+                    prefix = ctl->tau;
+                    remaining = ctl->pick[0];
+                    break;
+                }
             }
         }
-    }
-    const uint32_t tau = prefix;     // the nq-th largest key of the query (when nq > 0)
-    const int req_eq = remaining;    // keys equal to tau to take, lowest ids first
+        const uint32_t tau = prefix;     // the nq-th largest key (when nq > 0)
+        const int req_eq = remaining;    // keys equal to tau to take, lowest ids first
 
-    // ---- 4. placement: this CTA's winners after those of the lower ranks
-    const int chunk = (nloc + kIxThreads - 1) / kIxThreads;
-    const int i_lo = min(nloc, tid * chunk), i_hi = min(nloc, i_lo + chunk);
-    int gt = 0, eq = 0;
-    if (nq > 0)
-        for (int i = i_lo; i < i_hi; ++i) {
-            const uint32_t k = skeys[i];
-            gt += k > tau;
-            eq += k == tau;
+        // ---- 4. winners in ascending pool id: every key above tau, then the
+        // req_eq lowest-id keys equal to it
+        const int chunk = (P + kIxThreads - 1) / kIxThreads;
+        const int p_lo = min(P, tid * chunk), p_hi = min(P, p_lo + chunk);
+        int gt = 0, eq = 0;
+        if (nq > 0)
+            for (int p = p_lo; p < p_hi; ++p) {
+                const uint32_t k = akeys[p];
+                gt += k > tau;
+                eq += k == tau;
+            }
+        int tot_gt, tot_eq;
+        const int2 before = ix_excl_scan2(gt, eq, ctl->warp2, &tot_gt, &tot_eq);
+        if (nq > 0) {
+            int pos = before.x + min(before.y, req_eq);
+            int eqr = before.y;
+            for (int p = p_lo; p < p_hi; ++p) {
+                const uint32_t k = akeys[p];
+                if (k > tau) {
+                    slist[pos++] = p;
+                } else if (k == tau) {
+                    if (eqr < req_eq) slist[pos++] = p;
+                    ++eqr;
+                }
+            }
         }
-    int tot_gt, tot_eq;
-    const int2 before = ix_excl_scan2(gt, eq, ctl->warp2, &tot_gt, &tot_eq);
-    if (tid == 0) {
-        ctl->cnt[0] = tot_gt;
-        ctl->cnt[1] = tot_eq;
-    }
-    cluster_sync_all();
-    if (tid < 32) {
-        // counts of the lower-ranked CTAs, summed on one warp
-        int g = 0, e = 0;
-        if (tid < r) {
-            g = ld_cluster_s32(cluster_map(smem_u32(&ctl->cnt[0]), tid));
-            e = ld_cluster_s32(cluster_map(smem_u32(&ctl->cnt[1]), tid));
-        }
+        __syncthreads();
+        const size_t wrow = (size_t)SK * KP;
+        for (int j = tid; j < SK; j += kIxThreads) top_pools[(size_t)q * SK + j] = j < nq ? slist[j] : -1;
+        // expansion: four pool_idx gathers in flight per thread before the stores
+        for (int e0 = 0; e0 < SK * KP; e0 += 4 * kIxThreads) {
+            int32_t v[4];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            g += __shfl_xor_sync(0xffffffffu, g, off);
-            e += __shfl_xor_sync(0xffffffffu, e, off);
-        }
-        if (tid == 0) {
-            ctl->base[0] = g;
-            ctl->base[1] = e;
-        }
-    }
-    __syncthreads();
-    const int base_gt = ctl->base[0], base_eq = ctl->base[1];
-    const size_t wrow = (size_t)SK * KP;
-    if (nq > 0) {
-        const int eq0 = base_eq + before.y;
-        int pos = base_gt + before.x + min(eq0, req_eq);
-        int eqr = eq0;
-        for (int i = i_lo; i < i_hi; ++i) {
-            const uint32_t k = skeys[i];
-            bool take = false;
-            if (k > tau) {
-                take = true;
-            } else if (k == tau) {
-                take = eqr < req_eq;
-                ++eqr;
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + tid + u * kIxThreads;
+                const int j = e / KP, s = e - j * KP;
+                v[u] = -1;
+                if (e < SK * KP && j < nq) v[u] = __ldg(pool_idx + ((size_t)b * P + slist[j]) * KP + s);
             }
-            if (take) {
-                const int p = rg.p_lo + i;
-                top_pools[(size_t)q * SK + pos] = p;
-                const int32_t *src = pool_idx + ((size_t)b * P + p) * KP;
-                int32_t *dst = token_ids + (size_t)q * wrow + (size_t)pos * KP;
-                for (int s = 0; s < KP; ++s) dst[s] = __ldg(src + s);
-                ++pos;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + tid + u * kIxThreads;
+                if (e < SK * KP) token_ids[(size_t)q * wrow + e] = v[u];
             }
         }
-    }
-    // the -1 tail: slots nq .. SK-1, striped over the cluster
-    for (int j = nq + r * kIxThreads + tid; j < SK; j += C * kIxThreads) {
-        top_pools[(size_t)q * SK + j] = -1;
-        for (int s = 0; s < KP; ++s) token_ids[(size_t)q * wrow + (size_t)j * KP + s] = -1;
     }
 
     if (tid == 32) (void)mbar_wait(&ctl->q_bar, 0);   // the query rows' copy has landed
     tc::fence_before_sync();
-    cluster_sync_all();                           // no CTA leaves while a peer still reads it
+    __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, 32);
 }
-
-// Cluster size: 8 CTAs whatever P (the gate's K-split uses every CTA; one with no
-// pool tile only adds its gate slice and takes part in the select).
-inline int indexer_cluster(int) { return kIxMaxCluster; }
 
 inline int indexer_launch(const float *hidden, const float *w, int K, const void *q_idx,
                           const int32_t *q_req, const int32_t *q_pos, int Q, int H, int D,
@@ -545,7 +554,7 @@ inline int indexer_launch(const float *hidden, const float *w, int K, const void
         return DSA_ERR_INVALID_ARG;
     if (D != kD || H > kIxHeads || kpool > DSA_MAX_KPOOL || select_k > DSA_MAX_SELECT)
         return DSA_ERR_UNSUPPORTED;
-    if (max_pools > kIxMaxCluster * kIxMaxTilesPerCta * kIxTile) return DSA_ERR_UNSUPPORTED;
+    if (max_pools > kIxMaxPools) return DSA_ERR_UNSUPPORTED;
     if (Q == 0) return DSA_OK;
     if (Q > 65535 || (long long)B * max_pools >= (1ll << 31) || (long long)Q * H >= (1ll << 31))
         return DSA_ERR_UNSUPPORTED;
@@ -564,12 +573,12 @@ inline int indexer_launch(const float *hidden, const float *w, int K, const void
     if (!make_map_bf16_2d(&key_map, kbase, krows, kD, kD * 2, 64, kIxTile) ||
         !make_map_bf16_2d(&q_map, q_idx, (uint64_t)Q * H, kD, kD * 2, 64, kIxHeads))
         return DSA_ERR_CUDA;
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(indexer_kernel), kIxSmem)) return DSA_ERR_CUDA;
-    const int C = indexer_cluster(max_pools);
-    if (launch_pdl_cluster(indexer_kernel, dim3(C, Q), dim3(kIxThreads), kIxSmem, stream, C, key_map,
-                           q_map, hidden, w, K, H, q_req, q_pos, pool_valid, first_valid, pool_idx,
-                           B, kpool, max_pools, select_k, gate_w, scores, cand, top_pools,
-                           token_ids) != cudaSuccess)
+    const int smem = indexer_smem_bytes(max_pools, select_k);
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(indexer_kernel), smem)) return DSA_ERR_CUDA;
+    if (launch_pdl_cluster(indexer_kernel, dim3(kIxCluster, Q), dim3(kIxThreads), smem, stream,
+                           kIxCluster, key_map, q_map, hidden, w, K, H, q_req, q_pos, pool_valid,
+                           first_valid, pool_idx, B, kpool, max_pools, select_k, gate_w, scores,
+                           cand, top_pools, token_ids) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
 }

@@ -7,7 +7,11 @@
 // TMA-fed stream with all arithmetic in registers:
 //   * a persistent CTA owns a contiguous range of tiles; a tile is TP
 //     consecutive pools of one request, i.e. up to 128 contiguous token rows
-//     of k and of gate; a producer warp moves each tile with 1-D bulk copies
+//     of k and of gate. For up to 2048 requests (1152 above kpool 4) the CTAs
+//     first find every request's first valid token and split the tiles that
+//     hold pools evenly among themselves (requests of very different lengths
+//     then cost no imbalance, and pool slots past a request's span are written
+//     apart, without a trip through the pipeline); a producer warp moves each tile with 1-D bulk copies
 //     (cp.async.bulk) into a shared-memory ring -- the k rows, the gate rows
 //     and the 16-byte-aligned span of validity bytes covering them -- all
 //     completing on one mbarrier, so no consumer waits on a global load;
@@ -38,6 +42,9 @@ template <int KP> struct CmpCfg {
     static constexpr int kStageBytes = 2 * kTileTokens * 128 * 2;
 };
 constexpr int kD = DSA_INDEX_DIM;   // 128 channels
+// Requests the balanced partition handles (3 int32 a request in shared memory);
+// each thread of the CTA owns kCmpReqPerThread consecutive requests.
+constexpr int kCmpReqPerThread = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // First index in [0, T) of request rows [rs, rs+T) whose valid byte is nonzero;
@@ -252,7 +259,7 @@ template <int KP>
 __global__ void __launch_bounds__(CmpCfg<KP>::kThreads, 1)
 kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ gate,
                       const uint8_t *__restrict__ valid, const int32_t *__restrict__ req_start,
-                      int B, int max_pools, int tiles_per_req, int n_tiles,
+                      int B, int max_pools, int tiles_per_req, int n_tiles, int balanced,
                       const float *__restrict__ ape, const __nv_bfloat16 *__restrict__ ln_w,
                       const __nv_bfloat16 *__restrict__ ln_b, float eps,
                       __nv_bfloat16 *__restrict__ pool_keys, int32_t *__restrict__ pool_idx,
@@ -273,8 +280,14 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x;
-    const int t_begin = (int)((long long)blockIdx.x * n_tiles / G);
-    const int t_end = (int)((long long)(blockIdx.x + 1) * n_tiles / G);
+    // Unbalanced (many requests): contiguous ranges of every request's tile grid.
+    int t_begin = (int)((long long)blockIdx.x * n_tiles / G);
+    int t_end = (int)((long long)(blockIdx.x + 1) * n_tiles / G);
+    // Balanced: per request its first valid token, and prefix sums over the requests
+    // of the tiles holding pools in its span and of the pool slots past the span.
+    int32_t *s_f = reinterpret_cast<int32_t *>(cmp_smem + kCmpStages * kCmpStageBytes);
+    int32_t *s_pre = s_f + B;
+    int32_t *s_epre = s_pre + (B + 1);
 
     if (tid == 0) {
         for (int s = 0; s < kCmpStages; ++s) {
@@ -292,34 +305,158 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     // its first request's rows before the wait on the preceding kernel.
     long long total = 0;
     int first_rs = 0, first_re = 0;
-    if (warp == kCmpConsumers / 32 && t_begin < t_end) {
+    if (!balanced && warp == kCmpConsumers / 32 && t_begin < t_end) {
         const int b0 = t_begin / tiles_per_req;
         total = req_start[B];                       // rows of the validity array
         first_rs = req_start[b0];
         first_re = req_start[b0 + 1];
     }
+    // balanced: thread t owns requests [kCmpReqPerThread t, ... + kCmpReqPerThread)
+    int rq_rs[kCmpReqPerThread + 1];
+    const int rb0 = tid * kCmpReqPerThread;
+    if (balanced) {
+#pragma unroll
+        for (int u = 0; u <= kCmpReqPerThread; ++u) rq_rs[u] = rb0 + u <= B ? req_start[rb0 + u] : 0;
+        total = req_start[B];
+    }
     pdl_wait();
     pdl_launch_dependents();
+
+    int g_lo = 0, g_hi = 0, e_lo = 0, e_hi = 0;
+    if (balanced) {
+        // ---- each request's first valid token: the 16 validity bytes from its
+        // first row settle almost every request; a warp scans the rest
+#pragma unroll
+        for (int u = 0; u < kCmpReqPerThread; ++u) {
+            const int b = rb0 + u;
+            if (b >= B) break;
+            const long long rs = rq_rs[u], re = rq_rs[u + 1];
+            const int T = (int)max(0ll, re - rs);
+            int f = -1;
+            if (T == 0) {
+                f = 0;
+            } else {
+                const long long c0 = rs & ~15ll;
+                int hit = -1;
+                if (c0 + 16 <= total) {
+                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(valid + c0));
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int q = 3; q >= 0; --q)
+#pragma unroll
+                        for (int bb = 3; bb >= 0; --bb) {
+                            const long long pos = c0 + 4 * q + bb;
+                            if (pos >= rs && pos < re && ((w4[q] >> (8 * bb)) & 0xFF)) hit = (int)(pos - rs);
+                        }
+                    if (hit >= 0) f = hit;
+                    else if (c0 + 16 >= re) f = T;
+                }
+            }
+            s_f[b] = f;
+        }
+        __syncthreads();
+        for (int b = warp; b < B; b += kCmpThreads / 32) {
+            if (s_f[b] >= 0) continue;                     // warp-uniform
+            const int rs = req_start[b];
+            const int T = max(0, req_start[b + 1] - rs);
+            const int f = first_valid_scan(valid, rs, T);
+            if (lane == 0) s_f[b] = f;
+        }
+        __syncthreads();
+        // ---- per request: tiles of pools in its span, pool slots past it; prefix sums
+        int tl[kCmpReqPerThread], em[kCmpReqPerThread], st = 0, se = 0;
+#pragma unroll
+        for (int u = 0; u < kCmpReqPerThread; ++u) {
+            const int b = rb0 + u;
+            tl[u] = em[u] = 0;
+            if (b < B) {
+                const int T = (int)max(0ll, (long long)rq_rs[u + 1] - rq_rs[u]);
+                const int n_span = max(0, min(max_pools, (T - s_f[b]) / KP));
+                tl[u] = (n_span + TP - 1) / TP;
+                em[u] = max_pools - n_span;
+            }
+            st += tl[u];
+            se += em[u];
+        }
+        __shared__ int2 s_w2[kCmpThreads / 32];
+        int x = st, y = se;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, x, off), c = __shfl_up_sync(0xffffffffu, y, off);
+            if (lane >= off) { x += a; y += c; }
+        }
+        if (lane == 31) s_w2[warp] = make_int2(x, y);
+        __syncthreads();
+        int bx = 0, by = 0, R = 0, E = 0;
+        for (int w2 = 0; w2 < kCmpThreads / 32; ++w2) {
+            const int2 v = s_w2[w2];
+            if (w2 < warp) { bx += v.x; by += v.y; }
+            R += v.x;
+            E += v.y;
+        }
+        int px = bx + x - st, py = by + y - se;
+#pragma unroll
+        for (int u = 0; u < kCmpReqPerThread; ++u) {
+            const int b = rb0 + u;
+            if (b < B) {
+                s_pre[b] = px;
+                s_epre[b] = py;
+                if (b == B - 1) { s_pre[B] = px + tl[u]; s_epre[B] = py + em[u]; }
+            }
+            px += tl[u];
+            py += em[u];
+        }
+        __syncthreads();
+        g_lo = (int)((long long)blockIdx.x * R / G);
+        g_hi = (int)((long long)(blockIdx.x + 1) * R / G);
+        e_lo = (int)((long long)blockIdx.x * E / G);
+        e_hi = (int)((long long)(blockIdx.x + 1) * E / G);
+        t_begin = 0;
+        t_end = g_hi - g_lo;                       // this CTA's tiles, in order
+        // first_valid: this CTA's share of the requests
+        const int b_lo = (int)((long long)blockIdx.x * B / G), b_hi = (int)((long long)(blockIdx.x + 1) * B / G);
+        for (int b = b_lo + tid; b < b_hi; b += kCmpThreads) first_valid[b] = s_f[b];
+    }
 
     if (warp == kCmpConsumers / 32) {
         // ---------------------------------------------------------------- producer warp
         int cur_b = -1, cur_f = 0, cur_rs = 0, cur_T = 0;
+        // balanced: the first request holding real tile g_lo (s_pre is non-decreasing)
+        int bb = 0;
+        if (balanced) {
+            int lo = 0, hi = B - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_pre[mid] <= g_lo) lo = mid; else hi = mid - 1;
+            }
+            bb = lo;
+        }
         for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
             const int s = i % kCmpStages;
             bool ok = true;
             if (i >= kCmpStages) ok = mbar_wait(&empty[s], ((i / kCmpStages) - 1) & 1);
             if (!__all_sync(0xffffffffu, ok)) break;
-            const int b = t / tiles_per_req, j = t - b * tiles_per_req;
+            int b, j;
+            if (balanced) {
+                const int g = g_lo + t;
+                while (s_pre[bb + 1] <= g) ++bb;
+                b = bb;
+                j = g - s_pre[bb];
+            } else {
+                b = t / tiles_per_req;
+                j = t - b * tiles_per_req;
+            }
             if (b != cur_b) {
-                const bool first = i == 0;
+                const bool first = i == 0 && !balanced;
                 cur_rs = first ? first_rs : req_start[b];
                 cur_T = max(0, (first ? first_re : req_start[b + 1]) - cur_rs);
-                cur_f = first_valid_scan(valid, cur_rs, cur_T);
+                cur_f = balanced ? s_f[b] : first_valid_scan(valid, cur_rs, cur_T);
                 cur_b = b;
             }
             const int p0 = j * TP;
-            const int p1 = min(p0 + TP, max_pools);
             const int n_span = min(max_pools, (cur_T - cur_f) / KP);
+            // balanced tiles end at the span (the slots past it are written apart)
+            const int p1 = balanced ? min(p0 + TP, n_span) : min(p0 + TP, max_pools);
             const int n_in = max(0, min(p1, n_span) - p0);
             // The tile's rows of k and gate, and the 16-byte-aligned span of
             // validity bytes covering them, arrive together by bulk copy; the
@@ -348,6 +485,30 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
                 }
             }
             __syncwarp();
+        }
+        if (balanced) {
+            // pool slots past each request's span: index -1, invalid (the key rows
+            // there are not written); this CTA's share of them, request by request
+            int b = 0;
+            {
+                int lo = 0, hi = B - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (s_epre[mid] <= e_lo) lo = mid; else hi = mid - 1;
+                }
+                b = lo;
+            }
+            for (int e = e_lo; e < e_hi && b < B;) {
+                while (b < B && s_epre[b + 1] <= e) ++b;
+                if (b >= B) break;
+                const int first_p = max_pools - (s_epre[b + 1] - s_epre[b]);    // = n_span
+                const int p_a = first_p + (e - s_epre[b]);
+                const int cnt = min(e_hi, s_epre[b + 1]) - e;
+                const size_t pb = (size_t)b * max_pools;
+                for (int x = lane; x < cnt * KP; x += 32) pool_idx[(pb + p_a) * KP + x] = -1;
+                for (int x = lane; x < cnt; x += 32) pool_valid[pb + p_a + x] = 0;
+                e += cnt;
+            }
         }
         return;
     }
@@ -385,7 +546,7 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
         const __nv_bfloat16 *sg = sk + kCmpTileTokens * kD;
         const size_t pool_base = (size_t)m.b * max_pools;
-        if (m.p0 == 0 && tid == 0) first_valid[m.b] = m.f;
+        if (!balanced && m.p0 == 0 && tid == 0) first_valid[m.b] = m.f;
 
         // Pools of this tile past the request's span: no key, index -1, invalid.
         for (int x = m.n_in * KP + tid; x < (m.p1 - m.p0) * KP; x += kCmpConsumers)
@@ -424,16 +585,20 @@ inline int kpool_compress_launch_kp(const __nv_bfloat16 *k, const __nv_bfloat16 
                                     int32_t *idx, uint8_t *pv, int32_t *fv, cudaStream_t stream) {
     using C = CmpCfg<KP>;
     constexpr int TP = C::kTP;
-    const int smem = C::kStages * C::kStageBytes;
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(kpool_compress_kernel<KP>), smem))
+    // Up to kCmpReqPerThread requests a thread, the CTA splits the tiles that hold
+    // pools evenly (balanced); beyond, contiguous ranges of every request's tile grid.
+    const int balanced = B <= kCmpReqPerThread * C::kThreads ? 1 : 0;
+    const int smem = C::kStages * C::kStageBytes + (balanced ? 4 * (3 * B + 2) : 0);
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(kpool_compress_kernel<KP>),
+                          C::kStages * C::kStageBytes + 4 * (3 * kCmpReqPerThread * C::kThreads + 2)))
         return DSA_ERR_CUDA;
     const int tiles_per_req = max(1, ceil_div(max_pools, TP));
     const long long n_tiles = (long long)tiles_per_req * B;
     if (n_tiles > (1ll << 30)) return DSA_ERR_UNSUPPORTED;
     const int grid = (int)std::min<long long>(n_tiles, sm_count());
     if (launch_pdl(kpool_compress_kernel<KP>, dim3(grid), dim3(C::kThreads), smem, stream, k, gate,
-                   valid, req_start, B, max_pools, tiles_per_req, (int)n_tiles, ape, ln_w, ln_b, eps,
-                   keys, idx, pv, fv) != cudaSuccess)
+                   valid, req_start, B, max_pools, tiles_per_req, (int)n_tiles, balanced, ape, ln_w,
+                   ln_b, eps, keys, idx, pv, fv) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
 }

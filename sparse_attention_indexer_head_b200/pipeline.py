@@ -22,6 +22,8 @@ from . import binding as B
 from .workloads import INDEX_DIM, INDEX_HEADS, KV_LORA, Workload
 
 QUERY_INPUTS = ("hidden", "q_idx", "q_mla", "q_req", "q_pos")
+INDEXER_MAX_POOLS = 32768          # dsa_indexer_select's pool limit
+AUTO_FUSED_MAX_QUERIES = 256       # "auto": the fused indexer up to this many queries
 
 
 def _bf16(a: np.ndarray) -> torch.Tensor:
@@ -72,8 +74,14 @@ class DecodeStep:
                  always_select_tail: bool = False, fused_indexer: bool = False):
         self.device = torch.device(device)
         # fused_indexer: gate, scores, top-k and expansion in one dsa_indexer_select
-        # call (not with always_select_tail, whose tail slots only dsa_topk_expand_tail writes)
-        self.fused = bool(fused_indexer) and not always_select_tail
+        # call (not with always_select_tail, whose tail slots only dsa_topk_expand_tail
+        # writes, nor above its pool limit). "auto" takes it for decode-sized batches:
+        # its cluster of 8 CTAs a query recomputes the gate and re-reads the request's
+        # pooled keys per query, which the separate calls amortise over many queries.
+        if fused_indexer == "auto":
+            fused_indexer = wl.Q <= AUTO_FUSED_MAX_QUERIES
+        self.fused = (bool(fused_indexer) and not always_select_tail
+                      and wl.max_pools <= INDEXER_MAX_POOLS)
         self.g = Geometry(wl.B, wl.Q, wl.kpool, wl.max_pools, wl.select_k, wl.hm, wl.eps,
                           wl.sm_scale, wl.kpool - 1 if always_select_tail else 0)
         src = host_tensors(wl) if inputs is None else inputs

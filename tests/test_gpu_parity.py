@@ -10,8 +10,9 @@ import pytest
 import torch
 
 import oracle as O
-from gpu_helpers import (assert_gate_close, assert_mla_close, dev_bits, device_status_clean,
-                         end_to_end, host_bits, mla_value_bound, run_step, stagewise, workload)
+from gpu_helpers import (assert_gate_close, assert_keys_close, assert_mla_close, dev_bits,
+                         device_status_clean, end_to_end, host_bits, mla_value_bound, run_step,
+                         stagewise, workload)
 from sparse_attention_indexer_head_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -97,6 +98,26 @@ def test_every_kpool_with_ragged_requests(B, kpool):
     stagewise(wl, g)
     assert g["first_valid"][4] == 129 and g["first_valid"][5] == 0
     assert (g["top_pools"][4] == -1).all() and (g["token_ids"][5] == -1).all()
+    device_status_clean(B)
+
+
+@pytest.mark.parametrize("kpool,n_req", [(4, 2100), (8, 1200), (3, 300)])
+def test_compress_partitions(B, kpool, n_req):
+    """Request counts past the balanced partition's limit (2048 requests at kpool <= 4,
+    1152 above) take the per-request tile grid; below it, the tiles holding pools are
+    split evenly. Lengths 0-60 with random padding, so many requests end in a partial
+    pool, have no valid token or are empty."""
+    rng = np.random.default_rng(n_req)
+    lengths = rng.integers(0, 61, n_req).tolist()
+    pads = [int(rng.integers(0, t + 1)) if t else 0 for t in lengths]
+    wl = _mini(kpool, lengths, pads, select_k=4, max_pools=16)
+    step, g = run_step(wl)
+    keys, idx, pv, fv = O.kpool_compress(wl.k, wl.gate, wl.valid, wl.req_start, wl.kpool,
+                                         wl.max_pools, wl.ape, wl.ln_w, wl.ln_b, wl.eps)
+    np.testing.assert_array_equal(g["first_valid"], fv)
+    np.testing.assert_array_equal(g["pool_valid"], pv)
+    np.testing.assert_array_equal(g["pool_idx"], idx)
+    assert_keys_close(g["pool_keys"], keys, pv, wl, fv)
     device_status_clean(B)
 
 
