@@ -67,7 +67,13 @@ def algorithmic_bytes(wl) -> dict:
     scores = int((n_span * 2 * D).sum() + Q * (2 * H * D + 4 * H + P * (1 + 4 + 1) + 8))
     n_sel = np.minimum(wl.select_k, n_span[wl.q_req])          # pools selected (decode: all cand)
     topk = int(Q * P * 5 + (n_sel * kp * 4).sum() + Q * (4 * wl.select_k + 4 * wl.out_width + 4))
-    mla = int((n_sel * kp * L * 2).sum() + Q * (wl.hm * L * 2 * 2 + 4 * wl.out_width + 4 * wl.hm + 4))
+    # MLA: each request's latent rows once, the rows its queries select together; at
+    # most every row of its span (prefill's 2048 queries re-read their shared rows
+    # from L2), and exactly the selected rows at decode (one query a request)
+    rows_b = np.zeros(wl.B, dtype=np.int64)
+    np.add.at(rows_b, wl.q_req, n_sel * kp)
+    rows_b = np.minimum(rows_b, n_span * kp)
+    mla = int(rows_b.sum() * L * 2 + Q * (wl.hm * L * 2 * 2 + 4 * wl.out_width + 4 * wl.hm + 4))
     out = dict(head_gate=gate, kpool_compress=compress, index_scores=scores,
                topk_expand=topk, sparse_mla=mla)
     # the fused indexer moves the three stages' bytes but the ones they pass each other

@@ -19,8 +19,9 @@
 //   3. the leader selects: an exact 8-bit MSB radix select of the n_q-th
 //      largest candidate key over the query's pools, with, after two passes,
 //      a one-warp rank of the at most 32 keys that share the answer's top 16
-//      bits; the winners are placed in ascending pool id and expanded to
-//      token ids, and the -1 tail is written.
+//      bits; the winners are placed in ascending pool id (warps over
+//      contiguous id ranges, ballot ranks) and expanded to token ids, and the
+//      -1 tail is written.
 // Pushes are distributed-shared-memory stores followed by a release arrive on
 // the receiver's mbarrier, so the only cluster-wide rendezvous is the one that
 // guarantees every CTA has started (its arrive is issued before the gate's
@@ -47,9 +48,11 @@ constexpr uint32_t kIxQAtom = kIxHeads * 128;               // 2 KB
 constexpr uint32_t kIxOffQ = 2 * kIxKeyTile;                // after the two-stage key ring
 constexpr uint32_t kIxOffKeys = kIxOffQ + 2 * kIxQAtom;     // the query's radix keys (leader)
 
-// Dynamic shared memory: the key ring, the query rows, P radix keys and the
-// select_k selected ids (used by the leader, sized alike on every CTA).
-inline int indexer_smem_bytes(int P, int SK) { return (int)kIxOffKeys + 4 * P + 4 * SK + 1024; }
+// Dynamic shared memory: the key ring (whose space also holds the leader's
+// select_k selected ids once its tiles are done), the query rows and P radix
+// keys (used by the leader, sized alike on every CTA).
+inline int indexer_smem_bytes(int P) { return (int)kIxOffKeys + 4 * P + 1024; }
+static_assert(4 * DSA_MAX_SELECT <= 2 * kIxKeyTile, "selected ids fit in the key ring");
 
 struct IxCtl {
     uint64_t q_bar, load_full[2], mma_done[2], d_empty[2];
@@ -61,6 +64,7 @@ struct IxCtl {
     float gate_in[kIxCluster][kIxHeads];// the cluster's gate partials, by rank
     float gate[kIxHeads];               // the query's gate weights
     int ncand_in[kIxCluster];           // the cluster's candidate counts, by rank (leader)
+    int hist_in[kIxCluster][256];       // the cluster's top-byte histograms, by rank (leader)
     int2 warp2[kIxWarps];
     int pick[3];                        // (digit, count above, count in it) of the current pass
     int ncand;                          // this CTA's candidates
@@ -131,31 +135,6 @@ DSA_DEVINL void cluster_arrive_relaxed() {
 }
 DSA_DEVINL void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
-// Exclusive prefix sums of (a, b) over the CTA's kIxThreads threads; *ta, *tb get the sums.
-DSA_DEVINL int2 ix_excl_scan2(int a, int b, int2 *s_warp2, int *ta, int *tb) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = a, y = b;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, x, off);
-        const int v = __shfl_up_sync(0xffffffffu, y, off);
-        if (lane >= off) { x += u; y += v; }
-    }
-    if (lane == 31) s_warp2[warp] = make_int2(x, y);
-    __syncthreads();
-    int2 before = make_int2(0, 0), tot = make_int2(0, 0);
-#pragma unroll
-    for (int w2 = 0; w2 < kIxWarps; ++w2) {
-        const int2 v = s_warp2[w2];
-        if (w2 < warp) { before.x += v.x; before.y += v.y; }
-        tot.x += v.x;
-        tot.y += v.y;
-    }
-    *ta = tot.x;
-    *tb = tot.y;
-    return make_int2(before.x + x - a, before.y + y - b);
-}
-
 __global__ void __launch_bounds__(kIxThreads, 1)
 indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constant__ CUtensorMap q_map,
                const float *__restrict__ hidden, const float *__restrict__ w, int K, int H,
@@ -171,13 +150,16 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = ix_smem_raw + (base - raw);
     uint32_t *akeys = reinterpret_cast<uint32_t *>(gbase + kIxOffKeys);                 // [P]
-    int32_t *slist = reinterpret_cast<int32_t *>(gbase + kIxOffKeys + 4 * (size_t)P);   // [SK]
+    int32_t *slist = reinterpret_cast<int32_t *>(gbase);   // [SK], in the key ring (leader, at the end)
     const uint32_t sQ = base + kIxOffQ;
 
     const int C = gridDim.x, r = blockIdx.x, q = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const IxRange rg = ix_range(r, C, P);
     const int ntile = rg.t1 - rg.t0;
+    // the query's request and position are step inputs: their loads go out first
+    const int b = q_req[q];
+    const int qp = q_pos[q];
 
     if (warp == 0) {
         tc::tmem_alloc(&ctl->tmem_base, 32);
@@ -249,9 +231,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
 #pragma unroll
         for (int e = 0; e < 4; ++e) ctl->red[kp][4 * hq + e] = acc[e];
     }
-    const int b = q_req[q];                       // a step input, like the query rows
     const bool req_ok = b >= 0 && b < B;
-    const int qp = q_pos[q];
     __syncthreads();
     if (tid < kIxHeads) {
         float gpart = 0.f;
@@ -370,15 +350,21 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
                 st_cluster_u32(lead_keys + 4u * (uint32_t)p, k);
                 local_cand += k != 0u;
             }
+            // this CTA's share of the first radix pass: the top bytes of its keys
+            const uint32_t dgt = p < P ? (score_key(score, is_cand) >> 24) : 0x100u;
+            const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
+            if (dgt != 0x100u && lane == __ffs(peers) - 1) atomicAdd(&ctl->hist[0][dgt], __popc(peers));
         }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) local_cand += __shfl_xor_sync(0xffffffffu, local_cand, off);
     if (lane == 0 && local_cand) atomicAdd(&ctl->ncand, local_cand);
     __syncthreads();
+    // this CTA's histogram and candidate count to the leader, then its release
+    // arrive (after every key this CTA pushed: the CTA barrier orders them before it)
+    st_cluster_u32(cluster_map(smem_u32(&ctl->hist_in[r][tid]), 0), (uint32_t)ctl->hist[0][tid]);
+    __syncthreads();
     if (tid == 0) {
-        // this CTA's candidate count to the leader, then its release arrive (after
-        // every key this CTA pushed: the CTA barrier above orders them before it)
         st_cluster_u32(cluster_map(smem_u32(&ctl->ncand_in[r]), 0), (uint32_t)ctl->ncand);
         asm volatile("fence.acq_rel.cluster;" ::: "memory");
         mbar_arrive_remote(cluster_map(smem_u32(&ctl->keys_bar), 0));
@@ -401,12 +387,12 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         uint32_t prefix = 0, pmask = 0;
         int remaining = nq;
         if (nq > 0) {
-            // pass 0's histogram: the top byte of every key
-            for (int p0 = 0; p0 < P; p0 += kIxThreads) {
-                const int p = p0 + tid;
-                const uint32_t dgt = p < P ? (akeys[p] >> 24) : 0x100u;
-                const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
-                if (dgt != 0x100u && lane == __ffs(peers) - 1) atomicAdd(&ctl->hist[0][dgt], __popc(peers));
+            // pass 0's histogram: the cluster's top-byte histograms added up
+            {
+                int t = 0;
+                for (int c = 0; c < C; ++c) t += ctl->hist_in[c][tid];
+                __syncthreads();
+                ctl->hist[0][tid] = t;
             }
             __syncthreads();
 #pragma unroll 1
@@ -492,29 +478,38 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         const int req_eq = remaining;    // keys equal to tau to take, lowest ids first
 
         // ---- 4. winners in ascending pool id: every key above tau, then the
-        // req_eq lowest-id keys equal to it
-        const int chunk = (P + kIxThreads - 1) / kIxThreads;
-        const int p_lo = min(P, tid * chunk), p_hi = min(P, p_lo + chunk);
-        int gt = 0, eq = 0;
+        // req_eq lowest-id keys equal to it. Warp w places the keys of a contiguous
+        // range, 32 consecutive keys a step (conflict-free reads, ballot ranks).
+        const int span = (((P + kIxWarps - 1) / kIxWarps) + 31) & ~31;
+        const int wlo = min(P, warp * span), whi = min(P, wlo + span);
+        const uint32_t below = (1u << lane) - 1u;
+        int wgt = 0, weq = 0;
         if (nq > 0)
-            for (int p = p_lo; p < p_hi; ++p) {
-                const uint32_t k = akeys[p];
-                gt += k > tau;
-                eq += k == tau;
+            for (int p0 = wlo; p0 < whi; p0 += 32) {
+                const int p = p0 + lane;
+                const uint32_t k = p < whi ? akeys[p] : 0u;
+                wgt += __popc(__ballot_sync(0xffffffffu, p < whi && k > tau));
+                weq += __popc(__ballot_sync(0xffffffffu, p < whi && k == tau));
             }
-        int tot_gt, tot_eq;
-        const int2 before = ix_excl_scan2(gt, eq, ctl->warp2, &tot_gt, &tot_eq);
+        if (lane == 0) ctl->warp2[warp] = make_int2(wgt, weq);
+        __syncthreads();
+        int gt_before = 0, eq_before = 0;
+        for (int w2 = 0; w2 < warp; ++w2) {
+            gt_before += ctl->warp2[w2].x;
+            eq_before += ctl->warp2[w2].y;
+        }
         if (nq > 0) {
-            int pos = before.x + min(before.y, req_eq);
-            int eqr = before.y;
-            for (int p = p_lo; p < p_hi; ++p) {
-                const uint32_t k = akeys[p];
-                if (k > tau) {
-                    slist[pos++] = p;
-                } else if (k == tau) {
-                    if (eqr < req_eq) slist[pos++] = p;
-                    ++eqr;
-                }
+            int pos = gt_before + min(eq_before, req_eq), eqs = eq_before;
+            for (int p0 = wlo; p0 < whi; p0 += 32) {
+                const int p = p0 + lane;
+                const uint32_t k = p < whi ? akeys[p] : 0u;
+                const bool g = p < whi && k > tau, e = p < whi && k == tau;
+                const uint32_t be = __ballot_sync(0xffffffffu, e);
+                const bool take = g || (e && eqs + __popc(be & below) < req_eq);
+                const uint32_t bt = __ballot_sync(0xffffffffu, take);
+                if (take) slist[pos + __popc(bt & below)] = p;
+                pos += __popc(bt);
+                eqs += __popc(be);
             }
         }
         __syncthreads();
@@ -573,7 +568,7 @@ inline int indexer_launch(const float *hidden, const float *w, int K, const void
     if (!make_map_bf16_2d(&key_map, kbase, krows, kD, kD * 2, 64, kIxTile) ||
         !make_map_bf16_2d(&q_map, q_idx, (uint64_t)Q * H, kD, kD * 2, 64, kIxHeads))
         return DSA_ERR_CUDA;
-    const int smem = indexer_smem_bytes(max_pools, select_k);
+    const int smem = indexer_smem_bytes(max_pools);
     if (!ensure_smem_attr(reinterpret_cast<const void *>(indexer_kernel), smem)) return DSA_ERR_CUDA;
     if (launch_pdl_cluster(indexer_kernel, dim3(kIxCluster, Q), dim3(kIxThreads), smem, stream,
                            kIxCluster, key_map, q_map, hidden, w, K, H, q_req, q_pos, pool_valid,

@@ -42,7 +42,7 @@ template <int KP> struct CmpCfg {
     static constexpr int kStageBytes = 2 * kTileTokens * 128 * 2;
 };
 constexpr int kD = DSA_INDEX_DIM;   // 128 channels
-// Requests the balanced partition handles (3 int32 a request in shared memory);
+// Requests the balanced partition handles (4 int32 a request in shared memory);
 // each thread of the CTA owns kCmpReqPerThread consecutive requests.
 constexpr int kCmpReqPerThread = 4;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -288,6 +288,7 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     int32_t *s_f = reinterpret_cast<int32_t *>(cmp_smem + kCmpStages * kCmpStageBytes);
     int32_t *s_pre = s_f + B;
     int32_t *s_epre = s_pre + (B + 1);
+    int32_t *s_rs = s_epre + (B + 1);                // req_start, B + 1 entries
 
     if (tid == 0) {
         for (int s = 0; s < kCmpStages; ++s) {
@@ -324,41 +325,60 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
 
     int g_lo = 0, g_hi = 0, e_lo = 0, e_hi = 0;
     if (balanced) {
-        // ---- each request's first valid token: the 16 validity bytes from its
-        // first row settle almost every request; a warp scans the rest
+        // ---- each request's first valid token: the 64 validity bytes from its
+        // first row settle almost every request (all loads in flight at once);
+        // a warp scans the rest
+        uint4 vq[kCmpReqPerThread][4];
+#pragma unroll
+        for (int u = 0; u < kCmpReqPerThread; ++u) {
+            const long long c0 = (long long)rq_rs[u] & ~15ll;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const long long c = c0 + 16 * j;
+                vq[u][j] = (rb0 + u < B && c + 16 <= total && c < rq_rs[u + 1])
+                               ? __ldg(reinterpret_cast<const uint4 *>(valid + c))
+                               : make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
 #pragma unroll
         for (int u = 0; u < kCmpReqPerThread; ++u) {
             const int b = rb0 + u;
             if (b >= B) break;
             const long long rs = rq_rs[u], re = rq_rs[u + 1];
             const int T = (int)max(0ll, re - rs);
+            s_rs[b] = (int)rs;
+            if (b == B - 1) s_rs[B] = (int)re;
             int f = -1;
             if (T == 0) {
                 f = 0;
             } else {
                 const long long c0 = rs & ~15ll;
                 int hit = -1;
-                if (c0 + 16 <= total) {
-                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(valid + c0));
-                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                bool covered = true;          // every byte of [rs, min(re, c0 + 64)) was loaded
+#pragma unroll
+                for (int j = 3; j >= 0; --j) {
+                    const long long c = c0 + 16 * j;
+                    if (c >= re) continue;
+                    if (c + 16 > total) { covered = false; continue; }
+                    const uint32_t w4[4] = {vq[u][j].x, vq[u][j].y, vq[u][j].z, vq[u][j].w};
 #pragma unroll
                     for (int q = 3; q >= 0; --q)
 #pragma unroll
                         for (int bb = 3; bb >= 0; --bb) {
-                            const long long pos = c0 + 4 * q + bb;
+                            const long long pos = c + 4 * q + bb;
                             if (pos >= rs && pos < re && ((w4[q] >> (8 * bb)) & 0xFF)) hit = (int)(pos - rs);
                         }
-                    if (hit >= 0) f = hit;
-                    else if (c0 + 16 >= re) f = T;
                 }
+                if (hit >= 0 && covered) f = hit;
+                else if (covered && c0 + 64 >= re) f = T;
             }
             s_f[b] = f;
         }
         __syncthreads();
         for (int b = warp; b < B; b += kCmpThreads / 32) {
             if (s_f[b] >= 0) continue;                     // warp-uniform
-            const int rs = req_start[b];
-            const int T = max(0, req_start[b + 1] - rs);
+            const int rs = s_rs[b];
+            const int T = max(0, s_rs[b + 1] - rs);
             const int f = first_valid_scan(valid, rs, T);
             if (lane == 0) s_f[b] = f;
         }
@@ -448,8 +468,8 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             }
             if (b != cur_b) {
                 const bool first = i == 0 && !balanced;
-                cur_rs = first ? first_rs : req_start[b];
-                cur_T = max(0, (first ? first_re : req_start[b + 1]) - cur_rs);
+                cur_rs = balanced ? s_rs[b] : first ? first_rs : req_start[b];
+                cur_T = max(0, (balanced ? s_rs[b + 1] : first ? first_re : req_start[b + 1]) - cur_rs);
                 cur_f = balanced ? s_f[b] : first_valid_scan(valid, cur_rs, cur_T);
                 cur_b = b;
             }
@@ -588,9 +608,9 @@ inline int kpool_compress_launch_kp(const __nv_bfloat16 *k, const __nv_bfloat16 
     // Up to kCmpReqPerThread requests a thread, the CTA splits the tiles that hold
     // pools evenly (balanced); beyond, contiguous ranges of every request's tile grid.
     const int balanced = B <= kCmpReqPerThread * C::kThreads ? 1 : 0;
-    const int smem = C::kStages * C::kStageBytes + (balanced ? 4 * (3 * B + 2) : 0);
+    const int smem = C::kStages * C::kStageBytes + (balanced ? 4 * (4 * B + 3) : 0);
     if (!ensure_smem_attr(reinterpret_cast<const void *>(kpool_compress_kernel<KP>),
-                          C::kStages * C::kStageBytes + 4 * (3 * kCmpReqPerThread * C::kThreads + 2)))
+                          C::kStages * C::kStageBytes + 4 * (4 * kCmpReqPerThread * C::kThreads + 3)))
         return DSA_ERR_CUDA;
     const int tiles_per_req = max(1, ceil_div(max_pools, TP));
     const long long n_tiles = (long long)tiles_per_req * B;

@@ -10,11 +10,12 @@
 // The S partials (O, running max m, running sum l) of a (query, head group)
 // are merged in split order, so results do not depend on scheduling:
 //   S == 1       the CTA normalises and writes bf16 out and the lse itself;
-//   2 <= S <= 8  the S CTAs form a thread-block cluster and merge through
+//   2 <= S <= 16 the S CTAs form a thread-block cluster and merge through
 //                distributed shared memory, each CTA writing its share of the
-//                heads (no partials in global memory, no second launch);
-//   S > 8        (few queries) the partials go to the workspace and a combine
-//                kernel merges them.
+//                heads (no partials in global memory, no second launch), when
+//                all the launch's clusters fit on the device at once;
+//   otherwise    the partials go to the workspace and a combine kernel merges
+//                them.
 #pragma once
 
 #include <atomic>
@@ -80,7 +81,9 @@ constexpr int kSParts = 2;
 constexpr uint32_t kSCol = 256;                     // S buffers: [256, 256 + 2 * kSParts * chunk)
 static_assert(kSCol + 2 * kSParts * kTcChunk <= kTmemCols, "tensor memory columns");
 constexpr float kLazyRescale = 8.0f;                // log2 units
-constexpr int kMaxClusterSplits = 8;                // portable cluster size
+// Splits merged inside a cluster: up to 8 (the portable size) or, where the
+// device fits them, up to 16 (non-portable sizes are allowed on the kernel).
+constexpr int kMaxClusterSplits = 16;
 constexpr int kSmTarget = 148;                      // CTAs of one full wave (one CTA per SM)
 // The cluster merge reads each CTA's O^T, copied as fp32 [64 heads][512] into
 // the (then idle) gathered-row ring.
@@ -154,33 +157,43 @@ DSA_DEVINL void mla_cluster_merge(const TcCtl *ctl, uint32_t sO, int S, int nh, 
     for (int h = hb + (tid >> 7); h < he; h += 2) {
         const uint32_t am = smem_u32(&ctl->mfin[h]), al = smem_u32(&ctl->lsum[h]);
         const uint32_t ao = sO + (uint32_t)h * (kL * 4) + c4 * 16;
-        float ms[kMaxClusterSplits], ls[kMaxClusterSplits];
-        float4 v[kMaxClusterSplits];
+        // the splits' maxima first, then their rows in two rounds of eight (all of a
+        // round's remote loads in flight at once), in split order
+        float ms[kMaxClusterSplits];
 #pragma unroll
-        for (int r = 0; r < kMaxClusterSplits; ++r) {
-            ms[r] = -INFINITY;
-            ls[r] = 0.f;
-            v[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (r < S) {
-                ms[r] = ld_cluster_f32(cluster_map(am, r));
-                ls[r] = ld_cluster_f32(cluster_map(al, r));
-                v[r] = ld_cluster_f32x4(cluster_map(ao, r));   // unused where m is -inf
-            }
-        }
+        for (int r = 0; r < kMaxClusterSplits; ++r)
+            ms[r] = r < S ? ld_cluster_f32(cluster_map(am, r)) : -INFINITY;
         float M = -INFINITY;
 #pragma unroll
         for (int r = 0; r < kMaxClusterSplits; ++r) M = fmaxf(M, ms[r]);
         float o[4] = {0.f, 0.f, 0.f, 0.f};
         float lsum = 0.f;
 #pragma unroll
-        for (int r = 0; r < kMaxClusterSplits; ++r) {
-            if (ms[r] == -INFINITY) continue;
-            const float w = ex2(ms[r] - M);
-            lsum = fmaf(ls[r], w, lsum);
-            o[0] = fmaf(v[r].x, w, o[0]);
-            o[1] = fmaf(v[r].y, w, o[1]);
-            o[2] = fmaf(v[r].z, w, o[2]);
-            o[3] = fmaf(v[r].w, w, o[3]);
+        for (int r0 = 0; r0 < kMaxClusterSplits; r0 += 8) {
+            if (r0 >= S) break;
+            float ls[8];
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int r = r0 + u;
+                ls[u] = 0.f;
+                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (r < S && ms[r] != -INFINITY) {
+                    ls[u] = ld_cluster_f32(cluster_map(al, r));
+                    v[u] = ld_cluster_f32x4(cluster_map(ao, r));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int r = r0 + u;
+                if (r >= S || ms[r] == -INFINITY) continue;
+                const float w = ex2(ms[r] - M);
+                lsum = fmaf(ls[u], w, lsum);
+                o[0] = fmaf(v[u].x, w, o[0]);
+                o[1] = fmaf(v[u].y, w, o[1]);
+                o[2] = fmaf(v[u].z, w, o[2]);
+                o[3] = fmaf(v[u].w, w, o[3]);
+            }
         }
         const float inv = lsum > 0.f ? out_scale / lsum : 0.f;
         uint2 packed;
@@ -242,6 +255,19 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
     const int ntok = j1 - j0;
     const int nch = (ntok + kTcChunk - 1) / kTcChunk;
     const int h0 = hg * kTcHeads, nh = min(kTcHeads, Hm - h0);
+    // Request geometry is a step input: its loads go out before the set-up and are
+    // used after the wait on the predecessor.
+    const int b = q_req[qi];
+    const bool req_ok = b >= 0 && b < B;
+    int rs = 0, T = 0;
+    if (req_ok) {
+        if constexpr (kPaged) {
+            T = max(0, map.seq_len[b]);
+        } else {
+            rs = map.req_start[b];
+            T = max(0, map.req_start[b + 1] - rs);
+        }
+    }
 
     if (warp >= 4 && warp < 8) {
         // Q tile (a step input): 64 rows x 64 16-byte chunks into the swizzled
@@ -282,18 +308,6 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
-    // Request geometry is a step input: read before the wait on the predecessor.
-    const int b = q_req[qi];
-    const bool req_ok = b >= 0 && b < B;
-    int rs = 0, T = 0;
-    if (req_ok) {
-        if constexpr (kPaged) {
-            T = max(0, map.seq_len[b]);
-        } else {
-            rs = map.req_start[b];
-            T = max(0, map.req_start[b + 1] - rs);
-        }
-    }
     pdl_wait();                       // token ids come from the predecessor grid
     pdl_launch_dependents();
 
@@ -801,6 +815,15 @@ mla_combine_kernel(const uint8_t *__restrict__ part, int Hm, int S, float out_sc
         lse[(size_t)q * Hm + h] = lsum > 0.f ? (M + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
 }
 
+// Raise the cluster kernel's shared-memory limit and allow cluster sizes above
+// the portable 8 (once per device; false if the runtime refuses).
+template <bool kPaged, bool kFp8>
+inline bool mla_prepare_cluster_kernel() {
+    const void *f = reinterpret_cast<const void *>(mla_tc_kernel<true, kPaged, kFp8>);
+    if (!ensure_smem_attr(f, kTcSmemBytes)) return false;
+    return cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+}
+
 // How many clusters of `splits` CTAs of the cluster kernel can be resident at
 // once on the current device (asked once per device and size, after the
 // kernel's shared-memory limit is raised); 0 when none or unknown.
@@ -828,7 +851,7 @@ inline int mla_max_clusters(int splits) {
     return n;
 }
 
-// The launch: a plan of 2 or more splits runs as clusters of at most 8 CTAs
+// The launch: a plan of 2 or more splits runs as clusters of at most 16 CTAs
 // when all of a grid's clusters can be resident at once, shrinking the cluster
 // (more chunks per CTA) while that costs at most two chunks per CTA over the
 // plan -- about what the global merge and its second launch cost; otherwise
@@ -853,8 +876,7 @@ inline MlaGeom mla_launch_geometry(int Q, int Hm, int W) {
 // split kernel, plus the combine when the splits merge through the workspace.
 inline int sparse_mla_launch_count(int Q, int Hm, int W) {
     if (Q <= 0 || Hm <= 0 || W < 0) return 0;
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, false, false>), kTcSmemBytes))
-        return 0;
+    if (!mla_prepare_cluster_kernel<false, false>()) return 0;
     const MlaGeom g = mla_launch_geometry(Q, Hm, W);
     return (g.S > 1 && !g.cluster) ? 2 : 1;
 }
@@ -886,9 +908,9 @@ inline int sparse_mla_launch_map(const void *q, const void *kv, int64_t kv_rows,
         return DSA_ERR_ALIGNMENT;
     const size_t need = mla_workspace_bytes(Q, Hm, W);
     if (need > 0 && (!ws || ws_bytes < need)) return DSA_ERR_WORKSPACE;
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, kPaged, kFp8>), kTcSmemBytes) ||
+    if (!mla_prepare_cluster_kernel<kPaged, kFp8>() ||
         !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<false, kPaged, kFp8>), kTcSmemBytes) ||
-        !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<true, false, false>), kTcSmemBytes))
+        !mla_prepare_cluster_kernel<false, false>())
         return DSA_ERR_CUDA;
     const MlaGeom g = mla_launch_geometry(Q, Hm, W);
     // fp8: S = sm_scale * q . (s k8) = (sm_scale * s) q . k8, and O = s * (P V8)

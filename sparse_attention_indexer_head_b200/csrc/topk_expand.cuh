@@ -8,9 +8,9 @@
 // radix select finds the n_q-th largest key tau exactly: two passes, then,
 // when at most 32 keys share those 16 bits with tau, a rank among them on one
 // warp, else two more passes; the winners are
-// every key above tau plus the lowest-id keys equal to tau (an id-ordered
-// block scan), written in ascending pool id, so the result is bit-exact and
-// deterministic. The expansion gathers pool_idx rows and writes every slot of
+// every key above tau plus the lowest-id keys equal to tau (placed by warps
+// over contiguous id ranges with ballot ranks), written in ascending pool id,
+// so the result is bit-exact and deterministic. The expansion gathers pool_idx rows and writes every slot of
 // the [select_k * kpool] row, -1 past n_q.
 #pragma once
 
@@ -28,35 +28,6 @@ DSA_DEVINL uint32_t score_key(float s, bool is_cand) {
     if (s == 0.f) s = 0.f;          // -0 ranks as +0
     const uint32_t u = __float_as_uint(s);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Exclusive prefix sums of (a, b) over the block in one pass; *ta, *tb get the sums.
-DSA_DEVINL int2 block_excl_scan2(int a, int b, int2 *s_warp2, int *ta, int *tb) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = a, y = b;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, x, off);
-        const int v = __shfl_up_sync(0xffffffffu, y, off);
-        if (lane >= off) { x += u; y += v; }
-    }
-    if (lane == 31) s_warp2[warp] = make_int2(x, y);
-    __syncthreads();
-    if (warp == 0) {
-        int2 w = lane < kTopkWarps ? s_warp2[lane] : make_int2(0, 0);
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int u = __shfl_up_sync(0xffffffffu, w.x, off);
-            const int v = __shfl_up_sync(0xffffffffu, w.y, off);
-            if (lane >= off) { w.x += u; w.y += v; }
-        }
-        if (lane < kTopkWarps) s_warp2[lane] = w;   // inclusive warp totals
-    }
-    __syncthreads();
-    const int2 before = warp ? s_warp2[warp - 1] : make_int2(0, 0);
-    *ta = s_warp2[kTopkWarps - 1].x;
-    *tb = s_warp2[kTopkWarps - 1].y;
-    return make_int2(before.x + x - a, before.y + y - b);
 }
 
 // Tail slots (always_select_tail): after the K * KP pool slots, a row carries
@@ -243,32 +214,40 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     const uint32_t tau = prefix;   // the nq-th largest key (when nq > 0)
     const int r = remaining;       // keys equal to tau to take, lowest ids first
 
-    // Selection in id order over contiguous per-thread chunks.
-    const int chunk = (P + kTopkThreads - 1) / kTopkThreads;
-    const int p_lo = min(P, tid * chunk), p_hi = min(P, p_lo + chunk);
-    int gt = 0, eq = 0;
+    // Selection in id order: warp w places the keys of a contiguous range, 32
+    // consecutive keys a step (conflict-free reads, ballot ranks): every key above
+    // tau, then the r lowest-id keys equal to it.
+    const int lane = tid & 31, warp = tid >> 5;
+    const int span = (((P + kTopkWarps - 1) / kTopkWarps) + 31) & ~31;
+    const int wlo = min(P, warp * span), whi = min(P, wlo + span);
+    const uint32_t below = (1u << lane) - 1u;
+    int wgt = 0, weq = 0;
     if (nq > 0)
-        for (int p = p_lo; p < p_hi; ++p) {
-            const uint32_t k = key_at(p);
-            gt += k > tau;
-            eq += k == tau;
+        for (int p0 = wlo; p0 < whi; p0 += 32) {
+            const int p = p0 + lane;
+            const uint32_t k = p < whi ? key_at(p) : 0u;
+            wgt += __popc(__ballot_sync(0xffffffffu, p < whi && k > tau));
+            weq += __popc(__ballot_sync(0xffffffffu, p < whi && k == tau));
         }
-    int tot_gt, tot_eq;
-    const int2 before = block_excl_scan2(gt, eq, s_warp2, &tot_gt, &tot_eq);
-    const int gt_before = before.x, eq_before = before.y;
-    // The winners in ascending pool id: every key above tau, then the r lowest-id
-    // keys equal to tau, each placed at its id-order position.
+    if (lane == 0) s_warp2[warp] = make_int2(wgt, weq);
+    __syncthreads();
+    int gt_before = 0, eq_before = 0;
+    for (int w2 = 0; w2 < warp; ++w2) {
+        gt_before += s_warp2[w2].x;
+        eq_before += s_warp2[w2].y;
+    }
     if (nq > 0) {
-        int pos = gt_before + min(eq_before, r);
-        int eqr = eq_before;
-        for (int p = p_lo; p < p_hi; ++p) {
-            const uint32_t k = key_at(p);
-            if (k > tau) {
-                slist[pos++] = p;
-            } else if (k == tau) {
-                if (eqr < r) slist[pos++] = p;
-                ++eqr;
-            }
+        int pos = gt_before + min(eq_before, r), eqs = eq_before;
+        for (int p0 = wlo; p0 < whi; p0 += 32) {
+            const int p = p0 + lane;
+            const uint32_t k = p < whi ? key_at(p) : 0u;
+            const bool g = p < whi && k > tau, e = p < whi && k == tau;
+            const uint32_t be = __ballot_sync(0xffffffffu, e);
+            const bool take = g || (e && eqs + __popc(be & below) < r);
+            const uint32_t bt = __ballot_sync(0xffffffffu, take);
+            if (take) slist[pos + __popc(bt & below)] = p;
+            pos += __popc(bt);
+            eqs += __popc(be);
         }
     }
     __syncthreads();
