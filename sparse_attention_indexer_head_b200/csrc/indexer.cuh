@@ -515,20 +515,32 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         __syncthreads();
         const size_t wrow = (size_t)SK * KP;
         for (int j = tid; j < SK; j += kIxThreads) top_pools[(size_t)q * SK + j] = j < nq ? slist[j] : -1;
-        // expansion: four pool_idx gathers in flight per thread before the stores
-        for (int e0 = 0; e0 < SK * KP; e0 += 4 * kIxThreads) {
-            int32_t v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + tid + u * kIxThreads;
-                const int j = e / KP, s = e - j * KP;
-                v[u] = -1;
-                if (e < SK * KP && j < nq) v[u] = __ldg(pool_idx + ((size_t)b * P + slist[j]) * KP + s);
+        // expansion: with kpool a multiple of 4 and 16-byte aligned rows, a
+        // selected pool's ids move as kpool/4 vector loads and stores; otherwise
+        // four scalar gathers in flight per thread before the stores
+        if ((KP & 3) == 0 && aligned16(pool_idx) && aligned16(token_ids)) {
+            const int nv = KP >> 2;                         // 16-byte pieces a pool
+            const int4 *src = reinterpret_cast<const int4 *>(pool_idx + (size_t)b * P * KP);
+            int4 *dst = reinterpret_cast<int4 *>(token_ids + (size_t)q * wrow);
+            for (int e = tid; e < SK * nv; e += kIxThreads) {
+                const int j = e / nv, u = e - j * nv;
+                dst[e] = j < nq ? __ldg(src + (size_t)slist[j] * nv + u) : make_int4(-1, -1, -1, -1);
             }
+        } else {
+            for (int e0 = 0; e0 < SK * KP; e0 += 4 * kIxThreads) {
+                int32_t v[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + tid + u * kIxThreads;
-                if (e < SK * KP) token_ids[(size_t)q * wrow + e] = v[u];
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + tid + u * kIxThreads;
+                    const int j = e / KP, s = e - j * KP;
+                    v[u] = -1;
+                    if (e < SK * KP && j < nq) v[u] = __ldg(pool_idx + ((size_t)b * P + slist[j]) * KP + s);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + tid + u * kIxThreads;
+                    if (e < SK * KP) token_ids[(size_t)q * wrow + e] = v[u];
+                }
             }
         }
     }

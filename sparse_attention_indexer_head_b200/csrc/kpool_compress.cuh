@@ -33,10 +33,12 @@ namespace dsa {
 // 4); larger pools (more live registers) 8 warps and floor(128 / kpool) pools.
 // A stage holds the tile's k rows then its gate rows; three stages in the ring.
 template <int KP> struct CmpCfg {
-    static constexpr int kWarps = KP <= 4 ? 15 : 8;             // consumer warps
+    static constexpr int kPoolWarps = KP <= 4 ? 12 : 6;         // a half-warp per pool
+    static constexpr int kStatWarps = KP <= 4 ? 3 : 2;          // LayerNorm statistics, a tile ahead
+    static constexpr int kWarps = kPoolWarps + kStatWarps;      // consumer warps
     static constexpr int kConsumers = kWarps * 32;
     static constexpr int kThreads = kConsumers + 32;            // + 1 producer warp
-    static constexpr int kTP = KP <= 4 ? 120 / KP : 128 / KP;   // pools per tile
+    static constexpr int kTP = 2 * kPoolWarps;                  // pools per tile
     static constexpr int kTileTokens = kTP * KP;
     static constexpr int kStages = 3;
     static constexpr int kStageBytes = 2 * kTileTokens * 128 * 2;
@@ -46,6 +48,14 @@ constexpr int kD = DSA_INDEX_DIM;   // 128 channels
 // each thread of the CTA owns kCmpReqPerThread consecutive requests.
 constexpr int kCmpReqPerThread = 4;
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Bit i of the result is set iff byte i of w is nonzero: (low seven bits + 0x7F)
+// carries into a byte's top bit iff those bits are not all zero, and the OR adds
+// the byte's own top bit; no carry crosses into the next byte.
+DSA_DEVINL uint32_t nonzero_bytes(uint32_t w) {
+    const uint32_t h = (((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w) & 0x80808080u;
+    return ((h >> 7) & 1u) | ((h >> 14) & 2u) | ((h >> 21) & 4u) | ((h >> 28) & 8u);
+}
 
 // First index in [0, T) of request rows [rs, rs+T) whose valid byte is nonzero;
 // T if none. Executed by one full warp; the result is returned to every lane.
@@ -259,7 +269,7 @@ template <int KP>
 __global__ void __launch_bounds__(CmpCfg<KP>::kThreads, 1)
 kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ gate,
                       const uint8_t *__restrict__ valid, const int32_t *__restrict__ req_start,
-                      int B, int max_pools, int tiles_per_req, int n_tiles, int balanced,
+                      int B, int max_pools, int tiles_per_req, int n_tiles, int balance_ok,
                       const float *__restrict__ ape, const __nv_bfloat16 *__restrict__ ln_w,
                       const __nv_bfloat16 *__restrict__ ln_b, float eps,
                       __nv_bfloat16 *__restrict__ pool_keys, int32_t *__restrict__ pool_idx,
@@ -274,9 +284,10 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     extern __shared__ __align__(128) uint8_t cmp_smem[];
     __shared__ __align__(16) float s_ape[KP * kD];   // ape * log2(e), [slot][half][lane][4]
     __shared__ __align__(16) float2 s_stat[kCmpStages][kCmpTileTokens];   // (rstd, -mu*rstd)
-    __shared__ __align__(8) uint64_t full[kCmpStages], empty[kCmpStages];
+    __shared__ __align__(8) uint64_t full[kCmpStages], empty[kCmpStages], stat_full[kCmpStages];
     __shared__ CmpMeta meta[kCmpStages];
     __shared__ __align__(16) uint8_t s_valid[kCmpStages][kCmpValidWindow];
+    __shared__ int s_np_lo, s_np_hi;      // fewest and most pools a request holds
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x;
@@ -293,17 +304,41 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     if (tid == 0) {
         for (int s = 0; s < kCmpStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kCmpConsumers / 32);
+            mbar_init(&empty[s], C::kPoolWarps);
+            mbar_init(&stat_full[s], C::kStatWarps);
         }
         fence_mbarrier_init();
+        s_np_lo = INT_MAX;
+        s_np_hi = 0;
     }
     for (int i = tid; i < KP * kD; i += kCmpThreads) {
         const int sl = i / kD, c = i % kD;
         s_ape[(sl * 2 + ((c >> 2) & 1)) * 64 + 4 * (c >> 3) + (c & 3)] = ape[i] * kLog2e;
     }
     __syncthreads();
-    // Request offsets are a step input the path never writes: the producer has
-    // its first request's rows before the wait on the preceding kernel.
+    // Request offsets and validity bytes are step inputs the path never writes:
+    // the producer has its first request's rows, and the balanced partition is
+    // complete, before the wait on the preceding kernel.
+    // The balanced partition pays only where the requests' pool counts differ by
+    // more than a tile; otherwise every request's tile grid holds about as many
+    // real tiles and contiguous ranges of the grids are even already.
+    bool balanced = false;
+    if (balance_ok) {
+        int lo = INT_MAX, hi = 0;
+        for (int b = tid; b < B; b += kCmpThreads) {
+            const int np = min(max_pools, max(0, req_start[b + 1] - req_start[b]) / KP);
+            lo = min(lo, np);
+            hi = max(hi, np);
+        }
+        lo = __reduce_min_sync(0xffffffffu, lo);
+        hi = __reduce_max_sync(0xffffffffu, hi);
+        if (lane == 0) {
+            atomicMin(&s_np_lo, lo);
+            atomicMax(&s_np_hi, hi);
+        }
+        __syncthreads();
+        balanced = s_np_hi - s_np_lo > TP;
+    }
     long long total = 0;
     int first_rs = 0, first_re = 0;
     if (!balanced && warp == kCmpConsumers / 32 && t_begin < t_end) {
@@ -312,67 +347,41 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         first_rs = req_start[b0];
         first_re = req_start[b0 + 1];
     }
-    // balanced: thread t owns requests [kCmpReqPerThread t, ... + kCmpReqPerThread)
-    int rq_rs[kCmpReqPerThread + 1];
-    const int rb0 = tid * kCmpReqPerThread;
-    if (balanced) {
-#pragma unroll
-        for (int u = 0; u <= kCmpReqPerThread; ++u) rq_rs[u] = rb0 + u <= B ? req_start[rb0 + u] : 0;
-        total = req_start[B];
-    }
-    pdl_wait();
-    pdl_launch_dependents();
-
     int g_lo = 0, g_hi = 0, e_lo = 0, e_hi = 0;
     if (balanced) {
-        // ---- each request's first valid token: the 64 validity bytes from its
-        // first row settle almost every request (all loads in flight at once);
-        // a warp scans the rest
-        uint4 vq[kCmpReqPerThread][4];
-#pragma unroll
-        for (int u = 0; u < kCmpReqPerThread; ++u) {
-            const long long c0 = (long long)rq_rs[u] & ~15ll;
+        total = req_start[B];
+        // ---- each request's first valid token, a thread a request: the first 64
+        // validity bytes from the request's first row (four 16-byte loads, a
+        // nonzero-byte mask) settle almost every request; a warp scans the rest
+#pragma unroll 1
+        for (int b = tid; b < B; b += kCmpThreads) {
+            const long long rs = req_start[b], re = req_start[b + 1];
+            const long long c0 = rs & ~15ll;
+            uint4 v[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const long long c = c0 + 16 * j;
-                vq[u][j] = (rb0 + u < B && c + 16 <= total && c < rq_rs[u + 1])
-                               ? __ldg(reinterpret_cast<const uint4 *>(valid + c))
-                               : make_uint4(0u, 0u, 0u, 0u);
+                v[j] = c < re && c + 16 <= total ? __ldg(reinterpret_cast<const uint4 *>(valid + c))
+                                                 : make_uint4(0u, 0u, 0u, 0u);
             }
-        }
+            uint64_t m = 0;             // bit i: validity byte c0 + i is nonzero
 #pragma unroll
-        for (int u = 0; u < kCmpReqPerThread; ++u) {
-            const int b = rb0 + u;
-            if (b >= B) break;
-            const long long rs = rq_rs[u], re = rq_rs[u + 1];
+            for (int j = 0; j < 4; ++j)
+                m |= (uint64_t)(nonzero_bytes(v[j].x) | nonzero_bytes(v[j].y) << 4 |
+                                nonzero_bytes(v[j].z) << 8 | nonzero_bytes(v[j].w) << 12) << (16 * j);
+            const long long wend = min(re, c0 + 64);      // the window's end within the request
+            m &= ~0ull << (int)(rs - c0);
+            if (wend - c0 < 64) m &= (1ull << (int)max(0ll, wend - c0)) - 1ull;
             const int T = (int)max(0ll, re - rs);
+            const bool covered = wend <= (total & ~15ll);  // every chunk of the window was loaded
+            int f;
+            if (T == 0) f = 0;
+            else if (!covered) f = -1;
+            else if (m) f = (int)(c0 + __ffsll((long long)m) - 1 - rs);
+            else f = wend == re ? T : -1;
+            s_f[b] = f;
             s_rs[b] = (int)rs;
             if (b == B - 1) s_rs[B] = (int)re;
-            int f = -1;
-            if (T == 0) {
-                f = 0;
-            } else {
-                const long long c0 = rs & ~15ll;
-                int hit = -1;
-                bool covered = true;          // every byte of [rs, min(re, c0 + 64)) was loaded
-#pragma unroll
-                for (int j = 3; j >= 0; --j) {
-                    const long long c = c0 + 16 * j;
-                    if (c >= re) continue;
-                    if (c + 16 > total) { covered = false; continue; }
-                    const uint32_t w4[4] = {vq[u][j].x, vq[u][j].y, vq[u][j].z, vq[u][j].w};
-#pragma unroll
-                    for (int q = 3; q >= 0; --q)
-#pragma unroll
-                        for (int bb = 3; bb >= 0; --bb) {
-                            const long long pos = c + 4 * q + bb;
-                            if (pos >= rs && pos < re && ((w4[q] >> (8 * bb)) & 0xFF)) hit = (int)(pos - rs);
-                        }
-                }
-                if (hit >= 0 && covered) f = hit;
-                else if (covered && c0 + 64 >= re) f = T;
-            }
-            s_f[b] = f;
         }
         __syncthreads();
         for (int b = warp; b < B; b += kCmpThreads / 32) {
@@ -383,14 +392,16 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             if (lane == 0) s_f[b] = f;
         }
         __syncthreads();
-        // ---- per request: tiles of pools in its span, pool slots past it; prefix sums
+        // ---- per request: tiles of pools in its span, pool slots past it; prefix
+        // sums (thread t owns requests kCmpReqPerThread t, ... + kCmpReqPerThread)
+        const int rb0 = tid * kCmpReqPerThread;
         int tl[kCmpReqPerThread], em[kCmpReqPerThread], st = 0, se = 0;
 #pragma unroll
         for (int u = 0; u < kCmpReqPerThread; ++u) {
             const int b = rb0 + u;
             tl[u] = em[u] = 0;
             if (b < B) {
-                const int T = (int)max(0ll, (long long)rq_rs[u + 1] - rq_rs[u]);
+                const int T = max(0, s_rs[b + 1] - s_rs[b]);
                 const int n_span = max(0, min(max_pools, (T - s_f[b]) / KP));
                 tl[u] = (n_span + TP - 1) / TP;
                 em[u] = max_pools - n_span;
@@ -433,6 +444,10 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         e_hi = (int)((long long)(blockIdx.x + 1) * E / G);
         t_begin = 0;
         t_end = g_hi - g_lo;                       // this CTA's tiles, in order
+    }
+    pdl_wait();
+    pdl_launch_dependents();
+    if (balanced) {
         // first_valid: this CTA's share of the requests
         const int b_lo = (int)((long long)blockIdx.x * B / G), b_hi = (int)((long long)(blockIdx.x + 1) * B / G);
         for (int b = b_lo + tid; b < b_hi; b += kCmpThreads) first_valid[b] = s_f[b];
@@ -534,34 +549,33 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     }
 
     // -------------------------------------------------------------------- consumer warps
+    // Warp-specialised: kStatWarps warps take each tile's LayerNorm statistics as
+    // soon as it lands (a tile ahead of the pools), kPoolWarps warps compress its
+    // pools once the statistics are in; mbarriers hand the tiles over, so no
+    // barrier spans all consumers.
+    if (warp >= C::kPoolWarps) {
+        const int stid = tid - C::kPoolWarps * 32;
+        for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
+            const int s = i % kCmpStages;
+            const bool ok = mbar_wait(&full[s], (i / kCmpStages) & 1);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
+            token_stats(sk, meta[s].n_in * KP, eps, &s_stat[s][0], stid, C::kStatWarps * 32);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&stat_full[s]);
+        }
+        return;
+    }
     const int hw = tid >> 4;     // half-warp: one pool at a time
     const int l = tid & 15;      // channels 8l .. 8l+7
     float2 lw[4], lb[4];
     unpack8x2(ldg_nc_v4(ln_w + 8 * l), lw);
     unpack8x2(ldg_nc_v4(ln_b + 8 * l), lb);
-
-    // Consumer-wide barrier (named barrier 1) that also ORs a stop flag, so every
-    // consumer thread takes the same decision to leave.
-    auto bar_or = [&](bool v) -> bool {
-        uint32_t r;
-        asm volatile(
-            "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-            "bar.red.or.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-            : "=r"(r)
-            : "r"((uint32_t)v), "n"(kCmpConsumers)
-            : "memory");
-        return r != 0;
-    };
-    // Per tile: wait for its data, its LayerNorm statistics, the barrier (which
-    // also decides, for every consumer alike, whether a wait gave up), its pools.
+    constexpr int kPoolThreads = C::kPoolWarps * 32;
     for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
         const int s = i % kCmpStages;
-        const bool bad = __any_sync(0xffffffffu, !mbar_wait(&full[s], (i / kCmpStages) & 1));
-        if (!bad) {
-            const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
-            token_stats(sk, meta[s].n_in * KP, eps, &s_stat[s][0], tid, kCmpConsumers);
-        }
-        if (bar_or(bad)) break;
+        const bool ok = mbar_wait(&stat_full[s], (i / kCmpStages) & 1);
+        if (!__all_sync(0xffffffffu, ok)) break;
         const CmpMeta m = meta[s];
         const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
         const __nv_bfloat16 *sg = sk + kCmpTileTokens * kD;
@@ -569,28 +583,27 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         if (!balanced && m.p0 == 0 && tid == 0) first_valid[m.b] = m.f;
 
         // Pools of this tile past the request's span: no key, index -1, invalid.
-        for (int x = m.n_in * KP + tid; x < (m.p1 - m.p0) * KP; x += kCmpConsumers)
+        for (int x = m.n_in * KP + tid; x < (m.p1 - m.p0) * KP; x += kPoolThreads)
             pool_idx[(pool_base + m.p0) * KP + x] = -1;
-        for (int x = m.n_in + tid; x < m.p1 - m.p0; x += kCmpConsumers)
+        for (int x = m.n_in + tid; x < m.p1 - m.p0; x += kPoolThreads)
             pool_valid[pool_base + m.p0 + x] = 0;
 
         // Warp-uniform loop: the two half-warps of a warp take pools ii and ii+1;
         // a half-warp past the tile computes on a loaded row and stores nothing.
-        for (int ii = 2 * warp; ii < m.n_in; ii += kCmpConsumers / 16) {
+        for (int ii = 2 * warp; ii < m.n_in; ii += kPoolThreads / 16) {
             const bool active = ii + (hw & 1) < m.n_in;
             const int pi = active ? ii + (hw & 1) : ii;
             const int p = m.p0 + pi;
-            // pool valid iff every slot token is valid (read from the stage's window)
-            bool ok = true;
+            bool okp = true;
 #pragma unroll
-            for (int ss = 0; ss < KP; ++ss) ok = ok && s_valid[s][m.voff + pi * KP + ss] != 0;
+            for (int ss = 0; ss < KP; ++ss) okp = okp && s_valid[s][m.voff + pi * KP + ss] != 0;
             const uint4 o = compress_pool<KP>(sk + (size_t)pi * KP * kD + 8 * l,
                                               sg + (size_t)pi * KP * kD + 8 * l,
-                                              &s_stat[s][pi * KP], s_ape, lw, lb, l, ok);
+                                              &s_stat[s][pi * KP], s_ape, lw, lb, l, okp);
             if (!active) continue;
             *reinterpret_cast<uint4 *>(pool_keys + (pool_base + p) * kD + 8 * l) = o;
-            if (l < KP) pool_idx[(pool_base + p) * KP + l] = ok ? m.f + p * KP + l : -1;
-            if (l == 0) pool_valid[pool_base + p] = ok ? 1 : 0;
+            if (l < KP) pool_idx[(pool_base + p) * KP + l] = okp ? m.f + p * KP + l : -1;
+            if (l == 0) pool_valid[pool_base + p] = okp ? 1 : 0;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
@@ -605,10 +618,11 @@ inline int kpool_compress_launch_kp(const __nv_bfloat16 *k, const __nv_bfloat16 
                                     int32_t *idx, uint8_t *pv, int32_t *fv, cudaStream_t stream) {
     using C = CmpCfg<KP>;
     constexpr int TP = C::kTP;
-    // Up to kCmpReqPerThread requests a thread, the CTA splits the tiles that hold
-    // pools evenly (balanced); beyond, contiguous ranges of every request's tile grid.
-    const int balanced = B <= kCmpReqPerThread * C::kThreads ? 1 : 0;
-    const int smem = C::kStages * C::kStageBytes + (balanced ? 4 * (4 * B + 3) : 0);
+    // Up to kCmpReqPerThread requests a thread, the CTA may split the tiles that
+    // hold pools evenly (balanced, where request lengths differ); beyond, always
+    // contiguous ranges of every request's tile grid.
+    const int balance_ok = B <= kCmpReqPerThread * C::kThreads ? 1 : 0;
+    const int smem = C::kStages * C::kStageBytes + (balance_ok ? 4 * (4 * B + 3) : 0);
     if (!ensure_smem_attr(reinterpret_cast<const void *>(kpool_compress_kernel<KP>),
                           C::kStages * C::kStageBytes + 4 * (4 * kCmpReqPerThread * C::kThreads + 3)))
         return DSA_ERR_CUDA;
@@ -617,7 +631,7 @@ inline int kpool_compress_launch_kp(const __nv_bfloat16 *k, const __nv_bfloat16 
     if (n_tiles > (1ll << 30)) return DSA_ERR_UNSUPPORTED;
     const int grid = (int)std::min<long long>(n_tiles, sm_count());
     if (launch_pdl(kpool_compress_kernel<KP>, dim3(grid), dim3(C::kThreads), smem, stream, k, gate,
-                   valid, req_start, B, max_pools, tiles_per_req, (int)n_tiles, balanced, ape, ln_w,
+                   valid, req_start, B, max_pools, tiles_per_req, (int)n_tiles, balance_ok, ape, ln_w,
                    ln_b, eps, keys, idx, pv, fv) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();

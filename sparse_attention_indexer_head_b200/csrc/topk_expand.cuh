@@ -268,7 +268,19 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
     }
     for (int j = tid; j < K; j += kTopkThreads)
         top_pools[(size_t)q * K + j] = j < nq ? slist[j] : -1;
-    // Expansion: four pool_idx gathers in flight per thread before the stores.
+    // Expansion: with kpool a multiple of 4, no tail slots and 16-byte aligned
+    // rows, a selected pool's ids move as kpool/4 vector loads and stores;
+    // otherwise four scalar gathers in flight per thread before the stores.
+    if (tail.slots == 0 && (KP & 3) == 0 && aligned16(pool_idx) && aligned16(token_ids)) {
+        const int nv = KP >> 2;
+        const int4 *src = reinterpret_cast<const int4 *>(pool_idx + (size_t)(req_ok ? b : 0) * P * KP);
+        int4 *dst = reinterpret_cast<int4 *>(token_ids + (size_t)q * wout);
+        for (int e = tid; e < K * nv; e += kTopkThreads) {
+            const int j = e / nv, u = e - j * nv;
+            dst[e] = j < nq ? __ldg(src + (size_t)slist[j] * nv + u) : make_int4(-1, -1, -1, -1);
+        }
+        return;
+    }
     for (int e0 = 0; e0 < K * KP; e0 += 4 * kTopkThreads) {
         int32_t v[4];
 #pragma unroll

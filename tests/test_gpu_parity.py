@@ -101,16 +101,19 @@ def test_every_kpool_with_ragged_requests(B, kpool):
     device_status_clean(B)
 
 
-@pytest.mark.parametrize("kpool,n_req", [(4, 2100), (8, 1200), (3, 300)])
-def test_compress_partitions(B, kpool, n_req):
+@pytest.mark.parametrize("kpool,n_req,max_len,max_pools",
+                         [(4, 2100, 60, 16), (8, 1200, 60, 16), (3, 300, 60, 16),
+                          (4, 300, 2000, 512), (8, 90, 3000, 400)])
+def test_compress_partitions(B, kpool, n_req, max_len, max_pools):
     """Request counts past the balanced partition's limit (2048 requests at kpool <= 4,
-    1152 above) take the per-request tile grid; below it, the tiles holding pools are
-    split evenly. Lengths 0-60 with random padding, so many requests end in a partial
-    pool, have no valid token or are empty."""
+    1152 above) take the per-request tile grid, and so do requests whose pool counts
+    lie within a tile of one another (lengths 0-60); lengths spread over hundreds of
+    pools below the limit split the tiles holding pools evenly. Random padding, so
+    many requests end in a partial pool, have no valid token or are empty."""
     rng = np.random.default_rng(n_req)
-    lengths = rng.integers(0, 61, n_req).tolist()
-    pads = [int(rng.integers(0, t + 1)) if t else 0 for t in lengths]
-    wl = _mini(kpool, lengths, pads, select_k=4, max_pools=16)
+    lengths = rng.integers(0, max_len + 1, n_req).tolist()
+    pads = [int(rng.integers(0, min(t, 100) + 1)) if t else 0 for t in lengths]
+    wl = _mini(kpool, lengths, pads, select_k=4, max_pools=max_pools)
     step, g = run_step(wl)
     keys, idx, pv, fv = O.kpool_compress(wl.k, wl.gate, wl.valid, wl.req_start, wl.kpool,
                                          wl.max_pools, wl.ape, wl.ln_w, wl.ln_b, wl.eps)
