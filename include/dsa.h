@@ -277,10 +277,12 @@ int dsa_topk_expand_tail(const float *scores, const uint8_t *cand, const int32_t
  * (as dsa_index_scores, from this gate_w), top_pools int32 [Q, select_k] and
  * token_ids int32 [Q, select_k * kpool] (as dsa_topk_expand, from these
  * scores: the same ranking, ties and -1 tail).
- * One thread-block cluster of up to 8 CTAs per query splits K for the gate and
- * the pools for the scores; partial gates and the top-k histograms meet
- * through distributed shared memory, so nothing but the outputs goes to
- * global memory and results are deterministic. The gate's K-split differs from
+ * One thread-block cluster per query -- 8 CTAs, or 16 when so few queries
+ * would leave most of the device idle and the device holds that many such
+ * clusters at once -- splits K for the gate and the pools for the scores and
+ * the select; partial gates, the radix histograms of every pass and the
+ * winners' counts are exchanged through distributed shared memory, so nothing
+ * but the outputs goes to global memory and results are deterministic. The gate's K-split differs from
  * dsa_head_gate's, so gate_w (and the scores after it) may differ from the
  * separate calls' in the last bits; both are held to the same tolerance.
  * hidden, w, q_idx, q_req and q_pos are read before the wait on the preceding

@@ -6,28 +6,34 @@
 // to fourth arrows: [Q, P] scores with candidate validity, the top-k select,
 // the expansion to a [Q, select_k * kpool] token-id row; trap 6).
 //
-// One thread-block cluster of 8 CTAs per query. CTA r of the cluster
+// One thread-block cluster per query: 8 CTAs, or 16 where few queries leave
+// most of the device idle. CTA r of the cluster
 //   1. sums its K-slice of the query's head gate (hidden[q] . w) before the
 //      wait on the preceding kernel (both are step inputs the path never
 //      writes) and pushes the partial into every CTA's shared memory; each CTA
-//      adds the 8 partials in rank order, so all hold the same gate_w[q];
-//   2. scores its share of the pools, 128-pool tiles of TMA-loaded pooled keys
-//      on the tensor cores (D[128 pools x 16 heads] = keys . q_idx^T), one
-//      thread per pool summing g_h * relu(dot_h) in head order; it writes
-//      scores and cand and pushes each pool's radix key into the shared
-//      memory of the cluster's first CTA (the leader);
-//   3. the leader selects: an exact 8-bit MSB radix select of the n_q-th
-//      largest candidate key over the query's pools, with, after two passes,
-//      a one-warp rank of the at most 32 keys that share the answer's top 16
-//      bits; the winners are placed in ascending pool id (warps over
-//      contiguous id ranges, ballot ranks) and expanded to token ids, and the
-//      -1 tail is written.
-// Pushes are distributed-shared-memory stores followed by a release arrive on
-// the receiver's mbarrier, so the only cluster-wide rendezvous is the one that
-// guarantees every CTA has started (its arrive is issued before the gate's
-// loads). The selection is the one dsa_topk_expand makes (ties to the lowest
-// pool id, -0 equal to +0, NaN as -inf), so results are deterministic.
+//      adds the C partials in rank order, so all hold the same gate_w[q];
+//   2. scores its contiguous range of pools, 128-pool tiles of TMA-loaded
+//      pooled keys on the tensor cores (D[128 pools x 16 heads] = keys .
+//      q_idx^T), one thread per pool summing g_h * relu(dot_h) in head order;
+//      it writes scores and cand and keeps each pool's radix key in its own
+//      shared memory;
+//   3. the cluster selects together: an exact 8-bit MSB radix select of the
+//      n_q-th largest candidate key. Each pass every CTA counts the digit over
+//      its own keys and sends the 256 counts to every CTA, so all CTAs add the
+//      same histogram and take the same digit; after two passes, when at most
+//      32 keys share the answer's top 16 bits, those keys are exchanged and
+//      ranked on one warp instead of two more passes;
+//   4. every CTA counts its keys above the answer and equal to it, exchanges
+//      the counts, and writes its winners at their places in ascending pool id
+//      (ties to the lowest ids) with their token ids; the -1 tail is shared out.
+// An exchange is a set of asynchronous distributed-shared-memory stores into
+// slot r of every CTA's buffer, each completing its bytes on that CTA's
+// mbarrier (which expects the C ranks' bytes); two buffers alternate, so a CTA
+// never receives the next exchange into a buffer it is still reading. The selection is the one dsa_topk_expand makes (ties to the
+// lowest pool id, -0 equal to +0, NaN as -inf), so results are deterministic.
 #pragma once
+
+#include <atomic>
 
 #include "common.cuh"
 #include "tc_ptx.cuh"
@@ -41,39 +47,44 @@ constexpr int kIxWarps = kIxThreads / 32;
 constexpr int kIxTile = 128;                                // pools per MMA tile (M)
 constexpr int kIxHeads = DSA_MAX_INDEX_HEADS;               // 16 (N)
 constexpr int kIxCluster = 8;                               // CTAs per query
-constexpr int kIxMaxPools = 32768;                          // keys the leader holds
+constexpr int kIxMaxCluster = 16;                           // with few queries
+constexpr int kIxMaxPools = 32768;
+constexpr int kIxXWords = 260;                              // exchange: 256 counts + 4
+constexpr uint32_t kIxXBytes = 4 * kIxXWords;               // 65 16-byte pieces
 constexpr uint32_t kIxKeyAtom = kIxTile * 128;              // 16 KB: one 64-channel column
 constexpr uint32_t kIxKeyTile = 2 * kIxKeyAtom;             // 32 KB
 constexpr uint32_t kIxQAtom = kIxHeads * 128;               // 2 KB
 constexpr uint32_t kIxOffQ = 2 * kIxKeyTile;                // after the two-stage key ring
-constexpr uint32_t kIxOffKeys = kIxOffQ + 2 * kIxQAtom;     // the query's radix keys (leader)
+constexpr uint32_t kIxOffKeys = kIxOffQ + 2 * kIxQAtom;     // this CTA's radix keys
 
-// Dynamic shared memory: the key ring (whose space also holds the leader's
-// select_k selected ids once its tiles are done), the query rows and P radix
-// keys (used by the leader, sized alike on every CTA).
-inline int indexer_smem_bytes(int P) { return (int)kIxOffKeys + 4 * P + 1024; }
-static_assert(4 * DSA_MAX_SELECT <= 2 * kIxKeyTile, "selected ids fit in the key ring");
+// Dynamic shared memory: the key ring, the query rows and the radix keys of
+// this CTA's pools (whole tiles).
+inline int indexer_smem_bytes(int P, int C) {
+    const int tiles = (P + kIxTile - 1) / kIxTile;
+    return (int)kIxOffKeys + 4 * kIxTile * ((tiles + C - 1) / C) + 1024;
+}
 
 struct IxCtl {
     uint64_t q_bar, load_full[2], mma_done[2], d_empty[2];
     uint64_t gate_bar;                  // the cluster's gate partials have arrived
-    uint64_t keys_bar;                  // the cluster's radix keys have arrived (leader)
+    uint64_t xbar[2];                   // an exchange into buffer i has fully arrived
     uint32_t tmem_base;
-    int hist[2][256];
+    int hloc[256];                      // this CTA's counts of the current digit
     float red[64][kIxHeads];            // gate partials per row-part
-    float gate_in[kIxCluster][kIxHeads];// the cluster's gate partials, by rank
+    float gate_in[kIxMaxCluster][kIxHeads];   // the cluster's gate partials, by rank
     float gate[kIxHeads];               // the query's gate weights
-    int ncand_in[kIxCluster];           // the cluster's candidate counts, by rank (leader)
-    int hist_in[kIxCluster][256];       // the cluster's top-byte histograms, by rank (leader)
+    alignas(16) int xin[2][kIxMaxCluster][kIxXWords];   // exchange buffers: rank c's words
+    alignas(16) int xout[kIxXWords];    // this CTA's words of the current exchange
     int2 warp2[kIxWarps];
     int pick[3];                        // (digit, count above, count in it) of the current pass
     int ncand;                          // this CTA's candidates
     int nsmall;
-    uint32_t small[32];
+    uint32_t small[32];                 // this CTA's keys sharing the answer's top 16 bits
     uint32_t tau;
     int req;
     volatile int abort;
 };
+static_assert(sizeof(IxCtl) <= 46 * 1024, "static shared memory");
 
 // Pools [p_lo, p_hi) of cluster rank r: whole 128-pool tiles, split evenly.
 struct IxRange { int t0, t1, p_lo, p_hi; };
@@ -130,6 +141,16 @@ DSA_DEVINL void mbar_arrive_remote(uint32_t remote) {
 DSA_DEVINL void st_cluster_u32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+// 16 bytes into another CTA's shared memory (shared::cluster address), their
+// arrival completing 16 bytes of the transaction count of the mbarrier at
+// `remote_bar` (in the same CTA as the destination).
+DSA_DEVINL void st_async_v4(uint32_t remote, int4 v, uint32_t remote_bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.s32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+            remote),
+        "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(remote_bar)
+        : "memory");
+}
 DSA_DEVINL void cluster_arrive_relaxed() {
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
@@ -149,8 +170,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     const uint32_t raw = smem_u32(ix_smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = ix_smem_raw + (base - raw);
-    uint32_t *akeys = reinterpret_cast<uint32_t *>(gbase + kIxOffKeys);                 // [P]
-    int32_t *slist = reinterpret_cast<int32_t *>(gbase);   // [SK], in the key ring (leader, at the end)
+    uint32_t *akeys = reinterpret_cast<uint32_t *>(gbase + kIxOffKeys);   // this CTA's pools
     const uint32_t sQ = base + kIxOffQ;
 
     const int C = gridDim.x, r = blockIdx.x, q = blockIdx.y;
@@ -173,7 +193,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
             mbar_init(&ctl->d_empty[i], kIxTile);
         }
         mbar_init(&ctl->gate_bar, C);
-        mbar_init(&ctl->keys_bar, C);
+        mbar_init(&ctl->xbar[0], 1);       // own expect_tx; the other ranks' bytes complete it
+        mbar_init(&ctl->xbar[1], 1);
         ctl->abort = 0;
         ctl->ncand = 0;
         ctl->nsmall = 0;
@@ -183,7 +204,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         tma_load_2d(sQ, &q_map, 0, q * H, &ctl->q_bar);
         tma_load_2d(sQ + kIxQAtom, &q_map, 64, q * H, &ctl->q_bar);
     }
-    for (int i = tid; i < 2 * 256; i += kIxThreads) (&ctl->hist[0][0])[i] = 0;
+    for (int i = tid; i < 256; i += kIxThreads) ctl->hloc[i] = 0;
     // Every CTA of the cluster has started and initialised its barriers once the
     // cluster wait below returns; the arrive goes out now, so the rendezvous
     // overlaps the gate's loads.
@@ -242,9 +263,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     tc::fence_after_sync();
     __syncthreads();
     cluster_wait();
-    // push: thread (c, h) of warps 0-3 writes this CTA's partial of head h into
-    // slot r of CTA c; one thread per receiver then arrives on its barrier
-    if (warp < 4) {
+    // push: thread (c, h) writes this CTA's partial of head h into slot r of
+    // CTA c; one thread per receiver then arrives on its barrier
+    {
         const int c = tid >> 4, h = tid & 15;
         if (c < C) st_cluster_u32(cluster_map(smem_u32(&ctl->gate_in[r][h]), c), __float_as_uint(ctl->gate[h]));
     }
@@ -312,7 +333,6 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         if (!ok) ctl->abort = 1;
     }
 
-    const uint32_t lead_keys = cluster_map(smem_u32(akeys), 0);   // the leader's key array
     int local_cand = 0;
     if (warp < 4) {
         float g[kIxHeads];
@@ -347,208 +367,272 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
                 scores[(size_t)q * P + p] = is_cand ? score : -INFINITY;
                 cand[(size_t)q * P + p] = is_cand ? 1 : 0;
                 const uint32_t k = score_key(score, is_cand);
-                st_cluster_u32(lead_keys + 4u * (uint32_t)p, k);
+                akeys[p - rg.p_lo] = k;
                 local_cand += k != 0u;
             }
             // this CTA's share of the first radix pass: the top bytes of its keys
             const uint32_t dgt = p < P ? (score_key(score, is_cand) >> 24) : 0x100u;
             const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
-            if (dgt != 0x100u && lane == __ffs(peers) - 1) atomicAdd(&ctl->hist[0][dgt], __popc(peers));
+            if (dgt != 0x100u && lane == __ffs(peers) - 1) atomicAdd(&ctl->hloc[dgt], __popc(peers));
         }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) local_cand += __shfl_xor_sync(0xffffffffu, local_cand, off);
     if (lane == 0 && local_cand) atomicAdd(&ctl->ncand, local_cand);
     __syncthreads();
-    // this CTA's histogram and candidate count to the leader, then its release
-    // arrive (after every key this CTA pushed: the CTA barrier orders them before it)
-    st_cluster_u32(cluster_map(smem_u32(&ctl->hist_in[r][tid]), 0), (uint32_t)ctl->hist[0][tid]);
-    __syncthreads();
-    if (tid == 0) {
-        st_cluster_u32(cluster_map(smem_u32(&ctl->ncand_in[r]), 0), (uint32_t)ctl->ncand);
-        asm volatile("fence.acq_rel.cluster;" ::: "memory");
-        mbar_arrive_remote(cluster_map(smem_u32(&ctl->keys_bar), 0));
-    }
 
-    if (r == 0) {
-        // ---- 3. the leader selects over the query's P keys
-        if (tid == 0) {
-            int n = 0;
-            if (mbar_wait_cluster(&ctl->keys_bar, 0)) {
-                for (int c = 0; c < C; ++c) n += ctl->ncand_in[c];
-            } else {
-                ctl->abort = 1;
+    // ---- 3. the cluster selects
+    // Exchange: word t (thread t) and, from thread 0, word 256 go into slot r of
+    // every CTA's buffer xi & 1; returns the buffer once all C slots of this
+    // CTA's copy have arrived. Every CTA makes the same exchanges in the same
+    // order (each decision below is taken on exchanged data alike everywhere).
+    int xi = 0;
+    auto exchange = [&](int v, int extra) -> int {
+        const int bf = xi & 1;
+        ctl->xout[tid] = v;
+        if (tid < kIxXWords - 256) ctl->xout[256 + tid] = tid == 0 ? extra : 0;
+        if (tid == 0) mbar_arrive_expect_tx(&ctl->xbar[bf], (uint32_t)(C - 1) * kIxXBytes);
+        __syncthreads();
+        // thread t sends 16-byte piece t % 65 to rank t / 65; this CTA's own slot
+        // is a plain copy (seen by the CTA after the barrier below)
+        const uint32_t dst0 = smem_u32(&ctl->xin[bf][r][0]), bar0 = smem_u32(&ctl->xbar[bf]);
+        for (int t = tid; t < (int)(kIxXBytes / 16) * C; t += kIxThreads) {
+            const int c = t / (kIxXBytes / 16), u = t - c * (kIxXBytes / 16);
+            const int4 val = reinterpret_cast<const int4 *>(ctl->xout)[u];
+            if (c == r)
+                reinterpret_cast<int4 *>(&ctl->xin[bf][r][0])[u] = val;
+            else
+                st_async_v4(cluster_map(dst0 + 16u * (uint32_t)u, c), val, cluster_map(bar0, c));
+        }
+        if (tid == 0 && !mbar_wait_cluster(&ctl->xbar[bf], (xi >> 1) & 1)) ctl->abort = 1;
+        ++xi;
+        __syncthreads();
+        return bf;
+    };
+    const int nloc = max(0, rg.p_hi - rg.p_lo);
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = 0, nq = 0;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        if (pass > 0) {
+            // this CTA's counts of the digit over its keys that match the prefix
+            ctl->hloc[tid] = 0;
+            __syncthreads();
+            for (int i0 = warp * 32; i0 < nloc; i0 += kIxThreads) {
+                const int i = i0 + lane;
+                const uint32_t k = i < nloc ? akeys[i] : 0u;
+                const bool m = i < nloc && (k & pmask) == prefix;
+                const uint32_t d = m ? (k >> shift) & 0xFFu : 0x100u;
+                const uint32_t peers = __match_any_sync(0xffffffffu, d);
+                if (m && lane == __ffs(peers) - 1) atomicAdd(&ctl->hloc[d], __popc(peers));
             }
+            __syncthreads();
+        }
+        const int bf = exchange(ctl->hloc[tid], pass == 0 ? ctl->ncand : 0);
+        // the cluster's histogram (integer counts: the sum is the same everywhere)
+        int t = 0;
+        for (int c = 0; c < C; ++c) t += ctl->xin[bf][c][tid];
+        ctl->hloc[tid] = t;
+        if (pass == 0 && tid == 0) {
+            int n = 0;
+            for (int c = 0; c < C; ++c) n += ctl->xin[bf][c][256];
             ctl->req = ctl->abort ? 0 : n;
         }
         __syncthreads();
-        const int nq = min(SK, ctl->req);
-
-        uint32_t prefix = 0, pmask = 0;
-        int remaining = nq;
-        if (nq > 0) {
-            // pass 0's histogram: the cluster's top-byte histograms added up
-            {
-                int t = 0;
-                for (int c = 0; c < C; ++c) t += ctl->hist_in[c][tid];
-                __syncthreads();
-                ctl->hist[0][tid] = t;
+        if (pass == 0) {
+            nq = min(SK, ctl->req);
+            remaining = nq;
+            if (nq == 0) break;
+        }
+        if (tid < 32) {
+            // lane l owns bins 255-8l down to 248-8l
+            int cbin[8], sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                cbin[i] = ctl->hloc[255 - 8 * tid - i];
+                sum += cbin[i];
+            }
+            int above = sum;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, above, off);
+                if (tid >= off) above += y;
+            }
+            int run = above - sum;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (run < remaining && remaining <= run + cbin[i]) {
+                    ctl->pick[0] = 255 - 8 * tid - i;
+                    ctl->pick[1] = run;
+                    ctl->pick[2] = cbin[i];
+                }
+                run += cbin[i];
+            }
+        }
+        __syncthreads();
+        remaining -= ctl->pick[1];
+        prefix |= (uint32_t)ctl->pick[0] << shift;
+        pmask |= 0xFFu << shift;
+        if (pass == 1 && ctl->pick[2] <= 32) {
+            // At most 32 keys share the answer's top 16 bits: every CTA sends its
+            // own (at most 32) and all rank the same list on one warp.
+            if (tid == 0) ctl->nsmall = 0;
+            __syncthreads();
+            for (int i0 = warp * 32; i0 < nloc; i0 += kIxThreads) {
+                const int i = i0 + lane;
+                const uint32_t k = i < nloc ? akeys[i] : 0u;
+                const bool m = i < nloc && (k & pmask) == prefix;
+                const uint32_t bal = __ballot_sync(0xffffffffu, m);
+                if (bal) {
+                    int off = 0;
+                    if (lane == 0) off = atomicAdd(&ctl->nsmall, __popc(bal));
+                    off = __shfl_sync(0xffffffffu, off, 0);
+                    if (m) ctl->small[off + __popc(bal & ((1u << lane) - 1u))] = k;
+                }
             }
             __syncthreads();
-#pragma unroll 1
-            for (int pass = 0; pass < 4; ++pass) {
-                const int shift = 24 - 8 * pass, hb = pass & 1;
-                if (pass > 0) {
-                    for (int p = tid; p < P; p += kIxThreads) {
-                        const uint32_t k = akeys[p];
-                        if ((k & pmask) == prefix) atomicAdd(&ctl->hist[hb][(k >> shift) & 0xFF], 1);
-                    }
-                    __syncthreads();
+            const int ns = min(ctl->nsmall, 32);
+            const int bs = exchange(tid < ns ? (int)ctl->small[tid] : 0, ns);
+            if (tid < 32) {
+                // lane l takes the l-th key of the ranks' lists laid end to end
+                uint32_t mine = 0u;
+                int n = 0;
+                for (int c = 0; c < C; ++c) {
+                    const int nc = min(ctl->xin[bs][c][256], 32);
+                    if (tid >= n && tid < n + nc) mine = (uint32_t)ctl->xin[bs][c][tid - n];
+                    n += nc;
                 }
-                if (tid < 32) {
-                    // lane l owns bins 255-8l down to 248-8l
-                    int cbin[8], sum = 0;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        cbin[i] = ctl->hist[hb][255 - 8 * tid - i];
-                        sum += cbin[i];
-                    }
-                    int above = sum;
-#pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const int y = __shfl_up_sync(0xffffffffu, above, off);
-                        if (tid >= off) above += y;
-                    }
-                    int run = above - sum;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        if (run < remaining && remaining <= run + cbin[i]) {
-                            ctl->pick[0] = 255 - 8 * tid - i;
-                            ctl->pick[1] = run;
-                            ctl->pick[2] = cbin[i];
-                        }
-                        run += cbin[i];
-                    }
+                n = min(n, 32);
+                int gt = 0, ge = 0;
+                for (int j = 0; j < n; ++j) {
+                    const uint32_t kj = __shfl_sync(0xffffffffu, mine, j);
+                    gt += kj > mine;
+                    ge += kj >= mine;
                 }
-                __syncthreads();
-                remaining -= ctl->pick[1];
-                prefix |= (uint32_t)ctl->pick[0] << shift;
-                pmask |= 0xFFu << shift;
-                const int in_bin = ctl->pick[2];
-                for (int i = tid; i < 256; i += kIxThreads) ctl->hist[hb ^ 1][i] = 0;
-                __syncthreads();
-                if (pass == 1 && in_bin <= 32) {
-                    // At most 32 keys share the answer's top 16 bits: gather them and
-                    // rank them on one warp instead of two more passes.
-                    for (int base0 = (tid & ~31); base0 < P; base0 += kIxThreads) {
-                        const int p = base0 + lane;
-                        const uint32_t k = p < P ? akeys[p] : 0u;
-                        const bool m = p < P && (k & pmask) == prefix;
-                        const uint32_t bal = __ballot_sync(0xffffffffu, m);
-                        if (bal) {
-                            int off = 0;
-                            if (lane == 0) off = atomicAdd(&ctl->nsmall, __popc(bal));
-                            off = __shfl_sync(0xffffffffu, off, 0);
-                            if (m) ctl->small[off + __popc(bal & ((1u << lane) - 1u))] = k;
-                        }
-                    }
-                    __syncthreads();
-                    if (tid < 32) {
-                        const int n = ctl->nsmall;
-                        const uint32_t mine = tid < n ? ctl->small[tid] : 0u;
-                        int gt = 0, ge = 0;
-                        for (int j = 0; j < n; ++j) {
-                            const uint32_t kj = ctl->small[j];
-                            gt += kj > mine;
-                            ge += kj >= mine;
-                        }
-                        if (tid < n && gt < remaining && remaining <= ge) {
-                            ctl->tau = mine;
-                            ctl->pick[0] = remaining - gt;
-                        }
-                    }
-                    __syncthreads();
-                    prefix = ctl->tau;
-                    remaining = ctl->pick[0];
-                    break;
+                if (tid < n && gt < remaining && remaining <= ge) {
+                    ctl->tau = mine;
+                    ctl->pick[0] = remaining - gt;
                 }
             }
+            __syncthreads();
+            prefix = ctl->tau;
+            remaining = ctl->pick[0];
+            break;
         }
-        const uint32_t tau = prefix;     // the nq-th largest key (when nq > 0)
-        const int req_eq = remaining;    // keys equal to tau to take, lowest ids first
+    }
+    const uint32_t tau = prefix;     // the nq-th largest key (when nq > 0)
+    const int req_eq = remaining;    // keys equal to tau to take, lowest ids first
 
-        // ---- 4. winners in ascending pool id: every key above tau, then the
-        // req_eq lowest-id keys equal to it. Warp w places the keys of a contiguous
-        // range, 32 consecutive keys a step (conflict-free reads, ballot ranks).
-        const int span = (((P + kIxWarps - 1) / kIxWarps) + 31) & ~31;
-        const int wlo = min(P, warp * span), whi = min(P, wlo + span);
+    // ---- 4. winners in ascending pool id: every key above tau, then the req_eq
+    // lowest-id keys equal to it. Warp w of CTA r takes a contiguous range of the
+    // CTA's pools, 32 consecutive keys a step (ballot ranks); the places before it
+    // are the counts of the lower ranks and of the lower warps.
+    const size_t wrow = (size_t)SK * KP;
+    const bool vec = (KP & 3) == 0 && aligned16(pool_idx) && aligned16(token_ids);
+    if (nq > 0) {
+        const int span = (((nloc + kIxWarps - 1) / kIxWarps) + 31) & ~31;
+        const int wlo = min(nloc, warp * span), whi = min(nloc, wlo + span);
         const uint32_t below = (1u << lane) - 1u;
         int wgt = 0, weq = 0;
-        if (nq > 0)
-            for (int p0 = wlo; p0 < whi; p0 += 32) {
-                const int p = p0 + lane;
-                const uint32_t k = p < whi ? akeys[p] : 0u;
-                wgt += __popc(__ballot_sync(0xffffffffu, p < whi && k > tau));
-                weq += __popc(__ballot_sync(0xffffffffu, p < whi && k == tau));
-            }
+        for (int p0 = wlo; p0 < whi; p0 += 32) {
+            const int i = p0 + lane;
+            const uint32_t k = i < whi ? akeys[i] : 0u;
+            wgt += __popc(__ballot_sync(0xffffffffu, i < whi && k > tau));
+            weq += __popc(__ballot_sync(0xffffffffu, i < whi && k == tau));
+        }
         if (lane == 0) ctl->warp2[warp] = make_int2(wgt, weq);
         __syncthreads();
-        int gt_before = 0, eq_before = 0;
-        for (int w2 = 0; w2 < warp; ++w2) {
-            gt_before += ctl->warp2[w2].x;
-            eq_before += ctl->warp2[w2].y;
+        int cgt = 0, ceq = 0, gtw = 0, eqw = 0;
+        for (int w2 = 0; w2 < kIxWarps; ++w2) {
+            const int2 v = ctl->warp2[w2];
+            cgt += v.x;
+            ceq += v.y;
+            if (w2 < warp) { gtw += v.x; eqw += v.y; }
         }
-        if (nq > 0) {
-            int pos = gt_before + min(eq_before, req_eq), eqs = eq_before;
-            for (int p0 = wlo; p0 < whi; p0 += 32) {
-                const int p = p0 + lane;
-                const uint32_t k = p < whi ? akeys[p] : 0u;
-                const bool g = p < whi && k > tau, e = p < whi && k == tau;
-                const uint32_t be = __ballot_sync(0xffffffffu, e);
-                const bool take = g || (e && eqs + __popc(be & below) < req_eq);
-                const uint32_t bt = __ballot_sync(0xffffffffu, take);
-                if (take) slist[pos + __popc(bt & below)] = p;
-                pos += __popc(bt);
-                eqs += __popc(be);
-            }
+        const int bc = exchange(tid == 0 ? cgt : tid == 1 ? ceq : 0, 0);
+        int gtr = 0, eqr = 0;
+        for (int c = 0; c < r; ++c) {
+            gtr += ctl->xin[bc][c][0];
+            eqr += ctl->xin[bc][c][1];
         }
-        __syncthreads();
-        const size_t wrow = (size_t)SK * KP;
-        for (int j = tid; j < SK; j += kIxThreads) top_pools[(size_t)q * SK + j] = j < nq ? slist[j] : -1;
-        // expansion: with kpool a multiple of 4 and 16-byte aligned rows, a
-        // selected pool's ids move as kpool/4 vector loads and stores; otherwise
-        // four scalar gathers in flight per thread before the stores
-        if ((KP & 3) == 0 && aligned16(pool_idx) && aligned16(token_ids)) {
-            const int nv = KP >> 2;                         // 16-byte pieces a pool
-            const int4 *src = reinterpret_cast<const int4 *>(pool_idx + (size_t)b * P * KP);
-            int4 *dst = reinterpret_cast<int4 *>(token_ids + (size_t)q * wrow);
-            for (int e = tid; e < SK * nv; e += kIxThreads) {
-                const int j = e / nv, u = e - j * nv;
-                dst[e] = j < nq ? __ldg(src + (size_t)slist[j] * nv + u) : make_int4(-1, -1, -1, -1);
-            }
-        } else {
-            for (int e0 = 0; e0 < SK * KP; e0 += 4 * kIxThreads) {
-                int32_t v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = e0 + tid + u * kIxThreads;
-                    const int j = e / KP, s = e - j * KP;
-                    v[u] = -1;
-                    if (e < SK * KP && j < nq) v[u] = __ldg(pool_idx + ((size_t)b * P + slist[j]) * KP + s);
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = e0 + tid + u * kIxThreads;
-                    if (e < SK * KP) token_ids[(size_t)q * wrow + e] = v[u];
+        int eqs = eqr + eqw;
+        int pos = gtr + gtw + min(eqs, req_eq);
+        const int32_t *prow = pool_idx + (size_t)b * P * KP;
+        for (int p0 = wlo; p0 < whi; p0 += 32) {
+            const int i = p0 + lane;
+            const uint32_t k = i < whi ? akeys[i] : 0u;
+            const bool g = i < whi && k > tau, e = i < whi && k == tau;
+            const uint32_t be = __ballot_sync(0xffffffffu, e);
+            const bool take = g || (e && eqs + __popc(be & below) < req_eq);
+            const uint32_t bt = __ballot_sync(0xffffffffu, take);
+            if (take) {
+                const int j = pos + __popc(bt & below);
+                const int pid = rg.p_lo + i;
+                top_pools[(size_t)q * SK + j] = pid;
+                if (vec) {
+                    const int4 *src = reinterpret_cast<const int4 *>(prow + (size_t)pid * KP);
+                    int4 *dst = reinterpret_cast<int4 *>(token_ids + (size_t)q * wrow + (size_t)j * KP);
+                    for (int u = 0; u < (KP >> 2); ++u) dst[u] = __ldg(src + u);
+                } else {
+                    for (int u = 0; u < KP; ++u)
+                        token_ids[(size_t)q * wrow + (size_t)j * KP + u] = __ldg(prow + (size_t)pid * KP + u);
                 }
             }
+            pos += __popc(bt);
+            eqs += __popc(be);
         }
+    }
+    // the -1 tail, slots [nq, SK), shared out over the cluster
+    for (int j = nq + r * kIxThreads + tid; j < SK; j += C * kIxThreads) {
+        top_pools[(size_t)q * SK + j] = -1;
+        for (int u = 0; u < KP; ++u) token_ids[(size_t)q * wrow + (size_t)j * KP + u] = -1;
     }
 
     if (tid == 32) (void)mbar_wait(&ctl->q_bar, 0);   // the query rows' copy has landed
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, 32);
+}
+
+// Clusters of 16 CTAs the device holds at once with the largest shared-memory
+// size the kernel takes (asked once per device); 0 when none or unknown.
+inline int indexer_max_clusters16() {
+    static std::atomic<int> known[64];   // count + 1; 0 = not asked
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    const int k = known[dev].load(std::memory_order_relaxed);
+    if (k != 0) return k - 1;
+    const void *f = reinterpret_cast<const void *>(indexer_kernel);
+    const int smem = indexer_smem_bytes(kIxMaxPools, kIxMaxCluster);
+    int n = 0;
+    if (ensure_smem_attr(f, smem) &&
+        cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kIxMaxCluster, 1, 1);
+        cfg.blockDim = dim3(kIxThreads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kIxMaxCluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, indexer_kernel, &cfg) != cudaSuccess) n = 0;
+    }
+    (void)cudaGetLastError();
+    known[dev].store(n + 1, std::memory_order_relaxed);
+    return n;
+}
+
+// CTAs a query: 16 where clusters of 8 would leave most of the device idle (16
+// CTAs a query still fit in one wave), every CTA gets at least two tiles and
+// the device holds all Q clusters of 16 at once; 8 otherwise.
+inline int indexer_cluster_size(int Q, int P) {
+    const int tiles = (P + kIxTile - 1) / kIxTile;
+    if ((long long)Q * kIxMaxCluster > sm_count() || tiles < 2 * kIxMaxCluster) return kIxCluster;
+    return indexer_max_clusters16() >= Q ? kIxMaxCluster : kIxCluster;
 }
 
 inline int indexer_launch(const float *hidden, const float *w, int K, const void *q_idx,
@@ -580,10 +664,10 @@ inline int indexer_launch(const float *hidden, const float *w, int K, const void
     if (!make_map_bf16_2d(&key_map, kbase, krows, kD, kD * 2, 64, kIxTile) ||
         !make_map_bf16_2d(&q_map, q_idx, (uint64_t)Q * H, kD, kD * 2, 64, kIxHeads))
         return DSA_ERR_CUDA;
-    const int smem = indexer_smem_bytes(max_pools);
+    const int C = indexer_cluster_size(Q, max_pools);
+    const int smem = indexer_smem_bytes(max_pools, C);
     if (!ensure_smem_attr(reinterpret_cast<const void *>(indexer_kernel), smem)) return DSA_ERR_CUDA;
-    if (launch_pdl_cluster(indexer_kernel, dim3(kIxCluster, Q), dim3(kIxThreads), smem, stream,
-                           kIxCluster, key_map, q_map, hidden, w, K, H, q_req, q_pos, pool_valid,
+    if (launch_pdl_cluster(indexer_kernel, dim3(C, Q), dim3(kIxThreads), smem, stream, C, key_map, q_map, hidden, w, K, H, q_req, q_pos, pool_valid,
                            first_valid, pool_idx, B, kpool, max_pools, select_k, gate_w, scores,
                            cand, top_pools, token_ids) != cudaSuccess)
         return DSA_ERR_CUDA;

@@ -73,13 +73,16 @@ constexpr uint32_t kOffCtl = kOffP + 2 * kStageP;
 constexpr uint32_t kTmemCols = 512;
 // MMAs are issued by one thread in each of warps 0-3: a single issuing thread
 // starts about one tcgen05.mma every 128 cycles whatever the tile, and issuers
-// in different warps proceed in parallel. Warps 0 and 1 issue the two K-halves
-// of S into separate accumulators (added by the softmax); each of the four
-// issues the PV of one 128-latent block of O^T.
+// in different warps proceed in parallel. Each of the four issues one K-quarter
+// of S into its own accumulator (the softmax adds the four) and the PV of one
+// 128-latent block of O^T. The four S parts fill the columns O^T leaves, so S
+// has one buffer: S(c+1) waits only for the softmax to have read S(c).
 constexpr int kIssuers = 4;
-constexpr int kSParts = 2;
-constexpr uint32_t kSCol = 256;                     // S buffers: [256, 256 + 2 * kSParts * chunk)
-static_assert(kSCol + 2 * kSParts * kTcChunk <= kTmemCols, "tensor memory columns");
+constexpr int kSParts = 4;
+constexpr int kSBufs = 1;
+constexpr uint32_t kSCol = 256;                     // S: [256, 256 + kSBufs * kSParts * chunk)
+static_assert(kSCol + kSBufs * kSParts * kTcChunk <= kTmemCols, "tensor memory columns");
+static_assert(kSParts <= kIssuers && kSParts % 2 == 0, "S parts: one issuer each, read in pairs");
 constexpr float kLazyRescale = 8.0f;                // log2 units
 // Splits merged inside a cluster: up to 8 (the portable size) or, where the
 // device fits them, up to 16 (non-portable sizes are allowed on the kernel).
@@ -313,8 +316,8 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
 
     if (warp < kIssuers) {
         // ------------------------------------------------------------------ MMA issuers
-        // Lane 0 of warp w issues the PV of latent block w and, for w < 2, the
-        // K-half w of every S.
+        // Lane 0 of warp w issues the PV of latent block w and the K-quarter w of
+        // every S.
         if (lane == 0 && nch > 0) {
             const int w = warp;
             const bool s_issuer = w < kSParts;
@@ -341,17 +344,17 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
                 tc::mma_commit(&ctl->p_empty[pb]);
                 tc::mma_commit(&ctl->o_done);
             };
-            // S(c), K-half w = Q K^T over latent [256w, 256w + 256) of chunk c's 48
-            // tokens, into S buffer c & 1, part w.
+            // S(c), K-quarter w = Q K^T over latent [128w, 128w + 128) of chunk c's
+            // 48 tokens, into part w of the S buffer.
             auto issue_s = [&](int c) {
-                const int slot = c % kTcSlots, sb = c & 1;
+                const int slot = c % kTcSlots, sb = c % kSBufs;
                 tc::fence_after_sync();
                 tc::fence_proxy_async_smem();     // the slot was written by cp.async
                 const uint32_t d = tmem + kSCol + (uint32_t)((sb * kSParts + w) * kTcChunk);
-                constexpr int kHalf = kL / 16 / kSParts;
+                constexpr int kPart = kL / 16 / kSParts;
 #pragma unroll
-                for (int k2 = 0; k2 < kHalf; ++k2) {
-                    const int kk = w * kHalf + k2;
+                for (int k2 = 0; k2 < kPart; ++k2) {
+                    const int kk = w * kPart + k2;
                     const uint32_t qo = (kk >> 2) * 8192 + (kk & 3) * 32;
                     const uint32_t ko = (kk >> 2) * kAtomKV + slot * kSlotRows + (kk & 3) * 32;
                     tc::mma_bf16_ss(d, tc::desc_sw128(sQ + qo, 16, 1024),
@@ -373,7 +376,8 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
                 }
                 if (s_issuer && ns < nch) {
                     const bool ready = mbar_test(&ctl->kv_full[ns % kTcSlots], (ns / kTcSlots) & 1) &&
-                                       (ns < 2 || mbar_test(&ctl->s_empty[ns & 1], ((ns >> 1) - 1) & 1));
+                                       (ns < kSBufs ||
+                                        mbar_test(&ctl->s_empty[ns % kSBufs], ((ns / kSBufs) - 1) & 1));
                     if (ready) {
                         issue_s(ns++);
                         t_last = clock64();
@@ -537,20 +541,31 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
         float m_used = -INFINITY, l = 0.f;
         bool failed = false;
         for (int c = 0; c < nch; ++c) {
-            const int slot = c % kTcSlots, sb = c & 1;
+            const int slot = c % kTcSlots, sb = c & 1, sbuf = c % kSBufs;
             bool bad = !tc_wait(ctl, &ctl->kv_full[slot], (c / kTcSlots) & 1);
-            bad = bad || !tc_wait(ctl, &ctl->s_full[sb], (c >> 1) & 1);
+            bad = bad || !tc_wait(ctl, &ctl->s_full[sbuf], (c / kSBufs) & 1);
             tc::fence_after_sync();
-            // 48 columns of each S part: this thread's 24 tokens par + 2i, i < 24
-            uint32_t r[24], r2[24];
-            const uint32_t sc0 = tl + kSCol + (uint32_t)(sb * kSParts * kTcChunk);
-            tc::tmem_ld16x64b_x16(sc0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-            tc::tmem_ld16x64b_x8(sc0 + 32, *reinterpret_cast<uint32_t(*)[8]>(&r[16]));
-            tc::tmem_ld16x64b_x16(sc0 + kTcChunk, *reinterpret_cast<uint32_t(*)[16]>(&r2[0]));
-            tc::tmem_ld16x64b_x8(sc0 + kTcChunk + 32, *reinterpret_cast<uint32_t(*)[8]>(&r2[16]));
-            tc::tmem_wait_ld();
+            // 48 columns of each S part: this thread's 24 tokens par + 2i, i < 24;
+            // the parts are read two at a time and summed pairwise, (p0+p1)+(p2+p3)
+            float sacc[24];
+            const uint32_t sc0 = tl + kSCol + (uint32_t)(sbuf * kSParts * kTcChunk);
+#pragma unroll
+            for (int pp = 0; pp < kSParts; pp += 2) {
+                uint32_t r[24], r2[24];
+                const uint32_t a0 = sc0 + (uint32_t)(pp * kTcChunk);
+                tc::tmem_ld16x64b_x16(a0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                tc::tmem_ld16x64b_x8(a0 + 32, *reinterpret_cast<uint32_t(*)[8]>(&r[16]));
+                tc::tmem_ld16x64b_x16(a0 + kTcChunk, *reinterpret_cast<uint32_t(*)[16]>(&r2[0]));
+                tc::tmem_ld16x64b_x8(a0 + kTcChunk + 32, *reinterpret_cast<uint32_t(*)[8]>(&r2[16]));
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 24; ++i) {
+                    const float t2 = __uint_as_float(r[i]) + __uint_as_float(r2[i]);
+                    sacc[i] = pp == 0 ? t2 : sacc[i] + t2;
+                }
+            }
             tc::fence_before_sync();
-            mbar_arrive(&ctl->s_empty[sb]);
+            mbar_arrive(&ctl->s_empty[sbuf]);
 
             // validity of the chunk's 48 rows (12 per gather warp), then bit 2i: token par + 2i
             const uint64_t vm48 = (uint64_t)ctl->vmask[slot][0] | ((uint64_t)ctl->vmask[slot][1] << 12) |
@@ -560,8 +575,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
             float mx = -INFINITY;
 #pragma unroll
             for (int i = 0; i < 24; ++i) {
-                z[i] = ((vmp >> (2 * i)) & 1) ? (__uint_as_float(r[i]) + __uint_as_float(r2[i])) * scale_log2
-                                              : -INFINITY;
+                z[i] = ((vmp >> (2 * i)) & 1) ? sacc[i] * scale_log2 : -INFINITY;
                 mx = fmaxf(mx, z[i]);
             }
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
