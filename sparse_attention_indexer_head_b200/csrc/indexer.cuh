@@ -54,18 +54,23 @@ constexpr uint32_t kIxXBytes = 4 * kIxXWords;               // 65 16-byte pieces
 constexpr uint32_t kIxKeyAtom = kIxTile * 128;              // 16 KB: one 64-channel column
 constexpr uint32_t kIxKeyTile = 2 * kIxKeyAtom;             // 32 KB
 constexpr uint32_t kIxQAtom = kIxHeads * 128;               // 2 KB
-constexpr uint32_t kIxOffQ = 2 * kIxKeyTile;                // after the two-stage key ring
-constexpr uint32_t kIxOffKeys = kIxOffQ + 2 * kIxQAtom;     // this CTA's radix keys
+constexpr int kIxStages = 5;                                // deepest key ring (tiles in flight)
+constexpr uint32_t kIxTmemCols = 128;                       // up to kIxStages D[128 x 16]
+static_assert(kIxHeads * kIxStages <= (int)kIxTmemCols, "tensor memory columns");
+// Dynamic shared memory of a ring of ns stages: the ring, the query rows, the
+// radix keys of this CTA's pools (whole tiles).
+__host__ __device__ inline uint32_t ix_off_q(int ns) { return (uint32_t)ns * kIxKeyTile; }
+__host__ __device__ inline uint32_t ix_off_keys(int ns) { return ix_off_q(ns) + 2 * kIxQAtom; }
 
 // Dynamic shared memory: the key ring, the query rows and the radix keys of
 // this CTA's pools (whole tiles).
-inline int indexer_smem_bytes(int P, int C) {
+inline int indexer_smem_bytes(int P, int C, int ns) {
     const int tiles = (P + kIxTile - 1) / kIxTile;
-    return (int)kIxOffKeys + 4 * kIxTile * ((tiles + C - 1) / C) + 1024;
+    return (int)ix_off_keys(ns) + 5 * kIxTile * ((tiles + C - 1) / C) + 1024;   // keys, valid bytes
 }
 
 struct IxCtl {
-    uint64_t q_bar, load_full[2], mma_done[2], d_empty[2];
+    uint64_t q_bar, load_full[kIxStages], mma_done[kIxStages], d_empty[kIxStages];
     uint64_t gate_bar;                  // the cluster's gate partials have arrived
     uint64_t xbar[2];                   // an exchange into buffer i has fully arrived
     uint32_t tmem_base;
@@ -82,6 +87,8 @@ struct IxCtl {
     uint32_t small[32];                 // this CTA's keys sharing the answer's top 16 bits
     uint32_t tau;
     int req;
+    int gt16;                           // this CTA's keys above the answer's top 16 bits
+    int rank_gt, rank_eq;               // keys above / equal to tau on the lower ranks
     volatile int abort;
 };
 static_assert(sizeof(IxCtl) <= 46 * 1024, "static shared memory");
@@ -144,6 +151,11 @@ DSA_DEVINL void st_cluster_u32(uint32_t addr, uint32_t v) {
 // 16 bytes into another CTA's shared memory (shared::cluster address), their
 // arrival completing 16 bytes of the transaction count of the mbarrier at
 // `remote_bar` (in the same CTA as the destination).
+DSA_DEVINL void st_async_b32(uint32_t remote, uint32_t v, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote),
+                 "r"(v), "r"(remote_bar)
+                 : "memory");
+}
 DSA_DEVINL void st_async_v4(uint32_t remote, int4 v, uint32_t remote_bar) {
     asm volatile(
         "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.s32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
@@ -163,36 +175,40 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
                const uint8_t *__restrict__ pool_valid, const int32_t *__restrict__ first_valid,
                const int32_t *__restrict__ pool_idx, int B, int KP, int P, int SK,
                float *__restrict__ gate_w, float *__restrict__ scores, uint8_t *__restrict__ cand,
-               int32_t *__restrict__ top_pools, int32_t *__restrict__ token_ids) {
+               int32_t *__restrict__ top_pools, int32_t *__restrict__ token_ids, int NS) {
     extern __shared__ uint8_t ix_smem_raw[];
     __shared__ IxCtl ctl_s;
     IxCtl *ctl = &ctl_s;
     const uint32_t raw = smem_u32(ix_smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = ix_smem_raw + (base - raw);
-    uint32_t *akeys = reinterpret_cast<uint32_t *>(gbase + kIxOffKeys);   // this CTA's pools
-    const uint32_t sQ = base + kIxOffQ;
+    uint32_t *akeys = reinterpret_cast<uint32_t *>(gbase + ix_off_keys(NS));   // this CTA's pools
+    uint8_t *svalid;                     // their pool_valid bytes (after the keys)
+    const uint32_t sQ = base + ix_off_q(NS);
 
     const int C = gridDim.x, r = blockIdx.x, q = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const IxRange rg = ix_range(r, C, P);
     const int ntile = rg.t1 - rg.t0;
+    svalid = reinterpret_cast<uint8_t *>(akeys + (size_t)kIxTile * ((((P + kIxTile - 1) / kIxTile) + C - 1) / C));
     // the query's request and position are step inputs: their loads go out first
     const int b = q_req[q];
     const int qp = q_pos[q];
 
     if (warp == 0) {
-        tc::tmem_alloc(&ctl->tmem_base, 32);
+        tc::tmem_alloc(&ctl->tmem_base, kIxTmemCols);
         tc::tmem_relinquish();
     }
     if (tid == 32) {
         mbar_init(&ctl->q_bar, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kIxStages; ++i) {
             mbar_init(&ctl->load_full[i], 1);
             mbar_init(&ctl->mma_done[i], 1);
             mbar_init(&ctl->d_empty[i], kIxTile);
         }
-        mbar_init(&ctl->gate_bar, C);
+        mbar_init(&ctl->gate_bar, 1);
+        // the other ranks' partials arrive as asynchronous stores counted in bytes
+        mbar_arrive_expect_tx(&ctl->gate_bar, (uint32_t)(C - 1) * kIxHeads * 4);
         mbar_init(&ctl->xbar[0], 1);       // own expect_tx; the other ranks' bytes complete it
         mbar_init(&ctl->xbar[1], 1);
         ctl->abort = 0;
@@ -263,36 +279,60 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     tc::fence_after_sync();
     __syncthreads();
     cluster_wait();
-    // push: thread (c, h) writes this CTA's partial of head h into slot r of
-    // CTA c; one thread per receiver then arrives on its barrier
+    // push: thread (c, h) stores this CTA's partial of head h into slot r of CTA
+    // c, completing 4 bytes on that CTA's barrier (its own slot: a plain store)
     {
         const int c = tid >> 4, h = tid & 15;
-        if (c < C) st_cluster_u32(cluster_map(smem_u32(&ctl->gate_in[r][h]), c), __float_as_uint(ctl->gate[h]));
+        const uint32_t v = __float_as_uint(ctl->gate[h]);
+        if (c == r)
+            ctl->gate_in[r][h] = ctl->gate[h];
+        else if (c < C)
+            st_async_b32(cluster_map(smem_u32(&ctl->gate_in[r][h]), c), v,
+                         cluster_map(smem_u32(&ctl->gate_bar), c));
     }
     __syncthreads();
-    if (tid < C) {
-        asm volatile("fence.acq_rel.cluster;" ::: "memory");
-        mbar_arrive_remote(cluster_map(smem_u32(&ctl->gate_bar), tid));
-    }
 
     pdl_wait();                                   // pooled keys and flags come from compress
     pdl_launch_dependents();
 
-    // ---- 2. tiles: two issuing threads load keys and issue the MMAs, warps 0-3 drain
+    // ---- 2. tiles: a producer thread loads keys into an NS-deep ring, two
+    // issuing threads issue the MMAs (tile i into stage and accumulator i % NS),
+    // warps 0-3 drain the accumulators
     auto load = [&](int i) {
-        const int s = i & 1;
+        const int s = i % NS;
         mbar_arrive_expect_tx(&ctl->load_full[s], kIxKeyTile);
         const int row = b * P + (rg.t0 + i) * kIxTile;
         const uint32_t dst = base + s * kIxKeyTile;
         tma_load_2d(dst, &key_map, 0, row, &ctl->load_full[s]);
         tma_load_2d(dst + kIxKeyAtom, &key_map, 64, row, &ctl->load_full[s]);
     };
-    // tiles i = 0, 2, 4 ... go through stage 0 and the issuer in warp 4, tiles
-    // 1, 3, 5 ... through stage 1 and the issuer in warp 5 (a single thread
-    // starts about one MMA per 128 cycles; two in separate warps run in parallel)
+    // tiles i = 0, 2, 4 ... go to the issuer in warp 4, tiles 1, 3, 5 ... to the
+    // issuer in warp 5 (a single thread starts about one MMA per 128 cycles; two
+    // in separate warps run in parallel)
     const bool issuer = (tid == 128 || tid == 160) && req_ok;
+    const bool producer = tid == 192 && req_ok;
     const int my_s = (tid - 128) >> 5;
-    if (issuer && my_s < ntile) load(my_s);
+    if (producer)
+        for (int i = 0; i < min(ntile, NS); ++i) load(i);
+    // this CTA's pool_valid bytes, all loads in flight at once (seen by the
+    // epilogue after the barrier below)
+    if (req_ok) {
+        const uint8_t *vsrc = pool_valid + (size_t)b * P + rg.p_lo;
+        const int nv = max(0, rg.p_hi - rg.p_lo);
+        for (int i0 = 0; i0 < nv; i0 += 4 * kIxThreads) {
+            uint8_t v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * kIxThreads + tid;
+                v[u] = i < nv ? __ldg(vsrc + i) : (uint8_t)0;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * kIxThreads + tid;
+                if (i < nv) svalid[i] = v[u];
+            }
+        }
+    }
     // the cluster's gate partials, added in rank order
     if (tid < kIxHeads) {
         float g = 0.f;
@@ -310,9 +350,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         bool ok = my_s >= ntile || ix_wait(ctl, &ctl->q_bar, 0);
         constexpr uint32_t idesc = tc::idesc_bf16(kIxTile, kIxHeads, false, false);
         for (int i = my_s; ok && i < ntile; i += 2) {
-            const int s = i & 1;
-            ok = ix_wait(ctl, &ctl->load_full[s], (i >> 1) & 1);
-            if (ok && i >= 2) ok = ix_wait(ctl, &ctl->d_empty[s], ((i >> 1) - 1) & 1);
+            const int s = i % NS, ph = (i / NS) & 1;
+            ok = ix_wait(ctl, &ctl->load_full[s], ph);
+            if (ok && i >= NS) ok = ix_wait(ctl, &ctl->d_empty[s], ph ^ 1);
             if (!ok) break;
             tc::fence_after_sync();
             const uint32_t sK = base + s * kIxKeyTile;
@@ -320,15 +360,19 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
             for (int kk = 0; kk < kD / 16; ++kk) {
                 const uint32_t off_k = (kk >> 2) * kIxKeyAtom + (kk & 3) * 32;
                 const uint32_t off_q = (kk >> 2) * kIxQAtom + (kk & 3) * 32;
-                tc::mma_bf16_ss(tmem + 16 * s, tc::desc_sw128(sK + off_k, 16, 1024),
+                tc::mma_bf16_ss(tmem + kIxHeads * s, tc::desc_sw128(sK + off_k, 16, 1024),
                                 tc::desc_sw128(sQ + off_q, 16, 1024), idesc, kk > 0 ? 1u : 0u);
             }
             tc::mma_commit(&ctl->mma_done[s]);
-            if (i + 2 < ntile) {
-                // the stage is free once this tile's MMAs have read it
-                ok = ix_wait(ctl, &ctl->mma_done[s], (i >> 1) & 1);
-                if (ok) load(i + 2);
-            }
+        }
+        if (!ok) ctl->abort = 1;
+    } else if (producer) {
+        // tile i reuses stage i % NS once the MMAs of tile i - NS have read it
+        bool ok = true;
+        for (int i = NS; ok && i < ntile; ++i) {
+            const int s = i % NS;
+            ok = ix_wait(ctl, &ctl->mma_done[s], ((i / NS) - 1) & 1);
+            if (ok) load(i);
         }
         if (!ok) ctl->abort = 1;
     }
@@ -340,19 +384,19 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         for (int h = 0; h < kIxHeads; ++h) g[h] = ctl->gate[h];
         const long long f = req_ok ? (long long)first_valid[b] : 0;
         for (int i = 0; i < ntile; ++i) {
-            const int s = i & 1;
+            const int s = i % NS;
             const int p = (rg.t0 + i) * kIxTile + tid;
             bool is_cand = false;
             if (req_ok && p < P) {
                 const long long last = f + (long long)p * KP + KP - 1;
-                is_cand = pool_valid[(size_t)b * P + p] != 0 && last <= (long long)qp;
+                is_cand = svalid[p - rg.p_lo] != 0 && last <= (long long)qp;
             }
             float score = -INFINITY;
-            const bool ok = req_ok && __all_sync(0xffffffffu, ix_wait(ctl, &ctl->mma_done[s], (i >> 1) & 1));
+            const bool ok = req_ok && __all_sync(0xffffffffu, ix_wait(ctl, &ctl->mma_done[s], (i / NS) & 1));
             if (ok) {
                 tc::fence_after_sync();
                 uint32_t d[kIxHeads];
-                tc::tmem_ld16(tmem + 16 * s + ((uint32_t)(32 * warp) << 16), d);
+                tc::tmem_ld16(tmem + kIxHeads * s + ((uint32_t)(32 * warp) << 16), d);
                 tc::tmem_wait_ld();
                 tc::fence_before_sync();
                 mbar_arrive(&ctl->d_empty[s]);
@@ -370,10 +414,6 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
                 akeys[p - rg.p_lo] = k;
                 local_cand += k != 0u;
             }
-            // this CTA's share of the first radix pass: the top bytes of its keys
-            const uint32_t dgt = p < P ? (score_key(score, is_cand) >> 24) : 0x100u;
-            const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
-            if (dgt != 0x100u && lane == __ffs(peers) - 1) atomicAdd(&ctl->hloc[dgt], __popc(peers));
         }
     }
 #pragma unroll
@@ -382,15 +422,15 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     __syncthreads();
 
     // ---- 3. the cluster selects
-    // Exchange: word t (thread t) and, from thread 0, word 256 go into slot r of
+    // Exchange: word t (thread t) and words 256, 257 go into slot r of
     // every CTA's buffer xi & 1; returns the buffer once all C slots of this
     // CTA's copy have arrived. Every CTA makes the same exchanges in the same
     // order (each decision below is taken on exchanged data alike everywhere).
     int xi = 0;
-    auto exchange = [&](int v, int extra) -> int {
+    auto exchange = [&](int v, int extra, int extra2) -> int {
         const int bf = xi & 1;
         ctl->xout[tid] = v;
-        if (tid < kIxXWords - 256) ctl->xout[256 + tid] = tid == 0 ? extra : 0;
+        if (tid < kIxXWords - 256) ctl->xout[256 + tid] = tid == 0 ? extra : tid == 1 ? extra2 : 0;
         if (tid == 0) mbar_arrive_expect_tx(&ctl->xbar[bf], (uint32_t)(C - 1) * kIxXBytes);
         __syncthreads();
         // thread t sends 16-byte piece t % 65 to rank t / 65; this CTA's own slot
@@ -412,10 +452,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     const int nloc = max(0, rg.p_hi - rg.p_lo);
     uint32_t prefix = 0, pmask = 0;
     int remaining = 0, nq = 0;
+    bool counts_known = false;           // the lower ranks' counts came with the small list
 #pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
-        if (pass > 0) {
+        {
             // this CTA's counts of the digit over its keys that match the prefix
             ctl->hloc[tid] = 0;
             __syncthreads();
@@ -429,7 +470,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
             }
             __syncthreads();
         }
-        const int bf = exchange(ctl->hloc[tid], pass == 0 ? ctl->ncand : 0);
+        const int bf = exchange(ctl->hloc[tid], pass == 0 ? ctl->ncand : 0, 0);
         // the cluster's histogram (integer counts: the sum is the same everywhere)
         int t = 0;
         for (int c = 0; c < C; ++c) t += ctl->xin[bf][c][tid];
@@ -476,13 +517,20 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
         pmask |= 0xFFu << shift;
         if (pass == 1 && ctl->pick[2] <= 32) {
             // At most 32 keys share the answer's top 16 bits: every CTA sends its
-            // own (at most 32) and all rank the same list on one warp.
-            if (tid == 0) ctl->nsmall = 0;
+            // own (at most 32) with its count of keys above those 16 bits, and all
+            // rank the same list on one warp; the lists and counts also give every
+            // rank's keys above and equal to the answer, so no further exchange.
+            if (tid == 0) {
+                ctl->nsmall = 0;
+                ctl->gt16 = 0;
+            }
             __syncthreads();
+            int above16 = 0;
             for (int i0 = warp * 32; i0 < nloc; i0 += kIxThreads) {
                 const int i = i0 + lane;
                 const uint32_t k = i < nloc ? akeys[i] : 0u;
                 const bool m = i < nloc && (k & pmask) == prefix;
+                above16 += __popc(__ballot_sync(0xffffffffu, i < nloc && (k & pmask) > prefix));
                 const uint32_t bal = __ballot_sync(0xffffffffu, m);
                 if (bal) {
                     int off = 0;
@@ -491,9 +539,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
                     if (m) ctl->small[off + __popc(bal & ((1u << lane) - 1u))] = k;
                 }
             }
+            if (lane == 0 && above16) atomicAdd(&ctl->gt16, above16);
             __syncthreads();
             const int ns = min(ctl->nsmall, 32);
-            const int bs = exchange(tid < ns ? (int)ctl->small[tid] : 0, ns);
+            const int bs = exchange(tid < ns ? (int)ctl->small[tid] : 0, ns, ctl->gt16);
             if (tid < 32) {
                 // lane l takes the l-th key of the ranks' lists laid end to end
                 uint32_t mine = 0u;
@@ -518,6 +567,22 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
             __syncthreads();
             prefix = ctl->tau;
             remaining = ctl->pick[0];
+            if (tid == 0) {
+                int g = 0, e = 0;
+                for (int c = 0; c < r; ++c) {
+                    const int nc = min(ctl->xin[bs][c][256], 32);
+                    g += ctl->xin[bs][c][257];
+                    for (int j = 0; j < nc; ++j) {
+                        const uint32_t kj = (uint32_t)ctl->xin[bs][c][j];
+                        g += kj > prefix;
+                        e += kj == prefix;
+                    }
+                }
+                ctl->rank_gt = g;
+                ctl->rank_eq = e;
+            }
+            __syncthreads();
+            counts_known = true;
             break;
         }
     }
@@ -527,7 +592,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     // ---- 4. winners in ascending pool id: every key above tau, then the req_eq
     // lowest-id keys equal to it. Warp w of CTA r takes a contiguous range of the
     // CTA's pools, 32 consecutive keys a step (ballot ranks); the places before it
-    // are the counts of the lower ranks and of the lower warps.
+    // are the counts of the lower ranks and of the lower warps. The CTA's winners
+    // go to a list in the idle key ring, then their token ids are gathered with
+    // every row's loads in flight at once.
     const size_t wrow = (size_t)SK * KP;
     const bool vec = (KP & 3) == 0 && aligned16(pool_idx) && aligned16(token_ids);
     if (nq > 0) {
@@ -550,14 +617,22 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
             ceq += v.y;
             if (w2 < warp) { gtw += v.x; eqw += v.y; }
         }
-        const int bc = exchange(tid == 0 ? cgt : tid == 1 ? ceq : 0, 0);
         int gtr = 0, eqr = 0;
-        for (int c = 0; c < r; ++c) {
-            gtr += ctl->xin[bc][c][0];
-            eqr += ctl->xin[bc][c][1];
+        if (counts_known) {
+            gtr = ctl->rank_gt;
+            eqr = ctl->rank_eq;
+        } else {
+            const int bc = exchange(tid == 0 ? cgt : tid == 1 ? ceq : 0, 0, 0);
+            for (int c = 0; c < r; ++c) {
+                gtr += ctl->xin[bc][c][0];
+                eqr += ctl->xin[bc][c][1];
+            }
         }
         int eqs = eqr + eqw;
         int pos = gtr + gtw + min(eqs, req_eq);
+        const int c_start = gtr + min(eqr, req_eq);                 // this CTA's places
+        const int c_end = gtr + cgt + min(eqr + ceq, req_eq);
+        int32_t *tlist = reinterpret_cast<int32_t *>(gbase);        // at most SK ids
         const int32_t *prow = pool_idx + (size_t)b * P * KP;
         for (int p0 = wlo; p0 < whi; p0 += 32) {
             const int i = p0 + lane;
@@ -570,17 +645,27 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
                 const int j = pos + __popc(bt & below);
                 const int pid = rg.p_lo + i;
                 top_pools[(size_t)q * SK + j] = pid;
-                if (vec) {
-                    const int4 *src = reinterpret_cast<const int4 *>(prow + (size_t)pid * KP);
-                    int4 *dst = reinterpret_cast<int4 *>(token_ids + (size_t)q * wrow + (size_t)j * KP);
-                    for (int u = 0; u < (KP >> 2); ++u) dst[u] = __ldg(src + u);
-                } else {
-                    for (int u = 0; u < KP; ++u)
-                        token_ids[(size_t)q * wrow + (size_t)j * KP + u] = __ldg(prow + (size_t)pid * KP + u);
-                }
+                tlist[j - c_start] = pid;
             }
             pos += __popc(bt);
             eqs += __popc(be);
+        }
+        __syncthreads();
+        const int nt = c_end - c_start;
+        if (vec) {
+            const int nv = KP >> 2;                         // 16-byte pieces a pool
+            const int4 *src = reinterpret_cast<const int4 *>(prow);
+            int4 *dst = reinterpret_cast<int4 *>(token_ids + (size_t)q * wrow) + (size_t)c_start * nv;
+            for (int e = tid; e < nt * nv; e += kIxThreads) {
+                const int jj = e / nv, u = e - jj * nv;
+                dst[e] = __ldg(src + (size_t)tlist[jj] * nv + u);
+            }
+        } else {
+            int32_t *dst = token_ids + (size_t)q * wrow + (size_t)c_start * KP;
+            for (int e = tid; e < nt * KP; e += kIxThreads) {
+                const int jj = e / KP, u = e - jj * KP;
+                dst[e] = __ldg(prow + (size_t)tlist[jj] * KP + u);
+            }
         }
     }
     // the -1 tail, slots [nq, SK), shared out over the cluster
@@ -592,7 +677,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
     if (tid == 32) (void)mbar_wait(&ctl->q_bar, 0);   // the query rows' copy has landed
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, 32);
+    if (warp == 0) tc::tmem_dealloc(tmem, kIxTmemCols);
 }
 
 // Clusters of 16 CTAs the device holds at once with the largest shared-memory
@@ -604,7 +689,7 @@ inline int indexer_max_clusters16() {
     const int k = known[dev].load(std::memory_order_relaxed);
     if (k != 0) return k - 1;
     const void *f = reinterpret_cast<const void *>(indexer_kernel);
-    const int smem = indexer_smem_bytes(kIxMaxPools, kIxMaxCluster);
+    const int smem = indexer_smem_bytes(kIxMaxPools, kIxMaxCluster, kIxStages);
     int n = 0;
     if (ensure_smem_attr(f, smem) &&
         cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
@@ -665,11 +750,22 @@ inline int indexer_launch(const float *hidden, const float *w, int K, const void
         !make_map_bf16_2d(&q_map, q_idx, (uint64_t)Q * H, kD, kD * 2, 64, kIxHeads))
         return DSA_ERR_CUDA;
     const int C = indexer_cluster_size(Q, max_pools);
-    const int smem = indexer_smem_bytes(max_pools, C);
+    // ring depth: deep where the clusters fill at most one wave (each CTA then
+    // streams many tiles), two stages otherwise, so two CTAs share an SM
+    const int tpc = ceil_div(ceil_div(max_pools, kIxTile), C);
+    int NS = (long long)Q * C <= sm_count() ? std::max(2, std::min(kIxStages, tpc)) : 2;
+    // as deep as the block's shared-memory limit allows
+    cudaFuncAttributes fa;
+    int dev = 0, optin = 0;
+    if (cudaFuncGetAttributes(&fa, indexer_kernel) != cudaSuccess || cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    while (NS > 2 && (long long)fa.sharedSizeBytes + indexer_smem_bytes(max_pools, C, NS) > optin) --NS;
+    const int smem = indexer_smem_bytes(max_pools, C, NS);
     if (!ensure_smem_attr(reinterpret_cast<const void *>(indexer_kernel), smem)) return DSA_ERR_CUDA;
     if (launch_pdl_cluster(indexer_kernel, dim3(C, Q), dim3(kIxThreads), smem, stream, C, key_map, q_map, hidden, w, K, H, q_req, q_pos, pool_valid,
                            first_valid, pool_idx, B, kpool, max_pools, select_k, gate_w, scores,
-                           cand, top_pools, token_ids) != cudaSuccess)
+                           cand, top_pools, token_ids, NS) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
 }

@@ -156,3 +156,40 @@ def test_direct_call_odd_gate_shape(B):
     np.testing.assert_array_equal(top.cpu().numpy(), rt)
     np.testing.assert_array_equal(ids.cpu().numpy(), ri)
     device_status_clean(B)
+
+
+@pytest.mark.parametrize("Q", [4, 10])
+def test_direct_call_largest_pool_count(B, Q):
+    """32768 pools a request (the largest the fused call takes): 4 queries run as
+    clusters of 16 CTAs with a deep key ring, 10 as clusters of 8 whose ring the
+    shared-memory limit bounds; every output against the oracle stages."""
+    rng = np.random.default_rng(Q)
+    H, K, kp, P, SK, Bn = 16, 4096, 4, 32768, 512, Q
+    hidden = rng.standard_normal((Q, K), dtype=np.float32)
+    w = (rng.standard_normal((K, H)) / 64).astype(np.float32)
+    q_idx = W.f32_to_bf16_bits(rng.standard_normal((Q, H, 128)).astype(np.float32))
+    keys = W.f32_to_bf16_bits(rng.standard_normal((Bn, P, 128)).astype(np.float32))
+    pv = (rng.random((Bn, P)) < 0.95).astype(np.uint8)
+    fv = rng.integers(0, 4, Bn).astype(np.int32)
+    pidx = (np.arange(Bn * P * kp, dtype=np.int64).reshape(Bn, P, kp) % (1 << 30)).astype(np.int32)
+    q_req = np.arange(Q, dtype=np.int32)
+    q_pos = (fv + kp * P - 1 - rng.integers(0, 5000, Q)).astype(np.int32)
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    gate_w = torch.full((Q, H), float("nan"), device="cuda")
+    scores = torch.full((Q, P), float("nan"), device="cuda")
+    cand = torch.full((Q, P), 0x7F, dtype=torch.uint8, device="cuda")
+    top = torch.full((Q, SK), 0x7F7F7F7F, dtype=torch.int32, device="cuda")
+    ids = torch.full((Q, SK * kp), 0x7F7F7F7F, dtype=torch.int32, device="cuda")
+    B.dsa_indexer_select(d(hidden), d(w), K, bits(q_idx), d(q_req), d(q_pos), Q, H, 128, bits(keys),
+                         d(pv), d(fv), d(pidx), Bn, kp, P, SK, gate_w, scores, cand, top, ids)
+    torch.cuda.synchronize()
+    gw = gate_w.cpu().numpy()
+    assert_gate_close(gw, O.head_gate(hidden, w))
+    sc, cd = O.index_scores(q_idx, gw, q_req, q_pos, keys, pv, fv, kp)
+    np.testing.assert_array_equal(cand.cpu().numpy(), cd)
+    assert_scores_close(scores.cpu().numpy(), sc, cd, score_magnitude(q_idx, gw, keys, q_req))
+    rt, ri = O.topk_expand(scores.cpu().numpy(), cand.cpu().numpy(), pidx, q_req, SK)
+    np.testing.assert_array_equal(top.cpu().numpy(), rt)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ri)
+    device_status_clean(B)
