@@ -30,8 +30,8 @@
  *     start while the kernel before it on the stream drains, and waits for
  *     that kernel (griddepcontrol.wait) before reading anything an earlier
  *     stage of this path writes. Before that wait it already reads inputs the
- *     path never writes: hidden and w (head gate); ape and req_start
- *     (kpool_compress); ape (kpool_compress_tokens); q_idx and q_req
+ *     path never writes: hidden and w (head gate); ape, ln_w, ln_b,
+ *     req_start, valid, k and gate (kpool_compress); ape (kpool_compress_tokens); q_idx and q_req
  *     (index_scores); q_req (top-k); q, q_req and req_start (sparse MLA). Write those before
  *     the kernel that immediately precedes the call on the stream, or
  *     separate that kernel from the call by a copy, an event wait or a host
@@ -325,20 +325,18 @@ int dsa_indexer_select(const float *hidden, const float *w, int K, const dsa_bf1
  *   (16-byte aligned; contents need no initialisation; not shared between
  *   calls that may overlap).
  *   A query's ids are cut into splits so the grid fills at most one wave of
- *   148 CTAs. The workspace holds the splits' partial results for a merge
- *   in global memory; when a query has 2..8 splits and all the launch's
- *   clusters fit on the device at once, the splits of a query run as one
- *   thread-block cluster, merge in shared memory and leave the workspace
- *   untouched. Either way the splits are merged in split order.
+ *   148 CTAs, each split holding at least four 48-id chunks (half the row's
+ *   chunks when it has fewer than eight). The workspace holds the splits'
+ *   partial results, which a second kernel merges in split order.
  * Requires kv_lora == 512 and rope_dim == 0 (DSA_ERR_UNSUPPORTED otherwise,
  * as the page's config validation refuses any other latent width), Hm a
  * multiple of 16 with 16 <= Hm <= 128, W >= 0.
  */
 size_t dsa_sparse_mla_workspace_size(int Q, int Hm, int W);
 /*
- * Number of kernels dsa_sparse_mla_decode launches for this shape on the
- * current device (1, or 2 when the splits merge through the workspace); 0 for
- * an empty or invalid shape. An inspection aid for callers that account for
+ * Number of kernels dsa_sparse_mla_decode launches for this shape (1 for one
+ * split, 2 when the splits merge through the workspace); 0 for an empty or
+ * invalid shape. An inspection aid for callers that account for
  * launches; it launches nothing.
  */
 int dsa_sparse_mla_launch_count(int Q, int Hm, int W);

@@ -445,13 +445,11 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         t_begin = 0;
         t_end = g_hi - g_lo;                       // this CTA's tiles, in order
     }
-    pdl_wait();
+    // k, gate and the validity bytes are step inputs too: the producer streams
+    // tiles before the wait on the preceding kernel; a thread waits for it before
+    // its first write to an output (the pool warps, and the producer's stores of
+    // the slots past the spans).
     pdl_launch_dependents();
-    if (balanced) {
-        // first_valid: this CTA's share of the requests
-        const int b_lo = (int)((long long)blockIdx.x * B / G), b_hi = (int)((long long)(blockIdx.x + 1) * B / G);
-        for (int b = b_lo + tid; b < b_hi; b += kCmpThreads) first_valid[b] = s_f[b];
-    }
 
     if (warp == kCmpConsumers / 32) {
         // ---------------------------------------------------------------- producer warp
@@ -521,6 +519,7 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             }
             __syncwarp();
         }
+        pdl_wait();
         if (balanced) {
             // pool slots past each request's span: index -1, invalid (the key rows
             // there are not written); this CTA's share of them, request by request
@@ -572,6 +571,12 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     unpack8x2(ldg_nc_v4(ln_w + 8 * l), lw);
     unpack8x2(ldg_nc_v4(ln_b + 8 * l), lb);
     constexpr int kPoolThreads = C::kPoolWarps * 32;
+    pdl_wait();
+    if (balanced) {
+        // first_valid: this CTA's share of the requests
+        const int b_lo = (int)((long long)blockIdx.x * B / G), b_hi = (int)((long long)(blockIdx.x + 1) * B / G);
+        for (int b = b_lo + tid; b < b_hi; b += kPoolThreads) first_valid[b] = s_f[b];
+    }
     for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
         const int s = i % kCmpStages;
         const bool ok = mbar_wait(&stat_full[s], (i / kCmpStages) & 1);

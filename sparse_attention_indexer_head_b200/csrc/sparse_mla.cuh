@@ -8,17 +8,10 @@
 // are cut into S contiguous splits; one CTA per (split, query, 64-head group)
 // gathers its latent rows and runs an online softmax for every head.
 // The S partials (O, running max m, running sum l) of a (query, head group)
-// are merged in split order, so results do not depend on scheduling:
-//   S == 1       the CTA normalises and writes bf16 out and the lse itself;
-//   2 <= S <= 16 the S CTAs form a thread-block cluster and merge through
-//                distributed shared memory, each CTA writing its share of the
-//                heads (no partials in global memory, no second launch), when
-//                all the launch's clusters fit on the device at once;
-//   otherwise    the partials go to the workspace and a combine kernel merges
-//                them.
+// are merged in split order, so results do not depend on scheduling: with
+// S == 1 the CTA normalises and writes bf16 out and the lse itself; otherwise
+// the partials go to the workspace and a combine kernel merges them.
 #pragma once
-
-#include <atomic>
 
 #include "common.cuh"
 #include "tc_ptx.cuh"
@@ -35,29 +28,31 @@ constexpr size_t kPartRowBytes = kL * 2 + 8;
 // ---------------------------------------------------------------------------------------
 // tcgen05 split-KV kernel. One CTA per (split, query, group of 64 heads).
 //
-// Per chunk of 32 selected tokens:
-//   S[64 heads x 32 tokens]   = Q[64 x 512] . KV[32 x 512]^T   (M=64, N=32, 32 K-steps)
-//   softmax over the chunk's tokens, per head row, in registers (one thread per head)
-//   O^T[512 x 64 heads]      += KV^T[512 x 32] . P^T[32 x 64]  (4 x M=128, N=64, 2 K-steps)
+// Per chunk of 48 selected tokens:
+//   S[64 heads x 48 tokens]   = Q[64 x 512] . KV[48 x 512]^T   (M=64, N=48, 32 K-steps,
+//                               as four K-quarters into four accumulators)
+//   softmax over the chunk's tokens, per head row (two threads a head)
+//   O^T[512 x 64 heads]      += KV^T[512 x 48] . P^T[48 x 64]  (4 x M=128, N=64, 3 K-steps)
 // The latent row is both key and value (NoPE), so one 128B-swizzled shared tile
 // of the gathered rows serves as the K-major B operand of S and as the MN-major A
 // operand of O^T. Accumulators live in tensor memory: O^T in columns [0,256)
-// (all 128 lanes), S double-buffered in columns [256,320) (lanes 0-15 of each
+// (all 128 lanes), the four S parts in columns [256,448) (lanes 0-15 of each
 // 32-lane quadrant, the M=64 layout).
 //
-// Warp roles (512 threads): warp 0 allocates tensor memory and one lane issues
-// every MMA (an event loop over the barriers: a PV as soon as its P is ready, an
-// S as soon as its two stages have landed); warps 8-15 gather, two groups of
-// four warps filling alternate 32-token stages of a 4-stage ring with 16-byte
-// cp.async pieces straight into the 128B-swizzled layout (a zero fill for ids
-// that are -1 or outside the request). The copies' landing is tracked by the
-// stage's mbarrier (cp.async.mbarrier.arrive), so no gather warp waits for its
-// own copies. (Per-row TMA copies -- tile::gather4 or a 1-D bulk copy per 1 KB
-// row -- move only 12-20 GB/s per SM here, bounded by their per-instruction
-// cost; cp.async reaches about 37 GB/s per SM once a stage is spread over four
-// warps.) Warps 4-7 load Q, run the softmax, rescale O^T when a head's running
-// max grows by more than 2^8 (lazy rescaling), and write the epilogue. Warps
-// 1-3 take part only in the cluster merge.
+// Warp roles (512 threads): warp 0 allocates tensor memory; lane 0 of each of
+// warps 0-3 issues MMAs in an event loop over the barriers (its K-quarter of S
+// as soon as the chunk has landed and the softmax has read the previous S, its
+// 128-latent block of PV as soon as the chunk's P is ready); warps 8-15 gather,
+// two groups of four warps filling alternate 48-token slots of a 3-slot ring
+// with 16-byte cp.async pieces straight into the 128B-swizzled layout (a zero
+// fill for ids that are -1 or outside the request). The copies' landing is
+// tracked by the slot's mbarrier (cp.async.mbarrier.arrive), so no gather warp
+// waits for its own copies. (Per-row TMA copies -- tile::gather4 or a 1-D bulk
+// copy per 1 KB row -- move only 12-20 GB/s per SM here, bounded by their
+// per-instruction cost; cp.async reaches about 37 GB/s per SM once a slot is
+// spread over four warps.) Warps 4-7 load Q, run the softmax, rescale O^T when
+// a head's running max grows by more than 2^8 (lazy rescaling); all sixteen
+// warps write the epilogue.
 // ---------------------------------------------------------------------------------------
 constexpr int kTcThreads = 512;
 constexpr int kTcChunk = 48;                        // tokens per chunk (one S tile, one PV pass)
@@ -84,13 +79,8 @@ constexpr uint32_t kSCol = 256;                     // S: [256, 256 + kSBufs * k
 static_assert(kSCol + kSBufs * kSParts * kTcChunk <= kTmemCols, "tensor memory columns");
 static_assert(kSParts <= kIssuers && kSParts % 2 == 0, "S parts: one issuer each, read in pairs");
 constexpr float kLazyRescale = 8.0f;                // log2 units
-// Splits merged inside a cluster: up to 8 (the portable size) or, where the
-// device fits them, up to 16 (non-portable sizes are allowed on the kernel).
-constexpr int kMaxClusterSplits = 16;
 constexpr int kSmTarget = 148;                      // CTAs of one full wave (one CTA per SM)
-// The cluster merge reads each CTA's O^T, copied as fp32 [64 heads][512] into
-// the (then idle) gathered-row ring.
-static_assert(8 * kAtomKV >= kTcHeads * kL * 4, "merge buffer must fit the ring");
+constexpr int kMinSplitChunks = 4;                  // chunks a split holds, where there are enough
 static_assert(kOffP % 1024 == 0, "P buffers hold 128B-swizzle atoms");
 
 struct TcCtl {
@@ -111,20 +101,26 @@ static_assert(kTcSmemBytes <= 232448, "shared memory per block");
 struct MlaGeom {
     int S;         // splits per (query, head group)
     int per;       // selected-id slots per split (a multiple of the chunk)
-    bool cluster;  // splits merged inside a thread-block cluster
 };
 
 // The split plan, the same on every device: as many splits as keep the grid
-// within one wave of CTAs, no split holding more chunks than needed for that;
-// every split then holds at least one id. The workspace is sized for this plan
-// merged through global partials.
+// within one wave of CTAs, no split holding more chunks than needed for that,
+// but at least kMinSplitChunks chunks a split (half the row's chunks when it
+// has fewer): each CTA's first gather and its epilogue cost about as much as a
+// few chunks, so more splits of fewer chunks end later. Every split then holds
+// at least one id. Splits merge through global partials and the combine kernel
+// (a merge inside thread-block clusters, measured at the same split counts,
+// was slower on every workload).
 inline MlaGeom mla_plan(int Q, int Hm, int W) {
-    MlaGeom g{1, kTcChunk, false};
+    MlaGeom g{1, kTcChunk};
     if (Q <= 0 || W <= 0) return g;
     const long long ctas = (long long)Q * ((Hm + kTcHeads - 1) / kTcHeads);
     const int chunks = ceil_div(W, kTcChunk);
     int per_chunks = chunks;
-    if (ctas < kSmTarget) per_chunks = ceil_div(chunks, (int)(kSmTarget / ctas));
+    if (ctas < kSmTarget) {
+        per_chunks = ceil_div(chunks, (int)(kSmTarget / ctas));
+        per_chunks = std::max(per_chunks, std::min(kMinSplitChunks, ceil_div(chunks, 2)));
+    }
     g.per = per_chunks * kTcChunk;
     g.S = ceil_div(chunks, per_chunks);
     return g;
@@ -144,68 +140,6 @@ DSA_DEVINL bool tc_wait(TcCtl *ctl, uint64_t *bar, uint32_t parity) {
         return false;
     }
     return true;
-}
-
-// Cluster merge of the S split partials of one (query, head group), held in the
-// shared memory of the cluster's S CTAs (m, l in TcCtl; O^T as fp32
-// [64 heads][512] at sO). The CTA of cluster rank r writes heads
-// [r*hp, min(nh, (r+1)*hp)), hp = ceil(nh / S), 256 threads x 4 latents per
-// head; splits enter in rank order.
-DSA_DEVINL void mla_cluster_merge(const TcCtl *ctl, uint32_t sO, int S, int nh, int rank, int tid,
-                                  float out_scale, __nv_bfloat16 *__restrict__ ob,
-                                  float *__restrict__ lseb) {
-    const int hp = (nh + S - 1) / S;
-    const int hb = rank * hp, he = min(nh, hb + hp);
-    const int c4 = tid & 127;
-    for (int h = hb + (tid >> 7); h < he; h += 2) {
-        const uint32_t am = smem_u32(&ctl->mfin[h]), al = smem_u32(&ctl->lsum[h]);
-        const uint32_t ao = sO + (uint32_t)h * (kL * 4) + c4 * 16;
-        // the splits' maxima first, then their rows in two rounds of eight (all of a
-        // round's remote loads in flight at once), in split order
-        float ms[kMaxClusterSplits];
-#pragma unroll
-        for (int r = 0; r < kMaxClusterSplits; ++r)
-            ms[r] = r < S ? ld_cluster_f32(cluster_map(am, r)) : -INFINITY;
-        float M = -INFINITY;
-#pragma unroll
-        for (int r = 0; r < kMaxClusterSplits; ++r) M = fmaxf(M, ms[r]);
-        float o[4] = {0.f, 0.f, 0.f, 0.f};
-        float lsum = 0.f;
-#pragma unroll
-        for (int r0 = 0; r0 < kMaxClusterSplits; r0 += 8) {
-            if (r0 >= S) break;
-            float ls[8];
-            float4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int r = r0 + u;
-                ls[u] = 0.f;
-                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (r < S && ms[r] != -INFINITY) {
-                    ls[u] = ld_cluster_f32(cluster_map(al, r));
-                    v[u] = ld_cluster_f32x4(cluster_map(ao, r));
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int r = r0 + u;
-                if (r >= S || ms[r] == -INFINITY) continue;
-                const float w = ex2(ms[r] - M);
-                lsum = fmaf(ls[u], w, lsum);
-                o[0] = fmaf(v[u].x, w, o[0]);
-                o[1] = fmaf(v[u].y, w, o[1]);
-                o[2] = fmaf(v[u].z, w, o[2]);
-                o[3] = fmaf(v[u].w, w, o[3]);
-            }
-        }
-        const float inv = lsum > 0.f ? out_scale / lsum : 0.f;
-        uint2 packed;
-        packed.x = pack_bf16x2(o[0] * inv, o[1] * inv);
-        packed.y = pack_bf16x2(o[2] * inv, o[3] * inv);
-        *reinterpret_cast<uint2 *>(ob + (size_t)h * kL + 4 * c4) = packed;
-        if (lseb && c4 == 0)
-            lseb[h] = lsum > 0.f ? (M + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
-    }
 }
 
 // Two E4M3 values (low byte first) widened to a bf16 pair: through f16, exact
@@ -236,7 +170,7 @@ struct KvMap {
 // kv: the latent cache, kv_rows rows of 512 bf16, or of 512 E4M3 bytes (kFp8:
 // the MMA takes them widened to bf16, which is exact; the cache-wide scale is
 // folded into scale_log2 and out_scale).
-template <bool kCluster, bool kPaged, bool kFp8>
+template <bool kPaged, bool kFp8>
 __global__ void __launch_bounds__(kTcThreads, 1)
 mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_raw,
               const KvMap map, const int32_t *__restrict__ q_req,
@@ -650,34 +584,12 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
         }
         if (owner) ctl->lsum[hh] = l;
         tc::named_bar_sync(2, 128);
-        if constexpr (kCluster) {
-            // O^T -> fp32 [head][latent] in the ring (idle: every gathered chunk was
-            // consumed and every MMA has completed); merged after the cluster barrier.
-            if (owner) ctl->mfin[hh] = have_o ? m_used : -INFINITY;
-            if (have_o) {
-                tc::fence_after_sync();
-#pragma unroll 1
-                for (int blk = 0; blk < 8; ++blk) {
-                    uint32_t o[32];
-                    tc::tmem_ld32(tl + (blk >> 1) * 64 + (blk & 1) * 32, o);
-                    tc::tmem_wait_ld();
-                    const int L = (blk >> 1) * 128 + 32 * wq + lane;
-                    const uint32_t dst = sKV + ((uint32_t)((blk & 1) * 32) * kL + L) * 4;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        asm volatile("st.shared.f32 [%0], %1;" ::"r"(dst + (uint32_t)j * kL * 4),
-                                     "f"(__uint_as_float(o[j]))
-                                     : "memory");
-                }
-            }
-        } else {
-            // O^T is written after the CTA barrier below, by all sixteen warps.
-            if (owner) ctl->mfin[hh] = have_o ? m_used : -INFINITY;
-            if (tid == 128) ctl->have_o = have_o ? 1 : 0;
-            if (S == 1 && lse && owner && hh < nh)
-                lse[(size_t)qi * Hm + h0 + hh] =
-                    (have_o && l > 0.f) ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
-        }
+        // O^T is written after the CTA barrier below, by all sixteen warps.
+        if (owner) ctl->mfin[hh] = have_o ? m_used : -INFINITY;
+        if (tid == 128) ctl->have_o = have_o ? 1 : 0;
+        if (S == 1 && lse && owner && hh < nh)
+            lse[(size_t)qi * Hm + h0 + hh] =
+                (have_o && l > 0.f) ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
 
     // Every MMA of this CTA has completed before tensor memory is released.
@@ -685,7 +597,7 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if constexpr (!kCluster) {
+    {
         // O^T out of tensor memory by all sixteen warps: warp w reads the lane
         // quarter w % 4 (32 latent rows of each 128-row block) for two of the
         // eight (latent block, 32-head half) pieces; each store writes 32
@@ -743,13 +655,6 @@ mla_tc_kernel(const __nv_bfloat16 *__restrict__ qm, const void *__restrict__ kv_
         }
         tc::fence_before_sync();
         __syncthreads();              // every tensor-memory read is done before the release
-    }
-    if constexpr (kCluster) {
-        cluster_sync_all();           // every split's m, l and O^T are in place
-        if (tid < 256)
-            mla_cluster_merge(ctl, sKV, S, nh, split, tid, out_scale, out + ((size_t)qi * Hm + h0) * kL,
-                              lse ? lse + (size_t)qi * Hm + h0 : nullptr);
-        cluster_sync_all();           // no CTA leaves while a peer still reads it
     }
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
@@ -829,70 +734,11 @@ mla_combine_kernel(const uint8_t *__restrict__ part, int Hm, int S, float out_sc
         lse[(size_t)q * Hm + h] = lsum > 0.f ? (M + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
 }
 
-// Raise the cluster kernel's shared-memory limit and allow cluster sizes above
-// the portable 8 (once per device; false if the runtime refuses).
-template <bool kPaged, bool kFp8>
-inline bool mla_prepare_cluster_kernel() {
-    const void *f = reinterpret_cast<const void *>(mla_tc_kernel<true, kPaged, kFp8>);
-    if (!ensure_smem_attr(f, kTcSmemBytes)) return false;
-    return cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
-}
-
-// How many clusters of `splits` CTAs of the cluster kernel can be resident at
-// once on the current device (asked once per device and size, after the
-// kernel's shared-memory limit is raised); 0 when none or unknown.
-inline int mla_max_clusters(int splits) {
-    static std::atomic<int> known[64][kMaxClusterSplits + 1];   // count + 1; 0 = not asked
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    const int k = known[dev][splits].load(std::memory_order_relaxed);
-    if (k != 0) return k - 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(splits, 1, 1);
-    cfg.blockDim = dim3(kTcThreads);
-    cfg.dynamicSmemBytes = kTcSmemBytes;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel<true, false, false>, &cfg) != cudaSuccess) n = 0;
-    (void)cudaGetLastError();
-    known[dev][splits].store(n + 1, std::memory_order_relaxed);
-    return n;
-}
-
-// The launch: a plan of 2 or more splits runs as clusters of at most 16 CTAs
-// when all of a grid's clusters can be resident at once, shrinking the cluster
-// (more chunks per CTA) while that costs at most two chunks per CTA over the
-// plan -- about what the global merge and its second launch cost; otherwise
-// the plan runs with global partials.
-inline MlaGeom mla_launch_geometry(int Q, int Hm, int W) {
-    MlaGeom g = mla_plan(Q, Hm, W);
-    if (g.S < 2) return g;
-    const long long ctas = (long long)Q * ((Hm + kTcHeads - 1) / kTcHeads);
-    const int chunks = ceil_div(W, kTcChunk);
-    const int base = g.per / kTcChunk;
-    for (int s = std::min(g.S, kMaxClusterSplits); s >= 2; --s) {
-        const int pc = ceil_div(chunks, s);
-        if (pc > base + 2) break;
-        const int ss = ceil_div(chunks, pc);
-        if (ss < 2) break;
-        if ((long long)mla_max_clusters(ss) >= ctas) return MlaGeom{ss, pc * kTcChunk, true};
-    }
-    return g;
-}
-
-// Kernels sparse_mla_launch runs for this shape on the current device: the
-// split kernel, plus the combine when the splits merge through the workspace.
+// Kernels sparse_mla_launch runs for this shape: the split kernel, plus the
+// combine when a query's ids are split.
 inline int sparse_mla_launch_count(int Q, int Hm, int W) {
     if (Q <= 0 || Hm <= 0 || W < 0) return 0;
-    if (!mla_prepare_cluster_kernel<false, false>()) return 0;
-    const MlaGeom g = mla_launch_geometry(Q, Hm, W);
-    return (g.S > 1 && !g.cluster) ? 2 : 1;
+    return mla_plan(Q, Hm, W).S > 1 ? 2 : 1;
 }
 
 template <bool kPaged, bool kFp8>
@@ -922,11 +768,9 @@ inline int sparse_mla_launch_map(const void *q, const void *kv, int64_t kv_rows,
         return DSA_ERR_ALIGNMENT;
     const size_t need = mla_workspace_bytes(Q, Hm, W);
     if (need > 0 && (!ws || ws_bytes < need)) return DSA_ERR_WORKSPACE;
-    if (!mla_prepare_cluster_kernel<kPaged, kFp8>() ||
-        !ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<false, kPaged, kFp8>), kTcSmemBytes) ||
-        !mla_prepare_cluster_kernel<false, false>())
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(mla_tc_kernel<kPaged, kFp8>), kTcSmemBytes))
         return DSA_ERR_CUDA;
-    const MlaGeom g = mla_launch_geometry(Q, Hm, W);
+    const MlaGeom g = mla_plan(Q, Hm, W);
     // fp8: S = sm_scale * q . (s k8) = (sm_scale * s) q . k8, and O = s * (P V8)
     const float out_scale = kFp8 ? kv_scale : 1.0f;
     const float scale_log2 = (kFp8 ? sm_scale * kv_scale : sm_scale) * 1.4426950408889634f;
@@ -935,15 +779,7 @@ inline int sparse_mla_launch_map(const void *q, const void *kv, int64_t kv_rows,
     const auto *qb = reinterpret_cast<const __nv_bfloat16 *>(q);
     auto *ob = reinterpret_cast<__nv_bfloat16 *>(out);
     const dim3 grid(g.S, Q, groups);
-    if (g.cluster) {
-        if (launch_pdl_cluster(mla_tc_kernel<true, kPaged, kFp8>, grid, dim3(kTcThreads),
-                               kTcSmemBytes, stream, g.S, qb, kv, map, q_req, token_ids, B,
-                               (int)kv_rows, Hm, W, g.S, g.per, scale_log2, out_scale, part, ob,
-                               lse) != cudaSuccess)
-            return DSA_ERR_CUDA;
-        return launch_status();
-    }
-    if (launch_pdl(mla_tc_kernel<false, kPaged, kFp8>, grid, dim3(kTcThreads), kTcSmemBytes,
+    if (launch_pdl(mla_tc_kernel<kPaged, kFp8>, grid, dim3(kTcThreads), kTcSmemBytes,
                    stream, qb, kv, map, q_req, token_ids, B, (int)kv_rows, Hm, W, g.S, g.per,
                    scale_log2, out_scale, part, ob, lse) != cudaSuccess)
         return DSA_ERR_CUDA;

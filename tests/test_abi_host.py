@@ -193,11 +193,13 @@ def test_topk_expand_tail_refusals(B):
 
 def test_sparse_mla_refusals(B):
     L = B.lib
-    # partials of every split (the plan keeps the grid within 148 CTAs; 48-token
-    # chunks, 43 of them for 2048 ids): 2 queries -> 43 splits of one chunk;
-    # 16 queries -> 9 splits of 5 chunks
+    # partials of every split (the plan keeps the grid within 148 CTAs with at
+    # least four 48-token chunks a split, half the row when it has fewer than
+    # eight; 43 chunks for 2048 ids): 2 queries -> 11 splits of 4 chunks;
+    # 16 queries -> 9 splits of 5 chunks; 1 query of 64 ids -> 2 splits of 1
     ws = B.dsa_sparse_mla_workspace_size(2, 64, 2048)
-    assert ws == 2 * 43 * 64 * (512 * 2 + 8)
+    assert ws == 2 * 11 * 64 * (512 * 2 + 8)
+    assert B.dsa_sparse_mla_workspace_size(1, 16, 64) == 1 * 2 * 16 * (512 * 2 + 8)
     assert B.dsa_sparse_mla_workspace_size(16, 64, 2048) == 16 * 9 * 64 * (512 * 2 + 8)
     # at least 148 CTAs without splitting: one split, no workspace
     assert B.dsa_sparse_mla_workspace_size(148, 64, 2048) == 0

@@ -69,17 +69,17 @@ def _paged_call(B, step, pool, table, seq_len, page):
 
 
 def _workload(name):
-    if name == "cluster":
-        # 32 decode queries: each query's ids split 4 ways and merge inside a cluster
+    if name == "split4":
+        # 32 decode queries: each query's ids split 4 ways, merged by the combine
         lengths = [600 + 37 * i for i in range(32)]
-        return W.build("cluster", lengths=lengths, pads=[i % 5 for i in range(32)], kpool=4,
+        return W.build("split4", lengths=lengths, pads=[i % 5 for i in range(32)], kpool=4,
                        max_pools=(max(lengths) + 3) // 4, select_k=512, hm=64,
                        q_req=list(range(32)), q_pos=[t - 1 for t in lengths], seed=17)
     return W.make(name)
 
 
 @pytest.mark.parametrize("name,page", [("tiny", 16), ("tiny", 7), ("tiny", 1), ("batched", 64),
-                                       ("cluster", 32)])
+                                       ("split4", 32)])
 def test_paged_equals_contiguous(B, name, page):
     from sparse_attention_indexer_head_b200.pipeline import DecodeStep
     wl = _workload(name)
@@ -139,7 +139,7 @@ def _paged_call_fp8(B, step, pool8, scale, table, seq_len, page):
     return out.view(torch.int16).cpu().numpy().view(np.uint16), lse.cpu().numpy()
 
 
-@pytest.mark.parametrize("name,page", [("tiny", 16), ("batched", 64), ("cluster", 32)])
+@pytest.mark.parametrize("name,page", [("tiny", 16), ("batched", 64), ("split4", 32)])
 def test_paged_fp8_against_oracle_and_bf16(B, name, page):
     from sparse_attention_indexer_head_b200.pipeline import DecodeStep
     wl = _workload(name)
@@ -189,7 +189,7 @@ def test_paged_fp8_against_oracle_and_bf16(B, name, page):
     device_status_clean(B)
 
 
-def test_cluster_workload_takes_the_cluster_path(B):
-    """The 32-query case above merges its splits inside clusters: one MLA launch."""
-    assert B.dsa_sparse_mla_launch_count(32, 64, 2048) == 1
-    assert B.dsa_sparse_mla_workspace_size(32, 64, 2048) > 0      # sized for the global plan
+def test_split4_workload_plan(B):
+    """The 32-query case above: 4 splits a query (128 CTAs), merged by the combine."""
+    assert B.dsa_sparse_mla_launch_count(32, 64, 2048) == 2
+    assert B.dsa_sparse_mla_workspace_size(32, 64, 2048) == 32 * 4 * 64 * (1024 + 8)

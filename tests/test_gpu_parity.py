@@ -246,13 +246,13 @@ def test_mla_rows_past_kv_rows_are_not_read(B):
 
 
 def test_mla_launch_count(B):
-    # one split: the split kernel alone; more than 16 splits even after shrinking the
-    # plan: the workspace merge, so a combine kernel too; 2..16 splits: 1 or 2
-    # (clusters where all of them fit on the device at once)
+    # one split: the split kernel alone; more: the combine kernel too
     assert B.dsa_sparse_mla_launch_count(148, 64, 2048) == 1
+    assert B.dsa_sparse_mla_launch_count(2048, 64, 2048) == 1
     assert B.dsa_sparse_mla_launch_count(2, 64, 32768) == 2
-    assert B.dsa_sparse_mla_launch_count(2, 64, 2048) in (1, 2)
-    assert B.dsa_sparse_mla_launch_count(16, 64, 2048) in (1, 2)
+    assert B.dsa_sparse_mla_launch_count(2, 64, 2048) == 2
+    assert B.dsa_sparse_mla_launch_count(16, 64, 2048) == 2
+    assert B.dsa_sparse_mla_launch_count(1, 16, 64) == 2        # two chunks, a split each
     assert B.dsa_sparse_mla_launch_count(0, 64, 2048) == 0
 
 
