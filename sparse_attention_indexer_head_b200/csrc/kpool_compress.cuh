@@ -31,7 +31,7 @@ namespace dsa {
 // warps per scheduler, so 128 registers a thread) and 120-token tiles -- four
 // threads per row in the statistics phase, two pools per warp (30 pools at kpool
 // 4); larger pools (more live registers) 8 warps and floor(128 / kpool) pools.
-// A stage holds the tile's k rows then its gate rows; three stages in the ring.
+// A stage holds the tile's k rows then its gate rows; three or four stages in the ring.
 template <int KP> struct CmpCfg {
     static constexpr int kPoolWarps = KP <= 4 ? 12 : 6;         // a half-warp per pool
     static constexpr int kStatWarps = KP <= 4 ? 3 : 2;          // LayerNorm statistics, a tile ahead
@@ -40,7 +40,7 @@ template <int KP> struct CmpCfg {
     static constexpr int kThreads = kConsumers + 32;            // + 1 producer warp
     static constexpr int kTP = 2 * kPoolWarps;                  // pools per tile
     static constexpr int kTileTokens = kTP * KP;
-    static constexpr int kStages = 3;
+    static constexpr int kStages = 4;                           // most ring stages (3 or 4 run)
     static constexpr int kStageBytes = 2 * kTileTokens * 128 * 2;
 };
 constexpr int kD = DSA_INDEX_DIM;   // 128 channels
@@ -125,18 +125,20 @@ DSA_DEVINL float2 row_stats(const __nv_bfloat16 *row, int q, int rot, bool act, 
     }
     const float x0 = __shfl_sync(0xffffffffu, bf16lo(v[0].x), lane & ~3);
     const float2 nx0 = make_float2(-x0, -x0);
-    float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
+    // pairwise sums (a short dependency chain): per 16-byte piece, then over pieces
+    float2 p1[4], p2[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        float2 x[4];
+        float2 x[4], d[4];
         unpack8x2(v[i], x);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const float2 d = __fadd2_rn(x[c], nx0);
-            s1 = __fadd2_rn(s1, d);
-            s2 = __ffma2_rn(d, d, s2);
-        }
+        for (int c = 0; c < 4; ++c) d[c] = __fadd2_rn(x[c], nx0);
+        p1[i] = __fadd2_rn(__fadd2_rn(d[0], d[1]), __fadd2_rn(d[2], d[3]));
+        p2[i] = __fadd2_rn(__ffma2_rn(d[1], d[1], __fmul2_rn(d[0], d[0])),
+                           __ffma2_rn(d[3], d[3], __fmul2_rn(d[2], d[2])));
     }
+    const float2 s1 = __fadd2_rn(__fadd2_rn(p1[0], p1[1]), __fadd2_rn(p1[2], p1[3]));
+    const float2 s2 = __fadd2_rn(__fadd2_rn(p2[0], p2[1]), __fadd2_rn(p2[2], p2[3]));
     float a1 = __fadd_rn(s1.x, s1.y), a2 = __fadd_rn(s2.x, s2.y);
     a1 = __fadd_rn(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
     a2 = __fadd_rn(a2, __shfl_xor_sync(0xffffffffu, a2, 1));
@@ -157,11 +159,15 @@ DSA_DEVINL float2 row_stats(const __nv_bfloat16 *row, int q, int rot, bool act, 
 DSA_DEVINL void token_stats(const __nv_bfloat16 *sk, int ntok, float eps, float2 *stat, int ctid,
                             int nthreads) {
     const int q = ctid & 3;
-    for (int tok0 = 0; tok0 < ntok; tok0 += nthreads / 4) {
-        const int tok = tok0 + (ctid >> 2);
-        const bool act = tok < ntok;
-        const float2 st = row_stats(sk + (size_t)(act ? tok : 0) * kD, q, 4 * (tok & 1), act, eps);
-        if (act && q == 0) stat[tok] = st;
+    const int rows = nthreads / 4;
+    // two rows a thread group per step, so both rows' loads and sums overlap
+    for (int tok0 = 0; tok0 < ntok; tok0 += 2 * rows) {
+        const int ta = tok0 + (ctid >> 2), tb = ta + rows;
+        const bool aa = ta < ntok, ab = tb < ntok;
+        const float2 sa = row_stats(sk + (size_t)(aa ? ta : 0) * kD, q, 4 * (ta & 1), aa, eps);
+        const float2 sb = row_stats(sk + (size_t)(ab ? tb : 0) * kD, q, 4 * (tb & 1), ab, eps);
+        if (aa && q == 0) stat[ta] = sa;
+        if (ab && q == 0) stat[tb] = sb;
     }
 }
 
@@ -169,20 +175,18 @@ DSA_DEVINL void token_stats(const __nv_bfloat16 *sk, int ntok, float eps, float2
 // k rows and gate rows, with the rows' LayerNorm statistics st[s]. s_ape holds
 // ape * log2(e) laid out [slot][half][lane][4] so a half-warp's loads are
 // contiguous. Returns the packed bf16 chunk (zero when the pool is invalid).
+//
+// One pass over the slots: the per-channel softmax is shifted by slot 0's
+// logit instead of the slots' maximum (the same quotient), so each slot's
+// exp2 weight and weighted k_norm row are formed as the row streams by, with
+// no max pass and no logits held between passes. A weight that overflows
+// (logits more than 2^7 apart in log2 units) leaves a non-finite denominator;
+// the warp then redoes its pools shifted by the slots' maximum.
 template <int KP>
 DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *grow,
                                const float2 *st, const float *s_ape, const float2 (&lw)[4],
                                const float2 (&lb)[4], int l, bool ok) {
-    // Pass 1 forms the slot logits and their per-channel max; pass 2 forms the
-    // bf16 k_norm rows and the softmax-weighted sum. kpool <= 4 keeps the logits
-    // in registers between the passes, larger pools recompute them.
-    constexpr bool kKeep = KP <= 4;
     const float2 log2e2 = make_float2(kLog2e, kLog2e);
-    float2 lgk[kKeep ? KP : 1][4];
-    float2 mx2[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) mx2[c] = make_float2(-INFINITY, -INFINITY);
-
     auto knorm = [&](int s, float2 (&kn)[4]) {
         const float2 rs = st[s];
         const float2 r2 = make_float2(rs.x, rs.x), n2 = make_float2(rs.y, rs.y);
@@ -202,41 +206,53 @@ DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *g
         lg[2] = __ffma2_rn(g[2], log2e2, make_float2(a1.x, a1.y));
         lg[3] = __ffma2_rn(g[3], log2e2, make_float2(a1.z, a1.w));
     };
-
-#pragma unroll
-    for (int s = 0; s < KP; ++s) {
+    // slots a step (measured: unrolled fully the loop spills; one slot a step
+    // is fastest at kpool <= 4, two above)
+    constexpr int kSlotUnroll = KP <= 4 ? 1 : 2;
+    float2 nsh[4], den[4], acc[4];
+    {
         float2 lg[4];
-        logits(s, lg);
+        logits(0, lg);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) nsh[c] = make_float2(-lg[c].x, -lg[c].y);
+    }
+#pragma unroll 1
+    for (int attempt = 0;; ++attempt) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            mx2[c] = make_float2(fmaxf(mx2[c].x, lg[c].x), fmaxf(mx2[c].y, lg[c].y));
-            if constexpr (kKeep) lgk[s][c] = lg[c];
+            den[c] = make_float2(0.f, 0.f);
+            acc[c] = make_float2(0.f, 0.f);
         }
-    }
-    float2 nmx[4], den[4], acc[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        nmx[c] = make_float2(-mx2[c].x, -mx2[c].y);
-        den[c] = make_float2(0.f, 0.f);
-        acc[c] = make_float2(0.f, 0.f);
-    }
-#pragma unroll
-    for (int s = 0; s < KP; ++s) {
-        float2 kn[4], lg[4];
-        if constexpr (kKeep) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) lg[c] = lgk[s][c];
-        } else {
+#pragma unroll kSlotUnroll
+        for (int s = 0; s < KP; ++s) {
+            float2 kn[4], lg[4];
             logits(s, lg);
-        }
-        knorm(s, kn);
+            knorm(s, kn);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const float2 z = __fadd2_rn(lg[c], nmx[c]);
-            const float2 e = make_float2(ex2(z.x), ex2(z.y));
-            den[c] = __fadd2_rn(den[c], e);
-            acc[c] = __ffma2_rn(e, kn[c], acc[c]);
+            for (int c = 0; c < 4; ++c) {
+                const float2 z = __fadd2_rn(lg[c], nsh[c]);
+                const float2 e = make_float2(ex2(z.x), ex2(z.y));
+                den[c] = __fadd2_rn(den[c], e);
+                acc[c] = __ffma2_rn(e, kn[c], acc[c]);
+            }
         }
+        float dsum = 0.f;     // finite iff every denominator is (a NaN or inf carries through)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dsum += den[c].x + den[c].y;
+        if (attempt == 1 || !__any_sync(0xffffffffu, !(dsum < INFINITY))) break;
+        // overflow somewhere in the warp: shift by the slots' maximum instead
+        float2 mx[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mx[c] = make_float2(-INFINITY, -INFINITY);
+#pragma unroll
+        for (int s = 0; s < KP; ++s) {
+            float2 lg[4];
+            logits(s, lg);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) mx[c] = make_float2(fmaxf(mx[c].x, lg[c].x), fmaxf(mx[c].y, lg[c].y));
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) nsh[c] = make_float2(-mx[c].x, -mx[c].y);
     }
     uint4 o = make_uint4(0, 0, 0, 0);
     if (ok) {
@@ -269,14 +285,14 @@ template <int KP>
 __global__ void __launch_bounds__(CmpCfg<KP>::kThreads, 1)
 kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ gate,
                       const uint8_t *__restrict__ valid, const int32_t *__restrict__ req_start,
-                      int B, int max_pools, int tiles_per_req, int n_tiles, int balance_ok,
+                      int B, int max_pools, int tiles_per_req, int n_tiles, int balance_ok, int ns,
                       const float *__restrict__ ape, const __nv_bfloat16 *__restrict__ ln_w,
                       const __nv_bfloat16 *__restrict__ ln_b, float eps,
                       __nv_bfloat16 *__restrict__ pool_keys, int32_t *__restrict__ pool_idx,
                       uint8_t *__restrict__ pool_valid, int32_t *__restrict__ first_valid) {
     using C = CmpCfg<KP>;
     constexpr int TP = C::kTP;
-    constexpr int kCmpStages = C::kStages;
+    constexpr int kCmpStages = C::kStages;       // static arrays; ns stages are used
     constexpr int kCmpStageBytes = C::kStageBytes;
     constexpr int kCmpTileTokens = C::kTileTokens;
     constexpr int kCmpConsumers = C::kConsumers;
@@ -296,7 +312,7 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     int t_end = (int)((long long)(blockIdx.x + 1) * n_tiles / G);
     // Balanced: per request its first valid token, and prefix sums over the requests
     // of the tiles holding pools in its span and of the pool slots past the span.
-    int32_t *s_f = reinterpret_cast<int32_t *>(cmp_smem + kCmpStages * kCmpStageBytes);
+    int32_t *s_f = reinterpret_cast<int32_t *>(cmp_smem + ns * kCmpStageBytes);
     int32_t *s_pre = s_f + B;
     int32_t *s_epre = s_pre + (B + 1);
     int32_t *s_rs = s_epre + (B + 1);                // req_start, B + 1 entries
@@ -465,9 +481,9 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             bb = lo;
         }
         for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
-            const int s = i % kCmpStages;
+            const int s = i % ns;
             bool ok = true;
-            if (i >= kCmpStages) ok = mbar_wait(&empty[s], ((i / kCmpStages) - 1) & 1);
+            if (i >= ns) ok = mbar_wait(&empty[s], ((i / ns) - 1) & 1);
             if (!__all_sync(0xffffffffu, ok)) break;
             int b, j;
             if (balanced) {
@@ -555,8 +571,8 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     if (warp >= C::kPoolWarps) {
         const int stid = tid - C::kPoolWarps * 32;
         for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
-            const int s = i % kCmpStages;
-            const bool ok = mbar_wait(&full[s], (i / kCmpStages) & 1);
+            const int s = i % ns;
+            const bool ok = mbar_wait(&full[s], (i / ns) & 1);
             if (!__all_sync(0xffffffffu, ok)) break;
             const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
             token_stats(sk, meta[s].n_in * KP, eps, &s_stat[s][0], stid, C::kStatWarps * 32);
@@ -578,8 +594,8 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         for (int b = b_lo + tid; b < b_hi; b += kPoolThreads) first_valid[b] = s_f[b];
     }
     for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
-        const int s = i % kCmpStages;
-        const bool ok = mbar_wait(&stat_full[s], (i / kCmpStages) & 1);
+        const int s = i % ns;
+        const bool ok = mbar_wait(&stat_full[s], (i / ns) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
         const CmpMeta m = meta[s];
         const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
@@ -627,16 +643,27 @@ inline int kpool_compress_launch_kp(const __nv_bfloat16 *k, const __nv_bfloat16 
     // hold pools evenly (balanced, where request lengths differ); beyond, always
     // contiguous ranges of every request's tile grid.
     const int balance_ok = B <= kCmpReqPerThread * C::kThreads ? 1 : 0;
-    const int smem = C::kStages * C::kStageBytes + (balance_ok ? 4 * (4 * B + 3) : 0);
-    if (!ensure_smem_attr(reinterpret_cast<const void *>(kpool_compress_kernel<KP>),
-                          C::kStages * C::kStageBytes + 4 * (4 * kCmpReqPerThread * C::kThreads + 3)))
+    // Ring depth: each stage turns over in its load latency plus the consumers'
+    // time on it, so a fourth stage (more bytes in flight, less of the ring idle
+    // while a tile is worked on) where the block's shared memory has room for it
+    // next to the balanced partition's per-request arrays.
+    const void *f = reinterpret_cast<const void *>(kpool_compress_kernel<KP>);
+    cudaFuncAttributes fa;
+    int dev = 0, optin = 0;
+    if (cudaFuncGetAttributes(&fa, f) != cudaSuccess || cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
         return DSA_ERR_CUDA;
+    const int extra = balance_ok ? 4 * (4 * B + 3) : 0;
+    int ns = C::kStages;
+    while (ns > 3 && (long long)fa.sharedSizeBytes + ns * C::kStageBytes + extra > optin) --ns;
+    const int smem = ns * C::kStageBytes + extra;
+    if (!ensure_smem_attr(f, smem)) return DSA_ERR_CUDA;
     const int tiles_per_req = max(1, ceil_div(max_pools, TP));
     const long long n_tiles = (long long)tiles_per_req * B;
     if (n_tiles > (1ll << 30)) return DSA_ERR_UNSUPPORTED;
     const int grid = (int)std::min<long long>(n_tiles, sm_count());
     if (launch_pdl(kpool_compress_kernel<KP>, dim3(grid), dim3(C::kThreads), smem, stream, k, gate,
-                   valid, req_start, B, max_pools, tiles_per_req, (int)n_tiles, balance_ok, ape, ln_w,
+                   valid, req_start, B, max_pools, tiles_per_req, (int)n_tiles, balance_ok, ns, ape, ln_w,
                    ln_b, eps, keys, idx, pv, fv) != cudaSuccess)
         return DSA_ERR_CUDA;
     return launch_status();
