@@ -124,6 +124,27 @@ def test_compress_partitions(B, kpool, n_req, max_len, max_pools):
     device_status_clean(B)
 
 
+def test_compress_gate_logits_far_apart(B):
+    """Compress shifts each channel's softmax by slot 0's logit; where the slots'
+    logits lie more than 2^7 apart (log2 units) a weight overflows and the warp
+    redoes its pools shifted by the maximum. Gate logits of +-100 on some tokens
+    (and 0.5 elsewhere) take that path; the keys still match the oracle."""
+    for kpool in (4, 8):
+        wl = _mini(kpool, [640, 333], [0, 5], select_k=8)
+        g16 = wl.gate.copy()
+        hi, lo = np.uint16(0x42C8), np.uint16(0xC2C8)        # bf16 +100, -100
+        g16[3::7, ::3] = hi
+        g16[5::11, 1::3] = lo
+        wl.gate[:] = g16
+        step, g = run_step(wl)
+        keys, idx, pv, fv = O.kpool_compress(wl.k, wl.gate, wl.valid, wl.req_start, wl.kpool,
+                                             wl.max_pools, wl.ape, wl.ln_w, wl.ln_b, wl.eps)
+        np.testing.assert_array_equal(g["pool_valid"], pv)
+        np.testing.assert_array_equal(g["pool_idx"], idx)
+        assert_keys_close(g["pool_keys"], keys, pv, wl, fv)
+    device_status_clean(B)
+
+
 def test_select_more_than_candidates_and_sentinel(B):
     wl = _mini(4, [64, 40], [0, 10], select_k=64)
     step, g = run_step(wl)
