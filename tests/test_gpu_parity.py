@@ -10,7 +10,8 @@ import pytest
 import torch
 
 import oracle as O
-from gpu_helpers import (assert_gate_close, assert_keys_close, assert_mla_close, dev_bits,
+from gpu_helpers import (assert_gate_close, assert_keys_close, assert_mla_close, assert_scores_close,
+                         dev_bits, score_magnitude,
                          device_status_clean, end_to_end, host_bits, mla_value_bound, run_step,
                          stagewise, workload)
 from sparse_attention_indexer_head_b200 import workloads as W
@@ -162,6 +163,38 @@ def test_ties_break_to_lowest_pool_id(B):
     assert (g["gate_w"] == 0).all()
     stagewise(wl, g)
     assert list(g["top_pools"][0]) == list(range(32))
+    device_status_clean(B)
+
+
+@pytest.mark.parametrize("H", [16, 13])
+def test_scores_many_queries(B, H):
+    """300 queries (the many-query scores kernel at H = 16: groups of 16 queries
+    sharing key tiles; the one-query kernel at H = 13): runs of one request that
+    do not line up with the groups, queries naming no request, causal positions
+    from before the first pool to past the last, 1000 pools (a ragged last tile).
+    Every score and candidate flag against the oracle."""
+    rng = np.random.default_rng(31 + H)
+    Q, P, kp, Bn = 300, 1000, 4, 3
+    q_req = np.sort(rng.integers(0, Bn, Q)).astype(np.int32)
+    q_req[[5, 17, 200]] = [-1, 7, -3]
+    fv = np.array([0, 3, 11], np.int32)
+    q_pos = rng.integers(-5, P * kp + 20, Q).astype(np.int32)
+    q_idx = W.f32_to_bf16_bits(rng.standard_normal((Q, H, 128)).astype(np.float32))
+    keys = W.f32_to_bf16_bits(rng.standard_normal((Bn, P, 128)).astype(np.float32))
+    pv = (rng.random((Bn, P)) < 0.9).astype(np.uint8)
+    gw = rng.standard_normal((Q, H)).astype(np.float32)
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    scores = torch.full((Q, P), float("nan"), device="cuda")
+    cand = torch.full((Q, P), 0x7F, dtype=torch.uint8, device="cuda")
+    B.dsa_index_scores(dev_bits(q_idx), d(gw), d(q_req), d(q_pos), Q, H, 128, dev_bits(keys), d(pv),
+                       d(fv), Bn, kp, P, scores, cand)
+    torch.cuda.synchronize()
+    ok = (q_req >= 0) & (q_req < Bn)
+    gs, gc = scores.cpu().numpy(), cand.cpu().numpy()
+    assert (gc[~ok] == 0).all() and np.isneginf(gs[~ok]).all()      # no request: no candidates
+    sc, cd = O.index_scores(q_idx[ok], gw[ok], q_req[ok], q_pos[ok], keys, pv, fv, kp)
+    np.testing.assert_array_equal(gc[ok], cd)
+    assert_scores_close(gs[ok], sc, cd, score_magnitude(q_idx[ok], gw[ok], keys, q_req[ok]))
     device_status_clean(B)
 
 
