@@ -27,11 +27,12 @@
 
 namespace dsa {
 
-// Geometry per kpool. kpool <= 4: 15 consumer warps (with the producer, four
-// warps per scheduler, so 128 registers a thread) and 120-token tiles -- four
-// threads per row in the statistics phase, two pools per warp (30 pools at kpool
-// 4); larger pools (more live registers) 8 warps and floor(128 / kpool) pools.
-// A stage holds the tile's k rows then its gate rows; three or four stages in the ring.
+// Geometry per kpool. kpool <= 4: 12 pool warps (a half-warp a pool, so 24 pools,
+// 96 token rows at kpool 4, a tile) and 3 statistics warps (a thread a row);
+// with the producer four warps per scheduler, so up to 128 registers a thread.
+// Larger pools (more live registers): 6 pool warps (12 pools) and 2 statistics
+// warps. A stage holds the tile's k rows then its gate rows; three or four
+// stages in the ring.
 template <int KP> struct CmpCfg {
     static constexpr int kPoolWarps = KP <= 4 ? 12 : 6;         // a half-warp per pool
     static constexpr int kStatWarps = KP <= 4 ? 3 : 2;          // LayerNorm statistics, a tile ahead
@@ -107,43 +108,48 @@ DSA_DEVINL float2 round_bf16x2(float2 y) {
     return make_float2(bf16lo(p), bf16hi(p));
 }
 
-// LayerNorm statistics of one token row on a group of four lanes (q = 0..3,
-// lanes 4g..4g+3 of the warp): lane q sums the 16-byte pieces q, q+4, q+8, q+12,
-// rotated by rot (0 or 4) pieces. The moments are shifted by a sample of the row
-// (its element 8*rot), which lies within a few standard deviations of the mean,
-// so their difference does not cancel. Returns (rstd, -mu * rstd) to every lane
-// of the group; a lane with act false reads nothing and counts as zeros. Every
-// lane of the warp calls it (full-warp shuffles). The rounding is explicit, so
-// every kernel that calls it gets the same bits for the same row and rot.
-DSA_DEVINL float2 row_stats(const __nv_bfloat16 *row, int q, int rot, bool act, float eps) {
-    const int lane = threadIdx.x & 31;
-    uint4 v[4];
+// LayerNorm statistics of one token row on one thread. The row's sixteen
+// 16-byte pieces are read in the order j ^ rot (j = 0..15, rot in 0..7), so the
+// eight rows of consecutive rot that one shared-memory phase serves touch eight
+// distinct bank groups. The moments are shifted by a sample of the row (the
+// first element read, element 8 * rot), which lies within a few standard
+// deviations of the mean, so their difference does not cancel. Sums are
+// pairwise: within a piece, over four pieces, over the four groups. Returns
+// (rstd, -mu * rstd). The order is fixed, so every kernel that calls it gets
+// the same bits for the same row and rot.
+DSA_DEVINL float2 row_stats(const __nv_bfloat16 *row, int rot, float eps) {
+    float2 g1[4], g2[4];
+    float x0 = 0.f;
+    float2 nx0 = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int piece = (q + 4 * i + rot) & 15;
-        v[i] = act ? *reinterpret_cast<const uint4 *>(row + piece * 8) : make_uint4(0u, 0u, 0u, 0u);
+    for (int q = 0; q < 4; ++q) {
+        uint4 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int j = 4 * q + i;
+            v[i] = *reinterpret_cast<const uint4 *>(row + 8 * ((j & 8) | ((j & 7) ^ rot)));
+        }
+        if (q == 0) {
+            x0 = bf16lo(v[0].x);
+            nx0 = make_float2(-x0, -x0);
+        }
+        float2 p1[4], p2[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 x[4], d[4];
+            unpack8x2(v[i], x);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) d[c] = __fadd2_rn(x[c], nx0);
+            p1[i] = __fadd2_rn(__fadd2_rn(d[0], d[1]), __fadd2_rn(d[2], d[3]));
+            p2[i] = __fadd2_rn(__ffma2_rn(d[1], d[1], __fmul2_rn(d[0], d[0])),
+                               __ffma2_rn(d[3], d[3], __fmul2_rn(d[2], d[2])));
+        }
+        g1[q] = __fadd2_rn(__fadd2_rn(p1[0], p1[1]), __fadd2_rn(p1[2], p1[3]));
+        g2[q] = __fadd2_rn(__fadd2_rn(p2[0], p2[1]), __fadd2_rn(p2[2], p2[3]));
     }
-    const float x0 = __shfl_sync(0xffffffffu, bf16lo(v[0].x), lane & ~3);
-    const float2 nx0 = make_float2(-x0, -x0);
-    // pairwise sums (a short dependency chain): per 16-byte piece, then over pieces
-    float2 p1[4], p2[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float2 x[4], d[4];
-        unpack8x2(v[i], x);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) d[c] = __fadd2_rn(x[c], nx0);
-        p1[i] = __fadd2_rn(__fadd2_rn(d[0], d[1]), __fadd2_rn(d[2], d[3]));
-        p2[i] = __fadd2_rn(__ffma2_rn(d[1], d[1], __fmul2_rn(d[0], d[0])),
-                           __ffma2_rn(d[3], d[3], __fmul2_rn(d[2], d[2])));
-    }
-    const float2 s1 = __fadd2_rn(__fadd2_rn(p1[0], p1[1]), __fadd2_rn(p1[2], p1[3]));
-    const float2 s2 = __fadd2_rn(__fadd2_rn(p2[0], p2[1]), __fadd2_rn(p2[2], p2[3]));
-    float a1 = __fadd_rn(s1.x, s1.y), a2 = __fadd_rn(s2.x, s2.y);
-    a1 = __fadd_rn(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
-    a2 = __fadd_rn(a2, __shfl_xor_sync(0xffffffffu, a2, 1));
-    a1 = __fadd_rn(a1, __shfl_xor_sync(0xffffffffu, a1, 2));
-    a2 = __fadd_rn(a2, __shfl_xor_sync(0xffffffffu, a2, 2));
+    const float2 s1 = __fadd2_rn(__fadd2_rn(g1[0], g1[1]), __fadd2_rn(g1[2], g1[3]));
+    const float2 s2 = __fadd2_rn(__fadd2_rn(g2[0], g2[1]), __fadd2_rn(g2[2], g2[3]));
+    const float a1 = __fadd_rn(s1.x, s1.y), a2 = __fadd_rn(s2.x, s2.y);
     const float dm = __fmul_rn(a1, 1.0f / kD);
     const float var = fmaxf(fmaf(-dm, dm, __fmul_rn(a2, 1.0f / kD)), 0.f);
     const float mu = __fadd_rn(x0, dm);
@@ -151,24 +157,13 @@ DSA_DEVINL float2 row_stats(const __nv_bfloat16 *row, int q, int rot, bool act, 
     return make_float2(r, __fmul_rn(-mu, r));
 }
 
-// LayerNorm statistics of a tile's token rows, four threads per row; odd rows of
-// the tile are rotated by four pieces, so the eight threads of a shared-memory
-// phase touch eight distinct bank groups. Stores (rstd, -mu * rstd). Every
-// thread of the consumer group calls it (warp-uniform loop); ctid & 31 is the
-// thread's lane.
+// LayerNorm statistics of a tile's token rows, one thread a row, the row's
+// read order keyed by its index in the tile (rot = index mod 8). Stores
+// (rstd, -mu * rstd). Every thread of the statistics group calls it.
 DSA_DEVINL void token_stats(const __nv_bfloat16 *sk, int ntok, float eps, float2 *stat, int ctid,
                             int nthreads) {
-    const int q = ctid & 3;
-    const int rows = nthreads / 4;
-    // two rows a thread group per step, so both rows' loads and sums overlap
-    for (int tok0 = 0; tok0 < ntok; tok0 += 2 * rows) {
-        const int ta = tok0 + (ctid >> 2), tb = ta + rows;
-        const bool aa = ta < ntok, ab = tb < ntok;
-        const float2 sa = row_stats(sk + (size_t)(aa ? ta : 0) * kD, q, 4 * (ta & 1), aa, eps);
-        const float2 sb = row_stats(sk + (size_t)(ab ? tb : 0) * kD, q, 4 * (tb & 1), ab, eps);
-        if (aa && q == 0) stat[ta] = sa;
-        if (ab && q == 0) stat[tb] = sb;
-    }
+    for (int tok = ctid; tok < ntok; tok += nthreads)
+        stat[tok] = row_stats(sk + (size_t)tok * kD, tok & 7, eps);
 }
 
 // The pooled key chunk of lane l (channels 8l..8l+7) from the pool's kpool
@@ -268,10 +263,16 @@ DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *g
     return o;
 }
 
-struct CmpMeta {
+// A tile's description, read by every consumer thread as two 16-byte loads.
+struct __align__(16) CmpMeta {
     int b, p0, p1, n_in, f, rs;
     int voff;             // validity byte of the tile's first row in the stage's byte window
+    int pad;
 };
+DSA_DEVINL CmpMeta load_meta(const CmpMeta *m) {
+    const int4 a = reinterpret_cast<const int4 *>(m)[0], c = reinterpret_cast<const int4 *>(m)[1];
+    return CmpMeta{a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+}
 // A stage's validity window: the 16-byte-aligned span of validity bytes that
 // covers the tile's rows (at most 128 rows + 2 x 15 bytes of alignment).
 constexpr int kCmpValidWindow = 160;
@@ -480,10 +481,11 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             }
             bb = lo;
         }
-        for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
-            const int s = i % ns;
+        // ring position: stage s of pass ph (tile i uses stage i mod ns in pass i / ns)
+        for (int t = t_begin, i = 0, s = 0, ph = 0; t < t_end;
+             ++t, ++i, ph ^= (s + 1 == ns), s = (s + 1 == ns) ? 0 : s + 1) {
             bool ok = true;
-            if (i >= ns) ok = mbar_wait(&empty[s], ((i / ns) - 1) & 1);
+            if (i >= ns) ok = mbar_wait(&empty[s], ph ^ 1);
             if (!__all_sync(0xffffffffu, ok)) break;
             int b, j;
             if (balanced) {
@@ -521,7 +523,7 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
                     s_valid[s][r - vs] = valid[r];
             __syncwarp();
             if (lane == 0) {
-                meta[s] = CmpMeta{b, p0, p1, n_in, cur_f, cur_rs, (int)(row0 - vs)};
+                meta[s] = CmpMeta{b, p0, p1, n_in, cur_f, cur_rs, (int)(row0 - vs), 0};
                 if (n_in > 0) {
                     const uint32_t bytes = (uint32_t)(n_in * KP * kD * 2);
                     __nv_bfloat16 *sk = reinterpret_cast<__nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
@@ -570,9 +572,8 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     // barrier spans all consumers.
     if (warp >= C::kPoolWarps) {
         const int stid = tid - C::kPoolWarps * 32;
-        for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
-            const int s = i % ns;
-            const bool ok = mbar_wait(&full[s], (i / ns) & 1);
+        for (int t = t_begin, s = 0, ph = 0; t < t_end; ++t, ph ^= (s + 1 == ns), s = (s + 1 == ns) ? 0 : s + 1) {
+            const bool ok = mbar_wait(&full[s], ph);
             if (!__all_sync(0xffffffffu, ok)) break;
             const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
             token_stats(sk, meta[s].n_in * KP, eps, &s_stat[s][0], stid, C::kStatWarps * 32);
@@ -593,11 +594,10 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         const int b_lo = (int)((long long)blockIdx.x * B / G), b_hi = (int)((long long)(blockIdx.x + 1) * B / G);
         for (int b = b_lo + tid; b < b_hi; b += kPoolThreads) first_valid[b] = s_f[b];
     }
-    for (int t = t_begin, i = 0; t < t_end; ++t, ++i) {
-        const int s = i % ns;
-        const bool ok = mbar_wait(&stat_full[s], (i / ns) & 1);
+    for (int t = t_begin, s = 0, ph = 0; t < t_end; ++t, ph ^= (s + 1 == ns), s = (s + 1 == ns) ? 0 : s + 1) {
+        const bool ok = mbar_wait(&stat_full[s], ph);
         if (!__all_sync(0xffffffffu, ok)) break;
-        const CmpMeta m = meta[s];
+        const CmpMeta m = load_meta(&meta[s]);
         const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(cmp_smem + s * kCmpStageBytes);
         const __nv_bfloat16 *sg = sk + kCmpTileTokens * kD;
         const size_t pool_base = (size_t)m.b * max_pools;
@@ -615,9 +615,11 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             const bool active = ii + (hw & 1) < m.n_in;
             const int pi = active ? ii + (hw & 1) : ii;
             const int p = m.p0 + pi;
-            bool okp = true;
-#pragma unroll
-            for (int ss = 0; ss < KP; ++ss) okp = okp && s_valid[s][m.voff + pi * KP + ss] != 0;
+            // the pool is valid iff its KP validity bytes are all nonzero: lane l < KP
+            // of the half-warp tests byte l, one ballot gathers them
+            const bool vb = l >= KP || s_valid[s][m.voff + pi * KP + l] != 0;
+            const uint32_t vbits = (__ballot_sync(0xffffffffu, vb) >> (16 * (hw & 1))) & 0xFFFFu;
+            const bool okp = vbits == 0xFFFFu;
             const uint4 o = compress_pool<KP>(sk + (size_t)pi * KP * kD + 8 * l,
                                               sg + (size_t)pi * KP * kD + 8 * l,
                                               &s_stat[s][pi * KP], s_ape, lw, lb, l, okp);

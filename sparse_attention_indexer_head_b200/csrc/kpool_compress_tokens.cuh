@@ -17,9 +17,9 @@ namespace dsa {
 // recomputed.
 //
 // One CTA (four warps) per request; a half-warp per pool: its kpool k and gate
-// rows are staged in shared memory, their LayerNorm statistics taken four lanes
-// per row (row_stats, with the full kernel's rotation), then the same slot
-// softmax and pooling as the full kernel (compress_pool).
+// rows are staged in shared memory, their LayerNorm statistics taken a lane a
+// row (row_stats, in the full kernel's read order), then the same slot softmax
+// and pooling as the full kernel (compress_pool).
 constexpr int kTokWarps = 4;
 
 template <int KP>
@@ -89,17 +89,12 @@ kpool_compress_tokens_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfl
             }
         }
         __syncwarp();
-        // LayerNorm statistics of the pool's rows, four lanes per row (both halves
-        // run it). The full kernel rotates a row by the parity of its index in its
-        // tile of CmpCfg<KP>::kTP pools; the same rotation gives the same bits.
-#pragma unroll
-        for (int s0 = 0; s0 < KP; s0 += 4) {
-            const int sl = s0 + (l >> 2);
-            const bool ract = sl < KP;
-            const int tok_in_tile = (p % CmpCfg<KP>::kTP) * KP + sl;
-            const float2 st = row_stats(&s_rows[hw][0][ract ? sl : 0][0], l & 3,
-                                        4 * (tok_in_tile & 1), ract, eps);
-            if (ract && (l & 3) == 0) s_st[hw][sl] = st;
+        // LayerNorm statistics of the pool's rows, lane l < KP of each half-warp
+        // taking row l. The full kernel keys a row's read order by its index in
+        // its tile of CmpCfg<KP>::kTP pools; the same key gives the same bits.
+        if (in_span && l < KP) {
+            const int tok_in_tile = (p % CmpCfg<KP>::kTP) * KP + l;
+            s_st[hw][l] = row_stats(&s_rows[hw][0][l][0], tok_in_tile & 7, eps);
         }
         __syncwarp();
         // pool valid iff every slot token is valid
