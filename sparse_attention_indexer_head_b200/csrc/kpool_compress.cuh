@@ -157,34 +157,41 @@ DSA_DEVINL float2 row_stats(const __nv_bfloat16 *row, int rot, float eps) {
     return make_float2(r, __fmul_rn(-mu, r));
 }
 
+// The statistics as the pool warps read them: (rstd, rstd, -mu * rstd,
+// -mu * rstd), each value already paired for the packed fp32x2 arithmetic.
+DSA_DEVINL float4 stat_pairs(float2 st) { return make_float4(st.x, st.x, st.y, st.y); }
+
 // LayerNorm statistics of a tile's token rows, one thread a row, the row's
-// read order keyed by its index in the tile (rot = index mod 8). Stores
-// (rstd, -mu * rstd). Every thread of the statistics group calls it.
-DSA_DEVINL void token_stats(const __nv_bfloat16 *sk, int ntok, float eps, float2 *stat, int ctid,
+// read order keyed by its index in the tile (rot = index mod 8). Every thread
+// of the statistics group calls it.
+DSA_DEVINL void token_stats(const __nv_bfloat16 *sk, int ntok, float eps, float4 *stat, int ctid,
                             int nthreads) {
     for (int tok = ctid; tok < ntok; tok += nthreads)
-        stat[tok] = row_stats(sk + (size_t)tok * kD, tok & 7, eps);
+        stat[tok] = stat_pairs(row_stats(sk + (size_t)tok * kD, tok & 7, eps));
 }
 
 // The pooled key chunk of lane l (channels 8l..8l+7) from the pool's kpool
-// k rows and gate rows, with the rows' LayerNorm statistics st[s]. s_ape holds
+// k rows and gate rows, with the rows' LayerNorm statistics st[s] (as paired
+// by stat_pairs). s_ape holds
 // ape * log2(e) laid out [slot][half][lane][4] so a half-warp's loads are
 // contiguous. Returns the packed bf16 chunk (zero when the pool is invalid).
 //
 // One pass over the slots: the per-channel softmax is shifted by slot 0's
 // logit instead of the slots' maximum (the same quotient), so each slot's
 // exp2 weight and weighted k_norm row are formed as the row streams by, with
-// no max pass and no logits held between passes. A weight that overflows
+// no max pass and no logits held between passes; slot 0's own weight is
+// exactly 1 (0 + 1, so a non-finite logit still carries through as NaN), with
+// no exp2. A weight that overflows
 // (logits more than 2^7 apart in log2 units) leaves a non-finite denominator;
 // the warp then redoes its pools shifted by the slots' maximum.
 template <int KP>
 DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *grow,
-                               const float2 *st, const float *s_ape, const float2 (&lw)[4],
+                               const float4 *st, const float *s_ape, const float2 (&lw)[4],
                                const float2 (&lb)[4], int l, bool ok) {
     const float2 log2e2 = make_float2(kLog2e, kLog2e);
     auto knorm = [&](int s, float2 (&kn)[4]) {
-        const float2 rs = st[s];
-        const float2 r2 = make_float2(rs.x, rs.x), n2 = make_float2(rs.y, rs.y);
+        const float4 rs = st[s];
+        const float2 r2 = make_float2(rs.x, rs.y), n2 = make_float2(rs.z, rs.w);
         float2 x[4];
         unpack8x2(*reinterpret_cast<const uint4 *>(krow + s * kD), x);
 #pragma unroll
@@ -213,13 +220,28 @@ DSA_DEVINL uint4 compress_pool(const __nv_bfloat16 *krow, const __nv_bfloat16 *g
     }
 #pragma unroll 1
     for (int attempt = 0;; ++attempt) {
+        int s_first = 0;
+        if (attempt == 0) {
+            // slot 0 is the shift: its weight is (-nsh + nsh) + 1, i.e. 1, or NaN
+            // where its logit is not finite, as exp2 of the difference would give
+            float2 kn[4];
+            knorm(0, kn);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            den[c] = make_float2(0.f, 0.f);
-            acc[c] = make_float2(0.f, 0.f);
+            for (int c = 0; c < 4; ++c) {
+                const float2 z0 = __ffma2_rn(nsh[c], make_float2(-1.f, -1.f), nsh[c]);
+                den[c] = __fadd2_rn(z0, make_float2(1.f, 1.f));
+                acc[c] = __ffma2_rn(den[c], kn[c], make_float2(0.f, 0.f));
+            }
+            s_first = 1;
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                den[c] = make_float2(0.f, 0.f);
+                acc[c] = make_float2(0.f, 0.f);
+            }
         }
 #pragma unroll kSlotUnroll
-        for (int s = 0; s < KP; ++s) {
+        for (int s = s_first; s < KP; ++s) {
             float2 kn[4], lg[4];
             logits(s, lg);
             knorm(s, kn);
@@ -300,7 +322,7 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
     constexpr int kCmpThreads = C::kThreads;
     extern __shared__ __align__(128) uint8_t cmp_smem[];
     __shared__ __align__(16) float s_ape[KP * kD];   // ape * log2(e), [slot][half][lane][4]
-    __shared__ __align__(16) float2 s_stat[kCmpStages][kCmpTileTokens];   // (rstd, -mu*rstd)
+    __shared__ __align__(16) float4 s_stat[kCmpStages][kCmpTileTokens];   // stat_pairs
     __shared__ __align__(8) uint64_t full[kCmpStages], empty[kCmpStages], stat_full[kCmpStages];
     __shared__ CmpMeta meta[kCmpStages];
     __shared__ __align__(16) uint8_t s_valid[kCmpStages][kCmpValidWindow];
@@ -328,51 +350,61 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
         s_np_lo = INT_MAX;
         s_np_hi = 0;
     }
-    for (int i = tid; i < KP * kD; i += kCmpThreads) {
-        const int sl = i / kD, c = i % kD;
-        s_ape[(sl * 2 + ((c >> 2) & 1)) * 64 + 4 * (c >> 3) + (c & 3)] = ape[i] * kLog2e;
+    // Step inputs the path never writes, all read in one round trip before the
+    // wait on the preceding kernel: ape, the request offsets the partition
+    // choice needs, and the producer's first request (contiguous ranges).
+    constexpr int kApePerThread = (KP * kD + kCmpThreads - 1) / kCmpThreads;
+    float apev[kApePerThread];
+#pragma unroll
+    for (int u = 0; u < kApePerThread; ++u) {
+        const int i = tid + u * kCmpThreads;
+        apev[u] = i < KP * kD ? ape[i] : 0.f;
     }
-    __syncthreads();
-    // Request offsets and validity bytes are step inputs the path never writes:
-    // the producer has its first request's rows, and the balanced partition is
-    // complete, before the wait on the preceding kernel.
     // The balanced partition pays only where the requests' pool counts differ by
     // more than a tile; otherwise every request's tile grid holds about as many
     // real tiles and contiguous ranges of the grids are even already.
-    bool balanced = false;
+    int np_lo = INT_MAX, np_hi = 0;
     if (balance_ok) {
-        int lo = INT_MAX, hi = 0;
         for (int b = tid; b < B; b += kCmpThreads) {
-            const int np = min(max_pools, max(0, req_start[b + 1] - req_start[b]) / KP);
-            lo = min(lo, np);
-            hi = max(hi, np);
+            const int rs = req_start[b], re = req_start[b + 1];
+            s_rs[b] = rs;
+            if (b == B - 1) s_rs[B] = re;
+            const int np = min(max_pools, max(0, re - rs) / KP);
+            np_lo = min(np_lo, np);
+            np_hi = max(np_hi, np);
         }
-        lo = __reduce_min_sync(0xffffffffu, lo);
-        hi = __reduce_max_sync(0xffffffffu, hi);
-        if (lane == 0) {
-            atomicMin(&s_np_lo, lo);
-            atomicMax(&s_np_hi, hi);
-        }
-        __syncthreads();
-        balanced = s_np_hi - s_np_lo > TP;
+        np_lo = __reduce_min_sync(0xffffffffu, np_lo);
+        np_hi = __reduce_max_sync(0xffffffffu, np_hi);
     }
     long long total = 0;
     int first_rs = 0, first_re = 0;
-    if (!balanced && warp == kCmpConsumers / 32 && t_begin < t_end) {
+    if (warp == kCmpConsumers / 32 && t_begin < t_end) {
         const int b0 = t_begin / tiles_per_req;
         total = req_start[B];                       // rows of the validity array
         first_rs = req_start[b0];
         first_re = req_start[b0 + 1];
     }
+    __syncthreads();                                // barrier and counter initialisation
+#pragma unroll
+    for (int u = 0; u < kApePerThread; ++u) {
+        const int i = tid + u * kCmpThreads, sl = i / kD, c = i % kD;
+        if (i < KP * kD) s_ape[(sl * 2 + ((c >> 2) & 1)) * 64 + 4 * (c >> 3) + (c & 3)] = apev[u] * kLog2e;
+    }
+    if (balance_ok && lane == 0) {
+        atomicMin(&s_np_lo, np_lo);
+        atomicMax(&s_np_hi, np_hi);
+    }
+    __syncthreads();                                // s_ape, s_rs and the pool-count range
+    const bool balanced = balance_ok && s_np_hi - s_np_lo > TP;
     int g_lo = 0, g_hi = 0, e_lo = 0, e_hi = 0;
     if (balanced) {
-        total = req_start[B];
+        total = s_rs[B];
         // ---- each request's first valid token, a thread a request: the first 64
         // validity bytes from the request's first row (four 16-byte loads, a
         // nonzero-byte mask) settle almost every request; a warp scans the rest
 #pragma unroll 1
         for (int b = tid; b < B; b += kCmpThreads) {
-            const long long rs = req_start[b], re = req_start[b + 1];
+            const long long rs = s_rs[b], re = s_rs[b + 1];
             const long long c0 = rs & ~15ll;
             uint4 v[4];
 #pragma unroll
@@ -397,8 +429,6 @@ kpool_compress_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *
             else if (m) f = (int)(c0 + __ffsll((long long)m) - 1 - rs);
             else f = wend == re ? T : -1;
             s_f[b] = f;
-            s_rs[b] = (int)rs;
-            if (b == B - 1) s_rs[B] = (int)re;
         }
         __syncthreads();
         for (int b = warp; b < B; b += kCmpThreads / 32) {

@@ -35,7 +35,7 @@ kpool_compress_tokens_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfl
     constexpr int kHW = kTokWarps * 2;                     // half-warps: pools per round
     __shared__ __align__(16) float s_ape[KP * kD];         // ape * log2(e), [slot][half][lane][4]
     __shared__ __align__(16) __nv_bfloat16 s_rows[kHW][2][KP][kD];   // per half-warp: k rows, gate rows
-    __shared__ __align__(16) float2 s_st[kHW][KP];         // per half-warp: (rstd, -mu * rstd)
+    __shared__ __align__(16) float4 s_st[kHW][KP];         // per half-warp: stat_pairs
     __shared__ int s_f, s_fold, s_tb, s_te;
 
     const int b = blockIdx.x;
@@ -94,7 +94,7 @@ kpool_compress_tokens_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfl
         // its tile of CmpCfg<KP>::kTP pools; the same key gives the same bits.
         if (in_span && l < KP) {
             const int tok_in_tile = (p % CmpCfg<KP>::kTP) * KP + l;
-            s_st[hw][l] = row_stats(&s_rows[hw][0][l][0], tok_in_tile & 7, eps);
+            s_st[hw][l] = stat_pairs(row_stats(&s_rows[hw][0][l][0], tok_in_tile & 7, eps));
         }
         __syncwarp();
         // pool valid iff every slot token is valid
