@@ -464,9 +464,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constan
                 const int i = i0 + lane;
                 const uint32_t k = i < nloc ? akeys[i] : 0u;
                 const bool m = i < nloc && (k & pmask) == prefix;
-                const uint32_t d = m ? (k >> shift) & 0xFFu : 0x100u;
-                const uint32_t peers = __match_any_sync(0xffffffffu, d);
-                if (m && lane == __ffs(peers) - 1) atomicAdd(&ctl->hloc[d], __popc(peers));
+                hist_add_warp(ctl->hloc, m ? (k >> shift) & 0xFFu : 0x100u);
             }
             __syncthreads();
         }

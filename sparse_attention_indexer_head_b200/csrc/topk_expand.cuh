@@ -30,6 +30,23 @@ DSA_DEVINL uint32_t score_key(float s, bool is_cand) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Adds each lane's digit d (0x100: the lane has none) to a shared-memory
+// histogram: one atomic for the warp when every lane that has a digit has the
+// same one (the top digit of scores of one magnitude, or equal scores), else
+// one atomic a lane (digits spread over the bins). Exact integer counts either
+// way. Every lane of the warp calls it.
+DSA_DEVINL void hist_add_warp(int *h, uint32_t d) {
+    const uint32_t act = __ballot_sync(0xffffffffu, d != 0x100u);
+    if (act == 0u) return;
+    const int lead = __ffs(act) - 1;
+    const uint32_t dl = __shfl_sync(0xffffffffu, d, lead);
+    if (__all_sync(0xffffffffu, d == 0x100u || d == dl)) {
+        if ((int)(threadIdx.x & 31) == lead) atomicAdd(&h[dl], __popc(act));
+    } else if (d != 0x100u) {
+        atomicAdd(&h[d], 1);
+    }
+}
+
 // Tail slots (always_select_tail): after the K * KP pool slots, a row carries
 // KP - 1 slots for the query's trailing partial pool. With f the request's first
 // valid token and n = (q_pos - f + 1) mod KP tokens past the query's last
@@ -99,9 +116,7 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
             const uint32_t k = score_key(sv[u], cv[u] != 0);
             if (keys_in_smem && p < P) skeys[p] = k;
             cnt += k != 0u;
-            const uint32_t d = p < P ? (k >> 24) : 0x100u;
-            const uint32_t peers = __match_any_sync(0xffffffffu, d);
-            if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[0][d], __popc(peers));
+            hist_add_warp(hist[0], p < P ? (k >> 24) : 0x100u);
         }
     }
 #pragma unroll
@@ -123,8 +138,7 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
                 // the other buffer's pass is over (its pick was read): clear it for the next
                 if (tid < 256) hist[hb ^ 1][tid] = 0;
                 // Only keys under the chosen prefix count, and they spread over the
-                // next byte: plain shared atomics, except in a warp where many lanes
-                // match (crowded bins, e.g. equal scores), which aggregates per digit.
+                // next byte (crowded bins, e.g. equal scores, take one atomic a warp).
                 for (int base = (tid & ~31); base < P; base += kTopkThreads) {
                     const int p = base + (tid & 31);
                     uint32_t d = 0x100u;   // no bin
@@ -132,13 +146,7 @@ topk_expand_kernel(const float *__restrict__ scores, const uint8_t *__restrict__
                         const uint32_t k = key_at(p);
                         if ((k & pmask) == prefix) d = (k >> shift) & 0xFF;
                     }
-                    const uint32_t act = __ballot_sync(0xffffffffu, d != 0x100u);
-                    if (__popc(act) > 8) {
-                        const uint32_t peers = __match_any_sync(0xffffffffu, d);
-                        if (d != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[hb][d], __popc(peers));
-                    } else if (d != 0x100u) {
-                        atomicAdd(&hist[hb][d], 1);
-                    }
+                    hist_add_warp(hist[hb], d);
                 }
                 __syncthreads();
             }

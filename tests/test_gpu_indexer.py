@@ -86,6 +86,23 @@ def test_cluster_sizes_and_ragged_requests(B, kpool):
     device_status_clean(B)
 
 
+@pytest.mark.parametrize("kpool,lengths,pads,select_k", [
+    # 300 pool slots: 3 tiles, so five of the cluster's eight CTAs hold no pool
+    # and send empty counts; one request shorter than select_k, one all padding,
+    # one empty
+    (4, [37, 1200, 129, 0, 1100], [5, 17, 129, 0, 2], 100),
+    # 2048 pool slots (the batched decode's count): two tiles a CTA
+    (1, [2048, 700, 5], [0, 3, 5], 512),
+    (8, [16384, 9000], [7, 0], 512),
+])
+def test_small_pool_counts_and_idle_ranks(B, kpool, lengths, pads, select_k):
+    wl = _mini(kpool, lengths, pads, select_k=select_k, holes=[37 + 40, 37 + 41, 400])
+    assert wl.max_pools <= 2048
+    step, g = run_step(wl, fused=True)
+    stagewise(wl, g)
+    device_status_clean(B)
+
+
 def test_ties_and_more_slots_than_candidates(B):
     # a zero gate scores every candidate exactly 0: the lowest pool ids win, and a
     # request with fewer candidates than select_k gets the -1 tail
