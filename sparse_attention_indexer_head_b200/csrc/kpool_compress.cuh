@@ -5,22 +5,27 @@
 // B200 design. The op streams the k and gate caches once (256 B per token row
 // each) and writes one 256 B key per pool: it is HBM-bound, so the kernel is a
 // TMA-fed stream with all arithmetic in registers:
-//   * a persistent CTA owns a contiguous range of tiles; a tile is TP
+//   * a persistent CTA (one an SM) owns a range of tiles; a tile is TP
 //     consecutive pools of one request, i.e. up to 128 contiguous token rows
-//     of k and of gate. For up to 2048 requests (1152 above kpool 4) the CTAs
+//     of k and of gate. Where the requests' pool counts differ by more than a
+//     tile (and there are at most 2048 requests, 1152 above kpool 4) the CTAs
 //     first find every request's first valid token and split the tiles that
-//     hold pools evenly among themselves (requests of very different lengths
-//     then cost no imbalance, and pool slots past a request's span are written
-//     apart, without a trip through the pipeline); a producer warp moves each tile with 1-D bulk copies
-//     (cp.async.bulk) into a shared-memory ring -- the k rows, the gate rows
-//     and the 16-byte-aligned span of validity bytes covering them -- all
-//     completing on one mbarrier, so no consumer waits on a global load;
-//   * a half-warp handles one pool; lane l owns channels 8l..8l+7 (one 16-byte
-//     vector of each row), LayerNorm statistics are half-warp shuffle sums;
-//   * the per-channel softmax over the kpool slots is done in fp32 registers
-//     (max-subtracted, exp2 with log2(e) folded into the logits);
-//   * the first valid token of a request is found by a warp-wide ballot scan
-//     of its validity bytes (16-byte loads).
+//     hold pools evenly among themselves (pool slots past a request's span are
+//     then written apart, without a trip through the pipeline); otherwise each
+//     takes a contiguous range of every request's tile grid;
+//   * a producer warp moves each tile with 1-D bulk copies (cp.async.bulk) into
+//     a shared-memory ring -- the k rows, the gate rows and the 16-byte-aligned
+//     span of validity bytes covering them -- all completing on one mbarrier,
+//     so no consumer waits on a global load;
+//   * statistics warps take each landed tile's LayerNorm statistics, one thread
+//     a token row, and hand them to the pool warps by mbarrier;
+//   * a half-warp of a pool warp handles one pool; lane l owns channels
+//     8l..8l+7 (one 16-byte vector of each row); the per-channel softmax over
+//     the kpool slots runs in one pass in packed fp32x2, shifted by slot 0's
+//     logit (exp2 with log2(e) folded into the logits; a second pass shifted by
+//     the slots' maximum where a weight overflows);
+//   * the first valid token of a request is found from its validity bytes
+//     (16-byte loads, a ballot scan).
 #pragma once
 
 #include "common.cuh"
