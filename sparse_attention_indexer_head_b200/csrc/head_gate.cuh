@@ -151,6 +151,105 @@ head_gate_kernel(const float *__restrict__ hidden, const float *__restrict__ w,
                      : "memory");
 }
 
+// Many rows (chunked prefill): the row blocks alone fill the device, so a CTA
+// takes its 16 rows over the whole of K, with no cluster: the same staging,
+// lane mapping and fixed-order warp fold as above, the next slice's loads in
+// flight (registers) while the current slice is summed. Deterministic; the
+// order of the sum differs from the split kernel's only in where the K slices
+// meet.
+__global__ void __launch_bounds__(kGateThreads, 1)
+head_gate_rows_kernel(const float *__restrict__ hidden, const float *__restrict__ w,
+                      float *__restrict__ out, int M, int K, int N) {
+    extern __shared__ __align__(16) float gate_smem[];
+    float *hs = gate_smem;                                   // [16][513]
+    float *ws = hs + kGateRows * kGateHStride;               // [512][16], zero-padded columns
+    float *red = ws + kGateSlice * kGateMaxN;                // [16 warps][16][16]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int m0 = blockIdx.x * kGateRows;
+    const int rows = min(kGateRows, M - m0);
+    const int m = lane >> 1, n0 = (lane & 1) * 8;
+    const bool w_vec = N == kGateMaxN && aligned16(w);
+    constexpr int HV = kGateRows * kGateSlice / 4 / kGateThreads;    // 4 float4 of hidden
+    constexpr int WV = kGateSlice * kGateMaxN / 4 / kGateThreads;    // 4 float4 of w
+    float4 hv[HV], wv[WV];
+    auto load = [&](int k0) {
+        const int len = min(kGateSlice, K - k0);
+#pragma unroll
+        for (int u = 0; u < HV; ++u) {
+            const int i = tid + u * kGateThreads;          // i = r * 128 + c4
+            const int r = i >> 7, c4 = (i & 127) * 4;
+            hv[u] = (r < rows && c4 < len)
+                        ? __ldg(reinterpret_cast<const float4 *>(hidden + (size_t)(m0 + r) * K + k0 + c4))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (w_vec) {
+            const float4 *src = reinterpret_cast<const float4 *>(w + (size_t)k0 * kGateMaxN);
+#pragma unroll
+            for (int u = 0; u < WV; ++u) {
+                const int i = tid + u * kGateThreads;
+                wv[u] = i < len * 4 ? __ldg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < WV; ++u) {
+                const int i = tid + u * kGateThreads;      // float4 index: row i/4, cols 4(i%4)..
+                const int kk = i >> 2, c = (i & 3) * 4;
+                float t[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    t[e] = (kk < len && c + e < N) ? __ldg(w + (size_t)(k0 + kk) * N + c + e) : 0.f;
+                wv[u] = make_float4(t[0], t[1], t[2], t[3]);
+            }
+        }
+    };
+    float acc[8];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) acc[n] = 0.f;
+    load(0);
+    for (int k0 = 0; k0 < K; k0 += kGateSlice) {
+        const int len = min(kGateSlice, K - k0);
+        __syncthreads();   // the previous slice is done with hs / ws
+#pragma unroll
+        for (int u = 0; u < HV; ++u) {
+            const int i = tid + u * kGateThreads;
+            const int r = i >> 7, c4 = (i & 127) * 4;
+            float *d = hs + r * kGateHStride + c4;
+            d[0] = hv[u].x; d[1] = hv[u].y; d[2] = hv[u].z; d[3] = hv[u].w;
+        }
+#pragma unroll
+        for (int u = 0; u < WV; ++u)
+            reinterpret_cast<float4 *>(ws)[tid + u * kGateThreads] = wv[u];
+        __syncthreads();
+        if (k0 + kGateSlice < K) load(k0 + kGateSlice);   // in flight while this slice is summed
+        const float *hrow = hs + m * kGateHStride;
+#pragma unroll 4
+        for (int kk = warp; kk < len; kk += kGateWarps) {
+            const float h = hrow[kk];
+            const float4 wa = *reinterpret_cast<const float4 *>(ws + kk * kGateMaxN + n0);
+            const float4 wb = *reinterpret_cast<const float4 *>(ws + kk * kGateMaxN + n0 + 4);
+            acc[0] = fmaf(h, wa.x, acc[0]); acc[1] = fmaf(h, wa.y, acc[1]);
+            acc[2] = fmaf(h, wa.z, acc[2]); acc[3] = fmaf(h, wa.w, acc[3]);
+            acc[4] = fmaf(h, wb.x, acc[4]); acc[5] = fmaf(h, wb.y, acc[5]);
+            acc[6] = fmaf(h, wb.z, acc[6]); acc[7] = fmaf(h, wb.w, acc[7]);
+        }
+    }
+    // Loads and arithmetic above touch only the step's inputs; the output is
+    // written after the predecessor grid.
+    pdl_wait();
+    pdl_launch_dependents();
+#pragma unroll
+    for (int n = 0; n < 8; ++n) red[(warp * kGateRows + m) * kGateMaxN + n0 + n] = acc[n];
+    __syncthreads();
+    if (tid < kGateRows * kGateMaxN) {
+        const int r = tid / kGateMaxN, n = tid % kGateMaxN;
+        float sum = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < kGateWarps; ++w2) sum += red[w2 * kGateRows * kGateMaxN + tid];
+        if (r < rows && n < N) out[(size_t)(m0 + r) * N + n] = sum;
+    }
+}
+
 // The size checks of head_gate_launch, on their own (no pointer is looked at).
 inline int head_gate_shape_status(int M, int K, int N) {
     if (M < 0 || K <= 0 || N <= 0) return DSA_ERR_INVALID_ARG;
@@ -168,6 +267,16 @@ inline int head_gate_launch(const float *hidden, const float *w, float *out, int
     if (!aligned(hidden, 16) || !aligned(w, 4) || !aligned(out, 4)) return DSA_ERR_ALIGNMENT;
     const int row_blocks = ceil_div(M, kGateRows);
     if (row_blocks > 65535 * 16) return DSA_ERR_UNSUPPORTED;
+    // Where the split clusters would take more than two waves of the device,
+    // the row blocks alone fill it: one CTA a row block over the whole of K.
+    if ((long long)row_blocks * kGateSplit > 2ll * sm_count()) {
+        if (!ensure_smem_attr(reinterpret_cast<const void *>(head_gate_rows_kernel), kGateSmem))
+            return DSA_ERR_CUDA;
+        if (launch_pdl(head_gate_rows_kernel, dim3(row_blocks), dim3(kGateThreads), kGateSmem, stream,
+                       hidden, w, out, M, K, N) != cudaSuccess)
+            return DSA_ERR_CUDA;
+        return launch_status();
+    }
     dim3 grid(row_blocks, kGateSplit);
     if (!ensure_smem_attr(reinterpret_cast<const void *>(head_gate_kernel), kGateSmem))
         return DSA_ERR_CUDA;

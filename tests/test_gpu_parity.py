@@ -200,8 +200,12 @@ def test_scores_many_queries(B, H):
 
 def test_head_gate_shapes(B):
     rng = np.random.default_rng(5)
+    # up to 592 rows the K split over clusters of 8; above, a CTA a 16-row block
+    # over the whole of K (partial row blocks, K not a multiple of the 512-k
+    # slice, N below 16)
     for M, K, N in [(1, 4096, 16), (5, 4096, 16), (16, 4096, 16), (17, 4096, 16),
-                    (33, 1000, 8), (3, 4, 1), (2048, 4096, 16), (7, 8192, 13)]:
+                    (33, 1000, 8), (3, 4, 1), (2048, 4096, 16), (7, 8192, 13),
+                    (600, 4100, 16), (1000, 1000, 13), (2047, 516, 16)]:
         h = rng.standard_normal((M, K), dtype=np.float32)
         w = (rng.standard_normal((K, N)) / 64).astype(np.float32)
         out = torch.full((M, N), float("nan"), device="cuda")
