@@ -105,8 +105,10 @@ int dsa_abi_version(void);
  * a1. Indexer head gate [PR227]: out[m, n] = sum_k hidden[m, k] * w[k, n].
  *   hidden fp32 [M, K] row-major; w fp32 [K, N] row-major; out fp32 [M, N].
  *   fp32 products and fp32 accumulation; K is split over a cluster of CTAs and
- *   the partial sums are combined in a fixed order, so results are
- *   deterministic (they differ from a sequential sum only in rounding).
+ *   the partial sums are combined in a fixed order (for many rows, where the
+ *   clusters would take more than two waves of the device, one CTA takes 16
+ *   rows over the whole of K instead), so results are deterministic (they
+ *   differ from a sequential sum only in rounding).
  *   Requires 1 <= N <= 16, K >= 1 with K % 4 == 0; M == 0 is a no-op.
  *   Alignment: hidden 16 bytes; w and out 4 bytes.
  */
