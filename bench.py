@@ -175,9 +175,9 @@ def kernel_source_sha(kernel_file: str) -> str:
     return h.hexdigest()[:16]
 
 
-# kernel source of each stage (its DRAM traffic is valid only for that source)
 # Steps in flight in the end-to-end loop (StreamedDecode slots).
 E2E_SLOTS = 4
+# kernel source of each stage (its DRAM traffic is valid only for that source)
 STAGE_SOURCE = {"head_gate": "head_gate.cuh", "kpool_compress": "kpool_compress.cuh",
                 "index_scores": "index_scores.cuh", "topk_expand": "topk_expand.cuh",
                 "indexer": "indexer.cuh", "sparse_mla": "sparse_mla.cuh"}
